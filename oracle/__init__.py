@@ -1,0 +1,218 @@
+"""CPU oracle for Sparse Delta Memory (SDM).  TEST INFRASTRUCTURE ONLY.
+
+A plain, slow fp64 implementation (``sdm_oracle.c``) of what the SDM hot path
+computes: product-key scoring with top-W / top-R selection and softmax weights,
+and the sparse gated-delta recurrence over an N-slot memory that starts from M0.
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It shares no code with the CUDA path and
+never imports it.
+
+Readings of the method (the pages give prose, not equations) are written out in
+``sdm_oracle.c``'s header; each C function names the passage it follows.
+
+Parity status per function:
+  half_scores / topk / score ... pinned (brute force vs product key, numpy matmul
+                                 + argsort, exact-recall proof when k >= top)
+  softmax weights ............. pinned (sum to 1, order, closed form on 2 slots)
+  recur_dense ................. pinned (beta=0 closed form, one-hot write/read,
+                                 dense Gated DeltaNet matrix form, hand example)
+  recur_lazy .................. pinned (agrees with recur_dense to 1e-12)
+  materialize ................. pinned (beta=0 closed form)
+  prefill_pairs ............... pinned through score + recur_lazy
+The softmax temperature and the tie order are readings the pages do not fix
+(parity of those two choices is unpinned by the pages themselves).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(_HERE, "sdm_oracle.c")
+LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_default = None
+
+MODE_BRUTE = 0
+MODE_PK = 1
+
+
+def build(force: bool = False, src: str = SRC, out: str = LIB_PATH) -> str:
+    """Compile the oracle C source into a shared library with gcc (-O2, OpenMP)."""
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+        return out
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-o", tmp, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise ValueError(f"oracle {what} failed with code {rc}")
+
+
+class Oracle:
+    """numpy front end over one build of the oracle library."""
+
+    def __init__(self, lib_path: str = LIB_PATH):
+        lib = ctypes.CDLL(lib_path)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        D = ctypes.c_double
+        lib.sdm_oracle_half_scores.argtypes = [P, P, I, I, P, P]
+        lib.sdm_oracle_half_scores.restype = None
+        lib.sdm_oracle_topk_vec.argtypes = [P, P, I, I, I, I, I, P, P, P]
+        lib.sdm_oracle_topk_vec.restype = I
+        lib.sdm_oracle_score.argtypes = [P, P, I, I, I, I, I, I, I, I, P, P, P, I]
+        lib.sdm_oracle_score.restype = I
+        lib.sdm_oracle_recur_dense.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P]
+        lib.sdm_oracle_recur_dense.restype = I
+        lib.sdm_oracle_recur_lazy.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P]
+        lib.sdm_oracle_recur_lazy.restype = I
+        lib.sdm_oracle_materialize.argtypes = [I, I, P, P, D, P]
+        lib.sdm_oracle_materialize.restype = None
+        lib.sdm_oracle_prefill_pairs.argtypes = [I, I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P,
+                                                 I, P, P, I]
+        lib.sdm_oracle_prefill_pairs.restype = I
+        lib.sdm_oracle_max_threads.argtypes = []
+        lib.sdm_oracle_max_threads.restype = I
+        self.lib = lib
+
+    def max_threads(self) -> int:
+        return int(self.lib.sdm_oracle_max_threads())
+
+    def half_scores(self, x, sk):
+        """s1[i] = <x[:h], C1[i]>, s2[j] = <x[h:], C2[j]> for one vector x [2h], sk [2,n,h]."""
+        x, sk = _f64(x), _f64(sk)
+        n, hd = sk.shape[1], sk.shape[2]
+        assert x.shape == (2 * hd,)
+        s1 = np.empty(n, np.float64)
+        s2 = np.empty(n, np.float64)
+        self.lib.sdm_oracle_half_scores(_p(x), _p(sk), n, hd, _p(s1), _p(s2))
+        return s1, s2
+
+    def topk(self, x, sk, k_half: int, top: int, mode: int = MODE_PK):
+        """Best-first (idx, score, w) for one vector x [2h] against one role's tables sk [2,n,h]."""
+        x, sk = _f64(x), _f64(sk)
+        n, hd = sk.shape[1], sk.shape[2]
+        idx = np.empty(top, np.int32)
+        sc = np.empty(top, np.float64)
+        w = np.empty(top, np.float64)
+        _check(self.lib.sdm_oracle_topk_vec(_p(x), _p(sk), n, hd, k_half, top, mode, _p(idx), _p(sc),
+                                            _p(w)), "topk")
+        return idx, sc, w
+
+    def score(self, x, sk, k_half: int, top: int, mode: int = MODE_PK, nthreads: int = 0):
+        """Batched scoring: x [B,H,T,2h], sk [H,2,n,h] -> idx/score/w [B,H,T,top]."""
+        x, sk = _f64(x), _f64(sk)
+        B, H, T, dk = x.shape
+        n, hd = sk.shape[2], sk.shape[3]
+        assert dk == 2 * hd and sk.shape[0] == H and sk.shape[1] == 2
+        idx = np.empty((B, H, T, top), np.int32)
+        sc = np.empty((B, H, T, top), np.float64)
+        w = np.empty((B, H, T, top), np.float64)
+        _check(self.lib.sdm_oracle_score(_p(x), _p(sk), B, H, T, hd, n, k_half, top, mode, _p(idx),
+                                         _p(sc), _p(w), nthreads), "score")
+        return idx, sc, w
+
+    def recur_dense(self, v, alpha, beta, widx, ww, ridx, rw, M):
+        """Dense-decay recurrence for one (b,h).  Returns (out [T,dv], M_final [N,dv])."""
+        v, alpha, beta = _f64(v), _f64(alpha), _f64(beta)
+        widx, ridx, ww, rw = _i32(widx), _i32(ridx), _f64(ww), _f64(rw)
+        M = _f64(M).copy()
+        T, dv = v.shape
+        N = M.shape[0]
+        W, R = widx.shape[1], ridx.shape[1]
+        out = np.empty((T, dv), np.float64)
+        _check(self.lib.sdm_oracle_recur_dense(T, N, dv, W, R, _p(v), _p(alpha), _p(beta), _p(widx),
+                                               _p(ww), _p(ridx), _p(rw), _p(M), _p(out)),
+               "recur_dense")
+        return out, M
+
+    @staticmethod
+    def fresh_lazy_state(M0h):
+        """Lazy state of a fresh sequence: Mraw = M0 (copy), stamp = 0, Lambda = 0."""
+        M0h = _f64(M0h)
+        return {"Mraw": M0h.copy(), "stamp": np.zeros(M0h.shape[0], np.float64), "Lambda": 0.0}
+
+    def recur_lazy(self, v, alpha, beta, widx, ww, ridx, rw, state):
+        """Lazy-decay recurrence for one (b,h); `state` is updated in place.  Returns out [T,dv]."""
+        v, alpha, beta = _f64(v), _f64(alpha), _f64(beta)
+        widx, ridx, ww, rw = _i32(widx), _i32(ridx), _f64(ww), _f64(rw)
+        T, dv = v.shape
+        Mraw, stamp = state["Mraw"], state["stamp"]
+        assert Mraw.dtype == np.float64 and Mraw.flags.c_contiguous and stamp.flags.c_contiguous
+        N = Mraw.shape[0]
+        W, R = widx.shape[1], ridx.shape[1]
+        lam = ctypes.c_double(state["Lambda"])
+        out = np.empty((T, dv), np.float64)
+        _check(self.lib.sdm_oracle_recur_lazy(T, N, dv, W, R, _p(v), _p(alpha), _p(beta), _p(widx),
+                                              _p(ww), _p(ridx), _p(rw), _p(Mraw), _p(stamp),
+                                              ctypes.byref(lam), _p(out)), "recur_lazy")
+        state["Lambda"] = lam.value
+        return out
+
+    def materialize(self, state):
+        """Dense [N,dv] memory of a lazy state."""
+        Mraw, stamp = state["Mraw"], state["stamp"]
+        N, dv = Mraw.shape
+        M = np.empty_like(Mraw)
+        self.lib.sdm_oracle_materialize(N, dv, _p(Mraw), _p(stamp), float(state["Lambda"]), _p(M))
+        return M
+
+    def prefill_pairs(self, q, k, v, alpha, beta, skw, skr, M0, k_half: int, W: int, R: int, pairs,
+                      nthreads: int = 0):
+        """Score both roles and run the lazy recurrence from M0 for each (b,h) in `pairs`.
+
+        Returns out [len(pairs), T, dv].  Used for the timed CPU baseline.
+        """
+        q, k, v, alpha, beta = _f64(q), _f64(k), _f64(v), _f64(alpha), _f64(beta)
+        skw, skr, M0 = _f64(skw), _f64(skr), _f64(M0)
+        B, H, T, dk = q.shape
+        n, hd = skw.shape[2], skw.shape[3]
+        dv = v.shape[3]
+        pairs = _i32(np.asarray(pairs).reshape(-1, 2))
+        out = np.empty((pairs.shape[0], T, dv), np.float64)
+        _check(self.lib.sdm_oracle_prefill_pairs(B, H, T, hd, n, dv, k_half, W, R, _p(q), _p(k),
+                                                 _p(v), _p(alpha), _p(beta), _p(skw), _p(skr),
+                                                 _p(M0), pairs.shape[0], _p(pairs), _p(out),
+                                                 nthreads), "prefill_pairs")
+        return out
+
+
+def default() -> Oracle:
+    """The oracle built from sdm_oracle.c (compiled on first use)."""
+    global _default
+    with _lock:
+        if _default is None:
+            build()
+            _default = Oracle(LIB_PATH)
+        return _default
+
+
+def __getattr__(name):
+    # module-level shortcuts: oracle.score(...), oracle.recur_lazy(...), ...
+    if name in {"max_threads", "half_scores", "topk", "score", "recur_dense", "recur_lazy",
+                "materialize", "prefill_pairs"}:
+        return getattr(default(), name)
+    if name == "fresh_lazy_state":
+        return Oracle.fresh_lazy_state
+    raise AttributeError(name)

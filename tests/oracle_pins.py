@@ -1,0 +1,347 @@
+"""Checks that pin the CPU oracle to facts that do not come from the oracle itself.
+
+Each function takes an ``oracle.Oracle`` and raises AssertionError when the
+oracle disagrees with what the definition or the mathematics fixes.  They are
+run against the real oracle (tests/test_oracle_pins.py) and against planted
+mutants of its C source (tests/test_oracle_mutants.py), where at least one of
+them must fail for every mutant.
+
+Sources: "Sparse Delta Memory: Scaling the State of Linear RNNs through
+Sparsity" summary pages — §2 Background (Gated DeltaNet; Product Key Memory),
+§3 Method (sparse updates, sparse addressing, sparse retrieval, connection to
+GDN, learned initial state), §4 SDM Configuration (softmax-normalised
+activations).
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _random_case(rng, T, N, dv, W, R, a_lo=0.8, a_hi=1.0):
+    v = rng.standard_normal((T, dv))
+    alpha = rng.uniform(a_lo, a_hi, T)
+    beta = rng.uniform(0.0, 1.0, T)
+    widx = np.stack([rng.choice(N, W, replace=False) for _ in range(T)]).astype(np.int32)
+    ridx = np.stack([rng.choice(N, R, replace=False) for _ in range(T)]).astype(np.int32)
+    ww = rng.uniform(0.05, 1.0, (T, W))
+    ww /= ww.sum(1, keepdims=True)
+    rw = rng.uniform(0.05, 1.0, (T, R))
+    rw /= rw.sum(1, keepdims=True)
+    M0 = rng.standard_normal((N, dv)) * 0.5
+    return v, alpha, beta, widx, ww, ridx, rw, M0
+
+
+# ---------------------------------------------------------------- scoring ---
+
+def pin_pk_equals_brute(o):
+    """Product-key top-W equals brute-force top-W over all N slots when k >= W
+    (a pair with per-half ranks (a, b) is beaten by at least (a+1)(b+1)-1 pairs)."""
+    rng = _rng(1)
+    for (n, hd, k, top) in [(8, 4, 4, 4), (16, 8, 6, 5), (16, 16, 16, 16), (32, 8, 8, 8)]:
+        sk = rng.standard_normal((2, n, hd))
+        for _ in range(20):
+            x = rng.standard_normal(2 * hd)
+            ib, sb, wb = o.topk(x, sk, k, top, mode=0)
+            ip, sp, wp = o.topk(x, sk, k, top, mode=1)
+            assert np.array_equal(ib, ip), (n, hd, k, top, ib, ip)
+            assert np.array_equal(sb, sp)
+
+
+def pin_brute_matches_numpy(o):
+    """Brute-force ranking equals a numpy matmul + lexsort of all N = n^2 slot scores."""
+    rng = _rng(2)
+    n, hd, top = 12, 6, 7
+    sk = rng.standard_normal((2, n, hd))
+    for _ in range(30):
+        x = rng.standard_normal(2 * hd)
+        s1 = sk[0] @ x[:hd]
+        s2 = sk[1] @ x[hd:]
+        full = (s1[:, None] + s2[None, :]).reshape(-1)  # slot s = i*n + j
+        order = np.lexsort((np.arange(n * n), -full))[:top]
+        idx, sc, w = o.topk(x, sk, n, top, mode=0)
+        assert np.array_equal(idx, order), (idx, order)
+        np.testing.assert_allclose(sc, full[order], rtol=0, atol=1e-12)
+        e = np.exp(full[order] - full[order].max())
+        np.testing.assert_allclose(w, e / e.sum(), rtol=1e-13, atol=0)
+
+
+def pin_pk_depends_on_k(o):
+    """With k < W the product-key shortlist must miss some brute-force winners."""
+    rng = _rng(3)
+    n, hd, k, top = 16, 4, 2, 4
+    sk = rng.standard_normal((2, n, hd))
+    differs = 0
+    for _ in range(50):
+        x = rng.standard_normal(2 * hd)
+        ib, _, _ = o.topk(x, sk, k, top, mode=0)
+        ip, _, _ = o.topk(x, sk, k, top, mode=1)
+        differs += int(not np.array_equal(ib, ip))
+        # every product-key pick lies in the k x k shortlist
+        s1, s2 = o.half_scores(x, sk)
+        top1 = set(np.lexsort((np.arange(n), -s1))[:k].tolist())
+        top2 = set(np.lexsort((np.arange(n), -s2))[:k].tolist())
+        for s in ip.tolist():
+            assert s // n in top1 and s % n in top2
+    assert differs > 0
+
+
+def pin_tie_order(o):
+    """Equal scores rank the lower slot first (reading: the pages fix no tie rule)."""
+    hd, n = 2, 4
+    sk = np.zeros((2, n, hd))
+    sk[0] = [[1, 0], [2, 0], [1, 0], [0, 0]]   # s1 = [1, 2, 1, 0] for x[:2] = [1, 0]
+    sk[1] = [[0, 1], [0, 1], [0, 0], [0, 3]]   # s2 = [1, 1, 0, 3] for x[2:] = [0, 1]
+    x = np.array([1.0, 0.0, 0.0, 1.0])
+    # slot scores: s(i,j) = s1[i] + s2[j]; best is (1,3)=5, then (0,3)=(2,3)=4 tie, ...
+    idx, sc, _ = o.topk(x, sk, 4, 5, mode=0)
+    s1 = np.array([1, 2, 1, 0.0])
+    s2 = np.array([1, 1, 0, 3.0])
+    full = (s1[:, None] + s2[None, :]).reshape(-1)
+    expect = sorted(range(16), key=lambda s: (-full[s], s))[:5]
+    assert idx.tolist() == expect, (idx, expect)
+    assert idx.tolist()[:3] == [7, 3, 11]
+    idx2, _, _ = o.topk(x, sk, 4, 5, mode=1)
+    assert idx2.tolist() == expect
+
+
+def pin_hand_scoring(o):
+    """The hand-worked scoring example in tests/golden/hand_scoring.json."""
+    with open(os.path.join(GOLDEN, "hand_scoring.json")) as f:
+        g = json.load(f)
+    for mode in (0, 1):
+        idx, sc, w = o.topk(g["x"], g["subkeys"], g["k_half"], g["top"], mode=mode)
+        assert idx.tolist() == g["idx"]
+        assert sc.tolist() == g["score"]
+        np.testing.assert_allclose(w, g["w"], rtol=1e-15, atol=0)
+
+
+def pin_softmax(o):
+    """Weights are softmax of the selected scores: positive, sum 1, best-first,
+    and w_a / w_b = exp(s_a - s_b)."""
+    rng = _rng(4)
+    n, hd = 8, 4
+    sk = rng.standard_normal((2, n, hd))
+    for top in (1, 2, 5):
+        for _ in range(10):
+            x = rng.standard_normal(2 * hd)
+            idx, sc, w = o.topk(x, sk, n, top, mode=1)
+            assert np.all(w > 0)
+            assert abs(w.sum() - 1.0) < 1e-14
+            assert np.all(np.diff(sc) <= 0) and np.all(np.diff(w) <= 1e-16)
+            if top >= 2:
+                np.testing.assert_allclose(w[0] / w[1], np.exp(sc[0] - sc[1]), rtol=1e-12)
+            if top == 1:
+                assert w[0] == 1.0
+
+
+def pin_batched_score(o):
+    """Batched scoring equals per-vector scoring, with per-head tables."""
+    rng = _rng(5)
+    B, H, T, hd, n, k, top = 2, 3, 5, 4, 6, 3, 3
+    x = rng.standard_normal((B, H, T, 2 * hd))
+    sk = rng.standard_normal((H, 2, n, hd))
+    idx, sc, w = o.score(x, sk, k, top, mode=1)
+    for b in range(B):
+        for h in range(H):
+            for t in range(T):
+                i1, s1, w1 = o.topk(x[b, h, t], sk[h], k, top, mode=1)
+                assert np.array_equal(idx[b, h, t], i1)
+                assert np.array_equal(w[b, h, t], w1)
+
+
+# ------------------------------------------------------------- recurrence ---
+
+def pin_beta_zero(o):
+    """beta = 0: memory only decays, M_T = M0 * prod(alpha) and
+    o_t = sum_j u_j M0[r_j] * prod_{s<=t} alpha_s."""
+    rng = _rng(6)
+    T, N, dv, W, R = 17, 20, 3, 4, 5
+    v, alpha, beta, widx, ww, ridx, rw, M0 = _random_case(rng, T, N, dv, W, R)
+    beta = np.zeros(T)
+    cum = np.cumprod(alpha)
+    expect_out = np.stack([(rw[t][:, None] * M0[ridx[t]]).sum(0) * cum[t] for t in range(T)])
+    out_d, M_d = o.recur_dense(v, alpha, beta, widx, ww, ridx, rw, M0)
+    np.testing.assert_allclose(out_d, expect_out, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(M_d, M0 * cum[-1], rtol=1e-12, atol=1e-14)
+    st = o.fresh_lazy_state(M0)
+    out_l = o.recur_lazy(v, alpha, beta, widx, ww, ridx, rw, st)
+    np.testing.assert_allclose(out_l, expect_out, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(o.materialize(st), M0 * cum[-1], rtol=1e-12, atol=1e-14)
+
+
+def pin_one_hot_exact(o):
+    """alpha = 1, beta = 1, a single write slot with weight 1 and a read of that
+    slot right after: the read returns v exactly (delta rule overwrite)."""
+    rng = _rng(7)
+    T, N, dv = 9, 12, 4
+    v = rng.standard_normal((T, dv))
+    s = rng.permutation(N)[:T].astype(np.int32)[:, None]  # each token writes a fresh slot
+    ones = np.ones((T, 1))
+    for M0 in (np.zeros((N, dv)), ):
+        out_d, _ = o.recur_dense(v, np.ones(T), np.ones(T), s, ones, s, ones, M0)
+        assert np.array_equal(out_d, v)
+        st = o.fresh_lazy_state(M0)
+        out_l = o.recur_lazy(v, np.ones(T), np.ones(T), s, ones, s, ones, st)
+        assert np.array_equal(out_l, v)
+    # non-zero M0: exact up to the one rounding of M + (v - M)
+    M0 = rng.standard_normal((N, dv))
+    out_d, _ = o.recur_dense(v, np.ones(T), np.ones(T), s, ones, s, ones, M0)
+    np.testing.assert_allclose(out_d, v, rtol=0, atol=4 * np.finfo(float).eps * 8)
+
+
+def pin_convex_update(o):
+    """W = R = 1 at one slot: M <- alpha*M + beta*(v - alpha*M), a textbook
+    exponential-moving-average step, and the read returns it."""
+    rng = _rng(8)
+    T, N, dv = 12, 5, 3
+    v = rng.standard_normal((T, dv))
+    alpha = rng.uniform(0.5, 1.0, T)
+    beta = rng.uniform(0.0, 1.0, T)
+    s = np.full((T, 1), 2, np.int32)
+    ones = np.ones((T, 1))
+    M0 = rng.standard_normal((N, dv))
+    m = M0[2].copy()
+    expect = []
+    for t in range(T):
+        m = (1 - beta[t]) * alpha[t] * m + beta[t] * v[t]
+        expect.append(m.copy())
+    out_d, M_d = o.recur_dense(v, alpha, beta, s, ones, s, ones, M0)
+    np.testing.assert_allclose(out_d, np.stack(expect), rtol=1e-12, atol=1e-14)
+    others = [i for i in range(N) if i != 2]
+    np.testing.assert_allclose(M_d[others], M0[others] * np.prod(alpha), rtol=1e-12)
+
+
+def pin_dense_limit_gdn(o):
+    """All N slots selected (W = R = N, k = n): the sparse recurrence is exactly
+    Gated DeltaNet with the dense key k_t = softmax weights over all slots,
+    S_t = alpha_t (I - beta_t k k^T) S_{t-1} + beta_t k v^T, o_t = S_t^T q_t."""
+    rng = _rng(9)
+    n, hd, T, dv = 4, 3, 11, 5
+    N = n * n
+    skw = rng.standard_normal((2, n, hd))
+    skr = rng.standard_normal((2, n, hd))
+    kx = rng.standard_normal((T, 2 * hd))
+    qx = rng.standard_normal((T, 2 * hd))
+    v = rng.standard_normal((T, dv))
+    alpha = rng.uniform(0.7, 1.0, T)
+    beta = rng.uniform(0.0, 1.0, T)
+    M0 = rng.standard_normal((N, dv)) * 0.3
+
+    def dense_weights(x, sk):
+        s = (sk[0] @ x[:hd])[:, None] + (sk[1] @ x[hd:])[None, :]
+        e = np.exp(s.reshape(-1) - s.max())
+        return e / e.sum()
+
+    S = M0.copy()
+    expect = []
+    for t in range(T):
+        kv = dense_weights(kx[t], skw)
+        qv = dense_weights(qx[t], skr)
+        S = alpha[t] * (np.eye(N) - beta[t] * np.outer(kv, kv)) @ S + beta[t] * np.outer(kv, v[t])
+        expect.append(S.T @ qv)
+    widx, ww, ridx, rw = [], [], [], []
+    for t in range(T):
+        i, _, w = o.topk(kx[t], skw, n, N, mode=1)
+        widx.append(i); ww.append(w)
+        i, _, w = o.topk(qx[t], skr, n, N, mode=1)
+        ridx.append(i); rw.append(w)
+    out_d, M_d = o.recur_dense(v, alpha, beta, np.array(widx), np.array(ww), np.array(ridx),
+                               np.array(rw), M0)
+    np.testing.assert_allclose(out_d, np.stack(expect), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(M_d, S, rtol=1e-11, atol=1e-12)
+
+
+def pin_lazy_equals_dense(o):
+    """Lazy decay (per-slot stamps) equals literal dense decay to 1e-12."""
+    rng = _rng(10)
+    for (T, N, dv, W, R) in [(40, 12, 3, 3, 4), (64, 50, 4, 6, 6), (30, 9, 2, 9, 9)]:
+        v, alpha, beta, widx, ww, ridx, rw, M0 = _random_case(rng, T, N, dv, W, R, 0.5, 1.0)
+        out_d, M_d = o.recur_dense(v, alpha, beta, widx, ww, ridx, rw, M0)
+        st = o.fresh_lazy_state(M0)
+        out_l = o.recur_lazy(v, alpha, beta, widx, ww, ridx, rw, st)
+        scale = max(1.0, np.abs(out_d).max())
+        assert np.abs(out_l - out_d).max() <= 1e-12 * scale
+        assert np.abs(o.materialize(st) - M_d).max() <= 1e-12 * max(1.0, np.abs(M_d).max())
+
+
+def pin_split_invariance(o):
+    """One call over T tokens equals T1 tokens then T-T1 tokens, and equals T1
+    tokens then T-T1 single-token calls (the lazy state carries everything)."""
+    rng = _rng(11)
+    T, N, dv, W, R = 30, 15, 3, 3, 4
+    v, alpha, beta, widx, ww, ridx, rw, M0 = _random_case(rng, T, N, dv, W, R)
+    st = o.fresh_lazy_state(M0)
+    full = o.recur_lazy(v, alpha, beta, widx, ww, ridx, rw, st)
+    for T1 in (0, 1, 13, 29):
+        st2 = o.fresh_lazy_state(M0)
+        a = o.recur_lazy(v[:T1], alpha[:T1], beta[:T1], widx[:T1], ww[:T1], ridx[:T1], rw[:T1], st2)
+        b = o.recur_lazy(v[T1:], alpha[T1:], beta[T1:], widx[T1:], ww[T1:], ridx[T1:], rw[T1:], st2)
+        assert np.array_equal(np.concatenate([a, b]), full)
+        st3 = o.fresh_lazy_state(M0)
+        parts = [o.recur_lazy(v[:T1], alpha[:T1], beta[:T1], widx[:T1], ww[:T1], ridx[:T1],
+                              rw[:T1], st3)]
+        for t in range(T1, T):
+            sl = slice(t, t + 1)
+            parts.append(o.recur_lazy(v[sl], alpha[sl], beta[sl], widx[sl], ww[sl], ridx[sl],
+                                      rw[sl], st3))
+        assert np.array_equal(np.concatenate(parts), full)
+        assert np.array_equal(o.materialize(st3), o.materialize(st))
+    _, M_d = o.recur_dense(v, alpha, beta, widx, ww, ridx, rw, M0)
+    _, M_a = o.recur_dense(v[:7], alpha[:7], beta[:7], widx[:7], ww[:7], ridx[:7], rw[:7], M0)
+    _, M_b = o.recur_dense(v[7:], alpha[7:], beta[7:], widx[7:], ww[7:], ridx[7:], rw[7:], M_a)
+    assert np.array_equal(M_b, M_d)
+
+
+def pin_hand_recurrence(o):
+    """The hand-worked two-token example in tests/golden/hand_two_tokens.json."""
+    with open(os.path.join(GOLDEN, "hand_two_tokens.json")) as f:
+        g = json.load(f)
+    args = [np.array(g[k], dtype=float) for k in ("v", "alpha", "beta")]
+    widx, ridx = np.array(g["widx"]), np.array(g["ridx"])
+    ww, rw = np.array(g["ww"], float), np.array(g["rw"], float)
+    M0 = np.array(g["M0"], float)
+    out_d, M_d = o.recur_dense(*args, widx, ww, ridx, rw, M0)
+    assert out_d.tolist() == g["out"]
+    assert M_d.tolist() == g["M_final"]
+    st = o.fresh_lazy_state(M0)
+    out_l = o.recur_lazy(*args, widx, ww, ridx, rw, st)
+    assert out_l.tolist() == g["out"]
+    assert o.materialize(st).tolist() == g["M_final"]
+
+
+def pin_prefill_pairs(o):
+    """The batched prefill equals product-key scoring followed by the lazy recurrence."""
+    rng = _rng(12)
+    B, H, T, hd, n, dv, k, W, R = 2, 2, 9, 3, 5, 4, 3, 3, 2
+    q = rng.standard_normal((B, H, T, 2 * hd))
+    kk = rng.standard_normal((B, H, T, 2 * hd))
+    v = rng.standard_normal((B, H, T, dv))
+    alpha = rng.uniform(0.8, 1.0, (B, H, T))
+    beta = rng.uniform(0, 1, (B, H, T))
+    skw = rng.standard_normal((H, 2, n, hd))
+    skr = rng.standard_normal((H, 2, n, hd))
+    M0 = rng.standard_normal((H, n * n, dv))
+    pairs = [(1, 0), (0, 1)]
+    out = o.prefill_pairs(q, kk, v, alpha, beta, skw, skr, M0, k, W, R, pairs)
+    for pi, (b, h) in enumerate(pairs):
+        wi, _, wwt = o.score(kk[b:b + 1, h:h + 1], skw[h:h + 1], k, W)
+        ri, _, rwt = o.score(q[b:b + 1, h:h + 1], skr[h:h + 1], k, R)
+        st = o.fresh_lazy_state(M0[h])
+        ref = o.recur_lazy(v[b, h], alpha[b, h], beta[b, h], wi[0, 0], wwt[0, 0], ri[0, 0],
+                           rwt[0, 0], st)
+        assert np.array_equal(out[pi], ref)
+
+
+ALL_PINS = [pin_pk_equals_brute, pin_brute_matches_numpy, pin_pk_depends_on_k, pin_tie_order,
+            pin_hand_scoring, pin_softmax, pin_batched_score, pin_beta_zero, pin_one_hot_exact,
+            pin_convex_update, pin_dense_limit_gdn, pin_lazy_equals_dense, pin_split_invariance,
+            pin_hand_recurrence, pin_prefill_pairs]

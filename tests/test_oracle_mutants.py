@@ -1,0 +1,80 @@
+"""Plant plausible mistakes in the oracle's C source and check that the pins catch each one.
+
+Every mutant below is a copy of oracle/sdm_oracle.c with one planted error, built
+into a temporary library on the CPU.  At least one pin in tests/oracle_pins.py
+must fail for each, which shows the pins are strong enough to expose that class
+of mistake in the real oracle.
+"""
+import os
+
+import pytest
+
+import oracle
+from tests import oracle_pins
+
+MUTANTS = {
+    "error_sign_flipped": [
+        ("e[c] = v[(size_t)t * dv + c] - p[c];", "e[c] = p[c] - v[(size_t)t * dv + c];"),
+        ("e[c] = v[(size_t)t * dv + c] - p;", "e[c] = p - v[(size_t)t * dv + c];"),
+    ],
+    "decay_dropped": [
+        ("M[q] *= alpha[t];", "M[q] *= 1.0;"),
+        ("L += log(alpha[t]);", "L += 0.0;"),
+    ],
+    "beta_ignored": [
+        ("M[(size_t)ws[i] * dv + c] += beta[t] *", "M[(size_t)ws[i] * dv + c] += 1.0 *"),
+        ("seen[(size_t)i * dv + c] + beta[t] *", "seen[(size_t)i * dv + c] + 1.0 *"),
+    ],
+    "halves_swapped": [
+        ("s1[i] = dot(x, c1 + (size_t)i * hd, hd);", "s1[i] = dot(x + hd, c1 + (size_t)i * hd, hd);"),
+        ("s2[j] = dot(x + hd, c2 + (size_t)j * hd, hd);", "s2[j] = dot(x, c2 + (size_t)j * hd, hd);"),
+    ],
+    "slot_numbering_transposed": [
+        ("cand[i * n + j].id = i * n + j;", "cand[i * n + j].id = j * n + i;"),
+        ("cand[a * k_half + b].id = i * n + j;", "cand[a * k_half + b].id = j * n + i;"),
+    ],
+    "tie_order_reversed": [
+        ("if (a->id < b->id) return -1;\n    if (a->id > b->id) return 1;",
+         "if (a->id < b->id) return 1;\n    if (a->id > b->id) return -1;"),
+    ],
+    "softmax_unnormalised": [
+        ("for (int i = 0; i < m; ++i) w[i] /= z;", "for (int i = 0; i < m; ++i) w[i] /= 1.0;"),
+    ],
+    "first_weight_everywhere": [
+        ("p[c] += ww[(size_t)t * W + i] *", "p[c] += ww[(size_t)t * W] *"),
+        ("p += ww[(size_t)t * W + i] *", "p += ww[(size_t)t * W] *"),
+    ],
+    "lazy_stamp_not_updated": [
+        ("stamp[ws[i]] = L;", "(void)0;"),
+    ],
+    "pk_shortlist_short_by_one": [
+        ("for (int a = 0; a < k_half; ++a)\n            for (int b = 0; b < k_half; ++b) {",
+         "for (int a = 0; a < k_half; ++a)\n            for (int b = 0; b < k_half - (a == 0); ++b) {"),
+    ],
+    "read_weights_from_write": [
+        ("o += rw[(size_t)t * R + j] * M[(size_t)rs[j] * dv + c];",
+         "o += rw[(size_t)t * R + j] * M[(size_t)ws[j % W] * dv + c];"),
+        ("o += rw[(size_t)t * R + j] * Mraw[(size_t)rs[j] * dv + c] * exp(L - stamp[rs[j]]);",
+         "o += rw[(size_t)t * R + j] * Mraw[(size_t)ws[j % W] * dv + c] * exp(L - stamp[ws[j % W]]);"),
+    ],
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    with open(oracle.SRC) as f:
+        src = f.read()
+    for old, new in MUTANTS[name]:
+        assert old in src, f"mutation site not found for {name}: {old!r}"
+        src = src.replace(old, new)
+    path = tmp_path / f"mut_{name}.c"
+    path.write_text(src)
+    lib = oracle.build(force=True, src=str(path), out=str(tmp_path / f"libmut_{name}.so"))
+    o = oracle.Oracle(lib)
+    failed = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(o)
+        except (AssertionError, ValueError, IndexError):
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught mutant {name}"
