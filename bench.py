@@ -1,0 +1,455 @@
+"""Benchmark of the SDM (Sparse Delta Memory) prefill hot path on B200.
+
+One step = one fresh prefill of the mid-size workload (B=2 sequences, H=4 heads, T=4096
+tokens, d_k=128, n=256 sub-keys per half -> N=65,536 slots, d_v=128, k=W=R=32, bf16
+q/k/v, fp32 memory): state reset, product-key scoring of the keys (write slots) and the
+queries (read slots), the index-only plan and the recurrence row pass.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME]
+
+Under torchrun (N > 1) every rank runs its own independent batch (weak scaling, no
+collective on the data path); the timed region is bracketed by a barrier and a device
+synchronisation, and the reported time is the maximum over ranks.  Rank 0 prints one
+JSON line.  `--impl reference` times the CPU oracle on the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "SDM prefill tokens·heads/sec and achieved HBM GB/s (% of roofline), config 2"
+UNIT = "tokens·heads/s"
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+# DRAM traffic per launch of the recurrence row pass from an ncu capture (bytes), keyed by
+# the hash of the kernel sources it was taken with; None when not yet measured for the
+# current sources.  Filled from profiles/ (see the summary named there).
+MEASURED_TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_state_linear_score_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------ workload helpers ---
+
+def workload(name: str):
+    import sdm_synth as S
+    return S.WORKLOADS[name]
+
+
+def describe(wl) -> str:
+    return (f"{wl.name}: B={wl.B} H={wl.H} T={wl.T} d_k={wl.d_k} n={wl.n_sub} N={wl.N} "
+            f"d_v={wl.d_v} k={wl.k_half} W={wl.W} R={wl.R} q/k/v={wl.x_dtype}")
+
+
+def units_per_step(wl) -> int:
+    """tokens x heads processed by one step on one GPU."""
+    return wl.B * wl.H * wl.T
+
+
+def bytes_per_token_head(wl) -> dict:
+    """Algorithmic HBM bytes per token.head (no re-reads, no plan records)."""
+    xb = 2 if wl.x_dtype == "bf16" else 4
+    vb = 2 if wl.v_dtype == "bf16" else 4
+    rows = (2 * wl.W + wl.R) * wl.d_v * 4          # W gathers + W scatters + R gathers, fp32 rows
+    scoring_io = 2 * wl.d_k * xb + (wl.W + wl.R) * 8  # read q, k; write idx + weights
+    recur_io = (wl.W + wl.R) * 8 + wl.d_v * vb + 8 + wl.d_v * 4  # read idx+w, v, alpha+beta; write out
+    return {"rows": rows, "scoring_io": scoring_io, "recur_io": recur_io,
+            "recurrence_kernel": rows + recur_io, "step": rows + scoring_io + recur_io}
+
+
+def scoring_flops_per_token_head(wl) -> int:
+    return 2 * 2 * wl.n_sub * wl.hd * 2  # two roles x two halves x n x h MACs x 2
+
+
+def rank_seed(wl, rank: int) -> int:
+    """Each rank draws an independent batch of sequences (weak scaling)."""
+    return wl.seed + 7919 * rank
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+# --------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self._t:
+            self._t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- distributed ---
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(value: float, device) -> float:
+    """Maximum of a per-rank float over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------- GPU arm ---
+
+def run_gpu(args, wl, world, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    import sdm_synth as S
+    import sparse_state_linear_score_b200 as sdm
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    stream = torch.cuda.current_stream()
+
+    inp = S.generate(wl, device=device, seed=rank_seed(wl, rank))
+    d = sdm.Dims(wl.B, wl.H, wl.T, wl.d_k, wl.n_sub, wl.d_v, wl.k_half, wl.W, wl.R, wl.x_dtype,
+                 wl.v_dtype)
+    st = sdm.State(d, inp["M0"])
+    sel = sdm.selection_buffers(d, device)
+    widx, ww, ridx, rw = sel
+    out = torch.empty((wl.B, wl.H, wl.T, wl.d_v), dtype=torch.float32, device=device)
+    ws = sdm.workspace(d, device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def step(ev=None):
+        # ev: (start, after_scoring, before_run, end) events or None
+        if ev:
+            ev[0].record(stream)
+        sdm.state_reset(d, st)
+        sdm.score_topk(d, inp["k"], inp["skw"], wl.W, widx, ww)
+        sdm.score_topk(d, inp["q"], inp["skr"], wl.R, ridx, rw)
+        if ev:
+            ev[1].record(stream)
+        sdm.forward_plan(d, inp["alpha"], widx, ridx, st, ws)
+        if ev:
+            ev[2].record(stream)
+        sdm.forward_run(d, inp["v"], inp["beta"], widx, ww, ridx, rw, st, out, ws)
+        if ev:
+            ev[3].record(stream)
+
+    warm = max(3, args.warmup)
+    for _ in range(warm):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert sdm.device_error() == 0, "device error during warm-up"
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(device.index if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                          int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[device.index]))
+    clocks.start()
+    barrier(device)
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush.zero_()  # L2 flush between timed steps, outside the step's events
+        step(evs[k])
+    torch.cuda.synchronize()
+    barrier(device)
+    clk = clocks.stop()
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    score_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    plan_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    run_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms = reduce_max(sum(step_ms), device)
+    launches_per_step = 6  # reset, 2 x score, plan_local, plan_walk, run
+
+    # end to end through the public API with host buffers
+    e2e = run_e2e(args, wl, d, inp, st, sel, out, ws, device, sdm)
+    errs = sdm.device_error()
+
+    if world > 1:
+        dist.barrier(device_ids=[device.index])
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    units = units_per_step(wl) * world
+    peaks = measured_peaks()
+    bpt = bytes_per_token_head(wl)
+    run_avg_s = statistics.mean(run_ms) / 1e3
+    run_bytes = bpt["recurrence_kernel"] * units_per_step(wl)
+    achieved = run_bytes / run_avg_s / 1e9
+    step_avg_s = statistics.mean(step_ms) / 1e3
+    step_gbs = bpt["step"] * units_per_step(wl) / step_avg_s / 1e9
+    score_tflops = (scoring_flops_per_token_head(wl) * units_per_step(wl) /
+                    (statistics.mean(score_ms) / 1e3) / 1e12)
+    traffic = MEASURED_TRAFFIC.get(kernel_source_hash())
+    line = {
+        "metric": METRIC,
+        "value": units * args.steps / (total_ms / 1e3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": warm,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded; shapes and distributions of the mid-size prefill workload)",
+        "config": {"workload": describe(wl), "inputs": "bf16 q/k/v and sub-keys, fp32 gates",
+                   "state": "fp32 rows, fp64 stamps, reset every step",
+                   "l2": "flushed between timed steps (256 MB write outside the step events)",
+                   "parallelism": f"dp{world} (independent sequences per rank)"},
+        "roofline": {"bound": "hbm", "kernel": "recur_run_kernel (sdm_forward_run)",
+                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "peak_source": peaks["source"] + " (burst copy)",
+                     "algorithmic_bytes_per_launch": run_bytes},
+        "step_roofline": {"achieved_gbs": step_gbs, "frac": step_gbs / peaks["hbm_gbs"],
+                          "bytes_per_token_head": bpt["step"]},
+        "stages_ms": {"reset_and_scoring": statistics.mean(score_ms),
+                      "plan": statistics.mean(plan_ms), "run": statistics.mean(run_ms)},
+        "scoring": {"tflops": score_tflops, "frac_of_bf16_peak": score_tflops / peaks["bf16_tflops"]},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "device_errors": errs,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    return line
+
+
+def run_e2e(args, wl, d, inp, st, sel, out, ws, device, sdm):
+    """Same metric through sdm.prefill with pinned host inputs copied in and the output
+    copied out inside the timed region."""
+    import torch
+    names = ("q", "k", "v", "alpha", "beta")
+    host = {n: inp[n].cpu().pin_memory() for n in names}
+    dev = {n: torch.empty_like(inp[n]) for n in names}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    stream = torch.cuda.current_stream()
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    d2h = out_h.numel() * out_h.element_size()
+
+    def step():
+        for n in names:
+            dev[n].copy_(host[n], non_blocking=True)
+        sdm.state_reset(d, st)
+        sdm.prefill(d, dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], inp["skw"],
+                    inp["skr"], st, sel=sel, out=out, ws=ws)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    steps = max(1, args.steps)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(device)
+    ms = reduce_max(t0.elapsed_time(t1), device)
+    world = dist_world()
+    return {"value": units_per_step(wl) * world * steps / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms / steps}
+
+
+def dist_world() -> int:
+    import torch.distributed as dist
+    return dist.get_world_size() if dist.is_available() and dist.is_initialized() else 1
+
+
+# ------------------------------------------------------------ CPU oracle arm ---
+
+def cpu_baseline(wl, seconds: float = 15.0, seed: int | None = None) -> dict:
+    """The CPU oracle (fp64 C, OpenMP over sequences) timed on this host on a bounded
+    sample of the same workload: token prefixes of B*H sequences, product-key scoring of
+    both roles and the lazy recurrence from M0."""
+    import numpy as np
+
+    import oracle
+    import sdm_synth as S
+    orc = oracle.default()
+    cores = orc.max_threads()
+    pairs = [(b, h) for b in range(wl.B) for h in range(wl.H)]
+    # calibrate on a short prefix
+    T_cal = min(wl.T, 64)
+    small = S.generate(wl.scaled(T=T_cal), seed=seed)
+    arr = {k: v.double().numpy() for k, v in small.items()}
+    t0 = time.perf_counter()
+    orc.prefill_pairs(arr["q"], arr["k"], arr["v"], arr["alpha"], arr["beta"], arr["skw"],
+                      arr["skr"], arr["M0"], wl.k_half, wl.W, wl.R, pairs, nthreads=cores)
+    cal = time.perf_counter() - t0
+    per_token = cal / T_cal
+    T_s = int(max(T_cal, min(wl.T, seconds / max(per_token, 1e-9))))
+    samp = S.generate(wl.scaled(T=T_s), seed=seed)
+    arr = {k: v.double().numpy() for k, v in samp.items()}
+    t0 = time.perf_counter()
+    orc.prefill_pairs(arr["q"], arr["k"], arr["v"], arr["alpha"], arr["beta"], arr["skw"],
+                      arr["skr"], arr["M0"], wl.k_half, wl.W, wl.R, pairs, nthreads=cores)
+    el = time.perf_counter() - t0
+    units = len(pairs) * T_s
+    return {"value": units / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"first {T_s} of {wl.T} tokens of all {len(pairs)} (b,h) sequences "
+                      f"({units} token.heads, {el:.1f} s, fp64, OpenMP over sequences)"}
+
+
+def run_reference(args, wl, world, rank):
+    """--impl reference: the CPU oracle as it stands, on rank 0 only."""
+    if rank != 0:
+        return None
+    import oracle
+    cores = oracle.default().max_threads()
+    per_step = max(2.0, args.cpu_seconds / 4)
+    for _ in range(max(0, min(args.warmup, 1))):
+        cpu_baseline(wl, seconds=1.0)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r = cpu_baseline(wl, seconds=per_step)
+        vals.append(r)
+    el = time.perf_counter() - t0
+    value = statistics.mean(v["value"] for v in vals)
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / max(1, args.steps),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded; shapes and distributions of the mid-size prefill workload)",
+        "config": {"workload": describe(wl), "inputs": "bf16-rounded q/k/v and sub-keys, upcast to fp64",
+                   "parallelism": "CPU host cores (OpenMP over sequences)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": vals[-1]["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["sdm", "reference"], default="sdm")
+    ap.add_argument("--workload", default="mid_prefill")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    world, rank, local = dist_env()
+    if world != args.gpus and "WORLD_SIZE" in os.environ:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    wl = workload(args.workload)
+    if args.impl == "reference":
+        line = run_reference(args, wl, world, rank)
+    else:
+        line = run_gpu(args, wl, world, rank, local)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

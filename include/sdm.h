@@ -1,0 +1,220 @@
+/*
+ * sdm.h — C ABI of the Sparse Delta Memory (SDM) hot path on NVIDIA B200 (sm_100a).
+ *
+ * Sparse Delta Memory ("Sparse Delta Memory: Scaling the State of Linear RNNs
+ * through Sparsity", arXiv 2607.07386) replaces the dense Gated DeltaNet state
+ * with an N-slot memory table per head.  Each token selects W write slots from
+ * its key and R read slots from its query by product-key top-k scoring, applies
+ * a gated delta update to the W write slots and reads a weighted sum of the R
+ * read slots.  The library computes that path on the GPU:
+ *
+ *   sdm_score_topk   product-key scoring, per-half top-k, k x k combine,
+ *                    top-W (or top-R) slot indices and softmax weights
+ *   sdm_forward      the sparse gated-delta recurrence over T tokens (prefill)
+ *   sdm_decode_step  one token per sequence (scoring + recurrence)
+ *
+ * Notation: B sequences, H heads, T tokens, key width d_k (two halves of
+ * h = d_k/2), n sub-keys per half (N = n*n slots, slot s = i*n + j where i is
+ * the rank source of the first half), value width d_v, per-half top-k k_half,
+ * W write / R read slots per token, decay gate alpha in (0,1], input gate beta.
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer is caller-owned device memory (except where a comment says
+ *     host), contiguous, row-major, 16-byte aligned.  The library never allocates
+ *     device memory on a compute call; scratch comes from the caller through a
+ *     workspace whose size a *_workspace_bytes query returns.
+ *   - All GPU work is enqueued asynchronously on `stream` (a cudaStream_t; NULL
+ *     is the legacy default stream).  Arguments are validated on the host before
+ *     anything is enqueued; a failed validation enqueues nothing.
+ *   - Nothing aborts, traps or prints.  Problems found on the device (an
+ *     out-of-range slot index, a repeated write slot within one token, alpha <= 0)
+ *     set bits of a device error word, skip the offending access and let the
+ *     kernel finish; read the word with sdm_device_error.
+ *   - Dimensions supported: 1 <= W, R <= 64; 1 <= k_half <= min(n, 64);
+ *     top <= k_half^2; d_v a multiple of 4 with d_v <= 256; d_k even with
+ *     d_k/2 a multiple of 8 and d_k <= 256; 1 <= n <= 4096.
+ */
+#ifndef SDM_H
+#define SDM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st* sdm_stream_t;
+
+typedef enum {
+    SDM_OK = 0,
+    SDM_ERR_ARG = 1,        /* null pointer, negative size, unsupported option */
+    SDM_ERR_SHAPE = 2,      /* dimensions outside the supported ranges */
+    SDM_ERR_DTYPE = 3,      /* unknown dtype tag */
+    SDM_ERR_ALIGN = 4,      /* pointer not 16-byte aligned */
+    SDM_ERR_CUDA = 5,       /* a CUDA runtime call failed (launch, memset, ...) */
+    SDM_ERR_BAD_INDEX = 6,  /* returned by sdm_device_error when an index bit is set */
+    SDM_ERR_WORKSPACE = 7,  /* workspace missing or smaller than the query returned */
+    SDM_ERR_UNSUPPORTED = 8 /* valid request this build does not implement */
+} sdm_status;
+
+typedef enum { SDM_F32 = 0, SDM_BF16 = 1 } sdm_dtype;
+
+/* Bits of the device error word (sdm_device_error). */
+#define SDM_DEVERR_SLOT_RANGE 1u   /* a slot index outside [0, N) */
+#define SDM_DEVERR_DUP_WRITE 2u    /* a write slot repeated within one token */
+#define SDM_DEVERR_ALPHA 4u        /* alpha <= 0 (its log is undefined) */
+
+typedef struct {
+    int32_t B, H, T;   /* sequences, heads, tokens in this call (T = 1 for decode) */
+    int32_t d_k;       /* key / query width: two halves of d_k/2 */
+    int32_t n_sub;     /* sub-keys per half; N = n_sub^2 slots per head */
+    int32_t d_v;       /* value width = slot row width */
+    int32_t k_half;    /* per-half top-k */
+    int32_t W, R;      /* write and read slots per token */
+    int32_t x_dtype;   /* sdm_dtype of q, k and the sub-key tables */
+    int32_t v_dtype;   /* sdm_dtype of v */
+} sdm_dims;
+
+/*
+ * Memory state of B*H sequences, all caller-owned device memory.  It is kept in
+ * lazy-decay form so that no call ever sweeps the whole table:
+ *   M      [B][H][N][d_v] fp32  raw slot rows
+ *   stamp  [B][H][N]      fp64  log-decay prefix at the slot's last write;
+ *                               NaN marks a pristine slot whose value is M0
+ *   Lambda [B][H]         fp64  running log-decay prefix sum_t log(alpha_t)
+ *   M0     [H][N][d_v]    fp32  initial memory, shared by the batch (read only)
+ * The true value of slot s is  M[s] * exp(Lambda - stamp[s]),  or
+ * M0[h][s] * exp(Lambda) while the slot is pristine.  (The pages give the decay
+ * as a per-token multiplication of every slot; this form is equal to it.)
+ */
+typedef struct {
+    float* M;
+    double* stamp;
+    double* Lambda;
+    const float* M0;
+} sdm_state;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* sdm_status_str(int32_t status);
+
+/* ABI version of this library; bumped whenever a signature or layout changes. */
+int32_t sdm_abi_version(void);
+
+/*
+ * Bytes of each state array for `dims` (M, stamp, Lambda).  Host only.
+ * Returns SDM_ERR_ARG on NULL outputs, SDM_ERR_SHAPE on unsupported dims.
+ */
+sdm_status sdm_state_bytes(const sdm_dims* dims, size_t* M_bytes, size_t* stamp_bytes,
+                           size_t* lambda_bytes);
+
+/*
+ * Start B*H fresh sequences: every slot becomes pristine (its value is M0) and
+ * Lambda = 0.  Writes stamp and Lambda only — O(B*H*N) stamps, no row traffic.
+ * Source: §3 Method, "Learned initial state" (the memory starts from M0).
+ */
+sdm_status sdm_state_reset(const sdm_dims* dims, const sdm_state* st, sdm_stream_t stream);
+
+/*
+ * Dense memory of every sequence: M_out[b][h][s] = true value of slot s
+ * ([B][H][N][d_v] fp32, caller-owned device buffer, may not alias st->M).
+ * Sweeps the whole table; meant for checks, not for the hot path.
+ */
+sdm_status sdm_state_materialize(const sdm_dims* dims, const sdm_state* st, float* M_out,
+                                 sdm_stream_t stream);
+
+/*
+ * Product-key top-k scoring for one role (write: x = k, read: x = q).
+ * Source: §2 Background "Product Key Memory" and §3 Method "Sparse addressing";
+ * softmax weights per §4 "SDM Configuration".
+ *   x       [B][H][T][d_k]      dims->x_dtype
+ *   subkeys [H][2][n_sub][d_k/2] dims->x_dtype   (half 1 table, then half 2)
+ *   top     W for the write role, R for the read role (1 <= top <= 64)
+ *   idx     [B][H][T][top] int32 out: slot indices, best first
+ *   w       [B][H][T][top] fp32  out: softmax over the selected scores
+ * Score of slot s = i*n + j is <x[0:h], C1[i]> + <x[h:2h], C2[j]> (fp32
+ * accumulation of the stored inputs); larger first, equal scores to the lower
+ * slot.  The k_half best sub-keys per half are kept and their k_half^2 sums
+ * ranked; this equals ranking all N slots whenever k_half >= top.
+ */
+sdm_status sdm_score_topk(const sdm_dims* dims, const void* x, const void* subkeys, int32_t top,
+                          int32_t* idx, float* w, sdm_stream_t stream);
+
+/* Workspace bytes sdm_forward / sdm_prefill need for `dims` (0 on bad dims). */
+size_t sdm_forward_workspace_bytes(const sdm_dims* dims);
+
+/*
+ * Sparse gated-delta recurrence over T tokens (prefill), state updated in place.
+ * Source: §2 Background "Gated DeltaNet"; §3 Method "Sparse memory updates",
+ * "Sparse retrieval", "Connection to GDN".  Per token t, in order:
+ *   every slot decays by alpha_t; p = sum_i w_i M[s_i]; e = v_t - p;
+ *   M[s_i] += beta_t w_i e for the W (distinct) write slots;
+ *   out_t = sum_j u_j M[r_j]   (read after the write).
+ *   v      [B][H][T][d_v]  dims->v_dtype
+ *   alpha, beta [B][H][T]  fp32
+ *   widx, ww [B][H][T][W]  int32 / fp32   write slots and weights
+ *   ridx, rw [B][H][T][R]  int32 / fp32   read slots and weights
+ *   out    [B][H][T][d_v]  fp32 out
+ *   ws     workspace of at least sdm_forward_workspace_bytes(dims) bytes
+ * T = 0 is a valid no-op.
+ */
+sdm_status sdm_forward(const sdm_dims* dims, const void* v, const float* alpha, const float* beta,
+                       const int32_t* widx, const float* ww, const int32_t* ridx, const float* rw,
+                       const sdm_state* st, float* out, void* ws, size_t ws_bytes,
+                       sdm_stream_t stream);
+
+/*
+ * The two stages of sdm_forward, callable separately (same arguments):
+ *   sdm_forward_plan  index-only pass: per-occurrence decay factors from the
+ *                     slot stamps, in-chunk links between tokens that share a
+ *                     slot, new stamps and Lambda (writes ws, st->stamp,
+ *                     st->Lambda).
+ *   sdm_forward_run   the row pass: gathers, delta updates, scatters, outputs
+ *                     (reads ws, updates st->M, writes out).
+ * A run must follow the plan of the same call, on the same stream, with the
+ * same index arrays and unchanged ws.
+ */
+sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const int32_t* widx,
+                            const int32_t* ridx, const sdm_state* st, void* ws, size_t ws_bytes,
+                            sdm_stream_t stream);
+sdm_status sdm_forward_run(const sdm_dims* dims, const void* v, const float* beta,
+                           const int32_t* widx, const float* ww, const int32_t* ridx,
+                           const float* rw, const sdm_state* st, float* out, void* ws,
+                           size_t ws_bytes, sdm_stream_t stream);
+
+/*
+ * Prefill = sdm_score_topk(k, skw, W) + sdm_score_topk(q, skr, R) + sdm_forward.
+ *   q, k [B][H][T][d_k] (x_dtype); skw, skr [H][2][n_sub][d_k/2] (x_dtype)
+ *   widx/ww, ridx/rw: caller buffers that receive the selections (as above)
+ */
+sdm_status sdm_prefill(const sdm_dims* dims, const void* q, const void* k, const void* v,
+                       const float* alpha, const float* beta, const void* skw, const void* skr,
+                       const sdm_state* st, int32_t* widx, float* ww, int32_t* ridx, float* rw,
+                       float* out, void* ws, size_t ws_bytes, sdm_stream_t stream);
+
+/*
+ * One token for each of the B*H sequences (dims->T must be 1): scoring of k and
+ * q, then the same recurrence step as sdm_forward.  Layouts drop the T axis:
+ *   q, k [B][H][d_k]; v [B][H][d_v]; alpha, beta [B][H]; out [B][H][d_v];
+ *   widx/ww [B][H][W], ridx/rw [B][H][R] receive the selections.
+ * No workspace.  Equal to sdm_forward with T = 1 up to rounding order.
+ */
+sdm_status sdm_decode_step(const sdm_dims* dims, const void* q, const void* k, const void* v,
+                           const float* alpha, const float* beta, const void* skw,
+                           const void* skr, const sdm_state* st, int32_t* widx, float* ww,
+                           int32_t* ridx, float* rw, float* out, sdm_stream_t stream);
+
+/*
+ * Read the device error word into *bits (host pointer; SDM_DEVERR_* bits), then
+ * clear it when `clear` is non-zero.  Synchronises `stream`.  Returns SDM_OK when
+ * no bit is set, SDM_ERR_BAD_INDEX when any is, SDM_ERR_CUDA if the copy fails.
+ * The word is per device and shared by every call on that device.
+ */
+sdm_status sdm_device_error(uint32_t* bits, int32_t clear, sdm_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDM_H */

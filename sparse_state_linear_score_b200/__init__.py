@@ -1,0 +1,269 @@
+"""Sparse Delta Memory (SDM) hot path on NVIDIA B200 — Python binding of libsdm.so.
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels (see include/sdm.h).  PyTorch provides device memory and streams.  There
+is no CPU fallback: importing this package without a loadable libsdm.so raises.
+
+Typical use::
+
+    import sparse_state_linear_score_b200 as sdm
+    d = sdm.Dims(B, H, T, d_k, n_sub, d_v, k_half, W, R, x_dtype="bf16", v_dtype="bf16")
+    st = sdm.State(d, M0)                      # M0: [H, N, d_v] fp32 on the GPU
+    sdm.state_reset(d, st)
+    out, sel = sdm.prefill(d, q, k, v, alpha, beta, skw, skr, st)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+__all__ = ["Dims", "State", "SdmError", "state_reset", "state_materialize", "score_topk",
+           "forward_workspace_bytes", "forward", "forward_plan", "forward_run", "prefill",
+           "decode_step", "device_error", "lib_path", "DEVERR_SLOT_RANGE", "DEVERR_DUP_WRITE",
+           "DEVERR_ALPHA"]
+
+F32, BF16 = 0, 1
+_DT = {"f32": F32, "bf16": BF16, torch.float32: F32, torch.bfloat16: BF16}
+DEVERR_SLOT_RANGE, DEVERR_DUP_WRITE, DEVERR_ALPHA = 1, 2, 4
+
+
+class SdmError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_lib.sdm_status_str(status).decode()}")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "H", "T", "d_k", "n_sub", "d_v", "k_half", "W", "R", "x_dtype", "v_dtype")]
+
+    def __init__(self, B, H, T, d_k, n_sub, d_v, k_half, W, R, x_dtype="f32", v_dtype="f32"):
+        super().__init__(B, H, T, d_k, n_sub, d_v, k_half, W, R, _DT[x_dtype], _DT[v_dtype])
+
+    @property
+    def N(self) -> int:
+        return self.n_sub * self.n_sub
+
+    def with_T(self, T: int) -> "Dims":
+        x = Dims(self.B, self.H, T, self.d_k, self.n_sub, self.d_v, self.k_half, self.W, self.R)
+        x.x_dtype, x.v_dtype = self.x_dtype, self.v_dtype
+        return x
+
+
+class _CState(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_void_p), ("stamp", ctypes.c_void_p), ("Lambda", ctypes.c_void_p),
+                ("M0", ctypes.c_void_p)]
+
+
+def _load():
+    path = _build.LIB
+    if not os.path.exists(path) or not _build.up_to_date():
+        _build.build()  # raises if nvcc fails: no fallback path exists
+    lib = ctypes.CDLL(path)
+    P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    D = ctypes.POINTER(Dims)
+    S = ctypes.POINTER(_CState)
+    sig = {
+        "sdm_status_str": ([I32], ctypes.c_char_p),
+        "sdm_abi_version": ([], I32),
+        "sdm_state_bytes": ([D, P, P, P], I32),
+        "sdm_state_reset": ([D, S, P], I32),
+        "sdm_state_materialize": ([D, S, P, P], I32),
+        "sdm_score_topk": ([D, P, P, I32, P, P, P], I32),
+        "sdm_forward_workspace_bytes": ([D], SZ),
+        "sdm_forward": ([D, P, P, P, P, P, P, P, S, P, P, SZ, P], I32),
+        "sdm_forward_plan": ([D, P, P, P, S, P, SZ, P], I32),
+        "sdm_forward_run": ([D, P, P, P, P, P, P, S, P, P, SZ, P], I32),
+        "sdm_prefill": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P, SZ, P], I32),
+        "sdm_decode_step": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P], I32),
+        "sdm_device_error": ([ctypes.POINTER(ctypes.c_uint32), I32, P], I32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def _ptr(t: torch.Tensor | None, what: str, dtype=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{what} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ok(status: int, what: str):
+    if status != 0:
+        raise SdmError(status, what)
+
+
+def _xdt(d: Dims):
+    return torch.float32 if d.x_dtype == F32 else torch.bfloat16
+
+
+def _vdt(d: Dims):
+    return torch.float32 if d.v_dtype == F32 else torch.bfloat16
+
+
+class State:
+    """Lazy-decay memory state of B*H sequences (see include/sdm.h, sdm_state)."""
+
+    def __init__(self, d: Dims, M0: torch.Tensor, device=None):
+        device = M0.device if device is None else device
+        self.M = torch.empty((d.B, d.H, d.N, d.d_v), dtype=torch.float32, device=device)
+        self.stamp = torch.empty((d.B, d.H, d.N), dtype=torch.float64, device=device)
+        self.Lambda = torch.zeros((d.B, d.H), dtype=torch.float64, device=device)
+        if tuple(M0.shape) != (d.H, d.N, d.d_v):
+            raise ValueError(f"M0 must be [H, N, d_v] = {(d.H, d.N, d.d_v)}")
+        self.M0 = M0
+        self._c = _CState(_ptr(self.M, "M", torch.float32), _ptr(self.stamp, "stamp", torch.float64),
+                          _ptr(self.Lambda, "Lambda", torch.float64), _ptr(M0, "M0", torch.float32))
+
+    @property
+    def c(self) -> _CState:
+        return self._c
+
+
+def state_reset(d: Dims, st: State, stream=None):
+    _ok(_lib.sdm_state_reset(ctypes.byref(d), ctypes.byref(st.c), _stream(stream)), "sdm_state_reset")
+
+
+def state_materialize(d: Dims, st: State, out: torch.Tensor | None = None, stream=None):
+    if out is None:
+        out = torch.empty_like(st.M)
+    _ok(_lib.sdm_state_materialize(ctypes.byref(d), ctypes.byref(st.c), _ptr(out, "out"),
+                                   _stream(stream)), "sdm_state_materialize")
+    return out
+
+
+def score_topk(d: Dims, x, subkeys, top: int, idx=None, w=None, stream=None):
+    shape = (d.B, d.H, d.T, top)
+    if idx is None:
+        idx = torch.empty(shape, dtype=torch.int32, device=x.device)
+    if w is None:
+        w = torch.empty(shape, dtype=torch.float32, device=x.device)
+    _ok(_lib.sdm_score_topk(ctypes.byref(d), _ptr(x, "x", _xdt(d)), _ptr(subkeys, "subkeys", _xdt(d)),
+                            top, _ptr(idx, "idx", torch.int32), _ptr(w, "w", torch.float32),
+                            _stream(stream)), "sdm_score_topk")
+    return idx, w
+
+
+def forward_workspace_bytes(d: Dims) -> int:
+    return int(_lib.sdm_forward_workspace_bytes(ctypes.byref(d)))
+
+
+def workspace(d: Dims, device="cuda") -> torch.Tensor:
+    return torch.empty(max(16, forward_workspace_bytes(d)), dtype=torch.uint8, device=device)
+
+
+def _fw_args(d, v, alpha, beta, widx, ww, ridx, rw):
+    return (_ptr(v, "v", _vdt(d)), _ptr(alpha, "alpha", torch.float32), _ptr(beta, "beta", torch.float32),
+            _ptr(widx, "widx", torch.int32), _ptr(ww, "ww", torch.float32),
+            _ptr(ridx, "ridx", torch.int32), _ptr(rw, "rw", torch.float32))
+
+
+def forward(d: Dims, v, alpha, beta, widx, ww, ridx, rw, st: State, out=None, ws=None, stream=None):
+    if out is None:
+        out = torch.empty((d.B, d.H, d.T, d.d_v), dtype=torch.float32, device=v.device)
+    if ws is None:
+        ws = workspace(d, v.device)
+    a = _fw_args(d, v, alpha, beta, widx, ww, ridx, rw)
+    _ok(_lib.sdm_forward(ctypes.byref(d), *a, ctypes.byref(st.c), _ptr(out, "out", torch.float32),
+                         _ptr(ws, "ws"), ws.numel(), _stream(stream)), "sdm_forward")
+    return out
+
+
+def forward_plan(d: Dims, alpha, widx, ridx, st: State, ws, stream=None):
+    _ok(_lib.sdm_forward_plan(ctypes.byref(d), _ptr(alpha, "alpha", torch.float32),
+                              _ptr(widx, "widx", torch.int32), _ptr(ridx, "ridx", torch.int32),
+                              ctypes.byref(st.c), _ptr(ws, "ws"), ws.numel(), _stream(stream)),
+        "sdm_forward_plan")
+
+
+def forward_run(d: Dims, v, beta, widx, ww, ridx, rw, st: State, out, ws, stream=None):
+    _ok(_lib.sdm_forward_run(ctypes.byref(d), _ptr(v, "v", _vdt(d)), _ptr(beta, "beta", torch.float32),
+                             _ptr(widx, "widx", torch.int32), _ptr(ww, "ww", torch.float32),
+                             _ptr(ridx, "ridx", torch.int32), _ptr(rw, "rw", torch.float32),
+                             ctypes.byref(st.c), _ptr(out, "out", torch.float32), _ptr(ws, "ws"),
+                             ws.numel(), _stream(stream)), "sdm_forward_run")
+    return out
+
+
+def selection_buffers(d: Dims, device="cuda"):
+    """Caller buffers for the write / read selections of one call: widx, ww, ridx, rw."""
+    return (torch.empty((d.B, d.H, d.T, d.W), dtype=torch.int32, device=device),
+            torch.empty((d.B, d.H, d.T, d.W), dtype=torch.float32, device=device),
+            torch.empty((d.B, d.H, d.T, d.R), dtype=torch.int32, device=device),
+            torch.empty((d.B, d.H, d.T, d.R), dtype=torch.float32, device=device))
+
+
+def prefill(d: Dims, q, k, v, alpha, beta, skw, skr, st: State, sel=None, out=None, ws=None,
+            stream=None):
+    """Scoring of k and q, then the recurrence.  Returns (out, (widx, ww, ridx, rw))."""
+    dev = q.device
+    if sel is None:
+        sel = selection_buffers(d, dev)
+    if out is None:
+        out = torch.empty((d.B, d.H, d.T, d.d_v), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(d, dev)
+    widx, ww, ridx, rw = sel
+    xdt = _xdt(d)
+    _ok(_lib.sdm_prefill(ctypes.byref(d), _ptr(q, "q", xdt), _ptr(k, "k", xdt), _ptr(v, "v", _vdt(d)),
+                         _ptr(alpha, "alpha", torch.float32), _ptr(beta, "beta", torch.float32),
+                         _ptr(skw, "skw", xdt), _ptr(skr, "skr", xdt), ctypes.byref(st.c),
+                         _ptr(widx, "widx", torch.int32), _ptr(ww, "ww", torch.float32),
+                         _ptr(ridx, "ridx", torch.int32), _ptr(rw, "rw", torch.float32),
+                         _ptr(out, "out", torch.float32), _ptr(ws, "ws"), ws.numel(),
+                         _stream(stream)), "sdm_prefill")
+    return out, sel
+
+
+def decode_step(d: Dims, q, k, v, alpha, beta, skw, skr, st: State, sel=None, out=None,
+                stream=None):
+    """One token per sequence (d.T must be 1).  q, k: [B,H,d_k]; v: [B,H,d_v]; gates [B,H]."""
+    dev = q.device
+    if sel is None:
+        sel = selection_buffers(d, dev)
+    if out is None:
+        out = torch.empty((d.B, d.H, d.d_v), dtype=torch.float32, device=dev)
+    widx, ww, ridx, rw = sel
+    xdt = _xdt(d)
+    _ok(_lib.sdm_decode_step(ctypes.byref(d), _ptr(q, "q", xdt), _ptr(k, "k", xdt),
+                             _ptr(v, "v", _vdt(d)), _ptr(alpha, "alpha", torch.float32),
+                             _ptr(beta, "beta", torch.float32), _ptr(skw, "skw", xdt),
+                             _ptr(skr, "skr", xdt), ctypes.byref(st.c),
+                             _ptr(widx, "widx", torch.int32), _ptr(ww, "ww", torch.float32),
+                             _ptr(ridx, "ridx", torch.int32), _ptr(rw, "rw", torch.float32),
+                             _ptr(out, "out", torch.float32), _stream(stream)), "sdm_decode_step")
+    return out, sel
+
+
+def device_error(clear: bool = True, stream=None) -> int:
+    """The device error word (DEVERR_* bits); synchronises the stream."""
+    bits = ctypes.c_uint32(0)
+    st = _lib.sdm_device_error(ctypes.byref(bits), 1 if clear else 0, _stream(stream))
+    if st not in (0, 6):
+        raise SdmError(st, "sdm_device_error")
+    return int(bits.value)

@@ -1,0 +1,345 @@
+// Index-only planning pass of the prefill recurrence.
+//
+// The recurrence (§2 Background "Gated DeltaNet", §3 Method "Sparse memory updates")
+// is run chunk by chunk: C tokens gather their rows from the memory as it stood at
+// the chunk start, the dependencies between tokens of one chunk that share a slot
+// are resolved on chip, and every slot written in the chunk is stored once at the
+// chunk end.  Everything that depends only on indices and gates is computed here,
+// once per (b,h), and shared by all column blocks of the row pass:
+//
+//   plan_local (one CTA per chunk)
+//     lam[t]      = sum of log(alpha_u) from the chunk start to t (inclusive), fp32
+//     csum[j]     = the same sum over the whole chunk, fp64
+//     lk[o]       = for occurrence o (a write or read slot of a token in the chunk):
+//                   1 + the in-chunk index of the latest earlier write of that slot
+//                   (token < t for a write, token <= t for a read), 0 if none;
+//                   bit 16: o is the last write of its slot in the chunk (stores it);
+//                   bit 17: o's accumulated in-chunk delta must be kept (a later
+//                   occurrence links to it, or it stores and has a link)
+//     tmask[t]    = {write-link bits, read-link bits, keep-delta bits} over the W / R slots
+//     st0[o]      = the state's stamp of o's slot at call entry (NaN: pristine)
+//   plan_walk (one CTA per (b,h), chunks in order)
+//     Lstart[j]   = log-decay prefix at the start of chunk j (Lstart[0] = state Lambda)
+//     fe[o]       = exp(Lambda_t - stamp of the row o gathers); sign bit set when the
+//                   row is the pristine M0 row
+//     state stamps of the slots written in the call and the state Lambda are updated.
+//
+// In-chunk occurrence order: the nt*W write occurrences (token-major), then the nt*R
+// read occurrences.  In the per-(b,h) arrays fe / lk / st0 the T*W write entries come
+// first, then the T*R read entries.
+#pragma once
+
+#include <math.h>
+
+#include "common.cuh"
+
+namespace sdm {
+
+constexpr int PLAN_MAX_OCC = 2048;  // C*(W+R) never exceeds this
+constexpr int PLAN_HASH = 4096;     // hash buckets (>= 2 * max write occurrences)
+constexpr int PLAN_THREADS = 256;
+constexpr int WALK_THREADS = 1024;
+constexpr int WALK_MAXO = PLAN_MAX_OCC / WALK_THREADS;
+
+constexpr unsigned LK_OWNER = 1u << 16;
+constexpr unsigned LK_KEEP = 1u << 17;
+
+SDM_DEV int lk_link(int lk) { return (lk & 0xffff) - 1; }
+
+SDM_DEV unsigned slot_hash(int s) { return ((unsigned)s * 2654435761u) >> (32 - 12); }
+
+// Inclusive block-wide prefix sum of doubles held one per thread (blockDim.x <= 1024).
+SDM_DEV double block_inclusive_scan(double v, double* warp_tot) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const double u = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += u;
+    }
+    if (lane == 31) warp_tot[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        const int nwarps = blockDim.x >> 5;
+        double t = lane < nwarps ? warp_tot[lane] : 0.0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const double u = __shfl_up_sync(0xffffffffu, t, off);
+            if (lane >= off) t += u;
+        }
+        if (lane < nwarps) warp_tot[lane] = t;
+    }
+    __syncthreads();
+    if (warp > 0) v += warp_tot[warp - 1];
+    __syncthreads();
+    return v;
+}
+
+struct PlanPtrs {
+    float* lam;        // [BH][T]
+    double* csum;      // [BH][J]
+    double* Lstart;    // [BH][J+1]
+    double* st0;       // [BH][T*(W+R)]
+    float* fe;         // [BH][T*(W+R)]
+    int32_t* lk;       // [BH][T*(W+R)]
+    uint64_t* tmask;   // [BH][T][3]
+    int32_t* lastw;    // [BH][N] (only when the walk table does not fit in shared memory)
+};
+
+__global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
+    const float* __restrict__ alpha, const int32_t* __restrict__ widx,
+    const int32_t* __restrict__ ridx, const double* __restrict__ stamp, int T, int N, int W,
+    int R, int C, int J, PlanPtrs P) {
+    __shared__ double s_wtot[32];
+    __shared__ int s_slot[PLAN_MAX_OCC];
+    __shared__ short s_link[PLAN_MAX_OCC];
+    __shared__ int s_head[PLAN_HASH];  // atomicExch needs 32-bit words
+    __shared__ short s_next[PLAN_MAX_OCC];
+    __shared__ unsigned char s_need[PLAN_MAX_OCC];
+    __shared__ unsigned char s_owner[PLAN_MAX_OCC];
+    __shared__ unsigned long long s_mask[3 * PLAN_THREADS];
+
+    const int j = blockIdx.x;
+    const size_t bh = blockIdx.y;
+    const int tid = threadIdx.x;
+    const int t0 = j * C;
+    const int nt = min(C, T - t0);
+    const int nw = nt * W, no = nt * (W + R);
+    const size_t occ_base = bh * (size_t)T * (W + R);
+
+    // 1. chunk-relative log-decay prefix (C <= PLAN_THREADS tokens per chunk)
+    double la = 0.0;
+    if (tid < nt) {
+        const float a = alpha[bh * T + t0 + tid];
+        if (a > 0.f) {
+            la = log((double)a);
+        } else {
+            raise_err(SDM_DEVERR_ALPHA);  // treated as alpha = 1
+        }
+    }
+    const double pre = block_inclusive_scan(la, s_wtot);
+    if (tid < nt) P.lam[bh * T + t0 + tid] = (float)pre;
+    if (tid == nt - 1) P.csum[bh * J + j] = pre;
+
+    // 2. slots of the chunk, hash heads, masks
+    for (int o = tid; o < no; o += PLAN_THREADS) {
+        int s;
+        if (o < nw) s = widx[(bh * T + t0) * W + o];
+        else s = ridx[(bh * T + t0) * R + (o - nw)];
+        if (!slot_ok(s, N)) {
+            raise_err(SDM_DEVERR_SLOT_RANGE);
+            s = -1;
+        }
+        s_slot[o] = s;
+        s_need[o] = 0;
+        s_owner[o] = 0;
+    }
+    for (int i = tid; i < PLAN_HASH; i += PLAN_THREADS) s_head[i] = -1;
+    for (int i = tid; i < 3 * nt; i += PLAN_THREADS) s_mask[i] = 0ull;
+    __syncthreads();
+
+    // 3. insert the write occurrences into per-bucket lists
+    for (int o = tid; o < nw; o += PLAN_THREADS) {
+        const int s = s_slot[o];
+        if (s >= 0) s_next[o] = (short)atomicExch(&s_head[slot_hash(s)], o);
+    }
+    __syncthreads();
+
+    // 4. links: latest earlier write of the same slot; owner = no later write in chunk
+    for (int o = tid; o < no; o += PLAN_THREADS) {
+        const int s = s_slot[o];
+        int link = -1;
+        if (s >= 0) {
+            const bool is_w = o < nw;
+            const int tl = is_w ? o / W : (o - nw) / R;
+            int best_t = -1;
+            bool later = false;
+            for (int p = s_head[slot_hash(s)]; p >= 0; p = s_next[p]) {
+                if (s_slot[p] != s) continue;
+                const int tp = p / W;
+                if (is_w) {
+                    if (tp == tl && p != o) raise_err(SDM_DEVERR_DUP_WRITE);
+                    if (tp > tl) later = true;
+                    if (tp < tl && tp > best_t) {
+                        best_t = tp;
+                        link = p;
+                    }
+                } else if (tp <= tl && tp > best_t) {
+                    best_t = tp;
+                    link = p;
+                }
+            }
+            if (is_w && !later) s_owner[o] = 1;
+            if (link >= 0) s_need[link] = 1;
+        }
+        s_link[o] = (short)link;
+    }
+    __syncthreads();
+
+    // 5. per-token masks
+    for (int o = tid; o < no; o += PLAN_THREADS) {
+        const int link = s_link[o];
+        if (o < nw) {
+            const int tl = o / W, i = o % W;
+            if (link >= 0) atomicOr(&s_mask[3 * tl + 0], 1ull << i);
+            if (s_need[o] || (s_owner[o] && link >= 0)) atomicOr(&s_mask[3 * tl + 2], 1ull << i);
+        } else if (link >= 0) {
+            const int tl = (o - nw) / R, jj = (o - nw) % R;
+            atomicOr(&s_mask[3 * tl + 1], 1ull << jj);
+        }
+    }
+    __syncthreads();
+
+    // 6. write out
+    for (int o = tid; o < no; o += PLAN_THREADS) {
+        const int link = s_link[o];
+        unsigned v = (unsigned)(link + 1);
+        size_t g;
+        if (o < nw) {
+            const int tl = o / W;
+            if (s_owner[o]) v |= LK_OWNER;
+            if (s_need[o] || (s_owner[o] && link >= 0)) v |= LK_KEEP;
+            g = occ_base + (size_t)t0 * W + o;
+            (void)tl;
+        } else {
+            g = occ_base + (size_t)T * W + (size_t)t0 * R + (o - nw);
+        }
+        P.lk[g] = (int32_t)v;
+        const int s = s_slot[o];
+        P.st0[g] = s >= 0 ? stamp[bh * (size_t)N + s] : 0.0;
+    }
+    for (int i = tid; i < 3 * nt; i += PLAN_THREADS)
+        P.tmask[(bh * T + t0) * 3 + i] = s_mask[i];
+}
+
+// Sequential walk over the chunks of one (b,h).  Table: last chunk of this call that
+// wrote each slot (-1: none), in shared memory (int16) when N <= walk_smem_slots, else
+// in the global workspace (int32, set to -1 by the host before the launch).
+template <bool SMEM_TABLE>
+__global__ void __launch_bounds__(WALK_THREADS) plan_walk_kernel(
+    const int32_t* __restrict__ widx, const int32_t* __restrict__ ridx, double* __restrict__ stamp,
+    double* __restrict__ lambda, int T, int N, int W, int R, int C, int J, int lstart_smem,
+    PlanPtrs P) {
+    extern __shared__ __align__(16) unsigned char walk_smem[];
+    __shared__ double s_wtot[32];
+    const size_t bh = blockIdx.x;
+    const int tid = threadIdx.x;
+    double* s_L = reinterpret_cast<double*>(walk_smem);  // [J+1] when lstart_smem
+    short* s_tab = reinterpret_cast<short*>(walk_smem + (lstart_smem ? (size_t)(J + 1) * 8 : 0));
+    int32_t* g_tab = P.lastw + bh * (size_t)N;
+    double* Lg = P.Lstart + bh * (size_t)(J + 1);
+    const size_t occ_base = bh * (size_t)T * (W + R);
+
+    // 1. chunk-start prefixes: Lstart[0] = Lambda, Lstart[j+1] = Lstart[j] + csum[j]
+    {
+        const int per = (J + WALK_THREADS - 1) / WALK_THREADS;
+        const int a = tid * per, b = min(J, a + per);
+        double part = 0.0;
+        for (int i = a; i < b; ++i) part += P.csum[bh * J + i];
+        const double incl = block_inclusive_scan(part, s_wtot);
+        double run = lambda[bh] + (incl - part);
+        if (tid == 0) {
+            Lg[0] = lambda[bh];
+            if (lstart_smem) s_L[0] = lambda[bh];
+        }
+        for (int i = a; i < b; ++i) {
+            run += P.csum[bh * J + i];
+            Lg[i + 1] = run;
+            if (lstart_smem) s_L[i + 1] = run;
+        }
+    }
+    if (SMEM_TABLE)
+        for (int i = tid; i < N; i += WALK_THREADS) s_tab[i] = -1;
+    __syncthreads();
+    const double* Lr = lstart_smem ? s_L : Lg;
+
+    // 2. chunks in order; each thread owns occurrences tid and tid + WALK_THREADS
+    int cs[WALK_MAXO], ck[WALK_MAXO];
+    double cst[WALK_MAXO];
+    float clam[WALK_MAXO];
+    size_t cg[WALK_MAXO];
+    auto fetch = [&](int j, int* s_, int* k_, double* st_, float* lm_, size_t* g_) {
+        const int t0 = j * C, nt = min(C, T - t0), nw = nt * W, no = nt * (W + R);
+#pragma unroll
+        for (int m = 0; m < WALK_MAXO; ++m) {
+            const int o = tid + m * WALK_THREADS;
+            s_[m] = -1;
+            if (o < no) {
+                size_t g;
+                int t;
+                if (o < nw) {
+                    g = occ_base + (size_t)t0 * W + o;
+                    s_[m] = widx[(bh * T + t0) * W + o];
+                    t = t0 + o / W;
+                } else {
+                    g = occ_base + (size_t)T * W + (size_t)t0 * R + (o - nw);
+                    s_[m] = ridx[(bh * T + t0) * R + (o - nw)];
+                    t = t0 + (o - nw) / R;
+                }
+                k_[m] = P.lk[g];
+                st_[m] = P.st0[g];
+                lm_[m] = P.lam[bh * T + t];
+                g_[m] = g;
+            }
+        }
+    };
+    if (J > 0) fetch(0, cs, ck, cst, clam, cg);
+    for (int j = 0; j < J; ++j) {
+        int ns[WALK_MAXO], nk[WALK_MAXO];
+        double nst[WALK_MAXO];
+        float nlam[WALK_MAXO];
+        size_t ng[WALK_MAXO];
+        if (j + 1 < J) fetch(j + 1, ns, nk, nst, nlam, ng);
+        const double Lj = Lr[j];
+#pragma unroll
+        for (int m = 0; m < WALK_MAXO; ++m) {
+            const int s = cs[m];
+            if (!slot_ok(s, N)) {
+                if (tid + m * WALK_THREADS < min(C, T - j * C) * (W + R)) P.fe[cg[m]] = 0.f;
+                continue;
+            }
+            const int jw = SMEM_TABLE ? (int)s_tab[s] : __ldcg(g_tab + s);
+            double stp;
+            bool m0 = false;
+            if (jw >= 0) {
+                stp = Lr[jw + 1];
+            } else if (isnan(cst[m])) {
+                stp = 0.0;
+                m0 = true;
+            } else {
+                stp = cst[m];
+            }
+            const float f = (float)exp(Lj + (double)clam[m] - stp);
+            P.fe[cg[m]] = m0 ? -f : f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < WALK_MAXO; ++m) {
+            const int s = cs[m];
+            if (slot_ok(s, N) && (ck[m] & LK_OWNER)) {
+                if (SMEM_TABLE) s_tab[s] = (short)j;
+                else __stcg(g_tab + s, j);
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < WALK_MAXO; ++m) {
+            cs[m] = ns[m];
+            ck[m] = nk[m];
+            cst[m] = nst[m];
+            clam[m] = nlam[m];
+            cg[m] = ng[m];
+        }
+    }
+
+    // 3. final stamps of the slots written in this call, and the new Lambda
+    for (size_t o = tid; o < (size_t)T * W; o += WALK_THREADS) {
+        const int s = widx[bh * (size_t)T * W + o];
+        if (!slot_ok(s, N) || !(P.lk[occ_base + o] & LK_OWNER)) continue;
+        const int j = (int)(o / W) / C;
+        const int jw = SMEM_TABLE ? (int)s_tab[s] : __ldcg(g_tab + s);
+        if (jw == j) stamp[bh * (size_t)N + s] = Lr[j + 1];
+    }
+    if (tid == 0) lambda[bh] = Lr[J];
+}
+
+}  // namespace sdm

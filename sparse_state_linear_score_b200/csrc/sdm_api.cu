@@ -1,0 +1,379 @@
+// C ABI of the SDM hot path (declared in include/sdm.h): host-side validation,
+// workspace layout and kernel launches.  One translation unit holds every kernel.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "plan.cuh"
+#include "recur.cuh"
+#include "score_simt.cuh"
+#include "state.cuh"
+
+using namespace sdm;
+
+namespace {
+
+constexpr int kMaxTop = 64;
+constexpr size_t kSmemBudget = 200 * 1024;  // dynamic shared memory per CTA we plan for
+constexpr int kWalkSmemSlots = 65536;        // walk table in shared memory up to this N
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+sdm_status check_dims(const sdm_dims* d) {
+    if (!d) return SDM_ERR_ARG;
+    if (d->x_dtype != SDM_F32 && d->x_dtype != SDM_BF16) return SDM_ERR_DTYPE;
+    if (d->v_dtype != SDM_F32 && d->v_dtype != SDM_BF16) return SDM_ERR_DTYPE;
+    if (d->B < 1 || d->H < 1 || d->T < 0) return SDM_ERR_SHAPE;
+    if ((long long)d->B * d->H > 65535) return SDM_ERR_SHAPE;
+    if (d->d_k < 16 || d->d_k > 256 || (d->d_k / 2) % 8 != 0 || d->d_k % 2 != 0) return SDM_ERR_SHAPE;
+    if (d->n_sub < 1 || d->n_sub > 4096) return SDM_ERR_SHAPE;
+    if (d->d_v < 4 || d->d_v > 256 || d->d_v % 4 != 0) return SDM_ERR_SHAPE;
+    if (d->k_half < 1 || d->k_half > 64 || d->k_half > d->n_sub) return SDM_ERR_SHAPE;
+    if (d->W < 1 || d->W > kMaxTop || d->R < 1 || d->R > kMaxTop) return SDM_ERR_SHAPE;
+    if (d->W > d->k_half * d->k_half || d->R > d->k_half * d->k_half) return SDM_ERR_SHAPE;
+    return SDM_OK;
+}
+
+inline long long N_of(const sdm_dims* d) { return (long long)d->n_sub * d->n_sub; }
+inline long long BH_of(const sdm_dims* d) { return (long long)d->B * d->H; }
+inline int col_width(const sdm_dims* d) { return d->d_v % 8 == 0 ? 8 : 4; }
+
+// Tokens per chunk of the prefill recurrence: as many as fit the plan's occurrence
+// budget, the run kernel's shared memory and the 256-token scan of plan_local.
+int chunk_tokens(const sdm_dims* d) {
+    const int CW = col_width(d);
+    int C = PLAN_MAX_OCC / (d->W + d->R);
+    if (C > PLAN_THREADS) C = PLAN_THREADS;
+    while (C > 1 && run_smem_bytes(C, d->W, d->R, CW) > kSmemBudget) --C;
+    return C < 1 ? 1 : C;
+}
+
+struct WsLayout {
+    int C, J;
+    bool smem_table, lstart_smem;
+    size_t walk_smem;
+    size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_tmask, off_lastw, total;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+WsLayout ws_layout(const sdm_dims* d) {
+    WsLayout L{};
+    const size_t BH = (size_t)BH_of(d), T = (size_t)d->T, N = (size_t)N_of(d);
+    const size_t occ = T * (size_t)(d->W + d->R);
+    L.C = chunk_tokens(d);
+    L.J = (int)((T + L.C - 1) / L.C);
+    L.smem_table = N <= (size_t)kWalkSmemSlots && L.J <= 32767;
+    const size_t tab_bytes = L.smem_table ? N * 2 : 0;
+    L.lstart_smem = (size_t)(L.J + 1) * 8 + tab_bytes <= kSmemBudget;
+    L.walk_smem = (L.lstart_smem ? (size_t)(L.J + 1) * 8 : 0) + tab_bytes;
+    size_t o = 0;
+    L.off_lam = o;    o = up256(o + BH * T * 4);
+    L.off_csum = o;   o = up256(o + BH * L.J * 8);
+    L.off_Lstart = o; o = up256(o + BH * (L.J + 1) * 8);
+    L.off_st0 = o;    o = up256(o + BH * occ * 8);
+    L.off_fe = o;     o = up256(o + BH * occ * 4);
+    L.off_lk = o;     o = up256(o + BH * occ * 4);
+    L.off_tmask = o;  o = up256(o + BH * T * 3 * 8);
+    L.off_lastw = o;  o = up256(o + (L.smem_table ? 0 : BH * N * 4));
+    L.total = o;
+    return L;
+}
+
+PlanPtrs plan_ptrs(const WsLayout& L, void* ws) {
+    unsigned char* b = static_cast<unsigned char*>(ws);
+    PlanPtrs P;
+    P.lam = reinterpret_cast<float*>(b + L.off_lam);
+    P.csum = reinterpret_cast<double*>(b + L.off_csum);
+    P.Lstart = reinterpret_cast<double*>(b + L.off_Lstart);
+    P.st0 = reinterpret_cast<double*>(b + L.off_st0);
+    P.fe = reinterpret_cast<float*>(b + L.off_fe);
+    P.lk = reinterpret_cast<int32_t*>(b + L.off_lk);
+    P.tmask = reinterpret_cast<uint64_t*>(b + L.off_tmask);
+    P.lastw = reinterpret_cast<int32_t*>(b + L.off_lastw);
+    return P;
+}
+
+sdm_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? SDM_OK : SDM_ERR_CUDA;
+}
+
+template <typename K>
+bool set_smem(K kernel, size_t bytes) {
+    if (bytes <= 48 * 1024) return true;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) ==
+           cudaSuccess;
+}
+
+sdm_status check_state(const sdm_state* st) {
+    if (!st || !st->M || !st->stamp || !st->Lambda || !st->M0) return SDM_ERR_ARG;
+    if (!aligned16(st->M) || !aligned16(st->stamp) || !aligned16(st->M0)) return SDM_ERR_ALIGN;
+    if (((uintptr_t)st->Lambda & 7u) != 0) return SDM_ERR_ALIGN;
+    return SDM_OK;
+}
+
+sdm_status launch_score(const sdm_dims* d, const void* x, const void* sk, int top, int32_t* idx,
+                        float* w, cudaStream_t s) {
+    const long long rows = (long long)d->B * d->T;
+    if (rows == 0) return SDM_OK;
+    const int threads = 128, warps = threads / 32;
+    const size_t smem =
+        (size_t)warps * score_simt_warp_floats(d->d_k, d->n_sub, d->k_half, top) * sizeof(float);
+    long long gx = (rows + warps * 4 - 1) / (warps * 4);
+    if (gx > 65535LL * 16) gx = 65535LL * 16;
+    dim3 grid((unsigned)gx, (unsigned)d->H);
+    if (d->x_dtype == SDM_F32) {
+        if (!set_smem(score_simt_kernel<float>, smem)) return SDM_ERR_CUDA;
+        score_simt_kernel<float><<<grid, threads, smem, s>>>(
+            (const float*)x, (const float*)sk, d->B, d->H, d->T, d->d_k, d->n_sub, d->k_half, top,
+            idx, w);
+    } else {
+        if (!set_smem(score_simt_kernel<__nv_bfloat16>, smem)) return SDM_ERR_CUDA;
+        score_simt_kernel<__nv_bfloat16><<<grid, threads, smem, s>>>(
+            (const __nv_bfloat16*)x, (const __nv_bfloat16*)sk, d->B, d->H, d->T, d->d_k, d->n_sub,
+            d->k_half, top, idx, w);
+    }
+    return launch_status();
+}
+
+template <int CW, typename VT>
+sdm_status launch_run_t(const sdm_dims* d, const WsLayout& L, const PlanPtrs& P, const void* v,
+                        const float* beta, const int32_t* widx, const float* ww,
+                        const int32_t* ridx, const float* rw, const sdm_state* st, float* out,
+                        cudaStream_t s) {
+    const size_t smem = run_smem_bytes(L.C, d->W, d->R, CW);
+    auto kern = recur_run_kernel<CW, VT>;
+    if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
+    const long long grid = BH_of(d) * (d->d_v / CW);
+    kern<<<(unsigned)grid, RUN_THREADS, smem, s>>>(
+        (const VT*)v, beta, widx, ww, ridx, rw, P.fe, P.lk, P.lam,
+        reinterpret_cast<const unsigned long long*>(P.tmask), st->M, st->M0, out, d->H, d->T,
+        (int)N_of(d), d->d_v, d->W, d->R, L.C, L.J);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sdm_status_str(int32_t status) {
+    switch (status) {
+        case SDM_OK: return "SDM_OK";
+        case SDM_ERR_ARG: return "SDM_ERR_ARG: null pointer or invalid argument";
+        case SDM_ERR_SHAPE: return "SDM_ERR_SHAPE: dimensions outside the supported ranges";
+        case SDM_ERR_DTYPE: return "SDM_ERR_DTYPE: unknown dtype";
+        case SDM_ERR_ALIGN: return "SDM_ERR_ALIGN: pointer not 16-byte aligned";
+        case SDM_ERR_CUDA: return "SDM_ERR_CUDA: CUDA runtime call failed";
+        case SDM_ERR_BAD_INDEX: return "SDM_ERR_BAD_INDEX: device error word is set";
+        case SDM_ERR_WORKSPACE: return "SDM_ERR_WORKSPACE: workspace missing or too small";
+        case SDM_ERR_UNSUPPORTED: return "SDM_ERR_UNSUPPORTED: not implemented for these arguments";
+        default: return "SDM_ERR_UNKNOWN";
+    }
+}
+
+int32_t sdm_abi_version(void) { return 1; }
+
+sdm_status sdm_state_bytes(const sdm_dims* dims, size_t* M_bytes, size_t* stamp_bytes,
+                           size_t* lambda_bytes) {
+    if (!M_bytes || !stamp_bytes || !lambda_bytes) return SDM_ERR_ARG;
+    const sdm_status e = check_dims(dims);
+    if (e) return e;
+    const size_t BH = (size_t)BH_of(dims), N = (size_t)N_of(dims);
+    *M_bytes = BH * N * dims->d_v * sizeof(float);
+    *stamp_bytes = BH * N * sizeof(double);
+    *lambda_bytes = BH * sizeof(double);
+    return SDM_OK;
+}
+
+sdm_status sdm_state_reset(const sdm_dims* dims, const sdm_state* st, sdm_stream_t stream) {
+    sdm_status e = check_dims(dims);
+    if (e) return e;
+    if ((e = check_state(st))) return e;
+    const size_t n = (size_t)BH_of(dims) * N_of(dims);
+    const int threads = 256;
+    size_t blocks = (n / 2 + threads - 1) / threads;
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    if (blocks < 1) blocks = 1;
+    state_reset_kernel<<<(unsigned)blocks, threads, 0, stream>>>(st->stamp, n, st->Lambda,
+                                                                 (int)BH_of(dims));
+    return launch_status();
+}
+
+sdm_status sdm_state_materialize(const sdm_dims* dims, const sdm_state* st, float* M_out,
+                                 sdm_stream_t stream) {
+    sdm_status e = check_dims(dims);
+    if (e) return e;
+    if ((e = check_state(st))) return e;
+    if (!M_out) return SDM_ERR_ARG;
+    if (!aligned16(M_out)) return SDM_ERR_ALIGN;
+    if (M_out == st->M) return SDM_ERR_ARG;
+    const size_t rows = (size_t)BH_of(dims) * N_of(dims);
+    const size_t total = rows * (dims->d_v / 4);
+    const int threads = 256;
+    size_t blocks = (total + threads - 1) / threads;
+    if (blocks > 148 * 64) blocks = 148 * 64;
+    state_materialize_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+        st->M, st->stamp, st->Lambda, st->M0, dims->H, (int)N_of(dims), dims->d_v, rows, M_out);
+    return launch_status();
+}
+
+sdm_status sdm_score_topk(const sdm_dims* dims, const void* x, const void* subkeys, int32_t top,
+                          int32_t* idx, float* w, sdm_stream_t stream) {
+    const sdm_status e = check_dims(dims);
+    if (e) return e;
+    if (!x || !subkeys || !idx || !w) return SDM_ERR_ARG;
+    if (top < 1 || top > kMaxTop || top > dims->k_half * dims->k_half) return SDM_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(subkeys) || !aligned16(idx) || !aligned16(w)) return SDM_ERR_ALIGN;
+    return launch_score(dims, x, subkeys, top, idx, w, stream);
+}
+
+size_t sdm_forward_workspace_bytes(const sdm_dims* dims) {
+    if (check_dims(dims) != SDM_OK) return 0;
+    return ws_layout(dims).total;
+}
+
+sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const int32_t* widx,
+                            const int32_t* ridx, const sdm_state* st, void* ws, size_t ws_bytes,
+                            sdm_stream_t stream) {
+    sdm_status e = check_dims(dims);
+    if (e) return e;
+    if ((e = check_state(st))) return e;
+    if (dims->T == 0) return SDM_OK;
+    if (!alpha || !widx || !ridx) return SDM_ERR_ARG;
+    if (!aligned16(alpha) || !aligned16(widx) || !aligned16(ridx)) return SDM_ERR_ALIGN;
+    const WsLayout L = ws_layout(dims);
+    if (!ws || ws_bytes < L.total) return SDM_ERR_WORKSPACE;
+    if (!aligned16(ws)) return SDM_ERR_ALIGN;
+    const PlanPtrs P = plan_ptrs(L, ws);
+    const int N = (int)N_of(dims);
+    const size_t BH = (size_t)BH_of(dims);
+    if (!L.smem_table &&
+        cudaMemsetAsync(P.lastw, 0xff, BH * (size_t)N * 4, stream) != cudaSuccess)
+        return SDM_ERR_CUDA;
+    plan_local_kernel<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, 0, stream>>>(
+        alpha, widx, ridx, st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, P);
+    if ((e = launch_status())) return e;
+    if (L.smem_table) {
+        if (!set_smem(plan_walk_kernel<true>, L.walk_smem)) return SDM_ERR_CUDA;
+        plan_walk_kernel<true><<<(unsigned)BH, WALK_THREADS, L.walk_smem, stream>>>(
+            widx, ridx, st->stamp, st->Lambda, dims->T, N, dims->W, dims->R, L.C, L.J,
+            L.lstart_smem ? 1 : 0, P);
+    } else {
+        if (!set_smem(plan_walk_kernel<false>, L.walk_smem)) return SDM_ERR_CUDA;
+        plan_walk_kernel<false><<<(unsigned)BH, WALK_THREADS, L.walk_smem, stream>>>(
+            widx, ridx, st->stamp, st->Lambda, dims->T, N, dims->W, dims->R, L.C, L.J,
+            L.lstart_smem ? 1 : 0, P);
+    }
+    return launch_status();
+}
+
+sdm_status sdm_forward_run(const sdm_dims* dims, const void* v, const float* beta,
+                           const int32_t* widx, const float* ww, const int32_t* ridx,
+                           const float* rw, const sdm_state* st, float* out, void* ws,
+                           size_t ws_bytes, sdm_stream_t stream) {
+    sdm_status e = check_dims(dims);
+    if (e) return e;
+    if ((e = check_state(st))) return e;
+    if (dims->T == 0) return SDM_OK;
+    if (!v || !beta || !widx || !ww || !ridx || !rw || !out) return SDM_ERR_ARG;
+    if (!aligned16(v) || !aligned16(beta) || !aligned16(widx) || !aligned16(ww) ||
+        !aligned16(ridx) || !aligned16(rw) || !aligned16(out))
+        return SDM_ERR_ALIGN;
+    const WsLayout L = ws_layout(dims);
+    if (!ws || ws_bytes < L.total) return SDM_ERR_WORKSPACE;
+    if (!aligned16(ws)) return SDM_ERR_ALIGN;
+    const PlanPtrs P = plan_ptrs(L, ws);
+    const int CW = col_width(dims);
+    if (CW == 8) {
+        if (dims->v_dtype == SDM_BF16)
+            return launch_run_t<8, __nv_bfloat16>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, stream);
+        return launch_run_t<8, float>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, stream);
+    }
+    if (dims->v_dtype == SDM_BF16)
+        return launch_run_t<4, __nv_bfloat16>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, stream);
+    return launch_run_t<4, float>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, stream);
+}
+
+sdm_status sdm_forward(const sdm_dims* dims, const void* v, const float* alpha, const float* beta,
+                       const int32_t* widx, const float* ww, const int32_t* ridx, const float* rw,
+                       const sdm_state* st, float* out, void* ws, size_t ws_bytes,
+                       sdm_stream_t stream) {
+    sdm_status e = check_dims(dims);
+    if (e) return e;
+    if ((e = check_state(st))) return e;
+    if (dims->T == 0) return SDM_OK;
+    if (!v || !alpha || !beta || !widx || !ww || !ridx || !rw || !out) return SDM_ERR_ARG;
+    const WsLayout L = ws_layout(dims);
+    if (!ws || ws_bytes < L.total) return SDM_ERR_WORKSPACE;
+    if ((e = sdm_forward_plan(dims, alpha, widx, ridx, st, ws, ws_bytes, stream))) return e;
+    return sdm_forward_run(dims, v, beta, widx, ww, ridx, rw, st, out, ws, ws_bytes, stream);
+}
+
+sdm_status sdm_prefill(const sdm_dims* dims, const void* q, const void* k, const void* v,
+                       const float* alpha, const float* beta, const void* skw, const void* skr,
+                       const sdm_state* st, int32_t* widx, float* ww, int32_t* ridx, float* rw,
+                       float* out, void* ws, size_t ws_bytes, sdm_stream_t stream) {
+    sdm_status e = check_dims(dims);
+    if (e) return e;
+    if ((e = check_state(st))) return e;
+    if (dims->T == 0) return SDM_OK;
+    if (!q || !k || !v || !alpha || !beta || !skw || !skr || !widx || !ww || !ridx || !rw || !out)
+        return SDM_ERR_ARG;
+    const WsLayout L = ws_layout(dims);
+    if (!ws || ws_bytes < L.total) return SDM_ERR_WORKSPACE;
+    if ((e = sdm_score_topk(dims, k, skw, dims->W, widx, ww, stream))) return e;
+    if ((e = sdm_score_topk(dims, q, skr, dims->R, ridx, rw, stream))) return e;
+    return sdm_forward(dims, v, alpha, beta, widx, ww, ridx, rw, st, out, ws, ws_bytes, stream);
+}
+
+sdm_status sdm_decode_step(const sdm_dims* dims, const void* q, const void* k, const void* v,
+                           const float* alpha, const float* beta, const void* skw,
+                           const void* skr, const sdm_state* st, int32_t* widx, float* ww,
+                           int32_t* ridx, float* rw, float* out, sdm_stream_t stream) {
+    sdm_status e = check_dims(dims);
+    if (e) return e;
+    if (dims->T != 1) return SDM_ERR_SHAPE;
+    if ((e = check_state(st))) return e;
+    if (!q || !k || !v || !alpha || !beta || !skw || !skr || !widx || !ww || !ridx || !rw || !out)
+        return SDM_ERR_ARG;
+    if (!aligned16(v) || !aligned16(alpha) || !aligned16(beta) || !aligned16(out))
+        return SDM_ERR_ALIGN;
+    if ((e = sdm_score_topk(dims, k, skw, dims->W, widx, ww, stream))) return e;
+    if ((e = sdm_score_topk(dims, q, skr, dims->R, ridx, rw, stream))) return e;
+    const size_t smem = decode_smem_bytes(dims->W, dims->R, dims->d_v);
+    const unsigned grid = (unsigned)BH_of(dims);
+    if (dims->v_dtype == SDM_BF16) {
+        if (!set_smem(decode_kernel<__nv_bfloat16>, smem)) return SDM_ERR_CUDA;
+        decode_kernel<__nv_bfloat16><<<grid, DECODE_THREADS, smem, stream>>>(
+            (const __nv_bfloat16*)v, alpha, beta, widx, ww, ridx, rw, st->M, st->stamp,
+            st->Lambda, st->M0, out, dims->H, (int)N_of(dims), dims->d_v, dims->W, dims->R);
+    } else {
+        if (!set_smem(decode_kernel<float>, smem)) return SDM_ERR_CUDA;
+        decode_kernel<float><<<grid, DECODE_THREADS, smem, stream>>>(
+            (const float*)v, alpha, beta, widx, ww, ridx, rw, st->M, st->stamp, st->Lambda,
+            st->M0, out, dims->H, (int)N_of(dims), dims->d_v, dims->W, dims->R);
+    }
+    return launch_status();
+}
+
+sdm_status sdm_device_error(uint32_t* bits, int32_t clear, sdm_stream_t stream) {
+    if (!bits) return SDM_ERR_ARG;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, g_err, sizeof(v), 0, cudaMemcpyDeviceToHost, stream) !=
+        cudaSuccess)
+        return SDM_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return SDM_ERR_CUDA;
+    if (clear) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbolAsync(g_err, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice,
+                                    stream) != cudaSuccess)
+            return SDM_ERR_CUDA;
+        if (cudaStreamSynchronize(stream) != cudaSuccess) return SDM_ERR_CUDA;
+    }
+    *bits = v;
+    return v ? SDM_ERR_BAD_INDEX : SDM_OK;
+}
+
+}  // extern "C"

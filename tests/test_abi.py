@@ -1,0 +1,108 @@
+"""The C-ABI library on the CPU: it loads without a GPU, exports every entry point that
+include/sdm.h declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sdm.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(sdm_\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_state_linear_score_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "H", "T", "d_k", "n_sub", "d_v", "k_half", "W", "R", "x_dtype", "v_dtype")]
+
+
+def mid_dims(**kw):
+    d = dict(B=2, H=4, T=4096, d_k=128, n_sub=256, d_v=128, k_half=32, W=32, R=32, x_dtype=1,
+             v_dtype=1)
+    d.update(kw)
+    return Dims(**d)
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for must in ("sdm_score_topk", "sdm_forward", "sdm_decode_step", "sdm_prefill",
+                 "sdm_state_reset", "sdm_state_materialize", "sdm_forward_workspace_bytes",
+                 "sdm_device_error"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings(lib):
+    lib.sdm_status_str.restype = ctypes.c_char_p
+    for code in range(0, 9):
+        s = lib.sdm_status_str(code)
+        assert s and s.startswith(b"SDM_")
+    assert lib.sdm_abi_version() >= 1
+
+
+def test_workspace_and_state_sizes(lib):
+    lib.sdm_forward_workspace_bytes.restype = ctypes.c_size_t
+    d = mid_dims()
+    ws = lib.sdm_forward_workspace_bytes(ctypes.byref(d))
+    assert ws > 2 * 4 * 4096 * 64 * 8  # at least the per-occurrence plan records
+    bad = mid_dims(W=65)
+    assert lib.sdm_forward_workspace_bytes(ctypes.byref(bad)) == 0
+    m, s, l = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.sdm_state_bytes(ctypes.byref(d), ctypes.byref(m), ctypes.byref(s), ctypes.byref(l)) == 0
+    assert m.value == 2 * 4 * 65536 * 128 * 4
+    assert s.value == 2 * 4 * 65536 * 8 and l.value == 2 * 4 * 8
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("x_dtype", 7, 3), ("v_dtype", -1, 3), ("B", 0, 2), ("T", -1, 2), ("d_k", 30, 2),
+    ("d_k", 512, 2), ("n_sub", 0, 2), ("d_v", 6, 2), ("d_v", 512, 2), ("k_half", 65, 2),
+    ("k_half", 300, 2), ("W", 0, 2), ("R", 65, 2),
+])
+def test_bad_dims_rejected_on_host(lib, field, value, code):
+    d = mid_dims(**{field: value})
+    p = ctypes.c_void_p(0x1000)
+    assert lib.sdm_score_topk(ctypes.byref(d), p, p, 4, p, p, None) == code
+
+
+def test_null_and_misaligned_pointers(lib):
+    d = mid_dims()
+    p = ctypes.c_void_p(0x1000)
+    assert lib.sdm_score_topk(None, p, p, 4, p, p, None) == 1
+    assert lib.sdm_score_topk(ctypes.byref(d), None, p, 4, p, p, None) == 1
+    assert lib.sdm_score_topk(ctypes.byref(d), ctypes.c_void_p(0x1004), p, 4, p, p, None) == 4
+    assert lib.sdm_score_topk(ctypes.byref(d), p, p, 0, p, p, None) == 2
+    assert lib.sdm_score_topk(ctypes.byref(d), p, p, 65, p, p, None) == 2
+    assert lib.sdm_device_error(None, 0, None) == 1
+    assert lib.sdm_state_reset(ctypes.byref(d), None, None) == 1
+    # decode needs T == 1
+    assert lib.sdm_decode_step(ctypes.byref(d), p, p, p, p, p, p, p, None, p, p, p, p, p, None) == 2
+
+
+def test_forward_rejects_small_workspace(lib):
+    class State(ctypes.Structure):
+        _fields_ = [("M", ctypes.c_void_p), ("stamp", ctypes.c_void_p), ("Lambda", ctypes.c_void_p),
+                    ("M0", ctypes.c_void_p)]
+    d = mid_dims()
+    p = ctypes.c_void_p(0x1000)
+    st = State(0x1000, 0x2000, 0x3000, 0x4000)
+    assert lib.sdm_forward(ctypes.byref(d), p, p, p, p, p, p, p, ctypes.byref(st), p, p,
+                           ctypes.c_size_t(64), None) == 7
+    st_bad = State(0x1000, 0x2000, 0x3003, 0x4000)
+    assert lib.sdm_forward(ctypes.byref(d), p, p, p, p, p, p, p, ctypes.byref(st_bad), p, p,
+                           ctypes.c_size_t(1 << 40), None) == 4
