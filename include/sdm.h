@@ -206,6 +206,29 @@ sdm_status sdm_decode_step(const sdm_dims* dims, const void* q, const void* k, c
                            int32_t* ridx, float* rw, float* out, sdm_stream_t stream);
 
 /*
+ * sdm_forward without a caller workspace and without any allocation: for callers that
+ * cannot call cudaMalloc or hand out scratch memory themselves — for example a custom
+ * operator inside a host framework that owns the device allocator and forbids side
+ * allocations, or a loop whose memory budget is fixed when the process starts.  The paper
+ * has no counterpart of this call; it only changes where the scratch lives.
+ *   Arguments, layouts and results are those of sdm_forward.
+ *   Scratch: one fixed 64 MiB array in device memory, defined in the library and held by
+ *     every GPU that loads it until the process exits.  Calls whose workspace would
+ *     exceed it (sdm_forward_workspace_bytes(dims) > 64 MiB) return SDM_ERR_WORKSPACE and
+ *     enqueue nothing.  Each call writes every part of the array it later reads, so no
+ *     contents carry over from the previous call.
+ *   All calls on a device share the array: calls that can overlap on the GPU (different
+ *     streams, or several host threads) race on it and must be serialised by the caller.
+ *   The first call on a device looks up the array's device address (once per device, with
+ *     the stream's device current); make that first call before any stream capture.
+ *   Never calls cudaMalloc, cudaFree or any allocating routine.
+ */
+sdm_status sdm_forward_noalloc(const sdm_dims* dims, const void* v, const float* alpha,
+                               const float* beta, const int32_t* widx, const float* ww,
+                               const int32_t* ridx, const float* rw, const sdm_state* st,
+                               float* out, sdm_stream_t stream);
+
+/*
  * Read the device error word into *bits (host pointer; SDM_DEVERR_* bits), then
  * clear it when `clear` is non-zero.  Synchronises `stream`.  Returns SDM_OK when
  * no bit is set, SDM_ERR_BAD_INDEX when any is, SDM_ERR_CUDA if the copy fails.

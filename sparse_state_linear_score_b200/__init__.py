@@ -22,7 +22,7 @@ import torch
 from . import build as _build
 
 __all__ = ["Dims", "State", "SdmError", "state_reset", "state_materialize", "score_topk",
-           "forward_workspace_bytes", "forward", "forward_plan", "forward_run", "prefill",
+           "forward_workspace_bytes", "forward", "forward_noalloc", "forward_plan", "forward_run", "prefill",
            "decode_step", "device_error", "lib_path", "DEVERR_SLOT_RANGE", "DEVERR_DUP_WRITE",
            "DEVERR_ALPHA"]
 
@@ -81,6 +81,7 @@ def _load():
         "sdm_prefill": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P, SZ, P], I32),
         "sdm_decode_step": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P], I32),
         "sdm_device_error": ([ctypes.POINTER(ctypes.c_uint32), I32, P], I32),
+        "sdm_forward_noalloc": ([D, P, P, P, P, P, P, P, S, P, P], I32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -191,6 +192,17 @@ def forward(d: Dims, v, alpha, beta, widx, ww, ridx, rw, st: State, out=None, ws
     a = _fw_args(d, v, alpha, beta, widx, ww, ridx, rw)
     _ok(_lib.sdm_forward(ctypes.byref(d), *a, ctypes.byref(st.c), _ptr(out, "out", torch.float32),
                          _ptr(ws, "ws"), ws.numel(), _stream(stream)), "sdm_forward")
+    return out
+
+
+def forward_noalloc(d: Dims, v, alpha, beta, widx, ww, ridx, rw, st: State, out=None, stream=None):
+    """sdm_forward with the library's fixed 64 MiB device scratch instead of a workspace."""
+    if out is None:
+        out = torch.empty((d.B, d.H, d.T, d.d_v), dtype=torch.float32, device=v.device)
+    a = _fw_args(d, v, alpha, beta, widx, ww, ridx, rw)
+    _ok(_lib.sdm_forward_noalloc(ctypes.byref(d), *a, ctypes.byref(st.c),
+                                 _ptr(out, "out", torch.float32), _stream(stream)),
+        "sdm_forward_noalloc")
     return out
 
 

@@ -4,6 +4,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "decode.cuh"
 #include "plan.cuh"
@@ -152,6 +154,38 @@ sdm_status launch_run_t(const sdm_dims* d, const WsLayout& L, const PlanPtrs& P,
         reinterpret_cast<const unsigned long long*>(P.tmask), st->M, st->M0, out, d->H, d->T,
         (int)N_of(d), d->d_v, d->W, d->R, L.C, L.J);
     return launch_status();
+}
+
+// ---- workspace of sdm_forward_noalloc: a fixed array in device memory -------------------
+// Every GPU that loads the library holds this array until the process exits.
+constexpr size_t kNoAllocWorkspaceBytes = size_t(64) << 20;  // 64 MiB
+constexpr int kNoAllocMaxDevices = 64;
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_ws[kNoAllocWorkspaceBytes];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_ws on the current device.  In host code the array's name is
+// only a host-side stand-in, so the address is looked up once per device (with that device
+// current) and cached.
+sdm_status noalloc_workspace(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SDM_ERR_CUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return SDM_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_ws) != cudaSuccess || p == nullptr)
+            return SDM_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SDM_OK;
 }
 
 }  // namespace
@@ -356,6 +390,23 @@ sdm_status sdm_decode_step(const sdm_dims* dims, const void* q, const void* k, c
             st->M0, out, dims->H, (int)N_of(dims), dims->d_v, dims->W, dims->R);
     }
     return launch_status();
+}
+
+sdm_status sdm_forward_noalloc(const sdm_dims* dims, const void* v, const float* alpha,
+                               const float* beta, const int32_t* widx, const float* ww,
+                               const int32_t* ridx, const float* rw, const sdm_state* st,
+                               float* out, sdm_stream_t stream) {
+    sdm_status e = check_dims(dims);
+    if (e) return e;
+    if ((e = check_state(st))) return e;
+    if (dims->T == 0) return SDM_OK;
+    if (!v || !alpha || !beta || !widx || !ww || !ridx || !rw || !out) return SDM_ERR_ARG;
+    const WsLayout L = ws_layout(dims);
+    if (L.total > kNoAllocWorkspaceBytes) return SDM_ERR_WORKSPACE;
+    void* ws = nullptr;
+    if ((e = noalloc_workspace(&ws))) return e;
+    return sdm_forward(dims, v, alpha, beta, widx, ww, ridx, rw, st, out, ws,
+                       kNoAllocWorkspaceBytes, stream);
 }
 
 sdm_status sdm_device_error(uint32_t* bits, int32_t clear, sdm_stream_t stream) {
