@@ -65,6 +65,7 @@ typedef enum { SDM_F32 = 0, SDM_BF16 = 1 } sdm_dtype;
 #define SDM_DEVERR_SLOT_RANGE 1u   /* a slot index outside [0, N) */
 #define SDM_DEVERR_DUP_WRITE 2u    /* a write slot repeated within one token */
 #define SDM_DEVERR_ALPHA 4u        /* alpha <= 0 (its log is undefined) */
+#define SDM_DEVERR_TIMEOUT 8u      /* a bounded on-chip wait gave up (the call's results are invalid) */
 
 typedef struct {
     int32_t B, H, T;   /* sequences, heads, tokens in this call (T = 1 for decode) */

@@ -1,0 +1,442 @@
+// Product-key scoring on the 5th-generation tensor cores (tcgen05 + TMEM + TMA), bf16 inputs.
+//
+// One CTA scores a tile of 128 rows (tokens of one head, one role) against that role's two
+// sub-key tables (§2 Background "Product Key Memory", §3 Method "Sparse addressing"):
+//   - TMA loads the x tile (both halves, 128-byte swizzle) and, per round, up to 256 sub-keys
+//     of one half; one thread issues 4 tcgen05.mma (K = 64 = 4 x 16) into 256 TMEM columns:
+//     D[row][j] = <x_half[row], C[j]> in fp32.
+//   - Thread r owns row r (TMEM lane r).  It keeps the k best sub-keys of each half exactly:
+//     min/max pass, a 64-bin histogram to find the threshold bin, compaction of the bins
+//     above it plus the best of the threshold bin (refined with finer bins when crowded),
+//     then a register bitonic sort (best first; equal scores to the lower sub-index).
+//     Halves with more than 256 sub-keys merge the per-round lists.
+//   - The k x k combine walks the pairs in decreasing order with a max-heap over the rows
+//     of the first list (pairs with (a+1)(b+1) > top are never pushed: >= top pairs beat
+//     them), giving the top-W (or top-R) slots s = i*n + j best first, then the softmax of
+//     the selected scores (§4 "SDM Configuration").
+#pragma once
+
+#include <math.h>
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+
+namespace sdm {
+
+constexpr int TC_THREADS = 128;
+constexpr int TC_NB = 256;      // sub-keys per round = TMEM columns
+constexpr int TC_NBIN = 64;     // histogram bins
+constexpr int TC_BC = 10;       // boundary candidates ranked exactly
+constexpr int TC_MAXLEV = 4;    // histogram refinement levels
+constexpr int TC_KMAX = 32;     // largest k_half / top this kernel takes
+
+// Shared-memory map (bytes from a 1024-aligned base).
+constexpr uint32_t TC_OFF_A = 0;         // x tile: half 0 [0,16K), half 1 [16K,32K); later list R1
+constexpr uint32_t TC_OFF_B = 32768;     // sub-key round tile; selection scratch; combine heap
+constexpr uint32_t TC_OFF_HIST = 65536;  // u16 hist [64][128]; later the selected scores [top][128]
+constexpr uint32_t TC_OFF_R0 = 81920;    // list R0: f32 [K][128] + u16 [K][128]
+constexpr uint32_t TC_OFF_CTRL = 81920 + 24576;
+constexpr uint32_t TC_SMEM_BYTES = TC_OFF_CTRL + 64 + 1024;  // + alignment slack
+
+struct ScoreTcArgs {
+    int B, H, T, n, k_half, top;
+    int nbox;          // sub-key rows per TMA box = min(n, 256)
+    int bt, bb, n_tt;  // a tile holds bt tokens of bb sequences; t-tiles per sequence block
+    int32_t* idx;
+    float* w;
+};
+
+SDM_DEV int tc_bin(float v, float lo, float sc) {
+    int b = __float2int_rd((v - lo) * sc);
+    return min(max(b, 0), TC_NBIN - 1);
+}
+
+template <int KP>
+SDM_DEV void bitonic_sort_desc(float (&v)[KP], int (&ix)[KP]) {
+#pragma unroll
+    for (int k = 2; k <= KP; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll
+            for (int i = 0; i < KP; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const bool desc = (i & k) == 0;
+                    const bool sw = desc ? better(v[l], ix[l], v[i], ix[i])
+                                         : better(v[i], ix[i], v[l], ix[l]);
+                    const float tv = sw ? v[l] : v[i];
+                    const int ti = sw ? ix[l] : ix[i];
+                    v[l] = sw ? v[i] : v[l];
+                    ix[l] = sw ? ix[i] : ix[l];
+                    v[i] = tv;
+                    ix[i] = ti;
+                }
+            }
+        }
+    }
+}
+
+// Merge a sorted (best-first) list held in r[] with sorted a[]: r <- best KP of both, sorted.
+template <int KP>
+SDM_DEV void bitonic_merge_keep(float (&r)[KP], int (&ri)[KP], const float (&a)[KP],
+                                const int (&ai)[KP]) {
+#pragma unroll
+    for (int i = 0; i < KP; ++i) {
+        const bool take = better(a[KP - 1 - i], ai[KP - 1 - i], r[i], ri[i]);
+        r[i] = take ? a[KP - 1 - i] : r[i];
+        ri[i] = take ? ai[KP - 1 - i] : ri[i];
+    }
+#pragma unroll
+    for (int j = KP >> 1; j > 0; j >>= 1) {
+#pragma unroll
+        for (int i = 0; i < KP; ++i) {
+            const int l = i ^ j;
+            if (l > i) {
+                const bool sw = better(r[l], ri[l], r[i], ri[i]);
+                const float tv = sw ? r[l] : r[i];
+                const int ti = sw ? ri[l] : ri[i];
+                r[l] = sw ? r[i] : r[l];
+                ri[l] = sw ? ri[i] : ri[l];
+                r[i] = tv;
+                ri[i] = ti;
+            }
+        }
+    }
+}
+
+// The K best of this thread's NB TMEM columns (sub-index = col_base + column), returned
+// sorted best-first in a[0..K) (entries K..KP-1 are padding).  Per-thread shared arrays
+// are strided by TC_THREADS.  Every TMEM pass is executed by whole warps (tcgen05.ld is
+// warp-collective); the per-thread state only predicates the work inside a pass.
+template <int KP>
+SDM_DEV void tc_select(uint32_t trow, int NB, int K, int col_base, uint16_t* hist, float* Sv,
+                       uint16_t* Si, float* Bv, uint16_t* Bi, float (&a)[KP], int (&ai)[KP]) {
+    constexpr int S = TC_THREADS;
+    constexpr unsigned FULL = 0xffffffffu;
+    float mn = INFINITY, mx = -INFINITY;
+    for (int c = 0; c < NB; c += 32) {
+        float v[32];
+        ptx::tmem_ld32(trow + c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            mn = fminf(mn, v[i]);
+            mx = fmaxf(mx, v[i]);
+        }
+    }
+    int ns = 0, need = K;
+    // all scores equal (or not numbers): the first K sub-indices win the ties
+    const bool flat = !(mx > mn) || !isfinite((float)TC_NBIN / (mx - mn));
+    float lo[TC_MAXLEV], sc[TC_MAXLEV];
+    int tb[TC_MAXLEV];
+    lo[0] = flat ? 0.f : mn;
+    sc[0] = flat ? 0.f : (float)TC_NBIN / (mx - mn);
+    bool done = false;
+#pragma unroll
+    for (int L = 0; L < TC_MAXLEV; ++L) {
+        const bool hist_on = !done && !flat;
+        int t_b = 0, cum = 0, cnt_tb = 0;
+        if (__any_sync(FULL, hist_on)) {
+            if (hist_on)
+                for (int bn = 0; bn < TC_NBIN; ++bn) hist[bn * S] = 0;
+            for (int c = 0; c < NB; c += 32) {
+                float v[32];
+                ptx::tmem_ld32(trow + c, v);
+                if (hist_on) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        bool in = true;
+#pragma unroll
+                        for (int l = 0; l < L; ++l) in = in && tc_bin(v[i], lo[l], sc[l]) == tb[l];
+                        if (in) {
+                            const int bn = tc_bin(v[i], lo[L], sc[L]);
+                            hist[bn * S] = (uint16_t)(hist[bn * S] + 1);
+                        }
+                    }
+                }
+            }
+            if (hist_on) {
+                for (int bn = TC_NBIN - 1; bn >= 0; --bn) {
+                    const int cnt = hist[bn * S];
+                    if (cum + cnt >= need) {
+                        t_b = bn;
+                        break;
+                    }
+                    cum += cnt;
+                }
+                cnt_tb = hist[t_b * S];
+            }
+        }
+        tb[L] = t_b;
+        const bool small = cnt_tb <= TC_BC;
+        const bool last = small || L == TC_MAXLEV - 1;
+        const bool flat_take = flat && !done && L == 0;
+        const bool comp_on = hist_on || flat_take;
+        int nbd = 0;
+        int take_direct = flat_take ? need : (hist_on && last && !small ? need - cum : 0);
+        if (__any_sync(FULL, comp_on)) {
+            for (int c = 0; c < NB; c += 32) {
+                float v[32];
+                ptx::tmem_ld32(trow + c, v);
+                if (comp_on) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const uint16_t col = (uint16_t)(col_base + c + i);
+                        if (flat_take) {
+                            if (take_direct > 0) {
+                                Sv[ns * S] = v[i];
+                                Si[ns * S] = col;
+                                ++ns;
+                                --take_direct;
+                            }
+                            continue;
+                        }
+                        bool in = true;
+#pragma unroll
+                        for (int l = 0; l < L; ++l) in = in && tc_bin(v[i], lo[l], sc[l]) == tb[l];
+                        if (!in) continue;
+                        const int bn = tc_bin(v[i], lo[L], sc[L]);
+                        if (bn > t_b) {
+                            Sv[ns * S] = v[i];
+                            Si[ns * S] = col;
+                            ++ns;
+                        } else if (bn == t_b) {
+                            if (last && small) {
+                                Bv[nbd * S] = v[i];
+                                Bi[nbd * S] = col;
+                                ++nbd;
+                            } else if (take_direct > 0) {  // crowded last level: index order
+                                Sv[ns * S] = v[i];
+                                Si[ns * S] = col;
+                                ++ns;
+                                --take_direct;
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        if (flat_take) {
+            done = true;
+        } else if (hist_on) {
+            need -= cum;
+            if (last) {
+                if (small) {  // the `need` best of the boundary bin, by exact rank
+                    for (int e = 0; e < nbd; ++e) {
+                        const float ve = Bv[e * S];
+                        const int ie = Bi[e * S];
+                        int rank = 0;
+                        for (int f = 0; f < nbd; ++f) rank += better(Bv[f * S], Bi[f * S], ve, ie);
+                        if (rank < need) {
+                            Sv[ns * S] = ve;
+                            Si[ns * S] = (uint16_t)ie;
+                            ++ns;
+                        }
+                    }
+                }
+                done = true;
+            } else if (L + 1 < TC_MAXLEV) {
+                lo[L + 1] = lo[L] + (float)t_b / sc[L];
+                sc[L + 1] = sc[L] * (float)TC_NBIN;
+            }
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < KP; ++e) {
+        const bool ok = e < ns && e < K;
+        a[e] = ok ? Sv[e * S] : -INFINITY;
+        ai[e] = ok ? (int)Si[e * S] : 0x7fffffff;
+    }
+    bitonic_sort_desc<KP>(a, ai);
+}
+
+template <int KP>
+__global__ void __launch_bounds__(TC_THREADS, 2) score_tc_kernel(
+    const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap skmap,
+    ScoreTcArgs p) {
+    constexpr int S = TC_THREADS;
+    extern __shared__ unsigned char tc_smem_raw[];
+    unsigned char* sm = tc_smem_raw + ((1024 - (ptx::smem_u32(tc_smem_raw) & 1023)) & 1023);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int h = blockIdx.y;
+    const int bti = blockIdx.x / p.n_tt, tti = blockIdx.x % p.n_tt;
+    const int b0 = bti * p.bb, t0 = tti * p.bt;
+    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + TC_OFF_CTRL);
+    uint64_t* bar_mma = bar_tma + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 2);
+    int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+    if (warp == 0) ptx::tmem_alloc(tmem_slot, TC_NB);
+    if (tid == 0) {
+        ptx::mbar_init(bar_tma, 1);
+        ptx::mbar_init(bar_mma, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint64_t deadline = ptx::globaltimer_ns() + 2000000000ull;
+    uint32_t ph_tma = 0, ph_mma = 0;
+
+    const int bi = tid / p.bt, ti = tid % p.bt;
+    const int b = b0 + bi, t = t0 + ti;
+    const bool row_ok = bi < p.bb && b < p.B && t < p.T;
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const int K = p.k_half, n = p.n;
+    const int rounds = (n + TC_NB - 1) / TC_NB;
+    const uint32_t abox = 64u * 2u * (uint32_t)(p.bt * p.bb);
+
+    uint16_t* hist = reinterpret_cast<uint16_t*>(sm + TC_OFF_HIST) + tid;
+    float* Sv = reinterpret_cast<float*>(sm + TC_OFF_B) + tid;
+    uint16_t* Si = reinterpret_cast<uint16_t*>(sm + TC_OFF_B + K * S * 4) + tid;
+    float* Bv = reinterpret_cast<float*>(sm + TC_OFF_B + K * S * 6) + tid;
+    uint16_t* Bi = reinterpret_cast<uint16_t*>(sm + TC_OFF_B + K * S * 6 + TC_BC * S * 4) + tid;
+    float* R0v = reinterpret_cast<float*>(sm + TC_OFF_R0) + tid;
+    uint16_t* R0i = reinterpret_cast<uint16_t*>(sm + TC_OFF_R0 + K * S * 4) + tid;
+    float* R1v = reinterpret_cast<float*>(sm + TC_OFF_A) + tid;
+    uint16_t* R1i = reinterpret_cast<uint16_t*>(sm + TC_OFF_A + K * S * 4) + tid;
+
+    bool aborted = false;
+    for (int hf = 0; hf < 2 && !aborted; ++hf) {
+        float* Rv = hf ? R1v : R0v;
+        uint16_t* Ri = hf ? R1i : R0i;
+        for (int r = 0; r < rounds; ++r) {
+            const int nb = min(TC_NB, n - r * TC_NB);
+            if (tid == 0) {
+                // generic-proxy writes to the tile area (scratch, lists) precede this load
+                ptx::fence_proxy_async_smem();
+                const bool first = hf == 0 && r == 0;
+                ptx::mbar_arrive_expect_tx(bar_tma, (first ? 2u * abox : 0u) + 64u * 2u * (uint32_t)p.nbox);
+                if (first) {
+                    ptx::tma_load_4d(sm + TC_OFF_A, &xmap, 0, t0, h, b0, bar_tma);
+                    ptx::tma_load_4d(sm + TC_OFF_A + 16384, &xmap, 64, t0, h, b0, bar_tma);
+                }
+                ptx::tma_load_2d(sm + TC_OFF_B, &skmap, 0, (h * 2 + hf) * n + r * TC_NB, bar_tma);
+                if (ptx::mbar_wait_bounded(bar_tma, ph_tma, deadline)) {
+                    ptx::tc_fence_after();
+                    const uint64_t ad = ptx::umma_desc_kmajor_sw128(sm + TC_OFF_A + hf * 16384);
+                    const uint64_t bd = ptx::umma_desc_kmajor_sw128(sm + TC_OFF_B);
+                    const uint32_t id = ptx::idesc_bf16_f32(128, nb);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)  // K = 64 in steps of 16 (32 bytes)
+                        ptx::umma_bf16(tmem, ad + 2 * k, bd + 2 * k, id, k > 0 ? 1u : 0u);
+                    ptx::umma_commit(bar_mma);
+                } else {
+                    *abort_flag = 1;
+                }
+            }
+            ph_tma ^= 1;
+            if (!ptx::mbar_wait_bounded(bar_mma, ph_mma, deadline)) *abort_flag = 1;
+            ph_mma ^= 1;
+            ptx::tc_fence_after();
+            __syncthreads();
+            if (*abort_flag) {
+                aborted = true;
+                break;
+            }
+            float a[KP];
+            int ai[KP];
+            tc_select<KP>(trow, nb, K, r * TC_NB, hist, Sv, Si, Bv, Bi, a, ai);
+            if (r == 0) {
+#pragma unroll
+                for (int e = 0; e < KP; ++e)
+                    if (e < K) {
+                        Rv[e * S] = a[e];
+                        Ri[e * S] = (uint16_t)ai[e];
+                    }
+            } else {
+                float rv[KP];
+                int ri[KP];
+#pragma unroll
+                for (int e = 0; e < KP; ++e) {
+                    rv[e] = e < K ? Rv[e * S] : -INFINITY;
+                    ri[e] = e < K ? (int)Ri[e * S] : 0x7fffffff;
+                }
+                bitonic_merge_keep<KP>(rv, ri, a, ai);
+#pragma unroll
+                for (int e = 0; e < KP; ++e)
+                    if (e < K) {
+                        Rv[e * S] = rv[e];
+                        Ri[e * S] = (uint16_t)ri[e];
+                    }
+            }
+            ptx::fence_proxy_async_smem();  // these generic writes precede the next TMA write
+            ptx::tc_fence_before();
+            __syncthreads();
+        }
+    }
+
+    if (!aborted) {
+        // k x k combine: max-heap over rows a of R0 (column b advances along R1)
+        const int W = p.top;
+        float* hv = reinterpret_cast<float*>(sm + TC_OFF_B) + tid;
+        uint32_t* hab = reinterpret_cast<uint32_t*>(sm + TC_OFF_B + K * S * 4) + tid;
+        float* sv = reinterpret_cast<float*>(sm + TC_OFF_HIST) + tid;
+        int size = min(K, W);
+        const float r1_0 = R1v[0];
+        for (int e = 0; e < size; ++e) {
+            hv[e * S] = R0v[e * S] + r1_0;
+            hab[e * S] = (uint32_t)e << 16;
+        }
+        auto slot_of = [&](uint32_t ab) -> int {
+            return (int)R0i[(ab >> 16) * S] * n + (int)R1i[(ab & 0xffffu) * S];
+        };
+        auto hbetter = [&](int x, int y) -> bool {
+            const float vx = hv[x * S], vy = hv[y * S];
+            if (vx != vy) return vx > vy;
+            return slot_of(hab[x * S]) < slot_of(hab[y * S]);
+        };
+        const size_t row_off = ((size_t)b * p.H + h) * p.T + t;
+        for (int q = 0; q < W; ++q) {
+            if (size <= 0) {  // cannot happen for top <= k_half^2; keep outputs defined
+                sv[q * S] = -INFINITY;
+                if (row_ok) p.idx[row_off * W + q] = -1;
+                continue;
+            }
+            const uint32_t ab = hab[0];
+            sv[q * S] = hv[0];
+            if (row_ok) p.idx[row_off * W + q] = slot_of(ab);
+            const int ra = (int)(ab >> 16), cb = (int)(ab & 0xffffu) + 1;
+            if (cb < K && (ra + 1) * (cb + 1) <= W) {
+                hv[0] = R0v[ra * S] + R1v[cb * S];
+                hab[0] = ((uint32_t)ra << 16) | (uint32_t)cb;
+            } else {
+                --size;
+                hv[0] = hv[size * S];
+                hab[0] = hab[size * S];
+            }
+            int pos = 0;
+            while (true) {
+                const int c1 = 2 * pos + 1;
+                if (c1 >= size) break;
+                const int c2 = c1 + 1;
+                const int best = (c2 < size && hbetter(c2, c1)) ? c2 : c1;
+                if (!hbetter(best, pos)) break;
+                const float tv = hv[pos * S];
+                const uint32_t tab = hab[pos * S];
+                hv[pos * S] = hv[best * S];
+                hab[pos * S] = hab[best * S];
+                hv[best * S] = tv;
+                hab[best * S] = tab;
+                pos = best;
+            }
+        }
+        if (row_ok) {
+            const float mx = sv[0];
+            float z = 0.f;
+            for (int q = 0; q < W; ++q) z += expf(sv[q * S] - mx);
+            for (int q = 0; q < W; ++q) p.w[row_off * W + q] = expf(sv[q * S] - mx) / z;
+        }
+    } else if (tid == 0) {
+        raise_err(SDM_DEVERR_TIMEOUT);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, TC_NB);
+    }
+}
+
+}  // namespace sdm

@@ -11,6 +11,7 @@
 #include "plan.cuh"
 #include "recur.cuh"
 #include "score_simt.cuh"
+#include "score_tc.cuh"
 #include "state.cuh"
 
 using namespace sdm;
@@ -116,10 +117,95 @@ sdm_status check_state(const sdm_state* st) {
     return SDM_OK;
 }
 
+// ---- tensor-core scoring: TMA descriptors and dispatch ------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// Shapes the tensor-core kernel takes: bf16, 64-wide halves, sub-key count a multiple of 64,
+// at most 32 kept per half and selected, and enough tokens per sequence for full tiles
+// (single-token decode stays on the CUDA-core kernel, which spreads rows over all SMs).
+bool score_tc_eligible(const sdm_dims* d, int top) {
+    if (d->x_dtype != SDM_BF16 || d->d_k != 128) return false;
+    if (d->n_sub % 64 != 0 || d->n_sub > 4096) return false;
+    if (d->k_half > TC_KMAX || top > TC_KMAX) return false;
+    if (d->n_sub > TC_NB && d->k_half * TC_THREADS * 6 > 16384) return false;  // R1 beside x half 1
+    return d->T >= 64;
+}
+
+template <int KP>
+sdm_status launch_score_tc_t(const sdm_dims* d, const CUtensorMap& xm, const CUtensorMap& km,
+                             const ScoreTcArgs& a, dim3 grid, cudaStream_t s) {
+    auto kern = score_tc_kernel<KP>;
+    if (!set_smem(kern, TC_SMEM_BYTES)) return SDM_ERR_CUDA;
+    kern<<<grid, TC_THREADS, TC_SMEM_BYTES, s>>>(xm, km, a);
+    return launch_status();
+}
+
+sdm_status launch_score_tc(const sdm_dims* d, const void* x, const void* sk, int top,
+                           int32_t* idx, float* w, cudaStream_t s) {
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return SDM_ERR_CUDA;
+    ScoreTcArgs a{};
+    a.B = d->B; a.H = d->H; a.T = d->T; a.n = d->n_sub; a.k_half = d->k_half; a.top = top;
+    a.nbox = d->n_sub < TC_NB ? d->n_sub : TC_NB;
+    a.bt = d->T >= 128 ? 128 : d->T;
+    a.bb = 128 / a.bt;
+    if (a.bb > d->B) a.bb = d->B;
+    a.n_tt = (d->T + a.bt - 1) / a.bt;
+    a.idx = idx;
+    a.w = w;
+    const int n_bt = (d->B + a.bb - 1) / a.bb;
+    CUtensorMap xm, km;
+    {
+        const cuuint64_t dims[4] = {(cuuint64_t)d->d_k, (cuuint64_t)d->T, (cuuint64_t)d->H,
+                                    (cuuint64_t)d->B};
+        const cuuint64_t strides[3] = {(cuuint64_t)d->d_k * 2, (cuuint64_t)d->T * d->d_k * 2,
+                                       (cuuint64_t)d->H * d->T * d->d_k * 2};
+        const cuuint32_t box[4] = {64, (cuuint32_t)a.bt, 1, (cuuint32_t)a.bb};
+        const cuuint32_t es[4] = {1, 1, 1, 1};
+        if (enc(&xm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims, strides, box,
+                es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return SDM_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {64, (cuuint64_t)d->H * 2 * d->n_sub};
+        const cuuint64_t strides[1] = {64 * 2};
+        const cuuint32_t box[2] = {64, (cuuint32_t)a.nbox};
+        const cuuint32_t es[2] = {1, 1};
+        if (enc(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(sk), dims, strides, box,
+                es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return SDM_ERR_CUDA;
+    }
+    const dim3 grid((unsigned)(a.n_tt * n_bt), (unsigned)d->H);
+    const int k = d->k_half;
+    if (k <= 8) return launch_score_tc_t<8>(d, xm, km, a, grid, s);
+    if (k <= 16) return launch_score_tc_t<16>(d, xm, km, a, grid, s);
+    return launch_score_tc_t<32>(d, xm, km, a, grid, s);
+}
+
 sdm_status launch_score(const sdm_dims* d, const void* x, const void* sk, int top, int32_t* idx,
                         float* w, cudaStream_t s) {
     const long long rows = (long long)d->B * d->T;
     if (rows == 0) return SDM_OK;
+    if (score_tc_eligible(d, top)) return launch_score_tc(d, x, sk, top, idx, w, s);
     const int threads = 128, warps = threads / 32;
     const size_t smem =
         (size_t)warps * score_simt_warp_floats(d->d_k, d->n_sub, d->k_half, top) * sizeof(float);
