@@ -16,7 +16,10 @@
 //                   bit 16: o is the last write of its slot in the chunk (stores it);
 //                   bit 17: o's accumulated in-chunk delta must be kept (a later
 //                   occurrence links to it, or it stores and has a link)
-//     tmask[t]    = {write-link bits, read-link bits, keep-delta bits} over the W / R slots
+//     tmask[t]    = {write-link bits, read-link bits, keep-delta bits, level}: the bits run
+//                   over the token's W / R slots; level 0 = no in-chunk link, otherwise
+//                   1 + the largest level among the earlier tokens it links to (tokens of
+//                   one level can be resolved together once the lower levels are done)
 //     st0[o]      = the state's stamp of o's slot at call entry (NaN: pristine)
 //   plan_walk (one CTA per (b,h), chunks in order)
 //     Lstart[j]   = log-decay prefix at the start of chunk j (Lstart[0] = state Lambda)
@@ -81,7 +84,7 @@ struct PlanPtrs {
     double* st0;       // [BH][T*(W+R)]
     float* fe;         // [BH][T*(W+R)]
     int32_t* lk;       // [BH][T*(W+R)]
-    uint64_t* tmask;   // [BH][T][3]
+    uint64_t* tmask;   // [BH][T][4]
     int32_t* lastw;    // [BH][N] (only when the walk table does not fit in shared memory)
 };
 
@@ -97,6 +100,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
     __shared__ unsigned char s_need[PLAN_MAX_OCC];
     __shared__ unsigned char s_owner[PLAN_MAX_OCC];
     __shared__ unsigned long long s_mask[3 * PLAN_THREADS];
+    __shared__ int s_level[PLAN_THREADS];
 
     const int j = blockIdx.x;
     const size_t bh = blockIdx.y;
@@ -189,6 +193,28 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
     }
     __syncthreads();
 
+    // 5b. levels: longest chain of in-chunk links ending at each token
+    for (int t = tid; t < nt; t += PLAN_THREADS)
+        s_level[t] = (s_mask[3 * t] | s_mask[3 * t + 1]) ? 1 : 0;
+    __syncthreads();
+    for (int it = 0; it < nt; ++it) {
+        int changed = 0;
+        for (int o = tid; o < no; o += PLAN_THREADS) {
+            const int link = s_link[o];
+            if (link < 0) continue;
+            const int tl = o < nw ? o / W : (o - nw) / R;
+            const int tp = link / W;
+            if (tp < tl) {
+                const int want = s_level[tp] + 1;
+                if (s_level[tp] > 0 && want > s_level[tl]) {
+                    atomicMax(&s_level[tl], want);
+                    changed = 1;
+                }
+            }
+        }
+        if (!__syncthreads_or(changed)) break;
+    }
+
     // 6. write out
     for (int o = tid; o < no; o += PLAN_THREADS) {
         const int link = s_link[o];
@@ -207,8 +233,13 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
         const int s = s_slot[o];
         P.st0[g] = s >= 0 ? stamp[bh * (size_t)N + s] : 0.0;
     }
-    for (int i = tid; i < 3 * nt; i += PLAN_THREADS)
-        P.tmask[(bh * T + t0) * 3 + i] = s_mask[i];
+    for (int t = tid; t < nt; t += PLAN_THREADS) {
+        uint64_t* tm = P.tmask + (bh * T + t0 + t) * 4;
+        tm[0] = s_mask[3 * t];
+        tm[1] = s_mask[3 * t + 1];
+        tm[2] = s_mask[3 * t + 2];
+        tm[3] = (uint64_t)s_level[t];
+    }
 }
 
 // Sequential walk over the chunks of one (b,h).  Table: last chunk of this call that

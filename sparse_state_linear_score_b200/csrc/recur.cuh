@@ -13,7 +13,8 @@
 //   in-chunk writes are carried as accumulated deltas A[o] (value added to the slot by the
 //   writes of this chunk up to occurrence o, decayed to o's token):
 //            A[o]     = e^{lam_t - lam_tp} A[link(o)] + w_o d_t
-//   linked tokens, in token order (one warp, lanes = columns):
+//   linked tokens, level by level (the plan gives each token 1 + the largest level of the
+//   earlier tokens it links to; all tokens of one level are resolved in parallel):
 //            P_t      = P0_t + sum_{i linked} w_i e^{lam_t - lam_tp} A[link]
 //            d_t      = beta_t (v_t - P_t)
 //            o_t      = Q0_t + sum_{j linked} u_j e^{lam_t - lam_tp} A[link]   (read after write)
@@ -31,22 +32,32 @@
 
 namespace sdm {
 
-constexpr int RUN_THREADS = 256;
+constexpr int RUN_THREADS = 512;
+constexpr int RUN_PAD = 8;  // floats between token blocks: spreads a warp's rows over banks
+
+// Floats per token block of gathered rows (and of A): its slots' CW-wide slices + padding.
+__host__ __device__ inline int run_tok_stride(int per_tok, int CW) { return per_tok * CW + RUN_PAD; }
 
 __host__ __device__ inline size_t run_smem_bytes(int C, int W, int R, int CW) {
-    const size_t no = (size_t)C * (W + R), nw = (size_t)C * W;
+    const size_t tsw = (size_t)run_tok_stride(W, CW), tsr = (size_t)run_tok_stride(R, CW);
+    const size_t no = (size_t)C * (W + R);
     size_t b = 0;
-    b += no * CW * 4;                   // rows
-    b += nw * CW * 4;                   // A
+    b += (size_t)C * (tsw + tsr) * 4;   // rows: write blocks, then read blocks
+    b += (size_t)C * tsw * 4;           // A (accumulated in-chunk deltas of write occurrences)
     b += (size_t)4 * C * CW * 4;        // v, P, d, o
-    b += (size_t)3 * C * 8;             // masks
-    b += (size_t)2 * C * 4;             // lam, beta
+    b += (size_t)3 * C * 8;             // link masks
+    b += (size_t)3 * C * 4;             // lam, beta, level
     b += no * 4 * 5;                    // slot, coef, w, fe, lk
     return b;
 }
 
+SDM_DEV void cp_async4(void* smem_dst, const void* gmem_src) {
+    unsigned dst = (unsigned)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(gmem_src) : "memory");
+}
+
 template <int CW, typename VT>
-__global__ void __launch_bounds__(RUN_THREADS) recur_run_kernel(
+__global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
     const VT* __restrict__ v, const float* __restrict__ beta, const int32_t* __restrict__ widx,
     const float* __restrict__ ww, const int32_t* __restrict__ ridx, const float* __restrict__ rw,
     const float* __restrict__ fe, const int32_t* __restrict__ lk, const float* __restrict__ lam,
@@ -64,134 +75,164 @@ __global__ void __launch_bounds__(RUN_THREADS) recur_run_kernel(
     const float* M0h = M0 + (size_t)h * N * d_v;
     const size_t occ_base = bh * (size_t)T * (W + R);
     const int tid = threadIdx.x;
+    const int tsw = run_tok_stride(W, CW), tsr = run_tok_stride(R, CW);
 
-    const int nomax = C * (W + R), nwmax = C * W;
+    const int nomax = C * (W + R);
     float* s_rows = reinterpret_cast<float*>(run_smem);
-    float* s_A = s_rows + (size_t)nomax * CW;
-    float* s_v = s_A + (size_t)nwmax * CW;
+    float* s_rrows = s_rows + (size_t)C * tsw;  // read blocks
+    float* s_A = s_rrows + (size_t)C * tsr;
+    float* s_v = s_A + (size_t)C * tsw;
     float* s_P = s_v + C * CW;
     float* s_d = s_P + C * CW;
     float* s_o = s_d + C * CW;
     unsigned long long* s_mask = reinterpret_cast<unsigned long long*>(s_o + C * CW);
     float* s_lam = reinterpret_cast<float*>(s_mask + 3 * C);
     float* s_beta = s_lam + C;
-    int* s_slot = reinterpret_cast<int*>(s_beta + C);
+    int* s_lev = reinterpret_cast<int*>(s_beta + C);
+    int* s_slot = s_lev + C;
     float* s_coef = reinterpret_cast<float*>(s_slot + nomax);
     float* s_w = s_coef + nomax;
     float* s_fe = s_w + nomax;
     int* s_lk = reinterpret_cast<int*>(s_fe + nomax);
 
+    // position of a write occurrence's (or its A's) slice, and of a read occurrence's slice
+    auto wpos = [&](int o) { return (o / W) * tsw + (o % W) * CW; };
+    auto rpos = [&](int o) { return (o / R) * tsr + (o % R) * CW; };
+
     for (int j = 0; j < J; ++j) {
         const int t0 = j * C, nt = min(C, T - t0);
         const int nw = nt * W, no = nt * (W + R);
 
-        // 1. chunk metadata
+        // 1. chunk metadata, copied asynchronously
         for (int o = tid; o < no; o += RUN_THREADS) {
-            int s;
-            float w;
+            const int32_t* si;
+            const float* sw;
             size_t g;
             if (o < nw) {
                 const size_t gi = (bh * T + t0) * W + o;
-                s = widx[gi];
-                w = ww[gi];
+                si = widx + gi;
+                sw = ww + gi;
                 g = occ_base + (size_t)t0 * W + o;
             } else {
                 const size_t gi = (bh * T + t0) * R + (o - nw);
-                s = ridx[gi];
-                w = rw[gi];
+                si = ridx + gi;
+                sw = rw + gi;
                 g = occ_base + (size_t)T * W + (size_t)t0 * R + (o - nw);
             }
-            const float f = fe[g];
-            s_slot[o] = s;
-            s_w[o] = w;
-            s_fe[o] = f;
-            s_coef[o] = w * fabsf(f);
-            s_lk[o] = lk[g];
+            cp_async4(&s_slot[o], si);
+            cp_async4(&s_w[o], sw);
+            cp_async4(&s_fe[o], fe + g);
+            cp_async4(&s_lk[o], lk + g);
         }
-        for (int t = tid; t < nt; t += RUN_THREADS) {
-            s_lam[t] = lam[bh * T + t0 + t];
-            s_beta[t] = beta[bh * T + t0 + t];
-            s_mask[3 * t + 0] = tmask[(bh * T + t0 + t) * 3 + 0];
-            s_mask[3 * t + 1] = tmask[(bh * T + t0 + t) * 3 + 1];
-            s_mask[3 * t + 2] = tmask[(bh * T + t0 + t) * 3 + 2];
+        cp_async_commit();
+        if (tid < nt) {
+            const size_t tg = bh * T + t0 + tid;
+            s_lam[tid] = lam[tg];
+            s_beta[tid] = beta[tg];
+            s_mask[3 * tid + 0] = tmask[tg * 4 + 0];
+            s_mask[3 * tid + 1] = tmask[tg * 4 + 1];
+            s_mask[3 * tid + 2] = tmask[tg * 4 + 2];
+            s_lev[tid] = (int)tmask[tg * 4 + 3];
         }
         for (int e = tid; e < nt * CW; e += RUN_THREADS) {
             const int t = e / CW, c = e % CW;
             s_v[e] = to_f32(v[(bh * T + t0 + t) * d_v + c0 + c]);
         }
+        cp_async_wait_all();
         __syncthreads();
 
-        // 2. gather the row slices as stored at chunk start
-        for (int e = tid; e < no * Q; e += RUN_THREADS) {
-            const int o = e / Q, q = e % Q;
+        // 2. gather the row slices as stored at chunk start (from M, or M0 while pristine)
+        for (int o = tid; o < no; o += RUN_THREADS) {
+            const float f = s_fe[o];
+            s_coef[o] = s_w[o] * fabsf(f);
             const int s = s_slot[o];
             const bool ok = slot_ok(s, N);
-            const float* src = (signbit(s_fe[o]) ? M0h : Mb) + (ok ? (size_t)s * d_v : 0) + c0 + 4 * q;
-            cp_async16(&s_rows[(size_t)o * CW + 4 * q], src, ok);
+            const float* src = (signbit(f) ? M0h : Mb) + (ok ? (size_t)s * d_v : 0) + c0;
+            float* dst = o < nw ? s_rows + wpos(o) : s_rrows + rpos(o - nw);
+#pragma unroll
+            for (int q = 0; q < Q; ++q) cp_async16(dst + 4 * q, src + 4 * q, ok);
         }
         cp_async_commit();
         cp_async_wait_all();
         __syncthreads();
 
-        // 3. predictions and reads from the chunk-start memory
-        for (int e = tid; e < nt * CW; e += RUN_THREADS) {
+        // 3. predictions (writes) and reads from the chunk-start memory
+        for (int task = tid; task < 2 * nt * CW; task += RUN_THREADS) {
+            const bool rd = task >= nt * CW;
+            const int e = rd ? task - nt * CW : task;
             const int t = e / CW, c = e % CW;
-            float p = 0.f, qv = 0.f;
-            const int ow = t * W, orr = nw + t * R;
-            for (int i = 0; i < W; ++i) p = fmaf(s_coef[ow + i], s_rows[(size_t)(ow + i) * CW + c], p);
-            for (int i = 0; i < R; ++i) qv = fmaf(s_coef[orr + i], s_rows[(size_t)(orr + i) * CW + c], qv);
-            s_P[e] = p;
-            s_d[e] = s_beta[t] * (s_v[e] - p);
-            s_o[e] = qv;
-        }
-        __syncthreads();
-        // accumulated deltas of tokens without links: A = w d
-        for (int e = tid; e < nw * CW; e += RUN_THREADS) {
-            const int o = e / CW, c = e % CW;
-            const int t = o / W;
-            if ((s_lk[o] & LK_KEEP) && !(s_mask[3 * t] | s_mask[3 * t + 1]))
-                s_A[e] = s_w[o] * s_d[t * CW + c];
-        }
-        __syncthreads();
-
-        // 4. tokens with in-chunk links, in order
-        if (tid < 32) {
-            const int c = tid;
-            for (int t = 0; t < nt; ++t) {
-                const unsigned long long wm = s_mask[3 * t], rm = s_mask[3 * t + 1],
-                                         am = s_mask[3 * t + 2];
-                if (!(wm | rm)) continue;
-                if (c < CW) {
-                    const float lt = s_lam[t];
-                    float p = s_P[t * CW + c];
-                    for (unsigned long long m = wm; m; m &= m - 1) {
-                        const int o = t * W + (__ffsll((long long)m) - 1);
-                        const int L = lk_link(s_lk[o]);
-                        if (L < 0) continue;
-                        p = fmaf(s_w[o] * expf(lt - s_lam[L / W]), s_A[(size_t)L * CW + c], p);
-                    }
-                    const float d = s_beta[t] * (s_v[t * CW + c] - p);
-                    s_d[t * CW + c] = d;
-                    for (unsigned long long m = am; m; m &= m - 1) {
-                        const int o = t * W + (__ffsll((long long)m) - 1);
-                        const int L = lk_link(s_lk[o]);
-                        float a = s_w[o] * d;
-                        if (L >= 0) a = fmaf(expf(lt - s_lam[L / W]), s_A[(size_t)L * CW + c], a);
-                        s_A[(size_t)o * CW + c] = a;
-                    }
-                    float qv = s_o[t * CW + c];
-                    for (unsigned long long m = rm; m; m &= m - 1) {
-                        const int o = nw + t * R + (__ffsll((long long)m) - 1);
-                        const int L = lk_link(s_lk[o]);
-                        if (L < 0) continue;
-                        qv = fmaf(s_w[o] * expf(lt - s_lam[L / W]), s_A[(size_t)L * CW + c], qv);
-                    }
-                    s_o[t * CW + c] = qv;
-                }
-                __syncwarp();
+            float acc = 0.f;
+            if (!rd) {
+                const float* rr = s_rows + t * tsw + c;
+                const float* cf = s_coef + t * W;
+                for (int i = 0; i < W; ++i) acc = fmaf(cf[i], rr[i * CW], acc);
+                s_P[e] = acc;
+                s_d[e] = s_beta[t] * (s_v[e] - acc);
+            } else {
+                const float* rr = s_rrows + t * tsr + c;
+                const float* cf = s_coef + nw + t * R;
+                for (int i = 0; i < R; ++i) acc = fmaf(cf[i], rr[i * CW], acc);
+                s_o[e] = acc;
             }
         }
         __syncthreads();
+        // accumulated deltas of kept write occurrences of tokens without links: A = w d
+        for (int o = tid; o < nw; o += RUN_THREADS) {
+            const int t = o / W;
+            if (!(s_lk[o] & LK_KEEP) || s_lev[t] != 0) continue;
+            const float w = s_w[o];
+            float* a = s_A + wpos(o);
+            const float* dd = s_d + t * CW;
+#pragma unroll
+            for (int c = 0; c < CW; ++c) a[c] = w * dd[c];
+        }
+
+        // 4. tokens with in-chunk links, one level at a time (the barrier of each test
+        //    also closes the previous phase)
+        for (int lev = 1;; ++lev) {
+            const bool mine = tid < nt && s_lev[tid] == lev;
+            if (!__syncthreads_or(mine)) break;
+            for (int e = tid; e < nt * CW; e += RUN_THREADS) {
+                const int t = e / CW, c = e % CW;
+                if (s_lev[t] != lev) continue;
+                const float lt = s_lam[t];
+                float p = s_P[e];
+                for (unsigned long long m = s_mask[3 * t]; m; m &= m - 1) {
+                    const int o = t * W + (__ffsll((long long)m) - 1);
+                    const int L = lk_link(s_lk[o]);
+                    if (L < 0) continue;
+                    p = fmaf(s_w[o] * expf(lt - s_lam[L / W]), s_A[wpos(L) + c], p);
+                }
+                s_d[e] = s_beta[t] * (s_v[e] - p);
+            }
+            __syncthreads();
+            for (int e = tid; e < nt * CW; e += RUN_THREADS) {
+                const int t = e / CW, c = e % CW;
+                if (s_lev[t] != lev) continue;
+                const float lt = s_lam[t], d = s_d[e];
+                for (unsigned long long m = s_mask[3 * t + 2]; m; m &= m - 1) {
+                    const int o = t * W + (__ffsll((long long)m) - 1);
+                    const int L = lk_link(s_lk[o]);
+                    float a = s_w[o] * d;
+                    if (L >= 0) a = fmaf(expf(lt - s_lam[L / W]), s_A[wpos(L) + c], a);
+                    s_A[wpos(o) + c] = a;
+                }
+            }
+            __syncthreads();
+            for (int e = tid; e < nt * CW; e += RUN_THREADS) {
+                const int t = e / CW, c = e % CW;
+                if (s_lev[t] != lev) continue;
+                const float lt = s_lam[t];
+                float qv = s_o[e];
+                for (unsigned long long m = s_mask[3 * t + 1]; m; m &= m - 1) {
+                    const int o = nw + t * R + (__ffsll((long long)m) - 1);
+                    const int L = lk_link(s_lk[o]);
+                    if (L < 0) continue;
+                    qv = fmaf(s_w[o] * expf(lt - s_lam[L / W]), s_A[wpos(L) + c], qv);
+                }
+                s_o[e] = qv;
+            }
+        }
 
         // 5. outputs
         for (int e = tid; e < nt * Q; e += RUN_THREADS) {
@@ -203,14 +244,14 @@ __global__ void __launch_bounds__(RUN_THREADS) recur_run_kernel(
         const float lam_end = s_lam[nt - 1];
         for (int e = tid; e < nw * Q; e += RUN_THREADS) {
             const int o = e / Q, q = e % Q;
+            const int lko = s_lk[o];
             const int s = s_slot[o];
-            if (!(s_lk[o] & LK_OWNER) || !slot_ok(s, N)) continue;
-            const int t = o / W, i = o % W;
-            const bool linked = (s_mask[3 * t] >> i) & 1ull;
-            const float4 raw = reinterpret_cast<const float4*>(s_rows + (size_t)o * CW)[q];
+            if (!(lko & LK_OWNER) || !slot_ok(s, N)) continue;
+            const int t = o / W;
+            const float4 raw = reinterpret_cast<const float4*>(s_rows + wpos(o))[q];
             float4 a;
-            if (linked) {
-                a = reinterpret_cast<const float4*>(s_A + (size_t)o * CW)[q];
+            if (lk_link(lko) >= 0) {
+                a = reinterpret_cast<const float4*>(s_A + wpos(o))[q];
             } else {
                 const float4 dd = reinterpret_cast<const float4*>(s_d + t * CW)[q];
                 const float w = s_w[o];

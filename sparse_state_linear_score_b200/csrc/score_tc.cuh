@@ -104,10 +104,19 @@ SDM_DEV void bitonic_merge_keep(float (&r)[KP], int (&ri)[KP], const float (&a)[
     }
 }
 
+// Bin of v in the refinement chain lo/sc/tb[0..L): -1 when v is outside the chain (rare path).
+SDM_DEV int tc_chain_bin(float v, const float* lo, const float* sc, const int* tb, int L) {
+    for (int l = 0; l < L; ++l)
+        if (tc_bin(v, lo[l], sc[l]) != tb[l]) return -1;
+    return tc_bin(v, lo[L], sc[L]);
+}
+
 // The K best of this thread's NB TMEM columns (sub-index = col_base + column), returned
 // sorted best-first in a[0..K) (entries K..KP-1 are padding).  Per-thread shared arrays
 // are strided by TC_THREADS.  Every TMEM pass is executed by whole warps (tcgen05.ld is
 // warp-collective); the per-thread state only predicates the work inside a pass.
+// Level 0 (64 bins over [min, max]) is the fast path; the rare refinement levels (more
+// than TC_BC scores in the threshold bin, or all scores equal) run a compact generic loop.
 template <int KP>
 SDM_DEV void tc_select(uint32_t trow, int NB, int K, int col_base, uint16_t* hist, float* Sv,
                        uint16_t* Si, float* Bv, uint16_t* Bi, float (&a)[KP], int (&ai)[KP]) {
@@ -130,113 +139,149 @@ SDM_DEV void tc_select(uint32_t trow, int NB, int K, int col_base, uint16_t* his
     int tb[TC_MAXLEV];
     lo[0] = flat ? 0.f : mn;
     sc[0] = flat ? 0.f : (float)TC_NBIN / (mx - mn);
-    bool done = false;
+
+    // ---- level 0: histogram, threshold, compaction (fast path) ----
+    int t_b = 0, cum = 0, cnt_tb = 0;
+    if (!flat)
+        for (int bn = 0; bn < TC_NBIN; ++bn) hist[bn * S] = 0;
+    for (int c = 0; c < NB; c += 32) {
+        float v[32];
+        ptx::tmem_ld32(trow + c, v);
+        if (!flat) {
 #pragma unroll
-    for (int L = 0; L < TC_MAXLEV; ++L) {
-        const bool hist_on = !done && !flat;
-        int t_b = 0, cum = 0, cnt_tb = 0;
-        if (__any_sync(FULL, hist_on)) {
-            if (hist_on)
-                for (int bn = 0; bn < TC_NBIN; ++bn) hist[bn * S] = 0;
-            for (int c = 0; c < NB; c += 32) {
-                float v[32];
-                ptx::tmem_ld32(trow + c, v);
-                if (hist_on) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        bool in = true;
-#pragma unroll
-                        for (int l = 0; l < L; ++l) in = in && tc_bin(v[i], lo[l], sc[l]) == tb[l];
-                        if (in) {
-                            const int bn = tc_bin(v[i], lo[L], sc[L]);
-                            hist[bn * S] = (uint16_t)(hist[bn * S] + 1);
-                        }
-                    }
-                }
-            }
-            if (hist_on) {
-                for (int bn = TC_NBIN - 1; bn >= 0; --bn) {
-                    const int cnt = hist[bn * S];
-                    if (cum + cnt >= need) {
-                        t_b = bn;
-                        break;
-                    }
-                    cum += cnt;
-                }
-                cnt_tb = hist[t_b * S];
+            for (int i = 0; i < 32; ++i) {
+                const int bn = tc_bin(v[i], lo[0], sc[0]);
+                hist[bn * S] = (uint16_t)(hist[bn * S] + 1);
             }
         }
-        tb[L] = t_b;
-        const bool small = cnt_tb <= TC_BC;
-        const bool last = small || L == TC_MAXLEV - 1;
-        const bool flat_take = flat && !done && L == 0;
-        const bool comp_on = hist_on || flat_take;
-        int nbd = 0;
-        int take_direct = flat_take ? need : (hist_on && last && !small ? need - cum : 0);
-        if (__any_sync(FULL, comp_on)) {
-            for (int c = 0; c < NB; c += 32) {
-                float v[32];
-                ptx::tmem_ld32(trow + c, v);
-                if (comp_on) {
+    }
+    if (!flat) {
+        for (int bn = TC_NBIN - 1; bn >= 0; --bn) {
+            const int cnt = hist[bn * S];
+            if (cum + cnt >= need) {
+                t_b = bn;
+                break;
+            }
+            cum += cnt;
+        }
+        cnt_tb = hist[t_b * S];
+    }
+    tb[0] = t_b;
+    bool small = !flat && cnt_tb <= TC_BC;
+    int nbd = 0;
+    for (int c = 0; c < NB; c += 32) {
+        float v[32];
+        ptx::tmem_ld32(trow + c, v);
+        if (!flat) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const uint16_t col = (uint16_t)(col_base + c + i);
-                        if (flat_take) {
-                            if (take_direct > 0) {
-                                Sv[ns * S] = v[i];
-                                Si[ns * S] = col;
-                                ++ns;
-                                --take_direct;
-                            }
-                            continue;
-                        }
-                        bool in = true;
-#pragma unroll
-                        for (int l = 0; l < L; ++l) in = in && tc_bin(v[i], lo[l], sc[l]) == tb[l];
-                        if (!in) continue;
-                        const int bn = tc_bin(v[i], lo[L], sc[L]);
-                        if (bn > t_b) {
+            for (int i = 0; i < 32; ++i) {
+                const int bn = tc_bin(v[i], lo[0], sc[0]);
+                if (bn > t_b) {
+                    Sv[ns * S] = v[i];
+                    Si[ns * S] = (uint16_t)(col_base + c + i);
+                    ++ns;
+                } else if (small && bn == t_b) {
+                    Bv[nbd * S] = v[i];
+                    Bi[nbd * S] = (uint16_t)(col_base + c + i);
+                    ++nbd;
+                }
+            }
+        }
+    }
+    if (!flat) need -= cum;
+    bool done = small;
+
+    // ---- rare: refinement levels, or all-equal scores ----
+    // The loop condition is warp-uniform; inactive lanes still take part in the TMEM loads.
+    int L = 0;
+    while (__any_sync(FULL, !done)) {
+        const bool act = !done;
+        if (act && !flat) {  // refine inside the crowded threshold bin of level L
+            lo[L + 1] = lo[L] + (float)tb[L] / sc[L];
+            sc[L + 1] = sc[L] * (float)TC_NBIN;
+            ++L;
+        }
+        // flat rows, or the deepest level: take the chain members in index order
+        const bool last = act && (flat || L == TC_MAXLEV - 1);
+        const bool refine = act && !last;
+        int cum2 = 0, t2 = 0, cnt2 = 0;
+        if (refine)
+            for (int bn = 0; bn < TC_NBIN; ++bn) hist[bn * S] = 0;
+        for (int c = 0; c < NB; c += 32) {
+            float v[32];
+            ptx::tmem_ld32(trow + c, v);
+            if (refine) {
+#pragma unroll 1
+                for (int i = 0; i < 32; ++i) {
+                    const int bn = tc_chain_bin(v[i], lo, sc, tb, L);
+                    if (bn >= 0) hist[bn * S] = (uint16_t)(hist[bn * S] + 1);
+                }
+            }
+        }
+        if (refine) {
+            for (int bn = TC_NBIN - 1; bn >= 0; --bn) {
+                const int cnt = hist[bn * S];
+                if (cum2 + cnt >= need) {
+                    t2 = bn;
+                    break;
+                }
+                cum2 += cnt;
+            }
+            cnt2 = hist[t2 * S];
+            tb[L] = t2;
+        }
+        const bool small2 = refine && cnt2 <= TC_BC;
+        if (small2) nbd = 0;
+        int take_direct = last ? need : 0;
+        for (int c = 0; c < NB; c += 32) {
+            float v[32];
+            ptx::tmem_ld32(trow + c, v);
+            if (act) {
+#pragma unroll 1
+                for (int i = 0; i < 32; ++i) {
+                    const uint16_t col = (uint16_t)(col_base + c + i);
+                    const int bn = flat ? 0 : tc_chain_bin(v[i], lo, sc, tb, L);
+                    if (bn < 0) continue;
+                    if (last) {
+                        if (take_direct > 0) {
                             Sv[ns * S] = v[i];
                             Si[ns * S] = col;
                             ++ns;
-                        } else if (bn == t_b) {
-                            if (last && small) {
-                                Bv[nbd * S] = v[i];
-                                Bi[nbd * S] = col;
-                                ++nbd;
-                            } else if (take_direct > 0) {  // crowded last level: index order
-                                Sv[ns * S] = v[i];
-                                Si[ns * S] = col;
-                                ++ns;
-                                --take_direct;
-                            }
+                            --take_direct;
                         }
+                    } else if (bn > t2) {
+                        Sv[ns * S] = v[i];
+                        Si[ns * S] = col;
+                        ++ns;
+                    } else if (small2 && bn == t2) {
+                        Bv[nbd * S] = v[i];
+                        Bi[nbd * S] = col;
+                        ++nbd;
                     }
                 }
             }
         }
-        if (flat_take) {
+        if (last) {
             done = true;
-        } else if (hist_on) {
-            need -= cum;
-            if (last) {
-                if (small) {  // the `need` best of the boundary bin, by exact rank
-                    for (int e = 0; e < nbd; ++e) {
-                        const float ve = Bv[e * S];
-                        const int ie = Bi[e * S];
-                        int rank = 0;
-                        for (int f = 0; f < nbd; ++f) rank += better(Bv[f * S], Bi[f * S], ve, ie);
-                        if (rank < need) {
-                            Sv[ns * S] = ve;
-                            Si[ns * S] = (uint16_t)ie;
-                            ++ns;
-                        }
-                    }
-                }
+        } else if (refine) {
+            need -= cum2;
+            if (small2) {
                 done = true;
-            } else if (L + 1 < TC_MAXLEV) {
-                lo[L + 1] = lo[L] + (float)t_b / sc[L];
-                sc[L + 1] = sc[L] * (float)TC_NBIN;
+                small = true;  // pick the remaining `need` from this level's boundary list
+            }
+        }
+    }
+    // the `need` best of the boundary bin, by exact rank
+    if (small) {
+        for (int e = 0; e < nbd; ++e) {
+            const float ve = Bv[e * S];
+            const int ie = Bi[e * S];
+            int rank = 0;
+            for (int f = 0; f < nbd; ++f) rank += better(Bv[f * S], Bi[f * S], ve, ie);
+            if (rank < need) {
+                Sv[ns * S] = ve;
+                Si[ns * S] = (uint16_t)ie;
+                ++ns;
             }
         }
     }

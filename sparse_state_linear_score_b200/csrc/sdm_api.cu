@@ -79,7 +79,7 @@ WsLayout ws_layout(const sdm_dims* d) {
     L.off_st0 = o;    o = up256(o + BH * occ * 8);
     L.off_fe = o;     o = up256(o + BH * occ * 4);
     L.off_lk = o;     o = up256(o + BH * occ * 4);
-    L.off_tmask = o;  o = up256(o + BH * T * 3 * 8);
+    L.off_tmask = o;  o = up256(o + BH * T * 4 * 8);
     L.off_lastw = o;  o = up256(o + (L.smem_table ? 0 : BH * N * 4));
     L.total = o;
     return L;
