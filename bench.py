@@ -223,7 +223,7 @@ def run_gpu(args, wl, world, rank, local):
         sdm.score_topk(d, inp["q"], inp["skr"], wl.R, ridx, rw)
         if ev:
             ev[1].record(stream)
-        sdm.forward_plan(d, inp["alpha"], widx, ridx, st, ws)
+        sdm.forward_plan(d, inp["alpha"], inp["beta"], widx, ww, ridx, rw, st, ws)
         if ev:
             ev[2].record(stream)
         sdm.forward_run(d, inp["v"], inp["beta"], widx, ww, ridx, rw, st, out, ws)

@@ -167,17 +167,19 @@ sdm_status sdm_forward(const sdm_dims* dims, const void* v, const float* alpha, 
 
 /*
  * The two stages of sdm_forward, callable separately (same arguments):
- *   sdm_forward_plan  index-only pass: per-occurrence decay factors from the
- *                     slot stamps, in-chunk links between tokens that share a
- *                     slot, new stamps and Lambda (writes ws, st->stamp,
- *                     st->Lambda).
- *   sdm_forward_run   the row pass: gathers, delta updates, scatters, outputs
- *                     (reads ws, updates st->M, writes out).
- * A run must follow the plan of the same call, on the same stream, with the
- * same index arrays and unchanged ws.
+ *   sdm_forward_plan  pass over indices, weights and gates only (no rows): decay factors
+ *                     of the rows each token gathers (from the slot stamps), links between
+ *                     occurrences of the same slot inside each chunk, and per chunk the
+ *                     C x C matrices that resolve them (a triangular solve, the intra-chunk
+ *                     phase of the pages' Appendix A.1); writes ws, st->stamp and st->Lambda.
+ *   sdm_forward_run   the row pass: gathers, delta updates, stores, outputs (reads ws,
+ *                     updates st->M, writes out).
+ * A run must follow the plan of the same call, on the same stream, with the same index,
+ * weight and gate arrays and unchanged ws.
  */
-sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const int32_t* widx,
-                            const int32_t* ridx, const sdm_state* st, void* ws, size_t ws_bytes,
+sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const float* beta,
+                            const int32_t* widx, const float* ww, const int32_t* ridx,
+                            const float* rw, const sdm_state* st, void* ws, size_t ws_bytes,
                             sdm_stream_t stream);
 sdm_status sdm_forward_run(const sdm_dims* dims, const void* v, const float* beta,
                            const int32_t* widx, const float* ww, const int32_t* ridx,

@@ -76,7 +76,7 @@ def _load():
         "sdm_score_topk": ([D, P, P, I32, P, P, P], I32),
         "sdm_forward_workspace_bytes": ([D], SZ),
         "sdm_forward": ([D, P, P, P, P, P, P, P, S, P, P, SZ, P], I32),
-        "sdm_forward_plan": ([D, P, P, P, S, P, SZ, P], I32),
+        "sdm_forward_plan": ([D, P, P, P, P, P, P, S, P, SZ, P], I32),
         "sdm_forward_run": ([D, P, P, P, P, P, P, S, P, P, SZ, P], I32),
         "sdm_prefill": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P, SZ, P], I32),
         "sdm_decode_step": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P], I32),
@@ -206,11 +206,12 @@ def forward_noalloc(d: Dims, v, alpha, beta, widx, ww, ridx, rw, st: State, out=
     return out
 
 
-def forward_plan(d: Dims, alpha, widx, ridx, st: State, ws, stream=None):
+def forward_plan(d: Dims, alpha, beta, widx, ww, ridx, rw, st: State, ws, stream=None):
     _ok(_lib.sdm_forward_plan(ctypes.byref(d), _ptr(alpha, "alpha", torch.float32),
-                              _ptr(widx, "widx", torch.int32), _ptr(ridx, "ridx", torch.int32),
-                              ctypes.byref(st.c), _ptr(ws, "ws"), ws.numel(), _stream(stream)),
-        "sdm_forward_plan")
+                              _ptr(beta, "beta", torch.float32), _ptr(widx, "widx", torch.int32),
+                              _ptr(ww, "ww", torch.float32), _ptr(ridx, "ridx", torch.int32),
+                              _ptr(rw, "rw", torch.float32), ctypes.byref(st.c), _ptr(ws, "ws"),
+                              ws.numel(), _stream(stream)), "sdm_forward_plan")
 
 
 def forward_run(d: Dims, v, beta, widx, ww, ridx, rw, st: State, out, ws, stream=None):

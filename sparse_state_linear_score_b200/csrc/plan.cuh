@@ -1,25 +1,28 @@
-// Index-only planning pass of the prefill recurrence.
+// Planning pass of the prefill recurrence (indices, weights and gates only; no rows).
 //
-// The recurrence (§2 Background "Gated DeltaNet", §3 Method "Sparse memory updates")
-// is run chunk by chunk: C tokens gather their rows from the memory as it stood at
-// the chunk start, the dependencies between tokens of one chunk that share a slot
-// are resolved on chip, and every slot written in the chunk is stored once at the
-// chunk end.  Everything that depends only on indices and gates is computed here,
-// once per (b,h), and shared by all column blocks of the row pass:
+// The recurrence (§2 Background "Gated DeltaNet", §3 Method "Sparse memory updates") is run
+// chunk by chunk: C tokens gather their rows from the memory as it stood at the chunk start,
+// the dependencies between tokens of one chunk that share a slot are resolved on chip, and
+// every slot written in the chunk is stored once at the chunk end.  Inside a chunk, with the
+// chunk-start rows gathered (decayed to each token: P0, Q0) and d_t = beta_t (v_t - p_t):
+//     p_t = P0_t + sum_{tau<t} L[t][tau] d_tau,   L[t][tau] = e^{lam_t - lam_tau} sum_{s in W_t ^ W_tau} w_t,s w_tau,s
+//     =>  (I + diag(beta) L) d = beta (v - P0),   d = Minv beta (v - P0)
+//     o_t = Q0_t + sum_{tau<=t} G[t][tau] d_tau,  G[t][tau] = e^{lam_t - lam_tau} sum_{s in R_t ^ W_tau} u_t,s w_tau,s
+// (the intra-chunk phase of the pages' Appendix A.1; tokens interact only through shared
+// slots, Appendix A.2).  Minv and G depend on nothing but indices, weights and gates, so they
+// are built here once per (b,h, chunk) and shared by every column block of the row pass.
 //
 //   plan_local (one CTA per chunk)
 //     lam[t]      = sum of log(alpha_u) from the chunk start to t (inclusive), fp32
 //     csum[j]     = the same sum over the whole chunk, fp64
 //     lk[o]       = for occurrence o (a write or read slot of a token in the chunk):
-//                   1 + the in-chunk index of the latest earlier write of that slot
+//                   bits 0..15: 1 + the in-chunk index of the latest earlier write of that slot
 //                   (token < t for a write, token <= t for a read), 0 if none;
 //                   bit 16: o is the last write of its slot in the chunk (stores it);
-//                   bit 17: o's accumulated in-chunk delta must be kept (a later
-//                   occurrence links to it, or it stores and has a link)
-//     tmask[t]    = {write-link bits, read-link bits, keep-delta bits, level}: the bits run
-//                   over the token's W / R slots; level 0 = no in-chunk link, otherwise
-//                   1 + the largest level among the earlier tokens it links to (tokens of
-//                   one level can be resolved together once the lower levels are done)
+//                   bits 18..29: 1 + the index of the previous chunk's write occurrence
+//                   that stored o's slot at that chunk's end (0: not written there) — the
+//                   row pass gathers a chunk ahead and takes such rows from that store
+//     mats[j]     = Minv [C][C], then G [C][C] (fp32, row t = token, zero beyond the chunk)
 //     st0[o]      = the state's stamp of o's slot at call entry (NaN: pristine)
 //   plan_walk (one CTA per (b,h), chunks in order)
 //     Lstart[j]   = log-decay prefix at the start of chunk j (Lstart[0] = state Lambda)
@@ -39,17 +42,25 @@
 namespace sdm {
 
 constexpr int PLAN_MAX_OCC = 2048;  // C*(W+R) never exceeds this
+constexpr int PLAN_MAX_C = 32;      // tokens per chunk
 constexpr int PLAN_HASH = 4096;     // hash buckets (>= 2 * max write occurrences)
 constexpr int PLAN_THREADS = 256;
 constexpr int WALK_THREADS = 1024;
 constexpr int WALK_MAXO = PLAN_MAX_OCC / WALK_THREADS;
 
 constexpr unsigned LK_OWNER = 1u << 16;
-constexpr unsigned LK_KEEP = 1u << 17;
+constexpr int LK_PREV_SHIFT = 18;  // bits 18..29: 1 + previous chunk's owner of the slot
 
 SDM_DEV int lk_link(int lk) { return (lk & 0xffff) - 1; }
+SDM_DEV int lk_prev(int lk) { return ((lk >> LK_PREV_SHIFT) & 0xfff) - 1; }
 
 SDM_DEV unsigned slot_hash(int s) { return ((unsigned)s * 2654435761u) >> (32 - 12); }
+
+// Dynamic shared memory of plan_local (bytes).
+__host__ __device__ inline size_t plan_local_smem_bytes() {
+    return (size_t)3 * PLAN_MAX_C * PLAN_MAX_C * 4 + (size_t)2 * PLAN_MAX_C * 4 +
+           (size_t)PLAN_MAX_OCC * (4 + 4 + 4 + 2 + 2 + 2 + 1) + (size_t)PLAN_HASH * 4 * 2;
+}
 
 // Inclusive block-wide prefix sum of doubles held one per thread (blockDim.x <= 1024).
 SDM_DEV double block_inclusive_scan(double v, double* warp_tot) {
@@ -84,23 +95,31 @@ struct PlanPtrs {
     double* st0;       // [BH][T*(W+R)]
     float* fe;         // [BH][T*(W+R)]
     int32_t* lk;       // [BH][T*(W+R)]
-    uint64_t* tmask;   // [BH][T][4]
+    float* mats;       // [BH][J][2][C][C]
     int32_t* lastw;    // [BH][N] (only when the walk table does not fit in shared memory)
 };
 
 __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
-    const float* __restrict__ alpha, const int32_t* __restrict__ widx,
-    const int32_t* __restrict__ ridx, const double* __restrict__ stamp, int T, int N, int W,
-    int R, int C, int J, PlanPtrs P) {
+    const float* __restrict__ alpha, const float* __restrict__ beta,
+    const int32_t* __restrict__ widx, const float* __restrict__ ww,
+    const int32_t* __restrict__ ridx, const float* __restrict__ rw,
+    const double* __restrict__ stamp, int T, int N, int W, int R, int C, int J, PlanPtrs P) {
     __shared__ double s_wtot[32];
-    __shared__ int s_slot[PLAN_MAX_OCC];
-    __shared__ short s_link[PLAN_MAX_OCC];
-    __shared__ int s_head[PLAN_HASH];  // atomicExch needs 32-bit words
-    __shared__ short s_next[PLAN_MAX_OCC];
-    __shared__ unsigned char s_need[PLAN_MAX_OCC];
-    __shared__ unsigned char s_owner[PLAN_MAX_OCC];
-    __shared__ unsigned long long s_mask[3 * PLAN_THREADS];
-    __shared__ int s_level[PLAN_THREADS];
+    extern __shared__ __align__(16) unsigned char plan_smem[];
+    float* s_L = reinterpret_cast<float*>(plan_smem);         // [32][32] L, then Minv
+    float* s_G = s_L + PLAN_MAX_C * PLAN_MAX_C;               // [32][32]
+    float* s_X = s_G + PLAN_MAX_C * PLAN_MAX_C;               // [32][32] Minv (column solves)
+    float* s_lamc = s_X + PLAN_MAX_C * PLAN_MAX_C;            // [32] chunk-relative prefix
+    float* s_bet = s_lamc + PLAN_MAX_C;                       // [32]
+    int* s_slot = reinterpret_cast<int*>(s_bet + PLAN_MAX_C); // [2048]
+    int* s_slot2 = s_slot + PLAN_MAX_OCC;                     // previous chunk's write slots
+    float* s_wt = reinterpret_cast<float*>(s_slot2 + PLAN_MAX_OCC);  // [2048] weights
+    int* s_head = reinterpret_cast<int*>(s_wt + PLAN_MAX_OCC);       // [4096] (32-bit atomics)
+    int* s_head2 = s_head + PLAN_HASH;                               // [4096]
+    short* s_link = reinterpret_cast<short*>(s_head2 + PLAN_HASH);
+    short* s_next = s_link + PLAN_MAX_OCC;
+    short* s_next2 = s_next + PLAN_MAX_OCC;
+    unsigned char* s_owner = reinterpret_cast<unsigned char*>(s_next2 + PLAN_MAX_OCC);
 
     const int j = blockIdx.x;
     const size_t bh = blockIdx.y;
@@ -119,32 +138,57 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
         } else {
             raise_err(SDM_DEVERR_ALPHA);  // treated as alpha = 1
         }
+        s_bet[tid] = beta[bh * T + t0 + tid];
     }
     const double pre = block_inclusive_scan(la, s_wtot);
-    if (tid < nt) P.lam[bh * T + t0 + tid] = (float)pre;
+    if (tid < nt) {
+        P.lam[bh * T + t0 + tid] = (float)pre;
+        s_lamc[tid] = (float)pre;
+    }
     if (tid == nt - 1) P.csum[bh * J + j] = pre;
 
-    // 2. slots of the chunk, hash heads, masks
+    // 2. slots and weights of the chunk (and the previous chunk's write slots), hash heads
     for (int o = tid; o < no; o += PLAN_THREADS) {
         int s;
-        if (o < nw) s = widx[(bh * T + t0) * W + o];
-        else s = ridx[(bh * T + t0) * R + (o - nw)];
+        float w;
+        if (o < nw) {
+            s = widx[(bh * T + t0) * W + o];
+            w = ww[(bh * T + t0) * W + o];
+        } else {
+            s = ridx[(bh * T + t0) * R + (o - nw)];
+            w = rw[(bh * T + t0) * R + (o - nw)];
+        }
         if (!slot_ok(s, N)) {
             raise_err(SDM_DEVERR_SLOT_RANGE);
             s = -1;
         }
         s_slot[o] = s;
-        s_need[o] = 0;
+        s_wt[o] = w;
         s_owner[o] = 0;
     }
-    for (int i = tid; i < PLAN_HASH; i += PLAN_THREADS) s_head[i] = -1;
-    for (int i = tid; i < 3 * nt; i += PLAN_THREADS) s_mask[i] = 0ull;
+    for (int i = tid; i < PLAN_HASH; i += PLAN_THREADS) {
+        s_head[i] = -1;
+        s_head2[i] = -1;
+    }
+    for (int i = tid; i < PLAN_MAX_C * PLAN_MAX_C; i += PLAN_THREADS) {
+        s_L[i] = 0.f;
+        s_G[i] = 0.f;
+    }
+    const int nwp = j > 0 ? C * W : 0;  // the previous chunk is always full
+    for (int o = tid; o < nwp; o += PLAN_THREADS) {
+        const int sp = widx[(bh * T + (size_t)(j - 1) * C) * W + o];
+        s_slot2[o] = slot_ok(sp, N) ? sp : -1;
+    }
     __syncthreads();
 
-    // 3. insert the write occurrences into per-bucket lists
+    // 3. insert the write occurrences of this and of the previous chunk into bucket lists
     for (int o = tid; o < nw; o += PLAN_THREADS) {
         const int s = s_slot[o];
         if (s >= 0) s_next[o] = (short)atomicExch(&s_head[slot_hash(s)], o);
+    }
+    for (int o = tid; o < nwp; o += PLAN_THREADS) {
+        const int s = s_slot2[o];
+        if (s >= 0) s_next2[o] = (short)atomicExch(&s_head2[slot_hash(s)], o);
     }
     __syncthreads();
 
@@ -173,72 +217,84 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
                 }
             }
             if (is_w && !later) s_owner[o] = 1;
-            if (link >= 0) s_need[link] = 1;
         }
         s_link[o] = (short)link;
     }
     __syncthreads();
 
-    // 5. per-token masks
-    for (int o = tid; o < no; o += PLAN_THREADS) {
-        const int link = s_link[o];
-        if (o < nw) {
-            const int tl = o / W, i = o % W;
-            if (link >= 0) atomicOr(&s_mask[3 * tl + 0], 1ull << i);
-            if (s_need[o] || (s_owner[o] && link >= 0)) atomicOr(&s_mask[3 * tl + 2], 1ull << i);
-        } else if (link >= 0) {
-            const int tl = (o - nw) / R, jj = (o - nw) % R;
-            atomicOr(&s_mask[3 * tl + 1], 1ull << jj);
-        }
-    }
-    __syncthreads();
-
-    // 5b. levels: longest chain of in-chunk links ending at each token
-    for (int t = tid; t < nt; t += PLAN_THREADS)
-        s_level[t] = (s_mask[3 * t] | s_mask[3 * t + 1]) ? 1 : 0;
-    __syncthreads();
-    for (int it = 0; it < nt; ++it) {
-        int changed = 0;
-        for (int o = tid; o < no; o += PLAN_THREADS) {
-            const int link = s_link[o];
-            if (link < 0) continue;
-            const int tl = o < nw ? o / W : (o - nw) / R;
-            const int tp = link / W;
-            if (tp < tl) {
-                const int want = s_level[tp] + 1;
-                if (s_level[tp] > 0 && want > s_level[tl]) {
-                    atomicMax(&s_level[tl], want);
-                    changed = 1;
-                }
+    // 5. L and G rows: token t walks the link chain of each of its occurrences (every
+    //    earlier write of the slot in the chunk), in a fixed order (deterministic sums)
+    if (tid < nt) {
+        const int t = tid;
+        const float lt = s_lamc[t];
+        for (int i = 0; i < W; ++i) {
+            const int o = t * W + i;
+            const float wo = s_wt[o];
+            for (int L = s_link[o]; L >= 0; L = s_link[L]) {
+                const int tp = L / W;
+                s_L[t * PLAN_MAX_C + tp] += wo * s_wt[L] * expf(lt - s_lamc[tp]);
             }
         }
-        if (!__syncthreads_or(changed)) break;
+        for (int i = 0; i < R; ++i) {
+            const int o = nw + t * R + i;
+            const float uo = s_wt[o];
+            for (int L = s_link[o]; L >= 0; L = s_link[L]) {
+                const int tp = L / W;
+                s_G[t * PLAN_MAX_C + tp] += uo * s_wt[L] * expf(lt - s_lamc[tp]);
+            }
+        }
+    }
+    __syncthreads();
+    // 6. Minv = (I + diag(beta) L)^-1, one column per thread by forward substitution
+    if (tid < nt) {
+        const int k = tid;
+        for (int t = 0; t < nt; ++t) {
+            float x;
+            if (t < k) {
+                x = 0.f;
+            } else if (t == k) {
+                x = 1.f;
+            } else {
+                float acc = 0.f;
+                for (int tau = k; tau < t; ++tau)
+                    acc = fmaf(s_L[t * PLAN_MAX_C + tau], s_X[tau * PLAN_MAX_C + k], acc);
+                x = -s_bet[t] * acc;
+            }
+            s_X[t * PLAN_MAX_C + k] = x;
+        }
+    }
+    __syncthreads();
+    {
+        float* mats = P.mats + ((bh * J + j) * 2) * (size_t)(C * C);
+        for (int e = tid; e < C * C; e += PLAN_THREADS) {
+            const int t = e / C, tau = e % C;
+            const bool in = t < nt && tau < nt;
+            mats[e] = in ? s_X[t * PLAN_MAX_C + tau] : 0.f;
+            mats[C * C + e] = in ? s_G[t * PLAN_MAX_C + tau] : 0.f;
+        }
     }
 
-    // 6. write out
+    // 7. link words and entry stamps
     for (int o = tid; o < no; o += PLAN_THREADS) {
         const int link = s_link[o];
         unsigned v = (unsigned)(link + 1);
         size_t g;
         if (o < nw) {
-            const int tl = o / W;
             if (s_owner[o]) v |= LK_OWNER;
-            if (s_need[o] || (s_owner[o] && link >= 0)) v |= LK_KEEP;
             g = occ_base + (size_t)t0 * W + o;
-            (void)tl;
         } else {
             g = occ_base + (size_t)T * W + (size_t)t0 * R + (o - nw);
         }
+        // the previous chunk's last write of this slot (its store at that chunk's end)
+        const int sl = s_slot[o];
+        if (sl >= 0 && nwp > 0) {
+            int best = -1;
+            for (int p = s_head2[slot_hash(sl)]; p >= 0; p = s_next2[p])
+                if (s_slot2[p] == sl && p > best) best = p;  // larger index = later token
+            v |= (unsigned)(best + 1) << LK_PREV_SHIFT;
+        }
         P.lk[g] = (int32_t)v;
-        const int s = s_slot[o];
-        P.st0[g] = s >= 0 ? stamp[bh * (size_t)N + s] : 0.0;
-    }
-    for (int t = tid; t < nt; t += PLAN_THREADS) {
-        uint64_t* tm = P.tmask + (bh * T + t0 + t) * 4;
-        tm[0] = s_mask[3 * t];
-        tm[1] = s_mask[3 * t + 1];
-        tm[2] = s_mask[3 * t + 2];
-        tm[3] = (uint64_t)s_level[t];
+        P.st0[g] = sl >= 0 ? stamp[bh * (size_t)N + sl] : 0.0;
     }
 }
 

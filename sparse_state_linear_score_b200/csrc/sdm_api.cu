@@ -19,7 +19,7 @@ using namespace sdm;
 namespace {
 
 constexpr int kMaxTop = 64;
-constexpr size_t kSmemBudget = 200 * 1024;  // dynamic shared memory per CTA we plan for
+constexpr size_t kSmemBudget = 220 * 1024;  // dynamic shared memory per CTA we plan for
 constexpr int kWalkSmemSlots = 65536;        // walk table in shared memory up to this N
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
@@ -48,16 +48,18 @@ inline int col_width(const sdm_dims* d) { return d->d_v % 8 == 0 ? 8 : 4; }
 int chunk_tokens(const sdm_dims* d) {
     const int CW = col_width(d);
     int C = PLAN_MAX_OCC / (d->W + d->R);
-    if (C > PLAN_THREADS) C = PLAN_THREADS;
-    while (C > 1 && run_smem_bytes(C, d->W, d->R, CW) > kSmemBudget) --C;
-    return C < 1 ? 1 : C;
+    if (C > PLAN_MAX_C) C = PLAN_MAX_C;
+    if (C > RUN_THREADS / CW) C = RUN_THREADS / CW;  // one value per thread in the prefetch
+    C &= ~3;  // matrices move in 16-byte rows
+    while (C > 4 && run_smem_bytes(C, d->W, d->R, CW) > kSmemBudget) C -= 4;
+    return C < 4 ? 4 : C;
 }
 
 struct WsLayout {
     int C, J;
     bool smem_table, lstart_smem;
     size_t walk_smem;
-    size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_tmask, off_lastw, total;
+    size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_mats, off_lastw, total;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -79,7 +81,7 @@ WsLayout ws_layout(const sdm_dims* d) {
     L.off_st0 = o;    o = up256(o + BH * occ * 8);
     L.off_fe = o;     o = up256(o + BH * occ * 4);
     L.off_lk = o;     o = up256(o + BH * occ * 4);
-    L.off_tmask = o;  o = up256(o + BH * T * 4 * 8);
+    L.off_mats = o;   o = up256(o + BH * (size_t)L.J * 2 * L.C * L.C * 4);
     L.off_lastw = o;  o = up256(o + (L.smem_table ? 0 : BH * N * 4));
     L.total = o;
     return L;
@@ -94,7 +96,7 @@ PlanPtrs plan_ptrs(const WsLayout& L, void* ws) {
     P.st0 = reinterpret_cast<double*>(b + L.off_st0);
     P.fe = reinterpret_cast<float*>(b + L.off_fe);
     P.lk = reinterpret_cast<int32_t*>(b + L.off_lk);
-    P.tmask = reinterpret_cast<uint64_t*>(b + L.off_tmask);
+    P.mats = reinterpret_cast<float*>(b + L.off_mats);
     P.lastw = reinterpret_cast<int32_t*>(b + L.off_lastw);
     return P;
 }
@@ -236,8 +238,8 @@ sdm_status launch_run_t(const sdm_dims* d, const WsLayout& L, const PlanPtrs& P,
     if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
     const long long grid = BH_of(d) * (d->d_v / CW);
     kern<<<(unsigned)grid, RUN_THREADS, smem, s>>>(
-        (const VT*)v, beta, widx, ww, ridx, rw, P.fe, P.lk, P.lam,
-        reinterpret_cast<const unsigned long long*>(P.tmask), st->M, st->M0, out, d->H, d->T,
+        (const VT*)v, beta, widx, ww, ridx, rw, P.fe, P.lk, P.lam, P.mats, st->M, st->M0, out,
+        d->H, d->T,
         (int)N_of(d), d->d_v, d->W, d->R, L.C, L.J);
     return launch_status();
 }
@@ -293,7 +295,7 @@ const char* sdm_status_str(int32_t status) {
     }
 }
 
-int32_t sdm_abi_version(void) { return 1; }
+int32_t sdm_abi_version(void) { return 2; }
 
 sdm_status sdm_state_bytes(const sdm_dims* dims, size_t* M_bytes, size_t* stamp_bytes,
                            size_t* lambda_bytes) {
@@ -354,15 +356,18 @@ size_t sdm_forward_workspace_bytes(const sdm_dims* dims) {
     return ws_layout(dims).total;
 }
 
-sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const int32_t* widx,
-                            const int32_t* ridx, const sdm_state* st, void* ws, size_t ws_bytes,
+sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const float* beta,
+                            const int32_t* widx, const float* ww, const int32_t* ridx,
+                            const float* rw, const sdm_state* st, void* ws, size_t ws_bytes,
                             sdm_stream_t stream) {
     sdm_status e = check_dims(dims);
     if (e) return e;
     if ((e = check_state(st))) return e;
     if (dims->T == 0) return SDM_OK;
-    if (!alpha || !widx || !ridx) return SDM_ERR_ARG;
-    if (!aligned16(alpha) || !aligned16(widx) || !aligned16(ridx)) return SDM_ERR_ALIGN;
+    if (!alpha || !beta || !widx || !ww || !ridx || !rw) return SDM_ERR_ARG;
+    if (!aligned16(alpha) || !aligned16(beta) || !aligned16(widx) || !aligned16(ww) ||
+        !aligned16(ridx) || !aligned16(rw))
+        return SDM_ERR_ALIGN;
     const WsLayout L = ws_layout(dims);
     if (!ws || ws_bytes < L.total) return SDM_ERR_WORKSPACE;
     if (!aligned16(ws)) return SDM_ERR_ALIGN;
@@ -372,8 +377,10 @@ sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const int3
     if (!L.smem_table &&
         cudaMemsetAsync(P.lastw, 0xff, BH * (size_t)N * 4, stream) != cudaSuccess)
         return SDM_ERR_CUDA;
-    plan_local_kernel<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, 0, stream>>>(
-        alpha, widx, ridx, st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, P);
+    if (!set_smem(plan_local_kernel, plan_local_smem_bytes())) return SDM_ERR_CUDA;
+    plan_local_kernel<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, plan_local_smem_bytes(),
+                        stream>>>(
+        alpha, beta, widx, ww, ridx, rw, st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, P);
     if ((e = launch_status())) return e;
     if (L.smem_table) {
         if (!set_smem(plan_walk_kernel<true>, L.walk_smem)) return SDM_ERR_CUDA;
@@ -427,7 +434,8 @@ sdm_status sdm_forward(const sdm_dims* dims, const void* v, const float* alpha, 
     if (!v || !alpha || !beta || !widx || !ww || !ridx || !rw || !out) return SDM_ERR_ARG;
     const WsLayout L = ws_layout(dims);
     if (!ws || ws_bytes < L.total) return SDM_ERR_WORKSPACE;
-    if ((e = sdm_forward_plan(dims, alpha, widx, ridx, st, ws, ws_bytes, stream))) return e;
+    if ((e = sdm_forward_plan(dims, alpha, beta, widx, ww, ridx, rw, st, ws, ws_bytes, stream)))
+        return e;
     return sdm_forward_run(dims, v, beta, widx, ww, ridx, rw, st, out, ws, ws_bytes, stream);
 }
 
