@@ -33,6 +33,19 @@ __host__ __device__ inline int run_tok_stride(int per_tok, int CW) { return per_
 // Row stride of Minv / G in shared memory (16-byte rows, 4 floats apart in banks).
 __host__ __device__ inline int run_mat_stride(int C) { return C + 4; }
 
+// x / d for 0 <= x < 2^16 and 1 <= d <= 64 as one multiply-high: with m = ceil(2^32 / d),
+// m*d - 2^32 < d, so the rounding error x*(m*d - 2^32) < 2^22 never reaches 2^32.
+struct FastDiv {
+    unsigned m, d;
+    __host__ __device__ explicit FastDiv(unsigned dd) : m((unsigned)((0x100000000ull + dd - 1) / dd)), d(dd) {}
+    SDM_DEV int div(int x) const { return (int)__umulhi((unsigned)x, m); }
+    SDM_DEV int mod(int x) const { return x - div(x) * (int)d; }
+};
+
+// Row stride of a token's coefficients in shared memory: W + 1 (or R + 1) keeps the four
+// tokens a warp reads at once in different banks.
+__host__ __device__ inline int run_coef_stride(int per_tok) { return per_tok + 1; }
+
 __host__ __device__ inline size_t run_smem_bytes(int C, int W, int R, int CW) {
     const size_t tsw = (size_t)run_tok_stride(W, CW), tsr = (size_t)run_tok_stride(R, CW);
     const size_t no = (size_t)C * (W + R);
@@ -41,11 +54,14 @@ __host__ __device__ inline size_t run_smem_bytes(int C, int W, int R, int CW) {
     b += (size_t)2 * 2 * C * run_mat_stride(C) * 4; // Minv and G, two chunks
     b += (size_t)4 * C * CW * 4;                    // v, rhs, d, Q0
     b += (size_t)2 * C * 4;                         // lam, beta
-    b += no * 4 * 5;                                // slot, coef, w, fe, lk
+    b += no * 4 * 4;                                // slot, w, fe, lk
+    b += (size_t)C * (run_coef_stride(W) + run_coef_stride(R)) * 4;  // coef (padded rows)
     return b;
 }
 
 constexpr int RUN_OPT = PLAN_MAX_OCC / RUN_THREADS;  // occurrences per thread per chunk
+
+
 
 // One chunk's metadata held in registers while the previous chunk computes.
 struct RunPrefetch {
@@ -87,15 +103,23 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
     float* s_lam = s_q + C * CW;
     float* s_beta = s_lam + C;
     int* s_slot = reinterpret_cast<int*>(s_beta + C);
-    float* s_coef = reinterpret_cast<float*>(s_slot + nomax);
-    float* s_w = s_coef + nomax;
+    const int csw = run_coef_stride(W), csr = run_coef_stride(R);
+    float* s_coef = reinterpret_cast<float*>(s_slot + nomax);  // [C][W+1], then [C][R+1]
+    float* s_w = s_coef + C * (csw + csr);
     float* s_fe = s_w + nomax;
     int* s_lk = reinterpret_cast<int*>(s_fe + nomax);
 
+    const FastDiv fW((unsigned)W), fR((unsigned)R);
     // position of a write occurrence's slice, and of a read occurrence's slice
-    auto wpos = [&](int o) { return (o / W) * tsw + (o % W) * CW; };
-    auto rpos = [&](int o) { return C * tsw + (o / R) * tsr + (o % R) * CW; };
+    auto wpos = [&](int o) { const int t = fW.div(o); return t * tsw + (o - t * W) * CW; };
+    auto rpos = [&](int o) { const int t = fR.div(o); return C * tsw + t * tsr + (o - t * R) * CW; };
     auto pos = [&](int o, int nw) { return o < nw ? wpos(o) : rpos(o - nw); };
+    // padded coefficient index of occurrence o
+    auto cpos = [&](int o, int nw) {
+        if (o < nw) { const int t = fW.div(o); return t * csw + (o - t * W); }
+        const int r = o - nw, t = fR.div(r);
+        return C * csw + t * csr + (r - t * R);
+    };
 
     // registers <- metadata of chunk jn
     auto fetch = [&](int jn, RunPrefetch& F) {
@@ -130,7 +154,7 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
     };
     // shared <- registers (chunk jn's metadata)
     auto publish = [&](int jn, const RunPrefetch& F) {
-        const int t0 = jn * C, nt = min(C, T - t0), no = nt * (W + R);
+        const int t0 = jn * C, nt = min(C, T - t0), nw = nt * W, no = nt * (W + R);
 #pragma unroll
         for (int k = 0; k < RUN_OPT; ++k) {
             const int o = tid + k * RUN_THREADS;
@@ -138,7 +162,7 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
                 s_slot[o] = F.slot[k];
                 s_w[o] = F.w[k];
                 s_fe[o] = F.fe[k];
-                s_coef[o] = F.w[k] * fabsf(F.fe[k]);
+                s_coef[cpos(o, nw)] = F.w[k] * fabsf(F.fe[k]);
                 s_lk[o] = F.lk[k];
             }
         }
@@ -149,19 +173,29 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
         if (tid < nt * CW) s_v[tid] = F.v;
     };
     // chunk jn's row gathers (rows as stored now; the ones its previous chunk is about to
-    // store are replaced later from that chunk's stores) and its Minv / G
+    // store are replaced later from that chunk's stores) and its Minv / G.  The Q 16-byte
+    // pieces of one occurrence's slice are fetched by Q adjacent lanes in one instruction,
+    // so each slice is a single request to the memory system.
     auto gather = [&](int jn, const RunPrefetch& F, float* rbuf, float* mbuf) {
         const int t0 = jn * C, nt = min(C, T - t0), nw = nt * W, no = nt * (W + R);
+        const int lane = tid & 31, wbase = tid - lane;
+        constexpr int PER = 32 / Q;  // occurrences per instruction
 #pragma unroll
         for (int k = 0; k < RUN_OPT; ++k) {
-            const int o = tid + k * RUN_THREADS;
-            if (o >= no) continue;
-            const int s = F.slot[k];
-            const bool ok = slot_ok(s, N);
-            const float* src = (signbit(F.fe[k]) ? M0h : Mb) + (ok ? (size_t)s * d_v : 0) + c0;
-            float* dst = rbuf + pos(o, nw);
 #pragma unroll
-            for (int q = 0; q < Q; ++q) cp_async16(dst + 4 * q, src + 4 * q, ok);
+            for (int r = 0; r < Q; ++r) {
+                const int src_lane = r * PER + lane / Q;
+                const int s = __shfl_sync(0xffffffffu, F.slot[k], src_lane);
+                const float f = __shfl_sync(0xffffffffu, F.fe[k], src_lane);
+                const int o = wbase + k * RUN_THREADS + src_lane;
+                const int q = lane % Q;
+                if (o < no) {
+                    const bool ok = slot_ok(s, N);
+                    const float* src =
+                        (signbit(f) ? M0h : Mb) + (ok ? (size_t)s * d_v : 0) + c0 + 4 * q;
+                    cp_async16(rbuf + pos(o, nw) + 4 * q, src, ok);
+                }
+            }
         }
         const float* msrc = mats + ((bh * J + jn) * 2) * (size_t)(C * C);
         for (int e = tid; e < 2 * C * (C / 4); e += RUN_THREADS) {  // 16-byte pieces
@@ -197,8 +231,8 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
                 reinterpret_cast<float4*>(rows + pos(o, nw))[q] =
                     reinterpret_cast<const float4*>(prev_rows + wpos(pv))[q];
             }
-            __syncthreads();
         }
+        __syncthreads();
         // 2. the next chunk's gathers and matrices (overlap with this chunk's compute)
         if (j + 1 < J)
             gather(j + 1, F1, prev_rows, s_matbuf + (size_t)((j + 1) & 1) * matbuf);
@@ -211,7 +245,7 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
             const int t = e / CW, c = e % CW;
             // four independent partial sums per dot product (latency of the smem loads)
             const float* rr = rd ? rows + C * tsw + t * tsr + c : rows + t * tsw + c;
-            const float* cf = rd ? s_coef + nw + t * R : s_coef + t * W;
+            const float* cf = rd ? s_coef + C * csw + t * csr : s_coef + t * csw;
             const int n_i = rd ? R : W;
             float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
             int i = 0;
@@ -262,12 +296,12 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
             const int lko = s_lk[o];
             const int s = s_slot[o];
             if (!(lko & LK_OWNER) || !slot_ok(s, N)) continue;
-            const int t = o / W;
+            const int t = fW.div(o);
             const float lt = s_lam[t];
             // A: this write plus the chunk's earlier writes of the slot, decayed to t
             float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int L = o; L >= 0; L = lk_link(s_lk[L])) {
-                const int tp = L / W;
+                const int tp = fW.div(L);
                 const float cfa = s_w[L] * expf(lt - s_lam[tp]);
                 const float4 dd = reinterpret_cast<const float4*>(s_d + tp * CW)[q];
                 a.x = fmaf(cfa, dd.x, a.x);
