@@ -24,11 +24,18 @@
 //                   row pass gathers a chunk ahead and takes such rows from that store
 //     mats[j]     = Minv [C][C], then G [C][C] (fp32, row t = token, zero beyond the chunk)
 //     st0[o]      = the state's stamp of o's slot at call entry (NaN: pristine)
-//   plan_walk (one CTA per (b,h), chunks in order)
-//     Lstart[j]   = log-decay prefix at the start of chunk j (Lstart[0] = state Lambda)
-//     fe[o]       = exp(Lambda_t - stamp of the row o gathers); sign bit set when the
-//                   row is the pristine M0 row
-//     state stamps of the slots written in the call and the state Lambda are updated.
+//     occw[o]     = o's slot | OCC_OWNER when o stores it
+//   plan_prefix (one CTA per (b,h))
+//     Lstart[j]   = log-decay prefix at the start of chunk j (Lstart[0] = state Lambda);
+//                   the state Lambda becomes Lstart[J]
+//   plan_fe0 (one CTA per chunk)
+//     fe[o]       = exp(Lambda_t - stamp of the row o gathers) assuming the slot was not
+//                   written earlier in this call; sign bit set when the row is the pristine
+//                   M0 row
+//   plan_walk (one CTA per (b,h), chunks in order, packed words streamed through a ring)
+//     fe[o] is rewritten for slots written by an earlier chunk of this call (the row then
+//     carries the stamp of that chunk's end); the state stamps of the slots written in the
+//     call are updated.
 //
 // In-chunk occurrence order: the nt*W write occurrences (token-major), then the nt*R
 // read occurrences.  In the per-(b,h) arrays fe / lk / st0 the T*W write entries come
@@ -45,8 +52,11 @@ constexpr int PLAN_MAX_OCC = 2048;  // C*(W+R) never exceeds this
 constexpr int PLAN_MAX_C = 32;      // tokens per chunk
 constexpr int PLAN_HASH = 4096;     // hash buckets (>= 2 * max write occurrences)
 constexpr int PLAN_THREADS = 256;
-constexpr int WALK_THREADS = 1024;
+constexpr int WALK_THREADS = 512;
 constexpr int WALK_MAXO = PLAN_MAX_OCC / WALK_THREADS;
+constexpr int WALK_RING = 8;  // chunks of packed occurrence words prefetched by the walk
+constexpr uint32_t OCC_OWNER = 0x80000000u;
+constexpr uint32_t OCC_SLOT = 0x7fffffffu;  // slot, or OCC_SLOT when out of range
 
 constexpr unsigned LK_OWNER = 1u << 16;
 constexpr int LK_PREV_SHIFT = 18;  // bits 18..29: 1 + previous chunk's owner of the slot
@@ -96,7 +106,9 @@ struct PlanPtrs {
     float* fe;         // [BH][T*(W+R)]
     int32_t* lk;       // [BH][T*(W+R)]
     float* mats;       // [BH][J][2][C][C]
-    int32_t* lastw;    // [BH][N] (only when the walk table does not fit in shared memory)
+    uint32_t* occw;    // [BH][T*(W+R)] slot | OCC_OWNER (the walk's input)
+    unsigned long long* mask;  // [BH][N][MW] chunks of this call that stored each slot, or null
+    int MW;                    // 64-bit words per slot in mask
 };
 
 __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
@@ -245,23 +257,27 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
         }
     }
     __syncthreads();
-    // 6. Minv = (I + diag(beta) L)^-1, one column per thread by forward substitution
-    if (tid < nt) {
+    // 6. Minv = (I + diag(beta) L)^-1, one column per thread by forward substitution with the
+    //    column in registers (L is zero outside the chunk, so the full 32 x 32 form is exact)
+    if (tid < PLAN_MAX_C) {
         const int k = tid;
-        for (int t = 0; t < nt; ++t) {
-            float x;
-            if (t < k) {
-                x = 0.f;
-            } else if (t == k) {
-                x = 1.f;
-            } else {
-                float acc = 0.f;
-                for (int tau = k; tau < t; ++tau)
-                    acc = fmaf(s_L[t * PLAN_MAX_C + tau], s_X[tau * PLAN_MAX_C + k], acc);
-                x = -s_bet[t] * acc;
+        float x[PLAN_MAX_C];
+#pragma unroll
+        for (int t = 0; t < PLAN_MAX_C; ++t) {
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+            for (int tau = 0; tau < t; ++tau) {
+                const float l = s_L[t * PLAN_MAX_C + tau];
+                if ((tau & 3) == 0) a0 = fmaf(l, x[tau], a0);
+                else if ((tau & 3) == 1) a1 = fmaf(l, x[tau], a1);
+                else if ((tau & 3) == 2) a2 = fmaf(l, x[tau], a2);
+                else a3 = fmaf(l, x[tau], a3);
             }
-            s_X[t * PLAN_MAX_C + k] = x;
+            const float bt = t < nt ? s_bet[t] : 0.f;
+            x[t] = (t == k) ? 1.f : (t < k ? 0.f : -bt * ((a0 + a1) + (a2 + a3)));
         }
+#pragma unroll
+        for (int t = 0; t < PLAN_MAX_C; ++t) s_X[t * PLAN_MAX_C + k] = x[t];
     }
     __syncthreads();
     {
@@ -295,138 +311,185 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
         }
         P.lk[g] = (int32_t)v;
         P.st0[g] = sl >= 0 ? stamp[bh * (size_t)N + sl] : 0.0;
+        P.occw[g] = (sl >= 0 ? (uint32_t)sl : OCC_SLOT) | (o < nw && s_owner[o] ? OCC_OWNER : 0u);
+        if (P.mask && o < nw && s_owner[o] && sl >= 0)  // this chunk stores the slot
+            atomicOr(P.mask + (bh * (size_t)N + sl) * P.MW + (j >> 6), 1ull << (j & 63));
     }
 }
 
-// Sequential walk over the chunks of one (b,h).  Table: last chunk of this call that
-// wrote each slot (-1: none), in shared memory (int16) when N <= walk_smem_slots, else
-// in the global workspace (int32, set to -1 by the host before the launch).
-template <bool SMEM_TABLE>
-__global__ void __launch_bounds__(WALK_THREADS) plan_walk_kernel(
-    const int32_t* __restrict__ widx, const int32_t* __restrict__ ridx, double* __restrict__ stamp,
-    double* __restrict__ lambda, int T, int N, int W, int R, int C, int J, int lstart_smem,
-    PlanPtrs P) {
-    extern __shared__ __align__(16) unsigned char walk_smem[];
+// Chunk-start log-decay prefixes of one (b,h): Lstart[0] = Lambda, Lstart[j+1] = Lstart[j] +
+// csum[j]; the state Lambda advances to Lstart[J].
+__global__ void __launch_bounds__(1024) plan_prefix_kernel(double* __restrict__ lambda, int J,
+                                                           PlanPtrs P) {
     __shared__ double s_wtot[32];
     const size_t bh = blockIdx.x;
     const int tid = threadIdx.x;
-    double* s_L = reinterpret_cast<double*>(walk_smem);  // [J+1] when lstart_smem
-    short* s_tab = reinterpret_cast<short*>(walk_smem + (lstart_smem ? (size_t)(J + 1) * 8 : 0));
-    int32_t* g_tab = P.lastw + bh * (size_t)N;
     double* Lg = P.Lstart + bh * (size_t)(J + 1);
+    const double L0 = lambda[bh];
+    const int per = (J + 1023) / 1024;
+    const int a = tid * per, b = min(J, a + per);
+    double part = 0.0;
+    for (int i = a; i < b; ++i) part += P.csum[bh * J + i];
+    const double incl = block_inclusive_scan(part, s_wtot);
+    double run = L0 + (incl - part);
+    if (tid == 0) Lg[0] = L0;
+    for (int i = a; i < b; ++i) {
+        run += P.csum[bh * J + i];
+        Lg[i + 1] = run;
+    }
+    __syncthreads();
+    if (tid == 0) lambda[bh] = Lg[J];
+}
+
+// Decay factors of every occurrence.  Without a mask: as if its slot had not been written
+// earlier in this call (the walk corrects the others).  With the per-slot chunk masks: the
+// last earlier chunk that stored the slot is the highest set bit below this chunk, so every
+// factor is final here, and the owner in the slot's last chunk writes the slot's new stamp.
+__global__ void __launch_bounds__(PLAN_THREADS) plan_fe_kernel(double* __restrict__ stamp, int T,
+                                                               int N, int W, int R, int C, int J,
+                                                               PlanPtrs P) {
+    const int j = blockIdx.x;
+    const size_t bh = blockIdx.y;
+    const int t0 = j * C, nt = min(C, T - t0), nw = nt * W, no = nt * (W + R);
+    const size_t occ_base = bh * (size_t)T * (W + R);
+    const double* Lb = P.Lstart + bh * (size_t)(J + 1);
+    const double Lj = Lb[j];
+    for (int o = threadIdx.x; o < no; o += PLAN_THREADS) {
+        size_t g;
+        int t;
+        if (o < nw) {
+            g = occ_base + (size_t)t0 * W + o;
+            t = o / W;
+        } else {
+            g = occ_base + (size_t)T * W + (size_t)t0 * R + (o - nw);
+            t = (o - nw) / R;
+        }
+        const uint32_t w = P.occw[g];
+        const int s = (int)(w & OCC_SLOT);
+        if (s >= N) {
+            P.fe[g] = 0.f;
+            continue;
+        }
+        const double Lt = Lj + (double)P.lam[bh * T + t0 + t];
+        int jw = -1;
+        if (P.mask) {
+            const unsigned long long* m = P.mask + (bh * (size_t)N + s) * P.MW;
+            for (int wi = j >> 6; wi >= 0 && jw < 0; --wi) {
+                unsigned long long bits = m[wi];
+                if (wi == (j >> 6)) bits &= (j & 63) ? ((1ull << (j & 63)) - 1) : 0ull;
+                if (bits) jw = wi * 64 + 63 - __clzll((long long)bits);
+            }
+            if (w & OCC_OWNER) {  // the slot's last storing chunk sets its stamp
+                int jl = -1;
+                for (int wi = P.MW - 1; wi >= 0 && jl < 0; --wi) {
+                    const unsigned long long bits = m[wi];
+                    if (bits) jl = wi * 64 + 63 - __clzll((long long)bits);
+                }
+                if (jl == j) stamp[bh * (size_t)N + s] = Lb[j + 1];
+            }
+        }
+        if (jw >= 0) {
+            P.fe[g] = expf((float)(Lj - Lb[jw + 1]) + P.lam[bh * T + t0 + t]);
+        } else {
+            const double st = P.st0[g];
+            P.fe[g] = isnan(st) ? -(float)exp(Lt) : (float)exp(Lt - st);
+        }
+    }
+}
+
+// Sequential walk over the chunks of one (b,h), split over WALK_PARTS CTAs by slot
+// (slot % WALK_PARTS): each CTA keeps, for its slots only, the last chunk of this call that
+// wrote them (-1: none) in shared memory, and streams the chunks' packed occurrence words
+// and token prefixes through a ring filled WALK_RING chunks ahead by cp.async.
+constexpr int WALK_PARTS = 16;
+
+__global__ void __launch_bounds__(WALK_THREADS) plan_walk_kernel(
+    double* __restrict__ stamp, int T, int N, int W, int R, int C, int J, int lstart_smem,
+    PlanPtrs P) {
+    extern __shared__ __align__(16) unsigned char walk_smem[];
+    const int part = blockIdx.x;
+    const size_t bh = blockIdx.y;
+    const int tid = threadIdx.x;
+    const int stage = PLAN_MAX_OCC + PLAN_MAX_C;  // words per ring stage
+    const int nslot = (N + WALK_PARTS - 1) / WALK_PARTS;
+    uint32_t* s_ring = reinterpret_cast<uint32_t*>(walk_smem);  // [WALK_RING][stage]
+    double* s_L = reinterpret_cast<double*>(s_ring + WALK_RING * stage);  // [J+1] if lstart_smem
+    short* s_tab = reinterpret_cast<short*>(s_L + (lstart_smem ? J + 1 : 0));  // [nslot]
+    const double* Lg = P.Lstart + bh * (size_t)(J + 1);
     const size_t occ_base = bh * (size_t)T * (W + R);
 
-    // 1. chunk-start prefixes: Lstart[0] = Lambda, Lstart[j+1] = Lstart[j] + csum[j]
-    {
-        const int per = (J + WALK_THREADS - 1) / WALK_THREADS;
-        const int a = tid * per, b = min(J, a + per);
-        double part = 0.0;
-        for (int i = a; i < b; ++i) part += P.csum[bh * J + i];
-        const double incl = block_inclusive_scan(part, s_wtot);
-        double run = lambda[bh] + (incl - part);
-        if (tid == 0) {
-            Lg[0] = lambda[bh];
-            if (lstart_smem) s_L[0] = lambda[bh];
-        }
-        for (int i = a; i < b; ++i) {
-            run += P.csum[bh * J + i];
-            Lg[i + 1] = run;
-            if (lstart_smem) s_L[i + 1] = run;
-        }
-    }
-    if (SMEM_TABLE)
-        for (int i = tid; i < N; i += WALK_THREADS) s_tab[i] = -1;
-    __syncthreads();
+    if (lstart_smem)
+        for (int i = tid; i <= J; i += WALK_THREADS) s_L[i] = Lg[i];
+    for (int i = tid; i < nslot; i += WALK_THREADS) s_tab[i] = -1;
     const double* Lr = lstart_smem ? s_L : Lg;
 
-    // 2. chunks in order; each thread owns occurrences tid and tid + WALK_THREADS
-    int cs[WALK_MAXO], ck[WALK_MAXO];
-    double cst[WALK_MAXO];
-    float clam[WALK_MAXO];
-    size_t cg[WALK_MAXO];
-    auto fetch = [&](int j, int* s_, int* k_, double* st_, float* lm_, size_t* g_) {
-        const int t0 = j * C, nt = min(C, T - t0), nw = nt * W, no = nt * (W + R);
-#pragma unroll
-        for (int m = 0; m < WALK_MAXO; ++m) {
-            const int o = tid + m * WALK_THREADS;
-            s_[m] = -1;
-            if (o < no) {
-                size_t g;
-                int t;
-                if (o < nw) {
-                    g = occ_base + (size_t)t0 * W + o;
-                    s_[m] = widx[(bh * T + t0) * W + o];
-                    t = t0 + o / W;
-                } else {
-                    g = occ_base + (size_t)T * W + (size_t)t0 * R + (o - nw);
-                    s_[m] = ridx[(bh * T + t0) * R + (o - nw)];
-                    t = t0 + (o - nw) / R;
-                }
-                k_[m] = P.lk[g];
-                st_[m] = P.st0[g];
-                lm_[m] = P.lam[bh * T + t];
-                g_[m] = g;
+    auto load_stage = [&](int jn) {
+        if (jn < J) {
+            uint32_t* dst = s_ring + (jn % WALK_RING) * stage;
+            const int t0 = jn * C, nt = min(C, T - t0), nw = nt * W, no = nt * (W + R);
+            for (int o = tid; o < no; o += WALK_THREADS) {
+                const size_t g = o < nw ? occ_base + (size_t)t0 * W + o
+                                        : occ_base + (size_t)T * W + (size_t)t0 * R + (o - nw);
+                const unsigned d = (unsigned)__cvta_generic_to_shared(dst + o);
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(d), "l"(P.occw + g)
+                             : "memory");
+            }
+            for (int t = tid; t < nt; t += WALK_THREADS) {
+                const unsigned d = (unsigned)__cvta_generic_to_shared(dst + PLAN_MAX_OCC + t);
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(d),
+                             "l"(P.lam + bh * T + t0 + t)
+                             : "memory");
             }
         }
+        cp_async_commit();  // one group per stage, empty past the end
     };
-    if (J > 0) fetch(0, cs, ck, cst, clam, cg);
-    for (int j = 0; j < J; ++j) {
-        int ns[WALK_MAXO], nk[WALK_MAXO];
-        double nst[WALK_MAXO];
-        float nlam[WALK_MAXO];
-        size_t ng[WALK_MAXO];
-        if (j + 1 < J) fetch(j + 1, ns, nk, nst, nlam, ng);
-        const double Lj = Lr[j];
-#pragma unroll
-        for (int m = 0; m < WALK_MAXO; ++m) {
-            const int s = cs[m];
-            if (!slot_ok(s, N)) {
-                if (tid + m * WALK_THREADS < min(C, T - j * C) * (W + R)) P.fe[cg[m]] = 0.f;
-                continue;
-            }
-            const int jw = SMEM_TABLE ? (int)s_tab[s] : __ldcg(g_tab + s);
-            double stp;
-            bool m0 = false;
-            if (jw >= 0) {
-                stp = Lr[jw + 1];
-            } else if (isnan(cst[m])) {
-                stp = 0.0;
-                m0 = true;
-            } else {
-                stp = cst[m];
-            }
-            const float f = (float)exp(Lj + (double)clam[m] - stp);
-            P.fe[cg[m]] = m0 ? -f : f;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int m = 0; m < WALK_MAXO; ++m) {
-            const int s = cs[m];
-            if (slot_ok(s, N) && (ck[m] & LK_OWNER)) {
-                if (SMEM_TABLE) s_tab[s] = (short)j;
-                else __stcg(g_tab + s, j);
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int m = 0; m < WALK_MAXO; ++m) {
-            cs[m] = ns[m];
-            ck[m] = nk[m];
-            cst[m] = nst[m];
-            clam[m] = nlam[m];
-            cg[m] = ng[m];
-        }
-    }
 
-    // 3. final stamps of the slots written in this call, and the new Lambda
-    for (size_t o = tid; o < (size_t)T * W; o += WALK_THREADS) {
-        const int s = widx[bh * (size_t)T * W + o];
-        if (!slot_ok(s, N) || !(P.lk[occ_base + o] & LK_OWNER)) continue;
-        const int j = (int)(o / W) / C;
-        const int jw = SMEM_TABLE ? (int)s_tab[s] : __ldcg(g_tab + s);
-        if (jw == j) stamp[bh * (size_t)N + s] = Lr[j + 1];
+    __syncthreads();
+    for (int s = 0; s < WALK_RING - 1; ++s) load_stage(s);
+    for (int j = 0; j < J; ++j) {
+        load_stage(j + WALK_RING - 1);
+        asm volatile("cp.async.wait_group %0;\n" ::"n"(WALK_RING - 1) : "memory");
+        __syncthreads();
+        const uint32_t* ow = s_ring + (j % WALK_RING) * stage;
+        const float* lamc = reinterpret_cast<const float*>(ow + PLAN_MAX_OCC);
+        const int t0 = j * C, nt = min(C, T - t0), nw = nt * W, no = nt * (W + R);
+        const double Lj = Lr[j];
+        // rows of slots written by an earlier chunk carry that chunk's end stamp
+        for (int o = tid; o < no; o += WALK_THREADS) {
+            const int s = (int)(ow[o] & OCC_SLOT);
+            if (s >= N || s % WALK_PARTS != part) continue;
+            const int jw = s_tab[s / WALK_PARTS];
+            if (jw < 0) continue;
+            int t;
+            size_t g;
+            if (o < nw) {
+                t = o / W;
+                g = occ_base + (size_t)t0 * W + o;
+            } else {
+                t = (o - nw) / R;
+                g = occ_base + (size_t)T * W + (size_t)t0 * R + (o - nw);
+            }
+            P.fe[g] = expf((float)(Lj - Lr[jw + 1]) + lamc[t]);
+        }
+        __syncthreads();
+        for (int o = tid; o < nw; o += WALK_THREADS) {
+            const uint32_t w = ow[o];
+            const int s = (int)(w & OCC_SLOT);
+            if (!(w & OCC_OWNER) || s >= N || s % WALK_PARTS != part) continue;
+            s_tab[s / WALK_PARTS] = (short)j;
+        }
+        __syncthreads();
     }
-    if (tid == 0) lambda[bh] = Lr[J];
+    asm volatile("cp.async.wait_all;\n" ::: "memory");
+
+    // final stamps of this partition's slots written in this call
+    for (size_t o = tid; o < (size_t)T * W; o += WALK_THREADS) {
+        const uint32_t w = P.occw[occ_base + o];
+        const int s = (int)(w & OCC_SLOT);
+        if (!(w & OCC_OWNER) || s >= N || s % WALK_PARTS != part) continue;
+        const int j = (int)(o / W) / C;
+        if (s_tab[s / WALK_PARTS] == j) stamp[bh * (size_t)N + s] = Lr[j + 1];
+    }
 }
 
 }  // namespace sdm

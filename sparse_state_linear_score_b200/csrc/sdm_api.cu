@@ -20,7 +20,7 @@ namespace {
 
 constexpr int kMaxTop = 64;
 constexpr size_t kSmemBudget = 220 * 1024;  // dynamic shared memory per CTA we plan for
-constexpr int kWalkSmemSlots = 65536;        // walk table in shared memory up to this N
+constexpr size_t kMaskBudget = size_t(512) << 20;  // workspace bytes for per-slot chunk masks
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -57,9 +57,10 @@ int chunk_tokens(const sdm_dims* d) {
 
 struct WsLayout {
     int C, J;
-    bool smem_table, lstart_smem;
+    bool lstart_smem;
     size_t walk_smem;
-    size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_mats, off_lastw, total;
+    size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_mats, off_occw, off_mask, total;
+    int MW;  // mask words per slot, 0 when the walk is used
 };
 
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -70,10 +71,10 @@ WsLayout ws_layout(const sdm_dims* d) {
     const size_t occ = T * (size_t)(d->W + d->R);
     L.C = chunk_tokens(d);
     L.J = (int)((T + L.C - 1) / L.C);
-    L.smem_table = N <= (size_t)kWalkSmemSlots && L.J <= 32767;
-    const size_t tab_bytes = L.smem_table ? N * 2 : 0;
-    L.lstart_smem = (size_t)(L.J + 1) * 8 + tab_bytes <= kSmemBudget;
-    L.walk_smem = (L.lstart_smem ? (size_t)(L.J + 1) * 8 : 0) + tab_bytes;
+    const size_t ring = (size_t)WALK_RING * (PLAN_MAX_OCC + PLAN_MAX_C) * 4;
+    const size_t tab_bytes = ((N + WALK_PARTS - 1) / WALK_PARTS) * 2;
+    L.lstart_smem = ring + (size_t)(L.J + 1) * 8 + tab_bytes <= kSmemBudget;
+    L.walk_smem = ring + (L.lstart_smem ? (size_t)(L.J + 1) * 8 : 0) + tab_bytes;
     size_t o = 0;
     L.off_lam = o;    o = up256(o + BH * T * 4);
     L.off_csum = o;   o = up256(o + BH * L.J * 8);
@@ -82,7 +83,11 @@ WsLayout ws_layout(const sdm_dims* d) {
     L.off_fe = o;     o = up256(o + BH * occ * 4);
     L.off_lk = o;     o = up256(o + BH * occ * 4);
     L.off_mats = o;   o = up256(o + BH * (size_t)L.J * 2 * L.C * L.C * 4);
-    L.off_lastw = o;  o = up256(o + (L.smem_table ? 0 : BH * N * 4));
+    L.off_occw = o;   o = up256(o + BH * occ * 4);
+    // per-slot chunk masks replace the sequential walk when they stay small
+    const size_t mw = (size_t)(L.J + 63) / 64;
+    L.MW = (L.J <= 512 && BH * N * mw * 8 <= kMaskBudget) ? (int)mw : 0;
+    L.off_mask = o;   o = up256(o + BH * N * (size_t)L.MW * 8);
     L.total = o;
     return L;
 }
@@ -97,7 +102,9 @@ PlanPtrs plan_ptrs(const WsLayout& L, void* ws) {
     P.fe = reinterpret_cast<float*>(b + L.off_fe);
     P.lk = reinterpret_cast<int32_t*>(b + L.off_lk);
     P.mats = reinterpret_cast<float*>(b + L.off_mats);
-    P.lastw = reinterpret_cast<int32_t*>(b + L.off_lastw);
+    P.occw = reinterpret_cast<uint32_t*>(b + L.off_occw);
+    P.mask = L.MW ? reinterpret_cast<unsigned long long*>(b + L.off_mask) : nullptr;
+    P.MW = L.MW;
     return P;
 }
 
@@ -369,30 +376,29 @@ sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const floa
         !aligned16(ridx) || !aligned16(rw))
         return SDM_ERR_ALIGN;
     const WsLayout L = ws_layout(dims);
+    if (L.J > 32767) return SDM_ERR_SHAPE;  // chunk indices are 16-bit in the walk's table
     if (!ws || ws_bytes < L.total) return SDM_ERR_WORKSPACE;
     if (!aligned16(ws)) return SDM_ERR_ALIGN;
     const PlanPtrs P = plan_ptrs(L, ws);
     const int N = (int)N_of(dims);
     const size_t BH = (size_t)BH_of(dims);
-    if (!L.smem_table &&
-        cudaMemsetAsync(P.lastw, 0xff, BH * (size_t)N * 4, stream) != cudaSuccess)
+    if (P.mask &&
+        cudaMemsetAsync(P.mask, 0, BH * (size_t)N * L.MW * 8, stream) != cudaSuccess)
         return SDM_ERR_CUDA;
     if (!set_smem(plan_local_kernel, plan_local_smem_bytes())) return SDM_ERR_CUDA;
     plan_local_kernel<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, plan_local_smem_bytes(),
                         stream>>>(
         alpha, beta, widx, ww, ridx, rw, st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, P);
     if ((e = launch_status())) return e;
-    if (L.smem_table) {
-        if (!set_smem(plan_walk_kernel<true>, L.walk_smem)) return SDM_ERR_CUDA;
-        plan_walk_kernel<true><<<(unsigned)BH, WALK_THREADS, L.walk_smem, stream>>>(
-            widx, ridx, st->stamp, st->Lambda, dims->T, N, dims->W, dims->R, L.C, L.J,
-            L.lstart_smem ? 1 : 0, P);
-    } else {
-        if (!set_smem(plan_walk_kernel<false>, L.walk_smem)) return SDM_ERR_CUDA;
-        plan_walk_kernel<false><<<(unsigned)BH, WALK_THREADS, L.walk_smem, stream>>>(
-            widx, ridx, st->stamp, st->Lambda, dims->T, N, dims->W, dims->R, L.C, L.J,
-            L.lstart_smem ? 1 : 0, P);
-    }
+    plan_prefix_kernel<<<(unsigned)BH, 1024, 0, stream>>>(st->Lambda, L.J, P);
+    if ((e = launch_status())) return e;
+    plan_fe_kernel<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, 0, stream>>>(
+        st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, P);
+    if ((e = launch_status())) return e;
+    if (P.mask) return SDM_OK;  // factors and stamps are final
+    if (!set_smem(plan_walk_kernel, L.walk_smem)) return SDM_ERR_CUDA;
+    plan_walk_kernel<<<dim3(WALK_PARTS, (unsigned)BH), WALK_THREADS, L.walk_smem, stream>>>(
+        st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, L.lstart_smem ? 1 : 0, P);
     return launch_status();
 }
 

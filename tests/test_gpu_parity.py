@@ -154,6 +154,20 @@ def test_forward_shared_slots(sdm, orc, T, pool, W, R):
     _forward_case(sdm, orc, wl, inp, widx, ww, ridx, rw, TOL["f32"])
 
 
+def test_forward_long_call_walk_path(sdm, orc):
+    """More than 512 chunks in one call: the plan takes its sequential walk instead of the
+    per-slot chunk masks; results must not depend on which is used."""
+    wl = S.TINY.scaled(B=1, H=1, T=17000, n_sub=16, d_v=16, k_half=4, W=4, R=4,
+                       alpha=("uniform", 0.97, 1.0))
+    inp = to_dev(S.generate(wl))
+    g = torch.Generator().manual_seed(17)
+    widx = S.random_indices(1, 1, wl.T, wl.N, 4, g, pool=64).cuda()
+    ridx = S.random_indices(1, 1, wl.T, wl.N, 4, g, pool=64).cuda()
+    ww = S.random_weights(1, 1, wl.T, 4, g).cuda()
+    rw = S.random_weights(1, 1, wl.T, 4, g).cuda()
+    _forward_case(sdm, orc, wl, inp, widx, ww, ridx, rw, TOL["f32"])
+
+
 def test_prefill_end_to_end(sdm, orc):
     """Scoring + recurrence: selections against the oracle, outputs against the oracle's
     recurrence run on the GPU's selections (so a near tie cannot fail the output check)."""
