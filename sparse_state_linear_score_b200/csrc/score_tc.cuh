@@ -6,14 +6,15 @@
 //     of one half; one thread issues 4 tcgen05.mma (K = 64 = 4 x 16) into 256 TMEM columns:
 //     D[row][j] = <x_half[row], C[j]> in fp32.
 //   - Thread r owns row r (TMEM lane r).  It keeps the k best sub-keys of each half exactly:
-//     min/max pass, a 64-bin histogram to find the threshold bin, compaction of the bins
+//     min/max pass, a 64-bin histogram (shared-memory atomics) to find the threshold bin,
+//     compaction of the bins
 //     above it plus the best of the threshold bin (refined with finer bins when crowded),
 //     then a register bitonic sort (best first; equal scores to the lower sub-index).
 //     Halves with more than 256 sub-keys merge the per-round lists.
-//   - The k x k combine walks the pairs in decreasing order with a max-heap over the rows
-//     of the first list (pairs with (a+1)(b+1) > top are never pushed: >= top pairs beat
-//     them), giving the top-W (or top-R) slots s = i*n + j best first, then the softmax of
-//     the selected scores (§4 "SDM Configuration").
+//   - The k x k combine ranks the pairs (a, b) of the two sorted lists with
+//     (a+1)(b+1) <= k (any other pair is beaten by >= k >= top pairs) with the same exact
+//     selection, ids = slots s = i*n + j (equal sums: lower slot), giving the top-W (or
+//     top-R) slots best first, then the softmax of the selected scores (§4 "SDM Configuration").
 #pragma once
 
 #include <math.h>
@@ -31,9 +32,12 @@ constexpr int TC_MAXLEV = 4;    // histogram refinement levels
 constexpr int TC_KMAX = 32;     // largest k_half / top this kernel takes
 
 // Shared-memory map (bytes from a 1024-aligned base).
-constexpr uint32_t TC_OFF_A = 0;         // x tile: half 0 [0,16K), half 1 [16K,32K); later list R1
-constexpr uint32_t TC_OFF_B = 32768;     // sub-key round tile; selection scratch; combine heap
-constexpr uint32_t TC_OFF_HIST = 65536;  // u16 hist [64][128]; later the selected scores [top][128]
+constexpr uint32_t TC_OFF_A = 0;         // x tile: half 0 [0,16K), half 1 [16K,32K); later list
+                                         // R1 [0, K*768) and the combine's handles [24K, 32K)
+constexpr uint32_t TC_OFF_B = 32768;     // sub-key round tile, then: [0,16K) round-merge list or
+                                         // combine scores, [16K, 28.5K) boundary lists
+constexpr uint32_t TC_OFF_BND = TC_OFF_B + 16384;
+constexpr uint32_t TC_OFF_HIST = 65536;  // packed u16 histogram [32 words][128]
 constexpr uint32_t TC_OFF_R0 = 81920;    // list R0: f32 [K][128] + u16 [K][128]
 constexpr uint32_t TC_OFF_CTRL = 81920 + 24576;
 constexpr uint32_t TC_SMEM_BYTES = TC_OFF_CTRL + 64 + 1024;  // + alignment slack
@@ -111,151 +115,131 @@ SDM_DEV int tc_chain_bin(float v, const float* lo, const float* sc, const int* t
     return tc_bin(v, lo[L], sc[L]);
 }
 
-// The K best of this thread's NB TMEM columns (sub-index = col_base + column), returned
-// sorted best-first in a[0..K) (entries K..KP-1 are padding).  Per-thread shared arrays
-// are strided by TC_THREADS.  Every TMEM pass is executed by whole warps (tcgen05.ld is
-// warp-collective); the per-thread state only predicates the work inside a pass.
-// Level 0 (64 bins over [min, max]) is the fast path; the rare refinement levels (more
-// than TC_BC scores in the threshold bin, or all scores equal) run a compact generic loop.
-template <int KP>
-SDM_DEV void tc_select(uint32_t trow, int NB, int K, int col_base, uint16_t* hist, float* Sv,
-                       uint16_t* Si, float* Bv, uint16_t* Bi, float (&a)[KP], int (&ai)[KP]) {
+// Per-thread histogram of 64 bins packed as 16-bit counters in 32 shared words (one column per
+// thread).  Updates are shared-memory atomics without a return value, so consecutive scores do
+// not wait on each other.
+SDM_DEV void hist_clear(uint32_t* h) {
+#pragma unroll
+    for (int w = 0; w < TC_NBIN / 2; ++w) h[w * TC_THREADS] = 0u;
+}
+SDM_DEV void hist_add(uint32_t* h, int bn) {
+    atomicAdd(h + (bn >> 1) * TC_THREADS, 1u << ((bn & 1) * 16));
+}
+// Highest bin t_b whose bins above it hold fewer than `need` (count above -> cum, in it -> cnt).
+SDM_DEV void hist_threshold(const uint32_t* h, int need, int& t_b, int& cum, int& cnt) {
+    uint32_t w[TC_NBIN / 2];
+#pragma unroll
+    for (int i = 0; i < TC_NBIN / 2; ++i) w[i] = h[i * TC_THREADS];
+    int c = 0, tb = 0, above = 0, in_tb = 0;
+    bool found = false;
+#pragma unroll
+    for (int bn = TC_NBIN - 1; bn >= 0; --bn) {
+        const int k = (int)((w[bn >> 1] >> ((bn & 1) * 16)) & 0xffffu);
+        const bool hit = !found && c + k >= need;
+        tb = hit ? bn : tb;
+        above = hit ? c : above;
+        in_tb = hit ? k : in_tb;
+        found = found || hit;
+        c += k;
+    }
+    t_b = tb;
+    cum = above;
+    cnt = in_tb;
+}
+
+// Shared-memory stores performed only by the lanes whose p is set (predicated, no branch).
+SDM_DEV void st_shared_if(bool p, uint32_t addr, float v) {
+    asm volatile("{\n .reg .pred q;\n setp.ne.b32 q, %0, 0;\n @q st.shared.f32 [%1], %2;\n}\n" ::"r"(
+                     (int)p),
+                 "r"(addr), "f"(v)
+                 : "memory");
+}
+SDM_DEV void st_shared_if_u16(bool p, uint32_t addr, int v) {
+    asm volatile("{\n .reg .pred q;\n setp.ne.b32 q, %0, 0;\n @q st.shared.u16 [%1], %2;\n}\n" ::"r"(
+                     (int)p),
+                 "r"(addr), "h"((unsigned short)v)
+                 : "memory");
+}
+
+struct TcRefine {
+    int ns, nbd, need;
+    bool small;
+};
+
+// Refinement of the threshold bin by finer histograms over its interval, for the lanes that
+// are not done; called by whole warps (the loop condition is warp-uniform, and lanes that are
+// done still take part in src.load).  Kept out of line: it is rare, and inlined it would cost
+// the common path registers.
+template <bool GUARD, class Src>
+__device__ __noinline__ TcRefine tc_refine(const Src src, int NV, bool done, float lo, float sc,
+                                           int t_b, TcRefine io, uint32_t* hist, float* Sv,
+                                           uint16_t* Sh, float* Bv, uint16_t* Bh) {
     constexpr int S = TC_THREADS;
     constexpr unsigned FULL = 0xffffffffu;
-    float mn = INFINITY, mx = -INFINITY;
-    for (int c = 0; c < NB; c += 32) {
-        float v[32];
-        ptx::tmem_ld32(trow + c, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            mn = fminf(mn, v[i]);
-            mx = fmaxf(mx, v[i]);
-        }
-    }
-    int ns = 0, need = K;
-    // all scores equal (or not numbers): the first K sub-indices win the ties
-    const bool flat = !(mx > mn) || !isfinite((float)TC_NBIN / (mx - mn));
-    float lo[TC_MAXLEV], sc[TC_MAXLEV];
+    int ns = io.ns, nbd = io.nbd, need = io.need;
+    bool small = io.small;
+    float lv[TC_MAXLEV], sv[TC_MAXLEV];
     int tb[TC_MAXLEV];
-    lo[0] = flat ? 0.f : mn;
-    sc[0] = flat ? 0.f : (float)TC_NBIN / (mx - mn);
-
-    // ---- level 0: histogram, threshold, compaction (fast path) ----
-    int t_b = 0, cum = 0, cnt_tb = 0;
-    if (!flat)
-        for (int bn = 0; bn < TC_NBIN; ++bn) hist[bn * S] = 0;
-    for (int c = 0; c < NB; c += 32) {
-        float v[32];
-        ptx::tmem_ld32(trow + c, v);
-        if (!flat) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int bn = tc_bin(v[i], lo[0], sc[0]);
-                hist[bn * S] = (uint16_t)(hist[bn * S] + 1);
-            }
-        }
-    }
-    if (!flat) {
-        for (int bn = TC_NBIN - 1; bn >= 0; --bn) {
-            const int cnt = hist[bn * S];
-            if (cum + cnt >= need) {
-                t_b = bn;
-                break;
-            }
-            cum += cnt;
-        }
-        cnt_tb = hist[t_b * S];
-    }
+    lv[0] = lo;
+    sv[0] = sc;
     tb[0] = t_b;
-    bool small = !flat && cnt_tb <= TC_BC;
-    int nbd = 0;
-    for (int c = 0; c < NB; c += 32) {
-        float v[32];
-        ptx::tmem_ld32(trow + c, v);
-        if (!flat) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int bn = tc_bin(v[i], lo[0], sc[0]);
-                if (bn > t_b) {
-                    Sv[ns * S] = v[i];
-                    Si[ns * S] = (uint16_t)(col_base + c + i);
-                    ++ns;
-                } else if (small && bn == t_b) {
-                    Bv[nbd * S] = v[i];
-                    Bi[nbd * S] = (uint16_t)(col_base + c + i);
-                    ++nbd;
-                }
-            }
-        }
-    }
-    if (!flat) need -= cum;
-    bool done = small;
-
-    // ---- rare: refinement levels, or all-equal scores ----
-    // The loop condition is warp-uniform; inactive lanes still take part in the TMEM loads.
     int L = 0;
     while (__any_sync(FULL, !done)) {
         const bool act = !done;
-        if (act && !flat) {  // refine inside the crowded threshold bin of level L
-            lo[L + 1] = lo[L] + (float)tb[L] / sc[L];
-            sc[L + 1] = sc[L] * (float)TC_NBIN;
+        if (act) {
+            lv[L + 1] = lv[L] + (float)tb[L] / sv[L];
+            sv[L + 1] = fminf(sv[L] * (float)TC_NBIN, 1e38f);
             ++L;
         }
-        // flat rows, or the deepest level: take the chain members in index order
-        const bool last = act && (flat || L == TC_MAXLEV - 1);
+        // the deepest level takes the chain members in item order
+        const bool last = act && L == TC_MAXLEV - 1;
         const bool refine = act && !last;
         int cum2 = 0, t2 = 0, cnt2 = 0;
-        if (refine)
-            for (int bn = 0; bn < TC_NBIN; ++bn) hist[bn * S] = 0;
-        for (int c = 0; c < NB; c += 32) {
+        if (refine) hist_clear(hist);
+        for (int c = 0; c < NV; c += 32) {
             float v[32];
-            ptx::tmem_ld32(trow + c, v);
+            int hd[32];
+            src.load(c, v, hd);
             if (refine) {
 #pragma unroll 1
                 for (int i = 0; i < 32; ++i) {
-                    const int bn = tc_chain_bin(v[i], lo, sc, tb, L);
-                    if (bn >= 0) hist[bn * S] = (uint16_t)(hist[bn * S] + 1);
+                    if (GUARD && c + i >= NV) break;
+                    const int bn = tc_chain_bin(v[i], lv, sv, tb, L);
+                    if (bn >= 0) hist_add(hist, bn);
                 }
             }
         }
         if (refine) {
-            for (int bn = TC_NBIN - 1; bn >= 0; --bn) {
-                const int cnt = hist[bn * S];
-                if (cum2 + cnt >= need) {
-                    t2 = bn;
-                    break;
-                }
-                cum2 += cnt;
-            }
-            cnt2 = hist[t2 * S];
+            hist_threshold(hist, need, t2, cum2, cnt2);
             tb[L] = t2;
         }
         const bool small2 = refine && cnt2 <= TC_BC;
         if (small2) nbd = 0;
         int take_direct = last ? need : 0;
-        for (int c = 0; c < NB; c += 32) {
+        for (int c = 0; c < NV; c += 32) {
             float v[32];
-            ptx::tmem_ld32(trow + c, v);
+            int hd[32];
+            src.load(c, v, hd);
             if (act) {
 #pragma unroll 1
                 for (int i = 0; i < 32; ++i) {
-                    const uint16_t col = (uint16_t)(col_base + c + i);
-                    const int bn = flat ? 0 : tc_chain_bin(v[i], lo, sc, tb, L);
+                    if (GUARD && c + i >= NV) break;
+                    const int bn = tc_chain_bin(v[i], lv, sv, tb, L);
                     if (bn < 0) continue;
                     if (last) {
                         if (take_direct > 0) {
                             Sv[ns * S] = v[i];
-                            Si[ns * S] = col;
+                            Sh[ns * S] = (uint16_t)hd[i];
                             ++ns;
                             --take_direct;
                         }
                     } else if (bn > t2) {
                         Sv[ns * S] = v[i];
-                        Si[ns * S] = col;
+                        Sh[ns * S] = (uint16_t)hd[i];
                         ++ns;
                     } else if (small2 && bn == t2) {
                         Bv[nbd * S] = v[i];
-                        Bi[nbd * S] = col;
+                        Bh[nbd * S] = (uint16_t)hd[i];
                         ++nbd;
                     }
                 }
@@ -271,8 +255,99 @@ SDM_DEV void tc_select(uint32_t trow, int NB, int K, int col_base, uint16_t* his
             }
         }
     }
+    return TcRefine{ns, nbd, need, small};
+}
+
+// Exact top-K (value desc, id asc) of the NV items of src, which produces them 32 at a time:
+// src.load(c, v, hd) gives the values and 16-bit handles of items c..c+31 (c a multiple of 32;
+// called by whole warps with the same c, it may be warp-collective) and src.id_of(hd) the id
+// of a handle.  With GUARD, items c+i >= NV are skipped (otherwise NV is a multiple of 32).
+// src.bounds(lo, mx, fl) gives the maximum mx, a bound lo with at least K items at or above
+// it (so the K-th best is >= lo), and a bound fl no item lies below.  K <= 32.  The K winners
+// are left unsorted in Sv/Sh (strided by TC_THREADS), then returned sorted in a[0..K)
+// (padding beyond).
+//
+// A 64-bin histogram over [lo, mx] (items below lo counted in bin 0) finds the bin holding
+// the K-th best.  Items in higher bins are taken; the threshold bin is ranked exactly when it
+// holds <= TC_BC items, else refined with finer bins.  A lane whose threshold lands in bin 0
+// takes the histogram again over [fl, mx].
+template <int KP, bool GUARD, class Src>
+SDM_DEV void tc_select(const Src& src, int NV, int K, uint32_t* hist, float* Sv, uint16_t* Sh,
+                       float* Bv, int* Bi, uint16_t* Bh, float (&a)[KP], int (&ai)[KP]) {
+    constexpr int S = TC_THREADS;
+    constexpr unsigned FULL = 0xffffffffu;
+    float lo, mx, fl;
+    src.bounds(lo, mx, fl);
+    // all the items at or above lo equal the maximum: the K best are the first K of them
+    const bool flat = !(mx > lo);
+    float sc = flat ? 0.f : fminf((float)TC_NBIN / (mx - lo), 1e38f);
+
+    // ---- level 0 histogram ----
+    int t_b = 0, cum = 0, cnt_tb = 0;
+    bool redo = false;
+    for (int attempt = 0; attempt < 2; ++attempt) {
+        if (attempt == 1 && !__any_sync(FULL, redo)) break;
+        const bool act = !flat && (attempt == 0 || redo);
+        if (act) hist_clear(hist);
+        for (int c = 0; c < NV; c += 32) {
+            float v[32];
+            int hd[32];
+            src.load(c, v, hd);
+            if (act) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (!GUARD || c + i < NV) hist_add(hist, tc_bin(v[i], lo, sc));
+            }
+        }
+        if (act) {
+            hist_threshold(hist, K, t_b, cum, cnt_tb);
+            redo = attempt == 0 && t_b == 0 && lo > fl;
+            if (redo) {
+                lo = fl;
+                sc = fminf((float)TC_NBIN / (mx - fl), 1e38f);
+            }
+        }
+    }
+
+    // ---- compaction: bins above the threshold bin (flat rows: the first K maxima), and the
+    //      threshold bin itself when it is small ----
+    bool small = !flat && cnt_tb <= TC_BC;
+    int ns = 0, nbd = 0;
+    const uint32_t sv0 = ptx::smem_u32(Sv), sh0 = ptx::smem_u32(Sh);
+    const uint32_t bv0 = ptx::smem_u32(Bv), bh0 = ptx::smem_u32(Bh);
+    for (int c = 0; c < NV; c += 32) {
+        float v[32];
+        int hd[32];
+        src.load(c, v, hd);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const bool valid = !GUARD || c + i < NV;
+            const int bn = tc_bin(v[i], lo, sc);
+            const bool take = valid && (flat ? (v[i] == mx && ns < K) : bn > t_b);
+            st_shared_if(take, sv0 + ns * (S * 4), v[i]);
+            st_shared_if_u16(take, sh0 + ns * (S * 2), hd[i]);
+            ns += take ? 1 : 0;
+            const bool bnd = small && valid && bn == t_b;
+            st_shared_if(bnd, bv0 + nbd * (S * 4), v[i]);
+            st_shared_if_u16(bnd, bh0 + nbd * (S * 2), hd[i]);
+            nbd += bnd ? 1 : 0;
+        }
+    }
+    int need = flat ? 0 : K - cum;
+    const bool done = flat || small;
+
+    // ---- rare: refinement levels inside a crowded threshold bin (out of line) ----
+    if (__any_sync(FULL, !done)) {
+        const TcRefine r = tc_refine<GUARD>(src, NV, done, lo, sc, t_b, {ns, nbd, need, small},
+                                            hist, Sv, Sh, Bv, Bh);
+        ns = r.ns;
+        nbd = r.nbd;
+        need = r.need;
+        small = r.small;
+    }
     // the `need` best of the boundary bin, by exact rank
     if (small) {
+        for (int e = 0; e < nbd; ++e) Bi[e * S] = src.id_of(Bh[e * S]);
         for (int e = 0; e < nbd; ++e) {
             const float ve = Bv[e * S];
             const int ie = Bi[e * S];
@@ -280,7 +355,7 @@ SDM_DEV void tc_select(uint32_t trow, int NB, int K, int col_base, uint16_t* his
             for (int f = 0; f < nbd; ++f) rank += better(Bv[f * S], Bi[f * S], ve, ie);
             if (rank < need) {
                 Sv[ns * S] = ve;
-                Si[ns * S] = (uint16_t)ie;
+                Sh[ns * S] = Bh[e * S];
                 ++ns;
             }
         }
@@ -289,10 +364,105 @@ SDM_DEV void tc_select(uint32_t trow, int NB, int K, int col_base, uint16_t* his
     for (int e = 0; e < KP; ++e) {
         const bool ok = e < ns && e < K;
         a[e] = ok ? Sv[e * S] : -INFINITY;
-        ai[e] = ok ? (int)Si[e * S] : 0x7fffffff;
+        ai[e] = ok ? src.id_of(Sh[e * S]) : 0x7fffffff;
     }
     bitonic_sort_desc<KP>(a, ai);
 }
+
+// Scores of this thread's row from TMEM, 32 columns at a time (warp-collective loads);
+// handles are the columns inside the round.
+struct TmemSource {
+    uint32_t trow;
+    int col_base, NV;
+    SDM_DEV void load(int c, float (&v)[32], int (&hd)[32]) const {
+        ptx::tmem_ld32(trow + c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) hd[i] = c + i;
+    }
+    SDM_DEV int id_of(int hd) const { return col_base + hd; }
+    // lo = the smallest of the maxima of the 32 groups {c + i} (each group is non-empty, so
+    // at least 32 items are >= lo); fl = the minimum.
+    SDM_DEV void bounds(float& lo, float& mx, float& fl) const {
+        float gmax[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) gmax[i] = -INFINITY;
+        float mn = INFINITY;
+        for (int c = 0; c < NV; c += 32) {
+            float v[32];
+            ptx::tmem_ld32(trow + c, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                gmax[i] = fmaxf(gmax[i], v[i]);
+                mn = fminf(mn, v[i]);
+            }
+        }
+        lo = INFINITY;
+        mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            lo = fminf(lo, gmax[i]);
+            mx = fmaxf(mx, gmax[i]);
+        }
+        fl = mn;
+    }
+};
+
+// For each top <= TC_KMAX: the pairs (a, b) of positions in the two sorted half lists with
+// (a+1)(b+1) <= top, in (a, b) order.  Only these can reach the top `top` of the k x k sums:
+// any other pair is beaten by the (a+1)(b+1) - 1 >= top pairs (a' <= a, b' <= b), whose sums
+// are no smaller and whose slots are no larger on equal sums.  When all their sums are equal,
+// (a, b) order is slot order (equal half scores are listed lower sub-index first).
+constexpr int TC_PAIR_TOTAL = 1724;  // sum over top = 1..32 of sum_a floor(top / a)
+struct PairTab {
+    uint16_t ab[TC_PAIR_TOTAL];  // (a << 8) | b
+    int off[TC_KMAX + 1], cnt[TC_KMAX + 1];
+};
+constexpr PairTab make_pair_tab() {
+    PairTab t{};
+    int e = 0;
+    for (int top = 1; top <= TC_KMAX; ++top) {
+        t.off[top] = e;
+        for (int a = 0; a < top; ++a)
+            for (int b = 0; (a + 1) * (b + 1) <= top; ++b) t.ab[e++] = (uint16_t)((a << 8) | b);
+        t.cnt[top] = e - t.off[top];
+    }
+    return t;
+}
+static_assert(make_pair_tab().off[TC_KMAX] + make_pair_tab().cnt[TC_KMAX] == TC_PAIR_TOTAL,
+              "pair table size");
+__constant__ PairTab c_pair_tab = make_pair_tab();
+
+// Candidate pairs of the two sorted half lists (per-thread, strided by TC_THREADS in shared
+// memory); handles are (a << 8) | b.
+struct PairSource {
+    const float* R0v;
+    const uint16_t* R0i;
+    const float* R1v;
+    const uint16_t* R1i;
+    int tab0, NV, top, n;  // this top's pairs: c_pair_tab.ab[tab0 .. tab0 + NV)
+    SDM_DEV void load(int c, float (&v)[32], int (&hd)[32]) const {
+        constexpr int S = TC_THREADS;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int e = c + i;  // warp-uniform: constant-cache broadcast
+            const int ab = e < NV ? (int)c_pair_tab.ab[tab0 + e] : 0;
+            v[i] = e < NV ? R0v[(ab >> 8) * S] + R1v[(ab & 0xff) * S] : -INFINITY;
+            hd[i] = ab;
+        }
+    }
+    SDM_DEV int id_of(int hd) const {
+        return (int)R0i[(hd >> 8) * TC_THREADS] * n + (int)R1i[(hd & 0xff) * TC_THREADS];
+    }
+    // The pairs (0, b) and (a, 0), b, a < top, are candidates: lo = the larger of their
+    // smallest sums; fl = the sum of the top-th entries bounds every candidate from below.
+    SDM_DEV void bounds(float& lo, float& mx, float& fl) const {
+        const int q = (top - 1) * TC_THREADS;
+        const float a0 = R0v[0], b0 = R1v[0], aq = R0v[q], bq = R1v[q];
+        lo = fmaxf(a0 + bq, aq + b0);
+        mx = a0 + b0;
+        fl = aq + bq;
+    }
+};
 
 template <int KP>
 __global__ void __launch_bounds__(TC_THREADS, 2) score_tc_kernel(
@@ -332,15 +502,17 @@ __global__ void __launch_bounds__(TC_THREADS, 2) score_tc_kernel(
     const int rounds = (n + TC_NB - 1) / TC_NB;
     const uint32_t abox = 64u * 2u * (uint32_t)(p.bt * p.bb);
 
-    uint16_t* hist = reinterpret_cast<uint16_t*>(sm + TC_OFF_HIST) + tid;
-    float* Sv = reinterpret_cast<float*>(sm + TC_OFF_B) + tid;
-    uint16_t* Si = reinterpret_cast<uint16_t*>(sm + TC_OFF_B + K * S * 4) + tid;
-    float* Bv = reinterpret_cast<float*>(sm + TC_OFF_B + K * S * 6) + tid;
-    uint16_t* Bi = reinterpret_cast<uint16_t*>(sm + TC_OFF_B + K * S * 6 + TC_BC * S * 4) + tid;
+    uint32_t* hist = reinterpret_cast<uint32_t*>(sm + TC_OFF_HIST) + tid;
+    float* Bv = reinterpret_cast<float*>(sm + TC_OFF_BND) + tid;                  // [TC_BC]
+    int* Bi = reinterpret_cast<int*>(sm + TC_OFF_BND + TC_BC * S * 4) + tid;       // [TC_BC]
+    uint16_t* Bh = reinterpret_cast<uint16_t*>(sm + TC_OFF_BND + TC_BC * S * 8) + tid;
     float* R0v = reinterpret_cast<float*>(sm + TC_OFF_R0) + tid;
     uint16_t* R0i = reinterpret_cast<uint16_t*>(sm + TC_OFF_R0 + K * S * 4) + tid;
     float* R1v = reinterpret_cast<float*>(sm + TC_OFF_A) + tid;
     uint16_t* R1i = reinterpret_cast<uint16_t*>(sm + TC_OFF_A + K * S * 4) + tid;
+    // round-merge scratch list (multi-round halves, K * 768 <= 16K bytes)
+    float* Nv = reinterpret_cast<float*>(sm + TC_OFF_B) + tid;
+    uint16_t* Ni = reinterpret_cast<uint16_t*>(sm + TC_OFF_B + K * S * 4) + tid;
 
     bool aborted = false;
     for (int hf = 0; hf < 2 && !aborted; ++hf) {
@@ -382,15 +554,12 @@ __global__ void __launch_bounds__(TC_THREADS, 2) score_tc_kernel(
             }
             float a[KP];
             int ai[KP];
-            tc_select<KP>(trow, nb, K, r * TC_NB, hist, Sv, Si, Bv, Bi, a, ai);
-            if (r == 0) {
-#pragma unroll
-                for (int e = 0; e < KP; ++e)
-                    if (e < K) {
-                        Rv[e * S] = a[e];
-                        Ri[e * S] = (uint16_t)ai[e];
-                    }
-            } else {
+            TmemSource src{trow, r * TC_NB, nb};
+            // round 0 selects straight into the half's list; later rounds into scratch
+            float* Sv = r == 0 ? Rv : Nv;
+            uint16_t* Si = r == 0 ? Ri : Ni;
+            tc_select<KP, false>(src, nb, K, hist, Sv, Si, Bv, Bi, Bh, a, ai);
+            if (r > 0) {
                 float rv[KP];
                 int ri[KP];
 #pragma unroll
@@ -400,12 +569,17 @@ __global__ void __launch_bounds__(TC_THREADS, 2) score_tc_kernel(
                 }
                 bitonic_merge_keep<KP>(rv, ri, a, ai);
 #pragma unroll
-                for (int e = 0; e < KP; ++e)
-                    if (e < K) {
-                        Rv[e * S] = rv[e];
-                        Ri[e * S] = (uint16_t)ri[e];
-                    }
+                for (int e = 0; e < KP; ++e) {
+                    a[e] = rv[e];
+                    ai[e] = ri[e];
+                }
             }
+#pragma unroll
+            for (int e = 0; e < KP; ++e)
+                if (e < K) {
+                    Rv[e * S] = a[e];
+                    Ri[e * S] = (uint16_t)ai[e];
+                }
             ptx::fence_proxy_async_smem();  // these generic writes precede the next TMA write
             ptx::tc_fence_before();
             __syncthreads();
@@ -413,65 +587,27 @@ __global__ void __launch_bounds__(TC_THREADS, 2) score_tc_kernel(
     }
 
     if (!aborted) {
-        // k x k combine: max-heap over rows a of R0 (column b advances along R1)
+        // k x k combine: exact top-`top` of the candidate pairs, ids = slots (ties: lower slot)
         const int W = p.top;
-        float* hv = reinterpret_cast<float*>(sm + TC_OFF_B) + tid;
-        uint32_t* hab = reinterpret_cast<uint32_t*>(sm + TC_OFF_B + K * S * 4) + tid;
-        float* sv = reinterpret_cast<float*>(sm + TC_OFF_HIST) + tid;
-        int size = min(K, W);
-        const float r1_0 = R1v[0];
-        for (int e = 0; e < size; ++e) {
-            hv[e * S] = R0v[e * S] + r1_0;
-            hab[e * S] = (uint32_t)e << 16;
-        }
-        auto slot_of = [&](uint32_t ab) -> int {
-            return (int)R0i[(ab >> 16) * S] * n + (int)R1i[(ab & 0xffffu) * S];
-        };
-        auto hbetter = [&](int x, int y) -> bool {
-            const float vx = hv[x * S], vy = hv[y * S];
-            if (vx != vy) return vx > vy;
-            return slot_of(hab[x * S]) < slot_of(hab[y * S]);
-        };
-        const size_t row_off = ((size_t)b * p.H + h) * p.T + t;
-        for (int q = 0; q < W; ++q) {
-            if (size <= 0) {  // cannot happen for top <= k_half^2; keep outputs defined
-                sv[q * S] = -INFINITY;
-                if (row_ok) p.idx[row_off * W + q] = -1;
-                continue;
-            }
-            const uint32_t ab = hab[0];
-            sv[q * S] = hv[0];
-            if (row_ok) p.idx[row_off * W + q] = slot_of(ab);
-            const int ra = (int)(ab >> 16), cb = (int)(ab & 0xffffu) + 1;
-            if (cb < K && (ra + 1) * (cb + 1) <= W) {
-                hv[0] = R0v[ra * S] + R1v[cb * S];
-                hab[0] = ((uint32_t)ra << 16) | (uint32_t)cb;
-            } else {
-                --size;
-                hv[0] = hv[size * S];
-                hab[0] = hab[size * S];
-            }
-            int pos = 0;
-            while (true) {
-                const int c1 = 2 * pos + 1;
-                if (c1 >= size) break;
-                const int c2 = c1 + 1;
-                const int best = (c2 < size && hbetter(c2, c1)) ? c2 : c1;
-                if (!hbetter(best, pos)) break;
-                const float tv = hv[pos * S];
-                const uint32_t tab = hab[pos * S];
-                hv[pos * S] = hv[best * S];
-                hab[pos * S] = hab[best * S];
-                hv[best * S] = tv;
-                hab[best * S] = tab;
-                pos = best;
-            }
-        }
+        PairSource src{R0v, R0i, R1v, R1i, c_pair_tab.off[W], c_pair_tab.cnt[W], W, n};
+        float* Ov = reinterpret_cast<float*>(sm + TC_OFF_B) + tid;                 // [W]
+        uint16_t* Oh = reinterpret_cast<uint16_t*>(sm + TC_OFF_A + 24576) + tid;   // [W]
+        float a[KP];
+        int ai[KP];
+        tc_select<KP, true>(src, src.NV, W, hist, Ov, Oh, Bv, Bi, Bh, a, ai);
         if (row_ok) {
-            const float mx = sv[0];
+            const size_t row_off = ((size_t)b * p.H + h) * p.T + t;
+            const float mx = a[0];
             float z = 0.f;
-            for (int q = 0; q < W; ++q) z += expf(sv[q * S] - mx);
-            for (int q = 0; q < W; ++q) p.w[row_off * W + q] = expf(sv[q * S] - mx) / z;
+#pragma unroll
+            for (int q = 0; q < KP; ++q)
+                if (q < W) z += expf(a[q] - mx);
+#pragma unroll
+            for (int q = 0; q < KP; ++q)
+                if (q < W) {
+                    p.idx[row_off * W + q] = ai[q];
+                    p.w[row_off * W + q] = expf(a[q] - mx) / z;
+                }
         }
     } else if (tid == 0) {
         raise_err(SDM_DEVERR_TIMEOUT);

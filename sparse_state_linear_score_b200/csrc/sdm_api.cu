@@ -154,6 +154,7 @@ bool score_tc_eligible(const sdm_dims* d, int top) {
     if (d->n_sub % 64 != 0 || d->n_sub > 4096) return false;
     if (d->k_half > TC_KMAX || top > TC_KMAX) return false;
     if (d->n_sub > TC_NB && d->k_half * TC_THREADS * 6 > 16384) return false;  // R1 beside x half 1
+    if (top > d->k_half) return false;  // the pair staircase covers top <= k_half
     return d->T >= 64;
 }
 
