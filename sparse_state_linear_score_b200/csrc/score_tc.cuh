@@ -35,7 +35,7 @@ constexpr int TC_KMAX = 32;     // largest k_half / top this kernel takes
 constexpr uint32_t TC_OFF_A = 0;         // x tile: half 0 [0,16K), half 1 [16K,32K); later list
                                          // R1 [0, K*768) and the combine's handles [24K, 32K)
 constexpr uint32_t TC_OFF_B = 32768;     // sub-key round tile, then: [0,16K) round-merge list or
-                                         // combine scores, [16K, 28.5K) boundary lists
+                                         // combine scores, [16K, 23.5K) boundary list
 constexpr uint32_t TC_OFF_BND = TC_OFF_B + 16384;
 constexpr uint32_t TC_OFF_HIST = 65536;  // packed u16 histogram [32 words][128]
 constexpr uint32_t TC_OFF_R0 = 81920;    // list R0: f32 [K][128] + u16 [K][128]
@@ -53,6 +53,11 @@ struct ScoreTcArgs {
 SDM_DEV int tc_bin(float v, float lo, float sc) {
     int b = __float2int_rd((v - lo) * sc);
     return min(max(b, 0), TC_NBIN - 1);
+}
+
+// Level-0 bin: -1 (not counted) below lo.
+SDM_DEV int tc_bin0(float v, float lo, float sc) {
+    return v >= lo ? min(__float2int_rd((v - lo) * sc), TC_NBIN - 1) : -1;
 }
 
 template <int KP>
@@ -78,6 +83,35 @@ SDM_DEV void bitonic_sort_desc(float (&v)[KP], int (&ix)[KP]) {
             }
         }
     }
+}
+
+// Same order, cheaper: the network compares values alone (ids follow them); equal values,
+// rare, are then put in id order by the full comparison.
+template <int KP>
+SDM_DEV void sort_desc(float (&v)[KP], int (&ix)[KP]) {
+#pragma unroll
+    for (int k = 2; k <= KP; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll
+            for (int i = 0; i < KP; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const bool sw = (i & k) == 0 ? v[l] > v[i] : v[i] > v[l];
+                    const float tv = sw ? v[l] : v[i];
+                    const int ti = sw ? ix[l] : ix[i];
+                    v[l] = sw ? v[i] : v[l];
+                    ix[l] = sw ? ix[i] : ix[l];
+                    v[i] = tv;
+                    ix[i] = ti;
+                }
+            }
+        }
+    }
+    bool tie = false;
+#pragma unroll
+    for (int e = 0; e + 1 < KP; ++e) tie = tie || (v[e] == v[e + 1] && v[e] > -INFINITY);
+    if (__any_sync(0xffffffffu, tie)) bitonic_sort_desc<KP>(v, ix);
 }
 
 // Merge a sorted (best-first) list held in r[] with sorted a[]: r <- best KP of both, sorted.
@@ -110,7 +144,8 @@ SDM_DEV void bitonic_merge_keep(float (&r)[KP], int (&ri)[KP], const float (&a)[
 
 // Bin of v in the refinement chain lo/sc/tb[0..L): -1 when v is outside the chain (rare path).
 SDM_DEV int tc_chain_bin(float v, const float* lo, const float* sc, const int* tb, int L) {
-    for (int l = 0; l < L; ++l)
+    if (tc_bin0(v, lo[0], sc[0]) != tb[0]) return -1;
+    for (int l = 1; l < L; ++l)
         if (tc_bin(v, lo[l], sc[l]) != tb[l]) return -1;
     return tc_bin(v, lo[L], sc[L]);
 }
@@ -124,6 +159,13 @@ SDM_DEV void hist_clear(uint32_t* h) {
 }
 SDM_DEV void hist_add(uint32_t* h, int bn) {
     atomicAdd(h + (bn >> 1) * TC_THREADS, 1u << ((bn & 1) * 16));
+}
+// The same, performed only when p is set (a predicated reduction, no branch).
+SDM_DEV void hist_add_if(bool p, uint32_t h_addr, int bn) {
+    const uint32_t addr = h_addr + (uint32_t)((bn >> 1) & (TC_NBIN / 2 - 1)) * (TC_THREADS * 4);
+    asm volatile("{\n .reg .pred q;\n setp.ne.b32 q, %0, 0;\n @q red.shared.add.u32 [%1], %2;\n}\n" ::
+                     "r"((int)p),
+                 "r"(addr), "r"(1u << ((bn & 1) * 16)));
 }
 // Highest bin t_b whose bins above it hold fewer than `need` (count above -> cum, in it -> cnt).
 SDM_DEV void hist_threshold(const uint32_t* h, int need, int& t_b, int& cum, int& cnt) {
@@ -258,22 +300,48 @@ __device__ __noinline__ TcRefine tc_refine(const Src src, int NV, bool done, flo
     return TcRefine{ns, nbd, need, small};
 }
 
-// Exact top-K (value desc, id asc) of the NV items of src, which produces them 32 at a time:
-// src.load(c, v, hd) gives the values and 16-bit handles of items c..c+31 (c a multiple of 32;
-// called by whole warps with the same c, it may be warp-collective) and src.id_of(hd) the id
-// of a handle.  With GUARD, items c+i >= NV are skipped (otherwise NV is a multiple of 32).
-// src.bounds(lo, mx, fl) gives the maximum mx, a bound lo with at least K items at or above
-// it (so the K-th best is >= lo), and a bound fl no item lies below.  K <= 32.  The K winners
-// are left unsorted in Sv/Sh (strided by TC_THREADS), then returned sorted in a[0..K)
-// (padding beyond).
+// Rows whose items at or above lo all equal the maximum: the K best are the first K items (in
+// id order) equal to it.  Called by whole warps; only the lanes with `flat` set take items.
+template <bool GUARD, class Src>
+__device__ __noinline__ int tc_flat(const Src src, int NV, bool flat, float mx, int K,
+                                    float* Sv, uint16_t* Sh) {
+    constexpr int S = TC_THREADS;
+    int ns = 0;
+    for (int c = 0; c < NV; c += 32) {
+        float v[32];
+        int hd[32];
+        src.load(c, v, hd);
+        if (flat) {
+#pragma unroll 1
+            for (int i = 0; i < 32; ++i) {
+                if ((GUARD && c + i >= NV) || ns >= K) break;
+                if (v[i] == mx) {
+                    Sv[ns * S] = v[i];
+                    Sh[ns * S] = (uint16_t)hd[i];
+                    ++ns;
+                }
+            }
+        }
+    }
+    return ns;
+}
+
+// Exact top-K (value desc, id asc) of the items of src.  src.for_each(f) calls
+// f(value, handle, valid) for every item, in any order (for the TMEM source it is
+// warp-collective: whole warps call it); src.id_of(handle) gives an item's id;
+// src.bounds(lo, mx, fl) gives the maximum mx, a bound lo with at least K valid items at or
+// above it (so the K-th best is >= lo) and a bound fl no valid item lies below;
+// src.chunked() gives the same items 32 at a time, in id order among equal values, for the
+// rare paths.  K <= 32.
+// The K winners are left unsorted in Sv/Sh (strided by TC_THREADS), then returned sorted in
+// a[0..K) (padding beyond).
 //
-// A 64-bin histogram over [lo, mx] (items below lo counted in bin 0) finds the bin holding
-// the K-th best.  Items in higher bins are taken; the threshold bin is ranked exactly when it
-// holds <= TC_BC items, else refined with finer bins.  A lane whose threshold lands in bin 0
-// takes the histogram again over [fl, mx].
-template <int KP, bool GUARD, class Src>
-SDM_DEV void tc_select(const Src& src, int NV, int K, uint32_t* hist, float* Sv, uint16_t* Sh,
-                       float* Bv, int* Bi, uint16_t* Bh, float (&a)[KP], int (&ai)[KP]) {
+// A 64-bin histogram over [lo, mx] finds the bin holding the K-th best.  Items in higher bins
+// are taken; the threshold bin is ranked exactly when it holds <= TC_BC items, else refined
+// with finer bins.
+template <int KP, class Src>
+SDM_DEV void tc_select(const Src& src, int K, uint32_t* hist, float* Sv, uint16_t* Sh,
+                       float* Bv, uint16_t* Bh, float (&a)[KP], int (&ai)[KP]) {
     constexpr int S = TC_THREADS;
     constexpr unsigned FULL = 0xffffffffu;
     float lo, mx, fl;
@@ -284,29 +352,37 @@ SDM_DEV void tc_select(const Src& src, int NV, int K, uint32_t* hist, float* Sv,
 
     // ---- level 0 histogram ----
     int t_b = 0, cum = 0, cnt_tb = 0;
-    bool redo = false;
-    for (int attempt = 0; attempt < 2; ++attempt) {
-        if (attempt == 1 && !__any_sync(FULL, redo)) break;
-        const bool act = !flat && (attempt == 0 || redo);
-        if (act) hist_clear(hist);
-        for (int c = 0; c < NV; c += 32) {
-            float v[32];
-            int hd[32];
-            src.load(c, v, hd);
+    if constexpr (Src::kClampBelow) {
+        // Every item counted, those below lo in bin 0 (measured faster for dense TMEM rows).
+        // A lane whose threshold lands in bin 0 takes the histogram again over [fl, mx], so
+        // that bins >= the threshold bin hold no item below lo.
+        bool redo = false;
+        for (int attempt = 0; attempt < 2; ++attempt) {
+            if (attempt == 1 && !__any_sync(FULL, redo)) break;
+            const bool act = !flat && (attempt == 0 || redo);
+            if (act) hist_clear(hist);
+            src.for_each([&](float v, int, bool valid) {
+                if (act && valid) hist_add(hist, tc_bin(v, lo, sc));
+            });
             if (act) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (!GUARD || c + i < NV) hist_add(hist, tc_bin(v[i], lo, sc));
+                hist_threshold(hist, K, t_b, cum, cnt_tb);
+                redo = attempt == 0 && t_b == 0 && lo > fl;
+                if (redo) {
+                    lo = fl;
+                    sc = fminf((float)TC_NBIN / (mx - fl), 1e38f);
+                }
             }
         }
-        if (act) {
-            hist_threshold(hist, K, t_b, cum, cnt_tb);
-            redo = attempt == 0 && t_b == 0 && lo > fl;
-            if (redo) {
-                lo = fl;
-                sc = fminf((float)TC_NBIN / (mx - fl), 1e38f);
-            }
-        }
+    } else {
+        // only the items at or above lo counted
+        if (!flat) hist_clear(hist);
+        const uint32_t h0 = ptx::smem_u32(hist);
+        src.for_each([&](float v, int, bool valid) {
+            const int bn = tc_bin0(v, lo, sc);
+            hist_add_if(!flat && valid && bn >= 0, h0, bn);
+        });
+        asm volatile("" ::: "memory");  // the predicated shared-memory writes precede the scan
+        if (!flat) hist_threshold(hist, K, t_b, cum, cnt_tb);
     }
 
     // ---- compaction: bins above the threshold bin (flat rows: the first K maxima), and the
@@ -315,50 +391,60 @@ SDM_DEV void tc_select(const Src& src, int NV, int K, uint32_t* hist, float* Sv,
     int ns = 0, nbd = 0;
     const uint32_t sv0 = ptx::smem_u32(Sv), sh0 = ptx::smem_u32(Sh);
     const uint32_t bv0 = ptx::smem_u32(Bv), bh0 = ptx::smem_u32(Bh);
-    for (int c = 0; c < NV; c += 32) {
-        float v[32];
-        int hd[32];
-        src.load(c, v, hd);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const bool valid = !GUARD || c + i < NV;
-            const int bn = tc_bin(v[i], lo, sc);
-            const bool take = valid && (flat ? (v[i] == mx && ns < K) : bn > t_b);
-            st_shared_if(take, sv0 + ns * (S * 4), v[i]);
-            st_shared_if_u16(take, sh0 + ns * (S * 2), hd[i]);
-            ns += take ? 1 : 0;
-            const bool bnd = small && valid && bn == t_b;
-            st_shared_if(bnd, bv0 + nbd * (S * 4), v[i]);
-            st_shared_if_u16(bnd, bh0 + nbd * (S * 2), hd[i]);
-            nbd += bnd ? 1 : 0;
-        }
-    }
+    src.for_each([&](float v, int hd, bool valid) {
+        const int bn = tc_bin0(v, lo, sc);
+        const bool take = valid && !flat && bn > t_b;
+        st_shared_if(take, sv0 + ns * (S * 4), v);
+        st_shared_if_u16(take, sh0 + ns * (S * 2), hd);
+        ns += take ? 1 : 0;
+        const bool bnd = small && valid && bn == t_b;
+        st_shared_if(bnd, bv0 + nbd * (S * 4), v);
+        st_shared_if_u16(bnd, bh0 + nbd * (S * 2), hd);
+        nbd += bnd ? 1 : 0;
+    });
+    asm volatile("" ::: "memory");
     int need = flat ? 0 : K - cum;
     const bool done = flat || small;
+    if (__any_sync(FULL, flat)) {
+        const auto ch = src.chunked();
+        const int nf = tc_flat<decltype(ch)::kGuard>(ch, ch.NV, flat, mx, K, Sv, Sh);
+        if (flat) ns = nf;
+    }
 
     // ---- rare: refinement levels inside a crowded threshold bin (out of line) ----
     if (__any_sync(FULL, !done)) {
-        const TcRefine r = tc_refine<GUARD>(src, NV, done, lo, sc, t_b, {ns, nbd, need, small},
-                                            hist, Sv, Sh, Bv, Bh);
+        const auto ch = src.chunked();
+        const TcRefine r = tc_refine<decltype(ch)::kGuard>(ch, ch.NV, done, lo, sc, t_b,
+                                                           {ns, nbd, need, small}, hist, Sv, Sh,
+                                                           Bv, Bh);
         ns = r.ns;
         nbd = r.nbd;
         need = r.need;
         small = r.small;
     }
-    // the `need` best of the boundary bin, by exact rank
+    // the `need` best of the boundary bin (nbd <= TC_BC entries), by exact rank: the entry of
+    // rank q goes to slot ns + q
     if (small) {
-        for (int e = 0; e < nbd; ++e) Bi[e * S] = src.id_of(Bh[e * S]);
-        for (int e = 0; e < nbd; ++e) {
-            const float ve = Bv[e * S];
-            const int ie = Bi[e * S];
+        float bv[TC_BC];
+        int bi[TC_BC], bh[TC_BC];
+#pragma unroll
+        for (int e = 0; e < TC_BC; ++e) {
+            const bool ok = e < nbd;
+            bh[e] = ok ? (int)Bh[e * S] : 0;
+            bv[e] = ok ? Bv[e * S] : -INFINITY;
+            bi[e] = ok ? src.id_of(bh[e]) : 0x7fffffff;
+        }
+#pragma unroll
+        for (int e = 0; e < TC_BC; ++e) {
             int rank = 0;
-            for (int f = 0; f < nbd; ++f) rank += better(Bv[f * S], Bi[f * S], ve, ie);
-            if (rank < need) {
-                Sv[ns * S] = ve;
-                Sh[ns * S] = Bh[e * S];
-                ++ns;
+#pragma unroll
+            for (int f = 0; f < TC_BC; ++f) rank += better(bv[f], bi[f], bv[e], bi[e]) ? 1 : 0;
+            if (e < nbd && rank < need) {
+                Sv[(ns + rank) * S] = bv[e];
+                Sh[(ns + rank) * S] = (uint16_t)bh[e];
             }
         }
+        ns += need;
     }
 #pragma unroll
     for (int e = 0; e < KP; ++e) {
@@ -366,12 +452,14 @@ SDM_DEV void tc_select(const Src& src, int NV, int K, uint32_t* hist, float* Sv,
         a[e] = ok ? Sv[e * S] : -INFINITY;
         ai[e] = ok ? src.id_of(Sh[e * S]) : 0x7fffffff;
     }
-    bitonic_sort_desc<KP>(a, ai);
+    sort_desc<KP>(a, ai);
 }
 
 // Scores of this thread's row from TMEM, 32 columns at a time (warp-collective loads);
 // handles are the columns inside the round.
 struct TmemSource {
+    static constexpr bool kGuard = false;  // NV is a multiple of 32
+    static constexpr bool kClampBelow = true;
     uint32_t trow;
     int col_base, NV;
     SDM_DEV void load(int c, float (&v)[32], int (&hd)[32]) const {
@@ -379,6 +467,16 @@ struct TmemSource {
 #pragma unroll
         for (int i = 0; i < 32; ++i) hd[i] = c + i;
     }
+    template <class F>
+    SDM_DEV void for_each(F&& f) const {
+        for (int c = 0; c < NV; c += 32) {
+            float v[32];
+            ptx::tmem_ld32(trow + c, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) f(v[i], c + i, true);
+        }
+    }
+    SDM_DEV TmemSource chunked() const { return *this; }
     SDM_DEV int id_of(int hd) const { return col_base + hd; }
     // lo = the smallest of the maxima of the 32 groups {c + i} (each group is non-empty, so
     // at least 32 items are >= lo); fl = the minimum.
@@ -435,6 +533,7 @@ __constant__ PairTab c_pair_tab = make_pair_tab();
 // Candidate pairs of the two sorted half lists (per-thread, strided by TC_THREADS in shared
 // memory); handles are (a << 8) | b.
 struct PairSource {
+    static constexpr bool kGuard = true;
     const float* R0v;
     const uint16_t* R0i;
     const float* R1v;
@@ -454,7 +553,7 @@ struct PairSource {
         return (int)R0i[(hd >> 8) * TC_THREADS] * n + (int)R1i[(hd & 0xff) * TC_THREADS];
     }
     // The pairs (0, b) and (a, 0), b, a < top, are candidates: lo = the larger of their
-    // smallest sums; fl = the sum of the top-th entries bounds every candidate from below.
+    // smallest sums.
     SDM_DEV void bounds(float& lo, float& mx, float& fl) const {
         const int q = (top - 1) * TC_THREADS;
         const float a0 = R0v[0], b0 = R1v[0], aq = R0v[q], bq = R1v[q];
@@ -462,6 +561,42 @@ struct PairSource {
         mx = a0 + b0;
         fl = aq + bq;
     }
+};
+
+// The same candidates enumerated as segments: for x = 0, 1, ... with (x+1)^2 <= top, the
+// row (x, b), x <= b < top/(x+1), and the column (a, x), x < a < top/(x+1).  Each segment is a
+// fixed entry of one list plus a run of the other, read 8 at a time.
+struct PairSegSource {
+    PairSource sm;
+    template <class F>
+    SDM_DEV void for_each(F&& f) const {
+        constexpr int S = TC_THREADS;
+        const int top = sm.top;
+        int r = 0;
+        while ((r + 1) * (r + 1) <= top) ++r;
+        for (int sg = 0; sg < 2 * r; ++sg) {
+            const bool col = sg >= r;
+            const int x = col ? sg - r : sg;
+            const float fx = (col ? sm.R1v : sm.R0v)[x * S];
+            const float* run = col ? sm.R0v : sm.R1v;
+            const int beg = col ? x + 1 : x, end = top / (x + 1);
+            for (int j0 = beg; j0 < end; j0 += 8) {
+                // all 8 loads before f (whose shared-memory atomics would delay later loads)
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = fx + run[(j0 + j < end ? j0 + j : x) * S];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int y = j0 + j;
+                    f(v[j], col ? (y << 8) | x : (x << 8) | y, y < end);
+                }
+            }
+        }
+    }
+    SDM_DEV int id_of(int hd) const { return sm.id_of(hd); }
+    static constexpr bool kClampBelow = false;
+    SDM_DEV void bounds(float& lo, float& mx, float& fl) const { sm.bounds(lo, mx, fl); }
+    SDM_DEV PairSource chunked() const { return sm; }
 };
 
 template <int KP>
@@ -503,9 +638,8 @@ __global__ void __launch_bounds__(TC_THREADS, 2) score_tc_kernel(
     const uint32_t abox = 64u * 2u * (uint32_t)(p.bt * p.bb);
 
     uint32_t* hist = reinterpret_cast<uint32_t*>(sm + TC_OFF_HIST) + tid;
-    float* Bv = reinterpret_cast<float*>(sm + TC_OFF_BND) + tid;                  // [TC_BC]
-    int* Bi = reinterpret_cast<int*>(sm + TC_OFF_BND + TC_BC * S * 4) + tid;       // [TC_BC]
-    uint16_t* Bh = reinterpret_cast<uint16_t*>(sm + TC_OFF_BND + TC_BC * S * 8) + tid;
+    float* Bv = reinterpret_cast<float*>(sm + TC_OFF_BND) + tid;                     // [TC_BC]
+    uint16_t* Bh = reinterpret_cast<uint16_t*>(sm + TC_OFF_BND + TC_BC * S * 4) + tid;  // [TC_BC]
     float* R0v = reinterpret_cast<float*>(sm + TC_OFF_R0) + tid;
     uint16_t* R0i = reinterpret_cast<uint16_t*>(sm + TC_OFF_R0 + K * S * 4) + tid;
     float* R1v = reinterpret_cast<float*>(sm + TC_OFF_A) + tid;
@@ -558,7 +692,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2) score_tc_kernel(
             // round 0 selects straight into the half's list; later rounds into scratch
             float* Sv = r == 0 ? Rv : Nv;
             uint16_t* Si = r == 0 ? Ri : Ni;
-            tc_select<KP, false>(src, nb, K, hist, Sv, Si, Bv, Bi, Bh, a, ai);
+            tc_select<KP>(src, K, hist, Sv, Si, Bv, Bh, a, ai);
             if (r > 0) {
                 float rv[KP];
                 int ri[KP];
@@ -589,12 +723,13 @@ __global__ void __launch_bounds__(TC_THREADS, 2) score_tc_kernel(
     if (!aborted) {
         // k x k combine: exact top-`top` of the candidate pairs, ids = slots (ties: lower slot)
         const int W = p.top;
-        PairSource src{R0v, R0i, R1v, R1i, c_pair_tab.off[W], c_pair_tab.cnt[W], W, n};
+        const PairSegSource src{
+            PairSource{R0v, R0i, R1v, R1i, c_pair_tab.off[W], c_pair_tab.cnt[W], W, n}};
         float* Ov = reinterpret_cast<float*>(sm + TC_OFF_B) + tid;                 // [W]
         uint16_t* Oh = reinterpret_cast<uint16_t*>(sm + TC_OFF_A + 24576) + tid;   // [W]
         float a[KP];
         int ai[KP];
-        tc_select<KP, true>(src, src.NV, W, hist, Ov, Oh, Bv, Bi, Bh, a, ai);
+        tc_select<KP>(src, W, hist, Ov, Oh, Bv, Bh, a, ai);
         if (row_ok) {
             const size_t row_off = ((size_t)b * p.H + h) * p.T + t;
             const float mx = a[0];
