@@ -50,14 +50,27 @@ struct ScoreTcArgs {
     float* w;
 };
 
+// Bin position (v - lo) * sc, rounded the same way wherever it is used.
+SDM_DEV float tc_pos(float v, float lo, float sc) { return __fmul_rn(__fsub_rn(v, lo), sc); }
+
 SDM_DEV int tc_bin(float v, float lo, float sc) {
-    int b = __float2int_rd((v - lo) * sc);
+    int b = __float2int_rd(tc_pos(v, lo, sc));
     return min(max(b, 0), TC_NBIN - 1);
 }
 
 // Level-0 bin: -1 (not counted) below lo.
 SDM_DEV int tc_bin0(float v, float lo, float sc) {
-    return v >= lo ? min(__float2int_rd((v - lo) * sc), TC_NBIN - 1) : -1;
+    return v >= lo ? min(__float2int_rd(tc_pos(v, lo, sc)), TC_NBIN - 1) : -1;
+}
+
+// Smallest v with tc_pos(v, lo, sc) >= t, i.e. with bin >= t for 1 <= t < TC_NBIN (the
+// position is monotone in v): the quotient, then a walk of a few ulps.
+SDM_DEV float tc_edge(int t, float lo, float sc) {
+    const float ft = (float)t;
+    float v = lo + __fdividef(ft, sc);
+    for (int it = 0; it < 64 && tc_pos(v, lo, sc) >= ft; ++it) v = nextafterf(v, -INFINITY);
+    for (int it = 0; it < 64 && tc_pos(v, lo, sc) < ft; ++it) v = nextafterf(v, INFINITY);
+    return v;
 }
 
 template <int KP>
@@ -391,15 +404,21 @@ SDM_DEV void tc_select(const Src& src, int K, uint32_t* hist, float* Sv, uint16_
     int ns = 0, nbd = 0;
     const uint32_t sv0 = ptx::smem_u32(Sv), sh0 = ptx::smem_u32(Sh);
     const uint32_t bv0 = ptx::smem_u32(Bv), bh0 = ptx::smem_u32(Bh);
+    // bins above t_b are the values >= tau_take, bin t_b the values in [tau_bnd, tau_take)
+    // (items below lo, counted in bin 0 by the clamped histogram, are in bin t_b only when
+    // t_b = 0, and then no item lies below lo)
+    const float tau_take = flat ? INFINITY : (t_b >= TC_NBIN - 1 ? INFINITY : tc_edge(t_b + 1, lo, sc));
+    const float tau_bnd = !small ? INFINITY : (t_b == 0 ? lo : tc_edge(t_b, lo, sc));
     src.for_each([&](float v, int hd, bool valid) {
-        const int bn = tc_bin0(v, lo, sc);
-        const bool take = valid && !flat && bn > t_b;
-        st_shared_if(take, sv0 + ns * (S * 4), v);
-        st_shared_if_u16(take, sh0 + ns * (S * 2), hd);
+        const bool take = valid && v >= tau_take;
+        const uint32_t so = (uint32_t)min(ns, K - 1);  // ns < K by the histogram count
+        st_shared_if(take, sv0 + so * (S * 4), v);
+        st_shared_if_u16(take, sh0 + so * (S * 2), hd);
         ns += take ? 1 : 0;
-        const bool bnd = small && valid && bn == t_b;
-        st_shared_if(bnd, bv0 + nbd * (S * 4), v);
-        st_shared_if_u16(bnd, bh0 + nbd * (S * 2), hd);
+        const bool bnd = valid && !take && v >= tau_bnd;
+        const uint32_t bo = (uint32_t)min(nbd, TC_BC - 1);  // nbd <= TC_BC when small
+        st_shared_if(bnd, bv0 + bo * (S * 4), v);
+        st_shared_if_u16(bnd, bh0 + bo * (S * 2), hd);
         nbd += bnd ? 1 : 0;
     });
     asm volatile("" ::: "memory");
