@@ -28,7 +28,7 @@
 //   plan_prefix (one CTA per (b,h))
 //     Lstart[j]   = log-decay prefix at the start of chunk j (Lstart[0] = state Lambda);
 //                   the state Lambda becomes Lstart[J]
-//   plan_fe0 (one CTA per chunk)
+//   plan_fe (one CTA per chunk)
 //     fe[o]       = exp(Lambda_t - stamp of the row o gathers) assuming the slot was not
 //                   written earlier in this call; sign bit set when the row is the pristine
 //                   M0 row
@@ -36,6 +36,8 @@
 //     fe[o] is rewritten for slots written by an earlier chunk of this call (the row then
 //     carries the stamp of that chunk's end); the state stamps of the slots written in the
 //     call are updated.
+//   plan_pack (one CTA per chunk)
+//     rs, rc, rsc, ra, hz: what the row pass reads per occurrence (see PlanPtrs).
 //
 // In-chunk occurrence order: the nt*W write occurrences (token-major), then the nt*R
 // read occurrences.  In the per-(b,h) arrays fe / lk / st0 the T*W write entries come
@@ -109,6 +111,13 @@ struct PlanPtrs {
     uint32_t* occw;    // [BH][T*(W+R)] slot | OCC_OWNER (the walk's input)
     unsigned long long* mask;  // [BH][N][MW] chunks of this call that stored each slot, or null
     int MW;                    // 64-bit words per slot in mask
+    // the row pass's inputs, packed by plan_pack (same occurrence layout as fe / lk)
+    int32_t* rs;       // slot | bit 31 when the row gathered is the pristine M0 row
+    float* rc;         // w |fe|: the coefficient of the gathered row in p_t / o_t
+    float* rsc;        // writes: w e^{lam_end - lam_t} (the write's share of its slot's store)
+    float* ra;         // writes: |fe| e^{lam_end - lam_t} (the gathered row's share)
+    int32_t* hz;       // [BH][T*(W+R)], chunk j at j*C*(W+R): o | prev << 16 for the chunk's
+                       // occurrences whose row the previous chunk stores, then -1
 };
 
 __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
@@ -490,6 +499,55 @@ __global__ void __launch_bounds__(WALK_THREADS) plan_walk_kernel(
         const int j = (int)(o / W) / C;
         if (s_tab[s / WALK_PARTS] == j) stamp[bh * (size_t)N + s] = Lr[j + 1];
     }
+}
+
+// The row pass's per-occurrence inputs from the final decay factors: slot and pristine flag,
+// the gathered row's coefficient, the store coefficients of the writes, and the chunk's list
+// of occurrences whose row the previous chunk stores (order within the list is free).
+__global__ void __launch_bounds__(PLAN_THREADS) plan_pack_kernel(
+    const int32_t* __restrict__ widx, const float* __restrict__ ww,
+    const int32_t* __restrict__ ridx, const float* __restrict__ rw, int T, int N, int W, int R,
+    int C, PlanPtrs P) {
+    __shared__ float s_lam[PLAN_MAX_C];
+    __shared__ int s_cnt;
+    const int j = blockIdx.x;
+    const size_t bh = blockIdx.y;
+    const int tid = threadIdx.x;
+    const int t0 = j * C, nt = min(C, T - t0), nw = nt * W, no = nt * (W + R);
+    const size_t occ_base = bh * (size_t)T * (W + R);
+    int32_t* hz = P.hz + occ_base + (size_t)t0 * (W + R);
+    if (tid == 0) s_cnt = 0;
+    if (tid < nt) s_lam[tid] = P.lam[bh * T + t0 + tid];
+    __syncthreads();
+    const float lam_end = s_lam[nt - 1];
+    for (int o = tid; o < no; o += PLAN_THREADS) {
+        size_t g;
+        int s;
+        float w;
+        if (o < nw) {
+            g = occ_base + (size_t)t0 * W + o;
+            s = widx[(bh * T + t0) * W + o];
+            w = ww[(bh * T + t0) * W + o];
+        } else {
+            g = occ_base + (size_t)T * W + (size_t)t0 * R + (o - nw);
+            s = ridx[(bh * T + t0) * R + (o - nw)];
+            w = rw[(bh * T + t0) * R + (o - nw)];
+        }
+        const float f = P.fe[g];
+        const int lk = P.lk[g];
+        const bool ok = slot_ok(s, N);
+        P.rs[g] = ok ? (int32_t)((uint32_t)s | (signbit(f) ? 0x80000000u : 0u)) : 0x7fffffff;
+        P.rc[g] = ok ? w * fabsf(f) : 0.f;
+        if (o < nw) {
+            const float e = expf(lam_end - s_lam[o / W]);
+            P.rsc[g] = w * e;
+            P.ra[g] = fabsf(f) * e;
+        }
+        const int pv = lk_prev(lk);
+        if (pv >= 0) hz[atomicAdd(&s_cnt, 1)] = o | (pv << 16);
+    }
+    __syncthreads();
+    for (int i = s_cnt + tid; i < no; i += PLAN_THREADS) hz[i] = -1;
 }
 
 }  // namespace sdm

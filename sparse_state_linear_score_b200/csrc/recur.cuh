@@ -11,9 +11,9 @@
 //   dense    P0_t    = sum_i w_i |fe_i| raw[t,i],  Q0_t = sum_j u_j |fe_j| raw[t,j]
 //            d       = Minv (beta (v - P0))          (in-chunk writes seen by later predictions)
 //            o_t     = Q0_t + sum_tau G[t][tau] d_tau (read after write)
-//   store    the last write of each slot stores e^{lam_end - lam_t} (|fe| raw + A), where
-//            A = sum over the chunk's writes of that slot up to it of w e^{lam_t - lam_tau} d_tau
-//            (its stamp, the chunk-end prefix, is written by the plan).
+//   store    the last write of each slot stores e^{lam_end - lam_t} |fe| raw + sum over the
+//            chunk's writes of that slot up to it of w e^{lam_end - lam_tau} d_tau (both
+//            coefficients from the plan; its stamp, the chunk-end prefix, too).
 //
 // This is the dense-decay recurrence of §2 Background "Gated DeltaNet" restricted to the
 // selected slots (§3 Method "Sparse memory updates", "Sparse retrieval"), evaluated chunk by
@@ -53,8 +53,8 @@ __host__ __device__ inline size_t run_smem_bytes(int C, int W, int R, int CW) {
     b += (size_t)2 * C * (tsw + tsr) * 4;           // rows, two chunks: write blocks, read blocks
     b += (size_t)2 * 2 * C * run_mat_stride(C) * 4; // Minv and G, two chunks
     b += (size_t)4 * C * CW * 4;                    // v, rhs, d, Q0
-    b += (size_t)2 * C * 4;                         // lam, beta
-    b += no * 4 * 4;                                // slot, w, fe, lk
+    b += (size_t)C * 4;                             // beta
+    b += no * 5 * 4;                                // slot, sc, a, lk, hz
     b += (size_t)C * (run_coef_stride(W) + run_coef_stride(R)) * 4;  // coef (padded rows)
     return b;
 }
@@ -65,17 +65,16 @@ constexpr int RUN_OPT = PLAN_MAX_OCC / RUN_THREADS;  // occurrences per thread p
 
 // One chunk's metadata held in registers while the previous chunk computes.
 struct RunPrefetch {
-    int slot[RUN_OPT], lk[RUN_OPT];
-    float w[RUN_OPT], fe[RUN_OPT];
-    float lam, beta, v;
+    int slot[RUN_OPT], lk[RUN_OPT], hz[RUN_OPT];
+    float c[RUN_OPT], sc[RUN_OPT], a[RUN_OPT];
+    float beta, v;
 };
 
 template <int CW, typename VT>
 __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
-    const VT* __restrict__ v, const float* __restrict__ beta, const int32_t* __restrict__ widx,
-    const float* __restrict__ ww, const int32_t* __restrict__ ridx, const float* __restrict__ rw,
-    const float* __restrict__ fe, const int32_t* __restrict__ lk, const float* __restrict__ lam,
-    const float* __restrict__ mats, float* __restrict__ M, const float* __restrict__ M0,
+    const VT* __restrict__ v, const float* __restrict__ beta, const int32_t* __restrict__ rs,
+    const float* __restrict__ rc, const float* __restrict__ rsc, const float* __restrict__ ra,
+    const int32_t* __restrict__ lk, const int32_t* __restrict__ hz, const float* __restrict__ mats, float* __restrict__ M, const float* __restrict__ M0,
     float* __restrict__ out, int H, int T, int N, int d_v, int W, int R, int C, int J) {
     constexpr int Q = CW / 4;
     extern __shared__ __align__(16) unsigned char run_smem[];
@@ -100,14 +99,14 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
     float* s_rhs = s_v + C * CW;
     float* s_d = s_rhs + C * CW;
     float* s_q = s_d + C * CW;
-    float* s_lam = s_q + C * CW;
-    float* s_beta = s_lam + C;
+    float* s_beta = s_q + C * CW;
     int* s_slot = reinterpret_cast<int*>(s_beta + C);
     const int csw = run_coef_stride(W), csr = run_coef_stride(R);
     float* s_coef = reinterpret_cast<float*>(s_slot + nomax);  // [C][W+1], then [C][R+1]
-    float* s_w = s_coef + C * (csw + csr);
-    float* s_fe = s_w + nomax;
-    int* s_lk = reinterpret_cast<int*>(s_fe + nomax);
+    float* s_sc = s_coef + C * (csw + csr);  // writes: store coefficient of the write
+    float* s_a = s_sc + nomax;                // writes: store coefficient of the gathered row
+    int* s_lk = reinterpret_cast<int*>(s_a + nomax);
+    int* s_hz = s_lk + nomax;                 // occurrences whose row the previous chunk stores
 
     const FastDiv fW((unsigned)W), fR((unsigned)R);
     // position of a write occurrence's slice, and of a read occurrence's slice
@@ -127,27 +126,22 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
 #pragma unroll
         for (int k = 0; k < RUN_OPT; ++k) {
             const int o = tid + k * RUN_THREADS;
-            F.slot[k] = -1;
+            F.slot[k] = 0x7fffffff;
             if (o < no) {
-                size_t gi, g;
-                if (o < nw) {
-                    gi = (bh * T + t0) * W + o;
-                    g = occ_base + (size_t)t0 * W + o;
-                    F.slot[k] = widx[gi];
-                    F.w[k] = ww[gi];
-                } else {
-                    gi = (bh * T + t0) * R + (o - nw);
-                    g = occ_base + (size_t)T * W + (size_t)t0 * R + (o - nw);
-                    F.slot[k] = ridx[gi];
-                    F.w[k] = rw[gi];
-                }
-                F.fe[k] = fe[g];
+                const size_t g = o < nw ? occ_base + (size_t)t0 * W + o
+                                        : occ_base + (size_t)T * W + (size_t)t0 * R + (o - nw);
+                F.slot[k] = rs[g];
+                F.c[k] = rc[g];
                 F.lk[k] = lk[g];
+                F.hz[k] = hz[occ_base + (size_t)t0 * (W + R) + o];
+                if (o < nw) {
+                    F.sc[k] = rsc[g];
+                    F.a[k] = ra[g];
+                }
             }
         }
         if (tid < nt) {
             const size_t tg = bh * T + t0 + tid;
-            F.lam = lam[tg];
             F.beta = beta[tg];
         }
         if (tid < nt * CW) F.v = to_f32(v[(bh * T + t0 + tid / CW) * d_v + c0 + tid % CW]);
@@ -160,14 +154,16 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
             const int o = tid + k * RUN_THREADS;
             if (o < no) {
                 s_slot[o] = F.slot[k];
-                s_w[o] = F.w[k];
-                s_fe[o] = F.fe[k];
-                s_coef[cpos(o, nw)] = F.w[k] * fabsf(F.fe[k]);
+                s_coef[cpos(o, nw)] = F.c[k];
                 s_lk[o] = F.lk[k];
+                s_hz[o] = F.hz[k];
+                if (o < nw) {
+                    s_sc[o] = F.sc[k];
+                    s_a[o] = F.a[k];
+                }
             }
         }
         if (tid < nt) {
-            s_lam[tid] = F.lam;
             s_beta[tid] = F.beta;
         }
         if (tid < nt * CW) s_v[tid] = F.v;
@@ -185,14 +181,13 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
 #pragma unroll
             for (int r = 0; r < Q; ++r) {
                 const int src_lane = r * PER + lane / Q;
-                const int s = __shfl_sync(0xffffffffu, F.slot[k], src_lane);
-                const float f = __shfl_sync(0xffffffffu, F.fe[k], src_lane);
+                const int sw = __shfl_sync(0xffffffffu, F.slot[k], src_lane);
                 const int o = wbase + k * RUN_THREADS + src_lane;
                 const int q = lane % Q;
                 if (o < no) {
-                    const bool ok = slot_ok(s, N);
-                    const float* src =
-                        (signbit(f) ? M0h : Mb) + (ok ? (size_t)s * d_v : 0) + c0 + 4 * q;
+                    const int s = sw & 0x7fffffff;
+                    const bool ok = s < N;
+                    const float* src = (sw < 0 ? M0h : Mb) + (ok ? (size_t)s * d_v : 0) + c0 + 4 * q;
                     cp_async16(rbuf + pos(o, nw) + 4 * q, src, ok);
                 }
             }
@@ -225,9 +220,9 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
         // 1. rows the previous chunk stored after they were gathered: take its stored values
         if (j > 0) {
             for (int e = tid; e < no * Q; e += RUN_THREADS) {
-                const int o = e / Q, q = e % Q;
-                const int pv = lk_prev(s_lk[o]);
-                if (pv < 0) continue;
+                const int hv = s_hz[e / Q];
+                if (hv < 0) break;  // end of the chunk's list
+                const int o = hv & 0xffff, pv = hv >> 16, q = e % Q;
                 reinterpret_cast<float4*>(rows + pos(o, nw))[q] =
                     reinterpret_cast<const float4*>(prev_rows + wpos(pv))[q];
             }
@@ -290,19 +285,16 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
             }
             reinterpret_cast<float4*>(out + (bh * T + t0 + t) * d_v + c0)[q] = acc;
         }
-        const float lam_end = s_lam[nt - 1];
         for (int e = tid; e < nw * Q; e += RUN_THREADS) {
             const int o = e / Q, q = e % Q;
             const int lko = s_lk[o];
-            const int s = s_slot[o];
-            if (!(lko & LK_OWNER) || !slot_ok(s, N)) continue;
-            const int t = fW.div(o);
-            const float lt = s_lam[t];
-            // A: this write plus the chunk's earlier writes of the slot, decayed to t
+            const int s = s_slot[o] & 0x7fffffff;
+            if (!(lko & LK_OWNER) || s >= N) continue;
+            // this write plus the chunk's earlier writes of the slot, decayed to the chunk end
             float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int L = o; L >= 0; L = lk_link(s_lk[L])) {
                 const int tp = fW.div(L);
-                const float cfa = s_w[L] * expf(lt - s_lam[tp]);
+                const float cfa = s_sc[L];
                 const float4 dd = reinterpret_cast<const float4*>(s_d + tp * CW)[q];
                 a.x = fmaf(cfa, dd.x, a.x);
                 a.y = fmaf(cfa, dd.y, a.y);
@@ -311,13 +303,12 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
             }
             float4* rp = reinterpret_cast<float4*>(rows + wpos(o)) + q;
             const float4 raw = *rp;
-            const float f = fabsf(s_fe[o]);
-            const float g = expf(lam_end - lt);
+            const float f = s_a[o];
             float4 val;
-            val.x = g * fmaf(f, raw.x, a.x);
-            val.y = g * fmaf(f, raw.y, a.y);
-            val.z = g * fmaf(f, raw.z, a.z);
-            val.w = g * fmaf(f, raw.w, a.w);
+            val.x = fmaf(f, raw.x, a.x);
+            val.y = fmaf(f, raw.y, a.y);
+            val.z = fmaf(f, raw.z, a.z);
+            val.w = fmaf(f, raw.w, a.w);
             reinterpret_cast<float4*>(Mb + (size_t)s * d_v + c0)[q] = val;
             *rp = val;  // the next chunk forwards it
         }

@@ -59,7 +59,8 @@ struct WsLayout {
     int C, J;
     bool lstart_smem;
     size_t walk_smem;
-    size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_mats, off_occw, off_mask, total;
+    size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_mats, off_occw, off_mask;
+    size_t off_rs, off_rc, off_rsc, off_ra, off_hz, total;
     int MW;  // mask words per slot, 0 when the walk is used
 };
 
@@ -88,6 +89,11 @@ WsLayout ws_layout(const sdm_dims* d) {
     const size_t mw = (size_t)(L.J + 63) / 64;
     L.MW = (L.J <= 512 && BH * N * mw * 8 <= kMaskBudget) ? (int)mw : 0;
     L.off_mask = o;   o = up256(o + BH * N * (size_t)L.MW * 8);
+    L.off_rs = o;     o = up256(o + BH * occ * 4);
+    L.off_rc = o;     o = up256(o + BH * occ * 4);
+    L.off_rsc = o;    o = up256(o + BH * occ * 4);
+    L.off_ra = o;     o = up256(o + BH * occ * 4);
+    L.off_hz = o;     o = up256(o + BH * occ * 4);
     L.total = o;
     return L;
 }
@@ -105,6 +111,11 @@ PlanPtrs plan_ptrs(const WsLayout& L, void* ws) {
     P.occw = reinterpret_cast<uint32_t*>(b + L.off_occw);
     P.mask = L.MW ? reinterpret_cast<unsigned long long*>(b + L.off_mask) : nullptr;
     P.MW = L.MW;
+    P.rs = reinterpret_cast<int32_t*>(b + L.off_rs);
+    P.rc = reinterpret_cast<float*>(b + L.off_rc);
+    P.rsc = reinterpret_cast<float*>(b + L.off_rsc);
+    P.ra = reinterpret_cast<float*>(b + L.off_ra);
+    P.hz = reinterpret_cast<int32_t*>(b + L.off_hz);
     return P;
 }
 
@@ -246,9 +257,8 @@ sdm_status launch_run_t(const sdm_dims* d, const WsLayout& L, const PlanPtrs& P,
     if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
     const long long grid = BH_of(d) * (d->d_v / CW);
     kern<<<(unsigned)grid, RUN_THREADS, smem, s>>>(
-        (const VT*)v, beta, widx, ww, ridx, rw, P.fe, P.lk, P.lam, P.mats, st->M, st->M0, out,
-        d->H, d->T,
-        (int)N_of(d), d->d_v, d->W, d->R, L.C, L.J);
+        (const VT*)v, beta, P.rs, P.rc, P.rsc, P.ra, P.lk, P.hz, P.mats, st->M, st->M0, out,
+        d->H, d->T, (int)N_of(d), d->d_v, d->W, d->R, L.C, L.J);
     return launch_status();
 }
 
@@ -396,10 +406,14 @@ sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const floa
     plan_fe_kernel<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, 0, stream>>>(
         st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, P);
     if ((e = launch_status())) return e;
-    if (P.mask) return SDM_OK;  // factors and stamps are final
-    if (!set_smem(plan_walk_kernel, L.walk_smem)) return SDM_ERR_CUDA;
-    plan_walk_kernel<<<dim3(WALK_PARTS, (unsigned)BH), WALK_THREADS, L.walk_smem, stream>>>(
-        st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, L.lstart_smem ? 1 : 0, P);
+    if (!P.mask) {  // the walk finishes the factors and the stamps
+        if (!set_smem(plan_walk_kernel, L.walk_smem)) return SDM_ERR_CUDA;
+        plan_walk_kernel<<<dim3(WALK_PARTS, (unsigned)BH), WALK_THREADS, L.walk_smem, stream>>>(
+            st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, L.lstart_smem ? 1 : 0, P);
+        if ((e = launch_status())) return e;
+    }
+    plan_pack_kernel<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, 0, stream>>>(
+        widx, ww, ridx, rw, dims->T, N, dims->W, dims->R, L.C, P);
     return launch_status();
 }
 
