@@ -22,7 +22,8 @@
 //                   bits 18..29: 1 + the index of the previous chunk's write occurrence
 //                   that stored o's slot at that chunk's end (0: not written there) — the
 //                   row pass gathers a chunk ahead and takes such rows from that store
-//     mats[j]     = Minv [C][C], then G [C][C] (fp32, row t = token, zero beyond the chunk)
+//     mats[j]     = Minv [C][C], then GM = G Minv [C][C] (fp32, row t = token, zero beyond
+//                   the chunk): d = Minv beta (v - P0), o = Q0 + GM beta (v - P0)
 //     st0[o]      = the state's stamp of o's slot at call entry (NaN: pristine)
 //     occw[o]     = o's slot | OCC_OWNER when o stores it
 //   plan_prefix (one CTA per (b,h))
@@ -289,13 +290,21 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
         for (int t = 0; t < PLAN_MAX_C; ++t) s_X[t * PLAN_MAX_C + k] = x[t];
     }
     __syncthreads();
+    // GM = G Minv (lower triangular), so that o = Q0 + GM beta (v - P0) needs no d; into s_L
+    for (int e = tid; e < PLAN_MAX_C * PLAN_MAX_C; e += PLAN_THREADS) {
+        const int t = e / PLAN_MAX_C, tau = e % PLAN_MAX_C;
+        float acc = 0.f;
+        for (int k = tau; k <= t; ++k) acc = fmaf(s_G[t * PLAN_MAX_C + k], s_X[k * PLAN_MAX_C + tau], acc);
+        s_L[e] = acc;
+    }
+    __syncthreads();
     {
         float* mats = P.mats + ((bh * J + j) * 2) * (size_t)(C * C);
         for (int e = tid; e < C * C; e += PLAN_THREADS) {
             const int t = e / C, tau = e % C;
             const bool in = t < nt && tau < nt;
             mats[e] = in ? s_X[t * PLAN_MAX_C + tau] : 0.f;
-            mats[C * C + e] = in ? s_G[t * PLAN_MAX_C + tau] : 0.f;
+            mats[C * C + e] = in ? s_L[t * PLAN_MAX_C + tau] : 0.f;
         }
     }
 

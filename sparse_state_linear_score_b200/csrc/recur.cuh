@@ -11,6 +11,7 @@
 //   dense    P0_t    = sum_i w_i |fe_i| raw[t,i],  Q0_t = sum_j u_j |fe_j| raw[t,j]
 //            d       = Minv (beta (v - P0))          (in-chunk writes seen by later predictions)
 //            o_t     = Q0_t + sum_tau G[t][tau] d_tau (read after write)
+//                    = Q0_t + (GM beta (v - P0))_t    (GM = G Minv from the plan)
 //   store    the last write of each slot stores e^{lam_end - lam_t} |fe| raw + sum over the
 //            chunk's writes of that slot up to it of w e^{lam_end - lam_tau} d_tau (both
 //            coefficients from the plan; its stamp, the chunk-end prefix, too).
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
         float* rows = s_rowbuf + (size_t)(j & 1) * rowbuf;
         float* prev_rows = s_rowbuf + (size_t)((j + 1) & 1) * rowbuf;
         const float* Minv = s_matbuf + (size_t)(j & 1) * matbuf;
-        const float* G = Minv + C * MS;
+        const float* G = Minv + C * MS;  // GM = G Minv
         cp_async_wait_all();
         __syncthreads();
         // 1. rows the previous chunk stored after they were gathered: take its stored values
@@ -256,10 +257,12 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
             else s_q[e] = acc;
         }
         __syncthreads();
-        // 4. d = Minv rhs (Minv is unit lower triangular and zero beyond the chunk)
-        for (int e = tid; e < nt * CW; e += RUN_THREADS) {
+        // 4. d = Minv rhs and o = Q0 + GM rhs (both lower triangular, zero beyond the chunk)
+        for (int task = tid; task < 2 * nt * CW; task += RUN_THREADS) {
+            const bool oo = task >= nt * CW;
+            const int e = oo ? task - nt * CW : task;
             const int t = e / CW, c = e % CW;
-            const float* mr = Minv + t * MS;
+            const float* mr = (oo ? G : Minv) + t * MS;
             float a0 = 0.f, a1 = 0.f;
             int tau = 0;
             for (; tau + 2 <= t + 1; tau += 2) {
@@ -267,24 +270,11 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
                 a1 = fmaf(mr[tau + 1], s_rhs[(tau + 1) * CW + c], a1);
             }
             if (tau <= t) a0 = fmaf(mr[tau], s_rhs[tau * CW + c], a0);
-            s_d[e] = a0 + a1;
+            if (oo) out[(bh * T + t0 + t) * d_v + c0 + c] = s_q[e] + (a0 + a1);
+            else s_d[e] = a0 + a1;
         }
         __syncthreads();
-        // 5. outputs o = Q0 + G d, and the stores of the chunk's last writes
-        for (int e = tid; e < nt * Q; e += RUN_THREADS) {
-            const int t = e / Q, q = e % Q;
-            const float* gr = G + t * MS;
-            float4 acc = reinterpret_cast<const float4*>(s_q + t * CW)[q];
-            for (int tau = 0; tau <= t; ++tau) {
-                const float g = gr[tau];
-                const float4 dd = reinterpret_cast<const float4*>(s_d + tau * CW)[q];
-                acc.x = fmaf(g, dd.x, acc.x);
-                acc.y = fmaf(g, dd.y, acc.y);
-                acc.z = fmaf(g, dd.z, acc.z);
-                acc.w = fmaf(g, dd.w, acc.w);
-            }
-            reinterpret_cast<float4*>(out + (bh * T + t0 + t) * d_v + c0)[q] = acc;
-        }
+        // 5. the stores of the chunk's last writes
         for (int e = tid; e < nw * Q; e += RUN_THREADS) {
             const int o = e / Q, q = e % Q;
             const int lko = s_lk[o];
