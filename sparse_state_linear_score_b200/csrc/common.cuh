@@ -36,6 +36,11 @@ SDM_DEV void cp_async16(void* smem_dst, const void* gmem_src, bool pred) {
                  "r"(n)
                  : "memory");
 }
+// 8-byte copy (through L1; the 16-byte form bypasses it).
+SDM_DEV void cp_async8(void* smem_dst, const void* gmem_src) {
+    unsigned dst = (unsigned)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(dst), "l"(gmem_src) : "memory");
+}
 SDM_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 SDM_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 

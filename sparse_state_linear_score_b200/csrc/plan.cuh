@@ -38,7 +38,7 @@
 //     carries the stamp of that chunk's end); the state stamps of the slots written in the
 //     call are updated.
 //   plan_pack (one CTA per chunk)
-//     rs, rc, rsc, ra, hz: what the row pass reads per occurrence (see PlanPtrs).
+//     rs and the chunk image: what the row pass reads (see PlanPtrs, RunImg).
 //
 // In-chunk occurrence order: the nt*W write occurrences (token-major), then the nt*R
 // read occurrences.  In the per-(b,h) arrays fe / lk / st0 the T*W write entries come
@@ -112,14 +112,40 @@ struct PlanPtrs {
     uint32_t* occw;    // [BH][T*(W+R)] slot | OCC_OWNER (the walk's input)
     unsigned long long* mask;  // [BH][N][MW] chunks of this call that stored each slot, or null
     int MW;                    // 64-bit words per slot in mask
-    // the row pass's inputs, packed by plan_pack (same occurrence layout as fe / lk)
-    int32_t* rs;       // slot | bit 31 when the row gathered is the pristine M0 row
-    float* rc;         // w |fe|: the coefficient of the gathered row in p_t / o_t
-    float* rsc;        // writes: w e^{lam_end - lam_t} (the write's share of its slot's store)
-    float* ra;         // writes: |fe| e^{lam_end - lam_t} (the gathered row's share)
-    int32_t* hz;       // [BH][T*(W+R)], chunk j at j*C*(W+R): o | prev << 16 for the chunk's
-                       // occurrences whose row the previous chunk stores, then -1
+    // the row pass's inputs, packed by plan_pack
+    int32_t* rs;          // [BH][T*(W+R)] chunk j at j*C*(W+R), in-chunk occurrence order:
+                          // slot | bit 31 when the row gathered is the pristine M0 row
+    unsigned char* img;   // [BH][J][img bytes]: per-chunk image (RunImg)
 };
+
+// Per-chunk image of the row pass's column-independent inputs, written by plan_pack and
+// copied as is into the row pass's shared memory (16-byte aligned sections, byte offsets):
+//   coef  [C][W+1] then [C][R+1]: w |fe| of token t's i-th write (read) occurrence (the
+//         padded rows keep the tokens a warp reads at once in different banks)
+//   hz    [C*(W+R)]: o | prev << 16 for the occurrences whose row the previous chunk stores
+//         (prev: that chunk's write occurrence), then -1
+//   wslot [C*W]: slot of each write occurrence (0x7fffffff when out of range)
+//   wlk   [C*W]: its link word (LK_OWNER, in-chunk link)
+//   sc    [C*W]: w e^{lam_end - lam_t}: the write's share of its slot's chunk-end value
+//   a     [C*W]: |fe| e^{lam_end - lam_t}: the gathered row's share (owners)
+//   beta  [C]
+struct RunImg {
+    int coef, hz, wslot, wlk, sc, a, beta, bytes;
+};
+__host__ __device__ inline int up16i(int x) { return (x + 15) & ~15; }
+__host__ __device__ inline RunImg run_img(int C, int W, int R) {
+    RunImg m;
+    int o = 0;
+    m.coef = o;  o += up16i(C * (W + R + 2) * 4);
+    m.hz = o;    o += up16i(C * (W + R) * 4);
+    m.wslot = o; o += up16i(C * W * 4);
+    m.wlk = o;   o += up16i(C * W * 4);
+    m.sc = o;    o += up16i(C * W * 4);
+    m.a = o;     o += up16i(C * W * 4);
+    m.beta = o;  o += up16i(C * 4);
+    m.bytes = o;
+    return m;
+}
 
 __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
     const float* __restrict__ alpha, const float* __restrict__ beta,
@@ -510,13 +536,13 @@ __global__ void __launch_bounds__(WALK_THREADS) plan_walk_kernel(
     }
 }
 
-// The row pass's per-occurrence inputs from the final decay factors: slot and pristine flag,
-// the gathered row's coefficient, the store coefficients of the writes, and the chunk's list
-// of occurrences whose row the previous chunk stores (order within the list is free).
+// The row pass's inputs from the final decay factors: the gather words (slot, pristine flag)
+// and the chunk image (coefficients, store factors, links, the list of occurrences whose row
+// the previous chunk stores — in any order — and beta).
 __global__ void __launch_bounds__(PLAN_THREADS) plan_pack_kernel(
-    const int32_t* __restrict__ widx, const float* __restrict__ ww,
-    const int32_t* __restrict__ ridx, const float* __restrict__ rw, int T, int N, int W, int R,
-    int C, PlanPtrs P) {
+    const float* __restrict__ beta, const int32_t* __restrict__ widx,
+    const float* __restrict__ ww, const int32_t* __restrict__ ridx,
+    const float* __restrict__ rw, int T, int N, int W, int R, int C, int J, PlanPtrs P) {
     __shared__ float s_lam[PLAN_MAX_C];
     __shared__ int s_cnt;
     const int j = blockIdx.x;
@@ -524,39 +550,57 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_pack_kernel(
     const int tid = threadIdx.x;
     const int t0 = j * C, nt = min(C, T - t0), nw = nt * W, no = nt * (W + R);
     const size_t occ_base = bh * (size_t)T * (W + R);
-    int32_t* hz = P.hz + occ_base + (size_t)t0 * (W + R);
+    const RunImg m = run_img(C, W, R);
+    unsigned char* img = P.img + (bh * J + j) * (size_t)m.bytes;
+    float* coef = reinterpret_cast<float*>(img + m.coef);
+    int32_t* hz = reinterpret_cast<int32_t*>(img + m.hz);
+    int32_t* wslot = reinterpret_cast<int32_t*>(img + m.wslot);
+    int32_t* wlk = reinterpret_cast<int32_t*>(img + m.wlk);
+    float* sc = reinterpret_cast<float*>(img + m.sc);
+    float* sa = reinterpret_cast<float*>(img + m.a);
+    float* bt = reinterpret_cast<float*>(img + m.beta);
+    int32_t* rs = P.rs + occ_base + (size_t)t0 * (W + R);
     if (tid == 0) s_cnt = 0;
-    if (tid < nt) s_lam[tid] = P.lam[bh * T + t0 + tid];
+    if (tid < nt) {
+        s_lam[tid] = P.lam[bh * T + t0 + tid];
+        bt[tid] = beta[bh * T + t0 + tid];
+    }
     __syncthreads();
     const float lam_end = s_lam[nt - 1];
     for (int o = tid; o < no; o += PLAN_THREADS) {
         size_t g;
-        int s;
+        int s, ci;
         float w;
         if (o < nw) {
+            const int t = o / W;
             g = occ_base + (size_t)t0 * W + o;
             s = widx[(bh * T + t0) * W + o];
             w = ww[(bh * T + t0) * W + o];
+            ci = t * (W + 1) + (o - t * W);
         } else {
-            g = occ_base + (size_t)T * W + (size_t)t0 * R + (o - nw);
-            s = ridx[(bh * T + t0) * R + (o - nw)];
-            w = rw[(bh * T + t0) * R + (o - nw)];
+            const int r = o - nw, t = r / R;
+            g = occ_base + (size_t)T * W + (size_t)t0 * R + r;
+            s = ridx[(bh * T + t0) * R + r];
+            w = rw[(bh * T + t0) * R + r];
+            ci = C * (W + 1) + t * (R + 1) + (r - t * R);
         }
         const float f = P.fe[g];
         const int lk = P.lk[g];
         const bool ok = slot_ok(s, N);
-        P.rs[g] = ok ? (int32_t)((uint32_t)s | (signbit(f) ? 0x80000000u : 0u)) : 0x7fffffff;
-        P.rc[g] = ok ? w * fabsf(f) : 0.f;
+        rs[o] = ok ? (int32_t)((uint32_t)s | (signbit(f) ? 0x80000000u : 0u)) : 0x7fffffff;
+        coef[ci] = ok ? w * fabsf(f) : 0.f;
         if (o < nw) {
             const float e = expf(lam_end - s_lam[o / W]);
-            P.rsc[g] = w * e;
-            P.ra[g] = fabsf(f) * e;
+            wslot[o] = ok ? s : 0x7fffffff;
+            wlk[o] = lk;
+            sc[o] = w * e;
+            sa[o] = fabsf(f) * e;
         }
         const int pv = lk_prev(lk);
         if (pv >= 0) hz[atomicAdd(&s_cnt, 1)] = o | (pv << 16);
     }
     __syncthreads();
-    for (int i = s_cnt + tid; i < no; i += PLAN_THREADS) hz[i] = -1;
+    for (int i = s_cnt + tid; i < C * (W + R); i += PLAN_THREADS) hz[i] = -1;
 }
 
 }  // namespace sdm

@@ -49,9 +49,8 @@ int chunk_tokens(const sdm_dims* d) {
     const int CW = col_width(d);
     int C = PLAN_MAX_OCC / (d->W + d->R);
     if (C > PLAN_MAX_C) C = PLAN_MAX_C;
-    if (C > RUN_THREADS / CW) C = RUN_THREADS / CW;  // one value per thread in the prefetch
     C &= ~3;  // matrices move in 16-byte rows
-    while (C > 4 && run_smem_bytes(C, d->W, d->R, CW) > kSmemBudget) C -= 4;
+    while (C > 4 && run_smem_bytes(C, d->W, d->R, CW, 4) > kSmemBudget) C -= 4;
     return C < 4 ? 4 : C;
 }
 
@@ -60,7 +59,7 @@ struct WsLayout {
     bool lstart_smem;
     size_t walk_smem;
     size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_mats, off_occw, off_mask;
-    size_t off_rs, off_rc, off_rsc, off_ra, off_hz, total;
+    size_t off_rs, off_img, total;
     int MW;  // mask words per slot, 0 when the walk is used
 };
 
@@ -90,10 +89,7 @@ WsLayout ws_layout(const sdm_dims* d) {
     L.MW = (L.J <= 512 && BH * N * mw * 8 <= kMaskBudget) ? (int)mw : 0;
     L.off_mask = o;   o = up256(o + BH * N * (size_t)L.MW * 8);
     L.off_rs = o;     o = up256(o + BH * occ * 4);
-    L.off_rc = o;     o = up256(o + BH * occ * 4);
-    L.off_rsc = o;    o = up256(o + BH * occ * 4);
-    L.off_ra = o;     o = up256(o + BH * occ * 4);
-    L.off_hz = o;     o = up256(o + BH * occ * 4);
+    L.off_img = o;    o = up256(o + BH * (size_t)L.J * run_img(L.C, d->W, d->R).bytes);
     L.total = o;
     return L;
 }
@@ -112,10 +108,7 @@ PlanPtrs plan_ptrs(const WsLayout& L, void* ws) {
     P.mask = L.MW ? reinterpret_cast<unsigned long long*>(b + L.off_mask) : nullptr;
     P.MW = L.MW;
     P.rs = reinterpret_cast<int32_t*>(b + L.off_rs);
-    P.rc = reinterpret_cast<float*>(b + L.off_rc);
-    P.rsc = reinterpret_cast<float*>(b + L.off_rsc);
-    P.ra = reinterpret_cast<float*>(b + L.off_ra);
-    P.hz = reinterpret_cast<int32_t*>(b + L.off_hz);
+    P.img = b + L.off_img;
     return P;
 }
 
@@ -252,13 +245,13 @@ sdm_status launch_run_t(const sdm_dims* d, const WsLayout& L, const PlanPtrs& P,
                         const float* beta, const int32_t* widx, const float* ww,
                         const int32_t* ridx, const float* rw, const sdm_state* st, float* out,
                         cudaStream_t s) {
-    const size_t smem = run_smem_bytes(L.C, d->W, d->R, CW);
+    const size_t smem = run_smem_bytes(L.C, d->W, d->R, CW, (int)sizeof(VT));
     auto kern = recur_run_kernel<CW, VT>;
     if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
     const long long grid = BH_of(d) * (d->d_v / CW);
     kern<<<(unsigned)grid, RUN_THREADS, smem, s>>>(
-        (const VT*)v, beta, P.rs, P.rc, P.rsc, P.ra, P.lk, P.hz, P.mats, st->M, st->M0, out,
-        d->H, d->T, (int)N_of(d), d->d_v, d->W, d->R, L.C, L.J);
+        (const VT*)v, P.rs, P.img, P.mats, st->M, st->M0, out, d->H, d->T, (int)N_of(d), d->d_v,
+        d->W, d->R, L.C, L.J);
     return launch_status();
 }
 
@@ -413,7 +406,7 @@ sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const floa
         if ((e = launch_status())) return e;
     }
     plan_pack_kernel<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, 0, stream>>>(
-        widx, ww, ridx, rw, dims->T, N, dims->W, dims->R, L.C, P);
+        beta, widx, ww, ridx, rw, dims->T, N, dims->W, dims->R, L.C, L.J, P);
     return launch_status();
 }
 
