@@ -22,8 +22,8 @@
 //                   bits 18..29: 1 + the index of the previous chunk's write occurrence
 //                   that stored o's slot at that chunk's end (0: not written there) — the
 //                   row pass gathers a chunk ahead and takes such rows from that store
-//     mats[j]     = Minv [C][C], then GM = G Minv [C][C] (fp32, row t = token, zero beyond
-//                   the chunk): d = Minv beta (v - P0), o = Q0 + GM beta (v - P0)
+//     Minv, GM    = Minv and GM = G Minv (fp32 [C][C+4] rows, row t = token, zero beyond the
+//                   chunk), into the chunk image: d = Minv beta (v - P0), o = Q0 + GM beta (v - P0)
 //     st0[o]      = the state's stamp of o's slot at call entry (NaN: pristine)
 //     occw[o]     = o's slot | OCC_OWNER when o stores it
 //   plan_prefix (one CTA per (b,h))
@@ -108,7 +108,6 @@ struct PlanPtrs {
     double* st0;       // [BH][T*(W+R)]
     float* fe;         // [BH][T*(W+R)]
     int32_t* lk;       // [BH][T*(W+R)]
-    float* mats;       // [BH][J][2][C][C]
     uint32_t* occw;    // [BH][T*(W+R)] slot | OCC_OWNER (the walk's input)
     unsigned long long* mask;  // [BH][N][MW] chunks of this call that stored each slot, or null
     int MW;                    // 64-bit words per slot in mask
@@ -129,8 +128,10 @@ struct PlanPtrs {
 //   sc    [C*W]: w e^{lam_end - lam_t}: the write's share of its slot's chunk-end value
 //   a     [C*W]: |fe| e^{lam_end - lam_t}: the gathered row's share (owners)
 //   beta  [C]
+//   minv, gm [C][C+4]: Minv and GM = G Minv (rows padded to C+4 floats: 16-byte rows whose
+//         starts fall 4 banks apart)
 struct RunImg {
-    int coef, hz, wslot, wlk, sc, a, beta, bytes;
+    int coef, hz, wslot, wlk, sc, a, beta, minv, gm, bytes;
 };
 __host__ __device__ inline int up16i(int x) { return (x + 15) & ~15; }
 __host__ __device__ inline RunImg run_img(int C, int W, int R) {
@@ -143,6 +144,8 @@ __host__ __device__ inline RunImg run_img(int C, int W, int R) {
     m.sc = o;    o += up16i(C * W * 4);
     m.a = o;     o += up16i(C * W * 4);
     m.beta = o;  o += up16i(C * 4);
+    m.minv = o;  o += C * (C + 4) * 4;
+    m.gm = o;    o += C * (C + 4) * 4;
     m.bytes = o;
     return m;
 }
@@ -325,12 +328,16 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
     }
     __syncthreads();
     {
-        float* mats = P.mats + ((bh * J + j) * 2) * (size_t)(C * C);
-        for (int e = tid; e < C * C; e += PLAN_THREADS) {
-            const int t = e / C, tau = e % C;
+        const RunImg m = run_img(C, W, R);
+        unsigned char* img = P.img + (bh * J + j) * (size_t)m.bytes;
+        float* minv = reinterpret_cast<float*>(img + m.minv);
+        float* gm = reinterpret_cast<float*>(img + m.gm);
+        const int MS = C + 4;
+        for (int e = tid; e < C * MS; e += PLAN_THREADS) {
+            const int t = e / MS, tau = e % MS;
             const bool in = t < nt && tau < nt;
-            mats[e] = in ? s_X[t * PLAN_MAX_C + tau] : 0.f;
-            mats[C * C + e] = in ? s_L[t * PLAN_MAX_C + tau] : 0.f;
+            minv[e] = in ? s_X[t * PLAN_MAX_C + tau] : 0.f;
+            gm[e] = in ? s_L[t * PLAN_MAX_C + tau] : 0.f;
         }
     }
 

@@ -23,9 +23,10 @@
 //
 // Warp roles.  Warps 0..3 (producers) only move data: while the consumers compute chunk j
 // they gather chunk j+1's rows into the other row buffer (cp.async, 16-byte pieces, the Q
-// pieces of a slice fetched by adjacent lanes of one instruction), copy its image, matrices
-// and values into the other halves of the double buffers, and load chunk j+2's gather words
-// into registers.  Warps 4..15 (consumers) compute.  Named barriers hand the buffers over:
+// pieces of a slice fetched by adjacent lanes of one instruction), copy its image (one bulk
+// copy on an mbarrier) and values into the other halves of the double buffers, and load
+// chunk j+2's gather words into registers.  Warps 4..15 (consumers) compute.  Named barriers
+// hand the buffers over:
 //   BAR_READY  producers arrive when chunk j+1's inputs have landed; consumers wait on it
 //   BAR_FIXED  consumers arrive when chunk j's forwarded rows are taken from the other row
 //              buffer; producers wait on it before gathering into that buffer
@@ -36,6 +37,7 @@
 
 #include "common.cuh"
 #include "plan.cuh"
+#include "tc_ptx.cuh"
 
 namespace sdm {
 
@@ -55,7 +57,7 @@ SDM_DEV void named_arrive(int id, int count) {
 
 // Floats per token block of gathered rows: its slots' CW-wide slices + padding.
 __host__ __device__ inline int run_tok_stride(int per_tok, int CW) { return per_tok * CW + RUN_PAD; }
-// Row stride of Minv / GM in shared memory (16-byte rows, 4 floats apart in banks).
+// Row stride of Minv / GM in the chunk image (16-byte rows, 4 floats apart in banks).
 __host__ __device__ inline int run_mat_stride(int C) { return C + 4; }
 
 // x / d for 0 <= x < 2^16 and 1 <= d <= 64 as one multiply-high: with m = ceil(2^32 / d),
@@ -68,8 +70,8 @@ struct FastDiv {
 };
 
 // Shared memory of the row pass (bytes), in this order: rows [2][C*(tsw+tsr)] floats,
-// mats [2][2][C][MS] floats, images [2][img bytes], values [2][C*CW] of VT (16-byte padded),
-// rhs, d, Q0 [C*CW] floats each.
+// images [2][img bytes], values [2][C*CW] of VT (16-byte padded), rhs, d, Q0 [C*CW] floats
+// each, the image copies' mbarrier.
 __host__ __device__ inline int run_vst_bytes(int C, int CW, int vbytes) {
     return up16i(C * CW * vbytes);
 }
@@ -77,19 +79,18 @@ __host__ __device__ inline size_t run_smem_bytes(int C, int W, int R, int CW, in
     const size_t tsw = (size_t)run_tok_stride(W, CW), tsr = (size_t)run_tok_stride(R, CW);
     size_t b = 0;
     b += (size_t)2 * C * (tsw + tsr) * 4;            // rows, two chunks
-    b += (size_t)2 * 2 * C * run_mat_stride(C) * 4; // Minv and GM, two chunks
     b += (size_t)2 * run_img(C, W, R).bytes;         // chunk images, two chunks
     b += (size_t)2 * run_vst_bytes(C, CW, vbytes);   // values, two chunks
     b += (size_t)3 * C * CW * 4;                     // rhs, d, Q0
+    b += 16;                                         // mbarrier
     return b;
 }
 
 template <int CW, typename VT>
 __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
     const VT* __restrict__ v, const int32_t* __restrict__ rs,
-    const unsigned char* __restrict__ imgs, const float* __restrict__ mats,
-    float* __restrict__ M, const float* __restrict__ M0, float* __restrict__ out, int H, int T,
-    int N, int d_v, int W, int R, int C, int J) {
+    const unsigned char* __restrict__ imgs, float* __restrict__ M, const float* __restrict__ M0,
+    float* __restrict__ out, int H, int T, int N, int d_v, int W, int R, int C, int J) {
     constexpr int Q = CW / 4;
     extern __shared__ __align__(16) unsigned char run_smem[];
     const int ncb = d_v / CW;
@@ -107,14 +108,19 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
 
     float* s_rowbuf = reinterpret_cast<float*>(run_smem);  // [2][C*(tsw+tsr)]
     const int rowbuf = C * (tsw + tsr);
-    float* s_matbuf = s_rowbuf + 2 * (size_t)rowbuf;       // [2][2][C][MS]
-    const int matbuf = 2 * C * MS;
-    unsigned char* s_imgbuf = reinterpret_cast<unsigned char*>(s_matbuf + 2 * (size_t)matbuf);
+    unsigned char* s_imgbuf = reinterpret_cast<unsigned char*>(s_rowbuf + 2 * (size_t)rowbuf);
     unsigned char* s_vbuf = s_imgbuf + 2 * (size_t)im.bytes;
     const int vst = run_vst_bytes(C, CW, (int)sizeof(VT));
     float* s_rhs = reinterpret_cast<float*>(s_vbuf + 2 * (size_t)vst);
     float* s_d = s_rhs + C * CW;
     float* s_q = s_d + C * CW;
+    uint64_t* bar_img = reinterpret_cast<uint64_t*>(s_q + C * CW);
+
+    if (tid == 0) {
+        ptx::mbar_init(bar_img, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
 
     const FastDiv fW((unsigned)W), fR((unsigned)R);
     // position of a write occurrence's slice, and of a read occurrence's slice
@@ -158,17 +164,13 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
                     }
                 }
             }
-            // image
-            const unsigned char* isrc = imgs + (bh * J + jn) * (size_t)im.bytes;
-            unsigned char* idst = s_imgbuf + (size_t)(jn & 1) * im.bytes;
-            for (int e = tid; e < im.bytes / 16; e += RUN_PRODUCERS)
-                cp_async16(idst + 16 * e, isrc + 16 * e, true);
-            // Minv and GM (16-byte row pieces into padded rows)
-            const float* msrc = mats + ((bh * J + jn) * 2) * (size_t)(C * C);
-            float* mdst = s_matbuf + (size_t)(jn & 1) * matbuf;
-            for (int e = tid; e < 2 * C * (C / 4); e += RUN_PRODUCERS) {
-                const int row = e / (C / 4), piece = e % (C / 4);
-                cp_async16(mdst + row * MS + 4 * piece, msrc + row * C + 4 * piece, true);
+            // image (with Minv and GM): one bulk copy.  The consumers' reads of this buffer
+            // (chunk jn-2) precede it through BAR_FIXED.
+            if (tid == 0) {
+                ptx::fence_proxy_async_smem();
+                ptx::mbar_arrive_expect_tx(bar_img, (uint32_t)im.bytes);
+                ptx::bulk_load(s_imgbuf + (size_t)(jn & 1) * im.bytes,
+                               imgs + (bh * J + jn) * (size_t)im.bytes, (uint32_t)im.bytes, bar_img);
             }
             // values: nt rows of CW elements, in 16-byte (or, for 8-byte rows, 8-byte) pieces
             constexpr int VROW = CW * (int)sizeof(VT);
@@ -186,10 +188,18 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
             cp_async_commit();
         };
 
+        // chunk jn's copies have landed (the image's wait is bounded: past the deadline the
+        // device error word records it and the pass goes on, so no barrier is left waiting)
+        auto landed = [&](int jn) {
+            cp_async_wait_all();
+            const uint64_t deadline = ptx::globaltimer_ns() + 2000000000ull;
+            if (!ptx::mbar_wait_bounded(bar_img, (uint32_t)(jn & 1), deadline) && tid == 0)
+                raise_err(SDM_DEVERR_TIMEOUT);
+        };
         load_words(0);
         stage(0);
         if (J > 1) load_words(1);
-        cp_async_wait_all();
+        landed(0);
         named_arrive(BAR_READY, RUN_THREADS);
         for (int j = 0; j < J; ++j) {
             // the consumers have taken chunk j's forwarded rows: the other buffers are free
@@ -197,7 +207,7 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
             if (j + 1 < J) {
                 stage(j + 1);
                 if (j + 2 < J) load_words(j + 2);
-                cp_async_wait_all();
+                landed(j + 1);
                 named_arrive(BAR_READY, RUN_THREADS);
             }
         }
@@ -212,9 +222,9 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
         const int nw = nt * W, no = nt * (W + R);
         float* rows = s_rowbuf + (size_t)(j & 1) * rowbuf;
         const float* prev_rows = s_rowbuf + (size_t)((j + 1) & 1) * rowbuf;
-        const float* Minv = s_matbuf + (size_t)(j & 1) * matbuf;
-        const float* GM = Minv + C * MS;
         const unsigned char* img = s_imgbuf + (size_t)(j & 1) * im.bytes;
+        const float* Minv = reinterpret_cast<const float*>(img + im.minv);
+        const float* GM = reinterpret_cast<const float*>(img + im.gm);
         const float* s_coef = reinterpret_cast<const float*>(img + im.coef);
         const int* s_hz = reinterpret_cast<const int*>(img + im.hz);
         const int* s_wslot = reinterpret_cast<const int*>(img + im.wslot);

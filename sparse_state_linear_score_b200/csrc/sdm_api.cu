@@ -58,7 +58,7 @@ struct WsLayout {
     int C, J;
     bool lstart_smem;
     size_t walk_smem;
-    size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_mats, off_occw, off_mask;
+    size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_occw, off_mask;
     size_t off_rs, off_img, total;
     int MW;  // mask words per slot, 0 when the walk is used
 };
@@ -82,7 +82,6 @@ WsLayout ws_layout(const sdm_dims* d) {
     L.off_st0 = o;    o = up256(o + BH * occ * 8);
     L.off_fe = o;     o = up256(o + BH * occ * 4);
     L.off_lk = o;     o = up256(o + BH * occ * 4);
-    L.off_mats = o;   o = up256(o + BH * (size_t)L.J * 2 * L.C * L.C * 4);
     L.off_occw = o;   o = up256(o + BH * occ * 4);
     // per-slot chunk masks replace the sequential walk when they stay small
     const size_t mw = (size_t)(L.J + 63) / 64;
@@ -103,7 +102,6 @@ PlanPtrs plan_ptrs(const WsLayout& L, void* ws) {
     P.st0 = reinterpret_cast<double*>(b + L.off_st0);
     P.fe = reinterpret_cast<float*>(b + L.off_fe);
     P.lk = reinterpret_cast<int32_t*>(b + L.off_lk);
-    P.mats = reinterpret_cast<float*>(b + L.off_mats);
     P.occw = reinterpret_cast<uint32_t*>(b + L.off_occw);
     P.mask = L.MW ? reinterpret_cast<unsigned long long*>(b + L.off_mask) : nullptr;
     P.MW = L.MW;
@@ -250,7 +248,7 @@ sdm_status launch_run_t(const sdm_dims* d, const WsLayout& L, const PlanPtrs& P,
     if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
     const long long grid = BH_of(d) * (d->d_v / CW);
     kern<<<(unsigned)grid, RUN_THREADS, smem, s>>>(
-        (const VT*)v, P.rs, P.img, P.mats, st->M, st->M0, out, d->H, d->T, (int)N_of(d), d->d_v,
+        (const VT*)v, P.rs, P.img, st->M, st->M0, out, d->H, d->T, (int)N_of(d), d->d_v,
         d->W, d->R, L.C, L.J);
     return launch_status();
 }

@@ -71,6 +71,16 @@ SDM_DEV void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int 
         : "memory");
 }
 
+// Contiguous global -> shared copy of `bytes` (a multiple of 16, both addresses 16-byte
+// aligned) by the bulk-copy engine, completing on bar.
+SDM_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand stored with the 128-byte swizzle
 // (rows of 64 bf16 = 128 B, 8-row groups 1024 B apart; tile base 1024-byte aligned).
 SDM_DEV uint64_t umma_desc_kmajor_sw128(const void* tile) {
