@@ -248,48 +248,87 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
         named_arrive(BAR_FIXED, RUN_THREADS);
         named_sync(BAR_CONS, RUN_CONSUMERS);
 
-        // 2. predictions (writes) and reads from the chunk-start memory
-        for (int task = ctid; task < 2 * nt * CW; task += RUN_CONSUMERS) {
-            const bool rd = task >= nt * CW;
-            const int e = rd ? task - nt * CW : task;
-            const int t = e / CW, c = e % CW;
-            // four independent partial sums per dot product (latency of the smem loads)
+        // 2. predictions (writes) and reads from the chunk-start memory; a task is two
+        //    adjacent columns of one token
+        constexpr int CP = CW / 2;
+        for (int task = ctid; task < 2 * nt * CP; task += RUN_CONSUMERS) {
+            const bool rd = task >= nt * CP;
+            const int e = rd ? task - nt * CP : task;
+            const int t = e / CP, c = 2 * (e % CP);
+            // four independent partial sums per column (latency of the smem loads)
             const float* rr = rd ? rows + C * tsw + t * tsr + c : rows + t * tsw + c;
             const float* cf = rd ? s_coef + C * csw + t * csr : s_coef + t * csw;
             const int n_i = rd ? R : W;
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
             int i = 0;
             for (; i + 4 <= n_i; i += 4) {
-                a0 = fmaf(cf[i], rr[i * CW], a0);
-                a1 = fmaf(cf[i + 1], rr[(i + 1) * CW], a1);
-                a2 = fmaf(cf[i + 2], rr[(i + 2) * CW], a2);
-                a3 = fmaf(cf[i + 3], rr[(i + 3) * CW], a3);
+                const float2 r0 = *reinterpret_cast<const float2*>(rr + i * CW);
+                const float2 r1 = *reinterpret_cast<const float2*>(rr + (i + 1) * CW);
+                const float2 r2 = *reinterpret_cast<const float2*>(rr + (i + 2) * CW);
+                const float2 r3 = *reinterpret_cast<const float2*>(rr + (i + 3) * CW);
+                a0.x = fmaf(cf[i], r0.x, a0.x);
+                a0.y = fmaf(cf[i], r0.y, a0.y);
+                a1.x = fmaf(cf[i + 1], r1.x, a1.x);
+                a1.y = fmaf(cf[i + 1], r1.y, a1.y);
+                a2.x = fmaf(cf[i + 2], r2.x, a2.x);
+                a2.y = fmaf(cf[i + 2], r2.y, a2.y);
+                a3.x = fmaf(cf[i + 3], r3.x, a3.x);
+                a3.y = fmaf(cf[i + 3], r3.y, a3.y);
             }
-            for (; i < n_i; ++i) a0 = fmaf(cf[i], rr[i * CW], a0);
-            const float acc = (a0 + a1) + (a2 + a3);
-            if (!rd) s_rhs[e] = s_beta[t] * (to_f32(s_v[e]) - acc);
-            else s_q[e] = acc;
+            for (; i < n_i; ++i) {
+                const float2 r0 = *reinterpret_cast<const float2*>(rr + i * CW);
+                a0.x = fmaf(cf[i], r0.x, a0.x);
+                a0.y = fmaf(cf[i], r0.y, a0.y);
+            }
+            const float accx = (a0.x + a1.x) + (a2.x + a3.x);
+            const float accy = (a0.y + a1.y) + (a2.y + a3.y);
+            const int ev = t * CW + c;
+            if (!rd) {
+                const float b = s_beta[t];
+                s_rhs[ev] = b * (to_f32(s_v[ev]) - accx);
+                s_rhs[ev + 1] = b * (to_f32(s_v[ev + 1]) - accy);
+            } else {
+                *reinterpret_cast<float2*>(s_q + ev) = make_float2(accx, accy);
+            }
         }
         named_sync(BAR_CONS, RUN_CONSUMERS);
-        // 3. d = Minv rhs and o = Q0 + GM rhs (both lower triangular, zero beyond the chunk)
-        for (int task = ctid; task < 2 * nt * CW; task += RUN_CONSUMERS) {
-            const bool oo = task >= nt * CW;
-            const int e = oo ? task - nt * CW : task;
-            const int t = e / CW, c = e % CW;
+        // 3. d = Minv rhs and o = Q0 + GM rhs (both lower triangular, zero beyond the chunk);
+        //    a task is two adjacent columns of one token
+        for (int task = ctid; task < 2 * nt * CP; task += RUN_CONSUMERS) {
+            const bool oo = task >= nt * CP;
+            const int e = oo ? task - nt * CP : task;
+            const int t = e / CP, c = 2 * (e % CP);
             const float* mr = (oo ? GM : Minv) + t * MS;
-            float a0 = 0.f, a1 = 0.f;
+            float2 a0 = make_float2(0.f, 0.f), a1 = a0;
             int tau = 0;
             for (; tau + 2 <= t + 1; tau += 2) {
-                a0 = fmaf(mr[tau], s_rhs[tau * CW + c], a0);
-                a1 = fmaf(mr[tau + 1], s_rhs[(tau + 1) * CW + c], a1);
+                const float2 r0 = *reinterpret_cast<const float2*>(s_rhs + tau * CW + c);
+                const float2 r1 = *reinterpret_cast<const float2*>(s_rhs + (tau + 1) * CW + c);
+                a0.x = fmaf(mr[tau], r0.x, a0.x);
+                a0.y = fmaf(mr[tau], r0.y, a0.y);
+                a1.x = fmaf(mr[tau + 1], r1.x, a1.x);
+                a1.y = fmaf(mr[tau + 1], r1.y, a1.y);
             }
-            if (tau <= t) a0 = fmaf(mr[tau], s_rhs[tau * CW + c], a0);
-            if (oo) out[(bh * T + t0 + t) * d_v + c0 + c] = s_q[e] + (a0 + a1);
-            else s_d[e] = a0 + a1;
+            if (tau <= t) {
+                const float2 r0 = *reinterpret_cast<const float2*>(s_rhs + tau * CW + c);
+                a0.x = fmaf(mr[tau], r0.x, a0.x);
+                a0.y = fmaf(mr[tau], r0.y, a0.y);
+            }
+            const int ev = t * CW + c;
+            const float2 r = make_float2(a0.x + a1.x, a0.y + a1.y);
+            if (oo) {
+                const float2 q = *reinterpret_cast<const float2*>(s_q + ev);
+                *reinterpret_cast<float2*>(out + (bh * T + t0 + t) * d_v + c0 + c) =
+                    make_float2(q.x + r.x, q.y + r.y);
+            } else {
+                *reinterpret_cast<float2*>(s_d + ev) = r;
+            }
         }
         named_sync(BAR_CONS, RUN_CONSUMERS);
         // 4. the stores of the chunk's last writes (also written back to the rows, from where
         //    the next chunk takes the ones it gathered before they were stored)
+        //    The Q 16-byte pieces of a slice are handled by adjacent lanes, so that one store
+        //    instruction writes whole 32-byte sectors.
         for (int e = ctid; e < nw * Q; e += RUN_CONSUMERS) {
             const int o = e / Q, q = e % Q;
             const int lko = s_wlk[o];
