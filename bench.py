@@ -35,8 +35,8 @@ L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 # the hash of the kernel sources it was taken with; None when not yet measured for the
 # current sources.  Filled from profiles/ (see the summary named there).
 MEASURED_TRAFFIC = {
-    # profiles/recur_run_kernel_mid_prefill.md: dram read 706.26 MB + write 409.43 MB
-    "7d1696cf3c1c3940": 1_115_686_144,
+    # profiles/recur_run_kernel_mid_prefill.md: dram read 729.02 MB + write 407.74 MB
+    "d0d71db08613d40f": 1_136_753_664,
 }
 
 
@@ -44,7 +44,7 @@ def kernel_source_hash() -> str:
     """Hash of the sources that define the recurrence row-pass kernel."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_state_linear_score_b200", "csrc")
-    for name in ("common.cuh", "plan.cuh", "recur.cuh"):
+    for name in ("common.cuh", "plan.cuh", "recur.cuh", "tc_ptx.cuh"):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
