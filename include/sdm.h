@@ -171,9 +171,12 @@ sdm_status sdm_forward(const sdm_dims* dims, const void* v, const float* alpha, 
  *                     of the rows each token gathers (from the slot stamps), links between
  *                     occurrences of the same slot inside each chunk, and per chunk the
  *                     C x C matrices that resolve them (a triangular solve, the intra-chunk
- *                     phase of the pages' Appendix A.1); writes ws, st->stamp and st->Lambda.
- *   sdm_forward_run   the row pass: gathers, delta updates, stores, outputs (reads ws,
- *                     updates st->M, writes out).
+ *                     phase of the pages' Appendix A.1), packed with every other
+ *                     column-independent input of the row pass into ws; writes ws,
+ *                     st->stamp and st->Lambda.
+ *   sdm_forward_run   the row pass: gathers, delta updates, stores, outputs (reads v and ws
+ *                     -- the plan's packed copy of indices, weights and beta -- updates
+ *                     st->M, writes out).  widx/ww/ridx/rw are validated, not re-read.
  * A run must follow the plan of the same call, on the same stream, with the same index,
  * weight and gate arrays and unchanged ws.
  */
