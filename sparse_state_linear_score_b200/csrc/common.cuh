@@ -44,4 +44,13 @@ SDM_DEV void cp_async8(void* smem_dst, const void* gmem_src) {
 SDM_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 SDM_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 
+// x / d for 0 <= x < 2^16 and 1 <= d <= 64 as one multiply-high: with m = ceil(2^32 / d),
+// m*d - 2^32 < d, so the rounding error x*(m*d - 2^32) < 2^22 never reaches 2^32.
+struct FastDiv {
+    unsigned m, d;
+    __host__ __device__ explicit FastDiv(unsigned dd) : m((unsigned)((0x100000000ull + dd - 1) / dd)), d(dd) {}
+    SDM_DEV int div(int x) const { return (int)__umulhi((unsigned)x, m); }
+    SDM_DEV int mod(int x) const { return x - div(x) * (int)d; }
+};
+
 }  // namespace sdm

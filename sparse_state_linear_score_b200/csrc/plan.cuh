@@ -150,7 +150,7 @@ __host__ __device__ inline RunImg run_img(int C, int W, int R) {
     return m;
 }
 
-__global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
+__global__ void __launch_bounds__(PLAN_THREADS, 2) plan_local_kernel(
     const float* __restrict__ alpha, const float* __restrict__ beta,
     const int32_t* __restrict__ widx, const float* __restrict__ ww,
     const int32_t* __restrict__ ridx, const float* __restrict__ rw,
@@ -198,8 +198,15 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
     }
     if (tid == nt - 1) P.csum[bh * J + j] = pre;
 
-    // 2. slots and weights of the chunk (and the previous chunk's write slots), hash heads
-    for (int o = tid; o < no; o += PLAN_THREADS) {
+    // 2. slots and weights of the chunk (and the previous chunk's write slots), hash heads;
+    //    the slots' entry stamps are fetched now (registers) and written in step 7
+    constexpr int PO = PLAN_MAX_OCC / PLAN_THREADS;
+    double est[PO];
+#pragma unroll
+    for (int k = 0; k < PO; ++k) {
+        const int o = tid + k * PLAN_THREADS;
+        est[k] = 0.0;
+        if (o >= no) continue;
         int s;
         float w;
         if (o < nw) {
@@ -212,6 +219,8 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
         if (!slot_ok(s, N)) {
             raise_err(SDM_DEVERR_SLOT_RANGE);
             s = -1;
+        } else {
+            est[k] = stamp[bh * (size_t)N + s];
         }
         s_slot[o] = s;
         s_wt[o] = w;
@@ -244,17 +253,18 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
     __syncthreads();
 
     // 4. links: latest earlier write of the same slot; owner = no later write in chunk
+    const FastDiv fW((unsigned)W), fR((unsigned)R);
     for (int o = tid; o < no; o += PLAN_THREADS) {
         const int s = s_slot[o];
         int link = -1;
         if (s >= 0) {
             const bool is_w = o < nw;
-            const int tl = is_w ? o / W : (o - nw) / R;
+            const int tl = is_w ? fW.div(o) : fR.div(o - nw);
             int best_t = -1;
             bool later = false;
             for (int p = s_head[slot_hash(s)]; p >= 0; p = s_next[p]) {
                 if (s_slot[p] != s) continue;
-                const int tp = p / W;
+                const int tp = fW.div(p);
                 if (is_w) {
                     if (tp == tl && p != o) raise_err(SDM_DEVERR_DUP_WRITE);
                     if (tp > tl) later = true;
@@ -273,25 +283,38 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
     }
     __syncthreads();
 
-    // 5. L and G rows: token t walks the link chain of each of its occurrences (every
-    //    earlier write of the slot in the chunk), in a fixed order (deterministic sums)
-    if (tid < nt) {
-        const int t = tid;
-        const float lt = s_lamc[t];
-        for (int i = 0; i < W; ++i) {
-            const int o = t * W + i;
-            const float wo = s_wt[o];
-            for (int L = s_link[o]; L >= 0; L = s_link[L]) {
-                const int tp = L / W;
-                s_L[t * PLAN_MAX_C + tp] += wo * s_wt[L] * expf(lt - s_lamc[tp]);
-            }
-        }
-        for (int i = 0; i < R; ++i) {
-            const int o = nw + t * R + i;
-            const float uo = s_wt[o];
-            for (int L = s_link[o]; L >= 0; L = s_link[L]) {
-                const int tp = L / W;
-                s_G[t * PLAN_MAX_C + tp] += uo * s_wt[L] * expf(lt - s_lamc[tp]);
+    // 5. L and G rows: one warp per (role, token) t; its lanes walk the link chains of t's
+    //    occurrences (every earlier write of the slot in the chunk) in step, and the terms of
+    //    one step are added to row t in lane order (deterministic sums)
+    {
+        const int warp = tid >> 5, lane = tid & 31;
+        for (int task = warp; task < 2 * nt; task += PLAN_THREADS / 32) {
+            const bool rd = task >= nt;
+            const int t = rd ? task - nt : task;
+            const int n_i = rd ? R : W;
+            const int o0 = rd ? nw + t * R : t * W;
+            float* row = (rd ? s_G : s_L) + t * PLAN_MAX_C;
+            const float lt = s_lamc[t];
+            for (int base = 0; base < n_i; base += 32) {
+                const int o = o0 + base + lane;
+                const bool in = base + lane < n_i;
+                const float wo = in ? s_wt[o] : 0.f;
+                int L = in ? s_link[o] : -1;
+                while (__any_sync(0xffffffffu, L >= 0)) {
+                    int tp = 0;
+                    float val = 0.f;
+                    if (L >= 0) {
+                        tp = fW.div(L);
+                        val = wo * s_wt[L] * expf(lt - s_lamc[tp]);
+                    }
+                    for (unsigned m = __ballot_sync(0xffffffffu, L >= 0); m; m &= m - 1) {
+                        const int src = __ffs(m) - 1;
+                        const int tps = __shfl_sync(0xffffffffu, tp, src);
+                        const float vs = __shfl_sync(0xffffffffu, val, src);
+                        if (lane == 0) row[tps] += vs;
+                    }
+                    L = L >= 0 ? s_link[L] : -1;
+                }
             }
         }
     }
@@ -342,7 +365,10 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
     }
 
     // 7. link words and entry stamps
-    for (int o = tid; o < no; o += PLAN_THREADS) {
+#pragma unroll
+    for (int k = 0; k < PO; ++k) {
+        const int o = tid + k * PLAN_THREADS;
+        if (o >= no) continue;
         const int link = s_link[o];
         unsigned v = (unsigned)(link + 1);
         size_t g;
@@ -361,7 +387,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_local_kernel(
             v |= (unsigned)(best + 1) << LK_PREV_SHIFT;
         }
         P.lk[g] = (int32_t)v;
-        P.st0[g] = sl >= 0 ? stamp[bh * (size_t)N + sl] : 0.0;
+        P.st0[g] = est[k];
         P.occw[g] = (sl >= 0 ? (uint32_t)sl : OCC_SLOT) | (o < nw && s_owner[o] ? OCC_OWNER : 0u);
         if (P.mask && o < nw && s_owner[o] && sl >= 0)  // this chunk stores the slot
             atomicOr(P.mask + (bh * (size_t)N + sl) * P.MW + (j >> 6), 1ull << (j & 63));

@@ -60,15 +60,6 @@ __host__ __device__ inline int run_tok_stride(int per_tok, int CW) { return per_
 // Row stride of Minv / GM in the chunk image (16-byte rows, 4 floats apart in banks).
 __host__ __device__ inline int run_mat_stride(int C) { return C + 4; }
 
-// x / d for 0 <= x < 2^16 and 1 <= d <= 64 as one multiply-high: with m = ceil(2^32 / d),
-// m*d - 2^32 < d, so the rounding error x*(m*d - 2^32) < 2^22 never reaches 2^32.
-struct FastDiv {
-    unsigned m, d;
-    __host__ __device__ explicit FastDiv(unsigned dd) : m((unsigned)((0x100000000ull + dd - 1) / dd)), d(dd) {}
-    SDM_DEV int div(int x) const { return (int)__umulhi((unsigned)x, m); }
-    SDM_DEV int mod(int x) const { return x - div(x) * (int)d; }
-};
-
 // Shared memory of the row pass (bytes), in this order: rows [2][C*(tsw+tsr)] floats,
 // images [2][img bytes], values [2][C*CW] of VT (16-byte padded), rhs, d, Q0 [C*CW] floats
 // each, the image copies' mbarrier.
