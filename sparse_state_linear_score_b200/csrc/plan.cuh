@@ -388,7 +388,8 @@ __global__ void __launch_bounds__(PLAN_THREADS, 2) plan_local_kernel(
         }
         P.lk[g] = (int32_t)v;
         P.st0[g] = est[k];
-        P.occw[g] = (sl >= 0 ? (uint32_t)sl : OCC_SLOT) | (o < nw && s_owner[o] ? OCC_OWNER : 0u);
+        if (!P.mask)  // the walk's input
+            P.occw[g] = (sl >= 0 ? (uint32_t)sl : OCC_SLOT) | (o < nw && s_owner[o] ? OCC_OWNER : 0u);
         if (P.mask && o < nw && s_owner[o] && sl >= 0)  // this chunk stores the slot
             atomicOr(P.mask + (bh * (size_t)N + sl) * P.MW + (j >> 6), 1ull << (j & 63));
     }
@@ -418,6 +419,35 @@ __global__ void __launch_bounds__(1024) plan_prefix_kernel(double* __restrict__ 
     if (tid == 0) lambda[bh] = Lg[J];
 }
 
+// Decay factor of one occurrence (slot s < N, owner bit, token prefix lam_t, entry stamp st)
+// in chunk j.  With the masks it is final (and the slot's last storing chunk writes the new
+// stamp); without, it is as if the slot had not been written earlier in this call.
+SDM_DEV float occ_factor(double* __restrict__ stamp, const PlanPtrs& P, size_t bh, int N, int J,
+                         int j, int s, bool owner, float lam_t, double st) {
+    const double* Lb = P.Lstart + bh * (size_t)(J + 1);
+    const double Lj = Lb[j];
+    int jw = -1;
+    if (P.mask) {
+        const unsigned long long* m = P.mask + (bh * (size_t)N + s) * P.MW;
+        for (int wi = j >> 6; wi >= 0 && jw < 0; --wi) {
+            unsigned long long bits = m[wi];
+            if (wi == (j >> 6)) bits &= (j & 63) ? ((1ull << (j & 63)) - 1) : 0ull;
+            if (bits) jw = wi * 64 + 63 - __clzll((long long)bits);
+        }
+        if (owner) {  // the slot's last storing chunk sets its stamp
+            int jl = -1;
+            for (int wi = P.MW - 1; wi >= 0 && jl < 0; --wi) {
+                const unsigned long long bits = m[wi];
+                if (bits) jl = wi * 64 + 63 - __clzll((long long)bits);
+            }
+            if (jl == j) stamp[bh * (size_t)N + s] = Lb[j + 1];
+        }
+    }
+    if (jw >= 0) return expf((float)(Lj - Lb[jw + 1]) + lam_t);
+    const double Lt = Lj + (double)lam_t;
+    return isnan(st) ? -(float)exp(Lt) : (float)exp(Lt - st);
+}
+
 // Decay factors of every occurrence.  Without a mask: as if its slot had not been written
 // earlier in this call (the walk corrects the others).  With the per-slot chunk masks: the
 // last earlier chunk that stored the slot is the highest set bit below this chunk, so every
@@ -429,8 +459,6 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_fe_kernel(double* __restric
     const size_t bh = blockIdx.y;
     const int t0 = j * C, nt = min(C, T - t0), nw = nt * W, no = nt * (W + R);
     const size_t occ_base = bh * (size_t)T * (W + R);
-    const double* Lb = P.Lstart + bh * (size_t)(J + 1);
-    const double Lj = Lb[j];
     for (int o = threadIdx.x; o < no; o += PLAN_THREADS) {
         size_t g;
         int t;
@@ -447,30 +475,8 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_fe_kernel(double* __restric
             P.fe[g] = 0.f;
             continue;
         }
-        const double Lt = Lj + (double)P.lam[bh * T + t0 + t];
-        int jw = -1;
-        if (P.mask) {
-            const unsigned long long* m = P.mask + (bh * (size_t)N + s) * P.MW;
-            for (int wi = j >> 6; wi >= 0 && jw < 0; --wi) {
-                unsigned long long bits = m[wi];
-                if (wi == (j >> 6)) bits &= (j & 63) ? ((1ull << (j & 63)) - 1) : 0ull;
-                if (bits) jw = wi * 64 + 63 - __clzll((long long)bits);
-            }
-            if (w & OCC_OWNER) {  // the slot's last storing chunk sets its stamp
-                int jl = -1;
-                for (int wi = P.MW - 1; wi >= 0 && jl < 0; --wi) {
-                    const unsigned long long bits = m[wi];
-                    if (bits) jl = wi * 64 + 63 - __clzll((long long)bits);
-                }
-                if (jl == j) stamp[bh * (size_t)N + s] = Lb[j + 1];
-            }
-        }
-        if (jw >= 0) {
-            P.fe[g] = expf((float)(Lj - Lb[jw + 1]) + P.lam[bh * T + t0 + t]);
-        } else {
-            const double st = P.st0[g];
-            P.fe[g] = isnan(st) ? -(float)exp(Lt) : (float)exp(Lt - st);
-        }
+        P.fe[g] = occ_factor(stamp, P, bh, N, J, j, s, (w & OCC_OWNER) != 0,
+                             P.lam[bh * T + t0 + t], P.st0[g]);
     }
 }
 
@@ -573,7 +579,7 @@ __global__ void __launch_bounds__(WALK_THREADS) plan_walk_kernel(
 // and the chunk image (coefficients, store factors, links, the list of occurrences whose row
 // the previous chunk stores — in any order — and beta).
 __global__ void __launch_bounds__(PLAN_THREADS) plan_pack_kernel(
-    const float* __restrict__ beta, const int32_t* __restrict__ widx,
+    double* __restrict__ stamp, const float* __restrict__ beta, const int32_t* __restrict__ widx,
     const float* __restrict__ ww, const int32_t* __restrict__ ridx,
     const float* __restrict__ rw, int T, int N, int W, int R, int C, int J, PlanPtrs P) {
     __shared__ float s_lam[PLAN_MAX_C];
@@ -617,9 +623,14 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_pack_kernel(
             w = rw[(bh * T + t0) * R + r];
             ci = C * (W + 1) + t * (R + 1) + (r - t * R);
         }
-        const float f = P.fe[g];
         const int lk = P.lk[g];
         const bool ok = slot_ok(s, N);
+        // with the masks the factors are computed here (plan_fe is not run); after the walk
+        // they are read back
+        const float f = !ok ? 0.f
+                        : P.mask ? occ_factor(stamp, P, bh, N, J, j, s, (o < nw) && (lk & LK_OWNER),
+                                              s_lam[o < nw ? o / W : (o - nw) / R], P.st0[g])
+                                 : P.fe[g];
         rs[o] = ok ? (int32_t)((uint32_t)s | (signbit(f) ? 0x80000000u : 0u)) : 0x7fffffff;
         coef[ci] = ok ? w * fabsf(f) : 0.f;
         if (o < nw) {

@@ -394,17 +394,18 @@ sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const floa
     if ((e = launch_status())) return e;
     plan_prefix_kernel<<<(unsigned)BH, 1024, 0, stream>>>(st->Lambda, L.J, P);
     if ((e = launch_status())) return e;
-    plan_fe_kernel<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, 0, stream>>>(
-        st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, P);
-    if ((e = launch_status())) return e;
-    if (!P.mask) {  // the walk finishes the factors and the stamps
+    if (!P.mask) {  // factors as if unwritten in this call; the walk finishes them and the stamps
+        plan_fe_kernel<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, 0, stream>>>(
+            st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, P);
+        if ((e = launch_status())) return e;
         if (!set_smem(plan_walk_kernel, L.walk_smem)) return SDM_ERR_CUDA;
         plan_walk_kernel<<<dim3(WALK_PARTS, (unsigned)BH), WALK_THREADS, L.walk_smem, stream>>>(
             st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, L.lstart_smem ? 1 : 0, P);
         if ((e = launch_status())) return e;
     }
+    // with the masks, plan_pack computes the final factors and stamps itself
     plan_pack_kernel<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, 0, stream>>>(
-        beta, widx, ww, ridx, rw, dims->T, N, dims->W, dims->R, L.C, L.J, P);
+        st->stamp, beta, widx, ww, ridx, rw, dims->T, N, dims->W, dims->R, L.C, L.J, P);
     return launch_status();
 }
 
