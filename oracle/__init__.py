@@ -19,6 +19,8 @@ Parity status per function:
   recur_lazy .................. pinned (agrees with recur_dense to 1e-12)
   materialize ................. pinned (beta=0 closed form)
   prefill_pairs ............... pinned through score + recur_lazy
+  weight_stats ................ pinned (uniform and one-hot closed forms, two-point
+                                 entropy, numpy sort for the order statistics)
 The softmax temperature and the tie order are readings the pages do not fix
 (parity of those two choices is unpinned by the pages themselves).
 """
@@ -92,12 +94,33 @@ class Oracle:
         lib.sdm_oracle_prefill_pairs.argtypes = [I, I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P,
                                                  I, P, P, I]
         lib.sdm_oracle_prefill_pairs.restype = I
+        lib.sdm_oracle_weight_stats.argtypes = [I, I, P, P, P, P, P, I, P, P]
+        lib.sdm_oracle_weight_stats.restype = I
         lib.sdm_oracle_max_threads.argtypes = []
         lib.sdm_oracle_max_threads.restype = I
         self.lib = lib
 
     def max_threads(self) -> int:
         return int(self.lib.sdm_oracle_max_threads())
+
+    def weight_stats(self, w, probs=(0.1, 0.5, 0.9)):
+        """Memory-utilisation diagnostics (Appendix D.1) of weight rows w [..., K] given best
+        first: per-row cumulative mass and normalised effective keys exp(H)/K, their means,
+        and order statistics of exp(H)/K at floor(p*(rows-1)).  Returns a dict."""
+        w = _f64(w)
+        K = int(w.shape[-1])
+        rows = int(w.size // K)
+        cum = np.empty(w.shape, dtype=np.float64)
+        eff = np.empty(w.shape[:-1], dtype=np.float64)
+        mean_cum = np.empty(K, dtype=np.float64)
+        mean_eff = np.empty(1, dtype=np.float64)
+        pr = _f64(probs)
+        quant = np.empty(len(pr), dtype=np.float64)
+        _check(self.lib.sdm_oracle_weight_stats(rows, K, _p(w), _p(cum), _p(eff), _p(mean_cum),
+                                                _p(mean_eff), len(pr), _p(pr), _p(quant)),
+               "weight_stats")
+        return {"cum": cum, "eff": eff, "mean_cum": mean_cum, "mean_eff": float(mean_eff[0]),
+                "quant": quant}
 
     def half_scores(self, x, sk):
         """s1[i] = <x[:h], C1[i]>, s2[j] = <x[h:], C2[j]> for one vector x [2h], sk [2,n,h]."""

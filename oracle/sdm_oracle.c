@@ -355,6 +355,59 @@ int sdm_oracle_prefill_pairs(int B, int H, int T, int hd, int n, int dv, int k_h
     return rc;
 }
 
+/*
+ * Memory-utilisation diagnostics over post-softmax selected-slot weights (pages:
+ * Appendix D.1 "Memory Utilization and Access": cumulative top-k mass and an
+ * entropy-based effective-key measure, summarised by the mean and by token-level
+ * quantiles over batch, head and time).  For each of `rows` weight vectors of length
+ * K, given best first (the order sdm_oracle_topk_vec returns):
+ *   cum[r][k] = w[r][0] + ... + w[r][k]                 (mass of the k+1 largest)
+ *   eff[r]    = exp(H_r) / K,  H_r = -sum_i w[r][i] ln w[r][i]   (0 ln 0 = 0)
+ * eff = 1 for uniform weights, 1/K for a one-hot vector.  Summary: mean_cum[k] =
+ * mean over rows of cum[r][k]; mean_eff = mean of eff; quant[q] = the order
+ * statistic of eff at index floor(probs[q] * (rows - 1)) of the ascending sort.
+ * cum and eff may be NULL.
+ */
+static int cmp_double_asc(const void* pa, const void* pb) {
+    const double a = *(const double*)pa, b = *(const double*)pb;
+    return a < b ? -1 : (a > b ? 1 : 0);
+}
+
+int sdm_oracle_weight_stats(int rows, int K, const double* w, double* cum, double* eff,
+                            double* mean_cum, double* mean_eff, int nprobs,
+                            const double* probs, double* quant) {
+    if (rows < 1 || K < 1 || !w || !mean_cum || !mean_eff) return ORACLE_ERR_ARG;
+    double* e = (double*)malloc(sizeof(double) * (size_t)rows);
+    if (!e) return ORACLE_ERR_NOMEM;
+    for (int k = 0; k < K; ++k) mean_cum[k] = 0.0;
+    double sum_eff = 0.0;
+    for (int r = 0; r < rows; ++r) {
+        const double* wr = w + (size_t)r * K;
+        double c = 0.0, H = 0.0;
+        for (int k = 0; k < K; ++k) {
+            c += wr[k];
+            if (cum) cum[(size_t)r * K + k] = c;
+            mean_cum[k] += c;
+            if (wr[k] > 0.0) H -= wr[k] * log(wr[k]);
+        }
+        e[r] = exp(H) / K;
+        if (eff) eff[r] = e[r];
+        sum_eff += e[r];
+    }
+    for (int k = 0; k < K; ++k) mean_cum[k] /= rows;
+    *mean_eff = sum_eff / rows;
+    if (nprobs > 0) {
+        if (!probs || !quant) { free(e); return ORACLE_ERR_ARG; }
+        qsort(e, (size_t)rows, sizeof(double), cmp_double_asc);
+        for (int q = 0; q < nprobs; ++q) {
+            if (!(probs[q] >= 0.0 && probs[q] <= 1.0)) { free(e); return ORACLE_ERR_ARG; }
+            quant[q] = e[(size_t)floor(probs[q] * (rows - 1))];
+        }
+    }
+    free(e);
+    return ORACLE_OK;
+}
+
 int sdm_oracle_max_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -341,7 +341,55 @@ def pin_prefill_pairs(o):
         assert np.array_equal(out[pi], ref)
 
 
+# ------------------------------------------------------ utilisation diagnostics ---
+# Appendix D.1 "Memory Utilization and Access": cumulative top-k mass and an entropy-based
+# effective-key measure of the post-softmax selected-slot weights, with the mean and
+# token-level quantiles over batch, head and time.
+
+def pin_weight_stats_closed_forms(o):
+    K = 8
+    # uniform weights: mass k/K, exp(H)/K = 1
+    r = o.weight_stats(np.full((5, K), 1.0 / K))
+    assert np.allclose(r["cum"][0], np.arange(1, K + 1) / K, rtol=0, atol=1e-15)
+    assert np.allclose(r["eff"], 1.0, rtol=0, atol=1e-14)
+    # one-hot: mass 1 everywhere, exp(0)/K
+    w = np.zeros((3, K))
+    w[:, 0] = 1.0
+    r = o.weight_stats(w)
+    assert np.array_equal(r["cum"], np.ones((3, K)))
+    assert np.allclose(r["eff"], 1.0 / K, rtol=0, atol=1e-15)
+    # two-point weights (p, 1-p): H = -p ln p - (1-p) ln(1-p), natural log
+    p = 0.8
+    w = np.zeros((1, K))
+    w[0, :2] = [p, 1 - p]
+    r = o.weight_stats(w)
+    H = -p * np.log(p) - (1 - p) * np.log(1 - p)
+    assert abs(r["eff"][0] - np.exp(H) / K) < 1e-14
+    assert abs(r["cum"][0, 0] - p) < 1e-15 and abs(r["cum"][0, 1] - 1.0) < 1e-15
+
+
+def pin_weight_stats_summaries(o):
+    rng = _rng(77)
+    K, rows = 16, 1000  # p * (rows - 1) is not an integer for p = 0.1, 0.5, 0.9
+    w = rng.dirichlet(np.full(K, 0.7), rows)
+    w = -np.sort(-w, axis=1)  # best first
+    probs = (0.0, 0.1, 0.5, 0.9, 1.0)
+    r = o.weight_stats(w, probs)
+    # per row: cumulative sums and exp(entropy)/K written out with numpy
+    assert np.allclose(r["cum"], np.cumsum(w, axis=1), rtol=0, atol=1e-14)
+    H = -(w * np.log(w)).sum(1)
+    assert np.allclose(r["eff"], np.exp(H) / K, rtol=1e-13, atol=0)
+    assert np.allclose(r["mean_cum"], np.cumsum(w, axis=1).mean(0), rtol=0, atol=1e-14)
+    assert abs(r["mean_eff"] - (np.exp(H) / K).mean()) < 1e-13
+    # order statistics at floor(p (rows-1)) of the ascending sort
+    srt = np.sort(np.exp(H) / K)
+    for q, pq in zip(r["quant"], probs):
+        assert abs(q - srt[int(np.floor(pq * (rows - 1)))]) < 1e-13
+    assert abs(r["mean_cum"][-1] - 1.0) < 1e-12
+
+
 ALL_PINS = [pin_pk_equals_brute, pin_brute_matches_numpy, pin_pk_depends_on_k, pin_tie_order,
             pin_hand_scoring, pin_softmax, pin_batched_score, pin_beta_zero, pin_one_hot_exact,
             pin_convex_update, pin_dense_limit_gdn, pin_lazy_equals_dense, pin_split_invariance,
-            pin_hand_recurrence, pin_prefill_pairs]
+            pin_hand_recurrence, pin_prefill_pairs, pin_weight_stats_closed_forms,
+            pin_weight_stats_summaries]

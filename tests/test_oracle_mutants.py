@@ -51,6 +51,13 @@ MUTANTS = {
         ("for (int a = 0; a < k_half; ++a)\n            for (int b = 0; b < k_half; ++b) {",
          "for (int a = 0; a < k_half; ++a)\n            for (int b = 0; b < k_half - (a == 0); ++b) {"),
     ],
+    "entropy_in_bits": [
+        ("if (wr[k] > 0.0) H -= wr[k] * log(wr[k]);", "if (wr[k] > 0.0) H -= wr[k] * log2(wr[k]);"),
+    ],
+    "quantile_index_rounded_up": [
+        ("quant[q] = e[(size_t)floor(probs[q] * (rows - 1))];",
+         "quant[q] = e[(size_t)ceil(probs[q] * (rows - 1))];"),
+    ],
     "read_weights_from_write": [
         ("o += rw[(size_t)t * R + j] * M[(size_t)rs[j] * dv + c];",
          "o += rw[(size_t)t * R + j] * M[(size_t)ws[j % W] * dv + c];"),
