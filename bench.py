@@ -254,7 +254,26 @@ def run_gpu(args, wl, world, rank, local):
     plan_ms = [e[1].elapsed_time(e[2]) for e in evs]
     run_ms = [e[2].elapsed_time(e[3]) for e in evs]
     total_ms = reduce_max(sum(step_ms), device)
-    launches_per_step = 6  # reset, 2 x score, plan_local, plan_walk, run
+    # reset, 2 x score, plan_local, plan_prefix, plan_pack, run (the per-slot chunk masks
+    # fit this workload, so plan_fe and plan_walk are not launched)
+    launches_per_step = 7
+
+    # memory-utilisation diagnostics of the write weights (after the timed steps)
+    diag = None
+    if rank == 0:
+        sdm.weight_stats(sel[1])
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(5):
+            g = sdm.weight_stats(sel[1])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dms = e0.elapsed_time(e1) / 5
+        rows = sel[1].numel() // wl.W
+        diag = {"kernels": "weight_stats_rows + weight_stats_summary", "rows": rows, "K": wl.W,
+                "ms": dms, "mean_eff": float(g["mean_eff"]),
+                "quant_eff_p10_p50_p90": [float(x) for x in g["quant"]]}
 
     # end to end through the public API with host buffers
     e2e = run_e2e(args, wl, d, inp, st, sel, out, ws, device, sdm)
@@ -305,6 +324,7 @@ def run_gpu(args, wl, world, rank, local):
                       "plan": statistics.mean(plan_ms), "run": statistics.mean(run_ms)},
         "scoring": {"tflops": score_tflops, "frac_of_bf16_peak": score_tflops / peaks["bf16_tflops"]},
         "e2e": e2e,
+        "diagnostics": diag,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "device_errors": errs,

@@ -235,6 +235,28 @@ sdm_status sdm_forward_noalloc(const sdm_dims* dims, const void* v, const float*
                                float* out, sdm_stream_t stream);
 
 /*
+ * Memory-utilisation diagnostics of post-softmax selected-slot weights (the pages'
+ * Appendix D.1 "Memory Utilization and Access": cumulative top-k mass and an entropy-based
+ * effective-key measure, summarised by the mean and token-level quantiles over batch, head
+ * and time).  Rows are given best first, as sdm_score_topk writes them.
+ *   w     [rows][K] fp32 (e.g. the ww or rw of a prefill: rows = B*H*T, K = W or R)
+ *   cum   [rows][K] fp32, or NULL: cum[r][k] = w[r][0] + ... + w[r][k]
+ *   eff   [rows] fp32: exp(H_r) / K with H_r = -sum_k w[r][k] ln w[r][k] (0 ln 0 = 0):
+ *         1 for uniform weights, 1/K for one-hot
+ *   mean  [K+1] fp32: the means over rows of cum[.][k] for k < K, then of eff
+ *   probs HOST array of nprobs (0..16) values in [0, 1]
+ *   quant [nprobs] fp32: the order statistic of eff at index floor(probs[q] * (rows-1))
+ *         of its ascending sort (exact, ties included)
+ *   ws    device workspace of at least sdm_weight_stats_workspace_bytes(rows, K) bytes
+ * Requires rows >= 1, 1 <= K <= 64; device pointers 4-byte aligned.  Means are summed in a
+ * fixed order (run to run identical).  Three kernel launches.
+ */
+size_t sdm_weight_stats_workspace_bytes(int64_t rows, int32_t K);
+sdm_status sdm_weight_stats(int64_t rows, int32_t K, const float* w, float* cum, float* eff,
+                            float* mean, int32_t nprobs, const double* probs, float* quant,
+                            void* ws, size_t ws_bytes, sdm_stream_t stream);
+
+/*
  * Read the device error word into *bits (host pointer; SDM_DEVERR_* bits), then
  * clear it when `clear` is non-zero.  Synchronises `stream`.  Returns SDM_OK when
  * no bit is set, SDM_ERR_BAD_INDEX when any is, SDM_ERR_CUDA if the copy fails.

@@ -23,8 +23,8 @@ from . import build as _build
 
 __all__ = ["Dims", "State", "SdmError", "state_reset", "state_materialize", "score_topk",
            "forward_workspace_bytes", "forward", "forward_noalloc", "forward_plan", "forward_run", "prefill",
-           "decode_step", "device_error", "lib_path", "DEVERR_SLOT_RANGE", "DEVERR_DUP_WRITE",
-           "DEVERR_ALPHA"]
+           "decode_step", "device_error", "weight_stats", "lib_path", "DEVERR_SLOT_RANGE",
+           "DEVERR_DUP_WRITE", "DEVERR_ALPHA"]
 
 F32, BF16 = 0, 1
 _DT = {"f32": F32, "bf16": BF16, torch.float32: F32, torch.bfloat16: BF16}
@@ -82,6 +82,8 @@ def _load():
         "sdm_decode_step": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P], I32),
         "sdm_device_error": ([ctypes.POINTER(ctypes.c_uint32), I32, P], I32),
         "sdm_forward_noalloc": ([D, P, P, P, P, P, P, P, S, P, P], I32),
+        "sdm_weight_stats_workspace_bytes": ([ctypes.c_int64, I32], SZ),
+        "sdm_weight_stats": ([ctypes.c_int64, I32, P, P, P, P, I32, P, P, P, SZ, P], I32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -280,3 +282,25 @@ def device_error(clear: bool = True, stream=None) -> int:
     if st not in (0, 6):
         raise SdmError(st, "sdm_device_error")
     return int(bits.value)
+
+
+def weight_stats(w: torch.Tensor, probs=(0.1, 0.5, 0.9), cum: bool = True, stream=None) -> dict:
+    """Memory-utilisation diagnostics (sdm_weight_stats) of weight rows w [..., K] fp32 given
+    best first: per-row cumulative mass (if cum) and exp(entropy)/K, their means, and the
+    order statistics of exp(entropy)/K at floor(p * (rows - 1))."""
+    K = int(w.shape[-1])
+    rows = int(w.numel() // K) if K else 0
+    dev = w.device
+    eff = torch.empty(w.shape[:-1], dtype=torch.float32, device=dev)
+    cum_t = torch.empty(w.shape, dtype=torch.float32, device=dev) if cum else None
+    mean = torch.empty(K + 1, dtype=torch.float32, device=dev)
+    pr = (ctypes.c_double * max(1, len(probs)))(*probs)
+    quant = torch.empty(max(1, len(probs)), dtype=torch.float32, device=dev)
+    nbytes = _lib.sdm_weight_stats_workspace_bytes(rows, K)
+    ws = torch.empty(max(1, nbytes), dtype=torch.uint8, device=dev)
+    _ok(_lib.sdm_weight_stats(rows, K, _ptr(w, "w", torch.float32), _ptr(cum_t, "cum"),
+                              _ptr(eff, "eff"), _ptr(mean, "mean"), len(probs), pr,
+                              _ptr(quant, "quant"), _ptr(ws, "ws"), nbytes, _stream(stream)),
+        "sdm_weight_stats")
+    return {"cum": cum_t, "eff": eff, "mean_cum": mean[:K], "mean_eff": mean[K],
+            "quant": quant[:len(probs)]}

@@ -13,6 +13,7 @@
 #include "score_simt.cuh"
 #include "score_tc.cuh"
 #include "state.cuh"
+#include "stats.cuh"
 
 using namespace sdm;
 
@@ -304,7 +305,7 @@ const char* sdm_status_str(int32_t status) {
     }
 }
 
-int32_t sdm_abi_version(void) { return 2; }
+int32_t sdm_abi_version(void) { return 3; }
 
 sdm_status sdm_state_bytes(const sdm_dims* dims, size_t* M_bytes, size_t* stamp_bytes,
                            size_t* lambda_bytes) {
@@ -514,6 +515,40 @@ sdm_status sdm_forward_noalloc(const sdm_dims* dims, const void* v, const float*
     if ((e = noalloc_workspace(&ws))) return e;
     return sdm_forward(dims, v, alpha, beta, widx, ww, ridx, rw, st, out, ws,
                        kNoAllocWorkspaceBytes, stream);
+}
+
+size_t sdm_weight_stats_workspace_bytes(int64_t rows, int32_t K) {
+    if (rows < 1 || K < 1 || K > STATS_MAXK) return 0;
+    const size_t blocks = (size_t)((rows + STATS_THREADS - 1) / STATS_THREADS);
+    return blocks * (size_t)(K + 1) * sizeof(float);
+}
+
+sdm_status sdm_weight_stats(int64_t rows, int32_t K, const float* w, float* cum, float* eff,
+                            float* mean, int32_t nprobs, const double* probs, float* quant,
+                            void* ws, size_t ws_bytes, sdm_stream_t stream) {
+    if (rows < 1 || K < 1 || K > STATS_MAXK) return SDM_ERR_SHAPE;
+    if (nprobs < 0 || nprobs > STATS_MAXP) return SDM_ERR_ARG;
+    if (!w || !eff || !mean || (nprobs > 0 && (!probs || !quant))) return SDM_ERR_ARG;
+    const uintptr_t a = (uintptr_t)w | (uintptr_t)eff | (uintptr_t)mean | (uintptr_t)cum |
+                        (uintptr_t)quant | (uintptr_t)ws;
+    if (a & 3u) return SDM_ERR_ALIGN;
+    StatsProbs P{};
+    for (int q = 0; q < nprobs; ++q) {
+        if (!(probs[q] >= 0.0 && probs[q] <= 1.0)) return SDM_ERR_ARG;
+        P.p[q] = probs[q];
+    }
+    const size_t need = sdm_weight_stats_workspace_bytes(rows, K);
+    if (!ws || ws_bytes < need) return SDM_ERR_WORKSPACE;
+    const long long blocks = (rows + STATS_THREADS - 1) / STATS_THREADS;
+    if (blocks > 0x7fffffffLL) return SDM_ERR_SHAPE;
+    float* part = static_cast<float*>(ws);
+    weight_stats_rows_kernel<<<(unsigned)blocks, STATS_THREADS, 0, stream>>>(w, rows, K, cum,
+                                                                            eff, part);
+    sdm_status e = launch_status();
+    if (e) return e;
+    weight_stats_summary_kernel<<<1, 1024, 0, stream>>>(part, (int)blocks, rows, K, eff, mean,
+                                                        nprobs, P, quant);
+    return launch_status();
 }
 
 sdm_status sdm_device_error(uint32_t* bits, int32_t clear, sdm_stream_t stream) {
