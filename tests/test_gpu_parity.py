@@ -187,6 +187,27 @@ def test_prefill_end_to_end(sdm, orc):
         assert per_bh_rel_err(f64(out), ref) <= TOL[wl.v_dtype]
 
 
+def test_shared_subkey_tables(sdm, orc):
+    """One sub-key table for both roles (the same array passed as skw and skr): reads and
+    writes then address the same slots for q = k, and everything still matches the oracle."""
+    wl = S.MID.scaled(B=1, H=2, T=160)
+    inp = to_dev(S.generate(wl))
+    inp["q"] = inp["k"].clone()  # same key for reading and writing: same slots
+    d = dims_of(sdm, wl)
+    st = sdm.State(d, inp["M0"])
+    sdm.state_reset(d, st)
+    out, (widx, ww, ridx, rw) = sdm.prefill(d, inp["q"], inp["k"], inp["v"], inp["alpha"],
+                                            inp["beta"], inp["skw"], inp["skw"], st)
+    torch.cuda.synchronize()
+    check_selection(orc, inp["k"], inp["skw"], widx, ww, wl.k_half, wl.W, wl.n_sub)
+    check_selection(orc, inp["q"], inp["skw"], ridx, rw, wl.k_half, wl.R, wl.n_sub)
+    assert torch.equal(widx, ridx) and torch.equal(ww, rw)
+    pairs = [(b, h) for b in range(wl.B) for h in range(wl.H)]
+    outs, _ = oracle_recurrence(orc, inp, widx.cpu(), ww.cpu(), ridx.cpu(), rw.cpu(), pairs)
+    ref = np.stack(outs).reshape(wl.B, wl.H, wl.T, wl.d_v)
+    assert per_bh_rel_err(f64(out), ref) <= TOL[wl.v_dtype]
+
+
 def test_split_invariance(sdm, orc):
     """prefill(T) == prefill(T1) + prefill(T-T1) == prefill(T1) + (T-T1) decode steps."""
     wl = S.MID.scaled(B=2, H=2, T=90, n_sub=32, k_half=8, W=8, R=8, d_v=32)
