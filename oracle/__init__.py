@@ -21,6 +21,8 @@ Parity status per function:
   prefill_pairs ............... pinned through score + recur_lazy
   weight_stats ................ pinned (uniform and one-hot closed forms, two-point
                                  entropy, numpy sort for the order statistics)
+  layer_out ................... pinned (hand RMS-norm example, scale invariance, swish
+                                 closed forms, gate zero, head selection by Wo, matmul)
 The softmax temperature and the tie order are readings the pages do not fix
 (parity of those two choices is unpinned by the pages themselves).
 """
@@ -96,12 +98,29 @@ class Oracle:
         lib.sdm_oracle_prefill_pairs.restype = I
         lib.sdm_oracle_weight_stats.argtypes = [I, I, P, P, P, P, P, I, P, P]
         lib.sdm_oracle_weight_stats.restype = I
+        lib.sdm_oracle_layer_out.argtypes = [I, I, I, I, I, P, P, P, D, P, I, P, P]
+        lib.sdm_oracle_layer_out.restype = I
         lib.sdm_oracle_max_threads.argtypes = []
         lib.sdm_oracle_max_threads.restype = I
         self.lib = lib
 
     def max_threads(self) -> int:
         return int(self.lib.sdm_oracle_max_threads())
+
+    def layer_out(self, o, g, wn, Wo_t, eps: float = 1e-6, rows=None):
+        """Output side of an SDM layer: o [B,H,T,dv], g [B,T,H*dv], wn [dv], Wo_t [dm, H*dv]
+        -> y [B,T,dm], or [len(rows), dm] for the listed rows (b*T + t)."""
+        o = _f64(o)
+        B, H, T, dv = o.shape
+        Wo_t = _f64(Wo_t)
+        dm = int(Wo_t.shape[0])
+        full = rows is None
+        r = np.arange(B * T, dtype=np.int64) if full else np.ascontiguousarray(rows, dtype=np.int64)
+        y = np.empty((len(r), dm), dtype=np.float64)
+        _check(self.lib.sdm_oracle_layer_out(B, H, T, dv, dm, _p(o), _p(_f64(g)), _p(_f64(wn)),
+                                             float(eps), _p(Wo_t), len(r), _p(r), _p(y)),
+               "layer_out")
+        return y.reshape(B, T, dm) if full else y
 
     def weight_stats(self, w, probs=(0.1, 0.5, 0.9)):
         """Memory-utilisation diagnostics (Appendix D.1) of weight rows w [..., K] given best

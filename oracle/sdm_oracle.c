@@ -408,6 +408,51 @@ int sdm_oracle_weight_stats(int rows, int K, const double* w, double* cum, doubl
     return ORACLE_OK;
 }
 
+/*
+ * Output side of an SDM layer (paperlayer.ai §3 Method "Sparse retrieval": the read result
+ * is RMS-normalised, elementwise gated and mixed across heads by the output projection).
+ * Readings: RMS-norm over each head's d_v values with one weight vector wn shared by the
+ * heads, x / sqrt(mean x^2 + eps); the gate is swish(z) = z * sigmoid(z) of a given
+ * pre-activation g; the mix is the output projection Wo (given transposed).
+ *   o [B][H][T][dv], g [B][T][H*dv], wn [dv], Wo_t [dm][H*dv]  ->  y [B][T][dm]
+ * Only the rows listed in `rows` (indices b*T + t, nrows of them) are computed; y is then
+ * [nrows][dm].  OpenMP over rows.
+ */
+int sdm_oracle_layer_out(int B, int H, int T, int dv, int dm, const double* o, const double* g,
+                         const double* wn, double eps, const double* Wo_t, int nrows,
+                         const int64_t* rows, double* y) {
+    const int K = H * dv;
+    int rc = ORACLE_OK;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int ri = 0; ri < nrows; ++ri) {
+        const int64_t bt = rows[ri];
+        if (bt < 0 || bt >= (int64_t)B * T) { rc = ORACLE_ERR_ARG; continue; }
+        const int b = (int)(bt / T), t = (int)(bt % T);
+        double* a = (double*)malloc(sizeof(double) * (size_t)K);
+        if (!a) { rc = ORACLE_ERR_NOMEM; continue; }
+        for (int h = 0; h < H; ++h) {
+            const double* x = o + (((size_t)b * H + h) * T + t) * dv;
+            double ms = 0.0;
+            for (int c = 0; c < dv; ++c) ms += x[c] * x[c];
+            const double r = 1.0 / sqrt(ms / dv + eps);
+            for (int c = 0; c < dv; ++c) {
+                const double z = g[(size_t)bt * K + (size_t)h * dv + c];
+                const double sw = z / (1.0 + exp(-z));
+                a[h * dv + c] = x[c] * r * wn[c] * sw;
+            }
+        }
+        for (int n = 0; n < dm; ++n) {
+            double acc = 0.0;
+            for (int k = 0; k < K; ++k) acc += a[k] * Wo_t[(size_t)n * K + k];
+            y[(size_t)ri * dm + n] = acc;
+        }
+        free(a);
+    }
+    return rc;
+}
+
 int sdm_oracle_max_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -388,8 +388,65 @@ def pin_weight_stats_summaries(o):
     assert abs(r["mean_cum"][-1] - 1.0) < 1e-12
 
 
+# ------------------------------------------------------------- layer output ---
+# §3 Method "Sparse retrieval": RMS-normalised, elementwise gated, mixed across heads.
+
+def _sig(z):
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def pin_layer_out_hand_example(o):
+    # one head, d_v = 2, x = (3, 4): mean square 12.5, so the normalised row is
+    # (3, 4) / sqrt(12.5); gate pre-activation z = 1 on both channels: swish(1) = sigma(1);
+    # wn = (1, 2); Wo = identity
+    x = np.array([3.0, 4.0]).reshape(1, 1, 1, 2)
+    g = np.ones((1, 1, 2))
+    wn = np.array([1.0, 2.0])
+    y = o.layer_out(x, g, wn, np.eye(2), eps=0.0)
+    s1 = 1.0 / (1.0 + np.exp(-1.0))
+    exp = np.array([3.0, 8.0]) / np.sqrt(12.5) * s1
+    assert np.allclose(y.reshape(2), exp, rtol=1e-14, atol=0)
+
+
+def pin_layer_out_properties(o):
+    rng = _rng(91)
+    B, H, T, dv, dm = 2, 3, 5, 8, 7
+    x = rng.standard_normal((B, H, T, dv))
+    g = rng.standard_normal((B, T, H * dv))
+    wn = rng.uniform(0.5, 1.5, dv)
+    Wo = rng.standard_normal((dm, H * dv))
+    y = o.layer_out(x, g, wn, Wo, eps=0.0)
+    # RMS-norm makes each head's read scale-free
+    assert np.allclose(o.layer_out(x * 7.5, g, wn, Wo, eps=0.0), y, rtol=1e-12, atol=1e-12)
+    # a zero gate closes the output; swish(z) ~ z for large z, ~ 0 for very negative z
+    assert np.array_equal(o.layer_out(x, np.zeros_like(g), wn, Wo, eps=0.0), np.zeros((B, T, dm)))
+    big = o.layer_out(x, np.full_like(g, 40.0), wn, Wo, eps=0.0)
+    assert np.allclose(big, 40.0 * o.layer_out(x, np.full_like(g, 1e6), wn, Wo, eps=0.0) / 1e6,
+                       rtol=1e-12, atol=1e-12)
+    # Wo selecting one head and channel returns that head's gated normalised channel
+    h, c = 2, 5
+    sel = np.zeros((1, H * dv))
+    sel[0, h * dv + c] = 1.0
+    ys = o.layer_out(x, g, wn, sel, eps=0.0)[..., 0]
+    xn = x[:, h] / np.sqrt((x[:, h] ** 2).mean(-1, keepdims=True))
+    z = g[:, :, h * dv + c]
+    assert np.allclose(ys, xn[..., c] * wn[c] * z * _sig(z), rtol=1e-12, atol=1e-14)
+    # mixing across heads is a linear map of the gated reads (numpy matmul, row subset)
+    a = np.concatenate([x[:, hh] / np.sqrt((x[:, hh] ** 2).mean(-1, keepdims=True)) * wn
+                        for hh in range(H)], axis=-1) * g * _sig(g)
+    assert np.allclose(y, a @ Wo.T, rtol=1e-12, atol=1e-12)
+    rows = np.array([7, 0, 3])
+    assert np.allclose(o.layer_out(x, g, wn, Wo, eps=0.0, rows=rows), y.reshape(B * T, dm)[rows],
+                       rtol=0, atol=0)
+    # eps enters as mean square + eps
+    e = 0.3
+    ye = o.layer_out(x, g, wn, sel, eps=e)[..., 0]
+    xe = x[:, h] / np.sqrt((x[:, h] ** 2).mean(-1, keepdims=True) + e)
+    assert np.allclose(ye, xe[..., c] * wn[c] * z * _sig(z), rtol=1e-12, atol=1e-14)
+
+
 ALL_PINS = [pin_pk_equals_brute, pin_brute_matches_numpy, pin_pk_depends_on_k, pin_tie_order,
             pin_hand_scoring, pin_softmax, pin_batched_score, pin_beta_zero, pin_one_hot_exact,
             pin_convex_update, pin_dense_limit_gdn, pin_lazy_equals_dense, pin_split_invariance,
             pin_hand_recurrence, pin_prefill_pairs, pin_weight_stats_closed_forms,
-            pin_weight_stats_summaries]
+            pin_weight_stats_summaries, pin_layer_out_hand_example, pin_layer_out_properties]

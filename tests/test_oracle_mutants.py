@@ -58,6 +58,15 @@ MUTANTS = {
         ("quant[q] = e[(size_t)floor(probs[q] * (rows - 1))];",
          "quant[q] = e[(size_t)ceil(probs[q] * (rows - 1))];"),
     ],
+    "rms_without_mean": [
+        ("const double r = 1.0 / sqrt(ms / dv + eps);", "const double r = 1.0 / sqrt(ms + eps);"),
+    ],
+    "gate_sigmoid_only": [
+        ("const double sw = z / (1.0 + exp(-z));", "const double sw = 1.0 / (1.0 + exp(-z));"),
+    ],
+    "wo_not_transposed": [
+        ("acc += a[k] * Wo_t[(size_t)n * K + k];", "acc += a[k] * Wo_t[(size_t)k * dm + n];"),
+    ],
     "read_weights_from_write": [
         ("o += rw[(size_t)t * R + j] * M[(size_t)rs[j] * dv + c];",
          "o += rw[(size_t)t * R + j] * M[(size_t)ws[j % W] * dv + c];"),
