@@ -275,6 +275,43 @@ def run_gpu(args, wl, world, rank, local):
                 "ms": dms, "mean_eff": float(g["mean_eff"]),
                 "quant_eff_p10_p50_p90": [float(x) for x in g["quant"]]}
 
+    # output side of the layer on this step's read output: RMS-norm, swish gate and the
+    # head-mixing projection (d_model = 4*H*n) on the tensor cores
+    layer = None
+    if rank == 0:
+        dm = 4 * wl.H * wl.n_sub
+        gen = torch.Generator(device=device).manual_seed(wl.seed + 17)
+        gate = torch.randn(wl.B, wl.T, wl.H * wl.d_v, device=device, generator=gen).to(torch.bfloat16)
+        wn = torch.ones(wl.d_v, device=device)
+        Wo_t = (torch.randn(dm, wl.H * wl.d_v, device=device, generator=gen) /
+                (wl.H * wl.d_v) ** 0.5).to(torch.bfloat16)
+        yb = torch.empty(wl.B, wl.T, dm, device=device)
+        lws = torch.empty(max(16, wl.B * wl.T * wl.H * wl.d_v * 2), dtype=torch.uint8, device=device)
+        A = torch.randn(wl.B * wl.T, wl.H * wl.d_v, device=device, generator=gen).to(torch.bfloat16)
+        Cg = torch.empty(wl.B * wl.T, dm, device=device)
+        for _ in range(3):
+            sdm.layer_out(d, out, gate, wn, Wo_t, y=yb, ws=lws)
+            sdm.gemm_bf16(A, Wo_t, Cg)
+        torch.cuda.synchronize()
+        res = {}
+        for name, fn in (("layer_out", lambda: sdm.layer_out(d, out, gate, wn, Wo_t, y=yb, ws=lws)),
+                         ("gemm", lambda: sdm.gemm_bf16(A, Wo_t, Cg))):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(10):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            res[name] = e0.elapsed_time(e1) / 10
+        flops = 2.0 * wl.B * wl.T * wl.H * wl.d_v * dm
+        tf = flops / (res["gemm"] / 1e3) / 1e12
+        pk = measured_peaks()["bf16_tflops"]
+        layer = {"M": wl.B * wl.T, "K": wl.H * wl.d_v, "N": dm, "layer_out_ms": res["layer_out"],
+                 "gemm_ms": res["gemm"],
+                 "gemm_roofline": {"bound": "tensor", "achieved": tf, "peak": pk,
+                                   "unit": "TFLOP/s", "frac": tf / pk,
+                                   "note": "bf16 x bf16 -> fp32, tcgen05; peak = measured burst bf16"}}
+
     # end to end through the public API with host buffers
     e2e = run_e2e(args, wl, d, inp, st, sel, out, ws, device, sdm)
     errs = sdm.device_error()
@@ -325,6 +362,7 @@ def run_gpu(args, wl, world, rank, local):
         "scoring": {"tflops": score_tflops, "frac_of_bf16_peak": score_tflops / peaks["bf16_tflops"]},
         "e2e": e2e,
         "diagnostics": diag,
+        "layer_out": layer,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "device_errors": errs,

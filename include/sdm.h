@@ -235,6 +235,33 @@ sdm_status sdm_forward_noalloc(const sdm_dims* dims, const void* v, const float*
                                float* out, sdm_stream_t stream);
 
 /*
+ * Dense GEMM on the tensor cores (tcgen05, bf16 operands, fp32 accumulation):
+ *   C[M][N] fp32 = A[M][K] x Bt[N][K]^T,  A and Bt bf16 row-major (K contiguous)
+ * K a multiple of 8; M, N free.  Pointers 16-byte aligned.  One launch.
+ */
+sdm_status sdm_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* A, const void* Bt, float* C,
+                         sdm_stream_t stream);
+
+/*
+ * Output side of an SDM layer (§3 Method "Sparse retrieval": the read result is
+ * RMS-normalised, elementwise gated and mixed across heads by the output projection):
+ *   a[b,t][h*d_v + c] = x_c / sqrt(mean_c x_c^2 + eps) * wn[c] * swish(g[b,t][h*d_v + c])
+ *                       with x = o[b][h][t][:], swish(z) = z * sigmoid(z)
+ *   y[b,t][:] = a[b,t][:] @ Wo
+ *   o    [B][H][T][d_v] fp32 (the recurrence output)
+ *   g    [B][T][H*d_v] bf16 (the gate's pre-activation)
+ *   wn   [d_v] fp32 (the RMS-norm weight, shared by the heads); eps >= 0
+ *   Wo_t [d_model][H*d_v] bf16 (Wo transposed)
+ *   y    [B][T][d_model] fp32
+ *   ws   at least sdm_layer_out_workspace_bytes(dims) bytes (a, bf16)
+ * Requires H*d_v a multiple of 8.  Two launches: the prologue, then sdm_gemm_bf16.
+ */
+size_t sdm_layer_out_workspace_bytes(const sdm_dims* dims);
+sdm_status sdm_layer_out(const sdm_dims* dims, const float* o, const void* g, const float* wn,
+                         float eps, const void* Wo_t, int32_t d_model, float* y, void* ws,
+                         size_t ws_bytes, sdm_stream_t stream);
+
+/*
  * Memory-utilisation diagnostics of post-softmax selected-slot weights (the pages'
  * Appendix D.1 "Memory Utilization and Access": cumulative top-k mass and an entropy-based
  * effective-key measure, summarised by the mean and token-level quantiles over batch, head

@@ -23,7 +23,8 @@ from . import build as _build
 
 __all__ = ["Dims", "State", "SdmError", "state_reset", "state_materialize", "score_topk",
            "forward_workspace_bytes", "forward", "forward_noalloc", "forward_plan", "forward_run", "prefill",
-           "decode_step", "device_error", "weight_stats", "lib_path", "DEVERR_SLOT_RANGE",
+           "decode_step", "device_error", "weight_stats", "gemm_bf16", "layer_out", "lib_path",
+           "DEVERR_SLOT_RANGE",
            "DEVERR_DUP_WRITE", "DEVERR_ALPHA"]
 
 F32, BF16 = 0, 1
@@ -82,6 +83,9 @@ def _load():
         "sdm_decode_step": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P], I32),
         "sdm_device_error": ([ctypes.POINTER(ctypes.c_uint32), I32, P], I32),
         "sdm_forward_noalloc": ([D, P, P, P, P, P, P, P, S, P, P], I32),
+        "sdm_gemm_bf16": ([I32, I32, I32, P, P, P, P], I32),
+        "sdm_layer_out_workspace_bytes": ([D], SZ),
+        "sdm_layer_out": ([D, P, P, P, ctypes.c_float, P, I32, P, P, SZ, P], I32),
         "sdm_weight_stats_workspace_bytes": ([ctypes.c_int64, I32], SZ),
         "sdm_weight_stats": ([ctypes.c_int64, I32, P, P, P, P, I32, P, P, P, SZ, P], I32),
     }
@@ -304,3 +308,36 @@ def weight_stats(w: torch.Tensor, probs=(0.1, 0.5, 0.9), cum: bool = True, strea
         "sdm_weight_stats")
     return {"cum": cum_t, "eff": eff, "mean_cum": mean[:K], "mean_eff": mean[K],
             "quant": quant[:len(probs)]}
+
+
+def gemm_bf16(A: torch.Tensor, Bt: torch.Tensor, C: torch.Tensor | None = None, stream=None):
+    """C = A @ Bt.T on the tensor cores: A [M, K] bf16, Bt [N, K] bf16 -> C [M, N] fp32."""
+    M, K = A.shape
+    N = Bt.shape[0]
+    if Bt.shape[1] != K:
+        raise ValueError("A and Bt must share K")
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.float32, device=A.device)
+    _ok(_lib.sdm_gemm_bf16(M, N, K, _ptr(A, "A", torch.bfloat16), _ptr(Bt, "Bt", torch.bfloat16),
+                           _ptr(C, "C", torch.float32), _stream(stream)), "sdm_gemm_bf16")
+    return C
+
+
+def layer_out(d: Dims, o: torch.Tensor, g: torch.Tensor, wn: torch.Tensor, Wo_t: torch.Tensor,
+              eps: float = 1e-6, y: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+              stream=None):
+    """SDM layer output: RMS-norm of each head's read, swish gate, output projection.
+    o [B,H,T,d_v] fp32, g [B,T,H*d_v] bf16, wn [d_v] fp32, Wo_t [d_model, H*d_v] bf16
+    -> y [B,T,d_model] fp32."""
+    d_model = int(Wo_t.shape[0])
+    if y is None:
+        y = torch.empty((d.B, d.T, d_model), dtype=torch.float32, device=o.device)
+    nbytes = _lib.sdm_layer_out_workspace_bytes(ctypes.byref(d))
+    if ws is None:
+        ws = torch.empty(max(16, nbytes), dtype=torch.uint8, device=o.device)
+    _ok(_lib.sdm_layer_out(ctypes.byref(d), _ptr(o, "o", torch.float32), _ptr(g, "g", torch.bfloat16),
+                           _ptr(wn, "wn", torch.float32), float(eps),
+                           _ptr(Wo_t, "Wo_t", torch.bfloat16), d_model,
+                           _ptr(y, "y", torch.float32), _ptr(ws, "ws"), ws.numel(),
+                           _stream(stream)), "sdm_layer_out")
+    return y

@@ -14,6 +14,8 @@
 #include "score_tc.cuh"
 #include "state.cuh"
 #include "stats.cuh"
+#include "gemm_tc.cuh"
+#include "layer.cuh"
 
 using namespace sdm;
 
@@ -515,6 +517,83 @@ sdm_status sdm_forward_noalloc(const sdm_dims* dims, const void* v, const float*
     if ((e = noalloc_workspace(&ws))) return e;
     return sdm_forward(dims, v, alpha, beta, widx, ww, ridx, rw, st, out, ws,
                        kNoAllocWorkspaceBytes, stream);
+}
+
+sdm_status sdm_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* A, const void* Bt, float* C,
+                         sdm_stream_t stream) {
+    if (M < 1 || N < 1 || K < 8 || K % 8 != 0) return SDM_ERR_SHAPE;
+    if (!A || !Bt || !C) return SDM_ERR_ARG;
+    if (!aligned16(A) || !aligned16(Bt) || !aligned16(C)) return SDM_ERR_ALIGN;
+    if ((long long)(M + GEMM_BM - 1) / GEMM_BM > 65535) return SDM_ERR_SHAPE;
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return SDM_ERR_CUDA;
+    CUtensorMap am, bm;
+    const cuuint32_t es[2] = {1, 1};
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {GEMM_BK, GEMM_BM};
+        if (enc(&am, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(A), dims, strides, box,
+                es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return SDM_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {GEMM_BK, GEMM_BN};
+        if (enc(&bm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(Bt), dims, strides, box,
+                es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return SDM_ERR_CUDA;
+    }
+    if (!set_smem(gemm_bf16_tc_kernel, GEMM_SMEM_BYTES)) return SDM_ERR_CUDA;
+    const dim3 grid((unsigned)((N + GEMM_BN - 1) / GEMM_BN), (unsigned)((M + GEMM_BM - 1) / GEMM_BM));
+    gemm_bf16_tc_kernel<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(am, bm, C, M, N, K);
+    return launch_status();
+}
+
+size_t sdm_layer_out_workspace_bytes(const sdm_dims* dims) {
+    if (check_dims(dims) != SDM_OK) return 0;
+    return (size_t)dims->B * dims->T * dims->H * dims->d_v * 2;
+}
+
+sdm_status sdm_layer_out(const sdm_dims* dims, const float* o, const void* g, const float* wn,
+                         float eps, const void* Wo_t, int32_t d_model, float* y, void* ws,
+                         size_t ws_bytes, sdm_stream_t stream) {
+    sdm_status e = check_dims(dims);
+    if (e) return e;
+    if (dims->T == 0) return SDM_OK;
+    if (!o || !g || !wn || !Wo_t || !y) return SDM_ERR_ARG;
+    if (!(eps >= 0.f) || d_model < 1) return SDM_ERR_ARG;
+    const int K = dims->H * dims->d_v;
+    if (K % 8 != 0) return SDM_ERR_SHAPE;
+    if (!aligned16(o) || !aligned16(g) || !aligned16(wn) || !aligned16(Wo_t) || !aligned16(y))
+        return SDM_ERR_ALIGN;
+    const size_t need = sdm_layer_out_workspace_bytes(dims);
+    if (!ws || ws_bytes < need) return SDM_ERR_WORKSPACE;
+    if (!aligned16(ws)) return SDM_ERR_ALIGN;
+    const long long rows = (long long)dims->B * dims->T;
+    if (rows > 0x7fffffffLL) return SDM_ERR_SHAPE;
+    __nv_bfloat16* a = static_cast<__nv_bfloat16*>(ws);
+    const long long warps = rows * dims->H;
+    const long long blocks = (warps * 32 + LAYER_THREADS - 1) / LAYER_THREADS;
+    const int per = (dims->d_v + 31) / 32;
+    const __nv_bfloat16* gb = static_cast<const __nv_bfloat16*>(g);
+    if (per <= 1)
+        layer_prologue_kernel<1><<<(unsigned)blocks, LAYER_THREADS, 0, stream>>>(
+            o, gb, wn, eps, dims->B, dims->H, dims->T, dims->d_v, a);
+    else if (per <= 2)
+        layer_prologue_kernel<2><<<(unsigned)blocks, LAYER_THREADS, 0, stream>>>(
+            o, gb, wn, eps, dims->B, dims->H, dims->T, dims->d_v, a);
+    else if (per <= 4)
+        layer_prologue_kernel<4><<<(unsigned)blocks, LAYER_THREADS, 0, stream>>>(
+            o, gb, wn, eps, dims->B, dims->H, dims->T, dims->d_v, a);
+    else
+        layer_prologue_kernel<8><<<(unsigned)blocks, LAYER_THREADS, 0, stream>>>(
+            o, gb, wn, eps, dims->B, dims->H, dims->T, dims->d_v, a);
+    if ((e = launch_status())) return e;
+    return sdm_gemm_bf16((int32_t)rows, d_model, K, a, Wo_t, y, stream);
 }
 
 size_t sdm_weight_stats_workspace_bytes(int64_t rows, int32_t K) {
