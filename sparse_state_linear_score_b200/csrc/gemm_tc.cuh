@@ -6,8 +6,11 @@
 // tcgen05.mma (K = 16 each) per K-block accumulate into GEMM_BN TMEM columns and commit to
 // empty[s], which frees the stage for the load GEMM_STAGES blocks later; a last commit
 // signals the epilogue.  All four warps then read their 32 TMEM lanes (rows) 32 columns at
-// a time and store fp32 rows.  Two CTAs fit an SM (TMEM 2 x 256 columns, 2 x 97 KB smem), so
-// one CTA's epilogue overlaps the other's MMAs.  Every mbarrier wait is bounded; on timeout
+// a time into a 128 x 32 fp32 staging tile in the (now free) stage memory, laid out with the
+// 128-byte swizzle (16-byte chunk index XOR row % 8: conflict-free writes), and thread 0
+// stores each tile with one TMA store (two tiles in flight).  Without a C tensor map (N not
+// a multiple of 4) the threads store their rows directly.  Two CTAs fit an SM (TMEM 2 x 256
+// columns, 2 x 97 KB smem), so one CTA's epilogue overlaps the other's MMAs.  Every mbarrier wait is bounded; on timeout
 // the device error word gets SDM_DEVERR_TIMEOUT and the CTA skips its stores.
 //
 // Loads past M, N or K read zeros (TMA bounds), stores are guarded, so M and N are free;
@@ -31,7 +34,8 @@ constexpr uint32_t GEMM_SMEM_BYTES = GEMM_STAGES * GEMM_STAGE_BYTES + 64 + 1024;
 
 __global__ void __launch_bounds__(GEMM_THREADS, 2) gemm_bf16_tc_kernel(
     const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
-    float* __restrict__ C, int M, int N, int K) {
+    const __grid_constant__ CUtensorMap cmap, int cmap_ok, float* __restrict__ C, int M, int N,
+    int K) {
     extern __shared__ unsigned char gemm_smem_raw[];
     unsigned char* sm =
         gemm_smem_raw + ((1024 - (ptx::smem_u32(gemm_smem_raw) & 1023)) & 1023);
@@ -113,7 +117,33 @@ __global__ void __launch_bounds__(GEMM_THREADS, 2) gemm_bf16_tc_kernel(
     }
     ptx::tc_fence_after();
     __syncthreads();
-    if (!*abort_flag) {
+    if (!*abort_flag && cmap_ok) {
+        // epilogue through swizzled staging tiles and TMA stores; the stage memory was last
+        // touched by the async proxy (loads, MMA reads)
+        ptx::fence_proxy_async_smem();
+        const int r = warp * 32 + (tid & 31);  // row inside the tile = TMEM lane
+        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+        for (int c = 0; c < GEMM_BN; c += 32) {
+            const int buf = (c / 32) & 1;
+            unsigned char* tile = sm + buf * (GEMM_BM * 32 * 4);  // 16 KB, 1024-aligned
+            if (c >= 64 && tid == 0) ptx::bulk_wait_group_read<1>();  // tile buf is free
+            __syncthreads();
+            float v[32];
+            ptx::tmem_ld32(trow + c, v);
+            unsigned char* rowp = tile + r * 128;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<float4*>(rowp + ((j ^ (r & 7)) << 4)) =
+                    make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            ptx::fence_proxy_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                ptx::tma_store_2d(&cmap, n0 + c, m0, tile);
+                ptx::bulk_commit_group();
+            }
+        }
+        if (tid == 0) ptx::bulk_wait_group_read<0>();  // staging read before the CTA exits
+    } else if (!*abort_flag) {
         // epilogue: warp w holds rows m0 + 32 w .. + 31 (TMEM lanes), 32 columns per load
         const int row = m0 + warp * 32 + (tid & 31);
         const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);

@@ -547,9 +547,22 @@ sdm_status sdm_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* A, const v
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return SDM_ERR_CUDA;
     }
+    // C by TMA stores when its rows are 16-byte multiples
+    CUtensorMap cm;
+    memset(&cm, 0, sizeof(cm));
+    int cm_ok = 0;
+    if (N % 4 == 0) {
+        const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+        const cuuint64_t strides[1] = {(cuuint64_t)N * 4};
+        const cuuint32_t box[2] = {32, GEMM_BM};
+        cm_ok = enc(&cm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, C, dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    }
     if (!set_smem(gemm_bf16_tc_kernel, GEMM_SMEM_BYTES)) return SDM_ERR_CUDA;
     const dim3 grid((unsigned)((N + GEMM_BN - 1) / GEMM_BN), (unsigned)((M + GEMM_BM - 1) / GEMM_BM));
-    gemm_bf16_tc_kernel<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(am, bm, C, M, N, K);
+    gemm_bf16_tc_kernel<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(am, bm, cm, cm_ok, C, M,
+                                                                        N, K);
     return launch_status();
 }
 

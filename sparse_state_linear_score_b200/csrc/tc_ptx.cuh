@@ -71,6 +71,22 @@ SDM_DEV void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int 
         : "memory");
 }
 
+// Tiled shared -> global store of a 2D box (bulk-group completion; out-of-range parts of
+// the box are not written).
+SDM_DEV void tma_store_2d(const CUtensorMap* map, int c0, int c1, const void* src) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(c0), "r"(c1), "r"(smem_u32(src))
+        : "memory");
+}
+SDM_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's bulk groups still read their shared source.
+template <int N>
+SDM_DEV void bulk_wait_group_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
 // Contiguous global -> shared copy of `bytes` (a multiple of 16, both addresses 16-byte
 // aligned) by the bulk-copy engine, completing on bar.
 SDM_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
