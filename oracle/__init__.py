@@ -21,6 +21,8 @@ Parity status per function:
   prefill_pairs ............... pinned through score + recur_lazy
   weight_stats ................ pinned (uniform and one-hot closed forms, two-point
                                  entropy, numpy sort for the order statistics)
+  layer_in .................... pinned (one-hot routing of inputs to each output, gate
+                                 closed forms, linearity, matmul)
   layer_out ................... pinned (hand RMS-norm example, scale invariance, swish
                                  closed forms, gate zero, head selection by Wo, matmul)
 The softmax temperature and the tie order are readings the pages do not fix
@@ -100,6 +102,8 @@ class Oracle:
         lib.sdm_oracle_weight_stats.restype = I
         lib.sdm_oracle_layer_out.argtypes = [I, I, I, I, I, P, P, P, D, P, I, P, P]
         lib.sdm_oracle_layer_out.restype = I
+        lib.sdm_oracle_layer_in.argtypes = [I, I, I, I, I, I, P, P, P, P, I, P, P, P, P, P, P, P]
+        lib.sdm_oracle_layer_in.restype = I
         lib.sdm_oracle_max_threads.argtypes = []
         lib.sdm_oracle_max_threads.restype = I
         self.lib = lib
@@ -121,6 +125,27 @@ class Oracle:
                                              float(eps), _p(Wo_t), len(r), _p(r), _p(y)),
                "layer_out")
         return y.reshape(B, T, dm) if full else y
+
+    def layer_in(self, x, Win_t, A_log, dt_bias, H: int, dk: int, dv: int, rows=None):
+        """Input side of an SDM layer: x [B,T,dm], Win_t [H*(2dk+2dv+2), dm] -> dict of q, k
+        [B,H,T,dk], v [B,H,T,dv], g [B,T,H*dv], alpha, beta [B,H,T]; with rows (b*T + t) the
+        outputs are per listed row: q [n,H,dk], v [n,H,dv], g [n,H*dv], alpha/beta [n,H]."""
+        x = _f64(x)
+        B, T, dm = x.shape
+        full = rows is None
+        r = np.arange(B * T, dtype=np.int64) if full else np.ascontiguousarray(rows, dtype=np.int64)
+        n = len(r)
+        q = np.empty((n, H, dk)); k = np.empty((n, H, dk)); v = np.empty((n, H, dv))
+        g = np.empty((n, H * dv)); a = np.empty((n, H)); b = np.empty((n, H))
+        _check(self.lib.sdm_oracle_layer_in(B, H, T, dk, dv, dm, _p(x), _p(_f64(Win_t)),
+                                            _p(_f64(A_log)), _p(_f64(dt_bias)), n, _p(r), _p(q),
+                                            _p(k), _p(v), _p(g), _p(a), _p(b)), "layer_in")
+        if not full:
+            return {"q": q, "k": k, "v": v, "g": g, "alpha": a, "beta": b}
+        bht = lambda z: z.reshape(B, T, H, -1).transpose(0, 2, 1, 3)
+        return {"q": bht(q), "k": bht(k), "v": bht(v), "g": g.reshape(B, T, H * dv),
+                "alpha": a.reshape(B, T, H).transpose(0, 2, 1),
+                "beta": b.reshape(B, T, H).transpose(0, 2, 1)}
 
     def weight_stats(self, w, probs=(0.1, 0.5, 0.9)):
         """Memory-utilisation diagnostics (Appendix D.1) of weight rows w [..., K] given best

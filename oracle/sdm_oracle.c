@@ -453,6 +453,59 @@ int sdm_oracle_layer_out(int B, int H, int T, int dv, int dm, const double* o, c
     return rc;
 }
 
+/*
+ * Input side of an SDM layer: the projections of the layer input x into the per-head query,
+ * key, value, output-gate pre-activation and the two gates (paperlayer.ai §2 Background
+ * "Gated DeltaNet": decay gate alpha_t in (0,1), input gate beta_t in [0,1]; §4 "SDM
+ * Configuration": forget gate and time-step bias as in GDN/FLA; appendix "Gate dynamics":
+ * the forget gate is exp(g), the input gate sigma(b)).  Readings: per head h, the columns
+ * of P = x Win (Win given transposed, Win_t [Nin][dm]) are laid out as
+ *   [q (dk) | k (dk) | v (dv) | g (dv) | a | b],  Nin = H (2 dk + 2 dv + 2),
+ * alpha = exp(-exp(A_log[h]) * softplus(a + dt_bias[h])), beta = sigmoid(b);
+ * no short convolution and no q/k normalisation.
+ *   x [B][T][dm]  ->  q, k [B][H][T][dk], v [B][H][T][dv], g [B][T][H*dv],
+ *                     alpha, beta [B][H][T]
+ * Only the rows listed (b*T + t) are computed; outputs are then indexed by list position
+ * in place of (b, t): q [nrows][H][dk], v [nrows][H][dv], g [nrows][H*dv], alpha/beta
+ * [nrows][H].  OpenMP over rows.
+ */
+static double softplus_d(double z) { return z > 30.0 ? z : log1p(exp(z)); }
+
+int sdm_oracle_layer_in(int B, int H, int T, int dk, int dv, int dm, const double* x,
+                        const double* Win_t, const double* A_log, const double* dt_bias,
+                        int nrows, const int64_t* rows, double* q, double* k, double* v,
+                        double* g, double* alpha, double* beta) {
+    const int hs = 2 * dk + 2 * dv + 2, Nin = H * hs;
+    int rc = ORACLE_OK;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int ri = 0; ri < nrows; ++ri) {
+        const int64_t bt = rows[ri];
+        if (bt < 0 || bt >= (int64_t)B * T) { rc = ORACLE_ERR_ARG; continue; }
+        double* P = (double*)malloc(sizeof(double) * (size_t)Nin);
+        if (!P) { rc = ORACLE_ERR_NOMEM; continue; }
+        const double* xr = x + (size_t)bt * dm;
+        for (int n = 0; n < Nin; ++n) P[n] = dot(xr, Win_t + (size_t)n * dm, dm);
+        for (int h = 0; h < H; ++h) {
+            const double* ph = P + (size_t)h * hs;
+            for (int c = 0; c < dk; ++c) {
+                q[((size_t)ri * H + h) * dk + c] = ph[c];
+                k[((size_t)ri * H + h) * dk + c] = ph[dk + c];
+            }
+            for (int c = 0; c < dv; ++c) {
+                v[((size_t)ri * H + h) * dv + c] = ph[2 * dk + c];
+                g[(size_t)ri * H * dv + (size_t)h * dv + c] = ph[2 * dk + dv + c];
+            }
+            const double a = ph[2 * dk + 2 * dv], bb = ph[2 * dk + 2 * dv + 1];
+            alpha[(size_t)ri * H + h] = exp(-exp(A_log[h]) * softplus_d(a + dt_bias[h]));
+            beta[(size_t)ri * H + h] = 1.0 / (1.0 + exp(-bb));
+        }
+        free(P);
+    }
+    return rc;
+}
+
 int sdm_oracle_max_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -445,8 +445,67 @@ def pin_layer_out_properties(o):
     assert np.allclose(ye, xe[..., c] * wn[c] * z * _sig(z), rtol=1e-12, atol=1e-14)
 
 
+# -------------------------------------------------------------- layer input ---
+
+def pin_layer_in_routing_and_gates(o):
+    H, dk, dv, dm = 2, 3, 2, 5
+    hs = 2 * dk + 2 * dv + 2
+    rng = _rng(93)
+    B, T = 2, 3
+    x = rng.standard_normal((B, T, dm))
+    A_log = np.array([0.2, -0.7])
+    dt = np.array([0.5, -1.0])
+    # Win routes input dim (n mod dm) to output column n: every output is a known input value
+    Win = np.zeros((H * hs, dm))
+    for n in range(H * hs):
+        Win[n, n % dm] = 1.0
+    r = o.layer_in(x, Win, A_log, dt, H, dk, dv)
+    col = lambda n: x[..., n % dm]  # [B, T]
+    for h in range(H):
+        base = h * hs
+        for c in range(dk):
+            assert np.array_equal(r["q"][:, h, :, c], col(base + c))
+            assert np.array_equal(r["k"][:, h, :, c], col(base + dk + c))
+        for c in range(dv):
+            assert np.array_equal(r["v"][:, h, :, c], col(base + 2 * dk + c))
+            assert np.array_equal(r["g"][:, :, h * dv + c], col(base + 2 * dk + dv + c))
+        a = col(base + 2 * dk + 2 * dv)
+        b = col(base + 2 * dk + 2 * dv + 1)
+        sp = np.log1p(np.exp(a + dt[h]))
+        assert np.allclose(r["alpha"][:, h], np.exp(-np.exp(A_log[h]) * sp), rtol=1e-14, atol=0)
+        assert np.allclose(r["beta"][:, h], 1 / (1 + np.exp(-b)), rtol=1e-14, atol=0)
+    # gate ranges: alpha in (0, 1), beta in (0, 1); a very negative a gives alpha -> 1
+    assert ((r["alpha"] > 0) & (r["alpha"] < 1)).all() and ((r["beta"] > 0) & (r["beta"] < 1)).all()
+    Wa = np.zeros((H * hs, dm))
+    xs = np.full((1, 1, dm), -60.0)
+    Wa[2 * dk + 2 * dv, 0] = 1.0
+    assert abs(o.layer_in(xs, Wa, A_log, np.zeros(H), H, dk, dv)["alpha"][0, 0, 0] - 1.0) < 1e-20 + 1e-12
+
+
+def pin_layer_in_linear(o):
+    rng = _rng(94)
+    H, dk, dv, dm, B, T = 3, 4, 2, 6, 2, 4
+    hs = 2 * dk + 2 * dv + 2
+    x = rng.standard_normal((B, T, dm))
+    Win = rng.standard_normal((H * hs, dm))
+    A_log, dt = rng.standard_normal(H), rng.standard_normal(H)
+    r = o.layer_in(x, Win, A_log, dt, H, dk, dv)
+    P = x @ Win.T  # numpy matmul: the projection
+    for h in range(H):
+        base = h * hs
+        assert np.allclose(r["q"][:, h], P[..., base:base + dk], rtol=1e-12, atol=1e-12)
+        assert np.allclose(r["v"][:, h], P[..., base + 2 * dk:base + 2 * dk + dv], rtol=1e-12, atol=1e-12)
+    # projections are linear in x; the listed-rows form agrees with the full form
+    r2 = o.layer_in(2 * x, Win, A_log, dt, H, dk, dv)
+    assert np.allclose(r2["k"], 2 * r["k"], rtol=1e-12, atol=1e-12)
+    rows = np.array([5, 0])
+    rs = o.layer_in(x, Win, A_log, dt, H, dk, dv, rows=rows)
+    assert np.array_equal(rs["g"], r["g"].reshape(B * T, -1)[rows])
+
+
 ALL_PINS = [pin_pk_equals_brute, pin_brute_matches_numpy, pin_pk_depends_on_k, pin_tie_order,
             pin_hand_scoring, pin_softmax, pin_batched_score, pin_beta_zero, pin_one_hot_exact,
             pin_convex_update, pin_dense_limit_gdn, pin_lazy_equals_dense, pin_split_invariance,
             pin_hand_recurrence, pin_prefill_pairs, pin_weight_stats_closed_forms,
-            pin_weight_stats_summaries, pin_layer_out_hand_example, pin_layer_out_properties]
+            pin_weight_stats_summaries, pin_layer_out_hand_example, pin_layer_out_properties,
+            pin_layer_in_routing_and_gates, pin_layer_in_linear]

@@ -67,6 +67,13 @@ MUTANTS = {
     "wo_not_transposed": [
         ("acc += a[k] * Wo_t[(size_t)n * K + k];", "acc += a[k] * Wo_t[(size_t)k * dm + n];"),
     ],
+    "decay_gate_without_exp_scale": [
+        ("alpha[(size_t)ri * H + h] = exp(-exp(A_log[h]) * softplus_d(a + dt_bias[h]));",
+         "alpha[(size_t)ri * H + h] = exp(-A_log[h] * softplus_d(a + dt_bias[h]));"),
+    ],
+    "q_k_swapped": [
+        ("q[((size_t)ri * H + h) * dk + c] = ph[c];", "q[((size_t)ri * H + h) * dk + c] = ph[dk + c];"),
+    ],
     "read_weights_from_write": [
         ("o += rw[(size_t)t * R + j] * M[(size_t)rs[j] * dv + c];",
          "o += rw[(size_t)t * R + j] * M[(size_t)ws[j % W] * dv + c];"),
