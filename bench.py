@@ -303,14 +303,37 @@ def run_gpu(args, wl, world, rank, local):
             e1.record(stream)
             torch.cuda.synchronize()
             res[name] = e0.elapsed_time(e1) / 10
+        # input side: x [B,T,dm] -> q, k, v, g, alpha, beta (one GEMM with K = dm)
+        hs = 2 * wl.d_k + 2 * wl.d_v + 2
+        x = torch.randn(wl.B, wl.T, dm, device=device, generator=gen).to(torch.bfloat16)
+        Win_t = (torch.randn(wl.H * hs, dm, device=device, generator=gen) / dm ** 0.5).to(torch.bfloat16)
+        A_log = torch.zeros(wl.H, device=device)
+        dtb = torch.zeros(wl.H, device=device)
+        lin = sdm.layer_in(d, x, Win_t, A_log, dtb)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(10):
+            sdm.layer_in(d, x, Win_t, A_log, dtb, out=lin)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        res["layer_in"] = e0.elapsed_time(e1) / 10
         flops = 2.0 * wl.B * wl.T * wl.H * wl.d_v * dm
         tf = flops / (res["gemm"] / 1e3) / 1e12
+        tf_in = 2.0 * wl.B * wl.T * wl.H * hs * dm / (res["layer_in"] / 1e3) / 1e12
         pk = measured_peaks()["bf16_tflops"]
-        layer = {"M": wl.B * wl.T, "K": wl.H * wl.d_v, "N": dm, "layer_out_ms": res["layer_out"],
-                 "gemm_ms": res["gemm"],
-                 "gemm_roofline": {"bound": "tensor", "achieved": tf, "peak": pk,
-                                   "unit": "TFLOP/s", "frac": tf / pk,
-                                   "note": "bf16 x bf16 -> fp32, tcgen05; peak = measured burst bf16"}}
+        st_ms = statistics.mean(step_ms)
+        layer = {"d_model": dm, "layer_in_ms": res["layer_in"], "layer_out_ms": res["layer_out"],
+                 "layer_forward_ms": res["layer_in"] + st_ms + res["layer_out"],
+                 "layer_forward_tokens_per_s": wl.B * wl.T /
+                 ((res["layer_in"] + st_ms + res["layer_out"]) / 1e3),
+                 "gemm_out": {"M": wl.B * wl.T, "K": wl.H * wl.d_v, "N": dm, "ms": res["gemm"],
+                              "tflops": tf, "frac_of_bf16_peak": tf / pk},
+                 "gemm_in_with_split": {"M": wl.B * wl.T, "K": dm, "N": wl.H * hs,
+                                        "ms": res["layer_in"], "tflops": tf_in,
+                                        "frac_of_bf16_peak": tf_in / pk},
+                 "note": "bf16 x bf16 -> fp32 on tcgen05; peak = measured burst bf16; "
+                         "layer_forward = layer_in + the timed step + layer_out"}
 
     # end to end through the public API with host buffers
     e2e = run_e2e(args, wl, d, inp, st, sel, out, ws, device, sdm)

@@ -243,6 +243,26 @@ sdm_status sdm_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* A, const v
                          sdm_stream_t stream);
 
 /*
+ * Input side of an SDM layer: the projections of the layer input into the per-head query,
+ * key, value, output-gate pre-activation and the two gates (§2 Background "Gated DeltaNet":
+ * decay gate alpha in (0,1), input gate beta in [0,1]; §4 "SDM Configuration": gates as in
+ * GDN/FLA):
+ *   P = x @ Win  (tensor cores), per head the columns [q (d_k) | k (d_k) | v (d_v) | g (d_v) | a | b]
+ *   alpha = exp(-exp(A_log[h]) * softplus(a + dt_bias[h])),  beta = sigmoid(b)
+ *   x     [B][T][d_model] bf16 (d_model a multiple of 8)
+ *   Win_t [H*(2 d_k + 2 d_v + 2)][d_model] bf16 (Win transposed); A_log, dt_bias [H] fp32
+ *   q, k  [B][H][T][d_k] bf16 (dims->x_dtype must be bf16); v [B][H][T][d_v] (v_dtype)
+ *   g     [B][T][H*d_v] bf16 (for sdm_layer_out); alpha, beta [B][H][T] fp32
+ *   ws    at least sdm_layer_in_workspace_bytes(dims) bytes (P, fp32)
+ * No short convolution and no q/k normalisation.  Two launches.
+ */
+size_t sdm_layer_in_workspace_bytes(const sdm_dims* dims);
+sdm_status sdm_layer_in(const sdm_dims* dims, const void* x, const void* Win_t,
+                        const float* A_log, const float* dt_bias, int32_t d_model, void* q,
+                        void* k, void* v, void* g, float* alpha, float* beta, void* ws,
+                        size_t ws_bytes, sdm_stream_t stream);
+
+/*
  * Output side of an SDM layer (§3 Method "Sparse retrieval": the read result is
  * RMS-normalised, elementwise gated and mixed across heads by the output projection):
  *   a[b,t][h*d_v + c] = x_c / sqrt(mean_c x_c^2 + eps) * wn[c] * swish(g[b,t][h*d_v + c])

@@ -23,7 +23,7 @@ from . import build as _build
 
 __all__ = ["Dims", "State", "SdmError", "state_reset", "state_materialize", "score_topk",
            "forward_workspace_bytes", "forward", "forward_noalloc", "forward_plan", "forward_run", "prefill",
-           "decode_step", "device_error", "weight_stats", "gemm_bf16", "layer_out", "lib_path",
+           "decode_step", "device_error", "weight_stats", "gemm_bf16", "layer_in", "layer_out", "lib_path",
            "DEVERR_SLOT_RANGE",
            "DEVERR_DUP_WRITE", "DEVERR_ALPHA"]
 
@@ -84,6 +84,8 @@ def _load():
         "sdm_device_error": ([ctypes.POINTER(ctypes.c_uint32), I32, P], I32),
         "sdm_forward_noalloc": ([D, P, P, P, P, P, P, P, S, P, P], I32),
         "sdm_gemm_bf16": ([I32, I32, I32, P, P, P, P], I32),
+        "sdm_layer_in_workspace_bytes": ([D], SZ),
+        "sdm_layer_in": ([D, P, P, P, P, I32, P, P, P, P, P, P, P, SZ, P], I32),
         "sdm_layer_out_workspace_bytes": ([D], SZ),
         "sdm_layer_out": ([D, P, P, P, ctypes.c_float, P, I32, P, P, SZ, P], I32),
         "sdm_weight_stats_workspace_bytes": ([ctypes.c_int64, I32], SZ),
@@ -341,3 +343,33 @@ def layer_out(d: Dims, o: torch.Tensor, g: torch.Tensor, wn: torch.Tensor, Wo_t:
                            _ptr(y, "y", torch.float32), _ptr(ws, "ws"), ws.numel(),
                            _stream(stream)), "sdm_layer_out")
     return y
+
+
+def layer_in(d: Dims, x: torch.Tensor, Win_t: torch.Tensor, A_log: torch.Tensor,
+             dt_bias: torch.Tensor, out: dict | None = None, ws: torch.Tensor | None = None,
+             stream=None) -> dict:
+    """SDM layer input side: x [B,T,d_model] bf16, Win_t [H*(2dk+2dv+2), d_model] bf16,
+    A_log / dt_bias [H] fp32 -> q, k [B,H,T,d_k] bf16, v [B,H,T,d_v], g [B,T,H*d_v] bf16,
+    alpha, beta [B,H,T] fp32 (the inputs of prefill and layer_out)."""
+    dev = x.device
+    d_model = int(x.shape[-1])
+    vdt = torch.bfloat16 if d.v_dtype == BF16 else torch.float32
+    if out is None:
+        out = {"q": torch.empty((d.B, d.H, d.T, d.d_k), dtype=torch.bfloat16, device=dev),
+               "k": torch.empty((d.B, d.H, d.T, d.d_k), dtype=torch.bfloat16, device=dev),
+               "v": torch.empty((d.B, d.H, d.T, d.d_v), dtype=vdt, device=dev),
+               "g": torch.empty((d.B, d.T, d.H * d.d_v), dtype=torch.bfloat16, device=dev),
+               "alpha": torch.empty((d.B, d.H, d.T), dtype=torch.float32, device=dev),
+               "beta": torch.empty((d.B, d.H, d.T), dtype=torch.float32, device=dev)}
+    nbytes = _lib.sdm_layer_in_workspace_bytes(ctypes.byref(d))
+    if ws is None:
+        ws = torch.empty(max(16, nbytes), dtype=torch.uint8, device=dev)
+    _ok(_lib.sdm_layer_in(ctypes.byref(d), _ptr(x, "x", torch.bfloat16),
+                          _ptr(Win_t, "Win_t", torch.bfloat16), _ptr(A_log, "A_log", torch.float32),
+                          _ptr(dt_bias, "dt_bias", torch.float32), d_model,
+                          _ptr(out["q"], "q", torch.bfloat16), _ptr(out["k"], "k", torch.bfloat16),
+                          _ptr(out["v"], "v", vdt), _ptr(out["g"], "g", torch.bfloat16),
+                          _ptr(out["alpha"], "alpha", torch.float32),
+                          _ptr(out["beta"], "beta", torch.float32), _ptr(ws, "ws"), ws.numel(),
+                          _stream(stream)), "sdm_layer_in")
+    return out

@@ -566,6 +566,50 @@ sdm_status sdm_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* A, const v
     return launch_status();
 }
 
+size_t sdm_layer_in_workspace_bytes(const sdm_dims* dims) {
+    if (check_dims(dims) != SDM_OK) return 0;
+    const size_t hs = (size_t)(2 * dims->d_k + 2 * dims->d_v + 2);
+    return (size_t)dims->B * dims->T * dims->H * hs * 4;
+}
+
+sdm_status sdm_layer_in(const sdm_dims* dims, const void* x, const void* Win_t,
+                        const float* A_log, const float* dt_bias, int32_t d_model, void* q,
+                        void* k, void* v, void* g, float* alpha, float* beta, void* ws,
+                        size_t ws_bytes, sdm_stream_t stream) {
+    sdm_status e = check_dims(dims);
+    if (e) return e;
+    if (dims->T == 0) return SDM_OK;
+    if (dims->x_dtype != SDM_BF16) return SDM_ERR_DTYPE;  // q, k are written as bf16
+    if (!x || !Win_t || !A_log || !dt_bias || !q || !k || !v || !g || !alpha || !beta)
+        return SDM_ERR_ARG;
+    if (d_model < 8 || d_model % 8 != 0) return SDM_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(Win_t) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+        !aligned16(g) || !aligned16(alpha) || !aligned16(beta))
+        return SDM_ERR_ALIGN;
+    const size_t need = sdm_layer_in_workspace_bytes(dims);
+    if (!ws || ws_bytes < need) return SDM_ERR_WORKSPACE;
+    if (!aligned16(ws)) return SDM_ERR_ALIGN;
+    const long long rows = (long long)dims->B * dims->T;
+    const int Nin = dims->H * (2 * dims->d_k + 2 * dims->d_v + 2);
+    if (rows > 0x7fffffffLL) return SDM_ERR_SHAPE;
+    float* P = static_cast<float*>(ws);
+    if ((e = sdm_gemm_bf16((int32_t)rows, Nin, d_model, x, Win_t, P, stream))) return e;
+    const long long total = rows * Nin;
+    long long blocks = (total + LAYER_THREADS - 1) / LAYER_THREADS;
+    if (blocks > 148LL * 64) blocks = 148LL * 64;
+    if (dims->v_dtype == SDM_BF16)
+        layer_in_split_kernel<__nv_bfloat16><<<(unsigned)blocks, LAYER_THREADS, 0, stream>>>(
+            P, A_log, dt_bias, dims->B, dims->H, dims->T, dims->d_k, dims->d_v,
+            static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k),
+            static_cast<__nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(g), alpha, beta);
+    else
+        layer_in_split_kernel<float><<<(unsigned)blocks, LAYER_THREADS, 0, stream>>>(
+            P, A_log, dt_bias, dims->B, dims->H, dims->T, dims->d_k, dims->d_v,
+            static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k),
+            static_cast<float*>(v), static_cast<__nv_bfloat16*>(g), alpha, beta);
+    return launch_status();
+}
+
 size_t sdm_layer_out_workspace_bytes(const sdm_dims* dims) {
     if (check_dims(dims) != SDM_OK) return 0;
     return (size_t)dims->B * dims->T * dims->H * dims->d_v * 2;

@@ -111,3 +111,67 @@ def test_gemm_validation(sdm):
     A = torch.zeros(4, 12, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(sdm.SdmError):
         sdm.gemm_bf16(A, torch.zeros(4, 12, dtype=torch.bfloat16, device="cuda"))  # K % 8
+
+
+def _layer_in_case(sdm, B, H, T, dk, dv, dm, n_sub, vdt, seed):
+    gen = torch.Generator(device="cuda").manual_seed(seed)
+    hs = 2 * dk + 2 * dv + 2
+    x = torch.randn(B, T, dm, device="cuda", generator=gen).to(torch.bfloat16)
+    Win_t = (torch.randn(H * hs, dm, device="cuda", generator=gen) / np.sqrt(dm)).to(torch.bfloat16)
+    A_log = torch.randn(H, device="cuda", generator=gen) * 0.5
+    dt = torch.randn(H, device="cuda", generator=gen) * 0.5
+    d = sdm.Dims(B, H, T, dk, n_sub, dv, 8, 8, 8, "bf16", vdt)
+    return d, x, Win_t, A_log, dt
+
+
+@pytest.mark.parametrize("B,H,T,dk,dv,dm,vdt", [(2, 2, 50, 32, 16, 64, "bf16"),
+                                                (1, 4, 130, 128, 128, 512, "bf16"),
+                                                (2, 3, 9, 16, 8, 40, "f32")])
+def test_layer_in_vs_oracle(sdm, B, H, T, dk, dv, dm, vdt):
+    d, x, Win_t, A_log, dt = _layer_in_case(sdm, B, H, T, dk, dv, dm, 16, vdt, seed=T + dm)
+    r = sdm.layer_in(d, x, Win_t, A_log, dt)
+    torch.cuda.synchronize()
+    ref = oracle.default().layer_in(f64(x), f64(Win_t), f64(A_log), f64(dt), H, dk, dv)
+    for name in ("q", "k", "v", "g"):
+        assert normwise_rel_err(f64(r[name]), ref[name]) <= 1e-2, name  # bf16 outputs
+    # gates: fp32 from fp32 accumulation of exact bf16 products
+    assert np.abs(f64(r["alpha"]) - ref["alpha"]).max() <= 1e-4
+    assert np.abs(f64(r["beta"]) - ref["beta"]).max() <= 1e-4
+    assert sdm.device_error() == 0
+
+
+def test_layer_forward_chain(sdm):
+    """x -> layer_in -> prefill (scoring + recurrence) -> layer_out, mid-like shapes, each
+    stage against the oracle fed the GPU's previous stage (bf16 rounding at the stage
+    boundaries is the GPU's own)."""
+    orc = oracle.default()
+    B, H, T, dk, dv, n, k, W = 1, 2, 96, 128, 128, 64, 16, 16
+    dm = 4 * H * n
+    d, x, Win_t, A_log, dt = _layer_in_case(sdm, B, H, T, dk, dv, dm, n, "bf16", seed=5)
+    d = sdm.Dims(B, H, T, dk, n, dv, k, W, W, "bf16", "bf16")
+    gen = torch.Generator(device="cuda").manual_seed(6)
+    skw = (torch.randn(H, 2, n, dk // 2, device="cuda", generator=gen) / 8).to(torch.bfloat16)
+    skr = (torch.randn(H, 2, n, dk // 2, device="cuda", generator=gen) / 8).to(torch.bfloat16)
+    M0 = torch.randn(H, n * n, dv, device="cuda", generator=gen) * 0.02
+    wn = torch.rand(dv, device="cuda", generator=gen) + 0.5
+    Wo_t = (torch.randn(dm, H * dv, device="cuda", generator=gen) / np.sqrt(H * dv)).to(torch.bfloat16)
+    r = sdm.layer_in(d, x, Win_t, A_log, dt)
+    st = sdm.State(d, M0)
+    sdm.state_reset(d, st)
+    o, (widx, ww, ridx, rw) = sdm.prefill(d, r["q"], r["k"], r["v"], r["alpha"], r["beta"],
+                                          skw, skr, st)
+    y = sdm.layer_out(d, o, r["g"], wn, Wo_t)
+    torch.cuda.synchronize()
+    ref_in = orc.layer_in(f64(x), f64(Win_t), f64(A_log), f64(dt), H, dk, dv)
+    assert normwise_rel_err(f64(r["q"]), ref_in["q"]) <= 1e-2
+    outs = []
+    for h in range(H):
+        s = orc.fresh_lazy_state(f64(M0[h]))
+        outs.append(orc.recur_lazy(f64(r["v"][0, h]), f64(r["alpha"][0, h]), f64(r["beta"][0, h]),
+                                   widx[0, h].cpu().numpy(), f64(ww[0, h]), ridx[0, h].cpu().numpy(),
+                                   f64(rw[0, h]), s))
+    ref_o = np.stack(outs).reshape(B, H, T, dv)
+    assert normwise_rel_err(f64(o), ref_o) <= TOL["bf16"]
+    ref_y = orc.layer_out(f64(o), f64(r["g"]), f64(wn), f64(Wo_t))
+    assert normwise_rel_err(f64(y), ref_y) <= TOL["bf16"]
+    assert sdm.device_error() == 0
