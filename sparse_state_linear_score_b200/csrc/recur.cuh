@@ -21,11 +21,11 @@
 // selected slots (§3 Method "Sparse memory updates", "Sparse retrieval"), evaluated chunk by
 // chunk as in the pages' Appendix A.1 (intra-chunk triangular solve, sequential chunks).
 //
-// Warp roles.  Warps 0..3 (producers) only move data: while the consumers compute chunk j
+// Warp roles.  Warps 0..7 (producers) only move data: while the consumers compute chunk j
 // they gather chunk j+1's rows into the other row buffer (cp.async, 16-byte pieces, the Q
 // pieces of a slice fetched by adjacent lanes of one instruction), copy its image (one bulk
 // copy on an mbarrier) and values into the other halves of the double buffers, and load
-// chunk j+2's gather words into registers.  Warps 4..15 (consumers) compute.  Named barriers
+// chunk j+2's gather words into registers.  Warps 8..15 (consumers) compute.  Named barriers
 // hand the buffers over:
 //   BAR_READY  producers arrive when chunk j+1's inputs have landed; consumers wait on it
 //   BAR_FIXED  consumers arrive when chunk j's forwarded rows are taken from the other row
@@ -42,7 +42,7 @@
 namespace sdm {
 
 constexpr int RUN_THREADS = 512;
-constexpr int RUN_PRODUCERS = 128;  // warps 0..3
+constexpr int RUN_PRODUCERS = 256;  // warps 0..7
 constexpr int RUN_CONSUMERS = RUN_THREADS - RUN_PRODUCERS;
 constexpr int RUN_PAD = 8;  // floats between token blocks: spreads a warp's rows over banks
 constexpr int RUN_GW = PLAN_MAX_OCC / RUN_PRODUCERS;  // gather words per producer thread
