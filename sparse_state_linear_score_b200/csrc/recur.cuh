@@ -320,32 +320,53 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
         //    the next chunk takes the ones it gathered before they were stored)
         //    The Q 16-byte pieces of a slice are handled by adjacent lanes, so that one store
         //    instruction writes whole 32-byte sectors.
-        for (int e = ctid; e < nw * Q; e += RUN_CONSUMERS) {
-            const int o = e / Q, q = e % Q;
-            const int lko = s_wlk[o];
-            const int s = s_wslot[o];
-            if (!(lko & LK_OWNER) || s >= N) continue;
-            // this write plus the chunk's earlier writes of the slot, decayed to the chunk end
-            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int L = o; L >= 0; L = lk_link(s_wlk[L])) {
-                const int tp = fW.div(L);
-                const float cfa = s_sc[L];
-                const float4 dd = reinterpret_cast<const float4*>(s_d + tp * CW)[q];
-                a.x = fmaf(cfa, dd.x, a.x);
-                a.y = fmaf(cfa, dd.y, a.y);
-                a.z = fmaf(cfa, dd.z, a.z);
-                a.w = fmaf(cfa, dd.w, a.w);
+        //    Two tasks per step, their loads issued together (most chains are the write
+        //    itself; the links to earlier writes of the slot, rare, are followed after).
+        for (int e0 = ctid; e0 < nw * Q; e0 += 2 * RUN_CONSUMERS) {
+            int o[2], q[2], lk[2], sl[2];
+            bool own[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int e = e0 + u * RUN_CONSUMERS;
+                const bool in = e < nw * Q;
+                o[u] = in ? e / Q : 0;
+                q[u] = e % Q;
+                lk[u] = s_wlk[o[u]];
+                sl[u] = s_wslot[o[u]];
+                own[u] = in && (lk[u] & LK_OWNER) && sl[u] < N;
             }
-            float4* rp = reinterpret_cast<float4*>(rows + wpos(o)) + q;
-            const float4 raw = *rp;
-            const float f = s_a[o];
-            float4 val;
-            val.x = fmaf(f, raw.x, a.x);
-            val.y = fmaf(f, raw.y, a.y);
-            val.z = fmaf(f, raw.z, a.z);
-            val.w = fmaf(f, raw.w, a.w);
-            reinterpret_cast<float4*>(Mb + (size_t)s * d_v + c0)[q] = val;
-            *rp = val;  // the next chunk forwards it
+            float4 a[2], raw[2];
+            float f[2];
+            float4* rp[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const float cf = s_sc[o[u]];
+                const float4 dd = reinterpret_cast<const float4*>(s_d + fW.div(o[u]) * CW)[q[u]];
+                a[u] = make_float4(cf * dd.x, cf * dd.y, cf * dd.z, cf * dd.w);
+                rp[u] = reinterpret_cast<float4*>(rows + wpos(o[u])) + q[u];
+                raw[u] = *rp[u];
+                f[u] = s_a[o[u]];
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                if (!own[u]) continue;
+                // the chunk's earlier writes of the slot, decayed to the chunk end
+                for (int L = lk_link(lk[u]); L >= 0; L = lk_link(s_wlk[L])) {
+                    const float cfa = s_sc[L];
+                    const float4 dd = reinterpret_cast<const float4*>(s_d + fW.div(L) * CW)[q[u]];
+                    a[u].x = fmaf(cfa, dd.x, a[u].x);
+                    a[u].y = fmaf(cfa, dd.y, a[u].y);
+                    a[u].z = fmaf(cfa, dd.z, a[u].z);
+                    a[u].w = fmaf(cfa, dd.w, a[u].w);
+                }
+                float4 val;
+                val.x = fmaf(f[u], raw[u].x, a[u].x);
+                val.y = fmaf(f[u], raw[u].y, a[u].y);
+                val.z = fmaf(f[u], raw[u].z, a[u].z);
+                val.w = fmaf(f[u], raw[u].w, a[u].w);
+                reinterpret_cast<float4*>(Mb + (size_t)sl[u] * d_v + c0)[q[u]] = val;
+                *rp[u] = val;  // the next chunk forwards it
+            }
         }
         // the stores precede the gathers that follow the next BAR_FIXED arrival
         __threadfence_block();
