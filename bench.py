@@ -35,8 +35,8 @@ L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 # the hash of the kernel sources it was taken with; None when not yet measured for the
 # current sources.  Filled from profiles/ (see the summary named there).
 MEASURED_TRAFFIC = {
-    # profiles/recur_run_kernel_mid_prefill.md: dram read 729.02 MB + write 407.74 MB
-    "d0d71db08613d40f": 1_136_753_664,
+    # profiles/recur_run_kernel_mid_prefill.md: dram read 728.66 MB + write 406.20 MB
+    "be658b80668ed88a": 1_134_859_520,
 }
 
 
