@@ -16,12 +16,41 @@
 namespace sdm {
 
 constexpr int DECODE_THREADS = 256;
+constexpr int DECODE_WARPS = DECODE_THREADS / 32;
 
+// Layout of one CTA: warp w owns write rows i = w, w+8, ... and read rows j = w, w+8, ...;
+// lane l owns the float4 columns q = l (+32) of d_v.  The rows live in registers: every
+// row load of a warp is issued before the first is used, and the cross-warp sums (p, then
+// the output) go through two [8][d_v] partial arrays in shared memory.  A read slot that is
+// also written this step takes the written row: its weight is added to that write row's
+// output weight (read slots are distinct, so at most one read lands on a write row).
 __host__ __device__ inline size_t decode_smem_bytes(int W, int R, int d_v) {
-    return (size_t)(W + R) * d_v * 4 + (size_t)d_v * 4 + (size_t)(W + R) * 4 * 3 + (size_t)R * 4;
+    return (size_t)2 * DECODE_WARPS * d_v * 4 + (size_t)(W + R) * 12 + (size_t)W * 4 +
+           (size_t)R * 4;
 }
 
 template <typename VT>
+SDM_DEV float4 load_v4(const VT* p);
+template <>
+SDM_DEV float4 load_v4<float>(const float* p) {
+    return __ldg(reinterpret_cast<const float4*>(p));
+}
+template <>
+SDM_DEV float4 load_v4<__nv_bfloat16>(const __nv_bfloat16* p) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                       __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+}
+
+SDM_DEV void fma4(float4& acc, float c, const float4& x) {
+    acc.x = fmaf(c, x.x, acc.x);
+    acc.y = fmaf(c, x.y, acc.y);
+    acc.z = fmaf(c, x.z, acc.z);
+    acc.w = fmaf(c, x.w, acc.w);
+}
+
+// RPW: rows of each role per warp (ceil(max(W, R) / 8)); QPL: float4 columns per lane.
+template <typename VT, int RPW, int QPL>
 __global__ void __launch_bounds__(DECODE_THREADS) decode_kernel(
     const VT* __restrict__ v, const float* __restrict__ alpha, const float* __restrict__ beta,
     const int32_t* __restrict__ widx, const float* __restrict__ ww,
@@ -31,25 +60,34 @@ __global__ void __launch_bounds__(DECODE_THREADS) decode_kernel(
     extern __shared__ __align__(16) unsigned char dec_smem[];
     const size_t bh = blockIdx.x;
     const int h = (int)(bh % H);
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int no = W + R;
     const int Q = d_v / 4;
-    float* s_rows = reinterpret_cast<float*>(dec_smem);        // [W+R][d_v]
-    float* s_d = s_rows + (size_t)no * d_v;                    // [d_v]
-    int* s_slot = reinterpret_cast<int*>(s_d + d_v);           // [W+R]
-    float* s_w = reinterpret_cast<float*>(s_slot + no);        // [W+R]
-    float* s_fe = s_w + no;                                    // [W+R], sign: pristine
-    int* s_match = reinterpret_cast<int*>(s_fe + no);          // [R]
+    float* s_pp = reinterpret_cast<float*>(dec_smem);              // [8][d_v] partial p
+    float* s_po = s_pp + DECODE_WARPS * d_v;                       // [8][d_v] partial out
+    int* s_slot = reinterpret_cast<int*>(s_po + DECODE_WARPS * d_v);  // [W+R]
+    float* s_w = reinterpret_cast<float*>(s_slot + no);            // [W+R]
+    float* s_f = s_w + no;                                         // [W+R], sign: pristine
+    float* s_uw = s_f + no;                                        // [W] read weight on row i
+    int* s_rm = reinterpret_cast<int*>(s_uw + W);                  // [R] read j is written
 
     float* Mb = M + bh * (size_t)N * d_v;
     const float* M0h = M0 + (size_t)h * N * d_v;
     double* stb = stamp + bh * (size_t)N;
     const float a = alpha[bh];
+    const float bt = beta[bh];
     double la = 0.0;
     if (a > 0.f) la = log((double)a);
     else if (tid == 0) raise_err(SDM_DEVERR_ALPHA);
     const double Lnew = lambda[bh] + la;
+    float4 vv[QPL];
+#pragma unroll
+    for (int c = 0; c < QPL; ++c) {
+        const int q = lane + 32 * c;
+        vv[c] = q < Q ? load_v4<VT>(v + bh * d_v + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 
+    // ---- slots, weights and decay factors seen at this step ------------------------------
     if (tid < no) {
         int s;
         float w;
@@ -70,62 +108,138 @@ __global__ void __launch_bounds__(DECODE_THREADS) decode_kernel(
         }
         s_slot[tid] = s;
         s_w[tid] = w;
-        s_fe[tid] = f;
+        s_f[tid] = f;
     }
     __syncthreads();
+
+    // ---- every row load of this warp in flight --------------------------------------------
+    float4 wr[RPW][QPL], rd[RPW][QPL];
+#pragma unroll
+    for (int k = 0; k < RPW; ++k) {
+        const int i = warp + DECODE_WARPS * k, j = i;
+        const int si = i < W ? s_slot[i] : -1;
+        const int sj = j < R ? s_slot[W + j] : -1;
+        const float* srci = (si >= 0 && signbit(s_f[i])) ? M0h : Mb;
+        const float* srcj = (sj >= 0 && signbit(s_f[W + j])) ? M0h : Mb;
+#pragma unroll
+        for (int c = 0; c < QPL; ++c) {
+            const int q = lane + 32 * c;
+            wr[k][c] = (si >= 0 && q < Q)
+                           ? __ldg(reinterpret_cast<const float4*>(srci + (size_t)si * d_v) + q)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            rd[k][c] = (sj >= 0 && q < Q)
+                           ? __ldg(reinterpret_cast<const float4*>(srcj + (size_t)sj * d_v) + q)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+
+    // ---- while they land: duplicate writes, reads of written slots --------------------------
     if (tid < W) {
         const int s = s_slot[tid];
-        for (int i = 0; i < tid; ++i)
-            if (s >= 0 && s_slot[i] == s) raise_err(SDM_DEVERR_DUP_WRITE);
-    }
-    if (tid < R) {
-        const int s = s_slot[W + tid];
-        int m = -1;
-        for (int i = 0; i < W; ++i)
-            if (s >= 0 && s_slot[i] == s) m = i;
-        s_match[tid] = m;
-    }
-    for (int e = tid; e < no * Q; e += DECODE_THREADS) {
-        const int o = e / Q, q = e % Q;
-        const int s = s_slot[o];
-        float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+        float uw = 0.f;
         if (s >= 0) {
-            const float* src = signbit(s_fe[o]) ? M0h : Mb;
-            val = reinterpret_cast<const float4*>(src + (size_t)s * d_v)[q];
+            for (int i = 0; i < tid; ++i)
+                if (s_slot[i] == s) raise_err(SDM_DEVERR_DUP_WRITE);
+            for (int j = 0; j < R; ++j)
+                if (s_slot[W + j] == s) uw += s_w[W + j];
         }
-        reinterpret_cast<float4*>(s_rows + (size_t)o * d_v)[q] = val;
+        s_uw[tid] = uw;
+    } else if (tid < no) {
+        const int s = s_slot[tid];
+        int m = 0;
+        if (s >= 0)
+            for (int i = 0; i < W; ++i) m |= s_slot[i] == s;
+        s_rm[tid - W] = m;
+    }
+
+    // ---- p = sum_i w_i seen(s_i) ------------------------------------------------------------
+    {
+        float4 pp[QPL];
+#pragma unroll
+        for (int c = 0; c < QPL; ++c) pp[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < RPW; ++k) {
+            const int i = warp + DECODE_WARPS * k;
+            if (i < W) {
+                const float cw = s_w[i] * fabsf(s_f[i]);
+#pragma unroll
+                for (int c = 0; c < QPL; ++c) fma4(pp[c], cw, wr[k][c]);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < QPL; ++c) {
+            const int q = lane + 32 * c;
+            if (q < Q) reinterpret_cast<float4*>(s_pp + warp * d_v)[q] = pp[c];
+        }
     }
     __syncthreads();
-    for (int c = tid; c < d_v; c += DECODE_THREADS) {
-        float p = 0.f;
-        for (int i = 0; i < W; ++i) p = fmaf(s_w[i] * fabsf(s_fe[i]), s_rows[(size_t)i * d_v + c], p);
-        s_d[c] = beta[bh] * (to_f32(v[bh * d_v + c]) - p);
-    }
-    __syncthreads();
-    for (int e = tid; e < W * Q; e += DECODE_THREADS) {
-        const int i = e / Q, q = e % Q;
-        const int s = s_slot[i];
-        const float f = fabsf(s_fe[i]), w = s_w[i];
-        float4 r = reinterpret_cast<const float4*>(s_rows + (size_t)i * d_v)[q];
-        const float4 dd = reinterpret_cast<const float4*>(s_d)[q];
-        r.x = fmaf(f, r.x, w * dd.x);
-        r.y = fmaf(f, r.y, w * dd.y);
-        r.z = fmaf(f, r.z, w * dd.z);
-        r.w = fmaf(f, r.w, w * dd.w);
-        reinterpret_cast<float4*>(s_rows + (size_t)i * d_v)[q] = r;  // now the written value
-        if (s >= 0) reinterpret_cast<float4*>(Mb + (size_t)s * d_v)[q] = r;
+
+    // ---- d = beta (v - p); written rows, stores, partial outputs --------------------------
+    {
+        float4 dd[QPL], po[QPL];
+#pragma unroll
+        for (int c = 0; c < QPL; ++c) {
+            const int q = lane + 32 * c;
+            float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (q < Q)
+#pragma unroll
+                for (int w2 = 0; w2 < DECODE_WARPS; ++w2) {
+                    const float4 t = reinterpret_cast<const float4*>(s_pp + w2 * d_v)[q];
+                    p.x += t.x;
+                    p.y += t.y;
+                    p.z += t.z;
+                    p.w += t.w;
+                }
+            dd[c] = make_float4(bt * (vv[c].x - p.x), bt * (vv[c].y - p.y), bt * (vv[c].z - p.z),
+                                bt * (vv[c].w - p.w));
+            po[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int k = 0; k < RPW; ++k) {
+            const int i = warp + DECODE_WARPS * k;
+            if (i < W) {
+                const int s = s_slot[i];
+                const float f = fabsf(s_f[i]), w = s_w[i], uw = s_uw[i];
+#pragma unroll
+                for (int c = 0; c < QPL; ++c) {
+                    const int q = lane + 32 * c;
+                    float4 r = wr[k][c];
+                    r.x = fmaf(f, r.x, w * dd[c].x);
+                    r.y = fmaf(f, r.y, w * dd[c].y);
+                    r.z = fmaf(f, r.z, w * dd[c].z);
+                    r.w = fmaf(f, r.w, w * dd[c].w);
+                    if (s >= 0 && q < Q) reinterpret_cast<float4*>(Mb + (size_t)s * d_v)[q] = r;
+                    fma4(po[c], uw, r);
+                }
+            }
+            const int j = i;
+            if (j < R && !s_rm[j]) {
+                const float cu = s_w[W + j] * fabsf(s_f[W + j]);
+#pragma unroll
+                for (int c = 0; c < QPL; ++c) fma4(po[c], cu, rd[k][c]);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < QPL; ++c) {
+            const int q = lane + 32 * c;
+            if (q < Q) reinterpret_cast<float4*>(s_po + warp * d_v)[q] = po[c];
+        }
     }
     if (tid < W && s_slot[tid] >= 0) stb[s_slot[tid]] = Lnew;
     __syncthreads();
-    for (int c = tid; c < d_v; c += DECODE_THREADS) {
-        float o = 0.f;
-        for (int j = 0; j < R; ++j) {
-            const int m = s_match[j];
-            const float val = m >= 0 ? s_rows[(size_t)m * d_v + c]
-                                     : fabsf(s_fe[W + j]) * s_rows[(size_t)(W + j) * d_v + c];
-            o = fmaf(s_w[W + j], val, o);
+
+    // ---- out = sum of the partial outputs ----------------------------------------------------
+    for (int q = tid; q < Q; q += DECODE_THREADS) {
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w2 = 0; w2 < DECODE_WARPS; ++w2) {
+            const float4 t = reinterpret_cast<const float4*>(s_po + w2 * d_v)[q];
+            o.x += t.x;
+            o.y += t.y;
+            o.z += t.z;
+            o.w += t.w;
         }
-        out[bh * d_v + c] = o;
+        reinterpret_cast<float4*>(out + bh * d_v)[q] = o;
     }
     if (tid == 0) lambda[bh] = Lnew;
 }

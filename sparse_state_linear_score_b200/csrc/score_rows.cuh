@@ -1,0 +1,547 @@
+// Product-key scoring with the latency of one row in mind: a decode step scores a single token
+// per (b,h), so a row cannot wait behind others in a thread's queue.  Each CTA takes
+// SROW_G rows of one head (and one role: blockIdx.z picks write or read, so a decode step
+// scores both roles in one launch).
+//
+// Same definition as the other scoring paths (§2 Background "Product Key Memory", §3 Method
+// "Sparse addressing", §4 "SDM Configuration"):
+//   s1[i] = <x[0:h], C1[i]>,  s2[j] = <x[h:2h], C2[j]>     (fp32 FMA, d ascending)
+//   the k_half best of each half, best first, ties to the lower sub-index
+//   the pairs (a, b) of the two lists with (a+1)(b+1) <= top ranked by s1[a] + s2[b], ties to
+//   the lower slot i*n + j; weights = softmax of the `top` selected sums.
+// Scores are ranked through an order-preserving u32 key (-0 joins +0, NaN ranks as -inf);
+// key 0 marks padding.
+//
+// Phases, all in one CTA of 8 warps:
+//   1. dot products: thread t takes sub-keys of one half for all SROW_G rows, so every
+//      sub-key element is loaded and widened once per CTA; the loads of a block of 32 (bf16)
+//      or 16 (fp32) elements are issued together (the first block before x is staged).
+//   2. per-half top-k: one warp per (row, half).
+//      k_half, top <= 32: the n scores form ceil(n/32) columns of 32 lanes.  A threshold
+//      that at least 32 scores reach (from each lane's second-largest) prunes them to
+//      about 50 candidates, which are compacted into two columns; each column is sorted by
+//      a bitonic network across the lanes and the two are merged (elementwise best
+//      against the reversed partner, then a bitonic merge) into the top 32 in order.
+//      up to 64: lane l sorts the block [l*PL, l*PL+PL) in registers and the warp takes
+//      k_half rounds of "best lane head" (redux.sync max, ballot, lowest lane among equal
+//      heads, whose block holds the lower sub-indices).
+//   3. combine, one warp per row.  <= 32: the staircase candidates (at most 119) form four
+//      columns and go through the same pruning, sort and merge.  Up to 64: lane l owns staircase
+//      columns b = l, l + 32, whose candidates are already sorted along a, and `top` rounds
+//      of best-head selection take them in order (equal sums: redux.sync min over slots).
+#pragma once
+
+#include <math.h>
+
+#include "common.cuh"
+
+namespace sdm {
+
+constexpr int SROW_THREADS = 256;
+constexpr int SROW_G = 4;  // rows per CTA: two warps per row in phase 2
+
+struct ScoreRowsArgs {
+    const void* x[2];
+    const void* sk[2];
+    int top[2];
+    int32_t* idx[2];
+    float* w[2];
+    int B, H, T, d_k, n, k_half;
+};
+
+// Strictly increasing map of the floats onto u32 with -0 joined to +0 and NaN ranked as -inf,
+// so unsigned comparison orders scores; 0 is left free for "no candidate".
+SDM_DEV uint32_t order_key(float v) {
+    if (v == 0.f) v = 0.f;
+    if (v != v) v = -INFINITY;
+    const uint32_t u = __float_as_uint(v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+SDM_DEV float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
+}
+
+// Eight consecutive sub-key elements, loaded raw and widened to fp32 at use.
+template <typename XT>
+struct Chunk8;
+template <>
+struct Chunk8<__nv_bfloat16> {
+    uint4 u;
+    SDM_DEV void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
+    SDM_DEV void widen(float* k) const {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            k[2 * i] = __uint_as_float(w[i] << 16);
+            k[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+};
+template <>
+struct Chunk8<float> {
+    float4 a, b;
+    SDM_DEV void load(const float* p) {
+        a = __ldg(reinterpret_cast<const float4*>(p));
+        b = __ldg(reinterpret_cast<const float4*>(p + 4));
+    }
+    SDM_DEV void widen(float* k) const {
+        k[0] = a.x; k[1] = a.y; k[2] = a.z; k[3] = a.w;
+        k[4] = b.x; k[5] = b.y; k[6] = b.z; k[7] = b.w;
+    }
+};
+
+// (key a, index ia) ranks before (key b, index ib)
+SDM_DEV bool kv_better(uint32_t ka, uint32_t ia, uint32_t kb, uint32_t ib) {
+    return ka > kb || (ka == kb && ia < ib);
+}
+
+// Sorts each of the C columns (one register across the 32 lanes) best first: bitonic network,
+// lane pairs at distance j exchange through shuffles; in a pair the lane that keeps the
+// better element is the lower one in descending runs and the upper one in ascending runs.
+template <int C>
+SDM_DEV void column_sort(uint32_t (&k)[C], uint32_t (&id)[C], int lane) {
+#pragma unroll
+    for (int kk = 2; kk <= 32; kk <<= 1) {
+#pragma unroll
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+            const bool keep_better = ((lane & kk) == 0) == ((lane & j) == 0);
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                const uint32_t pk = __shfl_xor_sync(0xffffffffu, k[c], j);
+                const uint32_t pi = __shfl_xor_sync(0xffffffffu, id[c], j);
+                if (keep_better == kv_better(pk, pi, k[c], id[c])) {
+                    k[c] = pk;
+                    id[c] = pi;
+                }
+            }
+        }
+    }
+}
+
+// (ka, ia) <- the best 32 of two columns sorted best first, sorted best first: the
+// elementwise better of a and the reversed b is a bitonic sequence holding the best 32,
+// which a bitonic merge orders.
+SDM_DEV void column_merge(uint32_t& ka, uint32_t& ia, uint32_t kb, uint32_t ib, int lane) {
+    const uint32_t rk = __shfl_sync(0xffffffffu, kb, 31 - lane);
+    const uint32_t ri = __shfl_sync(0xffffffffu, ib, 31 - lane);
+    if (kv_better(rk, ri, ka, ia)) {
+        ka = rk;
+        ia = ri;
+    }
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) {
+        const bool keep_better = (lane & j) == 0;
+        const uint32_t pk = __shfl_xor_sync(0xffffffffu, ka, j);
+        const uint32_t pi = __shfl_xor_sync(0xffffffffu, ia, j);
+        if (keep_better == kv_better(pk, pi, ka, ia)) {
+            ka = pk;
+            ia = pi;
+        }
+    }
+}
+
+// Column 0 <- the best 32 of all C columns (C a power of two), in order.
+template <int C>
+SDM_DEV void top32_columns(uint32_t (&k)[C], uint32_t (&id)[C], int lane) {
+    column_sort<C>(k, id, lane);
+#pragma unroll
+    for (int st = 1; st < C; st <<= 1)
+#pragma unroll
+        for (int c = 0; c < C; c += 2 * st) column_merge(k[c], id[c], k[c + st], id[c + st], lane);
+}
+
+// (k0, i0) <- the best 32 of the C columns, in order, through a pruned candidate set: tau is
+// the 16th largest over the lanes of each lane's second-largest key, so at least 16 lanes
+// hold two keys >= tau and at least 32 keys are >= tau -- tau is at most the 32nd key, and
+// every element that can rank in the best 32 (ties included) passes.  When at most 64 pass
+// (nearly always for continuous scores) they are compacted into `scratch` (64 entries) and
+// sorted as two columns; otherwise all C columns are sorted.
+template <int C>
+SDM_DEV void top32_pruned(uint32_t (&k)[C], uint32_t (&id)[C], int2* scratch, int lane,
+                          uint32_t& k0, uint32_t& i0) {
+    uint32_t m1 = 0u, m2 = 0u;
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        m2 = max(m2, min(m1, k[c]));
+        m1 = max(m1, k[c]);
+    }
+#pragma unroll
+    for (int kk = 2; kk <= 32; kk <<= 1) {
+#pragma unroll
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+            const bool keep_larger = ((lane & kk) == 0) == ((lane & j) == 0);
+            const uint32_t p = __shfl_xor_sync(0xffffffffu, m2, j);
+            m2 = keep_larger ? max(m2, p) : min(m2, p);
+        }
+    }
+    const uint32_t tau = __shfl_sync(0xffffffffu, m2, 15);
+    const uint32_t below = (1u << lane) - 1u;
+    int m = 0;
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        const bool in = k[c] >= tau;
+        const uint32_t bal = __ballot_sync(0xffffffffu, in);
+        const int pos = m + __popc(bal & below);
+        if (in && pos < 64) scratch[pos] = make_int2((int)k[c], (int)id[c]);
+        m += __popc(bal);
+    }
+    if (m <= 64) {
+        __syncwarp();
+        uint32_t kk2[2], ii2[2];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const int e = c * 32 + lane;
+            if (e < m) {
+                const int2 v = scratch[e];
+                kk2[c] = (uint32_t)v.x;
+                ii2[c] = (uint32_t)v.y;
+            } else {
+                kk2[c] = 0u;
+                ii2[c] = 0x7fffff00u + (uint32_t)e;  // padding, distinct from every index
+            }
+        }
+        __syncwarp();  // scratch is free again
+        top32_columns<2>(kk2, ii2, lane);
+        k0 = kk2[0];
+        i0 = ii2[0];
+    } else {
+        top32_columns<C>(k, id, lane);
+        k0 = k[0];
+        i0 = id[0];
+    }
+}
+
+__host__ __device__ inline size_t srow_align16(size_t b) { return (b + 15) & ~(size_t)15; }
+
+constexpr int SROW_CAND = 128;  // staircase candidates when k_half, top <= 32 (at most 119)
+
+// Shared memory: x rows, the (row, half) score segments (reused for the sorted lane lists
+// of the wide variant), the per-half lists, the selected pairs and the staircase table.
+__host__ __device__ inline size_t score_rows_smem_bytes(int d_k, int PL, int KP) {
+    return srow_align16((size_t)SROW_G * d_k * 4) + (size_t)SROW_G * 2 * 32 * PL * 8 +
+           (size_t)SROW_G * 2 * KP * 8 + (size_t)SROW_G * KP * 8 + SROW_CAND * 4 + 16;
+}
+
+template <typename XT, int PL, int KP>
+__global__ void __launch_bounds__(SROW_THREADS, 3) score_rows_kernel(ScoreRowsArgs a) {
+    constexpr int NP = 32 * PL;    // sub-keys per half, padded to whole lanes
+    constexpr int CPL = KP / 32;   // staircase columns per lane (wide variant)
+    constexpr int NB = sizeof(XT) == 2 ? 4 : 2;  // 8-element chunks per load block
+    extern __shared__ __align__(16) unsigned char srow_smem[];
+    const int role = blockIdx.z;
+    const XT* __restrict__ x = static_cast<const XT*>(role ? a.x[1] : a.x[0]);
+    const XT* __restrict__ sk = static_cast<const XT*>(role ? a.sk[1] : a.sk[0]);
+    const int top = role ? a.top[1] : a.top[0];
+    int32_t* __restrict__ idx_out = role ? a.idx[1] : a.idx[0];
+    float* __restrict__ w_out = role ? a.w[1] : a.w[0];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.y, d_k = a.d_k, hd = d_k >> 1, n = a.n, kh = a.k_half;
+    const long long rows = (long long)a.B * a.T;
+    const long long r0 = (long long)blockIdx.x * SROW_G;
+
+    float* xs = reinterpret_cast<float*>(srow_smem);  // [G][d_k]
+    unsigned char* segs = srow_smem + srow_align16((size_t)SROW_G * d_k * 4);
+    float* tv = reinterpret_cast<float*>(segs + (size_t)SROW_G * 2 * NP * 8);  // [G][2][KP]
+    int* ti = reinterpret_cast<int*>(tv + SROW_G * 2 * KP);                     // [G][2][KP]
+    float* sv = reinterpret_cast<float*>(ti + SROW_G * 2 * KP);                 // [G][KP]
+    uint32_t* ss = reinterpret_cast<uint32_t*>(sv + SROW_G * KP);               // [G][KP]
+    int* cand = reinterpret_cast<int*>(ss + SROW_G * KP);                       // [SROW_CAND]
+    int* ncand = cand + SROW_CAND;
+
+    // ---- 1a. first sub-key block in flight while x is staged -----------------------------
+    const int hf1 = tid >> 7, j1 = tid & 127;  // threads 0..127 half 0, 128..255 half 1
+    const XT* tab = sk + (size_t)(h * 2 + hf1) * n * hd;
+    Chunk8<XT> r0c[NB], r1c[NB];
+    auto load_block = [&](int s0, int d0) {
+        const int s1 = s0 + 128 < n ? s0 + 128 : s0;
+#pragma unroll
+        for (int c = 0; c < NB; ++c)
+            if (d0 + 8 * c < hd) {
+                r0c[c].load(tab + (size_t)s0 * hd + d0 + 8 * c);
+                r1c[c].load(tab + (size_t)s1 * hd + d0 + 8 * c);
+            }
+    };
+    if (j1 < n) load_block(j1, 0);
+
+    // ---- 0. x rows (zeros past the last row); the staircase table ------------------------
+    for (int i = tid; i < SROW_G * d_k; i += SROW_THREADS) {
+        const int g = i / d_k, c = i - g * d_k;
+        const long long r = r0 + g;
+        float v = 0.f;
+        if (r < rows) {
+            const long long b = r / a.T, t = r - b * a.T;
+            v = to_f32(x[(((size_t)b * a.H + h) * a.T + t) * d_k + c]);
+        }
+        xs[i] = v;
+    }
+    if (KP == 32 && warp == SROW_THREADS / 32 - 1) {
+        // pairs (a, b) with (a+1)(b+1) <= top, a, b < k_half <= 32, row by row
+        int base = 0;
+        for (int a0 = 0; a0 < kh; ++a0) {
+            const int m = min(kh, top / (a0 + 1));
+            if (m <= 0) break;
+            if (lane < m) cand[base + lane] = (a0 << 8) | lane;
+            base += m;
+        }
+        if (lane == 0) *ncand = base;
+    }
+    __syncthreads();
+
+    // ---- 1b. dot products: sub-keys j, j + 128 (then + 256, + 384) of this thread's half --
+    {
+        const float* xh = xs + hf1 * hd;
+        for (int s0 = j1; s0 < n; s0 += 256) {
+            const int s1 = s0 + 128;
+            float acc0[SROW_G], acc1[SROW_G];
+#pragma unroll
+            for (int g = 0; g < SROW_G; ++g) acc0[g] = acc1[g] = 0.f;
+            for (int d0 = 0; d0 < hd; d0 += 8 * NB) {
+                if (d0 > 0) load_block(s0, d0);
+#pragma unroll
+                for (int c = 0; c < NB; ++c) {
+                    if (d0 + 8 * c >= hd) break;
+                    float k0[8], k1[8];
+                    r0c[c].widen(k0);
+                    r1c[c].widen(k1);
+                    const int d = d0 + 8 * c;
+#pragma unroll
+                    for (int g = 0; g < SROW_G; ++g) {
+                        const float4 xa = *reinterpret_cast<const float4*>(xh + g * d_k + d);
+                        const float4 xb = *reinterpret_cast<const float4*>(xh + g * d_k + d + 4);
+                        const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            acc0[g] = fmaf(xv[e], k0[e], acc0[g]);
+                            acc1[g] = fmaf(xv[e], k1[e], acc1[g]);
+                        }
+                    }
+                }
+            }
+            if (s0 + 256 < n) load_block(s0 + 256, 0);
+#pragma unroll
+            for (int g = 0; g < SROW_G; ++g) {
+                float* scf = reinterpret_cast<float*>(segs + (size_t)(g * 2 + hf1) * NP * 8);
+                scf[s0] = acc0[g];
+                if (s1 < n) scf[s1] = acc1[g];
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- 2. per-half top-k: warp (g, hf) ---------------------------------------------------
+    {
+        const int g = warp >> 1, hf = warp & 1;
+        const float* scf = reinterpret_cast<const float*>(segs + (size_t)(g * 2 + hf) * NP * 8);
+        float* tvo = tv + (g * 2 + hf) * KP;
+        int* tio = ti + (g * 2 + hf) * KP;
+        if constexpr (KP == 32) {
+            uint32_t key[PL], id[PL];
+#pragma unroll
+            for (int c = 0; c < PL; ++c) {
+                const int i = c * 32 + lane;
+                id[c] = (uint32_t)i;
+                key[c] = i < n ? order_key(scf[i]) : 0u;
+            }
+            uint32_t bk, bi;
+            if constexpr (PL <= 2) {
+                top32_columns<PL>(key, id, lane);
+                bk = key[0];
+                bi = id[0];
+            } else {  // the segment's second half (NP * 4 >= 512 bytes) is the scratch
+                int2* scr = reinterpret_cast<int2*>(segs + (size_t)(g * 2 + hf) * NP * 8 + NP * 4);
+                top32_pruned<PL>(key, id, scr, lane, bk, bi);
+            }
+            if (lane < kh) {
+                tvo[lane] = key_value(bk);
+                tio[lane] = (int)bi;
+            }
+        } else {
+            uint32_t key[PL];
+            int id[PL];
+#pragma unroll
+            for (int r = 0; r < PL; ++r) {
+                const int i = lane * PL + r;
+                id[r] = i;
+                key[r] = i < n ? order_key(scf[i]) : 0u;
+            }
+            // bitonic sort of the lane's block, best first (key desc, sub-index asc)
+#pragma unroll
+            for (int k = 2; k <= PL; k <<= 1) {
+#pragma unroll
+                for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll
+                    for (int i = 0; i < PL; ++i) {
+                        const int l = i ^ j;
+                        if (l > i) {
+                            const bool l_better =
+                                key[l] > key[i] || (key[l] == key[i] && id[l] < id[i]);
+                            if (((i & k) == 0) == l_better) {
+                                const uint32_t tk = key[i];
+                                key[i] = key[l];
+                                key[l] = tk;
+                                const int tix = id[i];
+                                id[i] = id[l];
+                                id[l] = tix;
+                            }
+                        }
+                    }
+                }
+            }
+            __syncwarp();  // every lane has read its scores: the segment now holds the lists
+            int2* lst = reinterpret_cast<int2*>(segs + (size_t)(g * 2 + hf) * NP * 8);  // [32][PL]
+#pragma unroll
+            for (int r = 2; r < PL; ++r) lst[lane * PL + r] = make_int2((int)key[r], id[r]);
+            __syncwarp();
+            uint32_t hk = key[0];
+            int hi = id[0];
+            uint32_t nk = PL > 1 ? key[PL > 1 ? 1 : 0] : 0u;
+            int ni = PL > 1 ? id[PL > 1 ? 1 : 0] : 0;
+            int p = 1;  // position of (nk, ni) in the lane's list
+            for (int q = 0; q < kh; ++q) {
+                const uint32_t mx = __reduce_max_sync(0xffffffffu, hk);
+                const uint32_t bal = __ballot_sync(0xffffffffu, hk == mx);
+                if (lane == __ffs(bal) - 1) {
+                    tvo[q] = key_value(hk);
+                    tio[q] = hi;
+                    hk = nk;
+                    hi = ni;
+                    ++p;
+                    if (p < PL) {
+                        const int2 e = lst[lane * PL + p];
+                        nk = (uint32_t)e.x;
+                        ni = e.y;
+                    } else {
+                        nk = 0u;
+                        ni = 0;
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- 3. combine and softmax: warp g --------------------------------------------------
+    if (warp >= SROW_G || r0 + warp >= rows) return;
+    const int g = warp;
+    const float* t1 = tv + (g * 2) * KP;
+    const int* i1 = ti + (g * 2) * KP;
+    const float* t2 = tv + (g * 2 + 1) * KP;
+    const int* i2 = ti + (g * 2 + 1) * KP;
+    const long long r = r0 + g;
+    const long long b = r / a.T, t = r - b * a.T;
+    const size_t row_off = ((size_t)b * a.H + h) * a.T + t;
+    if constexpr (KP == 32) {
+        constexpr int C = SROW_CAND / 32;
+        const int nc = *ncand;
+        uint32_t key[C], id[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            const int e = c * 32 + lane;
+            if (e < nc) {
+                const int pr = cand[e], pa = pr >> 8, pb = pr & 255;
+                key[c] = order_key(t1[pa] + t2[pb]);
+                id[c] = (uint32_t)i1[pa] * (uint32_t)n + (uint32_t)i2[pb];
+            } else {
+                key[c] = 0u;
+                id[c] = 0x40000000u + (uint32_t)e;  // padding, distinct from every slot
+            }
+        }
+        uint32_t bk, bi;
+        if (nc <= 64) {
+            uint32_t k2[2] = {key[0], key[1]}, i2c[2] = {id[0], id[1]};
+            top32_columns<2>(k2, i2c, lane);
+            bk = k2[0];
+            bi = i2c[0];
+        } else {  // scratch: the second half of the row's first score segment (free by now)
+            int2* scr = reinterpret_cast<int2*>(segs + (size_t)(g * 2) * NP * 8 + NP * 4);
+            top32_pruned<C>(key, id, scr, lane, bk, bi);
+        }
+        const float v = key_value(bk);
+        const float mx = __shfl_sync(0xffffffffu, v, 0);
+        const float ex = lane < top ? expf(v - mx) : 0.f;
+        float z = ex;
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) z += __shfl_xor_sync(0xffffffffu, z, m);
+        if (lane < top) {
+            idx_out[row_off * top + lane] = (int32_t)bi;
+            w_out[row_off * top + lane] = ex / z;
+        }
+    } else {
+        float* svo = sv + g * KP;
+        uint32_t* sso = ss + g * KP;
+        int ca[CPL], lim[CPL];
+        float v2[CPL], cv[CPL];
+        uint32_t j2[CPL], ck[CPL], cs[CPL];
+        auto head = [&](int c) {
+            if (ca[c] < lim[c]) {
+                cv[c] = t1[ca[c]] + v2[c];
+                ck[c] = order_key(cv[c]);
+                cs[c] = (uint32_t)i1[ca[c]] * (uint32_t)n + j2[c];
+            } else {
+                ck[c] = 0u;
+                cs[c] = 0xffffffffu;
+            }
+        };
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            const int bcol = lane + 32 * c;
+            ca[c] = 0;
+            lim[c] = bcol < kh ? min(kh, top / (bcol + 1)) : 0;
+            v2[c] = bcol < kh ? t2[bcol] : 0.f;
+            j2[c] = bcol < kh ? (uint32_t)i2[bcol] : 0u;
+            head(c);
+        }
+        for (int q = 0; q < top; ++q) {
+            uint32_t bk = ck[0], bs = cs[0];
+            float bv = cv[0];
+            int bc = 0;
+#pragma unroll
+            for (int c = 1; c < CPL; ++c)
+                if (ck[c] > bk || (ck[c] == bk && cs[c] < bs)) {
+                    bk = ck[c];
+                    bs = cs[c];
+                    bv = cv[c];
+                    bc = c;
+                }
+            const uint32_t mx = __reduce_max_sync(0xffffffffu, bk);
+            const bool eq = bk == mx;
+            uint32_t bal = __ballot_sync(0xffffffffu, eq);
+            if (__popc(bal) > 1) {  // equal sums: the lower slot first
+                const uint32_t ms = __reduce_min_sync(0xffffffffu, eq ? bs : 0xffffffffu);
+                bal = __ballot_sync(0xffffffffu, eq && bs == ms);
+            }
+            if (lane == __ffs(bal) - 1) {
+                svo[q] = bv;
+                sso[q] = bs;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c)
+                    if (c == bc) {
+                        ++ca[c];
+                        head(c);
+                    }
+            }
+        }
+        __syncwarp();
+        const float mx = svo[0];
+        float ex[CPL], z = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            const int q = lane + 32 * c;
+            ex[c] = q < top ? expf(svo[q] - mx) : 0.f;
+            z += ex[c];
+        }
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) z += __shfl_xor_sync(0xffffffffu, z, m);
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            const int q = lane + 32 * c;
+            if (q < top) {
+                idx_out[row_off * top + q] = (int32_t)sso[q];
+                w_out[row_off * top + q] = ex[c] / z;
+            }
+        }
+    }
+}
+
+}  // namespace sdm

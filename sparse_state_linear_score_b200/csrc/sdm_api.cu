@@ -10,6 +10,7 @@
 #include "decode.cuh"
 #include "plan.cuh"
 #include "recur.cuh"
+#include "score_rows.cuh"
 #include "score_simt.cuh"
 #include "score_tc.cuh"
 #include "state.cuh"
@@ -216,11 +217,79 @@ sdm_status launch_score_tc(const sdm_dims* d, const void* x, const void* sk, int
     return launch_score_tc_t<32>(d, xm, km, a, grid, s);
 }
 
+// The row scorer keeps a lane's block of n/32 half-scores in registers (at most 16) and the
+// selected lists in shared memory; check_dims already bounds k_half and top by 64 and makes
+// the half width a multiple of 8.
+bool score_rows_eligible(const sdm_dims* d) { return d->n_sub <= 32 * 16; }
+
+template <typename XT, int PL>
+sdm_status launch_score_rows_t(const ScoreRowsArgs& a, int kp, dim3 grid, cudaStream_t s) {
+    if (kp <= 32) {
+        auto kern = score_rows_kernel<XT, PL, 32>;
+        const size_t smem = score_rows_smem_bytes(a.d_k, PL, 32);
+        if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
+        kern<<<grid, SROW_THREADS, smem, s>>>(a);
+    } else {
+        auto kern = score_rows_kernel<XT, PL, 64>;
+        const size_t smem = score_rows_smem_bytes(a.d_k, PL, 64);
+        if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
+        kern<<<grid, SROW_THREADS, smem, s>>>(a);
+    }
+    return launch_status();
+}
+
+template <typename XT>
+sdm_status launch_score_rows_x(const ScoreRowsArgs& a, int kp, dim3 grid, cudaStream_t s) {
+    const int pl = (a.n + 31) / 32;
+    if (pl <= 1) return launch_score_rows_t<XT, 1>(a, kp, grid, s);
+    if (pl <= 2) return launch_score_rows_t<XT, 2>(a, kp, grid, s);
+    if (pl <= 4) return launch_score_rows_t<XT, 4>(a, kp, grid, s);
+    if (pl <= 8) return launch_score_rows_t<XT, 8>(a, kp, grid, s);
+    return launch_score_rows_t<XT, 16>(a, kp, grid, s);
+}
+
+// One launch for `roles` (1 or 2) scorings of the same shape: role r scores x[r] against
+// sk[r] into idx[r], w[r] with top[r] slots.
+sdm_status launch_score_rows(const sdm_dims* d, int roles, const void* const* x,
+                             const void* const* sk, const int* top, int32_t* const* idx,
+                             float* const* w, cudaStream_t s) {
+    ScoreRowsArgs a{};
+    int kp = d->k_half;
+    for (int r = 0; r < 2; ++r) {
+        const int q = r < roles ? r : 0;
+        a.x[r] = x[q];
+        a.sk[r] = sk[q];
+        a.top[r] = top[q];
+        a.idx[r] = idx[q];
+        a.w[r] = w[q];
+        if (top[q] > kp) kp = top[q];
+    }
+    a.B = d->B; a.H = d->H; a.T = d->T; a.d_k = d->d_k; a.n = d->n_sub; a.k_half = d->k_half;
+    const long long rows = (long long)d->B * d->T;
+    const dim3 grid((unsigned)((rows + SROW_G - 1) / SROW_G), (unsigned)d->H, (unsigned)roles);
+    if (d->x_dtype == SDM_F32) return launch_score_rows_x<float>(a, kp, grid, s);
+    return launch_score_rows_x<__nv_bfloat16>(a, kp, grid, s);
+}
+
+template <typename VT, int RPW, int QPL>
+sdm_status launch_decode(const sdm_dims* d, const void* v, const float* alpha, const float* beta,
+                         const sdm_state* st, const int32_t* widx, const float* ww,
+                         const int32_t* ridx, const float* rw, float* out, sdm_stream_t stream) {
+    auto kern = decode_kernel<VT, RPW, QPL>;
+    const size_t smem = decode_smem_bytes(d->W, d->R, d->d_v);
+    if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
+    kern<<<(unsigned)BH_of(d), DECODE_THREADS, smem, (cudaStream_t)stream>>>(
+        (const VT*)v, alpha, beta, widx, ww, ridx, rw, st->M, st->stamp, st->Lambda, st->M0, out,
+        d->H, (int)N_of(d), d->d_v, d->W, d->R);
+    return launch_status();
+}
+
 sdm_status launch_score(const sdm_dims* d, const void* x, const void* sk, int top, int32_t* idx,
                         float* w, cudaStream_t s) {
     const long long rows = (long long)d->B * d->T;
     if (rows == 0) return SDM_OK;
     if (score_tc_eligible(d, top)) return launch_score_tc(d, x, sk, top, idx, w, s);
+    if (score_rows_eligible(d)) return launch_score_rows(d, 1, &x, &sk, &top, &idx, &w, s);
     const int threads = 128, warps = threads / 32;
     const size_t smem =
         (size_t)warps * score_simt_warp_floats(d->d_k, d->n_sub, d->k_half, top) * sizeof(float);
@@ -467,8 +536,19 @@ sdm_status sdm_prefill(const sdm_dims* dims, const void* q, const void* k, const
         return SDM_ERR_ARG;
     const WsLayout L = ws_layout(dims);
     if (!ws || ws_bytes < L.total) return SDM_ERR_WORKSPACE;
-    if ((e = sdm_score_topk(dims, k, skw, dims->W, widx, ww, stream))) return e;
-    if ((e = sdm_score_topk(dims, q, skr, dims->R, ridx, rw, stream))) return e;
+    if (score_rows_eligible(dims) && aligned16(q) && aligned16(k) && aligned16(skw) &&
+        aligned16(skr) && aligned16(widx) && aligned16(ww) && aligned16(ridx) && aligned16(rw)) {
+        // both roles in one launch (grid.z = role)
+        const void* xs[2] = {k, q};
+        const void* sks[2] = {skw, skr};
+        const int tops[2] = {dims->W, dims->R};
+        int32_t* idxs[2] = {widx, ridx};
+        float* ws[2] = {ww, rw};
+        if ((e = launch_score_rows(dims, 2, xs, sks, tops, idxs, ws, stream))) return e;
+    } else {
+        if ((e = sdm_score_topk(dims, k, skw, dims->W, widx, ww, stream))) return e;
+        if ((e = sdm_score_topk(dims, q, skr, dims->R, ridx, rw, stream))) return e;
+    }
     return sdm_forward(dims, v, alpha, beta, widx, ww, ridx, rw, st, out, ws, ws_bytes, stream);
 }
 
@@ -486,20 +566,20 @@ sdm_status sdm_decode_step(const sdm_dims* dims, const void* q, const void* k, c
         return SDM_ERR_ALIGN;
     if ((e = sdm_score_topk(dims, k, skw, dims->W, widx, ww, stream))) return e;
     if ((e = sdm_score_topk(dims, q, skr, dims->R, ridx, rw, stream))) return e;
-    const size_t smem = decode_smem_bytes(dims->W, dims->R, dims->d_v);
-    const unsigned grid = (unsigned)BH_of(dims);
+    const int rpw = ((dims->W > dims->R ? dims->W : dims->R) + DECODE_WARPS - 1) / DECODE_WARPS;
+    const int qpl = (dims->d_v / 4 + 31) / 32;
     if (dims->v_dtype == SDM_BF16) {
-        if (!set_smem(decode_kernel<__nv_bfloat16>, smem)) return SDM_ERR_CUDA;
-        decode_kernel<__nv_bfloat16><<<grid, DECODE_THREADS, smem, stream>>>(
-            (const __nv_bfloat16*)v, alpha, beta, widx, ww, ridx, rw, st->M, st->stamp,
-            st->Lambda, st->M0, out, dims->H, (int)N_of(dims), dims->d_v, dims->W, dims->R);
+        if (rpw <= 4) e = qpl <= 1 ? launch_decode<__nv_bfloat16, 4, 1>(dims, v, alpha, beta, st, widx, ww, ridx, rw, out, stream)
+                                   : launch_decode<__nv_bfloat16, 4, 2>(dims, v, alpha, beta, st, widx, ww, ridx, rw, out, stream);
+        else e = qpl <= 1 ? launch_decode<__nv_bfloat16, 8, 1>(dims, v, alpha, beta, st, widx, ww, ridx, rw, out, stream)
+                          : launch_decode<__nv_bfloat16, 8, 2>(dims, v, alpha, beta, st, widx, ww, ridx, rw, out, stream);
     } else {
-        if (!set_smem(decode_kernel<float>, smem)) return SDM_ERR_CUDA;
-        decode_kernel<float><<<grid, DECODE_THREADS, smem, stream>>>(
-            (const float*)v, alpha, beta, widx, ww, ridx, rw, st->M, st->stamp, st->Lambda,
-            st->M0, out, dims->H, (int)N_of(dims), dims->d_v, dims->W, dims->R);
+        if (rpw <= 4) e = qpl <= 1 ? launch_decode<float, 4, 1>(dims, v, alpha, beta, st, widx, ww, ridx, rw, out, stream)
+                                   : launch_decode<float, 4, 2>(dims, v, alpha, beta, st, widx, ww, ridx, rw, out, stream);
+        else e = qpl <= 1 ? launch_decode<float, 8, 1>(dims, v, alpha, beta, st, widx, ww, ridx, rw, out, stream)
+                          : launch_decode<float, 8, 2>(dims, v, alpha, beta, st, widx, ww, ridx, rw, out, stream);
     }
-    return launch_status();
+    return e;
 }
 
 sdm_status sdm_forward_noalloc(const sdm_dims* dims, const void* v, const float* alpha,

@@ -278,6 +278,7 @@ def test_decode_vs_oracle(sdm, orc):
     for s, (wi, wv, ri, rv) in enumerate(sels):
         t = T0 + s
         check_selection(orc, inp["k"][:, :, t:t + 1], inp["skw"], wi, wv, wl.k_half, wl.W, wl.n_sub)
+        check_selection(orc, inp["q"][:, :, t:t + 1], inp["skr"], ri, rv, wl.k_half, wl.R, wl.n_sub)
     for b in range(wl.B):
         for h in range(wl.H):
             widx = np.concatenate([w0[b, h].cpu().numpy()] + [x[0][b, h].cpu().numpy() for x in sels])
@@ -443,6 +444,12 @@ def test_full_decode(sdm, orc):
         rws[s].copy_(sel[3].view(wl.B, wl.H, wl.R))
     torch.cuda.synchronize()
     assert sdm.device_error() == 0
+    # every row's selection of both roles at the first and the last step
+    for s in (0, steps - 1):
+        for x, sk, top, gi, gw in ((kd[s], inp["skw"], wl.W, wsel[s], wws[s]),
+                                   (qd[s], inp["skr"], wl.R, rsel[s], rws[s])):
+            check_selection(orc, x.unsqueeze(2), sk, gi.unsqueeze(2), gw.unsqueeze(2), wl.k_half,
+                            top, wl.n_sub)
     b, h = 5, 7
     widx = np.concatenate([sel0[0][b, h].cpu().numpy(), wsel[:, b, h].cpu().numpy()])
     ww = np.concatenate([f64(sel0[1][b, h]), f64(wws[:, b, h])])
