@@ -74,18 +74,24 @@ __global__ void __launch_bounds__(DECODE_THREADS) decode_kernel(
     float* Mb = M + bh * (size_t)N * d_v;
     const float* M0h = M0 + (size_t)h * N * d_v;
     double* stb = stamp + bh * (size_t)N;
-    const float a = alpha[bh];
+    // inputs that do not come from the scoring launch before this one: read them while it
+    // finishes (programmatic dependent launch), then wait for its indices and weights
     const float bt = beta[bh];
-    double la = 0.0;
-    if (a > 0.f) la = log((double)a);
-    else if (tid == 0) raise_err(SDM_DEVERR_ALPHA);
-    const double Lnew = lambda[bh] + la;
     float4 vv[QPL];
 #pragma unroll
     for (int c = 0; c < QPL; ++c) {
         const int q = lane + 32 * c;
         vv[c] = q < Q ? load_v4<VT>(v + bh * d_v + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    double Lnew = 0.0;  // Lambda' (needed by the threads that own a slot, and by thread 0)
+    if (tid < (no > 32 ? no : 32)) {
+        const float a = alpha[bh];
+        double la = 0.0;
+        if (a > 0.f) la = log((double)a);
+        else if (tid == 0) raise_err(SDM_DEVERR_ALPHA);
+        Lnew = lambda[bh] + la;
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // ---- slots, weights and decay factors seen at this step ------------------------------
     if (tid < no) {
@@ -137,12 +143,18 @@ __global__ void __launch_bounds__(DECODE_THREADS) decode_kernel(
     if (tid < W) {
         const int s = s_slot[tid];
         float uw = 0.f;
-        if (s >= 0) {
+        if (W <= 32) {  // the write slots are the lanes of warp 0
+            const unsigned lanes = W == 32 ? 0xffffffffu : (1u << W) - 1u;
+            const unsigned same = __match_any_sync(lanes, s);
+            if (s >= 0 && __popc(same) > 1 && (int)(__ffs(same) - 1) == tid)
+                raise_err(SDM_DEVERR_DUP_WRITE);
+        } else if (s >= 0) {
             for (int i = 0; i < tid; ++i)
                 if (s_slot[i] == s) raise_err(SDM_DEVERR_DUP_WRITE);
+        }
+        if (s >= 0)
             for (int j = 0; j < R; ++j)
                 if (s_slot[W + j] == s) uw += s_w[W + j];
-        }
         s_uw[tid] = uw;
     } else if (tid < no) {
         const int s = s_slot[tid];

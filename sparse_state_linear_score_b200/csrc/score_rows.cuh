@@ -40,6 +40,8 @@ namespace sdm {
 constexpr int SROW_THREADS = 256;
 constexpr int SROW_G = 4;  // rows per CTA: two warps per row in phase 2
 
+constexpr int SROW_CAND = 128;  // staircase candidates when k_half, top <= 32 (at most 119)
+
 struct ScoreRowsArgs {
     const void* x[2];
     const void* sk[2];
@@ -47,7 +49,20 @@ struct ScoreRowsArgs {
     int32_t* idx[2];
     float* w[2];
     int B, H, T, d_k, n, k_half;
+    // per role, when k_half, top <= 32: the pairs (a, b) with (a+1)(b+1) <= top, a, b < k_half,
+    // as (a << 8) | b, and their count
+    uint16_t cand[2][SROW_CAND];
+    int ncand[2];
 };
+
+// The staircase pairs of one role (host side; the same for every row).
+inline int score_rows_staircase(int k_half, int top, uint16_t* cand) {
+    int m = 0;
+    for (int a0 = 0; a0 < k_half; ++a0)
+        for (int b0 = 0; b0 < k_half && (a0 + 1) * (b0 + 1) <= top; ++b0)
+            if (m < SROW_CAND) cand[m++] = (uint16_t)((a0 << 8) | b0);
+    return m;
+}
 
 // Strictly increasing map of the floats onto u32 with -0 joined to +0 and NaN ranked as -inf,
 // so unsigned comparison orders scores; 0 is left free for "no candidate".
@@ -214,8 +229,6 @@ SDM_DEV void top32_pruned(uint32_t (&k)[C], uint32_t (&id)[C], int2* scratch, in
 
 __host__ __device__ inline size_t srow_align16(size_t b) { return (b + 15) & ~(size_t)15; }
 
-constexpr int SROW_CAND = 128;  // staircase candidates when k_half, top <= 32 (at most 119)
-
 // Shared memory: x rows, the (row, half) score segments (reused for the sorted lane lists
 // of the wide variant), the per-half lists, the selected pairs and the staircase table.
 __host__ __device__ inline size_t score_rows_smem_bytes(int d_k, int PL, int KP) {
@@ -224,10 +237,10 @@ __host__ __device__ inline size_t score_rows_smem_bytes(int d_k, int PL, int KP)
 }
 
 template <typename XT, int PL, int KP>
-__global__ void __launch_bounds__(SROW_THREADS, 3) score_rows_kernel(ScoreRowsArgs a) {
+__global__ void __launch_bounds__(SROW_THREADS, 4) score_rows_kernel(ScoreRowsArgs a) {
     constexpr int NP = 32 * PL;    // sub-keys per half, padded to whole lanes
     constexpr int CPL = KP / 32;   // staircase columns per lane (wide variant)
-    constexpr int NB = sizeof(XT) == 2 ? 4 : 2;  // 8-element chunks per load block
+    constexpr int NB = 2;  // 8-element chunks per load block
     extern __shared__ __align__(16) unsigned char srow_smem[];
     const int role = blockIdx.z;
     const XT* __restrict__ x = static_cast<const XT*>(role ? a.x[1] : a.x[0]);
@@ -235,6 +248,8 @@ __global__ void __launch_bounds__(SROW_THREADS, 3) score_rows_kernel(ScoreRowsAr
     const int top = role ? a.top[1] : a.top[0];
     int32_t* __restrict__ idx_out = role ? a.idx[1] : a.idx[0];
     float* __restrict__ w_out = role ? a.w[1] : a.w[0];
+    // a launch that reads this one's outputs may start now and wait for them itself
+    asm volatile("griddepcontrol.launch_dependents;");
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.y, d_k = a.d_k, hd = d_k >> 1, n = a.n, kh = a.k_half;
     const long long rows = (long long)a.B * a.T;
@@ -248,6 +263,11 @@ __global__ void __launch_bounds__(SROW_THREADS, 3) score_rows_kernel(ScoreRowsAr
     uint32_t* ss = reinterpret_cast<uint32_t*>(sv + SROW_G * KP);               // [G][KP]
     int* cand = reinterpret_cast<int*>(ss + SROW_G * KP);                       // [SROW_CAND]
     int* ncand = cand + SROW_CAND;
+    // element offset of row r = b*T + t in the [B,H,T,.] tensors: (b*H + h)*T + t
+    auto row_off = [&](long long r) -> size_t {
+        const long long b = a.T == 1 ? r : r / a.T;
+        return ((size_t)b * a.H + h) * a.T + (size_t)(r - b * a.T);
+    };
 
     // ---- 1a. first sub-key block in flight while x is staged -----------------------------
     const int hf1 = tid >> 7, j1 = tid & 127;  // threads 0..127 half 0, 128..255 half 1
@@ -265,26 +285,15 @@ __global__ void __launch_bounds__(SROW_THREADS, 3) score_rows_kernel(ScoreRowsAr
     if (j1 < n) load_block(j1, 0);
 
     // ---- 0. x rows (zeros past the last row); the staircase table ------------------------
-    for (int i = tid; i < SROW_G * d_k; i += SROW_THREADS) {
-        const int g = i / d_k, c = i - g * d_k;
-        const long long r = r0 + g;
-        float v = 0.f;
-        if (r < rows) {
-            const long long b = r / a.T, t = r - b * a.T;
-            v = to_f32(x[(((size_t)b * a.H + h) * a.T + t) * d_k + c]);
-        }
-        xs[i] = v;
+#pragma unroll
+    for (int g = 0; g < SROW_G; ++g) {
+        const bool live = r0 + g < rows;
+        for (int c = tid; c < d_k; c += SROW_THREADS)
+            xs[g * d_k + c] = live ? to_f32(x[row_off(r0 + g) * d_k + c]) : 0.f;
     }
-    if (KP == 32 && warp == SROW_THREADS / 32 - 1) {
-        // pairs (a, b) with (a+1)(b+1) <= top, a, b < k_half <= 32, row by row
-        int base = 0;
-        for (int a0 = 0; a0 < kh; ++a0) {
-            const int m = min(kh, top / (a0 + 1));
-            if (m <= 0) break;
-            if (lane < m) cand[base + lane] = (a0 << 8) | lane;
-            base += m;
-        }
-        if (lane == 0) *ncand = base;
+    if (KP == 32 && tid < SROW_CAND) {
+        cand[tid] = role ? a.cand[1][tid] : a.cand[0][tid];
+        if (tid == 0) *ncand = role ? a.ncand[1] : a.ncand[0];
     }
     __syncthreads();
 
@@ -428,9 +437,7 @@ __global__ void __launch_bounds__(SROW_THREADS, 3) score_rows_kernel(ScoreRowsAr
     const int* i1 = ti + (g * 2) * KP;
     const float* t2 = tv + (g * 2 + 1) * KP;
     const int* i2 = ti + (g * 2 + 1) * KP;
-    const long long r = r0 + g;
-    const long long b = r / a.T, t = r - b * a.T;
-    const size_t row_off = ((size_t)b * a.H + h) * a.T + t;
+    const size_t ro = row_off(r0 + g);
     if constexpr (KP == 32) {
         constexpr int C = SROW_CAND / 32;
         const int nc = *ncand;
@@ -464,8 +471,8 @@ __global__ void __launch_bounds__(SROW_THREADS, 3) score_rows_kernel(ScoreRowsAr
 #pragma unroll
         for (int m = 16; m > 0; m >>= 1) z += __shfl_xor_sync(0xffffffffu, z, m);
         if (lane < top) {
-            idx_out[row_off * top + lane] = (int32_t)bi;
-            w_out[row_off * top + lane] = ex / z;
+            idx_out[ro * top + lane] = (int32_t)bi;
+            w_out[ro * top + lane] = ex / z;
         }
     } else {
         float* svo = sv + g * KP;
@@ -473,16 +480,6 @@ __global__ void __launch_bounds__(SROW_THREADS, 3) score_rows_kernel(ScoreRowsAr
         int ca[CPL], lim[CPL];
         float v2[CPL], cv[CPL];
         uint32_t j2[CPL], ck[CPL], cs[CPL];
-        auto head = [&](int c) {
-            if (ca[c] < lim[c]) {
-                cv[c] = t1[ca[c]] + v2[c];
-                ck[c] = order_key(cv[c]);
-                cs[c] = (uint32_t)i1[ca[c]] * (uint32_t)n + j2[c];
-            } else {
-                ck[c] = 0u;
-                cs[c] = 0xffffffffu;
-            }
-        };
 #pragma unroll
         for (int c = 0; c < CPL; ++c) {
             const int bcol = lane + 32 * c;
@@ -490,8 +487,20 @@ __global__ void __launch_bounds__(SROW_THREADS, 3) score_rows_kernel(ScoreRowsAr
             lim[c] = bcol < kh ? min(kh, top / (bcol + 1)) : 0;
             v2[c] = bcol < kh ? t2[bcol] : 0.f;
             j2[c] = bcol < kh ? (uint32_t)i2[bcol] : 0u;
-            head(c);
         }
+        auto head = [&](int c) {
+            if (ca[c] < lim[c]) {
+                cv[c] = t1[ca[c]] + v2[c];
+                ck[c] = order_key(cv[c]);
+                cs[c] = (uint32_t)i1[ca[c]] * (uint32_t)n + j2[c];
+            } else {
+                cv[c] = 0.f;
+                ck[c] = 0u;
+                cs[c] = 0xffffffffu;
+            }
+        };
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) head(c);
         for (int q = 0; q < top; ++q) {
             uint32_t bk = ck[0], bs = cs[0];
             float bv = cv[0];
@@ -537,8 +546,8 @@ __global__ void __launch_bounds__(SROW_THREADS, 3) score_rows_kernel(ScoreRowsAr
         for (int c = 0; c < CPL; ++c) {
             const int q = lane + 32 * c;
             if (q < top) {
-                idx_out[row_off * top + q] = (int32_t)sso[q];
-                w_out[row_off * top + q] = ex[c] / z;
+                idx_out[ro * top + q] = (int32_t)sso[q];
+                w_out[ro * top + q] = ex[c] / z;
             }
         }
     }

@@ -262,6 +262,7 @@ sdm_status launch_score_rows(const sdm_dims* d, int roles, const void* const* x,
         a.top[r] = top[q];
         a.idx[r] = idx[q];
         a.w[r] = w[q];
+        a.ncand[r] = score_rows_staircase(d->k_half, top[q], a.cand[r]);
         if (top[q] > kp) kp = top[q];
     }
     a.B = d->B; a.H = d->H; a.T = d->T; a.d_k = d->d_k; a.n = d->n_sub; a.k_half = d->k_half;
@@ -278,9 +279,22 @@ sdm_status launch_decode(const sdm_dims* d, const void* v, const float* alpha, c
     auto kern = decode_kernel<VT, RPW, QPL>;
     const size_t smem = decode_smem_bytes(d->W, d->R, d->d_v);
     if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
-    kern<<<(unsigned)BH_of(d), DECODE_THREADS, smem, (cudaStream_t)stream>>>(
-        (const VT*)v, alpha, beta, widx, ww, ridx, rw, st->M, st->stamp, st->Lambda, st->M0, out,
-        d->H, (int)N_of(d), d->d_v, d->W, d->R);
+    // programmatic dependent launch: the kernel may start while the scoring launch before it
+    // finishes; it reads that launch's outputs only after griddepcontrol.wait
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)BH_of(d));
+    cfg.blockDim = dim3(DECODE_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = (cudaStream_t)stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, (const VT*)v, alpha, beta, widx, ww, ridx, rw, st->M,
+                           st->stamp, st->Lambda, (const float*)st->M0, out, d->H, (int)N_of(d),
+                           d->d_v, d->W, d->R) != cudaSuccess)
+        return SDM_ERR_CUDA;
     return launch_status();
 }
 
