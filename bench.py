@@ -339,6 +339,9 @@ def run_gpu(args, wl, world, rank, local):
     e2e = run_e2e(args, wl, d, inp, st, sel, out, ws, device, sdm)
     errs = sdm.device_error()
 
+    # the decode workload (single-token steps), on rank 0
+    dec = run_decode(device, sdm) if rank == 0 and not args.no_decode else None
+
     if world > 1:
         dist.barrier(device_ids=[device.index])
         dist.destroy_process_group()
@@ -386,6 +389,7 @@ def run_gpu(args, wl, world, rank, local):
         "e2e": e2e,
         "diagnostics": diag,
         "layer_out": layer,
+        "decode": dec,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "device_errors": errs,
@@ -393,6 +397,62 @@ def run_gpu(args, wl, world, rank, local):
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     return line
+
+
+def run_decode(device, sdm, steps: int = 64, warm: int = 3) -> dict:
+    """The decode workload at full size: a 512-token seeded prefill of every (b,h), then
+    `steps` timed single-token steps (sdm_decode_step: one scoring launch for both roles and
+    one recurrence launch each) on tokens after the warm-up.  The 34 GB state is far
+    larger than L2, and every step gathers new random rows of it."""
+    import torch
+
+    import sdm_synth as S
+
+    wl = S.DECODE.scaled(decode_steps=warm + steps)
+    inp = S.generate(wl, device=device)
+    d = sdm.Dims(wl.B, wl.H, wl.T, wl.d_k, wl.n_sub, wl.d_v, wl.k_half, wl.W, wl.R, wl.x_dtype,
+                 wl.v_dtype)
+    dd = sdm.Dims(wl.B, wl.H, 1, wl.d_k, wl.n_sub, wl.d_v, wl.k_half, wl.W, wl.R, wl.x_dtype,
+                  wl.v_dtype)
+    st = sdm.State(d, inp["M0"])
+    sdm.state_reset(d, st)
+    sl = lambda x: x[:, :, :wl.T].contiguous()
+    sdm.prefill(d, sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["alpha"]), sl(inp["beta"]),
+                inp["skw"], inp["skr"], st)
+    qd, kd, vd = (S.decode_layout(inp[k], wl.T) for k in ("q", "k", "v"))
+    ad, bd = (S.decode_layout(inp[k], wl.T) for k in ("alpha", "beta"))
+    sel = sdm.selection_buffers(dd, device)
+    out = torch.empty((wl.B, wl.H, wl.d_v), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+    for s in range(warm):
+        sdm.decode_step(dd, qd[s], kd[s], vd[s], ad[s], bd[s], inp["skw"], inp["skr"], st,
+                        sel=sel, out=out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(warm, warm + steps):
+        sdm.decode_step(dd, qd[s], kd[s], vd[s], ad[s], bd[s], inp["skw"], inp["skr"], st,
+                        sel=sel, out=out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    errs = sdm.device_error()
+    us = e0.elapsed_time(e1) * 1e3 / steps
+    rows = wl.B * wl.H
+    bpt = bytes_per_token_head(wl)
+    step_bytes = (bpt["step"] + (2 * wl.W + wl.R) * 8) * rows  # + stamp reads and writes
+    gbs = step_bytes / (us / 1e6) / 1e9
+    peak = measured_peaks()["hbm_gbs"]
+    res = {"workload": f"decode: B={wl.B} H={wl.H} d_k={wl.d_k} n={wl.n_sub} N={wl.N} "
+                       f"d_v={wl.d_v} k={wl.k_half} W={wl.W} R={wl.R} after a {wl.T}-token prefill",
+           "steps_timed": steps, "us_per_step": us, "token_heads_per_s": rows / (us / 1e6),
+           "gpu_launches_per_step": 2,
+           "roofline": {"bound": "hbm", "algorithmic_bytes_per_step": step_bytes,
+                        "achieved_gbs": gbs, "peak": peak, "frac": gbs / peak},
+           "note": "state 34 GB (fp32 rows) >> L2; each step scores new tokens, so its gathers "
+                   "miss L2", "device_errors": errs}
+    del inp, st, qd, kd, vd, ad, bd, sel, out
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_e2e(args, wl, d, inp, st, sel, out, ws, device, sdm):
@@ -562,6 +622,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="mid_prefill")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the decode-workload measurement (rank 0)")
     args = ap.parse_args(argv)
     world, rank, local = dist_env()
     if world != args.gpus and "WORLD_SIZE" in os.environ:
