@@ -106,6 +106,7 @@ def lib_path() -> str:
 
 
 def _ptr(t: torch.Tensor | None, what: str, dtype=None):
+    """Device address of a contiguous CUDA tensor (an int: the argtypes convert it)."""
     if t is None:
         return None
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
@@ -114,12 +115,20 @@ def _ptr(t: torch.Tensor | None, what: str, dtype=None):
         raise ValueError(f"{what} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
-    return ctypes.c_void_p(t.data_ptr())
+    return t.data_ptr()
+
+
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+_cur_device = getattr(torch._C, "_cuda_getDevice", None)
 
 
 def _stream(stream=None):
-    s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+    """cudaStream_t of `stream`, else of the current stream (without building a Stream)."""
+    if stream is not None:
+        return stream.cuda_stream
+    if _raw_stream is not None and _cur_device is not None:
+        return _raw_stream(_cur_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _ok(status: int, what: str):

@@ -83,8 +83,8 @@ __global__ void __launch_bounds__(DECODE_THREADS) decode_kernel(
         const int q = lane + 32 * c;
         vv[c] = q < Q ? load_v4<VT>(v + bh * d_v + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    double Lnew = 0.0;  // Lambda' (needed by the threads that own a slot, and by thread 0)
-    if (tid < (no > 32 ? no : 32)) {
+    double Lnew;  // Lambda'
+    {
         const float a = alpha[bh];
         double la = 0.0;
         if (a > 0.f) la = log((double)a);
@@ -93,40 +93,42 @@ __global__ void __launch_bounds__(DECODE_THREADS) decode_kernel(
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // ---- slots, weights and decay factors seen at this step ------------------------------
-    if (tid < no) {
-        int s;
-        float w;
-        if (tid < W) {
-            s = widx[bh * W + tid];
-            w = ww[bh * W + tid];
-        } else {
-            s = ridx[bh * R + (tid - W)];
-            w = rw[bh * R + (tid - W)];
+    // ---- this warp's rows: lane k fetches write row w + 8k, lane 16 + k read row w + 8k
+    //      (slot, weight, decay factor from the stamp), the warp shares them by shuffles and
+    //      puts every row load in flight before the first block barrier --------------------
+    int my_s = -1;
+    float my_f = 0.f;
+    {
+        const bool rl = lane >= 16;
+        const int k = lane & 15, i = warp + DECODE_WARPS * k;
+        if (k < RPW && i < (rl ? R : W)) {
+            int sl = rl ? ridx[bh * R + i] : widx[bh * W + i];
+            const float w = rl ? rw[bh * R + i] : ww[bh * W + i];
+            float f = 0.f;
+            if (!slot_ok(sl, N)) {
+                raise_err(SDM_DEVERR_SLOT_RANGE);
+                sl = -1;
+            } else {
+                const double st = stb[sl];
+                f = isnan(st) ? -(float)exp(Lnew) : (float)exp(Lnew - st);
+            }
+            my_s = sl;
+            my_f = f;
+            const int o = rl ? W + i : i;
+            s_slot[o] = sl;
+            s_w[o] = w;
+            s_f[o] = f;
         }
-        float f = 0.f;
-        if (!slot_ok(s, N)) {
-            raise_err(SDM_DEVERR_SLOT_RANGE);
-            s = -1;
-        } else {
-            const double st = stb[s];
-            f = isnan(st) ? -(float)exp(Lnew) : (float)exp(Lnew - st);
-        }
-        s_slot[tid] = s;
-        s_w[tid] = w;
-        s_f[tid] = f;
     }
-    __syncthreads();
-
-    // ---- every row load of this warp in flight --------------------------------------------
     float4 wr[RPW][QPL], rd[RPW][QPL];
 #pragma unroll
     for (int k = 0; k < RPW; ++k) {
-        const int i = warp + DECODE_WARPS * k, j = i;
-        const int si = i < W ? s_slot[i] : -1;
-        const int sj = j < R ? s_slot[W + j] : -1;
-        const float* srci = (si >= 0 && signbit(s_f[i])) ? M0h : Mb;
-        const float* srcj = (sj >= 0 && signbit(s_f[W + j])) ? M0h : Mb;
+        const int si = __shfl_sync(0xffffffffu, my_s, k);
+        const int sj = __shfl_sync(0xffffffffu, my_s, 16 + k);
+        const float fi = __shfl_sync(0xffffffffu, my_f, k);
+        const float fj = __shfl_sync(0xffffffffu, my_f, 16 + k);
+        const float* srci = (si >= 0 && signbit(fi)) ? M0h : Mb;
+        const float* srcj = (sj >= 0 && signbit(fj)) ? M0h : Mb;
 #pragma unroll
         for (int c = 0; c < QPL; ++c) {
             const int q = lane + 32 * c;
@@ -138,6 +140,7 @@ __global__ void __launch_bounds__(DECODE_THREADS) decode_kernel(
                            : make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
+    __syncthreads();  // every warp's slots are in shared memory
 
     // ---- while they land: duplicate writes, reads of written slots --------------------------
     if (tid < W) {
