@@ -31,9 +31,11 @@
 //      of best-head selection take them in order (equal sums: redux.sync min over slots).
 #pragma once
 
+#include <cuda.h>
 #include <math.h>
 
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace sdm {
 
@@ -229,18 +231,36 @@ SDM_DEV void top32_pruned(uint32_t (&k)[C], uint32_t (&id)[C], int2* scratch, in
 
 __host__ __device__ inline size_t srow_align16(size_t b) { return (b + 15) & ~(size_t)15; }
 
-// Shared memory: x rows, the (row, half) score segments (reused for the sorted lane lists
-// of the wide variant), the per-half lists, the selected pairs and the staircase table.
-__host__ __device__ inline size_t score_rows_smem_bytes(int d_k, int PL, int KP) {
-    return srow_align16((size_t)SROW_G * d_k * 4) + (size_t)SROW_G * 2 * 32 * PL * 8 +
-           (size_t)SROW_G * 2 * KP * 8 + (size_t)SROW_G * KP * 8 + SROW_CAND * 4 + 16;
+// Tensor-core dot products (bf16, d_k = 128): 128-sub-key chunks of the head's table stream
+// through two TMA buffers (128-byte swizzle) and the x rows form a 16-row operand, so each
+// chunk is one M=128, N=16, K=64 product into 16 TMEM columns (lane = sub-key, column = row).
+constexpr uint32_t SROW_TC_KBUF = 16384;                 // one chunk: 128 rows x 128 B
+constexpr uint32_t SROW_TC_XT = 2 * SROW_TC_KBUF;        // x: 2 halves x 16 rows x 128 B
+constexpr uint32_t SROW_TC_CTRL = SROW_TC_XT + 4096;     // mbarriers, TMEM address, abort
+constexpr uint32_t SROW_TC_HEAD = SROW_TC_CTRL + 64;     // the common area starts here
+
+// Bytes of one (row, half) score segment: the scores, then the 64-entry scratch of the
+// pruned selection (k_half, top <= 32), or the sorted lane lists (up to 64).
+__host__ __device__ inline size_t score_rows_seg_bytes(int PL, int KP) {
+    return KP == 32 ? (size_t)32 * PL * 4 + 512 : (size_t)32 * PL * 8;
 }
 
-template <typename XT, int PL, int KP>
-__global__ void __launch_bounds__(SROW_THREADS, 4) score_rows_kernel(ScoreRowsArgs a) {
+// Shared memory: x rows (CUDA-core dots) or the tensor-core staging (plus 1 KB for its
+// alignment), the score segments, the per-half lists, the selected pairs, the staircase.
+__host__ __device__ inline size_t score_rows_smem_bytes(int d_k, int PL, int KP, bool tcd) {
+    const size_t head = tcd ? SROW_TC_HEAD + 1024 : srow_align16((size_t)SROW_G * d_k * 4);
+    return head + (size_t)SROW_G * 2 * score_rows_seg_bytes(PL, KP) + (size_t)SROW_G * 2 * KP * 8 +
+           (size_t)SROW_G * KP * 8 + SROW_CAND * 4 + 16;
+}
+
+template <typename XT, int PL, int KP, bool TCD>
+__global__ void __launch_bounds__(SROW_THREADS, 4) score_rows_kernel(
+    const __grid_constant__ CUtensorMap km0, const __grid_constant__ CUtensorMap km1,
+    ScoreRowsArgs a) {
     constexpr int NP = 32 * PL;    // sub-keys per half, padded to whole lanes
     constexpr int CPL = KP / 32;   // staircase columns per lane (wide variant)
     constexpr int NB = 2;  // 8-element chunks per load block
+    constexpr size_t SEG = KP == 32 ? NP * 4 + 512 : NP * 8;
     extern __shared__ __align__(16) unsigned char srow_smem[];
     const int role = blockIdx.z;
     const XT* __restrict__ x = static_cast<const XT*>(role ? a.x[1] : a.x[0]);
@@ -255,9 +275,12 @@ __global__ void __launch_bounds__(SROW_THREADS, 4) score_rows_kernel(ScoreRowsAr
     const long long rows = (long long)a.B * a.T;
     const long long r0 = (long long)blockIdx.x * SROW_G;
 
-    float* xs = reinterpret_cast<float*>(srow_smem);  // [G][d_k]
-    unsigned char* segs = srow_smem + srow_align16((size_t)SROW_G * d_k * 4);
-    float* tv = reinterpret_cast<float*>(segs + (size_t)SROW_G * 2 * NP * 8);  // [G][2][KP]
+    unsigned char* base = srow_smem;
+    if constexpr (TCD) base += (1024 - (ptx::smem_u32(srow_smem) & 1023)) & 1023;
+    float* xs = reinterpret_cast<float*>(base);  // [G][d_k] (CUDA-core dots)
+    unsigned char* segs =
+        base + (TCD ? (size_t)SROW_TC_HEAD : srow_align16((size_t)SROW_G * d_k * 4));
+    float* tv = reinterpret_cast<float*>(segs + (size_t)SROW_G * 2 * SEG);      // [G][2][KP]
     int* ti = reinterpret_cast<int*>(tv + SROW_G * 2 * KP);                     // [G][2][KP]
     float* sv = reinterpret_cast<float*>(ti + SROW_G * 2 * KP);                 // [G][KP]
     uint32_t* ss = reinterpret_cast<uint32_t*>(sv + SROW_G * KP);               // [G][KP]
@@ -269,79 +292,187 @@ __global__ void __launch_bounds__(SROW_THREADS, 4) score_rows_kernel(ScoreRowsAr
         return ((size_t)b * a.H + h) * a.T + (size_t)(r - b * a.T);
     };
 
-    // ---- 1a. first sub-key block in flight while x is staged -----------------------------
-    const int hf1 = tid >> 7, j1 = tid & 127;  // threads 0..127 half 0, 128..255 half 1
-    const XT* tab = sk + (size_t)(h * 2 + hf1) * n * hd;
-    Chunk8<XT> r0c[NB], r1c[NB];
-    auto load_block = [&](int s0, int d0) {
-        const int s1 = s0 + 128 < n ? s0 + 128 : s0;
-#pragma unroll
-        for (int c = 0; c < NB; ++c)
-            if (d0 + 8 * c < hd) {
-                r0c[c].load(tab + (size_t)s0 * hd + d0 + 8 * c);
-                r1c[c].load(tab + (size_t)s1 * hd + d0 + 8 * c);
+    if constexpr (TCD) {
+        // ---- 1. tensor-core dot products ----------------------------------------------------
+        constexpr uint32_t TCOLS = 2 * ((NP + 127) / 128) * 16 <= 32
+                                       ? 32
+                                       : (2 * ((NP + 127) / 128) * 16 <= 64 ? 64 : 128);
+        uint64_t* bar_tma = reinterpret_cast<uint64_t*>(base + SROW_TC_CTRL);  // [2]
+        uint64_t* bar_mma = bar_tma + 2;                                       // [2]
+        uint64_t* bar_done = bar_mma + 2;
+        uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_done + 1);
+        int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+        const CUtensorMap* km = role ? &km1 : &km0;
+        const int cph = (n + 127) / 128, nch = 2 * cph;  // chunks per half, in all
+        auto chunk_row = [&](int c) { return (h * 2 + c / cph) * n + (c % cph) * 128; };
+        if (warp == 0) ptx::tmem_alloc(tmem_slot, TCOLS);
+        if (tid == 0) {
+            for (int i = 0; i < 2; ++i) {
+                ptx::mbar_init(bar_tma + i, 1);
+                ptx::mbar_init(bar_mma + i, 1);
             }
-    };
-    if (j1 < n) load_block(j1, 0);
+            ptx::mbar_init(bar_done, 1);
+            *abort_flag = 0;
+            ptx::fence_mbar_init();
+            for (int c = 0; c < 2 && c < nch; ++c) {
+                ptx::mbar_arrive_expect_tx(bar_tma + c, SROW_TC_KBUF);
+                ptx::tma_load_2d(base + c * SROW_TC_KBUF, km, 0, chunk_row(c), bar_tma + c);
+            }
+        }
+        {   // x operand: thread t writes 16 bytes of half t/128, row (t/8)%16 (zero past the
+            // CTA's rows), swizzled: 16-byte chunk index XOR row % 8
+            const int hx = tid >> 7, row = (tid >> 3) & 15, ch = tid & 7;
+            uint4 val = make_uint4(0u, 0u, 0u, 0u);
+            if (row < SROW_G && r0 + row < rows)
+                val = __ldg(reinterpret_cast<const uint4*>(x + row_off(r0 + row) * 128 + hx * 64 +
+                                                           ch * 8));
+            *reinterpret_cast<uint4*>(base + SROW_TC_XT + hx * 2048 + row * 128 +
+                                      ((ch ^ (row & 7)) << 4)) = val;
+        }
+        if (KP == 32 && tid < SROW_CAND) {
+            cand[tid] = role ? a.cand[1][tid] : a.cand[0][tid];
+            if (tid == 0) *ncand = role ? a.ncand[1] : a.ncand[0];
+        }
+        ptx::fence_proxy_async_smem();  // the x operand is read by the tensor cores
+        ptx::tc_fence_before();
+        __syncthreads();
+        ptx::tc_fence_after();
+        const uint32_t tmem = *tmem_slot;
+        const uint64_t deadline = ptx::globaltimer_ns() + 2000000000ull;
+        if (tid == 0) {
+            const uint32_t idesc = ptx::idesc_bf16_f32(128, 16);
+            bool ok = true;
+            for (int c = 0; c < nch && ok; ++c) {
+                const int bf = c & 1;
+                const uint32_t par = (uint32_t)(c >> 1) & 1u;
+                if (!ptx::mbar_wait_bounded(bar_tma + bf, par, deadline)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint64_t ad = ptx::umma_desc_kmajor_sw128(base + bf * SROW_TC_KBUF);
+                const uint64_t bd = ptx::umma_desc_kmajor_sw128(base + SROW_TC_XT + (c / cph) * 2048);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)  // K = 64 in steps of 16 (32 bytes)
+                    ptx::umma_bf16(tmem + 16u * (uint32_t)c, ad + 2 * k, bd + 2 * k, idesc,
+                                   k > 0 ? 1u : 0u);
+                ptx::umma_commit(bar_mma + bf);
+                if (c + 2 < nch) {  // buffer bf is free once this chunk's products are done
+                    if (!ptx::mbar_wait_bounded(bar_mma + bf, par, deadline)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::mbar_arrive_expect_tx(bar_tma + bf, SROW_TC_KBUF);
+                    ptx::tma_load_2d(base + bf * SROW_TC_KBUF, km, 0, chunk_row(c + 2), bar_tma + bf);
+                }
+            }
+            if (ok) {
+                ptx::umma_commit(bar_done);
+            } else {
+                *abort_flag = 1;
+                raise_err(SDM_DEVERR_TIMEOUT);
+            }
+        }
+        __syncthreads();  // thread 0 has issued everything (or given up)
+        bool aborted = *abort_flag != 0;
+        if (!aborted && !ptx::mbar_wait_bounded(bar_done, 0u, deadline)) {
+            aborted = true;
+            if (tid == 0) raise_err(SDM_DEVERR_TIMEOUT);
+        }
+        ptx::tc_fence_after();
+        if (!aborted) {  // warp w reads TMEM lanes 32 (w % 4) .. + 31 of every other chunk
+            const int q = warp & 3;
+            for (int c = warp >> 2; c < nch; c += 2) {
+                float v[4];
+                ptx::tmem_ld4(tmem + ((uint32_t)(32 * q) << 16) + 16u * (uint32_t)c, v);
+                const int hf = c / cph, sidx = (c % cph) * 128 + 32 * q + lane;
+                if (sidx < n)
+#pragma unroll
+                    for (int g = 0; g < SROW_G; ++g)
+                        reinterpret_cast<float*>(segs + (size_t)(g * 2 + hf) * SEG)[sidx] = v[g];
+            }
+        }
+        ptx::tc_fence_before();
+        __syncthreads();
+        if (warp == 0) {
+            ptx::tc_fence_after();
+            ptx::tmem_dealloc(tmem, TCOLS);
+        }
+    } else {
+        // ---- 1a. first sub-key block in flight while x is staged -----------------------------
+        const int hf1 = tid >> 7, j1 = tid & 127;  // threads 0..127 half 0, 128..255 half 1
+        const XT* tab = sk + (size_t)(h * 2 + hf1) * n * hd;
+        Chunk8<XT> r0c[NB], r1c[NB];
+        auto load_block = [&](int s0, int d0) {
+            const int s1 = s0 + 128 < n ? s0 + 128 : s0;
+    #pragma unroll
+            for (int c = 0; c < NB; ++c)
+                if (d0 + 8 * c < hd) {
+                    r0c[c].load(tab + (size_t)s0 * hd + d0 + 8 * c);
+                    r1c[c].load(tab + (size_t)s1 * hd + d0 + 8 * c);
+                }
+        };
+        if (j1 < n) load_block(j1, 0);
 
-    // ---- 0. x rows (zeros past the last row); the staircase table ------------------------
-#pragma unroll
-    for (int g = 0; g < SROW_G; ++g) {
-        const bool live = r0 + g < rows;
-        for (int c = tid; c < d_k; c += SROW_THREADS)
-            xs[g * d_k + c] = live ? to_f32(x[row_off(r0 + g) * d_k + c]) : 0.f;
-    }
-    if (KP == 32 && tid < SROW_CAND) {
-        cand[tid] = role ? a.cand[1][tid] : a.cand[0][tid];
-        if (tid == 0) *ncand = role ? a.ncand[1] : a.ncand[0];
-    }
-    __syncthreads();
+        // ---- 0. x rows (zeros past the last row); the staircase table ------------------------
+    #pragma unroll
+        for (int g = 0; g < SROW_G; ++g) {
+            const bool live = r0 + g < rows;
+            for (int c = tid; c < d_k; c += SROW_THREADS)
+                xs[g * d_k + c] = live ? to_f32(x[row_off(r0 + g) * d_k + c]) : 0.f;
+        }
+        if (KP == 32 && tid < SROW_CAND) {
+            cand[tid] = role ? a.cand[1][tid] : a.cand[0][tid];
+            if (tid == 0) *ncand = role ? a.ncand[1] : a.ncand[0];
+        }
+        __syncthreads();
 
-    // ---- 1b. dot products: sub-keys j, j + 128 (then + 256, + 384) of this thread's half --
-    {
-        const float* xh = xs + hf1 * hd;
-        for (int s0 = j1; s0 < n; s0 += 256) {
-            const int s1 = s0 + 128;
-            float acc0[SROW_G], acc1[SROW_G];
-#pragma unroll
-            for (int g = 0; g < SROW_G; ++g) acc0[g] = acc1[g] = 0.f;
-            for (int d0 = 0; d0 < hd; d0 += 8 * NB) {
-                if (d0 > 0) load_block(s0, d0);
-#pragma unroll
-                for (int c = 0; c < NB; ++c) {
-                    if (d0 + 8 * c >= hd) break;
-                    float k0[8], k1[8];
-                    r0c[c].widen(k0);
-                    r1c[c].widen(k1);
-                    const int d = d0 + 8 * c;
-#pragma unroll
-                    for (int g = 0; g < SROW_G; ++g) {
-                        const float4 xa = *reinterpret_cast<const float4*>(xh + g * d_k + d);
-                        const float4 xb = *reinterpret_cast<const float4*>(xh + g * d_k + d + 4);
-                        const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            acc0[g] = fmaf(xv[e], k0[e], acc0[g]);
-                            acc1[g] = fmaf(xv[e], k1[e], acc1[g]);
+        // ---- 1b. dot products: sub-keys j, j + 128 (then + 256, + 384) of this thread's half --
+        {
+            const float* xh = xs + hf1 * hd;
+            for (int s0 = j1; s0 < n; s0 += 256) {
+                const int s1 = s0 + 128;
+                float acc0[SROW_G], acc1[SROW_G];
+    #pragma unroll
+                for (int g = 0; g < SROW_G; ++g) acc0[g] = acc1[g] = 0.f;
+                for (int d0 = 0; d0 < hd; d0 += 8 * NB) {
+                    if (d0 > 0) load_block(s0, d0);
+    #pragma unroll
+                    for (int c = 0; c < NB; ++c) {
+                        if (d0 + 8 * c >= hd) break;
+                        float k0[8], k1[8];
+                        r0c[c].widen(k0);
+                        r1c[c].widen(k1);
+                        const int d = d0 + 8 * c;
+    #pragma unroll
+                        for (int g = 0; g < SROW_G; ++g) {
+                            const float4 xa = *reinterpret_cast<const float4*>(xh + g * d_k + d);
+                            const float4 xb = *reinterpret_cast<const float4*>(xh + g * d_k + d + 4);
+                            const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+    #pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                acc0[g] = fmaf(xv[e], k0[e], acc0[g]);
+                                acc1[g] = fmaf(xv[e], k1[e], acc1[g]);
+                            }
                         }
                     }
                 }
-            }
-            if (s0 + 256 < n) load_block(s0 + 256, 0);
-#pragma unroll
-            for (int g = 0; g < SROW_G; ++g) {
-                float* scf = reinterpret_cast<float*>(segs + (size_t)(g * 2 + hf1) * NP * 8);
-                scf[s0] = acc0[g];
-                if (s1 < n) scf[s1] = acc1[g];
+                if (s0 + 256 < n) load_block(s0 + 256, 0);
+    #pragma unroll
+                for (int g = 0; g < SROW_G; ++g) {
+                    float* scf = reinterpret_cast<float*>(segs + (size_t)(g * 2 + hf1) * SEG);
+                    scf[s0] = acc0[g];
+                    if (s1 < n) scf[s1] = acc1[g];
+                }
             }
         }
+        __syncthreads();
     }
-    __syncthreads();
 
     // ---- 2. per-half top-k: warp (g, hf) ---------------------------------------------------
     {
         const int g = warp >> 1, hf = warp & 1;
-        const float* scf = reinterpret_cast<const float*>(segs + (size_t)(g * 2 + hf) * NP * 8);
+        const float* scf = reinterpret_cast<const float*>(segs + (size_t)(g * 2 + hf) * SEG);
         float* tvo = tv + (g * 2 + hf) * KP;
         int* tio = ti + (g * 2 + hf) * KP;
         if constexpr (KP == 32) {
@@ -358,7 +489,7 @@ __global__ void __launch_bounds__(SROW_THREADS, 4) score_rows_kernel(ScoreRowsAr
                 bk = key[0];
                 bi = id[0];
             } else {  // the segment's second half (NP * 4 >= 512 bytes) is the scratch
-                int2* scr = reinterpret_cast<int2*>(segs + (size_t)(g * 2 + hf) * NP * 8 + NP * 4);
+                int2* scr = reinterpret_cast<int2*>(segs + (size_t)(g * 2 + hf) * SEG + NP * 4);
                 top32_pruned<PL>(key, id, scr, lane, bk, bi);
             }
             if (lane < kh) {
@@ -398,7 +529,7 @@ __global__ void __launch_bounds__(SROW_THREADS, 4) score_rows_kernel(ScoreRowsAr
                 }
             }
             __syncwarp();  // every lane has read its scores: the segment now holds the lists
-            int2* lst = reinterpret_cast<int2*>(segs + (size_t)(g * 2 + hf) * NP * 8);  // [32][PL]
+            int2* lst = reinterpret_cast<int2*>(segs + (size_t)(g * 2 + hf) * SEG);  // [32][PL]
 #pragma unroll
             for (int r = 2; r < PL; ++r) lst[lane * PL + r] = make_int2((int)key[r], id[r]);
             __syncwarp();
@@ -461,7 +592,7 @@ __global__ void __launch_bounds__(SROW_THREADS, 4) score_rows_kernel(ScoreRowsAr
             bk = k2[0];
             bi = i2c[0];
         } else {  // scratch: the second half of the row's first score segment (free by now)
-            int2* scr = reinterpret_cast<int2*>(segs + (size_t)(g * 2) * NP * 8 + NP * 4);
+            int2* scr = reinterpret_cast<int2*>(segs + (size_t)(g * 2) * SEG + NP * 4);
             top32_pruned<C>(key, id, scr, lane, bk, bi);
         }
         const float v = key_value(bk);

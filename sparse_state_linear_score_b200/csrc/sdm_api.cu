@@ -222,30 +222,45 @@ sdm_status launch_score_tc(const sdm_dims* d, const void* x, const void* sk, int
 // the half width a multiple of 8.
 bool score_rows_eligible(const sdm_dims* d) { return d->n_sub <= 32 * 16; }
 
-template <typename XT, int PL>
-sdm_status launch_score_rows_t(const ScoreRowsArgs& a, int kp, dim3 grid, cudaStream_t s) {
+struct RowMaps {
+    CUtensorMap km[2];
+};
+
+template <typename XT, int PL, bool TCD>
+sdm_status launch_score_rows_t(const RowMaps& m, const ScoreRowsArgs& a, int kp, dim3 grid,
+                               cudaStream_t s) {
     if (kp <= 32) {
-        auto kern = score_rows_kernel<XT, PL, 32>;
-        const size_t smem = score_rows_smem_bytes(a.d_k, PL, 32);
+        auto kern = score_rows_kernel<XT, PL, 32, TCD>;
+        const size_t smem = score_rows_smem_bytes(a.d_k, PL, 32, TCD);
         if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
-        kern<<<grid, SROW_THREADS, smem, s>>>(a);
+        kern<<<grid, SROW_THREADS, smem, s>>>(m.km[0], m.km[1], a);
     } else {
-        auto kern = score_rows_kernel<XT, PL, 64>;
-        const size_t smem = score_rows_smem_bytes(a.d_k, PL, 64);
+        auto kern = score_rows_kernel<XT, PL, 64, TCD>;
+        const size_t smem = score_rows_smem_bytes(a.d_k, PL, 64, TCD);
         if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
-        kern<<<grid, SROW_THREADS, smem, s>>>(a);
+        kern<<<grid, SROW_THREADS, smem, s>>>(m.km[0], m.km[1], a);
     }
     return launch_status();
 }
 
+// Dot products on the tensor cores for bf16 rows of d_k = 128 and n > 64 (the sub-key
+// tables then have 128-byte rows, one 128-byte swizzle span), on CUDA cores otherwise.
 template <typename XT>
-sdm_status launch_score_rows_x(const ScoreRowsArgs& a, int kp, dim3 grid, cudaStream_t s) {
+sdm_status launch_score_rows_x(const RowMaps& m, bool tcd, const ScoreRowsArgs& a, int kp,
+                               dim3 grid, cudaStream_t s) {
     const int pl = (a.n + 31) / 32;
-    if (pl <= 1) return launch_score_rows_t<XT, 1>(a, kp, grid, s);
-    if (pl <= 2) return launch_score_rows_t<XT, 2>(a, kp, grid, s);
-    if (pl <= 4) return launch_score_rows_t<XT, 4>(a, kp, grid, s);
-    if (pl <= 8) return launch_score_rows_t<XT, 8>(a, kp, grid, s);
-    return launch_score_rows_t<XT, 16>(a, kp, grid, s);
+    if constexpr (sizeof(XT) == 2) {
+        if (tcd) {
+            if (pl <= 4) return launch_score_rows_t<XT, 4, true>(m, a, kp, grid, s);
+            if (pl <= 8) return launch_score_rows_t<XT, 8, true>(m, a, kp, grid, s);
+            return launch_score_rows_t<XT, 16, true>(m, a, kp, grid, s);
+        }
+    }
+    if (pl <= 1) return launch_score_rows_t<XT, 1, false>(m, a, kp, grid, s);
+    if (pl <= 2) return launch_score_rows_t<XT, 2, false>(m, a, kp, grid, s);
+    if (pl <= 4) return launch_score_rows_t<XT, 4, false>(m, a, kp, grid, s);
+    if (pl <= 8) return launch_score_rows_t<XT, 8, false>(m, a, kp, grid, s);
+    return launch_score_rows_t<XT, 16, false>(m, a, kp, grid, s);
 }
 
 // One launch for `roles` (1 or 2) scorings of the same shape: role r scores x[r] against
@@ -268,8 +283,53 @@ sdm_status launch_score_rows(const sdm_dims* d, int roles, const void* const* x,
     a.B = d->B; a.H = d->H; a.T = d->T; a.d_k = d->d_k; a.n = d->n_sub; a.k_half = d->k_half;
     const long long rows = (long long)d->B * d->T;
     const dim3 grid((unsigned)((rows + SROW_G - 1) / SROW_G), (unsigned)d->H, (unsigned)roles);
-    if (d->x_dtype == SDM_F32) return launch_score_rows_x<float>(a, kp, grid, s);
-    return launch_score_rows_x<__nv_bfloat16>(a, kp, grid, s);
+    RowMaps m;
+    memset(&m, 0, sizeof(m));
+    const bool tcd = d->x_dtype == SDM_BF16 && d->d_k == 128 && d->n_sub > 64;
+    if (tcd) {
+        EncodeTiledFn enc = encode_tiled();
+        if (!enc) return SDM_ERR_CUDA;
+        for (int r = 0; r < 2; ++r) {  // [H*2*n rows][64] bf16, boxes of 128 rows
+            const cuuint64_t dims[2] = {64, (cuuint64_t)d->H * 2 * d->n_sub};
+            const cuuint64_t strides[1] = {64 * 2};
+            const cuuint32_t box[2] = {64, 128};
+            const cuuint32_t es[2] = {1, 1};
+            if (enc(&m.km[r], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.sk[r]), dims,
+                    strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return SDM_ERR_CUDA;
+        }
+    }
+    if (d->x_dtype == SDM_F32) return launch_score_rows_x<float>(m, false, a, kp, grid, s);
+    return launch_score_rows_x<__nv_bfloat16>(m, tcd, a, kp, grid, s);
+}
+
+sdm_status launch_score(const sdm_dims* d, const void* x, const void* sk, int top, int32_t* idx,
+                        float* w, cudaStream_t s);
+
+// Both roles of one call (keys against the write tables, queries against the read tables):
+// two tensor-core launches when the shape takes them, else one row-scorer launch for both
+// roles (grid.z = role), else the generic path per role.  Arguments as sdm_score_topk.
+sdm_status score_both_roles(const sdm_dims* d, const void* q, const void* k, const void* skw,
+                            const void* skr, int32_t* widx, float* ww, int32_t* ridx, float* rw,
+                            cudaStream_t s) {
+    if (!q || !k || !skw || !skr || !widx || !ww || !ridx || !rw) return SDM_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(skw) || !aligned16(skr) ||
+        !aligned16(widx) || !aligned16(ww) || !aligned16(ridx) || !aligned16(rw))
+        return SDM_ERR_ALIGN;
+    if ((long long)d->B * d->T == 0) return SDM_OK;
+    if (!(score_tc_eligible(d, d->W) && score_tc_eligible(d, d->R)) && score_rows_eligible(d)) {
+        const void* xs[2] = {k, q};
+        const void* sks[2] = {skw, skr};
+        const int tops[2] = {d->W, d->R};
+        int32_t* idxs[2] = {widx, ridx};
+        float* wts[2] = {ww, rw};
+        return launch_score_rows(d, 2, xs, sks, tops, idxs, wts, s);
+    }
+    sdm_status e = launch_score(d, k, skw, d->W, widx, ww, s);
+    if (e) return e;
+    return launch_score(d, q, skr, d->R, ridx, rw, s);
 }
 
 template <typename VT, int RPW, int QPL>
@@ -550,19 +610,7 @@ sdm_status sdm_prefill(const sdm_dims* dims, const void* q, const void* k, const
         return SDM_ERR_ARG;
     const WsLayout L = ws_layout(dims);
     if (!ws || ws_bytes < L.total) return SDM_ERR_WORKSPACE;
-    if (score_rows_eligible(dims) && aligned16(q) && aligned16(k) && aligned16(skw) &&
-        aligned16(skr) && aligned16(widx) && aligned16(ww) && aligned16(ridx) && aligned16(rw)) {
-        // both roles in one launch (grid.z = role)
-        const void* xs[2] = {k, q};
-        const void* sks[2] = {skw, skr};
-        const int tops[2] = {dims->W, dims->R};
-        int32_t* idxs[2] = {widx, ridx};
-        float* ws[2] = {ww, rw};
-        if ((e = launch_score_rows(dims, 2, xs, sks, tops, idxs, ws, stream))) return e;
-    } else {
-        if ((e = sdm_score_topk(dims, k, skw, dims->W, widx, ww, stream))) return e;
-        if ((e = sdm_score_topk(dims, q, skr, dims->R, ridx, rw, stream))) return e;
-    }
+    if ((e = score_both_roles(dims, q, k, skw, skr, widx, ww, ridx, rw, stream))) return e;
     return sdm_forward(dims, v, alpha, beta, widx, ww, ridx, rw, st, out, ws, ws_bytes, stream);
 }
 
@@ -578,8 +626,7 @@ sdm_status sdm_decode_step(const sdm_dims* dims, const void* q, const void* k, c
         return SDM_ERR_ARG;
     if (!aligned16(v) || !aligned16(alpha) || !aligned16(beta) || !aligned16(out))
         return SDM_ERR_ALIGN;
-    if ((e = sdm_score_topk(dims, k, skw, dims->W, widx, ww, stream))) return e;
-    if ((e = sdm_score_topk(dims, q, skr, dims->R, ridx, rw, stream))) return e;
+    if ((e = score_both_roles(dims, q, k, skw, skr, widx, ww, ridx, rw, stream))) return e;
     const int rpw = ((dims->W > dims->R ? dims->W : dims->R) + DECODE_WARPS - 1) / DECODE_WARPS;
     const int qpl = (dims->d_v / 4 + 31) / 32;
     if (dims->v_dtype == SDM_BF16) {
