@@ -399,7 +399,8 @@ def run_gpu(args, wl, world, rank, local):
     return line
 
 
-def run_decode(device, sdm, steps: int = 64, warm: int = 3) -> dict:
+def run_decode(device, sdm, steps: int = 64, warm: int = 3, n_sub: int | None = None,
+               d_v: int | None = None) -> dict:
     """The decode workload at full size: a 512-token seeded prefill of every (b,h), then
     single-token steps (sdm_decode_step: one scoring launch for both roles and one
     recurrence launch each).  `steps` steps are timed as issued from Python one call at a
@@ -411,6 +412,10 @@ def run_decode(device, sdm, steps: int = 64, warm: int = 3) -> dict:
     import sdm_synth as S
 
     wl = S.DECODE.scaled(decode_steps=warm + 2 * steps)
+    if n_sub is not None:  # a smaller table (and state), for captures under a profiler
+        wl = wl.scaled(n_sub=n_sub)
+    if d_v is not None:  # narrower rows: a smaller state, the same scoring launches
+        wl = wl.scaled(d_v=d_v)
     inp = S.generate(wl, device=device)
     d = sdm.Dims(wl.B, wl.H, wl.T, wl.d_k, wl.n_sub, wl.d_v, wl.k_half, wl.W, wl.R, wl.x_dtype,
                  wl.v_dtype)
@@ -643,7 +648,23 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the decode-workload measurement (rank 0)")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the decode workload (--steps timed steps after --warmup) and "
+                         "print its object")
+    ap.add_argument("--decode-n-sub", type=int, default=None,
+                    help="sub-keys per half for --decode-only (default: the workload's 256)")
+    ap.add_argument("--decode-d-v", type=int, default=None,
+                    help="row width for --decode-only (default: the workload's 128)")
     args = ap.parse_args(argv)
+    if args.decode_only:
+        import torch
+
+        import sparse_state_linear_score_b200 as sdm
+        res = run_decode(torch.device("cuda", 0), sdm, steps=args.steps,
+                         warm=max(3, args.warmup), n_sub=args.decode_n_sub,
+                         d_v=args.decode_d_v)
+        print(json.dumps({"decode": res}), flush=True)
+        return
     world, rank, local = dist_env()
     if world != args.gpus and "WORLD_SIZE" in os.environ:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
