@@ -39,6 +39,19 @@
 
 namespace sdm {
 
+// 4 consecutive fp32 columns of this thread's TMEM lane (tcgen05.ld, 32 lanes x 32 bits, x4).
+SDM_DEV void tmem_ld4(uint32_t taddr, float (&v)[4]) {
+    uint32_t r0, r1, r2, r3;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    v[0] = __uint_as_float(r0);
+    v[1] = __uint_as_float(r1);
+    v[2] = __uint_as_float(r2);
+    v[3] = __uint_as_float(r3);
+}
+
 constexpr int SROW_THREADS = 256;
 constexpr int SROW_G = 4;  // rows per CTA: two warps per row in phase 2
 
@@ -384,7 +397,7 @@ __global__ void __launch_bounds__(SROW_THREADS, 4) score_rows_kernel(
             const int q = warp & 3;
             for (int c = warp >> 2; c < nch; c += 2) {
                 float v[4];
-                ptx::tmem_ld4(tmem + ((uint32_t)(32 * q) << 16) + 16u * (uint32_t)c, v);
+                tmem_ld4(tmem + ((uint32_t)(32 * q) << 16) + 16u * (uint32_t)c, v);
                 const int hf = c / cph, sidx = (c % cph) * 128 + 32 * q + lane;
                 if (sidx < n)
 #pragma unroll

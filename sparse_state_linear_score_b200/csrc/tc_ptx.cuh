@@ -152,19 +152,6 @@ SDM_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 SDM_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 SDM_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 4 consecutive fp32 columns of this thread's TMEM lane.
-SDM_DEV void tmem_ld4(uint32_t taddr, float (&v)[4]) {
-    uint32_t r0, r1, r2, r3;
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-    v[0] = __uint_as_float(r0);
-    v[1] = __uint_as_float(r1);
-    v[2] = __uint_as_float(r2);
-    v[3] = __uint_as_float(r3);
-}
-
 // 32 consecutive fp32 columns of this thread's TMEM lane.
 SDM_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     uint32_t r[32];
