@@ -17,6 +17,9 @@ Parity status per function:
   recur_dense ................. pinned (beta=0 closed form, one-hot write/read,
                                  dense Gated DeltaNet matrix form, hand example)
   recur_lazy .................. pinned (agrees with recur_dense to 1e-12)
+  recur_touched ............... pinned (hand example, alpha = 1 equals recur_dense,
+                                 all slots written = recur_dense (Gated DeltaNet),
+                                 beta = 0 closed form with unwritten slots at M0)
   materialize ................. pinned (beta=0 closed form)
   prefill_pairs ............... pinned through score + recur_lazy
   weight_stats ................ pinned (uniform and one-hot closed forms, two-point
@@ -91,6 +94,8 @@ class Oracle:
         lib.sdm_oracle_score.restype = I
         lib.sdm_oracle_recur_dense.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P]
         lib.sdm_oracle_recur_dense.restype = I
+        lib.sdm_oracle_recur_touched.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P]
+        lib.sdm_oracle_recur_touched.restype = I
         lib.sdm_oracle_recur_lazy.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P]
         lib.sdm_oracle_recur_lazy.restype = I
         lib.sdm_oracle_materialize.argtypes = [I, I, P, P, D, P]
@@ -212,6 +217,22 @@ class Oracle:
         _check(self.lib.sdm_oracle_recur_dense(T, N, dv, W, R, _p(v), _p(alpha), _p(beta), _p(widx),
                                                _p(ww), _p(ridx), _p(rw), _p(M), _p(out)),
                "recur_dense")
+        return out, M
+
+    def recur_touched(self, v, alpha, beta, widx, ww, ridx, rw, M):
+        """Touched-slots decay (alpha scales only the write slots) for one (b,h).
+
+        Returns (out [T,dv], M_final [N,dv])."""
+        v, alpha, beta = _f64(v), _f64(alpha), _f64(beta)
+        widx, ridx, ww, rw = _i32(widx), _i32(ridx), _f64(ww), _f64(rw)
+        M = _f64(M).copy()
+        T, dv = v.shape
+        N = M.shape[0]
+        W, R = widx.shape[1], ridx.shape[1]
+        out = np.empty((T, dv), np.float64)
+        _check(self.lib.sdm_oracle_recur_touched(T, N, dv, W, R, _p(v), _p(alpha), _p(beta),
+                                                 _p(widx), _p(ww), _p(ridx), _p(rw), _p(M),
+                                                 _p(out)), "recur_touched")
         return out, M
 
     @staticmethod

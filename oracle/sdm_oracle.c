@@ -236,6 +236,58 @@ int sdm_oracle_recur_dense(int T, int N, int dv, int W, int R, const double* v,
 }
 
 /*
+ * Touched-slots decay: the other reading of §3 Method "Sparse memory updates"
+ * (the gated delta update, its decay gate included, acts only on the W slots the
+ * keys select).  Per token t:
+ *   (i')  M[s_i] <- alpha_t * M[s_i]             (the W write slots only)
+ *   (ii)  p  = sum_i w_i M[s_i]
+ *   (iii) e  = v_t - p
+ *   (iv)  M[s_i] <- M[s_i] + beta_t * w_i * e
+ *   (v)   o_t = sum_j u_j M[r_j]                (read after the write)
+ * Every other slot keeps its value, so a slot never written still holds M0.  With
+ * every slot written at every token (W = N) this is the dense form above (Gated
+ * DeltaNet, "Connection to GDN"); with alpha = 1 the two readings coincide.
+ * M [N][dv] in/out; out [T][dv].
+ */
+int sdm_oracle_recur_touched(int T, int N, int dv, int W, int R, const double* v,
+                             const double* alpha, const double* beta, const int32_t* widx,
+                             const double* ww, const int32_t* ridx, const double* rw,
+                             double* M, double* out) {
+    if (T < 0 || N <= 0 || dv <= 0 || W <= 0 || R <= 0) return ORACLE_ERR_ARG;
+    double* p = (double*)malloc(sizeof(double) * (size_t)dv);
+    double* e = (double*)malloc(sizeof(double) * (size_t)dv);
+    if (!p || !e) { free(p); free(e); return ORACLE_ERR_NOMEM; }
+    int rc = ORACLE_OK;
+    for (int t = 0; t < T; ++t) {
+        const int32_t* ws = widx + (size_t)t * W;
+        const int32_t* rs = ridx + (size_t)t * R;
+        if (!check_slots(ws, W, N) || !check_slots(rs, R, N)) { rc = ORACLE_ERR_ARG; break; }
+        /* (i') decay the write slots */
+        for (int i = 0; i < W; ++i)
+            for (int c = 0; c < dv; ++c) M[(size_t)ws[i] * dv + c] *= alpha[t];
+        /* (ii) prediction */
+        for (int c = 0; c < dv; ++c) p[c] = 0.0;
+        for (int i = 0; i < W; ++i)
+            for (int c = 0; c < dv; ++c) p[c] += ww[(size_t)t * W + i] * M[(size_t)ws[i] * dv + c];
+        /* (iii) error */
+        for (int c = 0; c < dv; ++c) e[c] = v[(size_t)t * dv + c] - p[c];
+        /* (iv) gated delta write on the W slots */
+        for (int i = 0; i < W; ++i)
+            for (int c = 0; c < dv; ++c)
+                M[(size_t)ws[i] * dv + c] += beta[t] * ww[(size_t)t * W + i] * e[c];
+        /* (v) read after the write */
+        for (int c = 0; c < dv; ++c) {
+            double o = 0.0;
+            for (int j = 0; j < R; ++j) o += rw[(size_t)t * R + j] * M[(size_t)rs[j] * dv + c];
+            out[(size_t)t * dv + c] = o;
+        }
+    }
+    free(p);
+    free(e);
+    return rc;
+}
+
+/*
  * Lazy-decay recurrence, the same steps with decay applied only when a slot is
  * touched.  State: Mraw [N][dv], stamp [N] (log-decay prefix at the slot's last
  * write), *Lambda (running log-decay prefix).  The true slot value at the current

@@ -318,6 +318,72 @@ def pin_hand_recurrence(o):
     assert o.materialize(st).tolist() == g["M_final"]
 
 
+# ------------------------------------------- touched-slots decay variant ---
+
+def pin_touched_hand(o):
+    """The hand-worked three-token example in tests/golden/hand_touched_three_tokens.json."""
+    with open(os.path.join(GOLDEN, "hand_touched_three_tokens.json")) as f:
+        g = json.load(f)
+    args = [np.array(g[k], dtype=float) for k in ("v", "alpha", "beta")]
+    widx, ridx = np.array(g["widx"]), np.array(g["ridx"])
+    ww, rw = np.array(g["ww"], float), np.array(g["rw"], float)
+    out, M = o.recur_touched(*args, widx, ww, ridx, rw, np.array(g["M0"], float))
+    assert out.tolist() == g["out"]
+    assert M.tolist() == g["M_final"]
+
+
+def pin_touched_alpha_one(o):
+    """alpha = 1: no slot decays under either reading, so the touched-slots recurrence
+    performs the dense one's arithmetic exactly."""
+    rng = _rng(13)
+    T, N, dv, W, R = 25, 14, 3, 4, 5
+    v, alpha, beta, widx, ww, ridx, rw, M0 = _random_case(rng, T, N, dv, W, R)
+    ones = np.ones(T)
+    out_t, M_t = o.recur_touched(v, ones, beta, widx, ww, ridx, rw, M0)
+    out_d, M_d = o.recur_dense(v, ones, beta, widx, ww, ridx, rw, M0)
+    assert np.array_equal(out_t, out_d) and np.array_equal(M_t, M_d)
+
+
+def pin_touched_all_slots_gdn(o):
+    """Every slot written at every token (W = N, a fresh permutation per token): every
+    slot decays once per token, which is the dense form (Gated DeltaNet)."""
+    rng = _rng(14)
+    T, N, dv, R = 12, 7, 3, 4
+    v = rng.standard_normal((T, dv))
+    alpha = rng.uniform(0.5, 1.0, T)
+    beta = rng.uniform(0.0, 1.0, T)
+    widx = np.stack([rng.permutation(N) for _ in range(T)]).astype(np.int32)
+    ww = rng.dirichlet(np.ones(N), T)
+    ridx = np.stack([rng.permutation(N)[:R] for _ in range(T)]).astype(np.int32)
+    rw = rng.dirichlet(np.ones(R), T)
+    M0 = rng.standard_normal((N, dv))
+    out_t, M_t = o.recur_touched(v, alpha, beta, widx, ww, ridx, rw, M0)
+    out_d, M_d = o.recur_dense(v, alpha, beta, widx, ww, ridx, rw, M0)
+    np.testing.assert_allclose(out_t, out_d, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(M_t, M_d, rtol=1e-13, atol=1e-14)
+
+
+def pin_touched_beta_zero(o):
+    """beta = 0: a slot is multiplied by alpha_t exactly at the tokens that write it, so
+    M_T[s] = M0[s] * prod_{t: s written at t} alpha_t, and o_t reads that product up to
+    token t (slots never written keep M0)."""
+    rng = _rng(15)
+    T, N, dv, W, R = 19, 16, 3, 3, 4
+    v, alpha, beta, widx, ww, ridx, rw, M0 = _random_case(rng, T, N, dv, W, R, 0.5, 1.0)
+    widx = np.stack([rng.permutation(10)[:W] for _ in range(T)]).astype(np.int32)  # 10..15 unwritten
+    fac = np.ones((T + 1, N))
+    for t in range(T):
+        fac[t + 1] = fac[t]
+        fac[t + 1, widx[t]] *= alpha[t]
+    expect = np.stack([(rw[t][:, None] * (M0[ridx[t]] * fac[t + 1, ridx[t]][:, None])).sum(0)
+                       for t in range(T)])
+    out_t, M_t = o.recur_touched(v, alpha, np.zeros(T), widx, ww, ridx, rw, M0)
+    np.testing.assert_allclose(out_t, expect, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(M_t, M0 * fac[T][:, None], rtol=1e-12, atol=1e-14)
+    untouched = np.setdiff1d(np.arange(N), widx.reshape(-1))
+    assert untouched.size > 0 and np.array_equal(M_t[untouched], M0[untouched])
+
+
 def pin_prefill_pairs(o):
     """The batched prefill equals product-key scoring followed by the lazy recurrence."""
     rng = _rng(12)
@@ -508,4 +574,5 @@ ALL_PINS = [pin_pk_equals_brute, pin_brute_matches_numpy, pin_pk_depends_on_k, p
             pin_convex_update, pin_dense_limit_gdn, pin_lazy_equals_dense, pin_split_invariance,
             pin_hand_recurrence, pin_prefill_pairs, pin_weight_stats_closed_forms,
             pin_weight_stats_summaries, pin_layer_out_hand_example, pin_layer_out_properties,
-            pin_layer_in_routing_and_gates, pin_layer_in_linear]
+            pin_layer_in_routing_and_gates, pin_layer_in_linear, pin_touched_hand,
+            pin_touched_alpha_one, pin_touched_all_slots_gdn, pin_touched_beta_zero]

@@ -20,6 +20,27 @@ MUTANTS = {
     "decay_dropped": [
         ("M[q] *= alpha[t];", "M[q] *= 1.0;"),
         ("L += log(alpha[t]);", "L += 0.0;"),
+        ("for (int c = 0; c < dv; ++c) M[(size_t)ws[i] * dv + c] *= alpha[t];",
+         "for (int c = 0; c < dv; ++c) M[(size_t)ws[i] * dv + c] *= 1.0;"),
+    ],
+    "touched_decay_hits_every_slot": [
+        ("for (int c = 0; c < dv; ++c) M[(size_t)ws[i] * dv + c] *= alpha[t];",
+         "if (i == 0) for (size_t q = 0; q < (size_t)N * dv; ++q) M[q] *= alpha[t];"),
+    ],
+    "touched_decay_after_prediction": [
+        ("        /* (i') decay the write slots */\n"
+         "        for (int i = 0; i < W; ++i)\n"
+         "            for (int c = 0; c < dv; ++c) M[(size_t)ws[i] * dv + c] *= alpha[t];\n"
+         "        /* (ii) prediction */\n"
+         "        for (int c = 0; c < dv; ++c) p[c] = 0.0;\n"
+         "        for (int i = 0; i < W; ++i)\n"
+         "            for (int c = 0; c < dv; ++c) p[c] += ww[(size_t)t * W + i] * M[(size_t)ws[i] * dv + c];\n",
+         "        /* (ii) prediction */\n"
+         "        for (int c = 0; c < dv; ++c) p[c] = 0.0;\n"
+         "        for (int i = 0; i < W; ++i)\n"
+         "            for (int c = 0; c < dv; ++c) p[c] += ww[(size_t)t * W + i] * M[(size_t)ws[i] * dv + c];\n"
+         "        for (int i = 0; i < W; ++i)\n"
+         "            for (int c = 0; c < dv; ++c) M[(size_t)ws[i] * dv + c] *= alpha[t];\n"),
     ],
     "beta_ignored": [
         ("M[(size_t)ws[i] * dv + c] += beta[t] *", "M[(size_t)ws[i] * dv + c] += 1.0 *"),
