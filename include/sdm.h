@@ -61,6 +61,19 @@ typedef enum {
 
 typedef enum { SDM_F32 = 0, SDM_BF16 = 1 } sdm_dtype;
 
+/*
+ * Which slots the decay gate alpha_t scales at token t.  The pages (Sparse Delta Memory
+ * summary, §3 Method "Sparse memory updates") say the gated delta updates act only on the
+ * W selected slots and (§3 "Connection to GDN") that selecting every slot gives Gated
+ * DeltaNet; they leave open whether the decay reaches the other slots.
+ *   SDM_DECAY_ALL     every slot, every token (the dense Gated DeltaNet rule, applied
+ *                     lazily through Lambda and the stamps)            -- the default
+ *   SDM_DECAY_TOUCHED only the token's write slots, at the write; a slot that is not
+ *                     written keeps its value, and one never written stays M0
+ * With alpha = 1, or with every slot written at every token, the two agree.
+ */
+typedef enum { SDM_DECAY_ALL = 0, SDM_DECAY_TOUCHED = 1 } sdm_decay;
+
 /* Bits of the device error word (sdm_device_error). */
 #define SDM_DEVERR_SLOT_RANGE 1u   /* a slot index outside [0, N) */
 #define SDM_DEVERR_DUP_WRITE 2u    /* a write slot repeated within one token */
@@ -76,6 +89,7 @@ typedef struct {
     int32_t W, R;      /* write and read slots per token */
     int32_t x_dtype;   /* sdm_dtype of q, k and the sub-key tables */
     int32_t v_dtype;   /* sdm_dtype of v */
+    int32_t decay;     /* sdm_decay: which slots alpha scales (0 = every slot) */
 } sdm_dims;
 
 /*
@@ -88,7 +102,9 @@ typedef struct {
  *   M0     [H][N][d_v]    fp32  initial memory, shared by the batch (read only)
  * The true value of slot s is  M[s] * exp(Lambda - stamp[s]),  or
  * M0[h][s] * exp(Lambda) while the slot is pristine.  (The pages give the decay
- * as a per-token multiplication of every slot; this form is equal to it.)
+ * as a per-token multiplication of every slot; this form is equal to it.)  Under
+ * SDM_DECAY_TOUCHED the value is M[s] itself (M0[h][s] while pristine): the stamps
+ * then only mark pristine slots, and Lambda is kept but not used.
  */
 typedef struct {
     float* M;

@@ -38,12 +38,21 @@ class SdmError(RuntimeError):
         super().__init__(f"{what}: {_lib.sdm_status_str(status).decode()}")
 
 
-class Dims(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int32) for n in
-                ("B", "H", "T", "d_k", "n_sub", "d_v", "k_half", "W", "R", "x_dtype", "v_dtype")]
+DECAY_ALL, DECAY_TOUCHED = 0, 1
+_DECAY = {"all": DECAY_ALL, "touched": DECAY_TOUCHED}
 
-    def __init__(self, B, H, T, d_k, n_sub, d_v, k_half, W, R, x_dtype="f32", v_dtype="f32"):
-        super().__init__(B, H, T, d_k, n_sub, d_v, k_half, W, R, _DT[x_dtype], _DT[v_dtype])
+
+class Dims(ctypes.Structure):
+    """sdm_dims.  decay: "all" (alpha scales every slot at every token) or "touched"
+    (only the token's write slots); see sdm_decay in include/sdm.h."""
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "H", "T", "d_k", "n_sub", "d_v", "k_half", "W", "R", "x_dtype", "v_dtype",
+                 "decay")]
+
+    def __init__(self, B, H, T, d_k, n_sub, d_v, k_half, W, R, x_dtype="f32", v_dtype="f32",
+                 decay="all"):
+        super().__init__(B, H, T, d_k, n_sub, d_v, k_half, W, R, _DT[x_dtype], _DT[v_dtype],
+                         _DECAY[decay])
 
     @property
     def N(self) -> int:
@@ -51,7 +60,7 @@ class Dims(ctypes.Structure):
 
     def with_T(self, T: int) -> "Dims":
         x = Dims(self.B, self.H, T, self.d_k, self.n_sub, self.d_v, self.k_half, self.W, self.R)
-        x.x_dtype, x.v_dtype = self.x_dtype, self.v_dtype
+        x.x_dtype, x.v_dtype, x.decay = self.x_dtype, self.v_dtype, self.decay
         return x
 
 

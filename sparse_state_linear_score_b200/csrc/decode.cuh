@@ -4,6 +4,7 @@
 // Per sequence, following §2 Background "Gated DeltaNet" and §3 Method:
 //   Lambda' = Lambda + log(alpha)
 //   seen(s) = M[s] e^{Lambda' - stamp[s]}   (M0[s] e^{Lambda'} while pristine)
+//             [touched-slots decay: alpha M[s] for a write slot, M[s] for a read slot]
 //   p = sum_i w_i seen(s_i);  d = beta (v - p)
 //   M[s_i] = seen(s_i) + w_i d,  stamp[s_i] = Lambda'
 //   out = sum_j u_j (value of r_j after the write)
@@ -56,7 +57,7 @@ __global__ void __launch_bounds__(DECODE_THREADS) decode_kernel(
     const int32_t* __restrict__ widx, const float* __restrict__ ww,
     const int32_t* __restrict__ ridx, const float* __restrict__ rw, float* __restrict__ M,
     double* __restrict__ stamp, double* __restrict__ lambda, const float* __restrict__ M0,
-    float* __restrict__ out, int H, int N, int d_v, int W, int R) {
+    float* __restrict__ out, int H, int N, int d_v, int W, int R, int touched) {
     extern __shared__ __align__(16) unsigned char dec_smem[];
     const size_t bh = blockIdx.x;
     const int h = (int)(bh % H);
@@ -84,10 +85,10 @@ __global__ void __launch_bounds__(DECODE_THREADS) decode_kernel(
         vv[c] = q < Q ? load_v4<VT>(v + bh * d_v + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     double Lnew;  // Lambda'
+    const float a_t = alpha[bh];
     {
-        const float a = alpha[bh];
         double la = 0.0;
-        if (a > 0.f) la = log((double)a);
+        if (a_t > 0.f) la = log((double)a_t);
         else if (tid == 0) raise_err(SDM_DEVERR_ALPHA);
         Lnew = lambda[bh] + la;
     }
@@ -110,7 +111,12 @@ __global__ void __launch_bounds__(DECODE_THREADS) decode_kernel(
                 sl = -1;
             } else {
                 const double st = stb[sl];
-                f = isnan(st) ? -(float)exp(Lnew) : (float)exp(Lnew - st);
+                if (touched) {  // alpha scales the write slots only
+                    const float fv = rl ? 1.f : a_t;
+                    f = isnan(st) ? -fv : fv;
+                } else {
+                    f = isnan(st) ? -(float)exp(Lnew) : (float)exp(Lnew - st);
+                }
             }
             my_s = sl;
             my_f = f;

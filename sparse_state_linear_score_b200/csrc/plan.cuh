@@ -115,6 +115,12 @@ struct PlanPtrs {
     int32_t* rs;          // [BH][T*(W+R)] chunk j at j*C*(W+R), in-chunk occurrence order:
                           // slot | bit 31 when the row gathered is the pristine M0 row
     unsigned char* img;   // [BH][J][img bytes]: per-chunk image (RunImg)
+    // touched-slots decay only (null otherwise), per occurrence in the lk order:
+    float* vfc;  // product of alpha over the slot's writes in this chunk up to the occurrence's
+                 // token (the occurrence itself included when it is a write): the factor
+                 // of the gathered row
+    float* vsh;  // writes: product of alpha over the slot's later writes in this chunk (the
+                 // owner's included): its d's factor in the stored value
 };
 
 // Per-chunk image of the row pass's column-independent inputs, written by plan_pack and
@@ -156,6 +162,7 @@ __global__ void __launch_bounds__(PLAN_THREADS, 2) plan_local_kernel(
     const int32_t* __restrict__ ridx, const float* __restrict__ rw,
     const double* __restrict__ stamp, int T, int N, int W, int R, int C, int J, PlanPtrs P) {
     __shared__ double s_wtot[32];
+    __shared__ float s_alf[PLAN_MAX_C];  // alpha_t (touched-slots decay)
     extern __shared__ __align__(16) unsigned char plan_smem[];
     float* s_L = reinterpret_cast<float*>(plan_smem);         // [32][32] L, then Minv
     float* s_G = s_L + PLAN_MAX_C * PLAN_MAX_C;               // [32][32]
@@ -179,11 +186,13 @@ __global__ void __launch_bounds__(PLAN_THREADS, 2) plan_local_kernel(
     const int nt = min(C, T - t0);
     const int nw = nt * W, no = nt * (W + R);
     const size_t occ_base = bh * (size_t)T * (W + R);
+    const bool touched = P.vfc != nullptr;  // alpha scales only the write slots
 
     // 1. chunk-relative log-decay prefix (C <= PLAN_THREADS tokens per chunk)
     double la = 0.0;
     if (tid < nt) {
         const float a = alpha[bh * T + t0 + tid];
+        s_alf[tid] = a;
         if (a > 0.f) {
             la = log((double)a);
         } else {
@@ -285,7 +294,9 @@ __global__ void __launch_bounds__(PLAN_THREADS, 2) plan_local_kernel(
 
     // 5. L and G rows: one warp per (role, token) t; its lanes walk the link chains of t's
     //    occurrences (every earlier write of the slot in the chunk) in step, and the terms of
-    //    one step are added to row t in lane order (deterministic sums)
+    //    one step are added to row t in lane order (deterministic sums).  A term's decay from
+    //    the earlier write at tp to t is e^{lam_t - lam_tp}; with touched-slots decay it is the
+    //    product of alpha over the slot's writes after tp up to t (t's own write included)
     {
         const int warp = tid >> 5, lane = tid & 31;
         for (int task = warp; task < 2 * nt; task += PLAN_THREADS / 32) {
@@ -300,12 +311,18 @@ __global__ void __launch_bounds__(PLAN_THREADS, 2) plan_local_kernel(
                 const bool in = base + lane < n_i;
                 const float wo = in ? s_wt[o] : 0.f;
                 int L = in ? s_link[o] : -1;
+                float chain = rd ? 1.f : s_alf[t];  // touched: decay of the next term
                 while (__any_sync(0xffffffffu, L >= 0)) {
                     int tp = 0;
                     float val = 0.f;
                     if (L >= 0) {
                         tp = fW.div(L);
-                        val = wo * s_wt[L] * expf(lt - s_lamc[tp]);
+                        if (touched) {
+                            val = wo * s_wt[L] * chain;
+                            chain *= s_alf[tp];
+                        } else {
+                            val = wo * s_wt[L] * expf(lt - s_lamc[tp]);
+                        }
                     }
                     for (unsigned m = __ballot_sync(0xffffffffu, L >= 0); m; m &= m - 1) {
                         const int src = __ffs(m) - 1;
@@ -388,6 +405,24 @@ __global__ void __launch_bounds__(PLAN_THREADS, 2) plan_local_kernel(
         }
         P.lk[g] = (int32_t)v;
         P.st0[g] = est[k];
+        if (touched) {
+            // the gathered row's factor: alpha of every write of the slot in this chunk up to
+            // this occurrence (its own write included)
+            const bool is_w = o < nw;
+            float fc = is_w ? s_alf[fW.div(o)] : 1.f;
+            for (int L = link; L >= 0; L = s_link[L]) fc *= s_alf[fW.div(L)];
+            P.vfc[g] = fc;
+            if (is_w && sl < 0) P.vsh[g] = 0.f;
+            if (is_w && s_owner[o]) {
+                // down the slot's chain from its last write: each write's d reaches the stored
+                // value through the alpha of the slot's later writes
+                float sh = 1.f;
+                for (int L = o; L >= 0; L = s_link[L]) {
+                    P.vsh[occ_base + (size_t)t0 * W + L] = sh;
+                    sh *= s_alf[fW.div(L)];
+                }
+            }
+        }
         if (!P.mask)  // the walk's input
             P.occw[g] = (sl >= 0 ? (uint32_t)sl : OCC_SLOT) | (o < nw && s_owner[o] ? OCC_OWNER : 0u);
         if (P.mask && o < nw && s_owner[o] && sl >= 0)  // this chunk stores the slot
@@ -627,17 +662,20 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_pack_kernel(
         const bool ok = slot_ok(s, N);
         // with the masks the factors are computed here (plan_fe is not run); after the walk
         // they are read back
-        const float f = !ok ? 0.f
-                        : P.mask ? occ_factor(stamp, P, bh, N, J, j, s, (o < nw) && (lk & LK_OWNER),
-                                              s_lam[o < nw ? o / W : (o - nw) / R], P.st0[g])
-                                 : P.fe[g];
+        float f = !ok ? 0.f
+                  : P.mask ? occ_factor(stamp, P, bh, N, J, j, s, (o < nw) && (lk & LK_OWNER),
+                                        s_lam[o < nw ? o / W : (o - nw) / R], P.st0[g])
+                           : P.fe[g];
+        // touched-slots decay: the same pristine sign, the in-chunk product as the magnitude
+        if (P.vfc && ok) f = copysignf(P.vfc[g], f);
         rs[o] = ok ? (int32_t)((uint32_t)s | (signbit(f) ? 0x80000000u : 0u)) : 0x7fffffff;
         coef[ci] = ok ? w * fabsf(f) : 0.f;
         if (o < nw) {
-            const float e = expf(lam_end - s_lam[o / W]);
+            // shares of the stored (chunk-end) value: the d of this write, the gathered row
+            const float e = P.vfc ? 1.f : expf(lam_end - s_lam[o / W]);
             wslot[o] = ok ? s : 0x7fffffff;
             wlk[o] = lk;
-            sc[o] = w * e;
+            sc[o] = w * (P.vfc ? P.vsh[g] : e);
             sa[o] = fabsf(f) * e;
         }
         const int pv = lk_prev(lk);

@@ -458,7 +458,7 @@ SDM_DEV void tc_select(const Src& src, int K, uint32_t* hist, float* Sv, uint16_
             int rank = 0;
 #pragma unroll
             for (int f = 0; f < TC_BC; ++f) rank += better(bv[f], bi[f], bv[e], bi[e]) ? 1 : 0;
-            if (e < nbd && rank < need) {
+            if (e < nbd && rank < need && ns + rank < K) {
                 Sv[(ns + rank) * S] = bv[e];
                 Sh[(ns + rank) * S] = (uint16_t)bh[e];
             }

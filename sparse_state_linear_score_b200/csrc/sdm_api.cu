@@ -32,6 +32,7 @@ sdm_status check_dims(const sdm_dims* d) {
     if (!d) return SDM_ERR_ARG;
     if (d->x_dtype != SDM_F32 && d->x_dtype != SDM_BF16) return SDM_ERR_DTYPE;
     if (d->v_dtype != SDM_F32 && d->v_dtype != SDM_BF16) return SDM_ERR_DTYPE;
+    if (d->decay != SDM_DECAY_ALL && d->decay != SDM_DECAY_TOUCHED) return SDM_ERR_ARG;
     if (d->B < 1 || d->H < 1 || d->T < 0) return SDM_ERR_SHAPE;
     if ((long long)d->B * d->H > 65535) return SDM_ERR_SHAPE;
     if (d->d_k < 16 || d->d_k > 256 || (d->d_k / 2) % 8 != 0 || d->d_k % 2 != 0) return SDM_ERR_SHAPE;
@@ -63,7 +64,7 @@ struct WsLayout {
     bool lstart_smem;
     size_t walk_smem;
     size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_occw, off_mask;
-    size_t off_rs, off_img, total;
+    size_t off_rs, off_img, off_vfc, off_vsh, total;
     int MW;  // mask words per slot, 0 when the walk is used
 };
 
@@ -93,6 +94,10 @@ WsLayout ws_layout(const sdm_dims* d) {
     L.off_mask = o;   o = up256(o + BH * N * (size_t)L.MW * 8);
     L.off_rs = o;     o = up256(o + BH * occ * 4);
     L.off_img = o;    o = up256(o + BH * (size_t)L.J * run_img(L.C, d->W, d->R).bytes);
+    // touched-slots decay: in-chunk decay products of each occurrence (see PlanPtrs)
+    const size_t vt = d->decay == SDM_DECAY_TOUCHED ? BH * occ * 4 : 0;
+    L.off_vfc = o;    o = up256(o + vt);
+    L.off_vsh = o;    o = up256(o + vt);
     L.total = o;
     return L;
 }
@@ -111,6 +116,9 @@ PlanPtrs plan_ptrs(const WsLayout& L, void* ws) {
     P.MW = L.MW;
     P.rs = reinterpret_cast<int32_t*>(b + L.off_rs);
     P.img = b + L.off_img;
+    const bool touched = L.off_vsh != L.off_vfc;
+    P.vfc = touched ? reinterpret_cast<float*>(b + L.off_vfc) : nullptr;
+    P.vsh = touched ? reinterpret_cast<float*>(b + L.off_vsh) : nullptr;
     return P;
 }
 
@@ -180,9 +188,11 @@ sdm_status launch_score_tc(const sdm_dims* d, const void* x, const void* sk, int
     ScoreTcArgs a{};
     a.B = d->B; a.H = d->H; a.T = d->T; a.n = d->n_sub; a.k_half = d->k_half; a.top = top;
     a.nbox = d->n_sub < TC_NB ? d->n_sub : TC_NB;
-    a.bt = d->T >= 128 ? 128 : d->T;
+    // A tile is always 128 rows that the TMA fills: 128 tokens of one sequence, or 64 tokens
+    // of two when T = 64.  Rows past T or B are the load's zero fill, so the tensor cores
+    // never read rows that no load wrote.
+    a.bt = d->T == 64 ? 64 : 128;
     a.bb = 128 / a.bt;
-    if (a.bb > d->B) a.bb = d->B;
     a.n_tt = (d->T + a.bt - 1) / a.bt;
     a.idx = idx;
     a.w = w;
@@ -353,7 +363,7 @@ sdm_status launch_decode(const sdm_dims* d, const void* v, const float* alpha, c
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, (const VT*)v, alpha, beta, widx, ww, ridx, rw, st->M,
                            st->stamp, st->Lambda, (const float*)st->M0, out, d->H, (int)N_of(d),
-                           d->d_v, d->W, d->R) != cudaSuccess)
+                           d->d_v, d->W, d->R, (int)(d->decay == SDM_DECAY_TOUCHED)) != cudaSuccess)
         return SDM_ERR_CUDA;
     return launch_status();
 }
@@ -450,7 +460,7 @@ const char* sdm_status_str(int32_t status) {
     }
 }
 
-int32_t sdm_abi_version(void) { return 3; }
+int32_t sdm_abi_version(void) { return 4; }
 
 sdm_status sdm_state_bytes(const sdm_dims* dims, size_t* M_bytes, size_t* stamp_bytes,
                            size_t* lambda_bytes) {
@@ -492,7 +502,8 @@ sdm_status sdm_state_materialize(const sdm_dims* dims, const sdm_state* st, floa
     size_t blocks = (total + threads - 1) / threads;
     if (blocks > 148 * 64) blocks = 148 * 64;
     state_materialize_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
-        st->M, st->stamp, st->Lambda, st->M0, dims->H, (int)N_of(dims), dims->d_v, rows, M_out);
+        st->M, st->stamp, st->Lambda, st->M0, dims->H, (int)N_of(dims), dims->d_v, rows,
+        (int)(dims->decay == SDM_DECAY_TOUCHED), M_out);
     return launch_status();
 }
 

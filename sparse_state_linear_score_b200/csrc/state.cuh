@@ -21,11 +21,12 @@ __global__ void state_reset_kernel(double* __restrict__ stamp, size_t n_stamp,
 }
 
 // Dense memory: out[b,h,s,:] = M[b,h,s,:] * exp(Lambda - stamp) or M0[h,s,:] * exp(Lambda)
-// for a pristine slot.  One thread per float4 of a row.
+// for a pristine slot (touched-slots decay: M[b,h,s,:], or M0[h,s,:] while pristine).  One
+// thread per float4 of a row.
 __global__ void state_materialize_kernel(const float* __restrict__ M, const double* __restrict__ stamp,
                                          const double* __restrict__ lambda,
                                          const float* __restrict__ M0, int H, int N, int d_v,
-                                         size_t n_rows, float* __restrict__ out) {
+                                         size_t n_rows, int touched, float* __restrict__ out) {
     const int q_per_row = d_v / 4;
     const size_t total = n_rows * q_per_row;
     const size_t stride = (size_t)gridDim.x * blockDim.x;
@@ -41,10 +42,10 @@ __global__ void state_materialize_kernel(const float* __restrict__ M, const doub
         float f;
         if (isnan(st)) {
             val = reinterpret_cast<const float4*>(M0 + ((size_t)h * N + s) * d_v)[q];
-            f = (float)exp(L);
+            f = touched ? 1.f : (float)exp(L);
         } else {
             val = reinterpret_cast<const float4*>(M + row * d_v)[q];
-            f = (float)exp(L - st);
+            f = touched ? 1.f : (float)exp(L - st);
         }
         val.x *= f;
         val.y *= f;

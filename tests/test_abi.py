@@ -24,13 +24,15 @@ def lib():
 
 
 class Dims(ctypes.Structure):
+    """sdm_dims as include/sdm.h lays it out (twelve int32 fields)."""
     _fields_ = [(n, ctypes.c_int32) for n in
-                ("B", "H", "T", "d_k", "n_sub", "d_v", "k_half", "W", "R", "x_dtype", "v_dtype")]
+                ("B", "H", "T", "d_k", "n_sub", "d_v", "k_half", "W", "R", "x_dtype", "v_dtype",
+                 "decay")]
 
 
 def mid_dims(**kw):
     d = dict(B=2, H=4, T=4096, d_k=128, n_sub=256, d_v=128, k_half=32, W=32, R=32, x_dtype=1,
-             v_dtype=1)
+             v_dtype=1, decay=0)
     d.update(kw)
     return Dims(**d)
 
@@ -69,10 +71,20 @@ def test_workspace_and_state_sizes(lib):
     assert s.value == 2 * 4 * 65536 * 8 and l.value == 2 * 4 * 8
 
 
+def test_touched_decay_workspace(lib):
+    """decay = touched adds two fp32 records per occurrence (its in-chunk decay products)."""
+    lib.sdm_forward_workspace_bytes.restype = ctypes.c_size_t
+    a = lib.sdm_forward_workspace_bytes(ctypes.byref(mid_dims(decay=0)))
+    t = lib.sdm_forward_workspace_bytes(ctypes.byref(mid_dims(decay=1)))
+    occ = 2 * 4 * 4096 * 64
+    assert t - a == 2 * occ * 4  # both sizes are 256-byte multiples here
+    assert ctypes.sizeof(Dims) == 48
+
+
 @pytest.mark.parametrize("field,value,code", [
     ("x_dtype", 7, 3), ("v_dtype", -1, 3), ("B", 0, 2), ("T", -1, 2), ("d_k", 30, 2),
     ("d_k", 512, 2), ("n_sub", 0, 2), ("d_v", 6, 2), ("d_v", 512, 2), ("k_half", 65, 2),
-    ("k_half", 300, 2), ("W", 0, 2), ("R", 65, 2),
+    ("k_half", 300, 2), ("W", 0, 2), ("R", 65, 2), ("decay", 2, 1), ("decay", -1, 1),
 ])
 def test_bad_dims_rejected_on_host(lib, field, value, code):
     d = mid_dims(**{field: value})

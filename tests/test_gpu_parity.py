@@ -78,7 +78,9 @@ def check_selection(orc, x, sk, gpu_idx, gpu_w, k_half, top, n, max_near_frac=0.
     S.MID.scaled(B=1, H=2, T=333),
     S.HEADLINE.scaled(B=1, H=2, T=150),
     S.LONG.scaled(B=1, H=2, T=120),
-], ids=["tiny", "mid", "headline", "long"])
+    S.MID.scaled(B=3, H=2, T=70),   # one tensor-core tile per sequence, rows past T zero-filled
+    S.MID.scaled(B=3, H=1, T=64),   # two sequences per tile, the last tile's second one absent
+], ids=["tiny", "mid", "headline", "long", "mid_t70", "mid_t64_odd_b"])
 def test_score_vs_oracle(sdm, orc, wl):
     inp = to_dev(S.generate(wl, with_m0=False))
     d = dims_of(sdm, wl)
