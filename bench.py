@@ -35,8 +35,9 @@ L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 # the hash of the kernel sources it was taken with; None when not yet measured for the
 # current sources.  Filled from profiles/ (see the summary named there).
 MEASURED_TRAFFIC = {
-    # profiles/recur_run_kernel_mid_prefill.md: dram read 728.66 MB + write 406.20 MB
-    "be658b80668ed88a": 1_134_859_520,
+    # profiles/recur_run_kernel_mid_prefill.md: dram read 728.69 MB + write 405.89 MB (the
+    # plan sources changed for the touched-slots decay variant; the row pass did not)
+    "3d81af8743a81d65": 1_134_580_224,
 }
 
 
@@ -339,7 +340,8 @@ def run_gpu(args, wl, world, rank, local):
     e2e = run_e2e(args, wl, d, inp, st, sel, out, ws, device, sdm)
     errs = sdm.device_error()
 
-    # the decode workload (single-token steps), on rank 0
+    # the touched-slots decay variant of the same step, and the decode workload, on rank 0
+    touched = run_touched(wl, inp, device, sdm) if rank == 0 else None
     dec = run_decode(device, sdm) if rank == 0 and not args.no_decode else None
 
     if world > 1:
@@ -390,6 +392,7 @@ def run_gpu(args, wl, world, rank, local):
         "diagnostics": diag,
         "layer_out": layer,
         "decode": dec,
+        "touched_decay": touched,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "device_errors": errs,
@@ -475,6 +478,60 @@ def run_decode(device, sdm, steps: int = 64, warm: int = 3, n_sub: int | None = 
            "note": "state 34 GB (fp32 rows) >> L2; each step scores new tokens, so its gathers "
                    "miss L2", "device_errors": errs}
     del inp, st, qd, kd, vd, ad, bd, sel, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_touched(wl, inp, device, sdm, steps: int = 10, warm: int = 3) -> dict:
+    """The same prefill step with touched-slots decay (alpha scales only each token's write
+    slots): reset, both scorings, plan, row pass, timed per stage with the L2 flushed
+    between steps."""
+    import torch
+
+    d = sdm.Dims(wl.B, wl.H, wl.T, wl.d_k, wl.n_sub, wl.d_v, wl.k_half, wl.W, wl.R, wl.x_dtype,
+                 wl.v_dtype, decay="touched")
+    st = sdm.State(d, inp["M0"])
+    widx, ww, ridx, rw = sdm.selection_buffers(d, device)
+    out = torch.empty((wl.B, wl.H, wl.T, wl.d_v), dtype=torch.float32, device=device)
+    ws = sdm.workspace(d, device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        sdm.state_reset(d, st)
+        sdm.score_topk(d, inp["k"], inp["skw"], wl.W, widx, ww)
+        sdm.score_topk(d, inp["q"], inp["skr"], wl.R, ridx, rw)
+        if ev:
+            ev[1].record(stream)
+        sdm.forward_plan(d, inp["alpha"], inp["beta"], widx, ww, ridx, rw, st, ws)
+        if ev:
+            ev[2].record(stream)
+        sdm.forward_run(d, inp["v"], inp["beta"], widx, ww, ridx, rw, st, out, ws)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(warm):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for k in range(steps):
+        flush.zero_()
+        step(evs[k])
+    torch.cuda.synchronize()
+    errs = sdm.device_error()
+    ms = [statistics.mean(e[a].elapsed_time(e[b]) for e in evs) for a, b in ((0, 3), (0, 1), (1, 2), (2, 3))]
+    units = units_per_step(wl)
+    run_bytes = bytes_per_token_head(wl)["recurrence_kernel"] * units
+    gbs = run_bytes / (ms[3] / 1e3) / 1e9
+    peak = measured_peaks()["hbm_gbs"]
+    res = {"workload": describe(wl) + ", decay: write slots only", "steps_timed": steps,
+           "ms_per_step": ms[0], "token_heads_per_s": units / (ms[0] / 1e3),
+           "stages_ms": {"reset_and_scoring": ms[1], "plan": ms[2], "run": ms[3]},
+           "row_pass": {"achieved_gbs": gbs, "frac": gbs / peak}, "device_errors": errs}
+    del st, out, ws, flush
     torch.cuda.empty_cache()
     return res
 
