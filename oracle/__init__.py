@@ -17,6 +17,9 @@ Parity status per function:
   recur_dense ................. pinned (beta=0 closed form, one-hot write/read,
                                  dense Gated DeltaNet matrix form, hand example)
   recur_lazy .................. pinned (agrees with recur_dense to 1e-12)
+  recur_backward .............. pinned (central finite differences of recur_dense and
+                                 recur_touched for every input, beta = 0 and alpha = 1
+                                 closed form)
   recur_touched ............... pinned (hand example, alpha = 1 equals recur_dense,
                                  all slots written = recur_dense (Gated DeltaNet),
                                  beta = 0 closed form with unwritten slots at M0)
@@ -96,6 +99,8 @@ class Oracle:
         lib.sdm_oracle_recur_dense.restype = I
         lib.sdm_oracle_recur_touched.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P]
         lib.sdm_oracle_recur_touched.restype = I
+        lib.sdm_oracle_recur_backward.argtypes = [I, I, I, I, I, I] + [P] * 15
+        lib.sdm_oracle_recur_backward.restype = I
         lib.sdm_oracle_recur_lazy.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P]
         lib.sdm_oracle_recur_lazy.restype = I
         lib.sdm_oracle_materialize.argtypes = [I, I, P, P, D, P]
@@ -234,6 +239,24 @@ class Oracle:
                                                  _p(widx), _p(ww), _p(ridx), _p(rw), _p(M),
                                                  _p(out)), "recur_touched")
         return out, M
+
+    def recur_backward(self, v, alpha, beta, widx, ww, ridx, rw, M0, dout, touched=False):
+        """Gradients of one (b,h)'s recurrence for output gradient dout [T,dv] (selections
+        fixed).  Returns dict dv [T,dv], dalpha [T], dbeta [T], dww [T,W], drw [T,R],
+        dM0 [N,dv] (with respect to the state at the start)."""
+        v, alpha, beta = _f64(v), _f64(alpha), _f64(beta)
+        widx, ridx, ww, rw = _i32(widx), _i32(ridx), _f64(ww), _f64(rw)
+        M0, dout = _f64(M0), _f64(dout)
+        T, dv = v.shape
+        N = M0.shape[0]
+        W, R = widx.shape[1], ridx.shape[1]
+        g = {"dv": np.empty((T, dv)), "dalpha": np.empty(T), "dbeta": np.empty(T),
+             "dww": np.empty((T, W)), "drw": np.empty((T, R)), "dM0": np.empty((N, dv))}
+        _check(self.lib.sdm_oracle_recur_backward(
+            T, N, dv, W, R, 1 if touched else 0, _p(v), _p(alpha), _p(beta), _p(widx), _p(ww),
+            _p(ridx), _p(rw), _p(M0), _p(dout), _p(g["dv"]), _p(g["dalpha"]), _p(g["dbeta"]),
+            _p(g["dww"]), _p(g["drw"]), _p(g["dM0"])), "recur_backward")
+        return g
 
     @staticmethod
     def fresh_lazy_state(M0h):

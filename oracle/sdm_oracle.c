@@ -288,6 +288,126 @@ int sdm_oracle_recur_touched(int T, int N, int dv, int W, int R, const double* v
 }
 
 /*
+ * Gradients of the recurrence of one (b,h) with respect to its inputs, for a loss whose
+ * gradient with respect to the outputs is dout [T][dv]; the slot selections are fixed
+ * (they are not differentiated).  touched = 0: steps (i)-(v) of the dense form (every slot
+ * decays); touched = 1: step (i') instead (only the write slots decay).  Plain
+ * reverse-mode differentiation, token by token, from every state M_0..M_T kept in memory
+ * (small cases only); the pages' appendix A.3 ("Memory-Efficient Backward") recovers the
+ * states by undoing the in-place updates instead.  Per token t, backwards:
+ *   (v)   o = sum_j u_j M_t[r_j]:        du_j = <G, M_t[r_j]>,  dM[r_j] += u_j G
+ *   (iv)  M_t[s_i] = Mt[s_i] + beta w_i e  (Mt = the decayed state):
+ *         de = beta sum_i w_i dM[s_i],  dbeta = sum_i w_i <dM[s_i], e>,
+ *         dw_i = beta <dM[s_i], e>
+ *   (iii) e = v - p:                       dv = de,  dp = -de
+ *   (ii)  p = sum_i w_i Mt[s_i]:           dw_i += <dp, Mt[s_i]>,  dMt[s_i] = dM[s_i] + w_i dp
+ *   (i)   Mt = alpha M_{t-1}:              dalpha = <dMt, M_{t-1}> over every slot (the
+ *         write slots only when touched),   dM_{t-1} = alpha dMt (those slots only)
+ * G = dout[t].  Outputs: dv [T][dv], dalpha [T], dbeta [T], dww [T][W], drw [T][R] and dM0
+ * [N][dv], the gradient with respect to the state at the start of the call.
+ * §2 Background "Gated DeltaNet"; §3 Method "Sparse memory updates", "Sparse retrieval".
+ */
+int sdm_oracle_recur_backward(int T, int N, int dv, int W, int R, int touched, const double* v,
+                              const double* alpha, const double* beta, const int32_t* widx,
+                              const double* ww, const int32_t* ridx, const double* rw,
+                              const double* M0, const double* dout, double* dvv, double* dalpha,
+                              double* dbeta, double* dww, double* drw, double* dM0) {
+    if (T < 0 || N <= 0 || dv <= 0 || W <= 0 || R <= 0) return ORACLE_ERR_ARG;
+    const size_t ND = (size_t)N * dv;
+    double* S = (double*)malloc(sizeof(double) * ND * (size_t)(T + 1));  /* S[t] = M_t */
+    double* dM = (double*)calloc(ND, sizeof(double));
+    double* Mt = (double*)malloc(sizeof(double) * (size_t)W * dv);       /* decayed write rows */
+    double* p = (double*)malloc(sizeof(double) * (size_t)dv);
+    double* e = (double*)malloc(sizeof(double) * (size_t)dv);
+    double* de = (double*)malloc(sizeof(double) * (size_t)dv);
+    if (!S || !dM || !Mt || !p || !e || !de) {
+        free(S); free(dM); free(Mt); free(p); free(e); free(de);
+        return ORACLE_ERR_NOMEM;
+    }
+    int rc = ORACLE_OK;
+    memcpy(S, M0, sizeof(double) * ND);
+    for (int t = 0; t < T && rc == ORACLE_OK; ++t) {
+        const int32_t* ws = widx + (size_t)t * W;
+        const int32_t* rs = ridx + (size_t)t * R;
+        if (!check_slots(ws, W, N) || !check_slots(rs, R, N)) { rc = ORACLE_ERR_ARG; break; }
+        double* M = S + ND * (size_t)(t + 1);
+        memcpy(M, S + ND * (size_t)t, sizeof(double) * ND);
+        if (touched) {
+            for (int i = 0; i < W; ++i)
+                for (int c = 0; c < dv; ++c) M[(size_t)ws[i] * dv + c] *= alpha[t];
+        } else {
+            for (size_t q = 0; q < ND; ++q) M[q] *= alpha[t];
+        }
+        for (int c = 0; c < dv; ++c) {
+            double pc = 0.0;
+            for (int i = 0; i < W; ++i) pc += ww[(size_t)t * W + i] * M[(size_t)ws[i] * dv + c];
+            e[c] = v[(size_t)t * dv + c] - pc;
+        }
+        for (int i = 0; i < W; ++i)
+            for (int c = 0; c < dv; ++c)
+                M[(size_t)ws[i] * dv + c] += beta[t] * ww[(size_t)t * W + i] * e[c];
+    }
+    for (int t = T - 1; t >= 0 && rc == ORACLE_OK; --t) {
+        const int32_t* ws = widx + (size_t)t * W;
+        const int32_t* rs = ridx + (size_t)t * R;
+        const double* Mnow = S + ND * (size_t)(t + 1);
+        const double* Mprev = S + ND * (size_t)t;
+        const double* G = dout + (size_t)t * dv;
+        const double* wt = ww + (size_t)t * W;
+        /* (v) the read */
+        for (int j = 0; j < R; ++j) {
+            const double u = rw[(size_t)t * R + j];
+            drw[(size_t)t * R + j] = dot(G, Mnow + (size_t)rs[j] * dv, dv);
+            for (int c = 0; c < dv; ++c) dM[(size_t)rs[j] * dv + c] += u * G[c];
+        }
+        /* recompute the decayed write rows, p and e of this token */
+        for (int i = 0; i < W; ++i)
+            for (int c = 0; c < dv; ++c)
+                Mt[(size_t)i * dv + c] = alpha[t] * Mprev[(size_t)ws[i] * dv + c];
+        for (int c = 0; c < dv; ++c) {
+            double pc = 0.0;
+            for (int i = 0; i < W; ++i) pc += wt[i] * Mt[(size_t)i * dv + c];
+            p[c] = pc;
+            e[c] = v[(size_t)t * dv + c] - pc;
+        }
+        /* (iv) the write */
+        double db = 0.0;
+        for (int c = 0; c < dv; ++c) {
+            double s = 0.0;
+            for (int i = 0; i < W; ++i) s += wt[i] * dM[(size_t)ws[i] * dv + c];
+            de[c] = beta[t] * s;
+        }
+        for (int i = 0; i < W; ++i) {
+            const double ge = dot(dM + (size_t)ws[i] * dv, e, dv);
+            db += wt[i] * ge;
+            dww[(size_t)t * W + i] = beta[t] * ge;
+        }
+        dbeta[t] = db;
+        /* (iii), (ii) */
+        for (int c = 0; c < dv; ++c) dvv[(size_t)t * dv + c] = de[c];
+        for (int i = 0; i < W; ++i) {
+            dww[(size_t)t * W + i] -= dot(de, Mt + (size_t)i * dv, dv);
+            for (int c = 0; c < dv; ++c) dM[(size_t)ws[i] * dv + c] -= wt[i] * de[c];
+        }
+        /* (i) the decay */
+        double da = 0.0;
+        if (touched) {
+            for (int i = 0; i < W; ++i) {
+                da += dot(dM + (size_t)ws[i] * dv, Mprev + (size_t)ws[i] * dv, dv);
+                for (int c = 0; c < dv; ++c) dM[(size_t)ws[i] * dv + c] *= alpha[t];
+            }
+        } else {
+            for (size_t q = 0; q < ND; ++q) da += dM[q] * Mprev[q];
+            for (size_t q = 0; q < ND; ++q) dM[q] *= alpha[t];
+        }
+        dalpha[t] = da;
+    }
+    if (rc == ORACLE_OK) memcpy(dM0, dM, sizeof(double) * ND);
+    free(S); free(dM); free(Mt); free(p); free(e); free(de);
+    return rc;
+}
+
+/*
  * Lazy-decay recurrence, the same steps with decay applied only when a slot is
  * touched.  State: Mraw [N][dv], stamp [N] (log-decay prefix at the slot's last
  * write), *Lambda (running log-decay prefix).  The true slot value at the current

@@ -384,6 +384,75 @@ def pin_touched_beta_zero(o):
     assert untouched.size > 0 and np.array_equal(M_t[untouched], M0[untouched])
 
 
+# ----------------------------------------------------------------- backward ---
+
+def _fd_case(rng, T, N, dv, W, R):
+    v, alpha, beta, widx, ww, ridx, rw, M0 = _random_case(rng, T, N, dv, W, R, 0.5, 1.0)
+    # small N: slots repeat across tokens and reads meet this token's writes
+    widx = np.stack([rng.permutation(N)[:W] for _ in range(T)]).astype(np.int32)
+    ridx = np.stack([rng.permutation(N)[:R] for _ in range(T)]).astype(np.int32)
+    dout = rng.standard_normal((T, dv))
+    return v, alpha, beta, widx, ww, ridx, rw, M0, dout
+
+
+def _check_fd(o, touched, case):
+    """Central differences of L = sum(dout * out) through the forward oracle, every input."""
+    v, alpha, beta, widx, ww, ridx, rw, M0, dout = case
+    fwd = o.recur_touched if touched else o.recur_dense
+    g = o.recur_backward(v, alpha, beta, widx, ww, ridx, rw, M0, dout, touched=touched)
+
+    def loss(**kw):
+        a = dict(v=v, alpha=alpha, beta=beta, ww=ww, rw=rw, M0=M0)
+        a.update(kw)
+        out, _ = fwd(a["v"], a["alpha"], a["beta"], widx, a["ww"], ridx, a["rw"], a["M0"])
+        return float((dout * out).sum())
+
+    h = 1e-6
+    for name, arr, key in (("v", v, "dv"), ("alpha", alpha, "dalpha"), ("beta", beta, "dbeta"),
+                           ("ww", ww, "dww"), ("rw", rw, "drw"), ("M0", M0, "dM0")):
+        num = np.empty_like(arr)
+        for idx in np.ndindex(arr.shape):
+            ap, am = arr.copy(), arr.copy()
+            ap[idx] += h
+            am[idx] -= h
+            num[idx] = (loss(**{name: ap}) - loss(**{name: am})) / (2 * h)
+        np.testing.assert_allclose(g[key], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def pin_backward_finite_differences(o):
+    """The backward equals central differences of the forward (every slot decays)."""
+    rng = _rng(16)
+    _check_fd(o, False, _fd_case(rng, 7, 6, 3, 2, 3))
+    _check_fd(o, False, _fd_case(rng, 5, 4, 2, 4, 4))  # every slot written at every token
+
+
+def pin_backward_touched_finite_differences(o):
+    """The backward equals central differences of the forward (only the write slots decay)."""
+    rng = _rng(17)
+    _check_fd(o, True, _fd_case(rng, 7, 6, 3, 2, 3))
+    _check_fd(o, True, _fd_case(rng, 6, 9, 2, 3, 2))
+
+
+def pin_backward_frozen_memory(o):
+    """beta = 0, alpha = 1: the memory stays M0, so o_t = sum_j u_j M0[r_j] and
+    dM0[s] = sum over (t, j) with r_j = s of u_j dout_t, du_j = <dout_t, M0[r_j]>,
+    dv = dw = 0 (no write moves the memory)."""
+    rng = _rng(18)
+    T, N, dv, W, R = 9, 8, 3, 2, 3
+    v, alpha, beta, widx, ww, ridx, rw, M0, dout = _fd_case(rng, T, N, dv, W, R)
+    for touched in (False, True):
+        g = o.recur_backward(v, np.ones(T), np.zeros(T), widx, ww, ridx, rw, M0, dout,
+                             touched=touched)
+        expect = np.zeros_like(M0)
+        for t in range(T):
+            for j in range(R):
+                expect[ridx[t, j]] += rw[t, j] * dout[t]
+        np.testing.assert_allclose(g["dM0"], expect, rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(g["drw"], np.einsum("tc,tjc->tj", dout, M0[ridx]),
+                                   rtol=1e-13, atol=1e-14)
+        assert np.array_equal(g["dv"], np.zeros((T, dv))) and np.array_equal(g["dww"], np.zeros((T, W)))
+
+
 def pin_prefill_pairs(o):
     """The batched prefill equals product-key scoring followed by the lazy recurrence."""
     rng = _rng(12)
@@ -575,4 +644,6 @@ ALL_PINS = [pin_pk_equals_brute, pin_brute_matches_numpy, pin_pk_depends_on_k, p
             pin_hand_recurrence, pin_prefill_pairs, pin_weight_stats_closed_forms,
             pin_weight_stats_summaries, pin_layer_out_hand_example, pin_layer_out_properties,
             pin_layer_in_routing_and_gates, pin_layer_in_linear, pin_touched_hand,
-            pin_touched_alpha_one, pin_touched_all_slots_gdn, pin_touched_beta_zero]
+            pin_touched_alpha_one, pin_touched_all_slots_gdn, pin_touched_beta_zero,
+            pin_backward_finite_differences, pin_backward_touched_finite_differences,
+            pin_backward_frozen_memory]

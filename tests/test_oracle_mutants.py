@@ -23,6 +23,16 @@ MUTANTS = {
         ("for (int c = 0; c < dv; ++c) M[(size_t)ws[i] * dv + c] *= alpha[t];",
          "for (int c = 0; c < dv; ++c) M[(size_t)ws[i] * dv + c] *= 1.0;"),
     ],
+    "backward_prediction_term_dropped": [
+        ("dww[(size_t)t * W + i] -= dot(de, Mt + (size_t)i * dv, dv);", "(void)0;"),
+    ],
+    "backward_decay_not_propagated": [
+        ("for (size_t q = 0; q < ND; ++q) dM[q] *= alpha[t];", "(void)0;"),
+    ],
+    "backward_error_gradient_sign": [
+        ("for (int c = 0; c < dv; ++c) dM[(size_t)ws[i] * dv + c] -= wt[i] * de[c];",
+         "for (int c = 0; c < dv; ++c) dM[(size_t)ws[i] * dv + c] += wt[i] * de[c];"),
+    ],
     "touched_decay_hits_every_slot": [
         ("for (int c = 0; c < dv; ++c) M[(size_t)ws[i] * dv + c] *= alpha[t];",
          "if (i == 0) for (size_t q = 0; q < (size_t)N * dv; ++q) M[q] *= alpha[t];"),
