@@ -228,6 +228,36 @@ sdm_status sdm_decode_step(const sdm_dims* dims, const void* q, const void* k, c
                            int32_t* ridx, float* rw, float* out, sdm_stream_t stream);
 
 /*
+ * Backward of the recurrence over one call of T tokens (Sparse Delta Memory summary,
+ * appendix A.3 "Memory-Efficient Backward"): gradients with respect to v, alpha, beta and
+ * the write and read weights, and with respect to the memory at the start of the call, for
+ * an output gradient dout; the slot selections are fixed (not differentiated), under the
+ * dims' decay rule.
+ *   st    the state at the START of the call (as it was passed to the sdm_forward that
+ *         produced the outputs).  The call replays the T tokens in place, logging the raw
+ *         rows and stamps of each token's write slots before the write (the T*W*d_v record
+ *         of the workspace), then walks the tokens backwards, restoring each token's write
+ *         slots from the log: on return the state is again the start state (the memory is
+ *         never copied; peak memory O(N*d_v + T*W*d_v) per sequence).
+ *   dout  [B][H][T][d_v] fp32 gradient of the loss with respect to out
+ *   outputs, fp32, caller-allocated, every element written:
+ *         dv [B][H][T][d_v], dalpha [B][H][T], dbeta [B][H][T], dww [B][H][T][W],
+ *         drw [B][H][T][R], dM_in [B][H][N][d_v] (with respect to the true slot values at
+ *         the start; for a fresh state, summing it over b gives the gradient of M0)
+ *   ws    device workspace of at least sdm_backward_workspace_bytes(dims) bytes, 16-byte
+ *         aligned.
+ * This first version walks the tokens of each sequence one at a time (one CTA per (b,h)).
+ * Errors: as sdm_forward; W + R <= 128; the slots must be in range and distinct within a
+ * token.
+ */
+size_t sdm_backward_workspace_bytes(const sdm_dims* dims);
+sdm_status sdm_backward(const sdm_dims* dims, const void* v, const float* alpha, const float* beta,
+                        const int32_t* widx, const float* ww, const int32_t* ridx, const float* rw,
+                        const sdm_state* st, const float* dout, float* dv, float* dalpha,
+                        float* dbeta, float* dww, float* drw, float* dM_in, void* ws,
+                        size_t ws_bytes, sdm_stream_t stream);
+
+/*
  * sdm_forward without a caller workspace and without any allocation: for callers that
  * cannot call cudaMalloc or hand out scratch memory themselves — for example a custom
  * operator inside a host framework that owns the device allocator and forbids side

@@ -92,6 +92,8 @@ def _load():
         "sdm_decode_step": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P], I32),
         "sdm_device_error": ([ctypes.POINTER(ctypes.c_uint32), I32, P], I32),
         "sdm_forward_noalloc": ([D, P, P, P, P, P, P, P, S, P, P], I32),
+        "sdm_backward_workspace_bytes": ([D], SZ),
+        "sdm_backward": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P, P, P, SZ, P], I32),
         "sdm_gemm_bf16": ([I32, I32, I32, P, P, P, P], I32),
         "sdm_layer_in_workspace_bytes": ([D], SZ),
         "sdm_layer_in": ([D, P, P, P, P, I32, P, P, P, P, P, P, P, SZ, P], I32),
@@ -277,6 +279,38 @@ def prefill(d: Dims, q, k, v, alpha, beta, skw, skr, st: State, sel=None, out=No
                          _ptr(out, "out", torch.float32), _ptr(ws, "ws"), ws.numel(),
                          _stream(stream)), "sdm_prefill")
     return out, sel
+
+
+def backward_workspace_bytes(d: Dims) -> int:
+    return int(_lib.sdm_backward_workspace_bytes(ctypes.byref(d)))
+
+
+def backward(d: Dims, v, alpha, beta, widx, ww, ridx, rw, st: State, dout, ws=None, grads=None,
+             stream=None) -> dict:
+    """sdm_backward: gradients of the recurrence over one call for the output gradient dout
+    [B,H,T,d_v] fp32.  `st` must hold the state at the start of the call; it is replayed and
+    restored in place.  Returns dict dv, dalpha, dbeta, dww, drw, dM_in (fp32)."""
+    dev = v.device
+    if ws is None:
+        ws = torch.empty(max(16, backward_workspace_bytes(d)), dtype=torch.uint8, device=dev)
+    if grads is None:
+        f = dict(dtype=torch.float32, device=dev)
+        grads = {"dv": torch.empty((d.B, d.H, d.T, d.d_v), **f),
+                 "dalpha": torch.empty((d.B, d.H, d.T), **f),
+                 "dbeta": torch.empty((d.B, d.H, d.T), **f),
+                 "dww": torch.empty((d.B, d.H, d.T, d.W), **f),
+                 "drw": torch.empty((d.B, d.H, d.T, d.R), **f),
+                 "dM_in": torch.empty((d.B, d.H, d.N, d.d_v), **f)}
+    a = _fw_args(d, v, alpha, beta, widx, ww, ridx, rw)
+    g = grads
+    _ok(_lib.sdm_backward(ctypes.byref(d), *a, ctypes.byref(st.c),
+                          _ptr(dout, "dout", torch.float32), _ptr(g["dv"], "dv", torch.float32),
+                          _ptr(g["dalpha"], "dalpha", torch.float32),
+                          _ptr(g["dbeta"], "dbeta", torch.float32),
+                          _ptr(g["dww"], "dww", torch.float32), _ptr(g["drw"], "drw", torch.float32),
+                          _ptr(g["dM_in"], "dM_in", torch.float32), _ptr(ws, "ws"), ws.numel(),
+                          _stream(stream)), "sdm_backward")
+    return grads
 
 
 def decode_step(d: Dims, q, k, v, alpha, beta, skw, skr, st: State, sel=None, out=None,

@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "backward.cuh"
 #include "decode.cuh"
 #include "plan.cuh"
 #include "recur.cuh"
@@ -342,6 +343,45 @@ sdm_status score_both_roles(const sdm_dims* d, const void* q, const void* k, con
     return launch_score(d, q, skr, d->R, ridx, rw, s);
 }
 
+struct BwdLayout {
+    size_t off_rows, off_lstamp, off_lam, off_dM, off_dstamp, total;
+};
+
+BwdLayout bwd_layout(const sdm_dims* d) {
+    BwdLayout L{};
+    const size_t BH = (size_t)BH_of(d), T = (size_t)d->T, N = (size_t)N_of(d);
+    size_t o = 0;
+    L.off_rows = o;   o = up256(o + BH * T * (size_t)d->W * d->d_v * 4);
+    L.off_lstamp = o; o = up256(o + BH * T * (size_t)d->W * 8);
+    L.off_lam = o;    o = up256(o + BH * (T + 1) * 8);
+    L.off_dM = o;     o = up256(o + BH * N * (size_t)d->d_v * 4);
+    L.off_dstamp = o; o = up256(o + BH * N * 8);
+    L.total = o;
+    return L;
+}
+
+template <typename VT, int QPL, int WPW>
+sdm_status launch_backward_t(const sdm_dims* d, const BwdPtrs& P, const void* v,
+                             const float* alpha, const float* beta, const int32_t* widx,
+                             const float* ww, const int32_t* ridx, const float* rw,
+                             const sdm_state* st, const float* dout, float* dv, float* dalpha,
+                             float* dbeta, float* dww, float* drw, cudaStream_t s) {
+    const int touched = d->decay == SDM_DECAY_TOUCHED;
+    const size_t smem = bwd_smem_bytes(d->d_v);
+    auto rk = bwd_replay_kernel<VT, QPL, WPW>;
+    auto sk = bwd_sweep_kernel<VT, QPL, WPW>;
+    if (!set_smem(rk, smem) || !set_smem(sk, smem)) return SDM_ERR_CUDA;
+    const unsigned grid = (unsigned)BH_of(d);
+    rk<<<grid, BWD_THREADS, smem, s>>>((const VT*)v, alpha, beta, widx, ww, st->M, st->stamp,
+                                       st->Lambda, st->M0, P, d->H, (int)N_of(d), d->T, d->d_v,
+                                       d->W, touched);
+    sk<<<grid, BWD_THREADS, smem, s>>>((const VT*)v, alpha, beta, widx, ww, ridx, rw, st->M,
+                                       st->stamp, st->Lambda, st->M0, P, dout, dv, dalpha, dbeta,
+                                       dww, drw, d->H, (int)N_of(d), d->T, d->d_v, d->W, d->R,
+                                       touched);
+    return launch_status();
+}
+
 template <typename VT, int RPW, int QPL>
 sdm_status launch_decode(const sdm_dims* d, const void* v, const float* alpha, const float* beta,
                          const sdm_state* st, const int32_t* widx, const float* ww,
@@ -652,6 +692,68 @@ sdm_status sdm_decode_step(const sdm_dims* dims, const void* q, const void* k, c
                           : launch_decode<float, 8, 2>(dims, v, alpha, beta, st, widx, ww, ridx, rw, out, stream);
     }
     return e;
+}
+
+size_t sdm_backward_workspace_bytes(const sdm_dims* dims) {
+    if (check_dims(dims) != SDM_OK) return 0;
+    return bwd_layout(dims).total;
+}
+
+sdm_status sdm_backward(const sdm_dims* dims, const void* v, const float* alpha, const float* beta,
+                        const int32_t* widx, const float* ww, const int32_t* ridx, const float* rw,
+                        const sdm_state* st, const float* dout, float* dv, float* dalpha,
+                        float* dbeta, float* dww, float* drw, float* dM_in, void* ws,
+                        size_t ws_bytes, sdm_stream_t stream) {
+    sdm_status e = check_dims(dims);
+    if (e) return e;
+    if ((e = check_state(st))) return e;
+    if (!v || !alpha || !beta || !widx || !ww || !ridx || !rw || !dout || !dv || !dalpha ||
+        !dbeta || !dww || !drw || !dM_in)
+        return SDM_ERR_ARG;
+    if (!aligned16(v) || !aligned16(dout) || !aligned16(dv) || !aligned16(dM_in))
+        return SDM_ERR_ALIGN;
+    if (dims->W + dims->R > BWD_MAXO) return SDM_ERR_SHAPE;
+    const BwdLayout L = bwd_layout(dims);
+    if (!ws || ws_bytes < L.total) return SDM_ERR_WORKSPACE;
+    if (!aligned16(ws)) return SDM_ERR_ALIGN;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t rows = (size_t)BH_of(dims) * (size_t)N_of(dims);
+    unsigned char* b = static_cast<unsigned char*>(ws);
+    BwdPtrs P;
+    P.log_rows = reinterpret_cast<float*>(b + L.off_rows);
+    P.log_stamp = reinterpret_cast<double*>(b + L.off_lstamp);
+    P.log_lam = reinterpret_cast<double*>(b + L.off_lam);
+    P.dM = reinterpret_cast<float*>(b + L.off_dM);
+    P.dstamp = reinterpret_cast<double*>(b + L.off_dstamp);
+    const int threads = 256;
+    {   // every memory-gradient row starts at zero (NaN stamp)
+        size_t blocks = (rows + threads - 1) / threads;
+        if (blocks > 148 * 64) blocks = 148 * 64;
+        if (blocks == 0) blocks = 1;
+        state_reset_kernel<<<(unsigned)blocks, threads, 0, s>>>(P.dstamp, rows, nullptr, 0);
+    }
+    if (dims->T > 0) {
+        const int wpw = ((dims->W > dims->R ? dims->W : dims->R) + BWD_WARPS - 1) / BWD_WARPS;
+        const bool q2 = dims->d_v > 128;
+#define SDM_BWD(VT, Q, WP) launch_backward_t<VT, Q, WP>(dims, P, v, alpha, beta, widx, ww, ridx, rw, st, dout, dv, dalpha, dbeta, dww, drw, s)
+        if (dims->v_dtype == SDM_BF16) {
+            if (wpw <= 4) e = q2 ? SDM_BWD(__nv_bfloat16, 2, 4) : SDM_BWD(__nv_bfloat16, 1, 4);
+            else e = q2 ? SDM_BWD(__nv_bfloat16, 2, 8) : SDM_BWD(__nv_bfloat16, 1, 8);
+        } else {
+            if (wpw <= 4) e = q2 ? SDM_BWD(float, 2, 4) : SDM_BWD(float, 1, 4);
+            else e = q2 ? SDM_BWD(float, 2, 8) : SDM_BWD(float, 1, 8);
+        }
+#undef SDM_BWD
+        if (e) return e;
+    } else if (cudaMemsetAsync(P.log_lam, 0, (size_t)BH_of(dims) * 8, s) != cudaSuccess) {
+        return SDM_ERR_CUDA;  // no token: the dense gradient's final prefix is 0
+    }
+    size_t blocks = (rows * (dims->d_v / 4) + threads - 1) / threads;
+    if (blocks > 148 * 64) blocks = 148 * 64;
+    if (blocks == 0) blocks = 1;
+    bwd_dense_kernel<<<(unsigned)blocks, threads, 0, s>>>(P, dims->T, (int)N_of(dims), dims->d_v,
+                                                          rows, dM_in);
+    return launch_status();
 }
 
 sdm_status sdm_forward_noalloc(const sdm_dims* dims, const void* v, const float* alpha,
