@@ -35,9 +35,9 @@ L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 # the hash of the kernel sources it was taken with; None when not yet measured for the
 # current sources.  Filled from profiles/ (see the summary named there).
 MEASURED_TRAFFIC = {
-    # profiles/recur_run_kernel_mid_prefill.md: dram read 728.69 MB + write 405.89 MB (the
+    # profiles/recur_run_kernel_mid_prefill.md: dram read 728.75 MB + write 405.35 MB (the
     # plan sources changed for the touched-slots decay variant; the row pass did not)
-    "3d81af8743a81d65": 1_134_580_224,
+    "e64fe2a7f5e03e49": 1_134_104_064,
 }
 
 
@@ -342,6 +342,7 @@ def run_gpu(args, wl, world, rank, local):
 
     # the touched-slots decay variant of the same step, and the decode workload, on rank 0
     touched = run_touched(wl, inp, device, sdm) if rank == 0 else None
+    bwd = run_backward(wl, inp, sel, device, sdm) if rank == 0 else None
     dec = run_decode(device, sdm) if rank == 0 and not args.no_decode else None
 
     if world > 1:
@@ -393,6 +394,7 @@ def run_gpu(args, wl, world, rank, local):
         "layer_out": layer,
         "decode": dec,
         "touched_decay": touched,
+        "backward": bwd,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "device_errors": errs,
@@ -532,6 +534,50 @@ def run_touched(wl, inp, device, sdm, steps: int = 10, warm: int = 3) -> dict:
            "stages_ms": {"reset_and_scoring": ms[1], "plan": ms[2], "run": ms[3]},
            "row_pass": {"achieved_gbs": gbs, "frac": gbs / peak}, "device_errors": errs}
     del st, out, ws, flush
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_backward(wl, inp, sel, device, sdm, reps: int = 2) -> dict:
+    """Backward of the recurrence over the whole prefill call (sdm_backward: in-place replay
+    with the write-slot log, then the reverse sweep that restores the state), for the step's
+    selections and a seeded output gradient, timed with CUDA events."""
+    import torch
+
+    d = sdm.Dims(wl.B, wl.H, wl.T, wl.d_k, wl.n_sub, wl.d_v, wl.k_half, wl.W, wl.R, wl.x_dtype,
+                 wl.v_dtype)
+    st = sdm.State(d, inp["M0"])
+    sdm.state_reset(d, st)
+    gen = torch.Generator(device=device).manual_seed(wl.seed + 29)
+    dout = torch.randn(wl.B, wl.H, wl.T, wl.d_v, device=device, generator=gen)
+    ws = torch.empty(max(16, sdm.backward_workspace_bytes(d)), dtype=torch.uint8, device=device)
+    widx, ww, ridx, rw = sel
+    args = (inp["v"], inp["alpha"], inp["beta"], widx, ww, ridx, rw)
+    grads = sdm.backward(d, *args, st, dout, ws=ws)  # warm-up (also the first allocation)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        sdm.backward(d, *args, st, dout, ws=ws, grads=grads)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    errs = sdm.device_error()
+    ms = e0.elapsed_time(e1) / reps
+    units = units_per_step(wl)
+    # per token.head: replay 3W rows (gather, log, store); sweep 3R (M, dM in, dM out) and 5W
+    # (M_t, log, dM in, dM out, restore) rows of d_v fp32, plus the dense gradient once
+    rows = (8 * wl.W + 3 * wl.R) * wl.d_v * 4
+    total = rows * units + wl.B * wl.H * wl.N * wl.d_v * 4
+    gbs = total / (ms / 1e3) / 1e9
+    peak = measured_peaks()["hbm_gbs"]
+    res = {"workload": describe(wl) + ", backward of the recurrence (selections fixed)",
+           "ms": ms, "token_heads_per_s": units / (ms / 1e3),
+           "roofline": {"bound": "hbm", "algorithmic_bytes": total, "achieved_gbs": gbs,
+                        "peak": peak, "frac": gbs / peak},
+           "note": "first version: one CTA per (b,h) walks the tokens one at a time",
+           "device_errors": errs}
+    del st, ws, grads, dout
     torch.cuda.empty_cache()
     return res
 

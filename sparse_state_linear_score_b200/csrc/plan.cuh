@@ -156,6 +156,8 @@ __host__ __device__ inline RunImg run_img(int C, int W, int R) {
     return m;
 }
 
+// TOUCHED: touched-slots decay (PlanPtrs::vfc and vsh are set); the default decays every slot.
+template <bool TOUCHED>
 __global__ void __launch_bounds__(PLAN_THREADS, 2) plan_local_kernel(
     const float* __restrict__ alpha, const float* __restrict__ beta,
     const int32_t* __restrict__ widx, const float* __restrict__ ww,
@@ -186,13 +188,13 @@ __global__ void __launch_bounds__(PLAN_THREADS, 2) plan_local_kernel(
     const int nt = min(C, T - t0);
     const int nw = nt * W, no = nt * (W + R);
     const size_t occ_base = bh * (size_t)T * (W + R);
-    const bool touched = P.vfc != nullptr;  // alpha scales only the write slots
+    constexpr bool touched = TOUCHED;  // alpha scales only the write slots
 
     // 1. chunk-relative log-decay prefix (C <= PLAN_THREADS tokens per chunk)
     double la = 0.0;
     if (tid < nt) {
         const float a = alpha[bh * T + t0 + tid];
-        s_alf[tid] = a;
+        if (TOUCHED) s_alf[tid] = a;
         if (a > 0.f) {
             la = log((double)a);
         } else {
@@ -311,7 +313,7 @@ __global__ void __launch_bounds__(PLAN_THREADS, 2) plan_local_kernel(
                 const bool in = base + lane < n_i;
                 const float wo = in ? s_wt[o] : 0.f;
                 int L = in ? s_link[o] : -1;
-                float chain = rd ? 1.f : s_alf[t];  // touched: decay of the next term
+                float chain = TOUCHED ? (rd ? 1.f : s_alf[t]) : 0.f;  // decay of the next term
                 while (__any_sync(0xffffffffu, L >= 0)) {
                     int tp = 0;
                     float val = 0.f;
@@ -613,6 +615,7 @@ __global__ void __launch_bounds__(WALK_THREADS) plan_walk_kernel(
 // The row pass's inputs from the final decay factors: the gather words (slot, pristine flag)
 // and the chunk image (coefficients, store factors, links, the list of occurrences whose row
 // the previous chunk stores — in any order — and beta).
+template <bool TOUCHED>
 __global__ void __launch_bounds__(PLAN_THREADS) plan_pack_kernel(
     double* __restrict__ stamp, const float* __restrict__ beta, const int32_t* __restrict__ widx,
     const float* __restrict__ ww, const int32_t* __restrict__ ridx,
@@ -667,15 +670,15 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_pack_kernel(
                                         s_lam[o < nw ? o / W : (o - nw) / R], P.st0[g])
                            : P.fe[g];
         // touched-slots decay: the same pristine sign, the in-chunk product as the magnitude
-        if (P.vfc && ok) f = copysignf(P.vfc[g], f);
+        if (TOUCHED && ok) f = copysignf(P.vfc[g], f);
         rs[o] = ok ? (int32_t)((uint32_t)s | (signbit(f) ? 0x80000000u : 0u)) : 0x7fffffff;
         coef[ci] = ok ? w * fabsf(f) : 0.f;
         if (o < nw) {
             // shares of the stored (chunk-end) value: the d of this write, the gathered row
-            const float e = P.vfc ? 1.f : expf(lam_end - s_lam[o / W]);
+            const float e = TOUCHED ? 1.f : expf(lam_end - s_lam[o / W]);
             wslot[o] = ok ? s : 0x7fffffff;
             wlk[o] = lk;
-            sc[o] = w * (P.vfc ? P.vsh[g] : e);
+            sc[o] = w * (TOUCHED ? P.vsh[g] : e);
             sa[o] = fabsf(f) * e;
         }
         const int pv = lk_prev(lk);

@@ -584,9 +584,10 @@ sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const floa
     if (P.mask &&
         cudaMemsetAsync(P.mask, 0, BH * (size_t)N * L.MW * 8, stream) != cudaSuccess)
         return SDM_ERR_CUDA;
-    if (!set_smem(plan_local_kernel, plan_local_smem_bytes())) return SDM_ERR_CUDA;
-    plan_local_kernel<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, plan_local_smem_bytes(),
-                        stream>>>(
+    const bool touched = dims->decay == SDM_DECAY_TOUCHED;
+    auto local = touched ? plan_local_kernel<true> : plan_local_kernel<false>;
+    if (!set_smem(local, plan_local_smem_bytes())) return SDM_ERR_CUDA;
+    local<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, plan_local_smem_bytes(), stream>>>(
         alpha, beta, widx, ww, ridx, rw, st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, P);
     if ((e = launch_status())) return e;
     plan_prefix_kernel<<<(unsigned)BH, 1024, 0, stream>>>(st->Lambda, L.J, P);
@@ -601,7 +602,8 @@ sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const floa
         if ((e = launch_status())) return e;
     }
     // with the masks, plan_pack computes the final factors and stamps itself
-    plan_pack_kernel<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, 0, stream>>>(
+    auto pack = touched ? plan_pack_kernel<true> : plan_pack_kernel<false>;
+    pack<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, 0, stream>>>(
         st->stamp, beta, widx, ww, ridx, rw, dims->T, N, dims->W, dims->R, L.C, L.J, P);
     return launch_status();
 }
