@@ -20,6 +20,8 @@ Parity status per function:
   recur_backward .............. pinned (central finite differences of recur_dense and
                                  recur_touched for every input, beta = 0 and alpha = 1
                                  closed form)
+  score_backward .............. pinned (central finite differences of the softmax of the
+                                 selected slots' half-score sums, for x and the tables)
   recur_touched ............... pinned (hand example, alpha = 1 equals recur_dense,
                                  all slots written = recur_dense (Gated DeltaNet),
                                  beta = 0 closed form with unwritten slots at M0)
@@ -101,6 +103,8 @@ class Oracle:
         lib.sdm_oracle_recur_touched.restype = I
         lib.sdm_oracle_recur_backward.argtypes = [I, I, I, I, I, I] + [P] * 15
         lib.sdm_oracle_recur_backward.restype = I
+        lib.sdm_oracle_score_backward.argtypes = [P, P, I, I, I, I, P, P, P, P]
+        lib.sdm_oracle_score_backward.restype = I
         lib.sdm_oracle_recur_lazy.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P]
         lib.sdm_oracle_recur_lazy.restype = I
         lib.sdm_oracle_materialize.argtypes = [I, I, P, P, D, P]
@@ -239,6 +243,29 @@ class Oracle:
                                                  _p(widx), _p(ww), _p(ridx), _p(rw), _p(M),
                                                  _p(out)), "recur_touched")
         return out, M
+
+    def score_backward(self, x, sk, idx, dw):
+        """Gradient through the scoring with the selections idx [B,H,T,top] fixed.
+        x [B,H,T,2h], sk [H,2,n,h], dw [B,H,T,top].  Returns (dx like x, dsk like sk)."""
+        x, sk, dw = _f64(x), _f64(sk), _f64(dw)
+        idx = _i32(idx)
+        B, H, T, dk = x.shape
+        n, hd = sk.shape[2], sk.shape[3]
+        top = idx.shape[-1]
+        dx = np.empty_like(x)
+        dsk = np.zeros_like(sk)
+        for h in range(H):
+            xh = np.ascontiguousarray(x[:, h].reshape(B * T, dk))
+            ih = np.ascontiguousarray(idx[:, h].reshape(B * T, top))
+            dwh = np.ascontiguousarray(dw[:, h].reshape(B * T, top))
+            dxh = np.empty_like(xh)
+            dskh = np.zeros_like(sk[h])
+            _check(self.lib.sdm_oracle_score_backward(_p(xh), _p(np.ascontiguousarray(sk[h])),
+                                                      B * T, n, hd, top, _p(ih), _p(dwh),
+                                                      _p(dxh), _p(dskh)), "score_backward")
+            dx[:, h] = dxh.reshape(B, T, dk)
+            dsk[h] = dskh
+        return dx, dsk
 
     def recur_backward(self, v, alpha, beta, widx, ww, ridx, rw, M0, dout, touched=False):
         """Gradients of one (b,h)'s recurrence for output gradient dout [T,dv] (selections

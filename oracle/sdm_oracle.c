@@ -182,6 +182,56 @@ int sdm_oracle_score(const double* x, const double* sk, int B, int H, int T, int
     return rc;
 }
 
+/*
+ * Gradient through the scoring of `rows` vectors x [rows][2*hd] of one head against that
+ * head's sub-key tables sk [2][n][hd], the selected slots idx [rows][top] held fixed:
+ * with score_q = <x[0:hd], C1[i_q]> + <x[hd:2hd], C2[j_q]> (slot = i_q*n + j_q) and
+ * w = softmax(score) over the selected slots (§2 Background "Product Key Memory", §3
+ * Method "Sparse addressing", §4 "SDM Configuration"), for dw [rows][top]:
+ *   dscore_q = w_q (dw_q - sum_r w_r dw_r)
+ *   dx[0:hd] = sum_q dscore_q C1[i_q],   dx[hd:] = sum_q dscore_q C2[j_q]
+ *   dsk[0][i] += sum_{q: i_q = i} dscore_q x[0:hd],   dsk[1][j] likewise with x[hd:]
+ * The weights are recomputed from x and the tables.  dx [rows][2*hd] is written; dsk
+ * [2][n][hd] is added to.
+ */
+int sdm_oracle_score_backward(const double* x, const double* sk, int rows, int n, int hd,
+                              int top, const int32_t* idx, const double* dw, double* dx,
+                              double* dsk) {
+    if (rows < 0 || n <= 0 || hd <= 0 || top <= 0) return ORACLE_ERR_ARG;
+    double* sc = (double*)malloc(sizeof(double) * (size_t)top);
+    double* w = (double*)malloc(sizeof(double) * (size_t)top);
+    double* ds = (double*)malloc(sizeof(double) * (size_t)top);
+    if (!sc || !w || !ds) { free(sc); free(w); free(ds); return ORACLE_ERR_NOMEM; }
+    const double* c1 = sk;
+    const double* c2 = sk + (size_t)n * hd;
+    for (int r = 0; r < rows; ++r) {
+        const double* xr = x + (size_t)r * 2 * hd;
+        const int32_t* id = idx + (size_t)r * top;
+        for (int q = 0; q < top; ++q) {
+            if (id[q] < 0 || id[q] >= n * n) { free(sc); free(w); free(ds); return ORACLE_ERR_ARG; }
+            const int i = id[q] / n, j = id[q] % n;
+            sc[q] = dot(xr, c1 + (size_t)i * hd, hd) + dot(xr + hd, c2 + (size_t)j * hd, hd);
+        }
+        softmax(sc, top, w);
+        double s = 0.0;
+        for (int q = 0; q < top; ++q) s += w[q] * dw[(size_t)r * top + q];
+        for (int q = 0; q < top; ++q) ds[q] = w[q] * (dw[(size_t)r * top + q] - s);
+        double* dxr = dx + (size_t)r * 2 * hd;
+        for (int d = 0; d < 2 * hd; ++d) dxr[d] = 0.0;
+        for (int q = 0; q < top; ++q) {
+            const int i = id[q] / n, j = id[q] % n;
+            for (int d = 0; d < hd; ++d) {
+                dxr[d] += ds[q] * c1[(size_t)i * hd + d];
+                dxr[hd + d] += ds[q] * c2[(size_t)j * hd + d];
+                dsk[(size_t)i * hd + d] += ds[q] * xr[d];
+                dsk[(size_t)n * hd + (size_t)j * hd + d] += ds[q] * xr[hd + d];
+            }
+        }
+    }
+    free(sc); free(w); free(ds);
+    return ORACLE_OK;
+}
+
 /* ------------------------------------------------------------------------- */
 /* Recurrence for one (b,h).                                                  */
 /* ------------------------------------------------------------------------- */

@@ -453,6 +453,40 @@ def pin_backward_frozen_memory(o):
         assert np.array_equal(g["dv"], np.zeros((T, dv))) and np.array_equal(g["dww"], np.zeros((T, W)))
 
 
+def pin_score_backward_finite_differences(o):
+    """The scoring backward equals central differences of L = sum dw * softmax(scores of the
+    fixed selected slots), the scores written out here from the definition, for x and both
+    sub-key tables."""
+    rng = _rng(19)
+    B, H, T, n, hd, top = 2, 2, 3, 5, 3, 6
+    x = rng.standard_normal((B, H, T, 2 * hd))
+    sk = rng.standard_normal((H, 2, n, hd))
+    idx = np.stack([rng.permutation(n * n)[:top] for _ in range(B * H * T)]).reshape(B, H, T, top)
+    dw = rng.standard_normal((B, H, T, top))
+
+    def loss(x, sk):
+        tot = 0.0
+        for b in range(B):
+            for h in range(H):
+                for t in range(T):
+                    i, j = idx[b, h, t] // n, idx[b, h, t] % n
+                    sc = sk[h, 0, i] @ x[b, h, t, :hd] + sk[h, 1, j] @ x[b, h, t, hd:]
+                    e = np.exp(sc - sc.max())
+                    tot += float(dw[b, h, t] @ (e / e.sum()))
+        return tot
+
+    dx, dsk = o.score_backward(x, sk, idx, dw)
+    eps = 1e-6
+    for arr, g, isx in ((x, dx, True), (sk, dsk, False)):
+        num = np.empty_like(arr)
+        for ix in np.ndindex(arr.shape):
+            ap, am = arr.copy(), arr.copy()
+            ap[ix] += eps
+            am[ix] -= eps
+            num[ix] = ((loss(ap, sk) - loss(am, sk)) if isx else (loss(x, ap) - loss(x, am))) / (2 * eps)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8)
+
+
 def pin_prefill_pairs(o):
     """The batched prefill equals product-key scoring followed by the lazy recurrence."""
     rng = _rng(12)
@@ -646,4 +680,4 @@ ALL_PINS = [pin_pk_equals_brute, pin_brute_matches_numpy, pin_pk_depends_on_k, p
             pin_layer_in_routing_and_gates, pin_layer_in_linear, pin_touched_hand,
             pin_touched_alpha_one, pin_touched_all_slots_gdn, pin_touched_beta_zero,
             pin_backward_finite_differences, pin_backward_touched_finite_differences,
-            pin_backward_frozen_memory]
+            pin_backward_frozen_memory, pin_score_backward_finite_differences]

@@ -33,6 +33,13 @@ MUTANTS = {
         ("for (int c = 0; c < dv; ++c) dM[(size_t)ws[i] * dv + c] -= wt[i] * de[c];",
          "for (int c = 0; c < dv; ++c) dM[(size_t)ws[i] * dv + c] += wt[i] * de[c];"),
     ],
+    "score_backward_softmax_centre_dropped": [
+        ("for (int q = 0; q < top; ++q) ds[q] = w[q] * (dw[(size_t)r * top + q] - s);",
+         "for (int q = 0; q < top; ++q) ds[q] = w[q] * dw[(size_t)r * top + q];"),
+    ],
+    "score_backward_halves_crossed": [
+        ("dsk[(size_t)i * hd + d] += ds[q] * xr[d];", "dsk[(size_t)i * hd + d] += ds[q] * xr[hd + d];"),
+    ],
     "touched_decay_hits_every_slot": [
         ("for (int c = 0; c < dv; ++c) M[(size_t)ws[i] * dv + c] *= alpha[t];",
          "if (i == 0) for (size_t q = 0; q < (size_t)N * dv; ++q) M[q] *= alpha[t];"),
