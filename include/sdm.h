@@ -250,6 +250,22 @@ sdm_status sdm_decode_step(const sdm_dims* dims, const void* q, const void* k, c
  * Errors: as sdm_forward; W + R <= 128; the slots must be in range and distinct within a
  * token.
  */
+/*
+ * Gradient through the scoring of one role with the selected slots held fixed (the top-k
+ * choice is piecewise constant and has no gradient): with w the selection weights that
+ * sdm_score_topk returned for x (softmax of the selected scores) and dw their gradient,
+ *   dscore_q = w_q (dw_q - sum_r w_r dw_r); dx and the sub-key tables' gradient follow
+ *   through the two half-score dot products (slot = i*n + j: C1[i], C2[j]).
+ *   x, subkeys, top, idx, w   as given to / returned by sdm_score_topk
+ *   dw    [B][H][T][top] fp32 (e.g. dww or drw of sdm_backward)
+ *   dx    [B][H][T][d_k] fp32, written
+ *   dsubkeys [H][2][n][d_k/2] fp32, ADDED TO (zero it first; calls accumulate)
+ * One launch; the table gradient uses atomic adds, so its summation order is not fixed.
+ */
+sdm_status sdm_score_backward(const sdm_dims* dims, const void* x, const void* subkeys,
+                              int32_t top, const int32_t* idx, const float* w, const float* dw,
+                              float* dx, float* dsubkeys, sdm_stream_t stream);
+
 size_t sdm_backward_workspace_bytes(const sdm_dims* dims);
 sdm_status sdm_backward(const sdm_dims* dims, const void* v, const float* alpha, const float* beta,
                         const int32_t* widx, const float* ww, const int32_t* ridx, const float* rw,

@@ -93,6 +93,7 @@ def _load():
         "sdm_device_error": ([ctypes.POINTER(ctypes.c_uint32), I32, P], I32),
         "sdm_forward_noalloc": ([D, P, P, P, P, P, P, P, S, P, P], I32),
         "sdm_backward_workspace_bytes": ([D], SZ),
+        "sdm_score_backward": ([D, P, P, I32, P, P, P, P, P, P], I32),
         "sdm_backward": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P, P, P, SZ, P], I32),
         "sdm_gemm_bf16": ([I32, I32, I32, P, P, P, P], I32),
         "sdm_layer_in_workspace_bytes": ([D], SZ),
@@ -311,6 +312,25 @@ def backward(d: Dims, v, alpha, beta, widx, ww, ridx, rw, st: State, dout, ws=No
                           _ptr(g["dM_in"], "dM_in", torch.float32), _ptr(ws, "ws"), ws.numel(),
                           _stream(stream)), "sdm_backward")
     return grads
+
+
+def score_backward(d: Dims, x, subkeys, top: int, idx, w, dw, dx=None, dsubkeys=None,
+                   stream=None):
+    """sdm_score_backward: (dx [B,H,T,d_k], dsubkeys [H,2,n,d_k/2]) fp32 for the selection
+    weights' gradient dw, the selections idx / w held fixed.  dsubkeys is added to (a new
+    zero tensor when not given)."""
+    dev = x.device
+    if dx is None:
+        dx = torch.empty((d.B, d.H, d.T, d.d_k), dtype=torch.float32, device=dev)
+    if dsubkeys is None:
+        dsubkeys = torch.zeros((d.H, 2, d.n_sub, d.d_k // 2), dtype=torch.float32, device=dev)
+    xdt = _xdt(d)
+    _ok(_lib.sdm_score_backward(ctypes.byref(d), _ptr(x, "x", xdt), _ptr(subkeys, "subkeys", xdt),
+                                top, _ptr(idx, "idx", torch.int32), _ptr(w, "w", torch.float32),
+                                _ptr(dw, "dw", torch.float32), _ptr(dx, "dx", torch.float32),
+                                _ptr(dsubkeys, "dsubkeys", torch.float32), _stream(stream)),
+        "sdm_score_backward")
+    return dx, dsubkeys
 
 
 def decode_step(d: Dims, q, k, v, alpha, beta, skw, skr, st: State, sel=None, out=None,

@@ -11,6 +11,7 @@
 #include "decode.cuh"
 #include "plan.cuh"
 #include "recur.cuh"
+#include "score_bwd.cuh"
 #include "score_rows.cuh"
 #include "score_simt.cuh"
 #include "score_tc.cuh"
@@ -382,6 +383,30 @@ sdm_status launch_backward_t(const sdm_dims* d, const BwdPtrs& P, const void* v,
     return launch_status();
 }
 
+template <typename XT, int HPL, int TPL>
+sdm_status launch_score_bwd_t(const sdm_dims* d, const void* x, const void* sk, int top,
+                              const int32_t* idx, const float* w, const float* dw, float* dx,
+                              float* dsk, cudaStream_t s) {
+    const long long rows = (long long)d->B * d->T;
+    const dim3 grid((unsigned)((rows + SBWD_ROWS - 1) / SBWD_ROWS), (unsigned)d->H);
+    score_backward_kernel<XT, HPL, TPL><<<grid, SBWD_THREADS, 0, s>>>(
+        (const XT*)x, (const XT*)sk, idx, w, dw, d->B, d->H, d->T, d->d_k, d->n_sub, top, dx, dsk);
+    return launch_status();
+}
+
+template <typename XT>
+sdm_status launch_score_bwd_x(const sdm_dims* d, const void* x, const void* sk, int top,
+                              const int32_t* idx, const float* w, const float* dw, float* dx,
+                              float* dsk, cudaStream_t s) {
+    const int hpl = (d->d_k / 2 + 31) / 32;  // d_k <= 256: at most 4
+    const bool t2 = top > 32;
+#define SDM_SB(H, TP) launch_score_bwd_t<XT, H, TP>(d, x, sk, top, idx, w, dw, dx, dsk, s)
+    if (hpl <= 1) return t2 ? SDM_SB(1, 2) : SDM_SB(1, 1);
+    if (hpl <= 2) return t2 ? SDM_SB(2, 2) : SDM_SB(2, 1);
+    return t2 ? SDM_SB(4, 2) : SDM_SB(4, 1);
+#undef SDM_SB
+}
+
 template <typename VT, int RPW, int QPL>
 sdm_status launch_decode(const sdm_dims* d, const void* v, const float* alpha, const float* beta,
                          const sdm_state* st, const int32_t* widx, const float* ww,
@@ -694,6 +719,20 @@ sdm_status sdm_decode_step(const sdm_dims* dims, const void* q, const void* k, c
                           : launch_decode<float, 8, 2>(dims, v, alpha, beta, st, widx, ww, ridx, rw, out, stream);
     }
     return e;
+}
+
+sdm_status sdm_score_backward(const sdm_dims* dims, const void* x, const void* subkeys,
+                              int32_t top, const int32_t* idx, const float* w, const float* dw,
+                              float* dx, float* dsubkeys, sdm_stream_t stream) {
+    const sdm_status e = check_dims(dims);
+    if (e) return e;
+    if (!x || !subkeys || !idx || !w || !dw || !dx || !dsubkeys) return SDM_ERR_ARG;
+    if (top < 1 || top > kMaxTop || top > dims->k_half * dims->k_half) return SDM_ERR_SHAPE;
+    if ((long long)dims->B * dims->T == 0) return SDM_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (dims->x_dtype == SDM_F32)
+        return launch_score_bwd_x<float>(dims, x, subkeys, top, idx, w, dw, dx, dsubkeys, s);
+    return launch_score_bwd_x<__nv_bfloat16>(dims, x, subkeys, top, idx, w, dw, dx, dsubkeys, s);
 }
 
 size_t sdm_backward_workspace_bytes(const sdm_dims* dims) {
