@@ -562,8 +562,19 @@ def run_backward(wl, inp, sel, device, sdm, reps: int = 2) -> dict:
         sdm.backward(d, *args, st, dout, ws=ws, grads=grads)
     e1.record(stream)
     torch.cuda.synchronize()
-    errs = sdm.device_error()
     ms = e0.elapsed_time(e1) / reps
+    # the gradient through both scorings (keys with dww, queries with drw)
+    sb = lambda: (sdm.score_backward(d, inp["k"], inp["skw"], wl.W, widx, ww, grads["dww"]),
+                  sdm.score_backward(d, inp["q"], inp["skr"], wl.R, ridx, rw, grads["drw"]))
+    sb()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        sb()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_score = e0.elapsed_time(e1) / reps
+    errs = sdm.device_error()
     units = units_per_step(wl)
     # per token.head: replay 3W rows (gather, log, store); sweep 3R (M, dM in, dM out) and 5W
     # (M_t, log, dM in, dM out, restore) rows of d_v fp32, plus the dense gradient once
@@ -573,6 +584,7 @@ def run_backward(wl, inp, sel, device, sdm, reps: int = 2) -> dict:
     peak = measured_peaks()["hbm_gbs"]
     res = {"workload": describe(wl) + ", backward of the recurrence (selections fixed)",
            "ms": ms, "token_heads_per_s": units / (ms / 1e3),
+           "scoring_backward_ms": ms_score,
            "roofline": {"bound": "hbm", "algorithmic_bytes": total, "achieved_gbs": gbs,
                         "peak": peak, "frac": gbs / peak},
            "note": "first version: one CTA per (b,h) walks the tokens one at a time",

@@ -87,7 +87,9 @@ SDM_DEV float bwd_factor(double st, double L, int touched) {
 }
 
 // ---- replay with the log --------------------------------------------------------------
-// QPL: float4 columns per lane (d_v <= 128: 1, else 2); WPW: write rows per warp.
+// QPL: float4 columns per lane (d_v <= 128: 1, else 2); WPW: write rows per warp.  Each
+// token's loads go out in dependent rounds (its indices were fetched during the previous
+// token; then the stamps; then every row), and all stores follow the loads.
 template <typename VT, int QPL, int WPW>
 __global__ void __launch_bounds__(BWD_THREADS) bwd_replay_kernel(
     const VT* __restrict__ v, const float* __restrict__ alpha, const float* __restrict__ beta,
@@ -105,55 +107,75 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_replay_kernel(
     double* stb = stamp + bh * (size_t)N;
     double L = lambda[bh];
     if (tid == 0) P.log_lam[bh * (size_t)(T + 1)] = L;
+    // indices and weights of the next token
+    int nsl[WPW];
+    float nwi[WPW], na = 1.f, nb = 0.f;
+    auto fetch = [&](int t) {
+        const size_t bt = bh * (size_t)T + t;
+        na = alpha[bt];
+        nb = beta[bt];
+#pragma unroll
+        for (int k = 0; k < WPW; ++k) {
+            const int i = warp + BWD_WARPS * k;
+            nsl[k] = i < W ? widx[bt * W + i] : -1;
+            nwi[k] = i < W ? ww[bt * W + i] : 0.f;
+        }
+    };
+    if (T > 0) fetch(0);
     for (int t = 0; t < T; ++t) {
         const size_t bt = bh * (size_t)T + t;
-        const float a = alpha[bt], bta = beta[bt];
-        if (a > 0.f) L += log((double)a);
-        else if (tid == 0) raise_err(SDM_DEVERR_ALPHA);
-        float4 seen[WPW][QPL], vv[QPL];
+        const float a = na, bta = nb;
         int sl[WPW];
         float wi[WPW];
+#pragma unroll
+        for (int k = 0; k < WPW; ++k) {
+            sl[k] = nsl[k];
+            wi[k] = nwi[k];
+            if (sl[k] >= 0 && !slot_ok(sl[k], N)) {
+                if (lane == 0) raise_err(SDM_DEVERR_SLOT_RANGE);
+                sl[k] = -1;
+            }
+        }
+        if (a > 0.f) L += log((double)a);
+        else if (tid == 0) raise_err(SDM_DEVERR_ALPHA);
+        float4 vv[QPL];
 #pragma unroll
         for (int c = 0; c < QPL; ++c) {
             const int q = lane + 32 * c;
             vv[c] = q < Q ? bwd_load_v4<VT>(v + bt * d_v + 4 * q) : f4(0.f);
         }
+        double st[WPW];
+#pragma unroll
+        for (int k = 0; k < WPW; ++k) st[k] = sl[k] >= 0 ? stb[sl[k]] : 0.0;
+        float4 raw[WPW][QPL], mraw[WPW][QPL];
+        float fk[WPW];
+#pragma unroll
+        for (int k = 0; k < WPW; ++k) {
+            const int s = sl[k];
+            fk[k] = bwd_factor(st[k], L, touched) * (touched ? a : 1.f);
+#pragma unroll
+            for (int c = 0; c < QPL; ++c) {
+                const int q = lane + 32 * c;
+                raw[k][c] = mraw[k][c] = f4(0.f);
+                if (s >= 0 && q < Q) {
+                    mraw[k][c] = reinterpret_cast<const float4*>(Mb + (size_t)s * d_v)[q];
+                    raw[k][c] = signbit(fk[k])
+                                    ? reinterpret_cast<const float4*>(M0h + (size_t)s * d_v)[q]
+                                    : mraw[k][c];
+                }
+            }
+        }
+        if (t + 1 < T) fetch(t + 1);
         float4 pp[QPL];
 #pragma unroll
         for (int c = 0; c < QPL; ++c) pp[c] = f4(0.f);
 #pragma unroll
-        for (int k = 0; k < WPW; ++k) {
-            const int i = warp + BWD_WARPS * k;
-            sl[k] = -1;
-            wi[k] = 0.f;
-            if (i < W) {
-                int s = widx[bt * W + i];
-                if (!slot_ok(s, N)) {
-                    raise_err(SDM_DEVERR_SLOT_RANGE);
-                    s = -1;
-                }
-                sl[k] = s;
-                wi[k] = ww[bt * W + i];
-            }
-            const int s = sl[k];
-            const double st = s >= 0 ? stb[s] : 0.0;
-            const float f = bwd_factor(st, L, touched) * (touched ? a : 1.f);
-            const float* src = signbit(f) ? M0h : Mb;
-            const size_t lr = (bt * W + (i < W ? i : 0)) * (size_t)d_v;
+        for (int k = 0; k < WPW; ++k)
 #pragma unroll
             for (int c = 0; c < QPL; ++c) {
-                const int q = lane + 32 * c;
-                float4 raw = f4(0.f), mraw = f4(0.f);
-                if (s >= 0 && q < Q) {
-                    raw = reinterpret_cast<const float4*>(src + (size_t)s * d_v)[q];
-                    mraw = reinterpret_cast<const float4*>(Mb + (size_t)s * d_v)[q];
-                    reinterpret_cast<float4*>(P.log_rows + lr)[q] = mraw;
-                }
-                seen[k][c] = f4_scale(fabsf(f), raw);
-                pp[c] = f4_fma(wi[k], seen[k][c], pp[c]);
+                raw[k][c] = f4_scale(fabsf(fk[k]), raw[k][c]);  // the decayed row, "seen"
+                pp[c] = f4_fma(wi[k], raw[k][c], pp[c]);
             }
-            if (s >= 0 && lane == 0) P.log_stamp[bt * W + i] = st;
-        }
 #pragma unroll
         for (int c = 0; c < QPL; ++c) {
             const int q = lane + 32 * c;
@@ -173,19 +195,25 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_replay_kernel(
             dd[c] = make_float4(bta * (vv[c].x - p.x), bta * (vv[c].y - p.y), bta * (vv[c].z - p.z),
                                 bta * (vv[c].w - p.w));
         }
-        __syncthreads();  // s_pp is rewritten by the next token
 #pragma unroll
         for (int k = 0; k < WPW; ++k) {
             const int s = sl[k];
             if (s < 0) continue;
+            const int i = warp + BWD_WARPS * k;
+            const size_t lr = (bt * W + i) * (size_t)d_v;
 #pragma unroll
             for (int c = 0; c < QPL; ++c) {
                 const int q = lane + 32 * c;
-                if (q < Q)
+                if (q < Q) {
+                    reinterpret_cast<float4*>(P.log_rows + lr)[q] = mraw[k][c];
                     reinterpret_cast<float4*>(Mb + (size_t)s * d_v)[q] =
-                        f4_fma(wi[k], dd[c], seen[k][c]);
+                        f4_fma(wi[k], dd[c], raw[k][c]);
+                }
             }
-            if (lane == 0) stb[s] = L;
+            if (lane == 0) {
+                P.log_stamp[bt * W + i] = st[k];
+                stb[s] = L;
+            }
         }
         if (tid == 0) P.log_lam[bh * (size_t)(T + 1) + t + 1] = L;
         __syncthreads();  // this token's rows and stamps before the next token's gathers
@@ -194,6 +222,11 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_replay_kernel(
 }
 
 // ---- the backward sweep ---------------------------------------------------------------
+// Per token: its indices, weights, dout and v rows were fetched during the previous token;
+// the read rows' stamps, then their rows (M side and gradient side) go out together; the
+// write rows' M side (log stamps, current stamps, then log and current rows) is issued
+// before the read rows are processed, their gradient side after the barrier that publishes
+// the read rows' gradient updates.
 template <typename VT, int QPL, int WPW>
 __global__ void __launch_bounds__(BWD_THREADS) bwd_sweep_kernel(
     const VT* __restrict__ v, const float* __restrict__ alpha, const float* __restrict__ beta,
@@ -219,50 +252,128 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_sweep_kernel(
     const double* lamb = P.log_lam + bh * (size_t)(T + 1);
     double X = 0.0, Gam = 0.0;  // <dM, M> over every slot; backward log-decay prefix
     constexpr int RPW = WPW;
-    for (int t = T - 1; t >= 0; --t) {
+    // the next token's inputs
+    int nrs[RPW], nws[WPW];
+    float nu[RPW], nwi[WPW], na = 1.f, nb = 0.f;
+    float4 nG[QPL], nv[QPL];
+    auto fetch = [&](int t) {
         const size_t bt = bh * (size_t)T + t;
-        const float a = alpha[bt] > 0.f ? alpha[bt] : 1.f, bta = beta[bt];
-        const double Lt = lamb[t + 1], Lp = lamb[t];
-        float4 G[QPL], vv[QPL];
+        na = alpha[bt] > 0.f ? alpha[bt] : 1.f;
+        nb = beta[bt];
+#pragma unroll
+        for (int k = 0; k < RPW; ++k) {
+            const int j = warp + BWD_WARPS * k;
+            nrs[k] = j < R ? ridx[bt * R + j] : -1;
+            nu[k] = j < R ? rw[bt * R + j] : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < WPW; ++k) {
+            const int i = warp + BWD_WARPS * k;
+            nws[k] = i < W ? widx[bt * W + i] : -1;
+            nwi[k] = i < W ? ww[bt * W + i] : 0.f;
+        }
 #pragma unroll
         for (int c = 0; c < QPL; ++c) {
             const int q = lane + 32 * c;
-            G[c] = q < Q ? reinterpret_cast<const float4*>(dout + bt * d_v)[q] : f4(0.f);
-            vv[c] = q < Q ? bwd_load_v4<VT>(v + bt * d_v + 4 * q) : f4(0.f);
+            nG[c] = q < Q ? reinterpret_cast<const float4*>(dout + bt * d_v)[q] : f4(0.f);
+            nv[c] = q < Q ? bwd_load_v4<VT>(v + bt * d_v + 4 * q) : f4(0.f);
         }
+    };
+    if (T > 0) fetch(T - 1);
+    for (int t = T - 1; t >= 0; --t) {
+        const size_t bt = bh * (size_t)T + t;
+        const float a = na, bta = nb;
+        const double Lt = lamb[t + 1], Lp = lamb[t];
+        int rs[RPW], sl[WPW];
+        float u[RPW], wi[WPW];
+        float4 G[QPL], vv[QPL];
+#pragma unroll
+        for (int k = 0; k < RPW; ++k) {
+            rs[k] = slot_ok(nrs[k], N) ? nrs[k] : -1;  // the forward reported bad slots
+            u[k] = nu[k];
+        }
+#pragma unroll
+        for (int k = 0; k < WPW; ++k) {
+            sl[k] = slot_ok(nws[k], N) ? nws[k] : -1;
+            wi[k] = nwi[k];
+        }
+#pragma unroll
+        for (int c = 0; c < QPL; ++c) {
+            G[c] = nG[c];
+            vv[c] = nv[c];
+        }
+        // -- round 1: stamps of the read rows and of the write rows (M side)
+        double rst[RPW], rds[RPW], wso[WPW], wsn[WPW];
+#pragma unroll
+        for (int k = 0; k < RPW; ++k) {
+            rst[k] = rs[k] >= 0 ? stb[rs[k]] : 0.0;
+            rds[k] = rs[k] >= 0 ? dsb[rs[k]] : 0.0;
+        }
+#pragma unroll
+        for (int k = 0; k < WPW; ++k) {
+            const int i = warp + BWD_WARPS * k;
+            wso[k] = sl[k] >= 0 ? P.log_stamp[bt * W + i] : 0.0;
+            wsn[k] = sl[k] >= 0 ? stb[sl[k]] : 0.0;
+        }
+        // -- round 2: the read rows (M and dM) and the write rows' M side (log and current)
+        float4 rm[RPW][QPL], rg[RPW][QPL], mp[WPW][QPL], mt[WPW][QPL];
+        float fo[WPW], fn[WPW];
+#pragma unroll
+        for (int k = 0; k < RPW; ++k) {
+            const int s = rs[k];
+            const float f = bwd_factor(rst[k], Lt, touched);
+            const float gf = (s < 0 || isnan(rds[k])) ? 0.f : (float)exp(Gam - rds[k]);
+#pragma unroll
+            for (int c = 0; c < QPL; ++c) {
+                const int q = lane + 32 * c;
+                rm[k][c] = rg[k][c] = f4(0.f);
+                if (s >= 0 && q < Q) {
+                    const float* src = (signbit(f) ? M0h : Mb) + (size_t)s * d_v;
+                    rm[k][c] = f4_scale(fabsf(f), reinterpret_cast<const float4*>(src)[q]);
+                    if (gf != 0.f)
+                        rg[k][c] = f4_scale(gf, reinterpret_cast<const float4*>(dMb + (size_t)s * d_v)[q]);
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < WPW; ++k) {
+            const int s = sl[k], i = warp + BWD_WARPS * k;
+            fo[k] = bwd_factor(wso[k], Lp, touched);  // value factor at t-1
+            fn[k] = bwd_factor(wsn[k], Lt, touched);  // at t
+            const size_t lr = (bt * W + (i < W ? i : 0)) * (size_t)d_v;
+#pragma unroll
+            for (int c = 0; c < QPL; ++c) {
+                const int q = lane + 32 * c;
+                mp[k][c] = mt[k][c] = f4(0.f);
+                if (s >= 0 && q < Q) {
+                    const float* so_src = signbit(fo[k]) ? M0h + (size_t)s * d_v : P.log_rows + lr;
+                    mp[k][c] = f4_scale(fabsf(fo[k]), reinterpret_cast<const float4*>(so_src)[q]);
+                    const float* sn_src = (signbit(fn[k]) ? M0h : Mb) + (size_t)s * d_v;
+                    mt[k][c] = f4_scale(fabsf(fn[k]), reinterpret_cast<const float4*>(sn_src)[q]);
+                }
+            }
+        }
+        if (t > 0) fetch(t - 1);
         // -- read rows: du_j, dM[r_j] += u_j G, X += u_j du_j
         double xr = 0.0;
 #pragma unroll
         for (int k = 0; k < RPW; ++k) {
             const int j = warp + BWD_WARPS * k;
-            if (j >= R) continue;
-            int s = ridx[bt * R + j];
-            if (!slot_ok(s, N)) continue;  // the forward reported it
-            const float u = rw[bt * R + j];
-            const float f = bwd_factor(stb[s], Lt, touched);
-            const float* src = signbit(f) ? M0h : Mb;
-            const double ds = dsb[s];
-            const float gf = isnan(ds) ? 0.f : (float)exp(Gam - ds);
+            const int s = rs[k];
+            if (s < 0) continue;  // warp-uniform
             float acc = 0.f;
-            float4 ng[QPL];
 #pragma unroll
             for (int c = 0; c < QPL; ++c) {
-                const int q = lane + 32 * c;
-                float4 m = f4(0.f), g = f4(0.f);
-                if (q < Q) {
-                    m = f4_scale(fabsf(f), reinterpret_cast<const float4*>(src + (size_t)s * d_v)[q]);
-                    if (!isnan(ds)) g = f4_scale(gf, reinterpret_cast<const float4*>(dMb + (size_t)s * d_v)[q]);
-                }
-                acc += f4_dot(G[c], m);
-                ng[c] = f4_fma(u, G[c], g);
+                acc += f4_dot(G[c], rm[k][c]);
+                rg[k][c] = f4_fma(u[k], G[c], rg[k][c]);
             }
             const float du = warp_sum(acc);
             if (lane == 0) drw[bt * R + j] = du;
-            xr += (double)u * du;
+            xr += (double)u[k] * du;
 #pragma unroll
             for (int c = 0; c < QPL; ++c) {
                 const int q = lane + 32 * c;
-                if (q < Q) reinterpret_cast<float4*>(dMb + (size_t)s * d_v)[q] = ng[c];
+                if (q < Q) reinterpret_cast<float4*>(dMb + (size_t)s * d_v)[q] = rg[k][c];
             }
             __syncwarp();
             if (lane == 0) dsb[s] = Gam;
@@ -271,38 +382,24 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_sweep_kernel(
         __syncthreads();  // read rows of dM (and their stamps) before the write rows use them
         if (!touched)
             for (int w2 = 0; w2 < BWD_WARPS; ++w2) X += s_part[w2 * 4 + 0];
-        // -- write rows: M_t (current), M_{t-1} (log), dM_t
-        float4 mp[WPW][QPL], mt[WPW][QPL], dm[WPW][QPL];
-        int sl[WPW];
-        float wi[WPW];
+        // -- round 3: the write rows' gradient side
+        double wds[WPW];
+#pragma unroll
+        for (int k = 0; k < WPW; ++k) wds[k] = sl[k] >= 0 ? dsb[sl[k]] : 0.0;
+        float4 dm[WPW][QPL];
         float4 pp[QPL], pd[QPL];
 #pragma unroll
         for (int c = 0; c < QPL; ++c) pp[c] = pd[c] = f4(0.f);
 #pragma unroll
         for (int k = 0; k < WPW; ++k) {
-            const int i = warp + BWD_WARPS * k;
-            int s = i < W ? widx[bt * W + i] : -1;
-            if (s >= 0 && !slot_ok(s, N)) s = -1;
-            sl[k] = s;
-            wi[k] = (i < W) ? ww[bt * W + i] : 0.f;
-            const double so = s >= 0 ? P.log_stamp[bt * W + i] : 0.0;
-            const float fo = bwd_factor(so, Lp, touched);      // value factor at t-1
-            const float fn = bwd_factor(s >= 0 ? stb[s] : 0.0, Lt, touched);  // at t
-            const double ds = s >= 0 ? dsb[s] : 0.0;
-            const float gf = (s < 0 || isnan(ds)) ? 0.f : (float)exp(Gam - ds);
-            const size_t lr = (bt * W + (i < W ? i : 0)) * (size_t)d_v;
+            const int s = sl[k];
+            const float gf = (s < 0 || isnan(wds[k])) ? 0.f : (float)exp(Gam - wds[k]);
 #pragma unroll
             for (int c = 0; c < QPL; ++c) {
                 const int q = lane + 32 * c;
-                mp[k][c] = mt[k][c] = dm[k][c] = f4(0.f);
-                if (s >= 0 && q < Q) {
-                    const float* so_src = signbit(fo) ? M0h + (size_t)s * d_v : P.log_rows + lr;
-                    mp[k][c] = f4_scale(fabsf(fo), reinterpret_cast<const float4*>(so_src)[q]);
-                    const float* sn_src = (signbit(fn) ? M0h : Mb) + (size_t)s * d_v;
-                    mt[k][c] = f4_scale(fabsf(fn), reinterpret_cast<const float4*>(sn_src)[q]);
-                    if (gf != 0.f)
-                        dm[k][c] = f4_scale(gf, reinterpret_cast<const float4*>(dMb + (size_t)s * d_v)[q]);
-                }
+                dm[k][c] = f4(0.f);
+                if (gf != 0.f && q < Q)
+                    dm[k][c] = f4_scale(gf, reinterpret_cast<const float4*>(dMb + (size_t)s * d_v)[q]);
                 pp[c] = f4_fma(wi[k] * a, mp[k][c], pp[c]);
                 pd[c] = f4_fma(wi[k], dm[k][c], pd[c]);
             }
@@ -358,12 +455,12 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_sweep_kernel(
             s2 += gmp;
             // dM_{t-1}[s] = alpha dMt[s]: every-slot decay keeps alpha in the prefix Gam
             const float sc = touched ? a : 1.f;
+            const size_t lr = (bt * W + i) * (size_t)d_v;
 #pragma unroll
             for (int c = 0; c < QPL; ++c) {
                 const int q = lane + 32 * c;
                 if (q < Q) {
                     reinterpret_cast<float4*>(dMb + (size_t)s * d_v)[q] = f4_scale(sc, nd[c]);
-                    const size_t lr = (bt * W + i) * (size_t)d_v;
                     reinterpret_cast<float4*>(Mb + (size_t)s * d_v)[q] =
                         reinterpret_cast<const float4*>(P.log_rows + lr)[q];  // restore
                 }
@@ -371,7 +468,7 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_sweep_kernel(
             __syncwarp();
             if (lane == 0) {
                 dsb[s] = Gam;
-                stb[s] = P.log_stamp[bt * W + i];
+                stb[s] = wso[k];
             }
         }
         if (lane == 0) {
