@@ -79,11 +79,15 @@ SDM_DEV float4 bwd_load_v4<__nv_bfloat16>(const __nv_bfloat16* p) {
                        __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
 }
 
+// e^d for a log-decay difference d taken in fp64: the exponential in fp32 (the factor is
+// stored and used in fp32; rounding d to fp32 first moves it by |d| * 6e-8 relative).
+SDM_DEV float bwd_exp(double d) { return expf((float)d); }
+
 // Value factor of a slot at prefix L from its stamp (every-slot decay; the sign marks a
 // pristine slot, whose row is M0); touched-slots decay: 1.
 SDM_DEV float bwd_factor(double st, double L, int touched) {
     if (touched) return isnan(st) ? -1.f : 1.f;
-    return isnan(st) ? -(float)exp(L) : (float)exp(L - st);
+    return isnan(st) ? -bwd_exp(L) : bwd_exp(L - st);
 }
 
 // ---- replay with the log --------------------------------------------------------------
@@ -322,7 +326,7 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_sweep_kernel(
         for (int k = 0; k < RPW; ++k) {
             const int s = rs[k];
             const float f = bwd_factor(rst[k], Lt, touched);
-            const float gf = (s < 0 || isnan(rds[k])) ? 0.f : (float)exp(Gam - rds[k]);
+            const float gf = (s < 0 || isnan(rds[k])) ? 0.f : bwd_exp(Gam - rds[k]);
 #pragma unroll
             for (int c = 0; c < QPL; ++c) {
                 const int q = lane + 32 * c;
@@ -393,7 +397,7 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_sweep_kernel(
 #pragma unroll
         for (int k = 0; k < WPW; ++k) {
             const int s = sl[k];
-            const float gf = (s < 0 || isnan(wds[k])) ? 0.f : (float)exp(Gam - wds[k]);
+            const float gf = (s < 0 || isnan(wds[k])) ? 0.f : bwd_exp(Gam - wds[k]);
 #pragma unroll
             for (int c = 0; c < QPL; ++c) {
                 const int q = lane + 32 * c;
@@ -517,7 +521,7 @@ __global__ void bwd_dense_kernel(const BwdPtrs P, int T, int N, int d_v, size_t 
         const double ds = P.dstamp[row];
         float4 val = f4(0.f);
         if (!isnan(ds)) {
-            const float g = (float)exp(P.log_lam[bh * (size_t)(T + 1) + T] - ds);
+            const float g = bwd_exp(P.log_lam[bh * (size_t)(T + 1) + T] - ds);
             val = f4_scale(g, reinterpret_cast<const float4*>(P.dM + row * d_v)[q]);
         }
         reinterpret_cast<float4*>(out + row * d_v)[q] = val;
