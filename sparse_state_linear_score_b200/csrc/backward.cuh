@@ -2,10 +2,18 @@
 // "Memory-Efficient Backward": the sparse updates are applied in place and undone while
 // the gradients flow back, so no copy of the memory is kept per chunk).
 //
+// Parallel over value columns.  Once the slots and gates are fixed, the chain through the
+// tokens is per column: every row operation acts column by column, and only outputs (dalpha,
+// dbeta, dw, du) sum over columns.  Each (b,h) is therefore split into slices of 8 columns
+// (two float4), one warp per slice, and every slice walks the tokens one at a time on its
+// own.  Stamps belong to slots, not columns, and the slices run at their own pace, so each
+// slice keeps private copies of the slot stamps and of the gradient stamps (all copies hold
+// the same values at the same point of the walk).  Column sums are written per slice and
+// added in a fixed order by bwd_reduce_kernel.
+//
 // bwd_replay_kernel: from the state at the start of the call, the tokens are replayed in
-// place, one CTA per (b,h), and before every write the raw rows and stamps of the token's
-// W write slots go to a log (T*W rows + T*W stamps per (b,h): the O(T*W*d) record), with
-// Lambda after every token.
+// place, and before every write the raw rows and stamps of the token's W write slots go to a
+// log (T*W rows + T*W stamps per (b,h): the O(T*W*d) record), with Lambda after every token.
 //
 // bwd_sweep_kernel: the tokens backwards.  With G = dout[t], per token (decayed rows
 // Mt = alpha M_{t-1} on the write slots, as in the forward):
@@ -18,13 +26,17 @@
 //           dalpha = (X - sum_i <dM[s_i], M_t[s_i]>) / alpha + sum_i <dMt[s_i], M_{t-1}[s_i]>,
 //           then X <- alpha dalpha; dM_{t-1} = alpha dMt, kept lazily as raw rows, a
 //           backward log-decay prefix Gam (+= log alpha per token) and per-row stamps.
+//           X is linear in its terms, so each lane carries its own share of it.
 //           Touched-slots decay: dalpha = sum_i <dMt[s_i], M_{t-1}[s_i]> and only the write
 //           rows take the factor alpha.
-//   then the write slots' raw rows and stamps are restored from the log, and Lambda.
-// On return the state is again the state at the start of the call.
+//   then the write slots' raw rows and stamps are restored from the log.
+// On return the state is again the state at the start of the call (its stamps and Lambda
+// are never written: the slices work on their private stamp copies).
 //
-// Layout: warp w owns write rows w, w+8, ... and read rows w, w+8, ...; lane l owns the
-// float4 columns l (+32) of d_v; sums across warps go through [8][d_v] shared partials.
+// Lane layout in a slice: lane = 2 g + h2, h2 the float4 of the slice, g the row group;
+// lane owns write rows g, g+16, ... and read rows g, g+16, ...  A token's loads (stamps,
+// rows, log) all go out in one round; a slot both read and written in the token takes the
+// read's gradient update through a shared-memory list of the token's read slots.
 #pragma once
 
 #include <math.h>
@@ -33,22 +45,23 @@
 
 namespace sdm {
 
-constexpr int BWD_THREADS = 256;
-constexpr int BWD_WARPS = BWD_THREADS / 32;
-constexpr int BWD_MAXO = 128;  // W + R
+constexpr int BWD_MAXO = 128;      // W + R
+constexpr int BWD_SLICE_Q = 2;     // float4 columns per slice
 
-// Per-(b,h) records of one call (a byte layout in the workspace).
+// Per-(b,h) records of one call (a byte layout in the workspace); S = slices per (b,h).
 struct BwdPtrs {
     float* log_rows;     // [BH][T][W][d_v] raw rows of the write slots before the write
     double* log_stamp;   // [BH][T][W]      their stamps before the write
     double* log_lam;     // [BH][T+1]       Lambda at the start, then after every token
     float* dM;           // [BH][N][d_v]    raw memory gradient rows
-    double* dstamp;      // [BH][N]         their stamps (NaN: the row is zero)
+    double* pst;         // [S][BH][N]      private slot stamps
+    double* pds;         // [S][BH][N]      private gradient stamps (NaN: the row is zero)
+    float* p_dww;        // [S][BH*T][W]    per-slice shares of dww
+    float* p_drw;        // [S][BH*T][R]    of drw
+    double* p_db;        // [S][BH*T]       of dbeta
+    double* p_da;        // [S][BH*T]       of dalpha
+    double* gam;         // [BH]            the final backward prefix
 };
-
-__host__ __device__ inline size_t bwd_smem_bytes(int d_v) {
-    return (size_t)3 * BWD_WARPS * d_v * 4 + (size_t)BWD_MAXO * 16 + 64 * 8;
-}
 
 SDM_DEV float4 f4(float a) { return make_float4(a, a, a, a); }
 SDM_DEV float4 f4_fma(float s, const float4& x, const float4& y) {
@@ -57,14 +70,30 @@ SDM_DEV float4 f4_fma(float s, const float4& x, const float4& y) {
 SDM_DEV float f4_dot(const float4& a, const float4& b) {
     return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
 }
-SDM_DEV float warp_sum(float x) {
+SDM_DEV float4 f4_scale(float s, const float4& a) {
+    return make_float4(s * a.x, s * a.y, s * a.z, s * a.w);
+}
+SDM_DEV float4 f4_add(const float4& a, const float4& b) {
+    return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+// sum over the 16 row groups (lanes of equal h2)
+SDM_DEV float4 f4_sum_groups(float4 x) {
+#pragma unroll
+    for (int m = 2; m < 32; m <<= 1) {
+        x.x += __shfl_xor_sync(0xffffffffu, x.x, m);
+        x.y += __shfl_xor_sync(0xffffffffu, x.y, m);
+        x.z += __shfl_xor_sync(0xffffffffu, x.z, m);
+        x.w += __shfl_xor_sync(0xffffffffu, x.w, m);
+    }
+    return x;
+}
+SDM_DEV double warp_sum_d(double x) {
 #pragma unroll
     for (int m = 16; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
     return x;
 }
-SDM_DEV float4 f4_scale(float s, const float4& a) {
-    return make_float4(s * a.x, s * a.y, s * a.z, s * a.w);
-}
+// a row's dot product: the two lanes of one row group
+SDM_DEV float pair_sum(float x) { return x + __shfl_xor_sync(0xffffffffu, x, 1); }
 
 template <typename VT>
 SDM_DEV float4 bwd_load_v4(const VT* p);
@@ -90,37 +119,48 @@ SDM_DEV float bwd_factor(double st, double L, int touched) {
     return isnan(st) ? -bwd_exp(L) : bwd_exp(L - st);
 }
 
+// Private stamp copies for every slice, gradient stamps NaN, final prefixes 0.
+__global__ void bwd_init_kernel(const double* __restrict__ stamp, BwdPtrs P, size_t bhn,
+                                int S, int BH) {
+    const size_t total = (size_t)S * bhn;
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    const size_t i0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (size_t i = i0; i < total; i += stride) {
+        P.pst[i] = stamp[i % bhn];
+        P.pds[i] = __longlong_as_double(0x7ff8000000000000ll);
+    }
+    for (size_t i = i0; i < (size_t)BH; i += stride) P.gam[i] = 0.0;
+}
+
 // ---- replay with the log --------------------------------------------------------------
-// QPL: float4 columns per lane (d_v <= 128: 1, else 2); WPW: write rows per warp.  Each
-// token's loads go out in dependent rounds (its indices were fetched during the previous
-// token; then the stamps; then every row), and all stores follow the loads.
-template <typename VT, int QPL, int WPW>
-__global__ void __launch_bounds__(BWD_THREADS) bwd_replay_kernel(
+// One warp per (slice, b, h); KPL: write rows per lane (ceil(W / 16)).
+template <typename VT, int KPL>
+__global__ void __launch_bounds__(32) bwd_replay_kernel(
     const VT* __restrict__ v, const float* __restrict__ alpha, const float* __restrict__ beta,
     const int32_t* __restrict__ widx, const float* __restrict__ ww, float* __restrict__ M,
-    double* __restrict__ stamp, double* __restrict__ lambda, const float* __restrict__ M0,
-    BwdPtrs P, int H, int N, int T, int d_v, int W, int touched) {
-    extern __shared__ __align__(16) unsigned char bwd_smem[];
-    const size_t bh = blockIdx.x;
+    const double* __restrict__ lambda, const float* __restrict__ M0, BwdPtrs P, int H, int N,
+    int T, int d_v, int W, int S, int touched) {
+    const int sc = (int)(blockIdx.x % S);
+    const size_t bh = blockIdx.x / S, BH = gridDim.x / S;
     const int h = (int)(bh % H);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int Q = d_v / 4;
-    float* s_pp = reinterpret_cast<float*>(bwd_smem);  // [8][d_v]
+    const int lane = threadIdx.x, h2 = lane & 1, g = lane >> 1;
+    const int Q = d_v / 4, q = BWD_SLICE_Q * sc + h2;
+    const bool qok = q < Q;
+    const bool lead = sc == 0;  // slice 0 writes the column-free records
     float* Mb = M + bh * (size_t)N * d_v;
     const float* M0h = M0 + (size_t)h * N * d_v;
-    double* stb = stamp + bh * (size_t)N;
+    double* stb = P.pst + ((size_t)sc * BH + bh) * N;
     double L = lambda[bh];
-    if (tid == 0) P.log_lam[bh * (size_t)(T + 1)] = L;
-    // indices and weights of the next token
-    int nsl[WPW];
-    float nwi[WPW], na = 1.f, nb = 0.f;
+    if (lead && lane == 0) P.log_lam[bh * (size_t)(T + 1)] = L;
+    int nsl[KPL];
+    float nwi[KPL], na = 1.f, nb = 0.f;
     auto fetch = [&](int t) {
         const size_t bt = bh * (size_t)T + t;
         na = alpha[bt];
         nb = beta[bt];
 #pragma unroll
-        for (int k = 0; k < WPW; ++k) {
-            const int i = warp + BWD_WARPS * k;
+        for (int k = 0; k < KPL; ++k) {
+            const int i = g + 16 * k;
             nsl[k] = i < W ? widx[bt * W + i] : -1;
             nwi[k] = i < W ? ww[bt * W + i] : 0.f;
         }
@@ -129,158 +169,105 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_replay_kernel(
     for (int t = 0; t < T; ++t) {
         const size_t bt = bh * (size_t)T + t;
         const float a = na, bta = nb;
-        int sl[WPW];
-        float wi[WPW];
+        int sl[KPL];
+        float wi[KPL];
 #pragma unroll
-        for (int k = 0; k < WPW; ++k) {
+        for (int k = 0; k < KPL; ++k) {
             sl[k] = nsl[k];
             wi[k] = nwi[k];
             if (sl[k] >= 0 && !slot_ok(sl[k], N)) {
-                if (lane == 0) raise_err(SDM_DEVERR_SLOT_RANGE);
+                raise_err(SDM_DEVERR_SLOT_RANGE);
                 sl[k] = -1;
             }
         }
         if (a > 0.f) L += log((double)a);
-        else if (tid == 0) raise_err(SDM_DEVERR_ALPHA);
-        float4 vv[QPL];
+        else if (lane == 0) raise_err(SDM_DEVERR_ALPHA);
+        const float4 vv = qok ? bwd_load_v4<VT>(v + bt * d_v + 4 * q) : f4(0.f);
+        double st[KPL];
+        float4 mraw[KPL], m0[KPL];
 #pragma unroll
-        for (int c = 0; c < QPL; ++c) {
-            const int q = lane + 32 * c;
-            vv[c] = q < Q ? bwd_load_v4<VT>(v + bt * d_v + 4 * q) : f4(0.f);
-        }
-        double st[WPW];
-#pragma unroll
-        for (int k = 0; k < WPW; ++k) st[k] = sl[k] >= 0 ? stb[sl[k]] : 0.0;
-        float4 raw[WPW][QPL], mraw[WPW][QPL];
-        float fk[WPW];
-#pragma unroll
-        for (int k = 0; k < WPW; ++k) {
+        for (int k = 0; k < KPL; ++k) {
             const int s = sl[k];
-            fk[k] = bwd_factor(st[k], L, touched) * (touched ? a : 1.f);
-#pragma unroll
-            for (int c = 0; c < QPL; ++c) {
-                const int q = lane + 32 * c;
-                raw[k][c] = mraw[k][c] = f4(0.f);
-                if (s >= 0 && q < Q) {
-                    mraw[k][c] = reinterpret_cast<const float4*>(Mb + (size_t)s * d_v)[q];
-                    raw[k][c] = signbit(fk[k])
-                                    ? reinterpret_cast<const float4*>(M0h + (size_t)s * d_v)[q]
-                                    : mraw[k][c];
-                }
+            st[k] = s >= 0 ? stb[s] : 0.0;
+            mraw[k] = m0[k] = f4(0.f);
+            if (s >= 0 && qok) {
+                mraw[k] = reinterpret_cast<const float4*>(Mb + (size_t)s * d_v)[q];
+                m0[k] = reinterpret_cast<const float4*>(M0h + (size_t)s * d_v)[q];
             }
         }
         if (t + 1 < T) fetch(t + 1);
-        float4 pp[QPL];
+        float4 raw[KPL], pp = f4(0.f);
 #pragma unroll
-        for (int c = 0; c < QPL; ++c) pp[c] = f4(0.f);
-#pragma unroll
-        for (int k = 0; k < WPW; ++k)
-#pragma unroll
-            for (int c = 0; c < QPL; ++c) {
-                raw[k][c] = f4_scale(fabsf(fk[k]), raw[k][c]);  // the decayed row, "seen"
-                pp[c] = f4_fma(wi[k], raw[k][c], pp[c]);
-            }
-#pragma unroll
-        for (int c = 0; c < QPL; ++c) {
-            const int q = lane + 32 * c;
-            if (q < Q) reinterpret_cast<float4*>(s_pp + warp * d_v)[q] = pp[c];
+        for (int k = 0; k < KPL; ++k) {
+            const float fk = bwd_factor(st[k], L, touched) * (touched ? a : 1.f);
+            raw[k] = f4_scale(fabsf(fk), signbit(fk) ? m0[k] : mraw[k]);  // the decayed row
+            pp = f4_fma(wi[k], raw[k], pp);
         }
-        __syncthreads();
-        float4 dd[QPL];
+        const float4 p = f4_sum_groups(pp);
+        const float4 dd = make_float4(bta * (vv.x - p.x), bta * (vv.y - p.y), bta * (vv.z - p.z),
+                                      bta * (vv.w - p.w));
 #pragma unroll
-        for (int c = 0; c < QPL; ++c) {
-            const int q = lane + 32 * c;
-            float4 p = f4(0.f);
-            if (q < Q)
-                for (int w2 = 0; w2 < BWD_WARPS; ++w2) {
-                    const float4 x = reinterpret_cast<const float4*>(s_pp + w2 * d_v)[q];
-                    p = make_float4(p.x + x.x, p.y + x.y, p.z + x.z, p.w + x.w);
-                }
-            dd[c] = make_float4(bta * (vv[c].x - p.x), bta * (vv[c].y - p.y), bta * (vv[c].z - p.z),
-                                bta * (vv[c].w - p.w));
-        }
-#pragma unroll
-        for (int k = 0; k < WPW; ++k) {
+        for (int k = 0; k < KPL; ++k) {
             const int s = sl[k];
             if (s < 0) continue;
-            const int i = warp + BWD_WARPS * k;
-            const size_t lr = (bt * W + i) * (size_t)d_v;
-#pragma unroll
-            for (int c = 0; c < QPL; ++c) {
-                const int q = lane + 32 * c;
-                if (q < Q) {
-                    reinterpret_cast<float4*>(P.log_rows + lr)[q] = mraw[k][c];
-                    reinterpret_cast<float4*>(Mb + (size_t)s * d_v)[q] =
-                        f4_fma(wi[k], dd[c], raw[k][c]);
-                }
+            const int i = g + 16 * k;
+            if (qok) {
+                reinterpret_cast<float4*>(P.log_rows + (bt * W + i) * (size_t)d_v)[q] = mraw[k];
+                reinterpret_cast<float4*>(Mb + (size_t)s * d_v)[q] = f4_fma(wi[k], dd, raw[k]);
             }
-            if (lane == 0) {
-                P.log_stamp[bt * W + i] = st[k];
+            if (h2 == 0) {
                 stb[s] = L;
+                if (lead) P.log_stamp[bt * W + i] = st[k];
             }
         }
-        if (tid == 0) P.log_lam[bh * (size_t)(T + 1) + t + 1] = L;
-        __syncthreads();  // this token's rows and stamps before the next token's gathers
+        if (lead && lane == 0) P.log_lam[bh * (size_t)(T + 1) + t + 1] = L;
+        __syncwarp();  // this token's rows and stamps before the next token's loads
     }
-    if (tid == 0) lambda[bh] = L;
 }
 
 // ---- the backward sweep ---------------------------------------------------------------
-// Per token: its indices, weights, dout and v rows were fetched during the previous token;
-// the read rows' stamps, then their rows (M side and gradient side) go out together; the
-// write rows' M side (log stamps, current stamps, then log and current rows) is issued
-// before the read rows are processed, their gradient side after the barrier that publishes
-// the read rows' gradient updates.
-template <typename VT, int QPL, int WPW>
-__global__ void __launch_bounds__(BWD_THREADS) bwd_sweep_kernel(
+template <typename VT, int KPL>
+__global__ void __launch_bounds__(32) bwd_sweep_kernel(
     const VT* __restrict__ v, const float* __restrict__ alpha, const float* __restrict__ beta,
     const int32_t* __restrict__ widx, const float* __restrict__ ww,
     const int32_t* __restrict__ ridx, const float* __restrict__ rw, float* __restrict__ M,
-    double* __restrict__ stamp, double* __restrict__ lambda, const float* __restrict__ M0,
-    BwdPtrs P, const float* __restrict__ dout, float* __restrict__ dv_out,
-    float* __restrict__ dalpha, float* __restrict__ dbeta, float* __restrict__ dww,
-    float* __restrict__ drw, int H, int N, int T, int d_v, int W, int R, int touched) {
-    extern __shared__ __align__(16) unsigned char bwd_smem[];
-    const size_t bh = blockIdx.x;
+    const float* __restrict__ M0, BwdPtrs P, const float* __restrict__ dout,
+    float* __restrict__ dv_out, int H, int N, int T, int d_v, int W, int R, int S, int touched) {
+    __shared__ int s_rs[BWD_MAXO];
+    __shared__ float s_ru[BWD_MAXO];
+    const int sc = (int)(blockIdx.x % S);
+    const size_t bh = blockIdx.x / S, BH = gridDim.x / S;
+    const size_t BHT = BH * (size_t)T;
     const int h = (int)(bh % H);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int Q = d_v / 4;
-    float* s_pp = reinterpret_cast<float*>(bwd_smem);          // [8][d_v] partial p
-    float* s_pd = s_pp + BWD_WARPS * d_v;                      // [8][d_v] partial sum w dM
-    double* s_part = reinterpret_cast<double*>(s_pd + BWD_WARPS * d_v);  // [8][4] partial sums
+    const int lane = threadIdx.x, h2 = lane & 1, g = lane >> 1;
+    const int Q = d_v / 4, q = BWD_SLICE_Q * sc + h2;
+    const bool qok = q < Q;
     float* Mb = M + bh * (size_t)N * d_v;
     const float* M0h = M0 + (size_t)h * N * d_v;
-    double* stb = stamp + bh * (size_t)N;
+    double* stb = P.pst + ((size_t)sc * BH + bh) * N;
+    double* dsb = P.pds + ((size_t)sc * BH + bh) * N;
     float* dMb = P.dM + bh * (size_t)N * d_v;
-    double* dsb = P.dstamp + bh * (size_t)N;
     const double* lamb = P.log_lam + bh * (size_t)(T + 1);
-    double X = 0.0, Gam = 0.0;  // <dM, M> over every slot; backward log-decay prefix
-    constexpr int RPW = WPW;
+    double X = 0.0, Gam = 0.0;  // this lane's share of <dM, M>; backward log-decay prefix
     // the next token's inputs
-    int nrs[RPW], nws[WPW];
-    float nu[RPW], nwi[WPW], na = 1.f, nb = 0.f;
-    float4 nG[QPL], nv[QPL];
+    int nrs[KPL], nws[KPL];
+    float nu[KPL], nwi[KPL], na = 1.f, nb = 0.f;
+    float4 nG = f4(0.f), nv = f4(0.f);
     auto fetch = [&](int t) {
         const size_t bt = bh * (size_t)T + t;
         na = alpha[bt] > 0.f ? alpha[bt] : 1.f;
         nb = beta[bt];
 #pragma unroll
-        for (int k = 0; k < RPW; ++k) {
-            const int j = warp + BWD_WARPS * k;
+        for (int k = 0; k < KPL; ++k) {
+            const int j = g + 16 * k;
             nrs[k] = j < R ? ridx[bt * R + j] : -1;
             nu[k] = j < R ? rw[bt * R + j] : 0.f;
+            nws[k] = j < W ? widx[bt * W + j] : -1;
+            nwi[k] = j < W ? ww[bt * W + j] : 0.f;
         }
-#pragma unroll
-        for (int k = 0; k < WPW; ++k) {
-            const int i = warp + BWD_WARPS * k;
-            nws[k] = i < W ? widx[bt * W + i] : -1;
-            nwi[k] = i < W ? ww[bt * W + i] : 0.f;
-        }
-#pragma unroll
-        for (int c = 0; c < QPL; ++c) {
-            const int q = lane + 32 * c;
-            nG[c] = q < Q ? reinterpret_cast<const float4*>(dout + bt * d_v)[q] : f4(0.f);
-            nv[c] = q < Q ? bwd_load_v4<VT>(v + bt * d_v + 4 * q) : f4(0.f);
+        if (qok) {
+            nG = reinterpret_cast<const float4*>(dout + bt * d_v)[q];
+            nv = bwd_load_v4<VT>(v + bt * d_v + 4 * q);
         }
     };
     if (T > 0) fetch(T - 1);
@@ -288,228 +275,173 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_sweep_kernel(
         const size_t bt = bh * (size_t)T + t;
         const float a = na, bta = nb;
         const double Lt = lamb[t + 1], Lp = lamb[t];
-        int rs[RPW], sl[WPW];
-        float u[RPW], wi[WPW];
-        float4 G[QPL], vv[QPL];
+        int rs[KPL], sl[KPL];
+        float u[KPL], wi[KPL];
 #pragma unroll
-        for (int k = 0; k < RPW; ++k) {
+        for (int k = 0; k < KPL; ++k) {
             rs[k] = slot_ok(nrs[k], N) ? nrs[k] : -1;  // the forward reported bad slots
             u[k] = nu[k];
-        }
-#pragma unroll
-        for (int k = 0; k < WPW; ++k) {
             sl[k] = slot_ok(nws[k], N) ? nws[k] : -1;
             wi[k] = nwi[k];
         }
+        const float4 G = nG, vv = nv;
+        // this token's read slots, for the write rows that share one
+        if (h2 == 0)
 #pragma unroll
-        for (int c = 0; c < QPL; ++c) {
-            G[c] = nG[c];
-            vv[c] = nv[c];
-        }
-        // -- round 1: stamps of the read rows and of the write rows (M side)
-        double rst[RPW], rds[RPW], wso[WPW], wsn[WPW];
-#pragma unroll
-        for (int k = 0; k < RPW; ++k) {
-            rst[k] = rs[k] >= 0 ? stb[rs[k]] : 0.0;
-            rds[k] = rs[k] >= 0 ? dsb[rs[k]] : 0.0;
-        }
-#pragma unroll
-        for (int k = 0; k < WPW; ++k) {
-            const int i = warp + BWD_WARPS * k;
-            wso[k] = sl[k] >= 0 ? P.log_stamp[bt * W + i] : 0.0;
-            wsn[k] = sl[k] >= 0 ? stb[sl[k]] : 0.0;
-        }
-        // -- round 2: the read rows (M and dM) and the write rows' M side (log and current)
-        float4 rm[RPW][QPL], rg[RPW][QPL], mp[WPW][QPL], mt[WPW][QPL];
-        float fo[WPW], fn[WPW];
-#pragma unroll
-        for (int k = 0; k < RPW; ++k) {
-            const int s = rs[k];
-            const float f = bwd_factor(rst[k], Lt, touched);
-            const float gf = (s < 0 || isnan(rds[k])) ? 0.f : bwd_exp(Gam - rds[k]);
-#pragma unroll
-            for (int c = 0; c < QPL; ++c) {
-                const int q = lane + 32 * c;
-                rm[k][c] = rg[k][c] = f4(0.f);
-                if (s >= 0 && q < Q) {
-                    const float* src = (signbit(f) ? M0h : Mb) + (size_t)s * d_v;
-                    rm[k][c] = f4_scale(fabsf(f), reinterpret_cast<const float4*>(src)[q]);
-                    if (gf != 0.f)
-                        rg[k][c] = f4_scale(gf, reinterpret_cast<const float4*>(dMb + (size_t)s * d_v)[q]);
+            for (int k = 0; k < KPL; ++k) {
+                const int j = g + 16 * k;
+                if (j < R) {
+                    s_rs[j] = rs[k];
+                    s_ru[j] = u[k];
                 }
             }
-        }
+        // -- one round of loads: read rows (stamps, M, M0, dM), write rows (log, stamps,
+        //    current row, M0, dM)
+        double rst[KPL], rds[KPL], wso[KPL], wsn[KPL], wds[KPL];
+        float4 rM[KPL], rM0[KPL], rG[KPL], lrow[KPL], mc[KPL], m0[KPL], wdm[KPL];
 #pragma unroll
-        for (int k = 0; k < WPW; ++k) {
-            const int s = sl[k], i = warp + BWD_WARPS * k;
-            fo[k] = bwd_factor(wso[k], Lp, touched);  // value factor at t-1
-            fn[k] = bwd_factor(wsn[k], Lt, touched);  // at t
-            const size_t lr = (bt * W + (i < W ? i : 0)) * (size_t)d_v;
-#pragma unroll
-            for (int c = 0; c < QPL; ++c) {
-                const int q = lane + 32 * c;
-                mp[k][c] = mt[k][c] = f4(0.f);
-                if (s >= 0 && q < Q) {
-                    const float* so_src = signbit(fo[k]) ? M0h + (size_t)s * d_v : P.log_rows + lr;
-                    mp[k][c] = f4_scale(fabsf(fo[k]), reinterpret_cast<const float4*>(so_src)[q]);
-                    const float* sn_src = (signbit(fn[k]) ? M0h : Mb) + (size_t)s * d_v;
-                    mt[k][c] = f4_scale(fabsf(fn[k]), reinterpret_cast<const float4*>(sn_src)[q]);
-                }
+        for (int k = 0; k < KPL; ++k) {
+            const int s = rs[k], sw = sl[k], i = g + 16 * k;
+            rst[k] = s >= 0 ? stb[s] : 0.0;
+            rds[k] = s >= 0 ? dsb[s] : 0.0;
+            wso[k] = sw >= 0 ? P.log_stamp[bt * W + i] : 0.0;
+            wsn[k] = sw >= 0 ? stb[sw] : 0.0;
+            wds[k] = sw >= 0 ? dsb[sw] : 0.0;
+            rM[k] = rM0[k] = rG[k] = lrow[k] = mc[k] = m0[k] = wdm[k] = f4(0.f);
+            if (qok && s >= 0) {
+                rM[k] = reinterpret_cast<const float4*>(Mb + (size_t)s * d_v)[q];
+                rM0[k] = reinterpret_cast<const float4*>(M0h + (size_t)s * d_v)[q];
+                rG[k] = reinterpret_cast<const float4*>(dMb + (size_t)s * d_v)[q];
+            }
+            if (qok && sw >= 0) {
+                lrow[k] = reinterpret_cast<const float4*>(P.log_rows + (bt * W + i) * (size_t)d_v)[q];
+                mc[k] = reinterpret_cast<const float4*>(Mb + (size_t)sw * d_v)[q];
+                m0[k] = reinterpret_cast<const float4*>(M0h + (size_t)sw * d_v)[q];
+                wdm[k] = reinterpret_cast<const float4*>(dMb + (size_t)sw * d_v)[q];
             }
         }
         if (t > 0) fetch(t - 1);
         // -- read rows: du_j, dM[r_j] += u_j G, X += u_j du_j
         double xr = 0.0;
 #pragma unroll
-        for (int k = 0; k < RPW; ++k) {
-            const int j = warp + BWD_WARPS * k;
-            const int s = rs[k];
-            if (s < 0) continue;  // warp-uniform
-            float acc = 0.f;
-#pragma unroll
-            for (int c = 0; c < QPL; ++c) {
-                acc += f4_dot(G[c], rm[k][c]);
-                rg[k][c] = f4_fma(u[k], G[c], rg[k][c]);
+        for (int k = 0; k < KPL; ++k) {
+            const int s = rs[k], j = g + 16 * k;
+            const float f = bwd_factor(rst[k], Lt, touched);
+            const float4 rm = f4_scale(fabsf(f), signbit(f) ? rM0[k] : rM[k]);
+            const float gf = (s < 0 || isnan(rds[k])) ? 0.f : bwd_exp(Gam - rds[k]);
+            const float part = s >= 0 ? f4_dot(G, rm) : 0.f;
+            const float du = pair_sum(part);
+            if (h2 == 0 && j < R) P.p_drw[((size_t)sc * BHT + bt) * R + j] = du;
+            xr += (double)u[k] * part;
+            if (s >= 0) {
+                if (qok)
+                    reinterpret_cast<float4*>(dMb + (size_t)s * d_v)[q] =
+                        f4_fma(u[k], G, gf != 0.f ? f4_scale(gf, rG[k]) : f4(0.f));
+                if (h2 == 0) dsb[s] = Gam;
             }
-            const float du = warp_sum(acc);
-            if (lane == 0) drw[bt * R + j] = du;
-            xr += (double)u[k] * du;
-#pragma unroll
-            for (int c = 0; c < QPL; ++c) {
-                const int q = lane + 32 * c;
-                if (q < Q) reinterpret_cast<float4*>(dMb + (size_t)s * d_v)[q] = rg[k][c];
-            }
-            __syncwarp();
-            if (lane == 0) dsb[s] = Gam;
         }
-        if (lane == 0) s_part[warp * 4 + 0] = xr;
-        __syncthreads();  // read rows of dM (and their stamps) before the write rows use them
-        if (!touched)
-            for (int w2 = 0; w2 < BWD_WARPS; ++w2) X += s_part[w2 * 4 + 0];
-        // -- round 3: the write rows' gradient side
-        double wds[WPW];
+        __syncwarp();  // read slots listed; read rows' gradient stored before the write rows'
+        // -- write rows
+        float4 mp[KPL], mt[KPL], dm[KPL], pp = f4(0.f), pd = f4(0.f);
 #pragma unroll
-        for (int k = 0; k < WPW; ++k) wds[k] = sl[k] >= 0 ? dsb[sl[k]] : 0.0;
-        float4 dm[WPW][QPL];
-        float4 pp[QPL], pd[QPL];
-#pragma unroll
-        for (int c = 0; c < QPL; ++c) pp[c] = pd[c] = f4(0.f);
-#pragma unroll
-        for (int k = 0; k < WPW; ++k) {
+        for (int k = 0; k < KPL; ++k) {
             const int s = sl[k];
+            const float fo = bwd_factor(wso[k], Lp, touched);  // value factor at t-1
+            const float fn = bwd_factor(wsn[k], Lt, touched);  // at t
+            mp[k] = f4_scale(fabsf(fo), signbit(fo) ? m0[k] : lrow[k]);
+            mt[k] = f4_scale(fabsf(fn), signbit(fn) ? m0[k] : mc[k]);
             const float gf = (s < 0 || isnan(wds[k])) ? 0.f : bwd_exp(Gam - wds[k]);
-#pragma unroll
-            for (int c = 0; c < QPL; ++c) {
-                const int q = lane + 32 * c;
-                dm[k][c] = f4(0.f);
-                if (gf != 0.f && q < Q)
-                    dm[k][c] = f4_scale(gf, reinterpret_cast<const float4*>(dMb + (size_t)s * d_v)[q]);
-                pp[c] = f4_fma(wi[k] * a, mp[k][c], pp[c]);
-                pd[c] = f4_fma(wi[k], dm[k][c], pd[c]);
-            }
+            // a row never reached holds stale workspace: select zero, never scale it
+            dm[k] = gf != 0.f ? f4_scale(gf, wdm[k]) : f4(0.f);
+            if (s >= 0)
+                for (int j = 0; j < R; ++j)
+                    if (s_rs[j] == s) {  // read in this token too: its update comes first
+                        dm[k] = f4_fma(s_ru[j], G, dm[k]);
+                        break;
+                    }
+            if (s < 0) mp[k] = mt[k] = dm[k] = f4(0.f);
+            pp = f4_fma(wi[k] * a, mp[k], pp);
+            pd = f4_fma(wi[k], dm[k], pd);
         }
+        pp = f4_sum_groups(pp);
+        pd = f4_sum_groups(pd);
+        const float4 e = make_float4(vv.x - pp.x, vv.y - pp.y, vv.z - pp.z, vv.w - pp.w);
+        const float4 de = f4_scale(bta, pd);
+        if (g == 0 && qok) reinterpret_cast<float4*>(dv_out + bt * d_v)[q] = de;
+        double sb = 0.0, s1 = 0.0, s2 = 0.0;  // shares of dbeta, <dM, M_t>, <dMt, M_{t-1}>
+        const float scw = touched ? a : 1.f;  // every-slot decay keeps alpha in Gam
 #pragma unroll
-        for (int c = 0; c < QPL; ++c) {
-            const int q = lane + 32 * c;
-            if (q < Q) {
-                reinterpret_cast<float4*>(s_pp + warp * d_v)[q] = pp[c];
-                reinterpret_cast<float4*>(s_pd + warp * d_v)[q] = pd[c];
-            }
-        }
-        __syncthreads();
-        float4 e[QPL], de[QPL];
-#pragma unroll
-        for (int c = 0; c < QPL; ++c) {
-            const int q = lane + 32 * c;
-            float4 p = f4(0.f), d = f4(0.f);
-            if (q < Q)
-                for (int w2 = 0; w2 < BWD_WARPS; ++w2) {
-                    const float4 x = reinterpret_cast<const float4*>(s_pp + w2 * d_v)[q];
-                    const float4 y = reinterpret_cast<const float4*>(s_pd + w2 * d_v)[q];
-                    p = make_float4(p.x + x.x, p.y + x.y, p.z + x.z, p.w + x.w);
-                    d = make_float4(d.x + y.x, d.y + y.y, d.z + y.z, d.w + y.w);
-                }
-            e[c] = make_float4(vv[c].x - p.x, vv[c].y - p.y, vv[c].z - p.z, vv[c].w - p.w);
-            de[c] = f4_scale(bta, d);
-            if (warp == 0 && q < Q) reinterpret_cast<float4*>(dv_out + bt * d_v)[q] = de[c];
-        }
-        double sb = 0.0, s1 = 0.0, s2 = 0.0;  // dbeta; <dM, M_t>; <dMt, M_{t-1}> (write rows)
-#pragma unroll
-        for (int k = 0; k < WPW; ++k) {
-            const int i = warp + BWD_WARPS * k;
-            const int s = sl[k];
+        for (int k = 0; k < KPL; ++k) {
+            const int s = sl[k], i = g + 16 * k;
+            const float ge = f4_dot(dm[k], e), gm = f4_dot(de, mp[k]);
+            const float4 nd = f4_fma(-wi[k], de, dm[k]);  // dMt[s_i]
+            const float dw = bta * pair_sum(ge) - a * pair_sum(gm);
+            if (h2 == 0 && i < W) P.p_dww[((size_t)sc * BHT + bt) * W + i] = s >= 0 ? dw : 0.f;
             if (s < 0) continue;
-            float ge = 0.f, gm = 0.f, gmt = 0.f, gmp = 0.f;
-            float4 nd[QPL];
-#pragma unroll
-            for (int c = 0; c < QPL; ++c) {
-                ge += f4_dot(dm[k][c], e[c]);
-                gm += f4_dot(de[c], mp[k][c]);
-                gmt += f4_dot(dm[k][c], mt[k][c]);
-                nd[c] = f4_fma(-wi[k], de[c], dm[k][c]);  // dMt[s_i]
-                gmp += f4_dot(nd[c], mp[k][c]);
-            }
-            ge = warp_sum(ge);
-            gm = warp_sum(gm);
-            gmt = warp_sum(gmt);
-            gmp = warp_sum(gmp);
-            if (lane == 0) dww[bt * W + i] = bta * ge - a * gm;
             sb += (double)wi[k] * ge;
-            s1 += gmt;
-            s2 += gmp;
-            // dM_{t-1}[s] = alpha dMt[s]: every-slot decay keeps alpha in the prefix Gam
-            const float sc = touched ? a : 1.f;
-            const size_t lr = (bt * W + i) * (size_t)d_v;
-#pragma unroll
-            for (int c = 0; c < QPL; ++c) {
-                const int q = lane + 32 * c;
-                if (q < Q) {
-                    reinterpret_cast<float4*>(dMb + (size_t)s * d_v)[q] = f4_scale(sc, nd[c]);
-                    reinterpret_cast<float4*>(Mb + (size_t)s * d_v)[q] =
-                        reinterpret_cast<const float4*>(P.log_rows + lr)[q];  // restore
-                }
+            s1 += f4_dot(dm[k], mt[k]);
+            s2 += f4_dot(nd, mp[k]);
+            if (qok) {
+                reinterpret_cast<float4*>(dMb + (size_t)s * d_v)[q] = f4_scale(scw, nd);
+                reinterpret_cast<float4*>(Mb + (size_t)s * d_v)[q] = lrow[k];  // restore
             }
-            __syncwarp();
-            if (lane == 0) {
+            if (h2 == 0) {
                 dsb[s] = Gam;
                 stb[s] = wso[k];
             }
         }
-        if (lane == 0) {
-            s_part[warp * 4 + 1] = sb;
-            s_part[warp * 4 + 2] = s1;
-            s_part[warp * 4 + 3] = s2;
-        }
-        __syncthreads();
-        double SB = 0.0, S1 = 0.0, S2 = 0.0;
-        for (int w2 = 0; w2 < BWD_WARPS; ++w2) {
-            SB += s_part[w2 * 4 + 1];
-            S1 += s_part[w2 * 4 + 2];
-            S2 += s_part[w2 * 4 + 3];
-        }
         double da;
         if (touched) {
-            da = S2;
+            da = s2;
         } else {
-            da = (X - S1) / (double)a + S2;
+            X += xr;
+            da = (X - s1) / (double)a + s2;
             X = (double)a * da;
             Gam += log((double)a);
         }
-        if (tid == 0) {
-            dalpha[bt] = (float)da;
-            dbeta[bt] = (float)SB;
+        da = warp_sum_d(da);
+        sb = warp_sum_d(sb);
+        if (lane == 0) {
+            P.p_da[(size_t)sc * BHT + bt] = da;
+            P.p_db[(size_t)sc * BHT + bt] = sb;
         }
-        __syncthreads();  // s_part and s_pp are rewritten by the next token
+        __syncwarp();  // this token's stores and list reads before the next token's
     }
-    if (tid == 0) {
-        lambda[bh] = lamb[0];
-        P.log_lam[bh * (size_t)(T + 1) + T] = Gam;  // the final prefix, for the dense gradient
+    if (sc == 0 && lane == 0) P.gam[bh] = Gam;
+}
+
+// The per-slice shares summed in slice order: dww, drw, dbeta, dalpha.
+__global__ void bwd_reduce_kernel(const BwdPtrs P, int S, size_t BHT, int W, int R,
+                                  float* __restrict__ dww, float* __restrict__ drw,
+                                  float* __restrict__ dbeta, float* __restrict__ dalpha) {
+    const size_t nw = BHT * W, nr = BHT * R;
+    const size_t total = nw + nr + 2 * BHT;
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+        if (i < nw) {
+            float acc = 0.f;
+            for (int c = 0; c < S; ++c) acc += P.p_dww[c * nw + i];
+            dww[i] = acc;
+        } else if (i < nw + nr) {
+            const size_t k = i - nw;
+            float acc = 0.f;
+            for (int c = 0; c < S; ++c) acc += P.p_drw[c * nr + k];
+            drw[k] = acc;
+        } else {
+            const bool is_b = i < nw + nr + BHT;
+            const size_t k = i - nw - nr - (is_b ? 0 : BHT);
+            const double* src = is_b ? P.p_db : P.p_da;
+            double acc = 0.0;
+            for (int c = 0; c < S; ++c) acc += src[c * BHT + k];
+            (is_b ? dbeta : dalpha)[k] = (float)acc;
+        }
     }
 }
 
 // Dense gradient with respect to the state at the start of the call: dM_in[s] = raw *
-// e^{Gam_final - stamp} (zero for rows never reached).
-__global__ void bwd_dense_kernel(const BwdPtrs P, int T, int N, int d_v, size_t n_rows,
+// e^{Gam_final - stamp} (zero for rows never reached).  The gradient stamps of slice 0
+// (all slices end with the same ones).
+__global__ void bwd_dense_kernel(const BwdPtrs P, int N, int d_v, size_t n_rows,
                                  float* __restrict__ out) {
     const int Q = d_v / 4;
     const size_t total = n_rows * Q;
@@ -518,10 +450,10 @@ __global__ void bwd_dense_kernel(const BwdPtrs P, int T, int N, int d_v, size_t 
         const size_t row = i / Q;
         const int q = (int)(i % Q);
         const size_t bh = row / N;
-        const double ds = P.dstamp[row];
+        const double ds = P.pds[row];
         float4 val = f4(0.f);
         if (!isnan(ds)) {
-            const float g = bwd_exp(P.log_lam[bh * (size_t)(T + 1) + T] - ds);
+            const float g = bwd_exp(P.gam[bh] - ds);
             val = f4_scale(g, reinterpret_cast<const float4*>(P.dM + row * d_v)[q]);
         }
         reinterpret_cast<float4*>(out + row * d_v)[q] = val;

@@ -344,42 +344,48 @@ sdm_status score_both_roles(const sdm_dims* d, const void* q, const void* k, con
     return launch_score(d, q, skr, d->R, ridx, rw, s);
 }
 
+// column slices per (b,h) in the backward (8 columns each)
+int bwd_slices(const sdm_dims* d) { return (d->d_v / 4 + BWD_SLICE_Q - 1) / BWD_SLICE_Q; }
+
 struct BwdLayout {
-    size_t off_rows, off_lstamp, off_lam, off_dM, off_dstamp, total;
+    size_t off_rows, off_lstamp, off_lam, off_dM, off_pst, off_pds, off_pdww, off_pdrw, off_pdb,
+        off_pda, off_gam, total;
 };
 
 BwdLayout bwd_layout(const sdm_dims* d) {
     BwdLayout L{};
     const size_t BH = (size_t)BH_of(d), T = (size_t)d->T, N = (size_t)N_of(d);
+    const size_t S = (size_t)bwd_slices(d);
     size_t o = 0;
     L.off_rows = o;   o = up256(o + BH * T * (size_t)d->W * d->d_v * 4);
     L.off_lstamp = o; o = up256(o + BH * T * (size_t)d->W * 8);
     L.off_lam = o;    o = up256(o + BH * (T + 1) * 8);
     L.off_dM = o;     o = up256(o + BH * N * (size_t)d->d_v * 4);
-    L.off_dstamp = o; o = up256(o + BH * N * 8);
+    L.off_pst = o;    o = up256(o + S * BH * N * 8);
+    L.off_pds = o;    o = up256(o + S * BH * N * 8);
+    L.off_pdww = o;   o = up256(o + S * BH * T * (size_t)d->W * 4);
+    L.off_pdrw = o;   o = up256(o + S * BH * T * (size_t)d->R * 4);
+    L.off_pdb = o;    o = up256(o + S * BH * T * 8);
+    L.off_pda = o;    o = up256(o + S * BH * T * 8);
+    L.off_gam = o;    o = up256(o + BH * 8);
     L.total = o;
     return L;
 }
 
-template <typename VT, int QPL, int WPW>
+template <typename VT, int KPL>
 sdm_status launch_backward_t(const sdm_dims* d, const BwdPtrs& P, const void* v,
                              const float* alpha, const float* beta, const int32_t* widx,
                              const float* ww, const int32_t* ridx, const float* rw,
-                             const sdm_state* st, const float* dout, float* dv, float* dalpha,
-                             float* dbeta, float* dww, float* drw, cudaStream_t s) {
+                             const sdm_state* st, const float* dout, float* dv, cudaStream_t s) {
     const int touched = d->decay == SDM_DECAY_TOUCHED;
-    const size_t smem = bwd_smem_bytes(d->d_v);
-    auto rk = bwd_replay_kernel<VT, QPL, WPW>;
-    auto sk = bwd_sweep_kernel<VT, QPL, WPW>;
-    if (!set_smem(rk, smem) || !set_smem(sk, smem)) return SDM_ERR_CUDA;
-    const unsigned grid = (unsigned)BH_of(d);
-    rk<<<grid, BWD_THREADS, smem, s>>>((const VT*)v, alpha, beta, widx, ww, st->M, st->stamp,
-                                       st->Lambda, st->M0, P, d->H, (int)N_of(d), d->T, d->d_v,
-                                       d->W, touched);
-    sk<<<grid, BWD_THREADS, smem, s>>>((const VT*)v, alpha, beta, widx, ww, ridx, rw, st->M,
-                                       st->stamp, st->Lambda, st->M0, P, dout, dv, dalpha, dbeta,
-                                       dww, drw, d->H, (int)N_of(d), d->T, d->d_v, d->W, d->R,
-                                       touched);
+    const int S = bwd_slices(d);
+    const unsigned grid = (unsigned)((size_t)BH_of(d) * S);
+    bwd_replay_kernel<VT, KPL><<<grid, 32, 0, s>>>((const VT*)v, alpha, beta, widx, ww, st->M,
+                                                   st->Lambda, st->M0, P, d->H, (int)N_of(d),
+                                                   d->T, d->d_v, d->W, S, touched);
+    bwd_sweep_kernel<VT, KPL><<<grid, 32, 0, s>>>((const VT*)v, alpha, beta, widx, ww, ridx, rw,
+                                                  st->M, st->M0, P, dout, dv, d->H, (int)N_of(d),
+                                                  d->T, d->d_v, d->W, d->R, S, touched);
     return launch_status();
 }
 
@@ -759,41 +765,48 @@ sdm_status sdm_backward(const sdm_dims* dims, const void* v, const float* alpha,
     if (!aligned16(ws)) return SDM_ERR_ALIGN;
     cudaStream_t s = (cudaStream_t)stream;
     const size_t rows = (size_t)BH_of(dims) * (size_t)N_of(dims);
+    const int S = bwd_slices(dims);
+    if ((size_t)BH_of(dims) * S > 0x7fffffffull) return SDM_ERR_SHAPE;
     unsigned char* b = static_cast<unsigned char*>(ws);
     BwdPtrs P;
     P.log_rows = reinterpret_cast<float*>(b + L.off_rows);
     P.log_stamp = reinterpret_cast<double*>(b + L.off_lstamp);
     P.log_lam = reinterpret_cast<double*>(b + L.off_lam);
     P.dM = reinterpret_cast<float*>(b + L.off_dM);
-    P.dstamp = reinterpret_cast<double*>(b + L.off_dstamp);
+    P.pst = reinterpret_cast<double*>(b + L.off_pst);
+    P.pds = reinterpret_cast<double*>(b + L.off_pds);
+    P.p_dww = reinterpret_cast<float*>(b + L.off_pdww);
+    P.p_drw = reinterpret_cast<float*>(b + L.off_pdrw);
+    P.p_db = reinterpret_cast<double*>(b + L.off_pdb);
+    P.p_da = reinterpret_cast<double*>(b + L.off_pda);
+    P.gam = reinterpret_cast<double*>(b + L.off_gam);
     const int threads = 256;
-    {   // every memory-gradient row starts at zero (NaN stamp)
-        size_t blocks = (rows + threads - 1) / threads;
+    auto grid_for = [](size_t n) {
+        size_t blocks = (n + 255) / 256;
         if (blocks > 148 * 64) blocks = 148 * 64;
-        if (blocks == 0) blocks = 1;
-        state_reset_kernel<<<(unsigned)blocks, threads, 0, s>>>(P.dstamp, rows, nullptr, 0);
-    }
+        return (unsigned)(blocks == 0 ? 1 : blocks);
+    };
+    // private stamp copies per slice, every memory-gradient row at zero (NaN stamp)
+    bwd_init_kernel<<<grid_for((size_t)S * rows), threads, 0, s>>>(st->stamp, P, rows, S,
+                                                                   (int)BH_of(dims));
     if (dims->T > 0) {
-        const int wpw = ((dims->W > dims->R ? dims->W : dims->R) + BWD_WARPS - 1) / BWD_WARPS;
-        const bool q2 = dims->d_v > 128;
-#define SDM_BWD(VT, Q, WP) launch_backward_t<VT, Q, WP>(dims, P, v, alpha, beta, widx, ww, ridx, rw, st, dout, dv, dalpha, dbeta, dww, drw, s)
+        const int m = dims->W > dims->R ? dims->W : dims->R;
+#define SDM_BWD(VT, K) launch_backward_t<VT, K>(dims, P, v, alpha, beta, widx, ww, ridx, rw, st, dout, dv, s)
         if (dims->v_dtype == SDM_BF16) {
-            if (wpw <= 4) e = q2 ? SDM_BWD(__nv_bfloat16, 2, 4) : SDM_BWD(__nv_bfloat16, 1, 4);
-            else e = q2 ? SDM_BWD(__nv_bfloat16, 2, 8) : SDM_BWD(__nv_bfloat16, 1, 8);
+            e = m <= 16 ? SDM_BWD(__nv_bfloat16, 1) : m <= 32 ? SDM_BWD(__nv_bfloat16, 2)
+              : m <= 64 ? SDM_BWD(__nv_bfloat16, 4) : SDM_BWD(__nv_bfloat16, 8);
         } else {
-            if (wpw <= 4) e = q2 ? SDM_BWD(float, 2, 4) : SDM_BWD(float, 1, 4);
-            else e = q2 ? SDM_BWD(float, 2, 8) : SDM_BWD(float, 1, 8);
+            e = m <= 16 ? SDM_BWD(float, 1) : m <= 32 ? SDM_BWD(float, 2)
+              : m <= 64 ? SDM_BWD(float, 4) : SDM_BWD(float, 8);
         }
 #undef SDM_BWD
         if (e) return e;
-    } else if (cudaMemsetAsync(P.log_lam, 0, (size_t)BH_of(dims) * 8, s) != cudaSuccess) {
-        return SDM_ERR_CUDA;  // no token: the dense gradient's final prefix is 0
+        const size_t BHT = (size_t)BH_of(dims) * dims->T;
+        bwd_reduce_kernel<<<grid_for(BHT * (dims->W + dims->R + 2)), threads, 0, s>>>(
+            P, S, BHT, dims->W, dims->R, dww, drw, dbeta, dalpha);
     }
-    size_t blocks = (rows * (dims->d_v / 4) + threads - 1) / threads;
-    if (blocks > 148 * 64) blocks = 148 * 64;
-    if (blocks == 0) blocks = 1;
-    bwd_dense_kernel<<<(unsigned)blocks, threads, 0, s>>>(P, dims->T, (int)N_of(dims), dims->d_v,
-                                                          rows, dM_in);
+    bwd_dense_kernel<<<grid_for(rows * (dims->d_v / 4)), threads, 0, s>>>(P, (int)N_of(dims),
+                                                                          dims->d_v, rows, dM_in);
     return launch_status();
 }
 
