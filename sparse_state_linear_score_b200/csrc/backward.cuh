@@ -4,8 +4,8 @@
 //
 // Parallel over value columns.  Once the slots and gates are fixed, the chain through the
 // tokens is per column: every row operation acts column by column, and only outputs (dalpha,
-// dbeta, dw, du) sum over columns.  Each (b,h) is therefore split into slices of 8 columns
-// (two float4), one warp per slice, and every slice walks the tokens one at a time on its
+// dbeta, dw, du) sum over columns.  Each (b,h) is therefore split into slices of 4 columns
+// (one float4), one warp per slice, and every slice walks the tokens one at a time on its
 // own.  Stamps belong to slots, not columns, and the slices run at their own pace, so each
 // slice keeps private copies of the slot stamps and of the gradient stamps (all copies hold
 // the same values at the same point of the walk).  Column sums are written per slice and
@@ -25,7 +25,8 @@
 //           running X = <dM, M> (full inner product) that only the touched rows change:
 //           dalpha = (X - sum_i <dM[s_i], M_t[s_i]>) / alpha + sum_i <dMt[s_i], M_{t-1}[s_i]>,
 //           then X <- alpha dalpha; dM_{t-1} = alpha dMt, kept lazily as raw rows, a
-//           backward log-decay prefix Gam (+= log alpha per token) and per-row stamps.
+//           backward log-decay prefix Gam (the sum of log alpha over the later tokens)
+//           and per-row stamps.
 //           X is linear in its terms, so each lane carries its own share of it.
 //           Touched-slots decay: dalpha = sum_i <dMt[s_i], M_{t-1}[s_i]> and only the write
 //           rows take the factor alpha.
@@ -33,10 +34,10 @@
 // On return the state is again the state at the start of the call (its stamps and Lambda
 // are never written: the slices work on their private stamp copies).
 //
-// Lane layout in a slice: lane = 2 g + h2, h2 the float4 of the slice, g the row group;
-// lane owns write rows g, g+16, ... and read rows g, g+16, ...  A token's loads (stamps,
-// rows, log) all go out in one round; a slot both read and written in the token takes the
-// read's gradient update through a shared-memory list of the token's read slots.
+// Lane layout in a slice: lane l owns write rows l, l+32, ... and read rows l, l+32, ...
+// (the slice's float4 of each).  A token's loads (stamps, rows, log) all go out in one
+// round; a slot both read and written in the token takes the read's gradient update,
+// found through a small shared-memory hash of the token's read slots.
 #pragma once
 
 #include <math.h>
@@ -46,7 +47,8 @@
 namespace sdm {
 
 constexpr int BWD_MAXO = 128;      // W + R
-constexpr int BWD_SLICE_Q = 2;     // float4 columns per slice
+constexpr int BWD_SLICE_Q = 1;     // float4 columns per slice
+constexpr int BWD_HASH = 256;      // read-slot hash entries (> BWD_MAXO)
 
 // Per-(b,h) records of one call (a byte layout in the workspace); S = slices per (b,h).
 struct BwdPtrs {
@@ -76,10 +78,10 @@ SDM_DEV float4 f4_scale(float s, const float4& a) {
 SDM_DEV float4 f4_add(const float4& a, const float4& b) {
     return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
-// sum over the 16 row groups (lanes of equal h2)
-SDM_DEV float4 f4_sum_groups(float4 x) {
+// sum over the warp's rows
+SDM_DEV float4 f4_sum_rows(float4 x) {
 #pragma unroll
-    for (int m = 2; m < 32; m <<= 1) {
+    for (int m = 1; m < 32; m <<= 1) {
         x.x += __shfl_xor_sync(0xffffffffu, x.x, m);
         x.y += __shfl_xor_sync(0xffffffffu, x.y, m);
         x.z += __shfl_xor_sync(0xffffffffu, x.z, m);
@@ -92,8 +94,7 @@ SDM_DEV double warp_sum_d(double x) {
     for (int m = 16; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
     return x;
 }
-// a row's dot product: the two lanes of one row group
-SDM_DEV float pair_sum(float x) { return x + __shfl_xor_sync(0xffffffffu, x, 1); }
+SDM_DEV unsigned bwd_hash(int s) { return ((unsigned)s * 0x9E3779B1u) >> 24; }
 
 template <typename VT>
 SDM_DEV float4 bwd_load_v4(const VT* p);
@@ -143,9 +144,8 @@ __global__ void __launch_bounds__(32) bwd_replay_kernel(
     const int sc = (int)(blockIdx.x % S);
     const size_t bh = blockIdx.x / S, BH = gridDim.x / S;
     const int h = (int)(bh % H);
-    const int lane = threadIdx.x, h2 = lane & 1, g = lane >> 1;
-    const int Q = d_v / 4, q = BWD_SLICE_Q * sc + h2;
-    const bool qok = q < Q;
+    const int lane = threadIdx.x, g = lane;
+    const int q = sc;  // the slice's float4 column
     const bool lead = sc == 0;  // slice 0 writes the column-free records
     float* Mb = M + bh * (size_t)N * d_v;
     const float* M0h = M0 + (size_t)h * N * d_v;
@@ -154,13 +154,15 @@ __global__ void __launch_bounds__(32) bwd_replay_kernel(
     if (lead && lane == 0) P.log_lam[bh * (size_t)(T + 1)] = L;
     int nsl[KPL];
     float nwi[KPL], na = 1.f, nb = 0.f;
+    double nla = 0.0;  // log alpha of the next token (0 for a gate outside (0,1], reported)
     auto fetch = [&](int t) {
         const size_t bt = bh * (size_t)T + t;
         na = alpha[bt];
         nb = beta[bt];
+        nla = na > 0.f ? log((double)na) : 0.0;
 #pragma unroll
         for (int k = 0; k < KPL; ++k) {
-            const int i = g + 16 * k;
+            const int i = g + 32 * k;
             nsl[k] = i < W ? widx[bt * W + i] : -1;
             nwi[k] = i < W ? ww[bt * W + i] : 0.f;
         }
@@ -169,6 +171,7 @@ __global__ void __launch_bounds__(32) bwd_replay_kernel(
     for (int t = 0; t < T; ++t) {
         const size_t bt = bh * (size_t)T + t;
         const float a = na, bta = nb;
+        const double la = nla;
         int sl[KPL];
         float wi[KPL];
 #pragma unroll
@@ -180,9 +183,9 @@ __global__ void __launch_bounds__(32) bwd_replay_kernel(
                 sl[k] = -1;
             }
         }
-        if (a > 0.f) L += log((double)a);
-        else if (lane == 0) raise_err(SDM_DEVERR_ALPHA);
-        const float4 vv = qok ? bwd_load_v4<VT>(v + bt * d_v + 4 * q) : f4(0.f);
+        L += la;
+        if (!(a > 0.f) && lane == 0) raise_err(SDM_DEVERR_ALPHA);
+        const float4 vv = bwd_load_v4<VT>(v + bt * d_v + 4 * q);
         double st[KPL];
         float4 mraw[KPL], m0[KPL];
 #pragma unroll
@@ -190,7 +193,7 @@ __global__ void __launch_bounds__(32) bwd_replay_kernel(
             const int s = sl[k];
             st[k] = s >= 0 ? stb[s] : 0.0;
             mraw[k] = m0[k] = f4(0.f);
-            if (s >= 0 && qok) {
+            if (s >= 0) {
                 mraw[k] = reinterpret_cast<const float4*>(Mb + (size_t)s * d_v)[q];
                 m0[k] = reinterpret_cast<const float4*>(M0h + (size_t)s * d_v)[q];
             }
@@ -203,22 +206,18 @@ __global__ void __launch_bounds__(32) bwd_replay_kernel(
             raw[k] = f4_scale(fabsf(fk), signbit(fk) ? m0[k] : mraw[k]);  // the decayed row
             pp = f4_fma(wi[k], raw[k], pp);
         }
-        const float4 p = f4_sum_groups(pp);
+        const float4 p = f4_sum_rows(pp);
         const float4 dd = make_float4(bta * (vv.x - p.x), bta * (vv.y - p.y), bta * (vv.z - p.z),
                                       bta * (vv.w - p.w));
 #pragma unroll
         for (int k = 0; k < KPL; ++k) {
             const int s = sl[k];
             if (s < 0) continue;
-            const int i = g + 16 * k;
-            if (qok) {
-                reinterpret_cast<float4*>(P.log_rows + (bt * W + i) * (size_t)d_v)[q] = mraw[k];
-                reinterpret_cast<float4*>(Mb + (size_t)s * d_v)[q] = f4_fma(wi[k], dd, raw[k]);
-            }
-            if (h2 == 0) {
-                stb[s] = L;
-                if (lead) P.log_stamp[bt * W + i] = st[k];
-            }
+            const int i = g + 32 * k;
+            reinterpret_cast<float4*>(P.log_rows + (bt * W + i) * (size_t)d_v)[q] = mraw[k];
+            reinterpret_cast<float4*>(Mb + (size_t)s * d_v)[q] = f4_fma(wi[k], dd, raw[k]);
+            stb[s] = L;
+            if (lead) P.log_stamp[bt * W + i] = st[k];
         }
         if (lead && lane == 0) P.log_lam[bh * (size_t)(T + 1) + t + 1] = L;
         __syncwarp();  // this token's rows and stamps before the next token's loads
@@ -233,22 +232,27 @@ __global__ void __launch_bounds__(32) bwd_sweep_kernel(
     const int32_t* __restrict__ ridx, const float* __restrict__ rw, float* __restrict__ M,
     const float* __restrict__ M0, BwdPtrs P, const float* __restrict__ dout,
     float* __restrict__ dv_out, int H, int N, int T, int d_v, int W, int R, int S, int touched) {
-    __shared__ int s_rs[BWD_MAXO];
-    __shared__ float s_ru[BWD_MAXO];
     const int sc = (int)(blockIdx.x % S);
     const size_t bh = blockIdx.x / S, BH = gridDim.x / S;
     const size_t BHT = BH * (size_t)T;
     const int h = (int)(bh % H);
-    const int lane = threadIdx.x, h2 = lane & 1, g = lane >> 1;
-    const int Q = d_v / 4, q = BWD_SLICE_Q * sc + h2;
-    const bool qok = q < Q;
+    const int lane = threadIdx.x, g = lane;
+    const int q = sc;  // the slice's float4 column
     float* Mb = M + bh * (size_t)N * d_v;
     const float* M0h = M0 + (size_t)h * N * d_v;
     double* stb = P.pst + ((size_t)sc * BH + bh) * N;
     double* dsb = P.pds + ((size_t)sc * BH + bh) * N;
     float* dMb = P.dM + bh * (size_t)N * d_v;
     const double* lamb = P.log_lam + bh * (size_t)(T + 1);
-    double X = 0.0, Gam = 0.0;  // this lane's share of <dM, M>; backward log-decay prefix
+    // the token's read slots: key = token << 32 | slot (an entry of another token is free)
+    __shared__ unsigned long long h_key[BWD_HASH];
+    __shared__ float h_u[BWD_HASH];
+    for (int i = lane; i < BWD_HASH; i += 32) h_key[i] = ~0ull;
+    __syncwarp();
+    // this lane's share of <dM, M>; the backward log-decay prefix Gam = Lambda_T - Lambda_{t+1}
+    // before token t (sums of the same logs as the replay's prefix)
+    double X = 0.0;
+    const double LT = T > 0 ? lamb[T] : 0.0;
     // the next token's inputs
     int nrs[KPL], nws[KPL];
     float nu[KPL], nwi[KPL], na = 1.f, nb = 0.f;
@@ -259,22 +263,21 @@ __global__ void __launch_bounds__(32) bwd_sweep_kernel(
         nb = beta[bt];
 #pragma unroll
         for (int k = 0; k < KPL; ++k) {
-            const int j = g + 16 * k;
+            const int j = g + 32 * k;
             nrs[k] = j < R ? ridx[bt * R + j] : -1;
             nu[k] = j < R ? rw[bt * R + j] : 0.f;
             nws[k] = j < W ? widx[bt * W + j] : -1;
             nwi[k] = j < W ? ww[bt * W + j] : 0.f;
         }
-        if (qok) {
-            nG = reinterpret_cast<const float4*>(dout + bt * d_v)[q];
-            nv = bwd_load_v4<VT>(v + bt * d_v + 4 * q);
-        }
+        nG = reinterpret_cast<const float4*>(dout + bt * d_v)[q];
+        nv = bwd_load_v4<VT>(v + bt * d_v + 4 * q);
     };
     if (T > 0) fetch(T - 1);
     for (int t = T - 1; t >= 0; --t) {
         const size_t bt = bh * (size_t)T + t;
         const float a = na, bta = nb;
         const double Lt = lamb[t + 1], Lp = lamb[t];
+        const double Gam = touched ? 0.0 : LT - Lt;
         int rs[KPL], sl[KPL];
         float u[KPL], wi[KPL];
 #pragma unroll
@@ -285,35 +288,25 @@ __global__ void __launch_bounds__(32) bwd_sweep_kernel(
             wi[k] = nwi[k];
         }
         const float4 G = nG, vv = nv;
-        // this token's read slots, for the write rows that share one
-        if (h2 == 0)
-#pragma unroll
-            for (int k = 0; k < KPL; ++k) {
-                const int j = g + 16 * k;
-                if (j < R) {
-                    s_rs[j] = rs[k];
-                    s_ru[j] = u[k];
-                }
-            }
         // -- one round of loads: read rows (stamps, M, M0, dM), write rows (log, stamps,
         //    current row, M0, dM)
         double rst[KPL], rds[KPL], wso[KPL], wsn[KPL], wds[KPL];
         float4 rM[KPL], rM0[KPL], rG[KPL], lrow[KPL], mc[KPL], m0[KPL], wdm[KPL];
 #pragma unroll
         for (int k = 0; k < KPL; ++k) {
-            const int s = rs[k], sw = sl[k], i = g + 16 * k;
+            const int s = rs[k], sw = sl[k], i = g + 32 * k;
             rst[k] = s >= 0 ? stb[s] : 0.0;
             rds[k] = s >= 0 ? dsb[s] : 0.0;
             wso[k] = sw >= 0 ? P.log_stamp[bt * W + i] : 0.0;
             wsn[k] = sw >= 0 ? stb[sw] : 0.0;
             wds[k] = sw >= 0 ? dsb[sw] : 0.0;
             rM[k] = rM0[k] = rG[k] = lrow[k] = mc[k] = m0[k] = wdm[k] = f4(0.f);
-            if (qok && s >= 0) {
+            if (s >= 0) {
                 rM[k] = reinterpret_cast<const float4*>(Mb + (size_t)s * d_v)[q];
                 rM0[k] = reinterpret_cast<const float4*>(M0h + (size_t)s * d_v)[q];
                 rG[k] = reinterpret_cast<const float4*>(dMb + (size_t)s * d_v)[q];
             }
-            if (qok && sw >= 0) {
+            if (sw >= 0) {
                 lrow[k] = reinterpret_cast<const float4*>(P.log_rows + (bt * W + i) * (size_t)d_v)[q];
                 mc[k] = reinterpret_cast<const float4*>(Mb + (size_t)sw * d_v)[q];
                 m0[k] = reinterpret_cast<const float4*>(M0h + (size_t)sw * d_v)[q];
@@ -325,22 +318,51 @@ __global__ void __launch_bounds__(32) bwd_sweep_kernel(
         double xr = 0.0;
 #pragma unroll
         for (int k = 0; k < KPL; ++k) {
-            const int s = rs[k], j = g + 16 * k;
+            const int s = rs[k], j = g + 32 * k;
             const float f = bwd_factor(rst[k], Lt, touched);
             const float4 rm = f4_scale(fabsf(f), signbit(f) ? rM0[k] : rM[k]);
             const float gf = (s < 0 || isnan(rds[k])) ? 0.f : bwd_exp(Gam - rds[k]);
-            const float part = s >= 0 ? f4_dot(G, rm) : 0.f;
-            const float du = pair_sum(part);
-            if (h2 == 0 && j < R) P.p_drw[((size_t)sc * BHT + bt) * R + j] = du;
-            xr += (double)u[k] * part;
+            const float du = s >= 0 ? f4_dot(G, rm) : 0.f;
+            if (j < R) P.p_drw[((size_t)sc * BHT + bt) * R + j] = du;
+            xr += (double)u[k] * du;
             if (s >= 0) {
-                if (qok)
-                    reinterpret_cast<float4*>(dMb + (size_t)s * d_v)[q] =
-                        f4_fma(u[k], G, gf != 0.f ? f4_scale(gf, rG[k]) : f4(0.f));
-                if (h2 == 0) dsb[s] = Gam;
+                reinterpret_cast<float4*>(dMb + (size_t)s * d_v)[q] =
+                    f4_fma(u[k], G, gf != 0.f ? f4_scale(gf, rG[k]) : f4(0.f));
+                dsb[s] = Gam;
+                // list the read slot (entries of earlier tokens count as free)
+                const unsigned long long key =
+                    ((unsigned long long)(unsigned)t << 32) | (unsigned)s;
+                unsigned hpos = bwd_hash(s);
+                for (int probe = 0; probe < 2 * BWD_HASH; ++probe) {
+                    const unsigned long long old = h_key[hpos];
+                    if ((unsigned)(old >> 32) == (unsigned)t) {
+                        hpos = (hpos + 1) & (BWD_HASH - 1);
+                    } else if (atomicCAS(&h_key[hpos], old, key) == old) {
+                        h_u[hpos] = u[k];
+                        break;
+                    }
+                }
             }
         }
-        __syncwarp();  // read slots listed; read rows' gradient stored before the write rows'
+        __syncwarp();  // the read rows' gradient stores before the write rows' (same slot)
+        // a write slot that is also read in this token takes the read's weight (its update of
+        // the gradient row comes first); the read slots are distinct, so at most one matches
+        float hu[KPL];
+#pragma unroll
+        for (int k = 0; k < KPL; ++k) {
+            hu[k] = 0.f;
+            if (sl[k] < 0) continue;
+            unsigned hpos = bwd_hash(sl[k]);
+            for (int probe = 0; probe < BWD_HASH; ++probe) {
+                const unsigned long long e = h_key[hpos];
+                if ((unsigned)(e >> 32) != (unsigned)t) break;  // free: not read
+                if ((int)(unsigned)e == sl[k]) {
+                    hu[k] = h_u[hpos];
+                    break;
+                }
+                hpos = (hpos + 1) & (BWD_HASH - 1);
+            }
+        }
         // -- write rows
         float4 mp[KPL], mt[KPL], dm[KPL], pp = f4(0.f), pd = f4(0.f);
 #pragma unroll
@@ -353,42 +375,33 @@ __global__ void __launch_bounds__(32) bwd_sweep_kernel(
             const float gf = (s < 0 || isnan(wds[k])) ? 0.f : bwd_exp(Gam - wds[k]);
             // a row never reached holds stale workspace: select zero, never scale it
             dm[k] = gf != 0.f ? f4_scale(gf, wdm[k]) : f4(0.f);
-            if (s >= 0)
-                for (int j = 0; j < R; ++j)
-                    if (s_rs[j] == s) {  // read in this token too: its update comes first
-                        dm[k] = f4_fma(s_ru[j], G, dm[k]);
-                        break;
-                    }
+            dm[k] = f4_fma(hu[k], G, dm[k]);
             if (s < 0) mp[k] = mt[k] = dm[k] = f4(0.f);
             pp = f4_fma(wi[k] * a, mp[k], pp);
             pd = f4_fma(wi[k], dm[k], pd);
         }
-        pp = f4_sum_groups(pp);
-        pd = f4_sum_groups(pd);
+        pp = f4_sum_rows(pp);
+        pd = f4_sum_rows(pd);
         const float4 e = make_float4(vv.x - pp.x, vv.y - pp.y, vv.z - pp.z, vv.w - pp.w);
         const float4 de = f4_scale(bta, pd);
-        if (g == 0 && qok) reinterpret_cast<float4*>(dv_out + bt * d_v)[q] = de;
+        if (lane == 0) reinterpret_cast<float4*>(dv_out + bt * d_v)[q] = de;
         double sb = 0.0, s1 = 0.0, s2 = 0.0;  // shares of dbeta, <dM, M_t>, <dMt, M_{t-1}>
         const float scw = touched ? a : 1.f;  // every-slot decay keeps alpha in Gam
 #pragma unroll
         for (int k = 0; k < KPL; ++k) {
-            const int s = sl[k], i = g + 16 * k;
+            const int s = sl[k], i = g + 32 * k;
             const float ge = f4_dot(dm[k], e), gm = f4_dot(de, mp[k]);
             const float4 nd = f4_fma(-wi[k], de, dm[k]);  // dMt[s_i]
-            const float dw = bta * pair_sum(ge) - a * pair_sum(gm);
-            if (h2 == 0 && i < W) P.p_dww[((size_t)sc * BHT + bt) * W + i] = s >= 0 ? dw : 0.f;
+            const float dw = bta * ge - a * gm;
+            if (i < W) P.p_dww[((size_t)sc * BHT + bt) * W + i] = s >= 0 ? dw : 0.f;
             if (s < 0) continue;
             sb += (double)wi[k] * ge;
             s1 += f4_dot(dm[k], mt[k]);
             s2 += f4_dot(nd, mp[k]);
-            if (qok) {
-                reinterpret_cast<float4*>(dMb + (size_t)s * d_v)[q] = f4_scale(scw, nd);
-                reinterpret_cast<float4*>(Mb + (size_t)s * d_v)[q] = lrow[k];  // restore
-            }
-            if (h2 == 0) {
-                dsb[s] = Gam;
-                stb[s] = wso[k];
-            }
+            reinterpret_cast<float4*>(dMb + (size_t)s * d_v)[q] = f4_scale(scw, nd);
+            reinterpret_cast<float4*>(Mb + (size_t)s * d_v)[q] = lrow[k];  // restore
+            dsb[s] = Gam;
+            stb[s] = wso[k];
         }
         double da;
         if (touched) {
@@ -397,7 +410,6 @@ __global__ void __launch_bounds__(32) bwd_sweep_kernel(
             X += xr;
             da = (X - s1) / (double)a + s2;
             X = (double)a * da;
-            Gam += log((double)a);
         }
         da = warp_sum_d(da);
         sb = warp_sum_d(sb);
@@ -405,9 +417,9 @@ __global__ void __launch_bounds__(32) bwd_sweep_kernel(
             P.p_da[(size_t)sc * BHT + bt] = da;
             P.p_db[(size_t)sc * BHT + bt] = sb;
         }
-        __syncwarp();  // this token's stores and list reads before the next token's
+        __syncwarp();  // this token's stores before the next token's loads
     }
-    if (sc == 0 && lane == 0) P.gam[bh] = Gam;
+    if (sc == 0 && lane == 0) P.gam[bh] = touched || T == 0 ? 0.0 : LT - lamb[0];
 }
 
 // The per-slice shares summed in slice order: dww, drw, dbeta, dalpha.

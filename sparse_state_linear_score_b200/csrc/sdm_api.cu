@@ -344,7 +344,7 @@ sdm_status score_both_roles(const sdm_dims* d, const void* q, const void* k, con
     return launch_score(d, q, skr, d->R, ridx, rw, s);
 }
 
-// column slices per (b,h) in the backward (8 columns each)
+// column slices per (b,h) in the backward (4 columns each)
 int bwd_slices(const sdm_dims* d) { return (d->d_v / 4 + BWD_SLICE_Q - 1) / BWD_SLICE_Q; }
 
 struct BwdLayout {
@@ -793,11 +793,10 @@ sdm_status sdm_backward(const sdm_dims* dims, const void* v, const float* alpha,
         const int m = dims->W > dims->R ? dims->W : dims->R;
 #define SDM_BWD(VT, K) launch_backward_t<VT, K>(dims, P, v, alpha, beta, widx, ww, ridx, rw, st, dout, dv, s)
         if (dims->v_dtype == SDM_BF16) {
-            e = m <= 16 ? SDM_BWD(__nv_bfloat16, 1) : m <= 32 ? SDM_BWD(__nv_bfloat16, 2)
-              : m <= 64 ? SDM_BWD(__nv_bfloat16, 4) : SDM_BWD(__nv_bfloat16, 8);
+            e = m <= 32 ? SDM_BWD(__nv_bfloat16, 1) : m <= 64 ? SDM_BWD(__nv_bfloat16, 2)
+                                                    : SDM_BWD(__nv_bfloat16, 4);
         } else {
-            e = m <= 16 ? SDM_BWD(float, 1) : m <= 32 ? SDM_BWD(float, 2)
-              : m <= 64 ? SDM_BWD(float, 4) : SDM_BWD(float, 8);
+            e = m <= 32 ? SDM_BWD(float, 1) : m <= 64 ? SDM_BWD(float, 2) : SDM_BWD(float, 4);
         }
 #undef SDM_BWD
         if (e) return e;
