@@ -36,8 +36,9 @@
 //
 // Lane layout in a slice: lane l owns write rows l, l+32, ... and read rows l, l+32, ...
 // (the slice's float4 of each).  A token's loads (stamps, rows, log) all go out in one
-// round; a slot both read and written in the token takes the read's gradient update,
-// found through a small shared-memory hash of the token's read slots.
+// round; a slot both read and written in the token takes the read's gradient update: which
+// read shares each write row's slot does not depend on the column, so bwd_links_kernel
+// finds it once per call for all slices.
 #pragma once
 
 #include <math.h>
@@ -48,7 +49,6 @@ namespace sdm {
 
 constexpr int BWD_MAXO = 128;      // W + R
 constexpr int BWD_SLICE_Q = 1;     // float4 columns per slice
-constexpr int BWD_HASH = 256;      // read-slot hash entries (> BWD_MAXO)
 
 // Per-(b,h) records of one call (a byte layout in the workspace); S = slices per (b,h).
 struct BwdPtrs {
@@ -63,6 +63,7 @@ struct BwdPtrs {
     double* p_db;        // [S][BH*T]       of dbeta
     double* p_da;        // [S][BH*T]       of dalpha
     double* gam;         // [BH]            the final backward prefix
+    int8_t* rpart;       // [BH*T][W]       the read of the same token with the write's slot, or -1
 };
 
 SDM_DEV float4 f4(float a) { return make_float4(a, a, a, a); }
@@ -94,7 +95,6 @@ SDM_DEV double warp_sum_d(double x) {
     for (int m = 16; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
     return x;
 }
-SDM_DEV unsigned bwd_hash(int s) { return ((unsigned)s * 0x9E3779B1u) >> 24; }
 
 template <typename VT>
 SDM_DEV float4 bwd_load_v4(const VT* p);
@@ -131,6 +131,25 @@ __global__ void bwd_init_kernel(const double* __restrict__ stamp, BwdPtrs P, siz
         P.pds[i] = __longlong_as_double(0x7ff8000000000000ll);
     }
     for (size_t i = i0; i < (size_t)BH; i += stride) P.gam[i] = 0.0;
+}
+
+// For every write row, the read row of the same token that has its slot (reads are
+// distinct within a token), or -1.  One thread per (token, write row).
+__global__ void bwd_links_kernel(const int32_t* __restrict__ widx,
+                                 const int32_t* __restrict__ ridx, size_t BHT, int W, int R,
+                                 int8_t* __restrict__ rpart) {
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < BHT * W; e += stride) {
+        const size_t bt = e / W;
+        const int s = widx[e];
+        int j0 = -1;
+        for (int j = 0; j < R; ++j)
+            if (ridx[bt * R + j] == s) {
+                j0 = j;
+                break;
+            }
+        rpart[e] = (int8_t)j0;
+    }
 }
 
 // ---- replay with the log --------------------------------------------------------------
@@ -244,22 +263,19 @@ __global__ void __launch_bounds__(32) bwd_sweep_kernel(
     double* dsb = P.pds + ((size_t)sc * BH + bh) * N;
     float* dMb = P.dM + bh * (size_t)N * d_v;
     const double* lamb = P.log_lam + bh * (size_t)(T + 1);
-    // the token's read slots: key = token << 32 | slot (an entry of another token is free)
-    __shared__ unsigned long long h_key[BWD_HASH];
-    __shared__ float h_u[BWD_HASH];
-    for (int i = lane; i < BWD_HASH; i += 32) h_key[i] = ~0ull;
-    __syncwarp();
     // this lane's share of <dM, M>; the backward log-decay prefix Gam = Lambda_T - Lambda_{t+1}
     // before token t (sums of the same logs as the replay's prefix)
     double X = 0.0;
     const double LT = T > 0 ? lamb[T] : 0.0;
     // the next token's inputs
-    int nrs[KPL], nws[KPL];
+    int nrs[KPL], nws[KPL], npj[KPL];
     float nu[KPL], nwi[KPL], na = 1.f, nb = 0.f;
+    double nia = 1.0;  // 1 / alpha
     float4 nG = f4(0.f), nv = f4(0.f);
     auto fetch = [&](int t) {
         const size_t bt = bh * (size_t)T + t;
         na = alpha[bt] > 0.f ? alpha[bt] : 1.f;
+        nia = 1.0 / (double)na;
         nb = beta[bt];
 #pragma unroll
         for (int k = 0; k < KPL; ++k) {
@@ -268,6 +284,7 @@ __global__ void __launch_bounds__(32) bwd_sweep_kernel(
             nu[k] = j < R ? rw[bt * R + j] : 0.f;
             nws[k] = j < W ? widx[bt * W + j] : -1;
             nwi[k] = j < W ? ww[bt * W + j] : 0.f;
+            npj[k] = j < W ? (int)P.rpart[bt * W + j] : -1;
         }
         nG = reinterpret_cast<const float4*>(dout + bt * d_v)[q];
         nv = bwd_load_v4<VT>(v + bt * d_v + 4 * q);
@@ -276,9 +293,10 @@ __global__ void __launch_bounds__(32) bwd_sweep_kernel(
     for (int t = T - 1; t >= 0; --t) {
         const size_t bt = bh * (size_t)T + t;
         const float a = na, bta = nb;
+        const double ia = nia;
         const double Lt = lamb[t + 1], Lp = lamb[t];
         const double Gam = touched ? 0.0 : LT - Lt;
-        int rs[KPL], sl[KPL];
+        int rs[KPL], sl[KPL], pj[KPL];
         float u[KPL], wi[KPL];
 #pragma unroll
         for (int k = 0; k < KPL; ++k) {
@@ -286,6 +304,7 @@ __global__ void __launch_bounds__(32) bwd_sweep_kernel(
             u[k] = nu[k];
             sl[k] = slot_ok(nws[k], N) ? nws[k] : -1;
             wi[k] = nwi[k];
+            pj[k] = npj[k];
         }
         const float4 G = nG, vv = nv;
         // -- one round of loads: read rows (stamps, M, M0, dM), write rows (log, stamps,
@@ -329,38 +348,19 @@ __global__ void __launch_bounds__(32) bwd_sweep_kernel(
                 reinterpret_cast<float4*>(dMb + (size_t)s * d_v)[q] =
                     f4_fma(u[k], G, gf != 0.f ? f4_scale(gf, rG[k]) : f4(0.f));
                 dsb[s] = Gam;
-                // list the read slot (entries of earlier tokens count as free)
-                const unsigned long long key =
-                    ((unsigned long long)(unsigned)t << 32) | (unsigned)s;
-                unsigned hpos = bwd_hash(s);
-                for (int probe = 0; probe < 2 * BWD_HASH; ++probe) {
-                    const unsigned long long old = h_key[hpos];
-                    if ((unsigned)(old >> 32) == (unsigned)t) {
-                        hpos = (hpos + 1) & (BWD_HASH - 1);
-                    } else if (atomicCAS(&h_key[hpos], old, key) == old) {
-                        h_u[hpos] = u[k];
-                        break;
-                    }
-                }
             }
         }
         __syncwarp();  // the read rows' gradient stores before the write rows' (same slot)
-        // a write slot that is also read in this token takes the read's weight (its update of
-        // the gradient row comes first); the read slots are distinct, so at most one matches
+        // a write slot that is also read in this token takes that read's weight (its update of
+        // the gradient row comes first); read j sits in lane j % 32, row j / 32
         float hu[KPL];
 #pragma unroll
         for (int k = 0; k < KPL; ++k) {
             hu[k] = 0.f;
-            if (sl[k] < 0) continue;
-            unsigned hpos = bwd_hash(sl[k]);
-            for (int probe = 0; probe < BWD_HASH; ++probe) {
-                const unsigned long long e = h_key[hpos];
-                if ((unsigned)(e >> 32) != (unsigned)t) break;  // free: not read
-                if ((int)(unsigned)e == sl[k]) {
-                    hu[k] = h_u[hpos];
-                    break;
-                }
-                hpos = (hpos + 1) & (BWD_HASH - 1);
+#pragma unroll
+            for (int k2 = 0; k2 < KPL; ++k2) {
+                const float u2 = __shfl_sync(0xffffffffu, u[k2], pj[k] & 31);
+                if (pj[k] >= 0 && (pj[k] >> 5) == k2) hu[k] = u2;
             }
         }
         // -- write rows
@@ -408,7 +408,7 @@ __global__ void __launch_bounds__(32) bwd_sweep_kernel(
             da = s2;
         } else {
             X += xr;
-            da = (X - s1) / (double)a + s2;
+            da = (X - s1) * ia + s2;
             X = (double)a * da;
         }
         da = warp_sum_d(da);

@@ -349,7 +349,7 @@ int bwd_slices(const sdm_dims* d) { return (d->d_v / 4 + BWD_SLICE_Q - 1) / BWD_
 
 struct BwdLayout {
     size_t off_rows, off_lstamp, off_lam, off_dM, off_pst, off_pds, off_pdww, off_pdrw, off_pdb,
-        off_pda, off_gam, total;
+        off_pda, off_gam, off_rpart, total;
 };
 
 BwdLayout bwd_layout(const sdm_dims* d) {
@@ -368,6 +368,7 @@ BwdLayout bwd_layout(const sdm_dims* d) {
     L.off_pdb = o;    o = up256(o + S * BH * T * 8);
     L.off_pda = o;    o = up256(o + S * BH * T * 8);
     L.off_gam = o;    o = up256(o + BH * 8);
+    L.off_rpart = o;  o = up256(o + BH * T * (size_t)d->W);
     L.total = o;
     return L;
 }
@@ -780,6 +781,7 @@ sdm_status sdm_backward(const sdm_dims* dims, const void* v, const float* alpha,
     P.p_db = reinterpret_cast<double*>(b + L.off_pdb);
     P.p_da = reinterpret_cast<double*>(b + L.off_pda);
     P.gam = reinterpret_cast<double*>(b + L.off_gam);
+    P.rpart = reinterpret_cast<int8_t*>(b + L.off_rpart);
     const int threads = 256;
     auto grid_for = [](size_t n) {
         size_t blocks = (n + 255) / 256;
@@ -790,6 +792,9 @@ sdm_status sdm_backward(const sdm_dims* dims, const void* v, const float* alpha,
     bwd_init_kernel<<<grid_for((size_t)S * rows), threads, 0, s>>>(st->stamp, P, rows, S,
                                                                    (int)BH_of(dims));
     if (dims->T > 0) {
+        const size_t BHT = (size_t)BH_of(dims) * dims->T;
+        bwd_links_kernel<<<grid_for(BHT * dims->W), threads, 0, s>>>(widx, ridx, BHT, dims->W,
+                                                                     dims->R, P.rpart);
         const int m = dims->W > dims->R ? dims->W : dims->R;
 #define SDM_BWD(VT, K) launch_backward_t<VT, K>(dims, P, v, alpha, beta, widx, ww, ridx, rw, st, dout, dv, s)
         if (dims->v_dtype == SDM_BF16) {
@@ -800,7 +805,6 @@ sdm_status sdm_backward(const sdm_dims* dims, const void* v, const float* alpha,
         }
 #undef SDM_BWD
         if (e) return e;
-        const size_t BHT = (size_t)BH_of(dims) * dims->T;
         bwd_reduce_kernel<<<grid_for(BHT * (dims->W + dims->R + 2)), threads, 0, s>>>(
             P, S, BHT, dims->W, dims->R, dww, drw, dbeta, dalpha);
     }
