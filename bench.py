@@ -587,7 +587,7 @@ def run_backward(wl, inp, sel, device, sdm, reps: int = 2) -> dict:
            "scoring_backward_ms": ms_score,
            "roofline": {"bound": "hbm", "algorithmic_bytes": total, "achieved_gbs": gbs,
                         "peak": peak, "frac": gbs / peak},
-           "note": "first version: one CTA per (b,h) walks the tokens one at a time",
+           "note": "tokens one at a time per sequence, one warp per 4-column slice of d_v",
            "device_errors": errs}
     del st, ws, grads, dout
     torch.cuda.empty_cache()

@@ -246,7 +246,9 @@ sdm_status sdm_decode_step(const sdm_dims* dims, const void* q, const void* k, c
  *         the start; for a fresh state, summing it over b gives the gradient of M0)
  *   ws    device workspace of at least sdm_backward_workspace_bytes(dims) bytes, 16-byte
  *         aligned.
- * This first version walks the tokens of each sequence one at a time (one CTA per (b,h)).
+ * Each sequence's tokens are walked one at a time, split over 4-column slices of d_v (one warp
+ * per slice); the workspace holds the write log, private stamp copies per slice and
+ * per-slice shares of the column sums.
  * Errors: as sdm_forward; W + R <= 128; the slots must be in range and distinct within a
  * token.
  */
