@@ -118,3 +118,34 @@ def test_forward_rejects_small_workspace(lib):
     st_bad = State(0x1000, 0x2000, 0x3003, 0x4000)
     assert lib.sdm_forward(ctypes.byref(d), p, p, p, p, p, p, p, ctypes.byref(st_bad), p, p,
                            ctypes.c_size_t(1 << 40), None) == 4
+
+
+def test_backward_host_checks(lib):
+    """sdm_backward's workspace query covers the write log, the memory gradient and one
+    private stamp copy pair per 4-column slice; bad arguments are refused on the host."""
+    class State(ctypes.Structure):
+        _fields_ = [("M", ctypes.c_void_p), ("stamp", ctypes.c_void_p), ("Lambda", ctypes.c_void_p),
+                    ("M0", ctypes.c_void_p)]
+    lib.sdm_backward_workspace_bytes.restype = ctypes.c_size_t
+    d = mid_dims()
+    ws = lib.sdm_backward_workspace_bytes(ctypes.byref(d))
+    BH, T, N, W, dv = 2 * 4, 4096, 65536, 32, 128
+    log_rows, dM = BH * T * W * dv * 4, BH * N * dv * 4
+    stamps = 2 * (dv // 4) * BH * N * 8
+    assert ws >= log_rows + dM + stamps
+    assert lib.sdm_backward_workspace_bytes(ctypes.byref(mid_dims(W=65))) == 0
+    # twice the columns: twice the slices' stamp copies
+    ws2 = lib.sdm_backward_workspace_bytes(ctypes.byref(mid_dims(d_v=256)))
+    assert ws2 - ws >= log_rows + dM + stamps
+    p = ctypes.c_void_p(0x1000)
+    st = State(0x1000, 0x2000, 0x3000, 0x4000)
+    big = ctypes.c_size_t(1 << 44)
+
+    def call(v=p, dout=p, ws_ptr=p, ws_bytes=big, dims=d):
+        return lib.sdm_backward(ctypes.byref(dims), v, p, p, p, p, p, p, ctypes.byref(st), dout,
+                                p, p, p, p, p, p, ws_ptr, ws_bytes, None)
+    assert call(v=None) == 1                                  # SDM_ERR_ARG
+    assert call(dout=ctypes.c_void_p(0x1008)) == 4            # SDM_ERR_ALIGN
+    assert call(ws_bytes=ctypes.c_size_t(ws - 1)) == 7        # SDM_ERR_WORKSPACE
+    assert call(ws_ptr=None) == 7
+    assert call(dims=mid_dims(d_k=30)) == 2                   # SDM_ERR_SHAPE
