@@ -18,8 +18,9 @@ Parity status per function:
                                  dense Gated DeltaNet matrix form, hand example)
   recur_lazy .................. pinned (agrees with recur_dense to 1e-12)
   recur_backward .............. pinned (central finite differences of recur_dense and
-                                 recur_touched for every input, beta = 0 and alpha = 1
-                                 closed form)
+                                 recur_touched for every input, with and without a gradient
+                                 of the final memory; beta = 0 and alpha = 1 closed form;
+                                 beta = 0 decay closed form of that gradient)
   score_backward .............. pinned (central finite differences of the softmax of the
                                  selected slots' half-score sums, for x and the tables)
   recur_touched ............... pinned (hand example, alpha = 1 equals recur_dense,
@@ -101,7 +102,7 @@ class Oracle:
         lib.sdm_oracle_recur_dense.restype = I
         lib.sdm_oracle_recur_touched.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P]
         lib.sdm_oracle_recur_touched.restype = I
-        lib.sdm_oracle_recur_backward.argtypes = [I, I, I, I, I, I] + [P] * 15
+        lib.sdm_oracle_recur_backward.argtypes = [I, I, I, I, I, I] + [P] * 16
         lib.sdm_oracle_recur_backward.restype = I
         lib.sdm_oracle_score_backward.argtypes = [P, P, I, I, I, I, P, P, P, P]
         lib.sdm_oracle_score_backward.restype = I
@@ -267,9 +268,11 @@ class Oracle:
             dsk[h] = dskh
         return dx, dsk
 
-    def recur_backward(self, v, alpha, beta, widx, ww, ridx, rw, M0, dout, touched=False):
+    def recur_backward(self, v, alpha, beta, widx, ww, ridx, rw, M0, dout, touched=False,
+                       dM_end=None):
         """Gradients of one (b,h)'s recurrence for output gradient dout [T,dv] (selections
-        fixed).  Returns dict dv [T,dv], dalpha [T], dbeta [T], dww [T,W], drw [T,R],
+        fixed) and, optionally, gradient dM_end [N,dv] with respect to the memory after the
+        last token.  Returns dict dv [T,dv], dalpha [T], dbeta [T], dww [T,W], drw [T,R],
         dM0 [N,dv] (with respect to the state at the start)."""
         v, alpha, beta = _f64(v), _f64(alpha), _f64(beta)
         widx, ridx, ww, rw = _i32(widx), _i32(ridx), _f64(ww), _f64(rw)
@@ -281,7 +284,8 @@ class Oracle:
              "dww": np.empty((T, W)), "drw": np.empty((T, R)), "dM0": np.empty((N, dv))}
         _check(self.lib.sdm_oracle_recur_backward(
             T, N, dv, W, R, 1 if touched else 0, _p(v), _p(alpha), _p(beta), _p(widx), _p(ww),
-            _p(ridx), _p(rw), _p(M0), _p(dout), _p(g["dv"]), _p(g["dalpha"]), _p(g["dbeta"]),
+            _p(ridx), _p(rw), _p(M0), _p(dout), None if dM_end is None else _p(_f64(dM_end)),
+            _p(g["dv"]), _p(g["dalpha"]), _p(g["dbeta"]),
             _p(g["dww"]), _p(g["drw"]), _p(g["dM0"])), "recur_backward")
         return g
 

@@ -353,15 +353,19 @@ int sdm_oracle_recur_touched(int T, int N, int dv, int W, int R, const double* v
  *   (ii)  p = sum_i w_i Mt[s_i]:           dw_i += <dp, Mt[s_i]>,  dMt[s_i] = dM[s_i] + w_i dp
  *   (i)   Mt = alpha M_{t-1}:              dalpha = <dMt, M_{t-1}> over every slot (the
  *         write slots only when touched),   dM_{t-1} = alpha dMt (those slots only)
- * G = dout[t].  Outputs: dv [T][dv], dalpha [T], dbeta [T], dww [T][W], drw [T][R] and dM0
- * [N][dv], the gradient with respect to the state at the start of the call.
+ * G = dout[t].  dM_end [N][dv] (may be NULL: zero) is the loss's gradient with respect to
+ * the memory after the last token, for a loss that also reads the final state (a sequence
+ * processed in several calls: the next call's gradient of its start state); the sweep
+ * starts from it.  Outputs: dv [T][dv], dalpha [T], dbeta [T], dww [T][W], drw [T][R] and
+ * dM0 [N][dv], the gradient with respect to the state at the start of the call.
  * §2 Background "Gated DeltaNet"; §3 Method "Sparse memory updates", "Sparse retrieval".
  */
 int sdm_oracle_recur_backward(int T, int N, int dv, int W, int R, int touched, const double* v,
                               const double* alpha, const double* beta, const int32_t* widx,
                               const double* ww, const int32_t* ridx, const double* rw,
-                              const double* M0, const double* dout, double* dvv, double* dalpha,
-                              double* dbeta, double* dww, double* drw, double* dM0) {
+                              const double* M0, const double* dout, const double* dM_end,
+                              double* dvv, double* dalpha, double* dbeta, double* dww,
+                              double* drw, double* dM0) {
     if (T < 0 || N <= 0 || dv <= 0 || W <= 0 || R <= 0) return ORACLE_ERR_ARG;
     const size_t ND = (size_t)N * dv;
     double* S = (double*)malloc(sizeof(double) * ND * (size_t)(T + 1));  /* S[t] = M_t */
@@ -376,6 +380,7 @@ int sdm_oracle_recur_backward(int T, int N, int dv, int W, int R, int touched, c
     }
     int rc = ORACLE_OK;
     memcpy(S, M0, sizeof(double) * ND);
+    if (dM_end) memcpy(dM, dM_end, sizeof(double) * ND);
     for (int t = 0; t < T && rc == ORACLE_OK; ++t) {
         const int32_t* ws = widx + (size_t)t * W;
         const int32_t* rs = ridx + (size_t)t * R;

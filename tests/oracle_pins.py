@@ -395,17 +395,19 @@ def _fd_case(rng, T, N, dv, W, R):
     return v, alpha, beta, widx, ww, ridx, rw, M0, dout
 
 
-def _check_fd(o, touched, case):
-    """Central differences of L = sum(dout * out) through the forward oracle, every input."""
+def _check_fd(o, touched, case, G_end=None):
+    """Central differences of L = sum(dout * out) (+ sum(G_end * M_T), the final memory)
+    through the forward oracle, every input."""
     v, alpha, beta, widx, ww, ridx, rw, M0, dout = case
     fwd = o.recur_touched if touched else o.recur_dense
-    g = o.recur_backward(v, alpha, beta, widx, ww, ridx, rw, M0, dout, touched=touched)
+    g = o.recur_backward(v, alpha, beta, widx, ww, ridx, rw, M0, dout, touched=touched,
+                         dM_end=G_end)
 
     def loss(**kw):
         a = dict(v=v, alpha=alpha, beta=beta, ww=ww, rw=rw, M0=M0)
         a.update(kw)
-        out, _ = fwd(a["v"], a["alpha"], a["beta"], widx, a["ww"], ridx, a["rw"], a["M0"])
-        return float((dout * out).sum())
+        out, MT = fwd(a["v"], a["alpha"], a["beta"], widx, a["ww"], ridx, a["rw"], a["M0"])
+        return float((dout * out).sum()) + (0.0 if G_end is None else float((G_end * MT).sum()))
 
     h = 1e-6
     for name, arr, key in (("v", v, "dv"), ("alpha", alpha, "dalpha"), ("beta", beta, "dbeta"),
@@ -431,6 +433,30 @@ def pin_backward_touched_finite_differences(o):
     rng = _rng(17)
     _check_fd(o, True, _fd_case(rng, 7, 6, 3, 2, 3))
     _check_fd(o, True, _fd_case(rng, 6, 9, 2, 3, 2))
+
+
+def pin_backward_end_gradient(o):
+    """A gradient for the memory after the last token (a loss that also reads the final
+    state): central differences of L = sum(dout * out) + sum(G * M_T) for both decay rules;
+    with no token it passes through unchanged; with beta = 0 and no output gradient, every
+    slot decays, so M_T = M0 prod(alpha): dM0 = prod(alpha) G and
+    dalpha_t = <G, M0> prod over the other tokens of alpha."""
+    rng = _rng(20)
+    for touched in (False, True):
+        case = _fd_case(rng, 6, 5, 3, 2, 2)
+        _check_fd(o, touched, case, G_end=rng.standard_normal((5, 3)))
+    T, N, dv, W, R = 5, 6, 2, 2, 2
+    v, alpha, beta, widx, ww, ridx, rw, M0, dout = _fd_case(rng, T, N, dv, W, R)
+    G = rng.standard_normal((N, dv))
+    g0 = o.recur_backward(v[:0], alpha[:0], beta[:0], widx[:0], ww[:0], ridx[:0], rw[:0], M0,
+                          dout[:0], dM_end=G)
+    assert np.array_equal(g0["dM0"], G)
+    g = o.recur_backward(v, alpha, np.zeros(T), widx, ww, ridx, rw, M0, np.zeros((T, dv)),
+                         dM_end=G)
+    P = float(np.prod(alpha))
+    np.testing.assert_allclose(g["dM0"], P * G, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(g["dalpha"], float((G * M0).sum()) * P / alpha, rtol=1e-12)
+    assert np.array_equal(g["drw"], np.zeros((T, R)))
 
 
 def pin_backward_frozen_memory(o):
@@ -680,4 +706,4 @@ ALL_PINS = [pin_pk_equals_brute, pin_brute_matches_numpy, pin_pk_depends_on_k, p
             pin_layer_in_routing_and_gates, pin_layer_in_linear, pin_touched_hand,
             pin_touched_alpha_one, pin_touched_all_slots_gdn, pin_touched_beta_zero,
             pin_backward_finite_differences, pin_backward_touched_finite_differences,
-            pin_backward_frozen_memory, pin_score_backward_finite_differences]
+            pin_backward_frozen_memory, pin_backward_end_gradient, pin_score_backward_finite_differences]
