@@ -240,6 +240,9 @@ sdm_status sdm_decode_step(const sdm_dims* dims, const void* q, const void* k, c
  *         slots from the log: on return the state is again the start state (the memory is
  *         never copied; peak memory O(N*d_v + T*W*d_v) per sequence).
  *   dout  [B][H][T][d_v] fp32 gradient of the loss with respect to out
+ *   dM_end [B][H][N][d_v] fp32 gradient of the loss with respect to the true slot values
+ *         after the last token (a loss that also reads the final memory, e.g. the next
+ *         call's dM_in when a sequence is processed in several calls), or NULL for zero
  *   outputs, fp32, caller-allocated, every element written:
  *         dv [B][H][T][d_v], dalpha [B][H][T], dbeta [B][H][T], dww [B][H][T][W],
  *         drw [B][H][T][R], dM_in [B][H][N][d_v] (with respect to the true slot values at
@@ -271,9 +274,9 @@ sdm_status sdm_score_backward(const sdm_dims* dims, const void* x, const void* s
 size_t sdm_backward_workspace_bytes(const sdm_dims* dims);
 sdm_status sdm_backward(const sdm_dims* dims, const void* v, const float* alpha, const float* beta,
                         const int32_t* widx, const float* ww, const int32_t* ridx, const float* rw,
-                        const sdm_state* st, const float* dout, float* dv, float* dalpha,
-                        float* dbeta, float* dww, float* drw, float* dM_in, void* ws,
-                        size_t ws_bytes, sdm_stream_t stream);
+                        const sdm_state* st, const float* dout, const float* dM_end, float* dv,
+                        float* dalpha, float* dbeta, float* dww, float* drw, float* dM_in,
+                        void* ws, size_t ws_bytes, sdm_stream_t stream);
 
 /*
  * sdm_forward without a caller workspace and without any allocation: for callers that

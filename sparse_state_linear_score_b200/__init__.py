@@ -94,7 +94,7 @@ def _load():
         "sdm_forward_noalloc": ([D, P, P, P, P, P, P, P, S, P, P], I32),
         "sdm_backward_workspace_bytes": ([D], SZ),
         "sdm_score_backward": ([D, P, P, I32, P, P, P, P, P, P], I32),
-        "sdm_backward": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P, P, P, SZ, P], I32),
+        "sdm_backward": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P, P, P, P, SZ, P], I32),
         "sdm_gemm_bf16": ([I32, I32, I32, P, P, P, P], I32),
         "sdm_layer_in_workspace_bytes": ([D], SZ),
         "sdm_layer_in": ([D, P, P, P, P, I32, P, P, P, P, P, P, P, SZ, P], I32),
@@ -287,10 +287,11 @@ def backward_workspace_bytes(d: Dims) -> int:
 
 
 def backward(d: Dims, v, alpha, beta, widx, ww, ridx, rw, st: State, dout, ws=None, grads=None,
-             stream=None) -> dict:
+             stream=None, dM_end=None) -> dict:
     """sdm_backward: gradients of the recurrence over one call for the output gradient dout
-    [B,H,T,d_v] fp32.  `st` must hold the state at the start of the call; it is replayed and
-    restored in place.  Returns dict dv, dalpha, dbeta, dww, drw, dM_in (fp32)."""
+    [B,H,T,d_v] fp32 and, optionally, the gradient dM_end [B,H,N,d_v] fp32 of the memory
+    after the last token.  `st` must hold the state at the start of the call; it is replayed
+    and restored in place.  Returns dict dv, dalpha, dbeta, dww, drw, dM_in (fp32)."""
     dev = v.device
     if ws is None:
         ws = torch.empty(max(16, backward_workspace_bytes(d)), dtype=torch.uint8, device=dev)
@@ -305,7 +306,9 @@ def backward(d: Dims, v, alpha, beta, widx, ww, ridx, rw, st: State, dout, ws=No
     a = _fw_args(d, v, alpha, beta, widx, ww, ridx, rw)
     g = grads
     _ok(_lib.sdm_backward(ctypes.byref(d), *a, ctypes.byref(st.c),
-                          _ptr(dout, "dout", torch.float32), _ptr(g["dv"], "dv", torch.float32),
+                          _ptr(dout, "dout", torch.float32),
+                          None if dM_end is None else _ptr(dM_end, "dM_end", torch.float32),
+                          _ptr(g["dv"], "dv", torch.float32),
                           _ptr(g["dalpha"], "dalpha", torch.float32),
                           _ptr(g["dbeta"], "dbeta", torch.float32),
                           _ptr(g["dww"], "dww", torch.float32), _ptr(g["drw"], "drw", torch.float32),

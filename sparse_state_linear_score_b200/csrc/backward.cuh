@@ -64,6 +64,7 @@ struct BwdPtrs {
     double* p_da;        // [S][BH*T]       of dalpha
     double* gam;         // [BH]            the final backward prefix
     int8_t* rpart;       // [BH*T][W]       the read of the same token with the write's slot, or -1
+    double* x0;          // [BH][S]         each slice's share of <dM_end, M_T> (every-slot decay)
 };
 
 SDM_DEV float4 f4(float a) { return make_float4(a, a, a, a); }
@@ -120,17 +121,60 @@ SDM_DEV float bwd_factor(double st, double L, int touched) {
     return isnan(st) ? -bwd_exp(L) : bwd_exp(L - st);
 }
 
-// Private stamp copies for every slice, gradient stamps NaN, final prefixes 0.
+// Private stamp copies for every slice; the memory gradient at the end of the call: zero
+// (NaN gradient stamps) or dM_end (its rows, stamps 0 = the backward prefix at the end);
+// final prefixes and the slices' <dM_end, M_T> shares 0.
 __global__ void bwd_init_kernel(const double* __restrict__ stamp, BwdPtrs P, size_t bhn,
-                                int S, int BH) {
+                                int S, int BH, const float* __restrict__ dM_end, int d_v) {
     const size_t total = (size_t)S * bhn;
     const size_t stride = (size_t)gridDim.x * blockDim.x;
     const size_t i0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const double ds0 = dM_end ? 0.0 : __longlong_as_double(0x7ff8000000000000ll);
     for (size_t i = i0; i < total; i += stride) {
         P.pst[i] = stamp[i % bhn];
-        P.pds[i] = __longlong_as_double(0x7ff8000000000000ll);
+        P.pds[i] = ds0;
+    }
+    if (dM_end) {
+        const size_t n4 = bhn * (size_t)(d_v / 4);
+        for (size_t i = i0; i < n4; i += stride)
+            reinterpret_cast<float4*>(P.dM)[i] = reinterpret_cast<const float4*>(dM_end)[i];
     }
     for (size_t i = i0; i < (size_t)BH; i += stride) P.gam[i] = 0.0;
+    for (size_t i = i0; i < (size_t)BH * S; i += stride) P.x0[i] = 0.0;
+}
+
+// With an end-of-call gradient and every-slot decay, the sweep's running <dM, M> starts at
+// <dM_end, M_T> over the whole table (M_T = the memory the replay left, true values):
+// grid (BH * S, row blocks), each block adds its rows' share of one slice (float4 column).
+constexpr int BWD_X0_ROWS = 4096;
+__global__ void __launch_bounds__(256) bwd_x0_kernel(const BwdPtrs P, const float* __restrict__ M,
+                                                     const float* __restrict__ M0,
+                                                     const float* __restrict__ dM_end, int H,
+                                                     int N, int T, int d_v, int S) {
+    __shared__ double red[256];
+    const int sc = (int)(blockIdx.x % S);
+    const size_t bh = blockIdx.x / S;
+    const int h = (int)(bh % H);
+    const double LT = P.log_lam[bh * (size_t)(T + 1) + T];
+    const double* stb = P.pst + bh * (size_t)N;  // slice 0's copy: the stamps after the replay
+    const size_t r0 = (size_t)blockIdx.y * BWD_X0_ROWS;
+    double acc = 0.0;
+    for (size_t r = r0 + threadIdx.x; r < r0 + BWD_X0_ROWS && r < (size_t)N; r += blockDim.x) {
+        const double st = stb[r];
+        const float f = isnan(st) ? bwd_exp(LT) : bwd_exp(LT - st);
+        const float* src = (isnan(st) ? M0 + (size_t)h * N * d_v : M + bh * (size_t)N * d_v) +
+                           r * d_v + 4 * sc;
+        const float4 m = *reinterpret_cast<const float4*>(src);
+        const float4 g = *reinterpret_cast<const float4*>(dM_end + (bh * (size_t)N + r) * d_v + 4 * sc);
+        acc += (double)f * (double)f4_dot(g, m);
+    }
+    red[threadIdx.x] = acc;
+    __syncthreads();
+    for (int m = 128; m > 0; m >>= 1) {
+        if ((int)threadIdx.x < m) red[threadIdx.x] += red[threadIdx.x + m];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) atomicAdd(&P.x0[bh * (size_t)S + sc], red[0]);
 }
 
 // For every write row, the read row of the same token that has its slot (reads are
@@ -263,9 +307,10 @@ __global__ void __launch_bounds__(32) bwd_sweep_kernel(
     double* dsb = P.pds + ((size_t)sc * BH + bh) * N;
     float* dMb = P.dM + bh * (size_t)N * d_v;
     const double* lamb = P.log_lam + bh * (size_t)(T + 1);
-    // this lane's share of <dM, M>; the backward log-decay prefix Gam = Lambda_T - Lambda_{t+1}
-    // before token t (sums of the same logs as the replay's prefix)
-    double X = 0.0;
+    // this lane's share of <dM, M> (lane 0 starts with the slice's share of <dM_end, M_T>);
+    // the backward log-decay prefix Gam = Lambda_T - Lambda_{t+1} before token t (sums of the
+    // same logs as the replay's prefix)
+    double X = lane == 0 && !touched ? P.x0[bh * (size_t)S + sc] : 0.0;
     const double LT = T > 0 ? lamb[T] : 0.0;
     // the next token's inputs
     int nrs[KPL], nws[KPL], npj[KPL];

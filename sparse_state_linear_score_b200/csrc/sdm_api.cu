@@ -349,7 +349,7 @@ int bwd_slices(const sdm_dims* d) { return (d->d_v / 4 + BWD_SLICE_Q - 1) / BWD_
 
 struct BwdLayout {
     size_t off_rows, off_lstamp, off_lam, off_dM, off_pst, off_pds, off_pdww, off_pdrw, off_pdb,
-        off_pda, off_gam, off_rpart, total;
+        off_pda, off_gam, off_rpart, off_x0, total;
 };
 
 BwdLayout bwd_layout(const sdm_dims* d) {
@@ -369,6 +369,7 @@ BwdLayout bwd_layout(const sdm_dims* d) {
     L.off_pda = o;    o = up256(o + S * BH * T * 8);
     L.off_gam = o;    o = up256(o + BH * 8);
     L.off_rpart = o;  o = up256(o + BH * T * (size_t)d->W);
+    L.off_x0 = o;     o = up256(o + BH * S * 8);
     L.total = o;
     return L;
 }
@@ -377,13 +378,19 @@ template <typename VT, int KPL>
 sdm_status launch_backward_t(const sdm_dims* d, const BwdPtrs& P, const void* v,
                              const float* alpha, const float* beta, const int32_t* widx,
                              const float* ww, const int32_t* ridx, const float* rw,
-                             const sdm_state* st, const float* dout, float* dv, cudaStream_t s) {
+                             const sdm_state* st, const float* dout, const float* dM_end,
+                             float* dv, cudaStream_t s) {
     const int touched = d->decay == SDM_DECAY_TOUCHED;
     const int S = bwd_slices(d);
     const unsigned grid = (unsigned)((size_t)BH_of(d) * S);
     bwd_replay_kernel<VT, KPL><<<grid, 32, 0, s>>>((const VT*)v, alpha, beta, widx, ww, st->M,
                                                    st->Lambda, st->M0, P, d->H, (int)N_of(d),
                                                    d->T, d->d_v, d->W, S, touched);
+    if (dM_end && !touched) {
+        const dim3 xg(grid, (unsigned)((N_of(d) + BWD_X0_ROWS - 1) / BWD_X0_ROWS));
+        bwd_x0_kernel<<<xg, 256, 0, s>>>(P, st->M, st->M0, dM_end, d->H, (int)N_of(d), d->T,
+                                         d->d_v, S);
+    }
     bwd_sweep_kernel<VT, KPL><<<grid, 32, 0, s>>>((const VT*)v, alpha, beta, widx, ww, ridx, rw,
                                                   st->M, st->M0, P, dout, dv, d->H, (int)N_of(d),
                                                   d->T, d->d_v, d->W, d->R, S, touched);
@@ -749,16 +756,17 @@ size_t sdm_backward_workspace_bytes(const sdm_dims* dims) {
 
 sdm_status sdm_backward(const sdm_dims* dims, const void* v, const float* alpha, const float* beta,
                         const int32_t* widx, const float* ww, const int32_t* ridx, const float* rw,
-                        const sdm_state* st, const float* dout, float* dv, float* dalpha,
-                        float* dbeta, float* dww, float* drw, float* dM_in, void* ws,
-                        size_t ws_bytes, sdm_stream_t stream) {
+                        const sdm_state* st, const float* dout, const float* dM_end, float* dv,
+                        float* dalpha, float* dbeta, float* dww, float* drw, float* dM_in,
+                        void* ws, size_t ws_bytes, sdm_stream_t stream) {
     sdm_status e = check_dims(dims);
     if (e) return e;
     if ((e = check_state(st))) return e;
     if (!v || !alpha || !beta || !widx || !ww || !ridx || !rw || !dout || !dv || !dalpha ||
         !dbeta || !dww || !drw || !dM_in)
         return SDM_ERR_ARG;
-    if (!aligned16(v) || !aligned16(dout) || !aligned16(dv) || !aligned16(dM_in))
+    if (!aligned16(v) || !aligned16(dout) || !aligned16(dv) || !aligned16(dM_in) ||
+        (dM_end && !aligned16(dM_end)))
         return SDM_ERR_ALIGN;
     if (dims->W + dims->R > BWD_MAXO) return SDM_ERR_SHAPE;
     const BwdLayout L = bwd_layout(dims);
@@ -782,6 +790,7 @@ sdm_status sdm_backward(const sdm_dims* dims, const void* v, const float* alpha,
     P.p_da = reinterpret_cast<double*>(b + L.off_pda);
     P.gam = reinterpret_cast<double*>(b + L.off_gam);
     P.rpart = reinterpret_cast<int8_t*>(b + L.off_rpart);
+    P.x0 = reinterpret_cast<double*>(b + L.off_x0);
     const int threads = 256;
     auto grid_for = [](size_t n) {
         size_t blocks = (n + 255) / 256;
@@ -790,13 +799,14 @@ sdm_status sdm_backward(const sdm_dims* dims, const void* v, const float* alpha,
     };
     // private stamp copies per slice, every memory-gradient row at zero (NaN stamp)
     bwd_init_kernel<<<grid_for((size_t)S * rows), threads, 0, s>>>(st->stamp, P, rows, S,
-                                                                   (int)BH_of(dims));
+                                                                   (int)BH_of(dims), dM_end,
+                                                                   dims->d_v);
     if (dims->T > 0) {
         const size_t BHT = (size_t)BH_of(dims) * dims->T;
         bwd_links_kernel<<<grid_for(BHT * dims->W), threads, 0, s>>>(widx, ridx, BHT, dims->W,
                                                                      dims->R, P.rpart);
         const int m = dims->W > dims->R ? dims->W : dims->R;
-#define SDM_BWD(VT, K) launch_backward_t<VT, K>(dims, P, v, alpha, beta, widx, ww, ridx, rw, st, dout, dv, s)
+#define SDM_BWD(VT, K) launch_backward_t<VT, K>(dims, P, v, alpha, beta, widx, ww, ridx, rw, st, dout, dM_end, dv, s)
         if (dims->v_dtype == SDM_BF16) {
             e = m <= 32 ? SDM_BWD(__nv_bfloat16, 1) : m <= 64 ? SDM_BWD(__nv_bfloat16, 2)
                                                     : SDM_BWD(__nv_bfloat16, 4);

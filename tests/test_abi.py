@@ -143,9 +143,11 @@ def test_backward_host_checks(lib):
 
     def call(v=p, dout=p, ws_ptr=p, ws_bytes=big, dims=d):
         return lib.sdm_backward(ctypes.byref(dims), v, p, p, p, p, p, p, ctypes.byref(st), dout,
-                                p, p, p, p, p, p, ws_ptr, ws_bytes, None)
+                                None, p, p, p, p, p, p, ws_ptr, ws_bytes, None)
     assert call(v=None) == 1                                  # SDM_ERR_ARG
     assert call(dout=ctypes.c_void_p(0x1008)) == 4            # SDM_ERR_ALIGN
     assert call(ws_bytes=ctypes.c_size_t(ws - 1)) == 7        # SDM_ERR_WORKSPACE
     assert call(ws_ptr=None) == 7
     assert call(dims=mid_dims(d_k=30)) == 2                   # SDM_ERR_SHAPE
+    assert lib.sdm_backward(ctypes.byref(d), p, p, p, p, p, p, p, ctypes.byref(st), p,
+                            ctypes.c_void_p(0x1004), p, p, p, p, p, p, p, big, None) == 4
