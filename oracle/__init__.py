@@ -20,7 +20,8 @@ Parity status per function:
   recur_backward .............. pinned (central finite differences of recur_dense and
                                  recur_touched for every input, with and without a gradient
                                  of the final memory; beta = 0 and alpha = 1 closed form;
-                                 beta = 0 decay closed form of that gradient)
+                                 beta = 0 decay closed form of that gradient; two calls
+                                 chained through it = one call)
   score_backward .............. pinned (central finite differences of the softmax of the
                                  selected slots' half-score sums, for x and the tables)
   recur_touched ............... pinned (hand example, alpha = 1 equals recur_dense,

@@ -459,6 +459,27 @@ def pin_backward_end_gradient(o):
     assert np.array_equal(g["drw"], np.zeros((T, R)))
 
 
+def pin_backward_split_calls(o):
+    """A sequence taken back in two calls (the second call's start-state gradient passed to
+    the first as the gradient of its final memory) gives the single call's gradients."""
+    rng = _rng(21)
+    T, T1, N, dv, W, R = 10, 4, 6, 3, 2, 3
+    v, alpha, beta, widx, ww, ridx, rw, M0, dout = _fd_case(rng, T, N, dv, W, R)
+    for touched in (False, True):
+        fwd = o.recur_touched if touched else o.recur_dense
+        whole = o.recur_backward(v, alpha, beta, widx, ww, ridx, rw, M0, dout, touched=touched)
+        a, b = slice(0, T1), slice(T1, T)
+        _, M_mid = fwd(v[a], alpha[a], beta[a], widx[a], ww[a], ridx[a], rw[a], M0)
+        g2 = o.recur_backward(v[b], alpha[b], beta[b], widx[b], ww[b], ridx[b], rw[b], M_mid,
+                              dout[b], touched=touched)
+        g1 = o.recur_backward(v[a], alpha[a], beta[a], widx[a], ww[a], ridx[a], rw[a], M0,
+                              dout[a], touched=touched, dM_end=g2["dM0"])
+        for key in ("dv", "dalpha", "dbeta", "dww", "drw"):
+            np.testing.assert_allclose(np.concatenate([g1[key], g2[key]]), whole[key],
+                                       rtol=1e-12, atol=1e-13, err_msg=key)
+        np.testing.assert_allclose(g1["dM0"], whole["dM0"], rtol=1e-12, atol=1e-13)
+
+
 def pin_backward_frozen_memory(o):
     """beta = 0, alpha = 1: the memory stays M0, so o_t = sum_j u_j M0[r_j] and
     dM0[s] = sum over (t, j) with r_j = s of u_j dout_t, du_j = <dout_t, M0[r_j]>,
@@ -706,4 +727,4 @@ ALL_PINS = [pin_pk_equals_brute, pin_brute_matches_numpy, pin_pk_depends_on_k, p
             pin_layer_in_routing_and_gates, pin_layer_in_linear, pin_touched_hand,
             pin_touched_alpha_one, pin_touched_all_slots_gdn, pin_touched_beta_zero,
             pin_backward_finite_differences, pin_backward_touched_finite_differences,
-            pin_backward_frozen_memory, pin_backward_end_gradient, pin_score_backward_finite_differences]
+            pin_backward_frozen_memory, pin_backward_end_gradient, pin_backward_split_calls, pin_score_backward_finite_differences]
