@@ -112,6 +112,9 @@ MUTANTS = {
     "q_k_swapped": [
         ("q[((size_t)ri * H + h) * dk + c] = ph[c];", "q[((size_t)ri * H + h) * dk + c] = ph[dk + c];"),
     ],
+    "backward_end_gradient_ignored": [
+        ("if (dM_end) memcpy(dM, dM_end, sizeof(double) * ND);", "(void)dM_end;"),
+    ],
     "read_weights_from_write": [
         ("o += rw[(size_t)t * R + j] * M[(size_t)rs[j] * dv + c];",
          "o += rw[(size_t)t * R + j] * M[(size_t)ws[j % W] * dv + c];"),
