@@ -293,7 +293,9 @@ sdm_status sdm_backward(const sdm_dims* dims, const void* v, const float* alpha,
  *   All calls on a device share the array: calls that can overlap on the GPU (different
  *     streams, or several host threads) race on it and must be serialised by the caller.
  *   The first call on a device looks up the array's device address (once per device, with
- *     the stream's device current); make that first call before any stream capture.
+ *     the stream's device current); make that first call before any stream capture.  After
+ *     a device reset the device has a new context, and the next call looks the address up
+ *     again.
  *   Never calls cudaMalloc, cudaFree or any allocating routine.
  */
 sdm_status sdm_forward_noalloc(const sdm_dims* dims, const void* v, const float* alpha,

@@ -293,6 +293,13 @@ def backward(d: Dims, v, alpha, beta, widx, ww, ridx, rw, st: State, dout, ws=No
     after the last token.  `st` must hold the state at the start of the call; it is replayed
     and restored in place.  Returns dict dv, dalpha, dbeta, dww, drw, dM_in (fp32)."""
     dev = v.device
+    if dM_end is not None:
+        # the kernels read B*H*N*d_v floats from it: a smaller tensor would be read past its end
+        if tuple(dM_end.shape) != (d.B, d.H, d.N, d.d_v):
+            raise ValueError(f"dM_end must have shape {(d.B, d.H, d.N, d.d_v)}, "
+                             f"got {tuple(dM_end.shape)}")
+        if dM_end.device != dev:
+            raise ValueError(f"dM_end is on {dM_end.device}, the other inputs on {dev}")
     if ws is None:
         ws = torch.empty(max(16, backward_workspace_bytes(d)), dtype=torch.uint8, device=dev)
     if grads is None:

@@ -147,6 +147,9 @@ __global__ void bwd_init_kernel(const double* __restrict__ stamp, BwdPtrs P, siz
 // <dM_end, M_T> over the whole table (M_T = the memory the replay left, true values):
 // grid (BH * S, row blocks), each block adds its rows' share of one slice (float4 column).
 constexpr int BWD_X0_ROWS = 4096;
+// Each slice is one float4 column (offset 4*sc) and the replay's stamps sit in slice 0's
+// copy; a wider slice would need a loop over its columns here.
+static_assert(BWD_SLICE_Q == 1, "bwd_x0_kernel reads one float4 column per slice");
 __global__ void __launch_bounds__(256) bwd_x0_kernel(const BwdPtrs P, const float* __restrict__ M,
                                                      const float* __restrict__ M0,
                                                      const float* __restrict__ dM_end, int H,

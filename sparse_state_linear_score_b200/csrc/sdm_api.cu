@@ -500,23 +500,58 @@ static __device__ __align__(256) unsigned char g_noalloc_ws[kNoAllocWorkspaceByt
 namespace {
 
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+struct NoAllocSlot {
+    CUcontext ctx;  // the context the address belongs to
+    void* ptr;
+};
+NoAllocSlot g_noalloc_slot[kNoAllocMaxDevices] = {};
 
-// Device address of g_noalloc_ws on the current device.  In host code the array's name is
-// only a host-side stand-in, so the address is looked up once per device (with that device
-// current) and cached.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The driver's cuCtxGetCurrent, reached through the runtime (the library links no driver
+// library); null when the driver does not offer it.
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(f);
+    });
+    return fn;
+}
+
+CUcontext current_ctx() {
+    CUcontext c = nullptr;
+    const CtxGetCurrentFn fn = ctx_get_current();
+    if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
+// Device address of g_noalloc_ws in the current context.  In host code the array's name is
+// only a host-side stand-in, so the address is looked up with the device current and cached
+// per device together with the context it belongs to.  A device reset (or any teardown of the
+// primary context) gives the device a new context, in which the library's module is loaded
+// again and the array may sit elsewhere: the changed context makes the next call look the
+// address up again instead of launching on the old one.
 sdm_status noalloc_workspace(void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return SDM_ERR_CUDA;
     if (dev < 0 || dev >= kNoAllocMaxDevices) return SDM_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    NoAllocSlot& slot = g_noalloc_slot[dev];
+    const CUcontext ctx = current_ctx();
+    if (!slot.ptr || ctx == nullptr || ctx != slot.ctx) {
         void* p = nullptr;
+        // also makes the device's primary context current if no call has yet
         if (cudaGetSymbolAddress(&p, g_noalloc_ws) != cudaSuccess || p == nullptr)
             return SDM_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
+        slot.ptr = p;
+        slot.ctx = current_ctx();
     }
-    *out = g_noalloc_ptr[dev];
+    *out = slot.ptr;
     return SDM_OK;
 }
 

@@ -9,6 +9,8 @@ Tolerances (from the stated targets of the hot path):
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 
 SCORE_GAP = 1e-5
@@ -82,3 +84,16 @@ def compare_selection(orc, x, sk, gpu_idx, ora_idx, ora_score, n, gap=SCORE_GAP)
 def f64(t):
     """torch tensor (any device / dtype) -> fp64 numpy."""
     return t.detach().to("cpu").double().numpy()
+
+
+# Observed errors of every tolerance check in this process, (test id, what, error, tolerance),
+# printed by the terminal summary so that drift well inside a tolerance stays visible.
+OBSERVED: list[tuple[str, str, float, float]] = []
+
+
+def check_err(err: float, tol: float, what: str = "rel err") -> float:
+    """Record an observed error and fail, naming it, when it exceeds its tolerance."""
+    test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
+    OBSERVED.append((test, what, float(err), float(tol)))
+    assert err <= tol, f"{what}: max rel err {err:.3e} above tolerance {tol:.1e}"
+    return err

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import sdm_synth as S
-from tests.parity import TOL, f64, normwise_rel_err
+from tests.parity import TOL, check_err, f64, normwise_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -74,7 +74,7 @@ def _case(sdm, orc, wl, decay, pool, seed, start_tokens=0, end_grad=False):
             for key, gk in (("dv", "dv"), ("dalpha", "dalpha"), ("dbeta", "dbeta"),
                             ("dww", "dww"), ("drw", "drw"), ("dM0", "dM_in")):
                 err = normwise_rel_err(f64(grads[gk][b, h]), ref[key])
-                assert err <= tol, ((b, h), key, err)
+                check_err(err, tol, f"{key} (b,h)={(b, h)}")
 
 
 @pytest.mark.parametrize("decay", ["all", "touched"])

@@ -15,7 +15,7 @@ import torch
 
 import oracle
 import sdm_synth as S
-from tests.parity import TOL, f64, normwise_rel_err
+from tests.parity import TOL, check_err, f64, normwise_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -77,7 +77,7 @@ def test_layer_out_vs_oracle(sdm):
         y = sdm.layer_out(d, o, g, wn, Wo_t, eps=1e-6)
         torch.cuda.synchronize()
         ref = orc.layer_out(f64(o), f64(g), f64(wn), f64(Wo_t), eps=1e-6)
-        assert normwise_rel_err(f64(y), ref) <= TOL["bf16"]
+        check_err(normwise_rel_err(f64(y), ref), TOL["bf16"], "y")
 
 
 def test_layer_out_after_prefill(sdm):
@@ -103,7 +103,7 @@ def test_layer_out_after_prefill(sdm):
     rows = np.array([0, 1, 77, 255, 256, 300, 511])
     ref = orc.layer_out(f64(out), f64(g), f64(wn), f64(Wo_t), rows=rows)
     got = f64(y).reshape(wl.B * wl.T, dm)[rows]
-    assert normwise_rel_err(got, ref) <= TOL["bf16"]
+    check_err(normwise_rel_err(got, ref), TOL["bf16"])
     assert sdm.device_error() == 0
 
 
@@ -171,7 +171,7 @@ def test_layer_forward_chain(sdm):
                                    widx[0, h].cpu().numpy(), f64(ww[0, h]), ridx[0, h].cpu().numpy(),
                                    f64(rw[0, h]), s))
     ref_o = np.stack(outs).reshape(B, H, T, dv)
-    assert normwise_rel_err(f64(o), ref_o) <= TOL["bf16"]
+    check_err(normwise_rel_err(f64(o), ref_o), TOL["bf16"], "o")
     ref_y = orc.layer_out(f64(o), f64(r["g"]), f64(wn), f64(Wo_t))
-    assert normwise_rel_err(f64(y), ref_y) <= TOL["bf16"]
+    check_err(normwise_rel_err(f64(y), ref_y), TOL["bf16"], "y")
     assert sdm.device_error() == 0

@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import sdm_synth as S
-from tests.parity import TOL, compare_selection, f64, normwise_rel_err, per_bh_rel_err
+from tests.parity import TOL, check_err, compare_selection, f64, normwise_rel_err, per_bh_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -119,7 +119,8 @@ def _forward_case(sdm, orc, wl, inp, widx, ww, ridx, rw, tol):
     for (b, h), o_ref, st_ref in zip(pairs, outs, states):
         e_out = normwise_rel_err(f64(out[b, h]), o_ref)
         e_mem = normwise_rel_err(f64(M[b, h]), orc.materialize(st_ref))
-        assert e_out <= tol and e_mem <= tol, ((b, h), e_out, e_mem)
+        check_err(e_out, tol, f"out (b,h)={(b, h)}")
+        check_err(e_mem, tol, f"memory (b,h)={(b, h)}")
     lam_ref = np.array([s["Lambda"] for s in states])
     np.testing.assert_allclose(f64(st.Lambda).reshape(-1), lam_ref, rtol=1e-12, atol=1e-12)
     return out, st
@@ -186,7 +187,7 @@ def test_prefill_end_to_end(sdm, orc):
         pairs = [(b, h) for b in range(wl.B) for h in range(wl.H)]
         outs, _ = oracle_recurrence(orc, inp, widx.cpu(), ww.cpu(), ridx.cpu(), rw.cpu(), pairs)
         ref = np.stack(outs).reshape(wl.B, wl.H, wl.T, wl.d_v)
-        assert per_bh_rel_err(f64(out), ref) <= TOL[wl.v_dtype]
+        check_err(per_bh_rel_err(f64(out), ref), TOL[wl.v_dtype])
 
 
 def test_shared_subkey_tables(sdm, orc):
@@ -207,7 +208,7 @@ def test_shared_subkey_tables(sdm, orc):
     pairs = [(b, h) for b in range(wl.B) for h in range(wl.H)]
     outs, _ = oracle_recurrence(orc, inp, widx.cpu(), ww.cpu(), ridx.cpu(), rw.cpu(), pairs)
     ref = np.stack(outs).reshape(wl.B, wl.H, wl.T, wl.d_v)
-    assert per_bh_rel_err(f64(out), ref) <= TOL[wl.v_dtype]
+    check_err(per_bh_rel_err(f64(out), ref), TOL[wl.v_dtype])
 
 
 def test_split_invariance(sdm, orc):
@@ -235,8 +236,8 @@ def test_split_invariance(sdm, orc):
                                sl(inp["alpha"], a, b), sl(inp["beta"], a, b), inp["skw"],
                                inp["skr"], st2)
             outs.append(o)
-        assert per_bh_rel_err(f64(torch.cat(outs, 2)), f64(full)) <= tol
-        assert per_bh_rel_err(f64(sdm.state_materialize(d, st2)), f64(M_full)) <= tol
+        check_err(per_bh_rel_err(f64(torch.cat(outs, 2)), f64(full)), tol)
+        check_err(per_bh_rel_err(f64(sdm.state_materialize(d, st2)), f64(M_full)), tol)
         st3 = sdm.State(d, inp["M0"])
         sdm.state_reset(d, st3)
         d1 = dims_of(sdm, wl, T=T1)
@@ -250,8 +251,8 @@ def test_split_invariance(sdm, orc):
                                    inp["v"][:, :, t].contiguous(), inp["alpha"][:, :, t].contiguous(),
                                    inp["beta"][:, :, t].contiguous(), inp["skw"], inp["skr"], st3)
             outs.append(o.unsqueeze(2))
-        assert per_bh_rel_err(f64(torch.cat(outs, 2)), f64(full)) <= tol
-        assert per_bh_rel_err(f64(sdm.state_materialize(d, st3)), f64(M_full)) <= tol
+        check_err(per_bh_rel_err(f64(torch.cat(outs, 2)), f64(full)), tol)
+        check_err(per_bh_rel_err(f64(sdm.state_materialize(d, st3)), f64(M_full)), tol)
     assert sdm.device_error() == 0
 
 
@@ -291,9 +292,9 @@ def test_decode_vs_oracle(sdm, orc):
             ref = orc.recur_lazy(f64(inp["v"][b, h]), f64(inp["alpha"][b, h]), f64(inp["beta"][b, h]),
                                  widx, ww, ridx, rw, stt)
             got = np.concatenate([f64(out0[b, h])] + [f64(o[b, h])[None] for o in outs])
-            assert normwise_rel_err(got, ref) <= TOL[wl.v_dtype]
-            assert normwise_rel_err(f64(sdm.state_materialize(d, st)[b, h]),
-                                    orc.materialize(stt)) <= TOL[wl.v_dtype]
+            check_err(normwise_rel_err(got, ref), TOL[wl.v_dtype])
+            check_err(normwise_rel_err(f64(sdm.state_materialize(d, st)[b, h]),
+                                       orc.materialize(stt)), TOL[wl.v_dtype], "memory")
     assert sdm.device_error() == 0
 
 
@@ -394,7 +395,7 @@ def _full_case(sdm, orc, wl, n_rows=192, n_pairs=2, seed=0):
         ref = orc.recur_lazy(f64(inp["v"][b, h, :T0]), f64(inp["alpha"][b, h, :T0]),
                              f64(inp["beta"][b, h, :T0]), widx[b, h].cpu().numpy(), f64(ww[b, h]),
                              ridx[b, h].cpu().numpy(), f64(rw[b, h]), stt)
-        assert normwise_rel_err(f64(out[b, h]), ref) <= TOL[wl.v_dtype]
+        check_err(normwise_rel_err(f64(out[b, h]), ref), TOL[wl.v_dtype])
         d1 = sdm.Dims(1, 1, T0, wl.d_k, wl.n_sub, wl.d_v, wl.k_half, wl.W, wl.R, wl.x_dtype,
                       wl.v_dtype)
         # materialise just this sequence through a one-sequence view of the state
@@ -406,7 +407,7 @@ def _full_case(sdm, orc, wl, n_rows=192, n_pairs=2, seed=0):
         one._c = sdm._CState(one.M.data_ptr(), one.stamp.data_ptr(), one.Lambda.data_ptr(),
                              one.M0.data_ptr())
         Mone = sdm.state_materialize(d1, one)
-        assert normwise_rel_err(f64(Mone[0, 0]), orc.materialize(stt)) <= TOL[wl.v_dtype]
+        check_err(normwise_rel_err(f64(Mone[0, 0]), orc.materialize(stt)), TOL[wl.v_dtype])
         del one, Mone
     return inp, st, (widx, ww, ridx, rw)
 
@@ -460,7 +461,7 @@ def test_full_decode(sdm, orc):
     stt = orc.fresh_lazy_state(f64(inp["M0"][h]))
     ref = orc.recur_lazy(f64(inp["v"][b, h]), f64(inp["alpha"][b, h]), f64(inp["beta"][b, h]), widx,
                          ww, ridx, rw, stt)
-    assert normwise_rel_err(f64(outs[:, b, h]), ref[wl.T:]) <= TOL[wl.v_dtype]
+    check_err(normwise_rel_err(f64(outs[:, b, h]), ref[wl.T:]), TOL[wl.v_dtype])
     del inp, st
     torch.cuda.empty_cache()
 

@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import sdm_synth as S
-from tests.parity import f64, normwise_rel_err
+from tests.parity import check_err, f64, normwise_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -51,9 +51,9 @@ def test_score_backward_vs_oracle(sdm, orc, name):
         torch.cuda.synchronize()
         assert sdm.device_error() == 0
         dx_o, dsk_o = orc.score_backward(f64(x), f64(sk), idx.cpu().numpy(), f64(dw))
-        assert normwise_rel_err(f64(dx), dx_o) <= 1e-4
-        assert normwise_rel_err(f64(dsk), dsk_o) <= 1e-4
+        check_err(normwise_rel_err(f64(dx), dx_o), 1e-4, "dx")
+        check_err(normwise_rel_err(f64(dsk), dsk_o), 1e-4, "dsubkeys")
         # a second call adds to the table gradient
         _, dsk2 = sdm.score_backward(d, x, sk, top, idx, w, dw, dsubkeys=dsk.clone())
         torch.cuda.synchronize()
-        assert normwise_rel_err(f64(dsk2), 2 * dsk_o) <= 1e-4
+        check_err(normwise_rel_err(f64(dsk2), 2 * dsk_o), 1e-4, "dsubkeys accumulated")

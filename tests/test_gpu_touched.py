@@ -14,7 +14,7 @@ import torch
 
 import oracle
 import sdm_synth as S
-from tests.parity import TOL, f64, normwise_rel_err
+from tests.parity import TOL, check_err, f64, normwise_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -58,7 +58,8 @@ def _forward_touched(sdm, orc, wl, inp, widx, ww, ridx, rw, tol):
             o_ref, M_ref = _oracle_bh(orc, inp, b, h, wc, wwc, rc, rwc)
             e_out = normwise_rel_err(f64(out[b, h]), o_ref)
             e_mem = normwise_rel_err(f64(M[b, h]), M_ref)
-            assert e_out <= tol and e_mem <= tol, ((b, h), e_out, e_mem)
+            check_err(e_out, tol, f"out (b,h)={(b, h)}")
+            check_err(e_mem, tol, f"memory (b,h)={(b, h)}")
     return out, M
 
 
@@ -121,8 +122,8 @@ def test_touched_prefill_and_decode(sdm, orc):
     for b in range(wl.B):
         for h in range(wl.H):
             o_ref, M_ref = _oracle_bh(orc, inp, b, h, widx, ww, ridx, rw)
-            assert normwise_rel_err(f64(got[b, h]), o_ref) <= TOL[wl.v_dtype]
-            assert normwise_rel_err(f64(M[b, h]), M_ref) <= TOL[wl.v_dtype]
+            check_err(normwise_rel_err(f64(got[b, h]), o_ref), TOL[wl.v_dtype], "out")
+            check_err(normwise_rel_err(f64(M[b, h]), M_ref), TOL[wl.v_dtype], "memory")
     # the same tokens as two prefill calls from a fresh state
     st2 = sdm.State(d, inp["M0"])
     sdm.state_reset(d, st2)
