@@ -220,8 +220,7 @@ def run_gpu(args, wl, world, rank, local):
         if ev:
             ev[0].record(stream)
         sdm.state_reset(d, st)
-        sdm.score_topk(d, inp["k"], inp["skw"], wl.W, widx, ww)
-        sdm.score_topk(d, inp["q"], inp["skr"], wl.R, ridx, rw)
+        sdm.score_qk(d, inp["q"], inp["k"], inp["skw"], inp["skr"], (widx, ww, ridx, rw))
         if ev:
             ev[1].record(stream)
         sdm.forward_plan(d, inp["alpha"], inp["beta"], widx, ww, ridx, rw, st, ws)
@@ -255,9 +254,9 @@ def run_gpu(args, wl, world, rank, local):
     plan_ms = [e[1].elapsed_time(e[2]) for e in evs]
     run_ms = [e[2].elapsed_time(e[3]) for e in evs]
     total_ms = reduce_max(sum(step_ms), device)
-    # reset, 2 x score, plan_local, plan_prefix, plan_pack, run (the per-slot chunk masks
+    # reset, score (both roles), plan_local, plan_prefix, plan_pack, run (the per-slot chunk masks
     # fit this workload, so plan_fe and plan_walk are not launched)
-    launches_per_step = 7
+    launches_per_step = 6
 
     # memory-utilisation diagnostics of the write weights (after the timed steps)
     diag = None
@@ -503,8 +502,7 @@ def run_touched(wl, inp, device, sdm, steps: int = 10, warm: int = 3) -> dict:
         if ev:
             ev[0].record(stream)
         sdm.state_reset(d, st)
-        sdm.score_topk(d, inp["k"], inp["skw"], wl.W, widx, ww)
-        sdm.score_topk(d, inp["q"], inp["skr"], wl.R, ridx, rw)
+        sdm.score_qk(d, inp["q"], inp["k"], inp["skw"], inp["skr"], (widx, ww, ridx, rw))
         if ev:
             ev[1].record(stream)
         sdm.forward_plan(d, inp["alpha"], inp["beta"], widx, ww, ridx, rw, st, ws)

@@ -10,6 +10,7 @@
  *
  *   sdm_score_topk   product-key scoring, per-half top-k, k x k combine,
  *                    top-W (or top-R) slot indices and softmax weights
+ *   sdm_score_qk     both roles of one call (keys: writes, queries: reads)
  *   sdm_forward      the sparse gated-delta recurrence over T tokens (prefill)
  *   sdm_decode_step  one token per sequence (scoring + recurrence)
  *
@@ -157,6 +158,21 @@ sdm_status sdm_state_materialize(const sdm_dims* dims, const sdm_state* st, floa
  */
 sdm_status sdm_score_topk(const sdm_dims* dims, const void* x, const void* subkeys, int32_t top,
                           int32_t* idx, float* w, sdm_stream_t stream);
+
+/*
+ * Both scorings of one call: the keys against the write-role tables and the queries against
+ * the read-role tables (§3 Method "Sparse addressing": keys choose the slots written,
+ * queries the slots read), with the results of two sdm_score_topk calls but in one launch
+ * where the shape allows it.
+ *   q, k       [B][H][T][d_k]        dims->x_dtype
+ *   skw, skr   [H][2][n_sub][d_k/2]  dims->x_dtype (the same pointer twice shares one table)
+ *   widx, ww   [B][H][T][W]          int32 / fp32 out (write role, best first)
+ *   ridx, rw   [B][H][T][R]          int32 / fp32 out (read role, best first)
+ * Errors as sdm_score_topk.
+ */
+sdm_status sdm_score_qk(const sdm_dims* dims, const void* q, const void* k, const void* skw,
+                        const void* skr, int32_t* widx, float* ww, int32_t* ridx, float* rw,
+                        sdm_stream_t stream);
 
 /* Workspace bytes sdm_forward / sdm_prefill need for `dims` (0 on bad dims). */
 size_t sdm_forward_workspace_bytes(const sdm_dims* dims);

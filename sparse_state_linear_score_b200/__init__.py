@@ -21,7 +21,7 @@ import torch
 
 from . import build as _build
 
-__all__ = ["Dims", "State", "SdmError", "state_reset", "state_materialize", "score_topk",
+__all__ = ["Dims", "State", "SdmError", "state_reset", "state_materialize", "score_topk", "score_qk",
            "forward_workspace_bytes", "forward", "forward_noalloc", "forward_plan", "forward_run", "prefill",
            "decode_step", "device_error", "weight_stats", "gemm_bf16", "layer_in", "layer_out", "lib_path",
            "DEVERR_SLOT_RANGE",
@@ -84,6 +84,7 @@ def _load():
         "sdm_state_reset": ([D, S, P], I32),
         "sdm_state_materialize": ([D, S, P, P], I32),
         "sdm_score_topk": ([D, P, P, I32, P, P, P], I32),
+        "sdm_score_qk": ([D, P, P, P, P, P, P, P, P, P], I32),
         "sdm_forward_workspace_bytes": ([D], SZ),
         "sdm_forward": ([D, P, P, P, P, P, P, P, S, P, P, SZ, P], I32),
         "sdm_forward_plan": ([D, P, P, P, P, P, P, S, P, SZ, P], I32),
@@ -197,6 +198,20 @@ def score_topk(d: Dims, x, subkeys, top: int, idx=None, w=None, stream=None):
                             top, _ptr(idx, "idx", torch.int32), _ptr(w, "w", torch.float32),
                             _stream(stream)), "sdm_score_topk")
     return idx, w
+
+
+def score_qk(d: Dims, q, k, skw, skr, sel=None, stream=None):
+    """sdm_score_qk: both roles of one call.  Returns (widx, ww, ridx, rw)."""
+    if sel is None:
+        sel = selection_buffers(d, q.device)
+    widx, ww, ridx, rw = sel
+    xdt = _xdt(d)
+    _ok(_lib.sdm_score_qk(ctypes.byref(d), _ptr(q, "q", xdt), _ptr(k, "k", xdt),
+                          _ptr(skw, "skw", xdt), _ptr(skr, "skr", xdt),
+                          _ptr(widx, "widx", torch.int32), _ptr(ww, "ww", torch.float32),
+                          _ptr(ridx, "ridx", torch.int32), _ptr(rw, "rw", torch.float32),
+                          _stream(stream)), "sdm_score_qk")
+    return sel
 
 
 def forward_workspace_bytes(d: Dims) -> int:

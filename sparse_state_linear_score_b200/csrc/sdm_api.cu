@@ -12,6 +12,7 @@
 #include "plan.cuh"
 #include "recur.cuh"
 #include "score_bwd.cuh"
+#include "score_pk.cuh"
 #include "score_rows.cuh"
 #include "score_simt.cuh"
 #include "score_tc.cuh"
@@ -229,6 +230,80 @@ sdm_status launch_score_tc(const sdm_dims* d, const void* x, const void* sk, int
     return launch_score_tc_t<32>(d, xm, km, a, grid, s);
 }
 
+// Shapes the one-round tensor-core scorer takes: bf16, 64-wide halves, at most 256 sub-keys per
+// half (a multiple of 64), at most 32 kept per half, top <= k_half (the staircase), and calls
+// of at least 64 tokens (shorter ones go to the row scorer, which spreads rows over all SMs).
+bool score_pk_eligible(const sdm_dims* d, int top) {
+    if (d->x_dtype != SDM_BF16 || d->d_k != 128) return false;
+    if (d->n_sub % 64 != 0 || d->n_sub > PK_NMAX) return false;
+    if (d->k_half > 32 || top > d->k_half) return false;
+    return d->T >= 64;
+}
+
+bool encode_x_map(EncodeTiledFn enc, CUtensorMap* m, const sdm_dims* d, const void* x, int bt,
+                  int bb) {
+    const cuuint64_t dims[4] = {(cuuint64_t)d->d_k, (cuuint64_t)d->T, (cuuint64_t)d->H,
+                                (cuuint64_t)d->B};
+    const cuuint64_t strides[3] = {(cuuint64_t)d->d_k * 2, (cuuint64_t)d->T * d->d_k * 2,
+                                   (cuuint64_t)d->H * d->T * d->d_k * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)bt, 1, (cuuint32_t)bb};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_sk_map(EncodeTiledFn enc, CUtensorMap* m, const sdm_dims* d, const void* sk, int rows) {
+    const cuuint64_t dims[2] = {64, (cuuint64_t)d->H * 2 * d->n_sub};
+    const cuuint64_t strides[1] = {64 * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)rows};
+    const cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(sk), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KP>
+sdm_status launch_score_pk_t(const CUtensorMap (&xm)[2], const CUtensorMap (&km)[2],
+                             const PkArgs& a, dim3 grid, cudaStream_t s) {
+    auto kern = score_pk_kernel<KP>;
+    if (!set_smem(kern, PkCfg<KP>::SMEM)) return SDM_ERR_CUDA;
+    kern<<<grid, PK_THREADS, PkCfg<KP>::SMEM, s>>>(xm[0], xm[1], km[0], km[1], a);
+    return launch_status();
+}
+
+// `roles` (1 or 2) scorings of the same shape in one launch (grid.z = role): role r scores
+// x[r] against sk[r] into idx[r], w[r] with top[r] slots.
+sdm_status launch_score_pk(const sdm_dims* d, int roles, const void* const* x,
+                           const void* const* sk, const int* top, int32_t* const* idx,
+                           float* const* w, cudaStream_t s) {
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return SDM_ERR_CUDA;
+    PkArgs a{};
+    a.B = d->B; a.H = d->H; a.T = d->T; a.n = d->n_sub; a.k_half = d->k_half; a.d_k = d->d_k;
+    // a tile is always 128 rows that the TMA fills: 128 tokens of one sequence, or 64 tokens of
+    // two when T = 64; rows past T or B are the load's zero fill and are not selected
+    a.bt = d->T == 64 ? 64 : 128;
+    a.bb = 128 / a.bt;
+    a.n_tt = (d->T + a.bt - 1) / a.bt;
+    a.z0 = pk_z0(d->n_sub, d->k_half);
+    CUtensorMap xm[2], km[2];
+    for (int r = 0; r < 2; ++r) {
+        const int q = r < roles ? r : 0;
+        a.top[r] = top[q];
+        a.x[r] = static_cast<const __nv_bfloat16*>(x[q]);
+        a.sk[r] = static_cast<const __nv_bfloat16*>(sk[q]);
+        a.idx[r] = idx[q];
+        a.w[r] = w[q];
+        if (!encode_x_map(enc, &xm[r], d, x[q], a.bt, a.bb)) return SDM_ERR_CUDA;
+        if (!encode_sk_map(enc, &km[r], d, sk[q], d->n_sub)) return SDM_ERR_CUDA;
+    }
+    const int n_bt = (d->B + a.bb - 1) / a.bb;
+    const dim3 grid((unsigned)(a.n_tt * n_bt), (unsigned)d->H, (unsigned)roles);
+    if (d->k_half <= 16) return launch_score_pk_t<16>(xm, km, a, grid, s);
+    return launch_score_pk_t<32>(xm, km, a, grid, s);
+}
+
 // The row scorer keeps a lane's block of n/32 half-scores in registers (at most 16) and the
 // selected lists in shared memory; check_dims already bounds k_half and top by 64 and makes
 // the half width a multiple of 8.
@@ -331,6 +406,14 @@ sdm_status score_both_roles(const sdm_dims* d, const void* q, const void* k, con
         !aligned16(widx) || !aligned16(ww) || !aligned16(ridx) || !aligned16(rw))
         return SDM_ERR_ALIGN;
     if ((long long)d->B * d->T == 0) return SDM_OK;
+    if (score_pk_eligible(d, d->W) && score_pk_eligible(d, d->R)) {
+        const void* xs[2] = {k, q};
+        const void* sks[2] = {skw, skr};
+        const int tops[2] = {d->W, d->R};
+        int32_t* idxs[2] = {widx, ridx};
+        float* wts[2] = {ww, rw};
+        return launch_score_pk(d, 2, xs, sks, tops, idxs, wts, s);
+    }
     if (!(score_tc_eligible(d, d->W) && score_tc_eligible(d, d->R)) && score_rows_eligible(d)) {
         const void* xs[2] = {k, q};
         const void* sks[2] = {skw, skr};
@@ -451,6 +534,7 @@ sdm_status launch_score(const sdm_dims* d, const void* x, const void* sk, int to
                         float* w, cudaStream_t s) {
     const long long rows = (long long)d->B * d->T;
     if (rows == 0) return SDM_OK;
+    if (score_pk_eligible(d, top)) return launch_score_pk(d, 1, &x, &sk, &top, &idx, &w, s);
     if (score_tc_eligible(d, top)) return launch_score_tc(d, x, sk, top, idx, w, s);
     if (score_rows_eligible(d)) return launch_score_rows(d, 1, &x, &sk, &top, &idx, &w, s);
     const int threads = 128, warps = threads / 32;
@@ -629,6 +713,14 @@ sdm_status sdm_score_topk(const sdm_dims* dims, const void* x, const void* subke
     if (top < 1 || top > kMaxTop || top > dims->k_half * dims->k_half) return SDM_ERR_SHAPE;
     if (!aligned16(x) || !aligned16(subkeys) || !aligned16(idx) || !aligned16(w)) return SDM_ERR_ALIGN;
     return launch_score(dims, x, subkeys, top, idx, w, stream);
+}
+
+sdm_status sdm_score_qk(const sdm_dims* dims, const void* q, const void* k, const void* skw,
+                        const void* skr, int32_t* widx, float* ww, int32_t* ridx, float* rw,
+                        sdm_stream_t stream) {
+    const sdm_status e = check_dims(dims);
+    if (e) return e;
+    return score_both_roles(dims, q, k, skw, skr, widx, ww, ridx, rw, (cudaStream_t)stream);
 }
 
 size_t sdm_forward_workspace_bytes(const sdm_dims* dims) {

@@ -171,5 +171,27 @@ SDM_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 64 consecutive fp32 columns of this thread's TMEM lane: two loads, one wait.  The wait
+// names the destination registers so that no use can be scheduled before it.
+SDM_DEV void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+    uint32_t r[64];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr + 32u));
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0+0]), "+r"(r[0+1]), "+r"(r[0+2]), "+r"(r[0+3]), "+r"(r[0+4]), "+r"(r[0+5]), "+r"(r[0+6]), "+r"(r[0+7]), "+r"(r[0+8]), "+r"(r[0+9]), "+r"(r[0+10]), "+r"(r[0+11]), "+r"(r[0+12]), "+r"(r[0+13]), "+r"(r[0+14]), "+r"(r[0+15]), "+r"(r[0+16]), "+r"(r[0+17]), "+r"(r[0+18]), "+r"(r[0+19]), "+r"(r[0+20]), "+r"(r[0+21]), "+r"(r[0+22]), "+r"(r[0+23]), "+r"(r[0+24]), "+r"(r[0+25]), "+r"(r[0+26]), "+r"(r[0+27]), "+r"(r[0+28]), "+r"(r[0+29]), "+r"(r[0+30]), "+r"(r[0+31])
+                 :
+                 : "memory");
+    asm volatile(""
+                 : "+r"(r[32+0]), "+r"(r[32+1]), "+r"(r[32+2]), "+r"(r[32+3]), "+r"(r[32+4]), "+r"(r[32+5]), "+r"(r[32+6]), "+r"(r[32+7]), "+r"(r[32+8]), "+r"(r[32+9]), "+r"(r[32+10]), "+r"(r[32+11]), "+r"(r[32+12]), "+r"(r[32+13]), "+r"(r[32+14]), "+r"(r[32+15]), "+r"(r[32+16]), "+r"(r[32+17]), "+r"(r[32+18]), "+r"(r[32+19]), "+r"(r[32+20]), "+r"(r[32+21]), "+r"(r[32+22]), "+r"(r[32+23]), "+r"(r[32+24]), "+r"(r[32+25]), "+r"(r[32+26]), "+r"(r[32+27]), "+r"(r[32+28]), "+r"(r[32+29]), "+r"(r[32+30]), "+r"(r[32+31]));
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 }  // namespace ptx
 }  // namespace sdm

@@ -91,6 +91,21 @@ def test_score_vs_oracle(sdm, orc, wl):
     assert sdm.device_error() == 0
 
 
+@pytest.mark.parametrize("wl", [S.MID.scaled(B=2, H=2, T=300), S.TINY.scaled(B=2, H=2, T=100),
+                                S.HEADLINE.scaled(B=1, H=2, T=130)], ids=["mid", "tiny", "headline"])
+def test_score_qk_matches_score_topk(sdm, wl):
+    """Both roles in one call give exactly what two single-role calls give."""
+    inp = to_dev(S.generate(wl, with_m0=False))
+    d = dims_of(sdm, wl)
+    widx, ww, ridx, rw = sdm.score_qk(d, inp["q"], inp["k"], inp["skw"], inp["skr"])
+    wi2, ww2 = sdm.score_topk(d, inp["k"], inp["skw"], wl.W)
+    ri2, rw2 = sdm.score_topk(d, inp["q"], inp["skr"], wl.R)
+    torch.cuda.synchronize()
+    assert torch.equal(widx, wi2) and torch.equal(ridx, ri2)
+    assert torch.equal(ww, ww2) and torch.equal(rw, rw2)
+    assert sdm.device_error() == 0
+
+
 def test_score_brute_force_equivalence(sdm, orc):
     """k_half == top: GPU product-key selection equals the oracle's brute-force ranking."""
     wl = S.MID.scaled(B=1, H=1, T=64, n_sub=64, k_half=16, W=16, R=16)
