@@ -160,6 +160,17 @@ sdm_status sdm_score_topk(const sdm_dims* dims, const void* x, const void* subke
                           int32_t* idx, float* w, sdm_stream_t stream);
 
 /*
+ * Which scoring kernel sdm_score_topk / sdm_score_qk launch for `dims` and `top` (host-side
+ * query, no GPU work): SDM_SCORE_TC = the tensor-core kernel (TMA-fed tcgen05.mma into TMEM,
+ * exact per-row selection; bf16, d_k = 128, n_sub a multiple of 64 up to 1024, top <= k_half
+ * <= 64, T >= 64), SDM_SCORE_ROWS = the row scorer (short calls such as decode; n_sub <= 512),
+ * SDM_SCORE_WARP = one warp per row on CUDA cores (every other shape); negative: a status
+ * code (bad dims).
+ */
+enum { SDM_SCORE_TC = 1, SDM_SCORE_ROWS = 2, SDM_SCORE_WARP = 3 };
+int32_t sdm_score_path(const sdm_dims* dims, int32_t top);
+
+/*
  * Both scorings of one call: the keys against the write-role tables and the queries against
  * the read-role tables (§3 Method "Sparse addressing": keys choose the slots written,
  * queries the slots read), with the results of two sdm_score_topk calls but in one launch

@@ -85,6 +85,7 @@ def _load():
         "sdm_state_materialize": ([D, S, P, P], I32),
         "sdm_score_topk": ([D, P, P, I32, P, P, P], I32),
         "sdm_score_qk": ([D, P, P, P, P, P, P, P, P, P], I32),
+        "sdm_score_path": ([D, I32], I32),
         "sdm_forward_workspace_bytes": ([D], SZ),
         "sdm_forward": ([D, P, P, P, P, P, P, P, S, P, P, SZ, P], I32),
         "sdm_forward_plan": ([D, P, P, P, P, P, P, S, P, SZ, P], I32),
@@ -198,6 +199,18 @@ def score_topk(d: Dims, x, subkeys, top: int, idx=None, w=None, stream=None):
                             top, _ptr(idx, "idx", torch.int32), _ptr(w, "w", torch.float32),
                             _stream(stream)), "sdm_score_topk")
     return idx, w
+
+
+SCORE_TC, SCORE_ROWS, SCORE_WARP = 1, 2, 3
+
+
+def score_path(d: Dims, top: int) -> int:
+    """sdm_score_path: the scoring kernel a call of these dims launches (SCORE_TC: the
+    tensor-core kernel, SCORE_ROWS: the row scorer, SCORE_WARP: one warp per row)."""
+    r = int(_lib.sdm_score_path(ctypes.byref(d), top))
+    if r < 0:
+        raise SdmError(-r, "sdm_score_path")
+    return r
 
 
 def score_qk(d: Dims, q, k, skw, skr, sel=None, stream=None):

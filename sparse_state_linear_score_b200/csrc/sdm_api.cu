@@ -230,13 +230,13 @@ sdm_status launch_score_tc(const sdm_dims* d, const void* x, const void* sk, int
     return launch_score_tc_t<32>(d, xm, km, a, grid, s);
 }
 
-// Shapes the one-round tensor-core scorer takes: bf16, 64-wide halves, at most 256 sub-keys per
-// half (a multiple of 64), at most 32 kept per half, top <= k_half (the staircase), and calls
-// of at least 64 tokens (shorter ones go to the row scorer, which spreads rows over all SMs).
+// Shapes the tensor-core scorer takes: bf16, 64-wide halves, at most 1024 sub-keys per half (a
+// multiple of 64), at most 64 kept per half, top <= k_half (the staircase), and calls of at
+// least 64 tokens (shorter ones go to the row scorer, which spreads rows over all SMs).
 bool score_pk_eligible(const sdm_dims* d, int top) {
     if (d->x_dtype != SDM_BF16 || d->d_k != 128) return false;
     if (d->n_sub % 64 != 0 || d->n_sub > PK_NMAX) return false;
-    if (d->k_half > 32 || top > d->k_half) return false;
+    if (d->k_half > 64 || top > d->k_half) return false;
     return d->T >= 64;
 }
 
@@ -263,28 +263,31 @@ bool encode_sk_map(EncodeTiledFn enc, CUtensorMap* m, const sdm_dims* d, const v
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KP>
+template <int KP, int ROWS>
 sdm_status launch_score_pk_t(const CUtensorMap (&xm)[2], const CUtensorMap (&km)[2],
                              const PkArgs& a, dim3 grid, cudaStream_t s) {
-    auto kern = score_pk_kernel<KP>;
-    if (!set_smem(kern, PkCfg<KP>::SMEM)) return SDM_ERR_CUDA;
-    kern<<<grid, PK_THREADS, PkCfg<KP>::SMEM, s>>>(xm[0], xm[1], km[0], km[1], a);
+    auto kern = score_pk_kernel<KP, ROWS>;
+    constexpr size_t smem = PkCfg<KP, ROWS>::SMEM;
+    if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
+    kern<<<grid, 2 * ROWS, smem, s>>>(xm[0], xm[1], km[0], km[1], a);
     return launch_status();
 }
 
 // `roles` (1 or 2) scorings of the same shape in one launch (grid.z = role): role r scores
-// x[r] against sk[r] into idx[r], w[r] with top[r] slots.
+// x[r] against sk[r] into idx[r], w[r] with top[r] slots.  Lists of up to 32 per half take
+// tiles of 128 rows, longer ones tiles of 64 (their candidate lists fill the shared memory).
 sdm_status launch_score_pk(const sdm_dims* d, int roles, const void* const* x,
                            const void* const* sk, const int* top, int32_t* const* idx,
                            float* const* w, cudaStream_t s) {
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return SDM_ERR_CUDA;
+    const int rows = d->k_half <= 32 ? 128 : 64;
     PkArgs a{};
     a.B = d->B; a.H = d->H; a.T = d->T; a.n = d->n_sub; a.k_half = d->k_half; a.d_k = d->d_k;
-    // a tile is always 128 rows that the TMA fills: 128 tokens of one sequence, or 64 tokens of
-    // two when T = 64; rows past T or B are the load's zero fill and are not selected
-    a.bt = d->T == 64 ? 64 : 128;
-    a.bb = 128 / a.bt;
+    // a tile is always `rows` rows that the TMA fills: tokens of one sequence, or 64 tokens of
+    // two when T = 64 and rows = 128; rows past T or B are the load's zero fill, not selected
+    a.bt = (rows == 128 && d->T == 64) ? 64 : rows;
+    a.bb = rows / a.bt;
     a.n_tt = (d->T + a.bt - 1) / a.bt;
     a.z0 = pk_z0(d->n_sub, d->k_half);
     CUtensorMap xm[2], km[2];
@@ -296,12 +299,13 @@ sdm_status launch_score_pk(const sdm_dims* d, int roles, const void* const* x,
         a.idx[r] = idx[q];
         a.w[r] = w[q];
         if (!encode_x_map(enc, &xm[r], d, x[q], a.bt, a.bb)) return SDM_ERR_CUDA;
-        if (!encode_sk_map(enc, &km[r], d, sk[q], d->n_sub)) return SDM_ERR_CUDA;
+        if (!encode_sk_map(enc, &km[r], d, sk[q], d->n_sub < 256 ? d->n_sub : 256)) return SDM_ERR_CUDA;
     }
     const int n_bt = (d->B + a.bb - 1) / a.bb;
     const dim3 grid((unsigned)(a.n_tt * n_bt), (unsigned)d->H, (unsigned)roles);
-    if (d->k_half <= 16) return launch_score_pk_t<16>(xm, km, a, grid, s);
-    return launch_score_pk_t<32>(xm, km, a, grid, s);
+    if (d->k_half <= 16) return launch_score_pk_t<16, 128>(xm, km, a, grid, s);
+    if (d->k_half <= 32) return launch_score_pk_t<32, 128>(xm, km, a, grid, s);
+    return launch_score_pk_t<64, 64>(xm, km, a, grid, s);
 }
 
 // The row scorer keeps a lane's block of n/32 half-scores in registers (at most 16) and the
@@ -713,6 +717,15 @@ sdm_status sdm_score_topk(const sdm_dims* dims, const void* x, const void* subke
     if (top < 1 || top > kMaxTop || top > dims->k_half * dims->k_half) return SDM_ERR_SHAPE;
     if (!aligned16(x) || !aligned16(subkeys) || !aligned16(idx) || !aligned16(w)) return SDM_ERR_ALIGN;
     return launch_score(dims, x, subkeys, top, idx, w, stream);
+}
+
+int32_t sdm_score_path(const sdm_dims* dims, int32_t top) {
+    const sdm_status e = check_dims(dims);
+    if (e) return -(int32_t)e;
+    if (score_pk_eligible(dims, top)) return SDM_SCORE_TC;
+    if (score_tc_eligible(dims, top)) return SDM_SCORE_TC;
+    if (score_rows_eligible(dims)) return SDM_SCORE_ROWS;
+    return SDM_SCORE_WARP;
 }
 
 sdm_status sdm_score_qk(const sdm_dims* dims, const void* q, const void* k, const void* skw,

@@ -151,3 +151,22 @@ def test_backward_host_checks(lib):
     assert call(dims=mid_dims(d_k=30)) == 2                   # SDM_ERR_SHAPE
     assert lib.sdm_backward(ctypes.byref(d), p, p, p, p, p, p, p, ctypes.byref(st), p,
                             ctypes.c_void_p(0x1004), p, p, p, p, p, p, p, big, None) == 4
+
+
+def test_score_path_dispatch(lib):
+    """Which scorer each workload's shape takes (host-side query): every bf16 prefill shape of
+    the workloads, the long-context one (n = 1024, k = W = R = 64) included, goes to the
+    tensor-core kernel; decode steps (T = 1) to the row scorer; fp32 to the CUDA-core paths."""
+    import sparse_state_linear_score_b200 as sdm
+    import sdm_synth as S
+    for wl in (S.MID, S.HEADLINE, S.LONG):
+        d = sdm.Dims(wl.B, wl.H, wl.T, wl.d_k, wl.n_sub, wl.d_v, wl.k_half, wl.W, wl.R,
+                     wl.x_dtype, wl.v_dtype)
+        assert sdm.score_path(d, wl.W) == sdm.SCORE_TC, wl
+        assert sdm.score_path(d, wl.R) == sdm.SCORE_TC, wl
+        assert sdm.score_path(d.with_T(1), wl.W) == (sdm.SCORE_ROWS if wl.n_sub <= 512
+                                                     else sdm.SCORE_WARP)
+    wl = S.TINY
+    d = sdm.Dims(wl.B, wl.H, wl.T, wl.d_k, wl.n_sub, wl.d_v, wl.k_half, wl.W, wl.R,
+                 wl.x_dtype, wl.v_dtype)
+    assert sdm.score_path(d, wl.W) == sdm.SCORE_ROWS  # fp32

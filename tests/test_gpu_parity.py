@@ -106,6 +106,30 @@ def test_score_qk_matches_score_topk(sdm, wl):
     assert sdm.device_error() == 0
 
 
+@pytest.mark.parametrize("wl", [S.MID.scaled(B=1, H=2, T=300), S.LONG.scaled(B=1, H=1, T=100)],
+                         ids=["mid", "long"])
+def test_score_exact_ties(sdm, orc, wl):
+    """Sub-key tables whose rows come in identical pairs: every half-score has an exactly equal
+    twin and pair sums tie in groups of four, so the selections' boundaries fall on exact ties
+    again and again.  The oracle ranks exact ties by the lower index, as the kernel must: the
+    indices are compared bit for bit (no near-tie allowance)."""
+    inp = to_dev(S.generate(wl, with_m0=False))
+    for key in ("skw", "skr"):
+        sk = inp[key].clone()
+        sk[:, :, 1::2] = sk[:, :, 0::2]
+        inp[key] = sk.contiguous()
+    d = dims_of(sdm, wl)
+    for x, sk, top in ((inp["k"], inp["skw"], wl.W), (inp["q"], inp["skr"], wl.R)):
+        idx, w = sdm.score_topk(d, x, sk, top)
+        torch.cuda.synchronize()
+        idx_o, _, w_o = oracle_select(orc, x, sk, wl.k_half, top)
+        gi = idx.cpu().numpy()
+        same = np.all(gi == idx_o, axis=-1)
+        assert same.all(), f"{(~same).sum()} rows differ, first at {np.argwhere(~same)[:3].tolist()}"
+        check_err(float(np.abs(f64(w) - w_o).max()), 1e-5, "weights")
+    assert sdm.device_error() == 0
+
+
 def test_score_brute_force_equivalence(sdm, orc):
     """k_half == top: GPU product-key selection equals the oracle's brute-force ranking."""
     wl = S.MID.scaled(B=1, H=1, T=64, n_sub=64, k_half=16, W=16, R=16)
