@@ -343,6 +343,13 @@ def run_gpu(args, wl, world, rank, local):
     touched = run_touched(wl, inp, device, sdm) if rank == 0 else None
     bwd = run_backward(wl, inp, sel, device, sdm) if rank == 0 else None
     dec = run_decode(device, sdm) if rank == 0 and not args.no_decode else None
+    extra = {}
+    if rank == 0 and args.workloads:
+        del inp, st, sel, widx, ww, ridx, rw, out, ws
+        torch.cuda.empty_cache()
+        for name in [x for x in args.workloads.split(",") if x]:
+            extra[name] = run_workload(name, device, sdm,
+                                       cpu_seconds=0.0 if args.no_cpu_baseline else 10.0)
 
     if world > 1:
         dist.barrier(device_ids=[device.index])
@@ -392,6 +399,7 @@ def run_gpu(args, wl, world, rank, local):
         "diagnostics": diag,
         "layer_out": layer,
         "decode": dec,
+        "workloads": extra,
         "touched_decay": touched,
         "backward": bwd,
         "gpu_launches": launches_per_step * args.steps,
@@ -401,6 +409,87 @@ def run_gpu(args, wl, world, rank, local):
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     return line
+
+
+def run_workload(name: str, device, sdm, steps: int = 5, warm: int = 3,
+                 cpu_seconds: float = 10.0) -> dict:
+    """Another prefill workload at full size on one GPU: the same timed step as the headline
+    line (state reset, both scorings in one launch, plan, row pass), `steps` timed steps with
+    the L2 flushed between them, each stage timed by CUDA events; then a sampled CPU oracle
+    rate on a token prefix of one or two sequences (the full workloads hold 8-34 GB of memory
+    tables, and the oracle's rate per token.head does not depend on the number of
+    sequences)."""
+    import torch
+
+    import sdm_synth as S
+    wl = S.WORKLOADS[name]
+    stream = torch.cuda.current_stream()
+    inp = S.generate(wl, device=device)
+    d = sdm.Dims(wl.B, wl.H, wl.T, wl.d_k, wl.n_sub, wl.d_v, wl.k_half, wl.W, wl.R, wl.x_dtype,
+                 wl.v_dtype)
+    st = sdm.State(d, inp["M0"])
+    sel = sdm.selection_buffers(d, device)
+    widx, ww, ridx, rw = sel
+    out = torch.empty((wl.B, wl.H, wl.T, wl.d_v), dtype=torch.float32, device=device)
+    ws = sdm.workspace(d, device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        sdm.state_reset(d, st)
+        sdm.score_qk(d, inp["q"], inp["k"], inp["skw"], inp["skr"], sel)
+        if ev:
+            ev[1].record(stream)
+        sdm.forward_plan(d, inp["alpha"], inp["beta"], widx, ww, ridx, rw, st, ws)
+        if ev:
+            ev[2].record(stream)
+        sdm.forward_run(d, inp["v"], inp["beta"], widx, ww, ridx, rw, st, out, ws)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(warm):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for k in range(steps):
+        flush.zero_()
+        step(evs[k])
+    torch.cuda.synchronize()
+    errs = sdm.device_error()
+    step_ms = statistics.mean(e[0].elapsed_time(e[3]) for e in evs)
+    score_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    plan_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    run_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    units = units_per_step(wl)
+    bpt = bytes_per_token_head(wl)
+    peak = measured_peaks()["hbm_gbs"]
+    step_gbs = bpt["step"] * units / (step_ms / 1e3) / 1e9
+    run_gbs = bpt["recurrence_kernel"] * units / (run_ms / 1e3) / 1e9
+    flops = scoring_flops_per_token_head(wl) * units
+    res = {"workload": describe(wl), "steps_timed": steps, "ms_per_step": step_ms,
+           "token_heads_per_s": units / (step_ms / 1e3),
+           "stages_ms": {"reset_and_scoring": score_ms, "plan": plan_ms, "run": run_ms},
+           "step_roofline": {"bytes_per_token_head": bpt["step"], "achieved_gbs": step_gbs,
+                             "peak": peak, "frac": step_gbs / peak,
+                             "roofline_ms": bpt["step"] * units / (peak * 1e9) * 1e3},
+           "row_pass": {"algorithmic_bytes": bpt["recurrence_kernel"] * units,
+                        "achieved_gbs": run_gbs, "frac": run_gbs / peak},
+           "scoring": {"rows": 2 * units, "ms": score_ms,
+                       "tflops": flops / (score_ms / 1e3) / 1e12,
+                       "path": "tensor cores" if sdm.score_path(d, wl.W) == sdm.SCORE_TC
+                       else "CUDA cores"},
+           "l2": "flushed between timed steps", "device_errors": errs}
+    del inp, st, sel, out, ws, flush
+    torch.cuda.empty_cache()
+    if cpu_seconds > 0:
+        samp = wl.scaled(B=1, H=min(wl.H, 2))
+        cb = cpu_baseline(samp, seconds=cpu_seconds)
+        cb["sample"] = cb["sample"] + f"; the {wl.name} workload has {wl.B * wl.H} sequences"
+        cb["kind"] = "oracle (sampled)"
+        res["cpu_baseline"] = cb
+    return res
 
 
 def run_decode(device, sdm, steps: int = 64, warm: int = 3, n_sub: int | None = None,
@@ -781,6 +870,9 @@ def main(argv=None):
     ap.add_argument("--workload", default="mid_prefill")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workloads", default="headline_prefill,long_context",
+                    help="other prefill workloads measured after the timed step (rank 0), "
+                         "comma-separated; empty for none")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the decode-workload measurement (rank 0)")
     ap.add_argument("--decode-only", action="store_true",
