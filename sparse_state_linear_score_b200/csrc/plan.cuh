@@ -110,6 +110,7 @@ struct PlanPtrs {
     int32_t* lk;       // [BH][T*(W+R)]
     uint32_t* occw;    // [BH][T*(W+R)] slot | OCC_OWNER (the walk's input)
     unsigned long long* mask;  // [BH][N][MW] chunks of this call that stored each slot, or null
+    short* wtab;               // [BH][N] the walk's last storing chunk of each slot (no masks)
     int MW;                    // 64-bit words per slot in mask
     // the row pass's inputs, packed by plan_pack
     int32_t* rs;          // [BH][T*(W+R)] chunk j at j*C*(W+R), in-chunk occurrence order:
@@ -517,31 +518,29 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_fe_kernel(double* __restric
     }
 }
 
-// Sequential walk over the chunks of one (b,h), split over WALK_PARTS CTAs by slot
-// (slot % WALK_PARTS): each CTA keeps, for its slots only, the last chunk of this call that
-// wrote them (-1: none) in shared memory, and streams the chunks' packed occurrence words
-// and token prefixes through a ring filled WALK_RING chunks ahead by cp.async.
-constexpr int WALK_PARTS = 16;
-
+// Sequential walk over the chunks of one (b,h), split over `parts` CTAs by slot (slot % parts):
+// the last chunk of this call that stored each slot (-1: none) is kept in P.wtab (int16 per
+// slot in global memory, 2 bytes a slot: it stays in L2), so the CTAs need only the ring that
+// streams the chunks' packed occurrence words and token prefixes, filled WALK_RING chunks
+// ahead by cp.async, and every walk of the call runs at once.  Two barriers per chunk: after
+// the chunk's words land (the previous chunk's table writes are then visible, and the ring
+// stage it used may be refilled) and between the chunk's lookups and its own writes.
 __global__ void __launch_bounds__(WALK_THREADS) plan_walk_kernel(
-    double* __restrict__ stamp, int T, int N, int W, int R, int C, int J, int lstart_smem,
-    PlanPtrs P) {
+    double* __restrict__ stamp, int T, int N, int W, int R, int C, int J, int parts,
+    int lstart_smem, PlanPtrs P) {
     extern __shared__ __align__(16) unsigned char walk_smem[];
     const int part = blockIdx.x;
     const size_t bh = blockIdx.y;
     const int tid = threadIdx.x;
     const int stage = PLAN_MAX_OCC + PLAN_MAX_C;  // words per ring stage
-    const int nslot = (N + WALK_PARTS - 1) / WALK_PARTS;
     uint32_t* s_ring = reinterpret_cast<uint32_t*>(walk_smem);  // [WALK_RING][stage]
     double* s_L = reinterpret_cast<double*>(s_ring + WALK_RING * stage);  // [J+1] if lstart_smem
-    short* s_tab = reinterpret_cast<short*>(s_L + (lstart_smem ? J + 1 : 0));  // [nslot]
+    short* tab = P.wtab + bh * (size_t)N;
     const double* Lg = P.Lstart + bh * (size_t)(J + 1);
-    const size_t occ_base = bh * (size_t)T * (W + R);
-
     if (lstart_smem)
         for (int i = tid; i <= J; i += WALK_THREADS) s_L[i] = Lg[i];
-    for (int i = tid; i < nslot; i += WALK_THREADS) s_tab[i] = -1;
     const double* Lr = lstart_smem ? s_L : Lg;
+    const size_t occ_base = bh * (size_t)T * (W + R);
 
     auto load_stage = [&](int jn) {
         if (jn < J) {
@@ -564,22 +563,29 @@ __global__ void __launch_bounds__(WALK_THREADS) plan_walk_kernel(
         cp_async_commit();  // one group per stage, empty past the end
     };
 
-    __syncthreads();
     for (int s = 0; s < WALK_RING - 1; ++s) load_stage(s);
     for (int j = 0; j < J; ++j) {
-        load_stage(j + WALK_RING - 1);
-        asm volatile("cp.async.wait_group %0;\n" ::"n"(WALK_RING - 1) : "memory");
+        asm volatile("cp.async.wait_group %0;\n" ::"n"(WALK_RING - 2) : "memory");
         __syncthreads();
+        load_stage(j + WALK_RING - 1);  // into the stage chunk j - 1 used (finished by now)
         const uint32_t* ow = s_ring + (j % WALK_RING) * stage;
         const float* lamc = reinterpret_cast<const float*>(ow + PLAN_MAX_OCC);
         const int t0 = j * C, nt = min(C, T - t0), nw = nt * W, no = nt * (W + R);
         const double Lj = Lr[j];
-        // rows of slots written by an earlier chunk carry that chunk's end stamp
-        for (int o = tid; o < no; o += WALK_THREADS) {
-            const int s = (int)(ow[o] & OCC_SLOT);
-            if (s >= N || s % WALK_PARTS != part) continue;
-            const int jw = s_tab[s / WALK_PARTS];
-            if (jw < 0) continue;
+        // rows of slots written by an earlier chunk carry that chunk's end stamp: the table
+        // entries of this thread's occurrences are all requested before any is used
+        constexpr int PO = PLAN_MAX_OCC / WALK_THREADS;
+        int jw[PO];
+#pragma unroll
+        for (int k = 0; k < PO; ++k) {
+            const int o = tid + k * WALK_THREADS;
+            const int s = o < no ? (int)(ow[o] & OCC_SLOT) : N;
+            jw[k] = (s < N && s % parts == part) ? (int)tab[s] : -1;
+        }
+#pragma unroll
+        for (int k = 0; k < PO; ++k) {
+            const int o = tid + k * WALK_THREADS;
+            if (jw[k] < 0) continue;
             int t;
             size_t g;
             if (o < nw) {
@@ -589,26 +595,26 @@ __global__ void __launch_bounds__(WALK_THREADS) plan_walk_kernel(
                 t = (o - nw) / R;
                 g = occ_base + (size_t)T * W + (size_t)t0 * R + (o - nw);
             }
-            P.fe[g] = expf((float)(Lj - Lr[jw + 1]) + lamc[t]);
+            P.fe[g] = expf((float)(Lj - Lr[jw[k] + 1]) + lamc[t]);
         }
         __syncthreads();
         for (int o = tid; o < nw; o += WALK_THREADS) {
             const uint32_t w = ow[o];
             const int s = (int)(w & OCC_SLOT);
-            if (!(w & OCC_OWNER) || s >= N || s % WALK_PARTS != part) continue;
-            s_tab[s / WALK_PARTS] = (short)j;
+            if (!(w & OCC_OWNER) || s >= N || s % parts != part) continue;
+            tab[s] = (short)j;
         }
-        __syncthreads();
     }
     asm volatile("cp.async.wait_all;\n" ::: "memory");
 
+    __syncthreads();
     // final stamps of this partition's slots written in this call
     for (size_t o = tid; o < (size_t)T * W; o += WALK_THREADS) {
         const uint32_t w = P.occw[occ_base + o];
         const int s = (int)(w & OCC_SLOT);
-        if (!(w & OCC_OWNER) || s >= N || s % WALK_PARTS != part) continue;
+        if (!(w & OCC_OWNER) || s >= N || s % parts != part) continue;
         const int j = (int)(o / W) / C;
-        if (s_tab[s / WALK_PARTS] == j) stamp[bh * (size_t)N + s] = Lr[j + 1];
+        if (tab[s] == j) stamp[bh * (size_t)N + s] = Lr[j + 1];
     }
 }
 

@@ -64,9 +64,10 @@ int chunk_tokens(const sdm_dims* d) {
 
 struct WsLayout {
     int C, J;
+    int walk_parts;
     bool lstart_smem;
     size_t walk_smem;
-    size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_occw, off_mask;
+    size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_occw, off_mask, off_wtab;
     size_t off_rs, off_img, off_vfc, off_vsh, total;
     int MW;  // mask words per slot, 0 when the walk is used
 };
@@ -79,10 +80,14 @@ WsLayout ws_layout(const sdm_dims* d) {
     const size_t occ = T * (size_t)(d->W + d->R);
     L.C = chunk_tokens(d);
     L.J = (int)((T + L.C - 1) / L.C);
+    // the walk: one CTA per (b,h) and slot partition, the chunk-start prefixes in shared memory
+    // when they fit; as many partitions as keep every walk of the call in one wave
     const size_t ring = (size_t)WALK_RING * (PLAN_MAX_OCC + PLAN_MAX_C) * 4;
-    const size_t tab_bytes = ((N + WALK_PARTS - 1) / WALK_PARTS) * 2;
-    L.lstart_smem = ring + (size_t)(L.J + 1) * 8 + tab_bytes <= kSmemBudget;
-    L.walk_smem = ring + (L.lstart_smem ? (size_t)(L.J + 1) * 8 : 0) + tab_bytes;
+    L.lstart_smem = ring + (size_t)(L.J + 1) * 8 <= kSmemBudget;
+    L.walk_smem = ring + (L.lstart_smem ? (size_t)(L.J + 1) * 8 : 0);
+    const size_t per_sm = (size_t)(228 * 1024) / (L.walk_smem + 1024);
+    L.walk_parts = (int)(148 * (per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm)) / BH);
+    L.walk_parts = L.walk_parts < 1 ? 1 : (L.walk_parts > 16 ? 16 : L.walk_parts);
     size_t o = 0;
     L.off_lam = o;    o = up256(o + BH * T * 4);
     L.off_csum = o;   o = up256(o + BH * L.J * 8);
@@ -95,6 +100,7 @@ WsLayout ws_layout(const sdm_dims* d) {
     const size_t mw = (size_t)(L.J + 63) / 64;
     L.MW = (L.J <= 512 && BH * N * mw * 8 <= kMaskBudget) ? (int)mw : 0;
     L.off_mask = o;   o = up256(o + BH * N * (size_t)L.MW * 8);
+    L.off_wtab = o;   o = up256(o + (L.MW ? 0 : BH * N * 2));
     L.off_rs = o;     o = up256(o + BH * occ * 4);
     L.off_img = o;    o = up256(o + BH * (size_t)L.J * run_img(L.C, d->W, d->R).bytes);
     // touched-slots decay: in-chunk decay products of each occurrence (see PlanPtrs)
@@ -117,6 +123,7 @@ PlanPtrs plan_ptrs(const WsLayout& L, void* ws) {
     P.occw = reinterpret_cast<uint32_t*>(b + L.off_occw);
     P.mask = L.MW ? reinterpret_cast<unsigned long long*>(b + L.off_mask) : nullptr;
     P.MW = L.MW;
+    P.wtab = L.MW ? nullptr : reinterpret_cast<short*>(b + L.off_wtab);
     P.rs = reinterpret_cast<int32_t*>(b + L.off_rs);
     P.img = b + L.off_img;
     const bool touched = L.off_vsh != L.off_vfc;
@@ -775,9 +782,12 @@ sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const floa
         plan_fe_kernel<<<dim3((unsigned)L.J, (unsigned)BH), PLAN_THREADS, 0, stream>>>(
             st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, P);
         if ((e = launch_status())) return e;
+        if (cudaMemsetAsync(P.wtab, 0xff, BH * (size_t)N * 2, stream) != cudaSuccess)
+            return SDM_ERR_CUDA;
         if (!set_smem(plan_walk_kernel, L.walk_smem)) return SDM_ERR_CUDA;
-        plan_walk_kernel<<<dim3(WALK_PARTS, (unsigned)BH), WALK_THREADS, L.walk_smem, stream>>>(
-            st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J, L.lstart_smem ? 1 : 0, P);
+        plan_walk_kernel<<<dim3((unsigned)L.walk_parts, (unsigned)BH), WALK_THREADS, L.walk_smem,
+                           stream>>>(st->stamp, dims->T, N, dims->W, dims->R, L.C, L.J,
+                                     L.walk_parts, L.lstart_smem ? 1 : 0, P);
         if ((e = launch_status())) return e;
     }
     // with the masks, plan_pack computes the final factors and stamps itself
