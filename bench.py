@@ -318,6 +318,22 @@ def run_gpu(args, wl, world, rank, local):
         e1.record(stream)
         torch.cuda.synchronize()
         res["layer_in"] = e0.elapsed_time(e1) / 10
+        # the output side's RMS-norm and gate fused into the row pass (its read): the row pass
+        # with the epilogue, then the projection alone
+        abuf = torch.empty(wl.B, wl.T, wl.H * wl.d_v, dtype=torch.bfloat16, device=device)
+        gms = []
+        for k in range(6):
+            sdm.state_reset(d, st)
+            sdm.score_qk(d, inp["q"], inp["k"], inp["skw"], inp["skr"], sel)
+            sdm.forward_plan(d, inp["alpha"], inp["beta"], widx, ww, ridx, rw, st, ws)
+            e0.record(stream)
+            sdm.forward_run_gated(d, inp["v"], inp["beta"], widx, ww, ridx, rw, st, gate, wn,
+                                  1e-6, out=out, a=abuf, ws=ws)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if k > 0:
+                gms.append(e0.elapsed_time(e1))
+        res["run_gated"] = statistics.mean(gms)
         flops = 2.0 * wl.B * wl.T * wl.H * wl.d_v * dm
         tf = flops / (res["gemm"] / 1e3) / 1e12
         tf_in = 2.0 * wl.B * wl.T * wl.H * hs * dm / (res["layer_in"] / 1e3) / 1e12
@@ -329,6 +345,12 @@ def run_gpu(args, wl, world, rank, local):
                  ((res["layer_in"] + st_ms + res["layer_out"]) / 1e3),
                  "gemm_out": {"M": wl.B * wl.T, "K": wl.H * wl.d_v, "N": dm, "ms": res["gemm"],
                               "tflops": tf, "frac_of_bf16_peak": tf / pk},
+                 "fused_into_read": {
+                     "run_gated_ms": res["run_gated"], "run_ms": statistics.mean(run_ms),
+                     "epilogue_ms": res["run_gated"] - statistics.mean(run_ms),
+                     "layer_out_ms": res["run_gated"] - statistics.mean(run_ms) + res["gemm"],
+                     "note": "sdm_forward_run_gated: the RMS-norm and gate by the last column "
+                             "slice to finish each chunk; then the projection alone"},
                  "gemm_in_with_split": {"M": wl.B * wl.T, "K": dm, "N": wl.H * hs,
                                         "ms": res["layer_in"], "tflops": tf_in,
                                         "frac_of_bf16_peak": tf_in / pk},

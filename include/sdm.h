@@ -331,6 +331,26 @@ sdm_status sdm_forward_noalloc(const sdm_dims* dims, const void* v, const float*
                                float* out, sdm_stream_t stream);
 
 /*
+ * sdm_forward_run with the first step of the layer's output side fused into the read (§3
+ * Method "Sparse retrieval": the read result is RMS-normalised and elementwise gated, then
+ * mixed across heads by the output projection).  Besides out, it writes the projection's
+ * operand
+ *   a[b,t][h*d_v + c] = o_c / sqrt(mean_c o_c^2 + eps) * wn[c] * swish(g[b,t][h*d_v + c])
+ *                       with o = out[b][h][t][:], swish(z) = z * sigmoid(z)
+ * so that y = a @ Wo is one sdm_gemm_bf16(B*T, d_model, H*d_v, a, Wo_t, y).  The column
+ * slices of a sequence finish each chunk in any order; the last to finish a chunk normalises
+ * its tokens (no slice waits for another).
+ *   g  [B][T][H*d_v] bf16 (the gate's pre-activation); wn [d_v] fp32; eps >= 0
+ *   a  [B][T][H*d_v] bf16 out
+ * Other arguments, workspace and errors as sdm_forward_run.
+ */
+sdm_status sdm_forward_run_gated(const sdm_dims* dims, const void* v, const float* beta,
+                                 const int32_t* widx, const float* ww, const int32_t* ridx,
+                                 const float* rw, const sdm_state* st, float* out, const void* g,
+                                 const float* wn, float eps, void* a, void* ws, size_t ws_bytes,
+                                 sdm_stream_t stream);
+
+/*
  * Dense GEMM on the tensor cores (tcgen05, bf16 operands, fp32 accumulation):
  *   C[M][N] fp32 = A[M][K] x Bt[N][K]^T,  A and Bt bf16 row-major (K contiguous)
  * K a multiple of 8; M, N free.  Pointers 16-byte aligned.  One launch.

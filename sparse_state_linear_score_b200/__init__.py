@@ -22,7 +22,8 @@ import torch
 from . import build as _build
 
 __all__ = ["Dims", "State", "SdmError", "state_reset", "state_materialize", "score_topk", "score_qk",
-           "forward_workspace_bytes", "forward", "forward_noalloc", "forward_plan", "forward_run", "prefill",
+           "forward_workspace_bytes", "forward", "forward_noalloc", "forward_plan", "forward_run",
+           "forward_run_gated", "prefill",
            "decode_step", "device_error", "weight_stats", "gemm_bf16", "layer_in", "layer_out", "lib_path",
            "DEVERR_SLOT_RANGE",
            "DEVERR_DUP_WRITE", "DEVERR_ALPHA"]
@@ -90,6 +91,8 @@ def _load():
         "sdm_forward": ([D, P, P, P, P, P, P, P, S, P, P, SZ, P], I32),
         "sdm_forward_plan": ([D, P, P, P, P, P, P, S, P, SZ, P], I32),
         "sdm_forward_run": ([D, P, P, P, P, P, P, S, P, P, SZ, P], I32),
+        "sdm_forward_run_gated": ([D, P, P, P, P, P, P, S, P, P, P, ctypes.c_float, P, P, SZ, P],
+                                  I32),
         "sdm_prefill": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P, SZ, P], I32),
         "sdm_decode_step": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P], I32),
         "sdm_device_error": ([ctypes.POINTER(ctypes.c_uint32), I32, P], I32),
@@ -453,6 +456,30 @@ def layer_out(d: Dims, o: torch.Tensor, g: torch.Tensor, wn: torch.Tensor, Wo_t:
                            _ptr(y, "y", torch.float32), _ptr(ws, "ws"), ws.numel(),
                            _stream(stream)), "sdm_layer_out")
     return y
+
+
+def forward_run_gated(d: Dims, v, beta, widx, ww, ridx, rw, st: State, g, wn, eps: float = 1e-6,
+                      out=None, a=None, ws=None, stream=None):
+    """sdm_forward_run_gated: the row pass (after forward_plan on the same ws) with the layer
+    output side's RMS-norm and swish gate fused into the read.  g [B,T,H*d_v] bf16, wn [d_v]
+    fp32.  Returns (out [B,H,T,d_v] fp32, a [B,T,H*d_v] bf16); y = gemm_bf16(a, Wo_t)."""
+    dev = v.device
+    if out is None:
+        out = torch.empty((d.B, d.H, d.T, d.d_v), dtype=torch.float32, device=dev)
+    if a is None:
+        a = torch.empty((d.B, d.T, d.H * d.d_v), dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        raise ValueError("forward_run_gated needs the workspace forward_plan filled")
+    _ok(_lib.sdm_forward_run_gated(ctypes.byref(d), _ptr(v, "v", _vdt(d)),
+                                   _ptr(beta, "beta", torch.float32),
+                                   _ptr(widx, "widx", torch.int32), _ptr(ww, "ww", torch.float32),
+                                   _ptr(ridx, "ridx", torch.int32), _ptr(rw, "rw", torch.float32),
+                                   ctypes.byref(st.c),
+                                   _ptr(out, "out", torch.float32), _ptr(g, "g", torch.bfloat16),
+                                   _ptr(wn, "wn", torch.float32), float(eps),
+                                   _ptr(a, "a", torch.bfloat16), _ptr(ws, "ws"), ws.numel(),
+                                   _stream(stream)), "sdm_forward_run_gated")
+    return out, a
 
 
 def layer_in(d: Dims, x: torch.Tensor, Win_t: torch.Tensor, A_log: torch.Tensor,

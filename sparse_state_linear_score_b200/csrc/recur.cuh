@@ -74,14 +74,96 @@ __host__ __device__ inline size_t run_smem_bytes(int C, int W, int R, int CW, in
     b += (size_t)2 * run_vst_bytes(C, CW, vbytes);   // values, two chunks
     b += (size_t)3 * C * CW * 4;                     // rhs, d, Q0
     b += 16;                                         // mbarrier
+    b += 16;                                         // the epilogue's flag
     return b;
 }
 
-template <int CW, typename VT>
+// Optional epilogue of the row pass: the layer output side's RMS-norm and swish gate (§3
+// Method "Sparse retrieval"; the same arithmetic as layer_prologue_kernel)
+//   a[b,t][h*d_v + c] = o_c / sqrt(mean_c o_c^2 + eps) * wn[c] * swish(g[b,t][h*d_v + c])
+// needs a token's whole row, which d_v / CW column slices produce.  Each slice counts itself
+// finished with a chunk (an acquire-release atomic after its outputs); the slice that completes
+// the count reads the chunk's rows back (from L2) and writes a.  No slice waits for another.
+struct RunEpi {
+    const __nv_bfloat16* g;  // [B][T][H*d_v] gate pre-activation; null: no epilogue
+    const float* wn;         // [d_v] RMS-norm weight
+    float eps;
+    __nv_bfloat16* a;        // [B][T][H*d_v] out (bf16: the output projection's operand)
+    int* cnt;                // [B*H][J] slices finished with each chunk, zero at launch
+};
+
+// Atomic add with acquire-release semantics at GPU scope (returns the old value).
+SDM_DEV int atom_add_acq_rel(int* p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+                 : "memory");
+    return old;
+}
+
+// The epilogue of tokens t0..t0+nt-1 (nt <= 32) of sequence bh by the consumer warps: warp cw
+// takes tokens cw, cw+8, cw+16, cw+24, and every load of its four tokens (the rows from L2, the
+// gates) is issued before any is used.
+SDM_DEV void run_epilogue(const RunEpi& ep, const float* out, size_t bh, int H, int T, int d_v,
+                          int t0, int nt, int cw, int lane) {
+    constexpr int TPW = PLAN_MAX_C / (RUN_CONSUMERS / 32);  // tokens per consumer warp
+    const int b = (int)(bh / H), h = (int)(bh % H);
+    float4 x[TPW][2];
+    uint2 gr[TPW][2];
+#pragma unroll
+    for (int u = 0; u < TPW; ++u) {
+        const int t = cw + u * (RUN_CONSUMERS / 32);
+        const float4* orow = reinterpret_cast<const float4*>(out + (bh * T + t0 + t) * d_v);
+        const size_t grow = (((size_t)b * T + t0 + t) * H + h) * d_v;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int c4 = lane + 32 * k;
+            const bool in = t < nt && 4 * c4 < d_v;
+            x[u][k] = in ? __ldcg(orow + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            gr[u][k] = in ? *reinterpret_cast<const uint2*>(ep.g + grow + 4 * c4) : make_uint2(0, 0);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < TPW; ++u) {
+        const int t = cw + u * (RUN_CONSUMERS / 32);
+        float ss = 0.f;
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+            ss = fmaf(x[u][k].x, x[u][k].x, fmaf(x[u][k].y, x[u][k].y,
+                 fmaf(x[u][k].z, x[u][k].z, fmaf(x[u][k].w, x[u][k].w, ss))));
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+        if (t >= nt) continue;
+        const float r = rsqrtf(ss / (float)d_v + ep.eps);
+        const size_t grow = (((size_t)b * T + t0 + t) * H + h) * d_v;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int c = 4 * (lane + 32 * k);
+            if (c >= d_v) continue;
+            const float4 w4 = *reinterpret_cast<const float4*>(ep.wn + c);
+            const float xs[4] = {x[u][k].x, x[u][k].y, x[u][k].z, x[u][k].w};
+            const float ws[4] = {w4.x, w4.y, w4.z, w4.w};
+            const unsigned gw[2] = {gr[u][k].x, gr[u][k].y};
+            unsigned short ab[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float z = __bfloat162float(
+                    __ushort_as_bfloat16((unsigned short)(gw[e >> 1] >> ((e & 1) * 16))));
+                const float sw = z / (1.f + expf(-z));
+                ab[e] = __bfloat16_as_ushort(__float2bfloat16_rn(xs[e] * r * ws[e] * sw));
+            }
+            *reinterpret_cast<uint2*>(ep.a + grow + c) =
+                make_uint2((unsigned)ab[0] | ((unsigned)ab[1] << 16),
+                           (unsigned)ab[2] | ((unsigned)ab[3] << 16));
+        }
+    }
+}
+
+template <int CW, typename VT, bool EPI>
 __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
     const VT* __restrict__ v, const int32_t* __restrict__ rs,
     const unsigned char* __restrict__ imgs, float* __restrict__ M, const float* __restrict__ M0,
-    float* __restrict__ out, int H, int T, int N, int d_v, int W, int R, int C, int J) {
+    float* __restrict__ out, int H, int T, int N, int d_v, int W, int R, int C, int J,
+    RunEpi ep) {
     constexpr int Q = CW / 4;
     extern __shared__ __align__(16) unsigned char run_smem[];
     const int ncb = d_v / CW;
@@ -106,6 +188,7 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
     float* s_d = s_rhs + C * CW;
     float* s_q = s_d + C * CW;
     uint64_t* bar_img = reinterpret_cast<uint64_t*>(s_q + C * CW);
+    int* s_last = reinterpret_cast<int*>(bar_img + 1);  // this slice finished a chunk last
 
     if (tid == 0) {
         ptx::mbar_init(bar_img, 1);
@@ -316,6 +399,13 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
             }
         }
         named_sync(BAR_CONS, RUN_CONSUMERS);
+        if (EPI) {
+            // one acquire-release count per slice and chunk, after the barrier that orders every
+            // consumer's output stores before it: it publishes them and, for the last slice,
+            // makes the other slices' stores visible to the consumers after the next barrier
+            // (the epilogue itself follows the chunk's memory stores, below)
+            if (ctid == 0) *s_last = atom_add_acq_rel(ep.cnt + bh * J + j, 1) == ncb - 1;
+        }
         // 4. the stores of the chunk's last writes (also written back to the rows, from where
         //    the next chunk takes the ones it gathered before they were stored)
         //    The Q 16-byte pieces of a slice are handled by adjacent lanes, so that one store
@@ -370,6 +460,10 @@ __global__ void __launch_bounds__(RUN_THREADS, 1) recur_run_kernel(
         }
         // the stores precede the gathers that follow the next BAR_FIXED arrival
         __threadfence_block();
+        if (EPI) {
+            named_sync(BAR_CONS, RUN_CONSUMERS);
+            if (*s_last) run_epilogue(ep, out, bh, H, T, d_v, t0, nt, ctid >> 5, tid & 31);
+        }
     }
 }
 

@@ -67,7 +67,8 @@ struct WsLayout {
     int walk_parts;
     bool lstart_smem;
     size_t walk_smem;
-    size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_occw, off_mask, off_wtab;
+    size_t off_lam, off_csum, off_Lstart, off_st0, off_fe, off_lk, off_occw, off_mask, off_wtab,
+        off_cnt;
     size_t off_rs, off_img, off_vfc, off_vsh, total;
     int MW;  // mask words per slot, 0 when the walk is used
 };
@@ -101,6 +102,7 @@ WsLayout ws_layout(const sdm_dims* d) {
     L.MW = (L.J <= 512 && BH * N * mw * 8 <= kMaskBudget) ? (int)mw : 0;
     L.off_mask = o;   o = up256(o + BH * N * (size_t)L.MW * 8);
     L.off_wtab = o;   o = up256(o + (L.MW ? 0 : BH * N * 2));
+    L.off_cnt = o;    o = up256(o + BH * (size_t)L.J * 4);
     L.off_rs = o;     o = up256(o + BH * occ * 4);
     L.off_img = o;    o = up256(o + BH * (size_t)L.J * run_img(L.C, d->W, d->R).bytes);
     // touched-slots decay: in-chunk decay products of each occurrence (see PlanPtrs)
@@ -572,14 +574,14 @@ template <int CW, typename VT>
 sdm_status launch_run_t(const sdm_dims* d, const WsLayout& L, const PlanPtrs& P, const void* v,
                         const float* beta, const int32_t* widx, const float* ww,
                         const int32_t* ridx, const float* rw, const sdm_state* st, float* out,
-                        cudaStream_t s) {
+                        const RunEpi& ep, cudaStream_t s) {
     const size_t smem = run_smem_bytes(L.C, d->W, d->R, CW, (int)sizeof(VT));
-    auto kern = recur_run_kernel<CW, VT>;
+    auto kern = ep.g ? recur_run_kernel<CW, VT, true> : recur_run_kernel<CW, VT, false>;
     if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
     const long long grid = BH_of(d) * (d->d_v / CW);
     kern<<<(unsigned)grid, RUN_THREADS, smem, s>>>(
         (const VT*)v, P.rs, P.img, st->M, st->M0, out, d->H, d->T, (int)N_of(d), d->d_v,
-        d->W, d->R, L.C, L.J);
+        d->W, d->R, L.C, L.J, ep);
     return launch_status();
 }
 
@@ -797,10 +799,15 @@ sdm_status sdm_forward_plan(const sdm_dims* dims, const float* alpha, const floa
     return launch_status();
 }
 
-sdm_status sdm_forward_run(const sdm_dims* dims, const void* v, const float* beta,
-                           const int32_t* widx, const float* ww, const int32_t* ridx,
-                           const float* rw, const sdm_state* st, float* out, void* ws,
-                           size_t ws_bytes, sdm_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The row pass, with the layer epilogue when ep.g is set.
+sdm_status forward_run_impl(const sdm_dims* dims, const void* v, const float* beta,
+                            const int32_t* widx, const float* ww, const int32_t* ridx,
+                            const float* rw, const sdm_state* st, float* out, RunEpi ep, void* ws,
+                            size_t ws_bytes, cudaStream_t stream) {
     sdm_status e = check_dims(dims);
     if (e) return e;
     if ((e = check_state(st))) return e;
@@ -813,15 +820,49 @@ sdm_status sdm_forward_run(const sdm_dims* dims, const void* v, const float* bet
     if (!ws || ws_bytes < L.total) return SDM_ERR_WORKSPACE;
     if (!aligned16(ws)) return SDM_ERR_ALIGN;
     const PlanPtrs P = plan_ptrs(L, ws);
+    if (ep.g) {
+        ep.cnt = reinterpret_cast<int*>(static_cast<unsigned char*>(ws) + L.off_cnt);
+        if (cudaMemsetAsync(ep.cnt, 0, (size_t)BH_of(dims) * L.J * 4, stream) != cudaSuccess)
+            return SDM_ERR_CUDA;
+    }
     const int CW = col_width(dims);
     if (CW == 8) {
         if (dims->v_dtype == SDM_BF16)
-            return launch_run_t<8, __nv_bfloat16>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, stream);
-        return launch_run_t<8, float>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, stream);
+            return launch_run_t<8, __nv_bfloat16>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, ep, stream);
+        return launch_run_t<8, float>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, ep, stream);
     }
     if (dims->v_dtype == SDM_BF16)
-        return launch_run_t<4, __nv_bfloat16>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, stream);
-    return launch_run_t<4, float>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, stream);
+        return launch_run_t<4, __nv_bfloat16>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, ep, stream);
+    return launch_run_t<4, float>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, ep, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+sdm_status sdm_forward_run(const sdm_dims* dims, const void* v, const float* beta,
+                           const int32_t* widx, const float* ww, const int32_t* ridx,
+                           const float* rw, const sdm_state* st, float* out, void* ws,
+                           size_t ws_bytes, sdm_stream_t stream) {
+    return forward_run_impl(dims, v, beta, widx, ww, ridx, rw, st, out, RunEpi{}, ws, ws_bytes,
+                            (cudaStream_t)stream);
+}
+
+sdm_status sdm_forward_run_gated(const sdm_dims* dims, const void* v, const float* beta,
+                                 const int32_t* widx, const float* ww, const int32_t* ridx,
+                                 const float* rw, const sdm_state* st, float* out, const void* g,
+                                 const float* wn, float eps, void* a, void* ws, size_t ws_bytes,
+                                 sdm_stream_t stream) {
+    if (!g || !wn || !a) return SDM_ERR_ARG;
+    if (!(eps >= 0.f)) return SDM_ERR_ARG;
+    if (!aligned16(g) || !aligned16(wn) || !aligned16(a)) return SDM_ERR_ALIGN;
+    RunEpi ep{};
+    ep.g = static_cast<const __nv_bfloat16*>(g);
+    ep.wn = wn;
+    ep.eps = eps;
+    ep.a = static_cast<__nv_bfloat16*>(a);
+    return forward_run_impl(dims, v, beta, widx, ww, ridx, rw, st, out, ep, ws, ws_bytes,
+                            (cudaStream_t)stream);
 }
 
 sdm_status sdm_forward(const sdm_dims* dims, const void* v, const float* alpha, const float* beta,

@@ -107,6 +107,47 @@ def test_layer_out_after_prefill(sdm):
     assert sdm.device_error() == 0
 
 
+def test_layer_out_fused_into_the_read(sdm):
+    """The row pass with the output side's RMS-norm and swish gate fused into it: its fp32
+    read output equals the plain row pass's bit for bit, its bf16 operand a matches the
+    oracle's normalised and gated read, and y = a @ Wo matches the oracle's layer output."""
+    orc = oracle.default()
+    for wl in (S.MID.scaled(T=256), S.HEADLINE.scaled(B=2, H=2, T=200, n_sub=128)):
+        inp = S.generate(wl, device="cuda")
+        d = sdm.Dims(wl.B, wl.H, wl.T, wl.d_k, wl.n_sub, wl.d_v, wl.k_half, wl.W, wl.R,
+                     wl.x_dtype, wl.v_dtype)
+        sel = sdm.score_qk(d, inp["q"], inp["k"], inp["skw"], inp["skr"])
+        ws = sdm.workspace(d)
+        st = sdm.State(d, inp["M0"])
+        sdm.state_reset(d, st)
+        sdm.forward_plan(d, inp["alpha"], inp["beta"], *sel, st, ws)
+        out0 = torch.empty((wl.B, wl.H, wl.T, wl.d_v), device="cuda")
+        sdm.forward_run(d, inp["v"], inp["beta"], *sel, st, out0, ws)
+        gen = torch.Generator(device="cuda").manual_seed(5)
+        g = torch.randn(wl.B, wl.T, wl.H * wl.d_v, device="cuda", generator=gen).to(torch.bfloat16)
+        wn = 0.5 + torch.rand(wl.d_v, device="cuda", generator=gen)
+        st2 = sdm.State(d, inp["M0"])
+        sdm.state_reset(d, st2)
+        sdm.forward_plan(d, inp["alpha"], inp["beta"], *sel, st2, ws)
+        out1, a = sdm.forward_run_gated(d, inp["v"], inp["beta"], *sel, st2, g, wn, 1e-6, ws=ws)
+        dm = 4 * wl.H * wl.n_sub
+        Wo_t = (torch.randn(dm, wl.H * wl.d_v, device="cuda", generator=gen) /
+                np.sqrt(wl.H * wl.d_v)).to(torch.bfloat16)
+        y = sdm.gemm_bf16(a.reshape(wl.B * wl.T, wl.H * wl.d_v), Wo_t)
+        torch.cuda.synchronize()
+        assert torch.equal(out0, out1)
+        # a against the normalised, gated read computed from the same fp32 read in fp64
+        o64 = f64(out1).transpose(0, 2, 1, 3)  # [B,T,H,d_v]
+        rms = np.sqrt((o64 ** 2).mean(-1, keepdims=True) + 1e-6)
+        z = f64(g).reshape(wl.B, wl.T, wl.H, wl.d_v)
+        a_ref = (o64 / rms * f64(wn) * (z / (1 + np.exp(-z)))).reshape(wl.B, wl.T, -1)
+        check_err(normwise_rel_err(f64(a), a_ref), TOL["bf16"], "a")
+        rows = np.array([0, 1, 77, wl.B * wl.T - 1])
+        ref = orc.layer_out(f64(out1), f64(g), f64(wn), f64(Wo_t), rows=rows)
+        check_err(normwise_rel_err(f64(y).reshape(wl.B * wl.T, dm)[rows], ref), TOL["bf16"], "y")
+        assert sdm.device_error() == 0
+
+
 def test_gemm_validation(sdm):
     A = torch.zeros(4, 12, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(sdm.SdmError):
