@@ -35,9 +35,10 @@ L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 # the hash of the kernel sources it was taken with; None when not yet measured for the
 # current sources.  Filled from profiles/ (see the summary named there).
 MEASURED_TRAFFIC = {
-    # profiles/recur_run_kernel_mid_prefill.md: dram read 728.75 MB + write 405.35 MB (the
-    # plan sources changed for the touched-slots decay variant; the row pass did not)
-    "e64fe2a7f5e03e49": 1_134_104_064,
+    # profiles/recur_run_kernel_mid_prefill.md: dram read 728.85 MB + write 406.16 MB, taken
+    # after the row pass gained its fused layer-output variant (a separate instantiation;
+    # the plain one is unchanged)
+    "e719ce73f5a42202": 1_135_003_648,
 }
 
 
@@ -514,6 +515,46 @@ def run_workload(name: str, device, sdm, steps: int = 5, warm: int = 3,
     return res
 
 
+def run_score_only(name: str, device, sdm, tokens: int | None = None, steps: int = 5,
+                   warm: int = 3) -> dict:
+    """Both roles' scoring of one workload (`sdm_score_qk`) on its own: `tokens` replaces the
+    workload's T (same d_k, n, k and value distributions), so that a profiler capture of the
+    scorer holds a few hundred MB instead of the full workload.  L2 flushed between calls."""
+    import torch
+
+    import sdm_synth as S
+    wl = S.WORKLOADS[name]
+    if tokens:
+        wl = wl.scaled(T=tokens, decode_steps=0)
+    inp = S.generate(wl, device=device, with_m0=False)
+    d = sdm.Dims(wl.B, wl.H, wl.T, wl.d_k, wl.n_sub, wl.d_v, wl.k_half, wl.W, wl.R, wl.x_dtype,
+                 wl.v_dtype)
+    sel = sdm.selection_buffers(d, device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(warm):
+        flush.zero_()
+        sdm.score_qk(d, inp["q"], inp["k"], inp["skw"], inp["skr"], sel)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    for e in evs:
+        flush.zero_()
+        e[0].record(stream)
+        sdm.score_qk(d, inp["q"], inp["k"], inp["skw"], inp["skr"], sel)
+        e[1].record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    units = units_per_step(wl)
+    flops = scoring_flops_per_token_head(wl) * units
+    path = {sdm.SCORE_TC: "tensor cores (score_pk_kernel)", sdm.SCORE_ROWS: "row scorer",
+            sdm.SCORE_WARP: "one warp per row"}[sdm.score_path(d, wl.W)]
+    return {"workload": describe(wl), "calls_timed": steps, "ms": ms, "path": path,
+            "rows_per_s": 2 * units / (ms / 1e3),
+            "tflops": flops / (ms / 1e3) / 1e12,
+            "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / measured_peaks()["bf16_tflops"],
+            "device_errors": sdm.device_error()}
+
+
 def run_decode(device, sdm, steps: int = 64, warm: int = 3, n_sub: int | None = None,
                d_v: int | None = None) -> dict:
     """The decode workload at full size: a 512-token seeded prefill of every (b,h), then
@@ -904,7 +945,21 @@ def main(argv=None):
                     help="sub-keys per half for --decode-only (default: the workload's 256)")
     ap.add_argument("--decode-d-v", type=int, default=None,
                     help="row width for --decode-only (default: the workload's 128)")
+    ap.add_argument("--score-only", default=None, metavar="WORKLOAD",
+                    help="run only both roles' scoring of WORKLOAD (--steps timed calls after "
+                         "--warmup) and print its object")
+    ap.add_argument("--score-tokens", type=int, default=None,
+                    help="tokens per sequence for --score-only (default: the workload's T)")
     args = ap.parse_args(argv)
+    if args.score_only:
+        import torch
+
+        import sparse_state_linear_score_b200 as sdm
+        res = run_score_only(args.score_only, torch.device("cuda", 0), sdm,
+                             tokens=args.score_tokens, steps=args.steps,
+                             warm=max(3, args.warmup))
+        print(json.dumps({"scoring": res}), flush=True)
+        return
     if args.decode_only:
         import torch
 
