@@ -510,7 +510,7 @@ def run_workload(name: str, device, sdm, steps: int = 5, warm: int = 3,
         samp = wl.scaled(B=1, H=min(wl.H, 2))
         cb = cpu_baseline(samp, seconds=cpu_seconds)
         cb["sample"] = cb["sample"] + f"; the {wl.name} workload has {wl.B * wl.H} sequences"
-        cb["kind"] = "oracle (sampled)"
+        cb["kind"] = "oracle (sampled; rate per token·head extrapolated to the workload)"
         res["cpu_baseline"] = cb
     return res
 
