@@ -617,6 +617,7 @@ def run_decode(device, sdm, steps: int = 64, warm: int = 3, n_sub: int | None = 
     us = e0.elapsed_time(e1) * 1e3 / steps
     del g
     errs = sdm.device_error()
+    fused = sdm.decode_path(dd) == sdm.DECODE_FUSED
     rows = wl.B * wl.H
     bpt = bytes_per_token_head(wl)
     step_bytes = (bpt["step"] + (2 * wl.W + wl.R) * 8) * rows  # + stamp reads and writes
@@ -625,7 +626,10 @@ def run_decode(device, sdm, steps: int = 64, warm: int = 3, n_sub: int | None = 
     res = {"workload": f"decode: B={wl.B} H={wl.H} d_k={wl.d_k} n={wl.n_sub} N={wl.N} "
                        f"d_v={wl.d_v} k={wl.k_half} W={wl.W} R={wl.R} after a {wl.T}-token prefill",
            "steps_timed": steps, "us_per_step": us, "token_heads_per_s": rows / (us / 1e6),
-           "us_per_step_issued_one_call_at_a_time": us_eager, "gpu_launches_per_step": 2,
+           "us_per_step_issued_one_call_at_a_time": us_eager,
+           "gpu_launches_per_step": 1 if fused else 2,
+           "path": "one launch (scoring and recurrence steps in clusters of two CTAs)" if fused
+                   else "scoring launch + recurrence launch",
            "roofline": {"bound": "hbm", "algorithmic_bytes_per_step": step_bytes,
                         "achieved_gbs": gbs, "peak": peak, "frac": gbs / peak},
            "note": "state 34 GB (fp32 rows) >> L2; each step scores new tokens, so its gathers "

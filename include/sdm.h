@@ -248,11 +248,51 @@ sdm_status sdm_prefill(const sdm_dims* dims, const void* q, const void* k, const
  *   q, k [B][H][d_k]; v [B][H][d_v]; alpha, beta [B][H]; out [B][H][d_v];
  *   widx/ww [B][H][W], ridx/rw [B][H][R] receive the selections.
  * No workspace.  Equal to sdm_forward with T = 1 up to rounding order.
+ * Where sdm_decode_path says SDM_DECODE_FUSED (bf16 q and k with d_k = 128,
+ * 64 < n_sub <= 512, k_half, W, R <= 32, d_v <= 256) the step is one launch: each CTA
+ * scores the keys and queries of two sequences of one head and runs their recurrence
+ * steps from the selections it holds on chip; the selections are still written to
+ * widx/ww/ridx/rw.  Otherwise it is a scoring launch followed by the recurrence launch.
  */
 sdm_status sdm_decode_step(const sdm_dims* dims, const void* q, const void* k, const void* v,
                            const float* alpha, const float* beta, const void* skw,
                            const void* skr, const sdm_state* st, int32_t* widx, float* ww,
                            int32_t* ridx, float* rw, float* out, sdm_stream_t stream);
+
+/*
+ * Call log: what one call overwrites in the state, so that the state at the call's start can
+ * be put back after it (Sparse Delta Memory summary, appendix A.3 "Memory-Efficient
+ * Backward": the sparse updates are undone in place instead of keeping a copy of the
+ * memory; here across calls).  A sequence run as calls 1..C is differentiated from the last
+ * call back: restore call c's log, then sdm_backward over call c from that state, its dM_in
+ * the dM_end of call c-1.  A call (sdm_forward, sdm_prefill, sdm_decode_step) writes only
+ * the rows and stamps of its write slots and Lambda, so the log holds, for each write
+ * occurrence, the raw row and stamp of its slot before the call, and Lambda:
+ *   rows [B][H][T][W][d_v] fp32, stamps [B][H][T][W] fp64, Lambda [B][H] fp64
+ * (sdm_call_log_bytes: the size, sections 256-byte aligned; O(T*W*d_v) per call).
+ *   sdm_call_log_save     before the call, on its stream: copies from st into log.
+ *                         widx [B][H][T][W] int32 are the call's write slots (for a
+ *                         prefill, sdm_score_topk of the keys gives them before the call).
+ *   sdm_call_log_restore  after the call (and after every later call has been restored):
+ *                         copies log back into st, which then equals, bit for bit, the
+ *                         state before the call.
+ * log is caller-owned device memory of at least sdm_call_log_bytes(dims) bytes, 16-byte
+ * aligned (SDM_ERR_WORKSPACE if smaller).  Slots outside [0, N) are skipped and set
+ * SDM_DEVERR_SLOT_RANGE.
+ */
+size_t sdm_call_log_bytes(const sdm_dims* dims);
+sdm_status sdm_call_log_save(const sdm_dims* dims, const int32_t* widx, const sdm_state* st,
+                             void* log, size_t log_bytes, sdm_stream_t stream);
+sdm_status sdm_call_log_restore(const sdm_dims* dims, const int32_t* widx, const void* log,
+                                size_t log_bytes, const sdm_state* st, sdm_stream_t stream);
+
+/*
+ * The launches sdm_decode_step makes for these dims: SDM_DECODE_FUSED (one launch: scoring
+ * and recurrence step in the same CTAs) or SDM_DECODE_TWO (a scoring launch, then the
+ * recurrence launch); a negative sdm_status code for bad dims (dims->T is not looked at).
+ */
+enum { SDM_DECODE_FUSED = 1, SDM_DECODE_TWO = 2 };
+int32_t sdm_decode_path(const sdm_dims* dims);
 
 /*
  * Backward of the recurrence over one call of T tokens (Sparse Delta Memory summary,

@@ -87,6 +87,7 @@ def _load():
         "sdm_score_topk": ([D, P, P, I32, P, P, P], I32),
         "sdm_score_qk": ([D, P, P, P, P, P, P, P, P, P], I32),
         "sdm_score_path": ([D, I32], I32),
+        "sdm_decode_path": ([D], I32),
         "sdm_forward_workspace_bytes": ([D], SZ),
         "sdm_forward": ([D, P, P, P, P, P, P, P, S, P, P, SZ, P], I32),
         "sdm_forward_plan": ([D, P, P, P, P, P, P, S, P, SZ, P], I32),
@@ -98,6 +99,9 @@ def _load():
         "sdm_device_error": ([ctypes.POINTER(ctypes.c_uint32), I32, P], I32),
         "sdm_forward_noalloc": ([D, P, P, P, P, P, P, P, S, P, P], I32),
         "sdm_backward_workspace_bytes": ([D], SZ),
+        "sdm_call_log_bytes": ([D], SZ),
+        "sdm_call_log_save": ([D, P, S, P, SZ, P], I32),
+        "sdm_call_log_restore": ([D, P, P, SZ, S, P], I32),
         "sdm_score_backward": ([D, P, P, I32, P, P, P, P, P, P], I32),
         "sdm_backward": ([D, P, P, P, P, P, P, P, S, P, P, P, P, P, P, P, P, P, SZ, P], I32),
         "sdm_gemm_bf16": ([I32, I32, I32, P, P, P, P], I32),
@@ -192,6 +196,28 @@ def state_materialize(d: Dims, st: State, out: torch.Tensor | None = None, strea
     return out
 
 
+def call_log_bytes(d: Dims) -> int:
+    return int(_lib.sdm_call_log_bytes(ctypes.byref(d)))
+
+
+def call_log_save(d: Dims, widx, st: State, log=None, stream=None):
+    """sdm_call_log_save: before a call with write slots widx [B,H,T,W], record the rows,
+    stamps and Lambda it will overwrite.  Returns the log (uint8 device tensor)."""
+    if log is None:
+        log = torch.empty(max(16, call_log_bytes(d)), dtype=torch.uint8, device=st.M.device)
+    _ok(_lib.sdm_call_log_save(ctypes.byref(d), _ptr(widx, "widx", torch.int32),
+                               ctypes.byref(st.c), _ptr(log, "log"), log.numel(),
+                               _stream(stream)), "sdm_call_log_save")
+    return log
+
+
+def call_log_restore(d: Dims, widx, log, st: State, stream=None):
+    """sdm_call_log_restore: after the call, put back the state it started from."""
+    _ok(_lib.sdm_call_log_restore(ctypes.byref(d), _ptr(widx, "widx", torch.int32),
+                                  _ptr(log, "log"), log.numel(), ctypes.byref(st.c),
+                                  _stream(stream)), "sdm_call_log_restore")
+
+
 def score_topk(d: Dims, x, subkeys, top: int, idx=None, w=None, stream=None):
     shape = (d.B, d.H, d.T, top)
     if idx is None:
@@ -213,6 +239,18 @@ def score_path(d: Dims, top: int) -> int:
     r = int(_lib.sdm_score_path(ctypes.byref(d), top))
     if r < 0:
         raise SdmError(-r, "sdm_score_path")
+    return r
+
+
+DECODE_FUSED, DECODE_TWO = 1, 2
+
+
+def decode_path(d: Dims) -> int:
+    """sdm_decode_path: DECODE_FUSED when decode_step is one launch (scoring and recurrence
+    step in the same CTAs), DECODE_TWO when it is a scoring launch and a recurrence launch."""
+    r = int(_lib.sdm_decode_path(ctypes.byref(d)))
+    if r < 0:
+        raise SdmError(-r, "sdm_decode_path")
     return r
 
 

@@ -13,6 +13,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "score_rows.cuh"
 
 namespace sdm {
 
@@ -50,89 +51,67 @@ SDM_DEV void fma4(float4& acc, float c, const float4& x) {
     acc.w = fmaf(c, x.w, acc.w);
 }
 
-// RPW: rows of each role per warp (ceil(max(W, R) / 8)); QPL: float4 columns per lane.
+// Decode smem views (decode_smem_bytes): partial sums and the occurrences' slots, weights and
+// decay factors (the sign bit marks a pristine row, read from M0), writes first.
+struct DecSmem {
+    float* pp;   // [8][d_v] partial p
+    float* po;   // [8][d_v] partial out
+    int* slot;   // [W+R]
+    float* w;    // [W+R]
+    float* f;    // [W+R]
+    float* uw;   // [W] read weight that lands on write row i
+    int* rm;     // [R] read j is also written
+    SDM_DEV DecSmem(unsigned char* p, int W, int R, int d_v) {
+        pp = reinterpret_cast<float*>(p);
+        po = pp + DECODE_WARPS * d_v;
+        slot = reinterpret_cast<int*>(po + DECODE_WARPS * d_v);
+        w = reinterpret_cast<float*>(slot + W + R);
+        f = w + W + R;
+        uw = f + W + R;
+        rm = reinterpret_cast<int*>(uw + W);
+    }
+};
+
+// Decay factor of an occurrence's row from its slot's stamp (NaN: pristine, the sign bit set):
+// e^{Lambda' - stamp}, or under touched-slots decay alpha for a write slot and 1 for a read.
+SDM_DEV float decode_factor(double st, double Lnew, bool write, float a_t, int touched) {
+    if (touched) {
+        const float fv = write ? a_t : 1.f;
+        return isnan(st) ? -fv : fv;
+    }
+    return isnan(st) ? -(float)exp(Lnew) : (float)exp(Lnew - st);
+}
+
+// The rows of one sequence's step, once its occurrences (slot, weight, factor) are in d's
+// arrays -- each warp reads the entries of its own rows (written by itself, or by any thread
+// before a block barrier): p = sum_i w_i seen(s_i), d = beta (v - p), the written rows and
+// their stamps, out = sum_j u_j (r_j after the write), Lambda'.
 template <typename VT, int RPW, int QPL>
-__global__ void __launch_bounds__(DECODE_THREADS) decode_kernel(
-    const VT* __restrict__ v, const float* __restrict__ alpha, const float* __restrict__ beta,
-    const int32_t* __restrict__ widx, const float* __restrict__ ww,
-    const int32_t* __restrict__ ridx, const float* __restrict__ rw, float* __restrict__ M,
-    double* __restrict__ stamp, double* __restrict__ lambda, const float* __restrict__ M0,
-    float* __restrict__ out, int H, int N, int d_v, int W, int R, int touched) {
-    extern __shared__ __align__(16) unsigned char dec_smem[];
-    const size_t bh = blockIdx.x;
+SDM_DEV void decode_apply(size_t bh, const float4 (&vv)[QPL], float bt, double Lnew, const DecSmem& d,
+                          float* __restrict__ M, double* __restrict__ stamp,
+                          double* __restrict__ lambda, const float* __restrict__ M0,
+                          float* __restrict__ out, int H, int N, int d_v, int W, int R) {
     const int h = (int)(bh % H);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int no = W + R;
     const int Q = d_v / 4;
-    float* s_pp = reinterpret_cast<float*>(dec_smem);              // [8][d_v] partial p
-    float* s_po = s_pp + DECODE_WARPS * d_v;                       // [8][d_v] partial out
-    int* s_slot = reinterpret_cast<int*>(s_po + DECODE_WARPS * d_v);  // [W+R]
-    float* s_w = reinterpret_cast<float*>(s_slot + no);            // [W+R]
-    float* s_f = s_w + no;                                         // [W+R], sign: pristine
-    float* s_uw = s_f + no;                                        // [W] read weight on row i
-    int* s_rm = reinterpret_cast<int*>(s_uw + W);                  // [R] read j is written
-
+    float* s_pp = d.pp;
+    float* s_po = d.po;
+    int* s_slot = d.slot;
+    float* s_w = d.w;
+    float* s_f = d.f;
+    float* s_uw = d.uw;
+    int* s_rm = d.rm;
     float* Mb = M + bh * (size_t)N * d_v;
     const float* M0h = M0 + (size_t)h * N * d_v;
     double* stb = stamp + bh * (size_t)N;
-    // inputs that do not come from the scoring launch before this one: read them while it
-    // finishes (programmatic dependent launch), then wait for its indices and weights
-    const float bt = beta[bh];
-    float4 vv[QPL];
-#pragma unroll
-    for (int c = 0; c < QPL; ++c) {
-        const int q = lane + 32 * c;
-        vv[c] = q < Q ? load_v4<VT>(v + bh * d_v + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    double Lnew;  // Lambda'
-    const float a_t = alpha[bh];
-    {
-        double la = 0.0;
-        if (a_t > 0.f) la = log((double)a_t);
-        else if (tid == 0) raise_err(SDM_DEVERR_ALPHA);
-        Lnew = lambda[bh] + la;
-    }
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-
-    // ---- this warp's rows: lane k fetches write row w + 8k, lane 16 + k read row w + 8k
-    //      (slot, weight, decay factor from the stamp), the warp shares them by shuffles and
-    //      puts every row load in flight before the first block barrier --------------------
-    int my_s = -1;
-    float my_f = 0.f;
-    {
-        const bool rl = lane >= 16;
-        const int k = lane & 15, i = warp + DECODE_WARPS * k;
-        if (k < RPW && i < (rl ? R : W)) {
-            int sl = rl ? ridx[bh * R + i] : widx[bh * W + i];
-            const float w = rl ? rw[bh * R + i] : ww[bh * W + i];
-            float f = 0.f;
-            if (!slot_ok(sl, N)) {
-                raise_err(SDM_DEVERR_SLOT_RANGE);
-                sl = -1;
-            } else {
-                const double st = stb[sl];
-                if (touched) {  // alpha scales the write slots only
-                    const float fv = rl ? 1.f : a_t;
-                    f = isnan(st) ? -fv : fv;
-                } else {
-                    f = isnan(st) ? -(float)exp(Lnew) : (float)exp(Lnew - st);
-                }
-            }
-            my_s = sl;
-            my_f = f;
-            const int o = rl ? W + i : i;
-            s_slot[o] = sl;
-            s_w[o] = w;
-            s_f[o] = f;
-        }
-    }
+    __syncwarp();
     float4 wr[RPW][QPL], rd[RPW][QPL];
 #pragma unroll
     for (int k = 0; k < RPW; ++k) {
-        const int si = __shfl_sync(0xffffffffu, my_s, k);
-        const int sj = __shfl_sync(0xffffffffu, my_s, 16 + k);
-        const float fi = __shfl_sync(0xffffffffu, my_f, k);
-        const float fj = __shfl_sync(0xffffffffu, my_f, 16 + k);
+        const int i = warp + DECODE_WARPS * k;
+        const int si = i < W ? s_slot[i] : -1, sj = i < R ? s_slot[W + i] : -1;
+        const float fi = i < W ? s_f[i] : 0.f, fj = i < R ? s_f[W + i] : 0.f;
         const float* srci = (si >= 0 && signbit(fi)) ? M0h : Mb;
         const float* srcj = (sj >= 0 && signbit(fj)) ? M0h : Mb;
 #pragma unroll
@@ -263,6 +242,253 @@ __global__ void __launch_bounds__(DECODE_THREADS) decode_kernel(
         reinterpret_cast<float4*>(out + bh * d_v)[q] = o;
     }
     if (tid == 0) lambda[bh] = Lnew;
+}
+
+// The step of sequence bh by the whole CTA (DECODE_THREADS threads; dec_smem holds
+// decode_smem_bytes).  wi / wv and ri / rv are the token's W write and R read slots and
+// weights.  With dep_wait the CTA waits for the launch before it (programmatic dependent
+// launch) after reading v, alpha and beta and before anything that launch writes.  RPW: rows
+// of each role per warp (ceil(max(W, R) / 8)); QPL: float4 columns per lane.
+template <typename VT, int RPW, int QPL>
+SDM_DEV void decode_seq_step(size_t bh, const VT* __restrict__ v, const float* __restrict__ alpha,
+                             const float* __restrict__ beta, const int32_t* wi, const float* wv,
+                             const int32_t* ri, const float* rv, float* __restrict__ M,
+                             double* __restrict__ stamp, double* __restrict__ lambda,
+                             const float* __restrict__ M0, float* __restrict__ out, int H, int N,
+                             int d_v, int W, int R, int touched, unsigned char* dec_smem,
+                             bool dep_wait) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int Q = d_v / 4;
+    const DecSmem d(dec_smem, W, R, d_v);
+    double* stb = stamp + bh * (size_t)N;
+    // inputs that do not come from the scoring launch before this one: read them while it
+    // finishes (programmatic dependent launch), then wait for its indices and weights
+    const float bt = beta[bh];
+    float4 vv[QPL];
+#pragma unroll
+    for (int c = 0; c < QPL; ++c) {
+        const int q = lane + 32 * c;
+        vv[c] = q < Q ? load_v4<VT>(v + bh * d_v + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const float a_t = alpha[bh];
+    double la = 0.0;
+    if (a_t > 0.f) la = log((double)a_t);
+    else if (tid == 0) raise_err(SDM_DEVERR_ALPHA);
+    if (dep_wait) asm volatile("griddepcontrol.wait;" ::: "memory");
+    const double Lnew = lambda[bh] + la;  // Lambda'
+    // lane k fetches write row w + 8k, lane 16 + k read row w + 8k: slot, weight, and the
+    // decay factor from the slot's stamp
+    {
+        const bool rl = lane >= 16;
+        const int k = lane & 15, i = warp + DECODE_WARPS * k;
+        if (k < RPW && i < (rl ? R : W)) {
+            int sl = rl ? ri[i] : wi[i];
+            const float w = rl ? rv[i] : wv[i];
+            float f = 0.f;
+            if (!slot_ok(sl, N)) {
+                raise_err(SDM_DEVERR_SLOT_RANGE);
+                sl = -1;
+            } else {
+                f = decode_factor(stb[sl], Lnew, !rl, a_t, touched);
+            }
+            const int o = rl ? W + i : i;
+            d.slot[o] = sl;
+            d.w[o] = w;
+            d.f[o] = f;
+        }
+    }
+    decode_apply<VT, RPW, QPL>(bh, vv, bt, Lnew, d, M, stamp, lambda, M0, out, H, N, d_v, W, R);
+}
+
+// One CTA per sequence, launched after the scoring launch as its programmatic dependent: the
+// prologue (v, alpha, beta) overlaps the scorer's tail, the slots are read after the wait.
+template <typename VT, int RPW, int QPL>
+__global__ void __launch_bounds__(DECODE_THREADS) decode_kernel(
+    const VT* __restrict__ v, const float* __restrict__ alpha, const float* __restrict__ beta,
+    const int32_t* __restrict__ widx, const float* __restrict__ ww,
+    const int32_t* __restrict__ ridx, const float* __restrict__ rw, float* __restrict__ M,
+    double* __restrict__ stamp, double* __restrict__ lambda, const float* __restrict__ M0,
+    float* __restrict__ out, int H, int N, int d_v, int W, int R, int touched) {
+    extern __shared__ __align__(16) unsigned char dec_smem[];
+    const size_t bh = blockIdx.x;
+    decode_seq_step<VT, RPW, QPL>(bh, v, alpha, beta, widx + bh * W, ww + bh * W, ridx + bh * R,
+                                  rw + bh * R, M, stamp, lambda, M0, out, H, N, d_v, W, R, touched,
+                                  dec_smem, true);
+}
+
+// ---- the whole decode step in one launch --------------------------------------------------
+//
+// A cluster of two CTAs takes four sequences b0..b0+3 of one head.  CTA rank r scores the four
+// rows of role r (rank 0: the keys against the write tables, rank 1: the queries against the
+// read tables) with the row scorer's phases (tensor-core dot products, per-half top-k,
+// staircase combine, softmax), writes the selections out, and right away fetches the stamps
+// of its selected slots into decay factors.  After a cluster barrier each CTA copies, through
+// distributed shared memory, the other role's selections of the two sequences it steps (rank
+// r: b0 + 2r and b0 + 2r + 1), and runs their recurrence steps (decode_apply).  The
+// selections never make a round trip through memory, each CTA streams one sub-key table,
+// and there is one launch per step.  k_half, W, R <= 32; bf16 x with d_k = 128 and
+// 64 < n <= 32 * PL.
+struct DecArgs {
+    const void* v;
+    const float* alpha;
+    const float* beta;
+    float* M;
+    double* stamp;
+    double* lambda;
+    const float* M0;
+    float* out;
+    int N, d_v, touched;
+};
+
+// Shared memory of the fused step: the row scorer's (tensor-core head and common area) and
+// the four rows' selections (slot, weight, factor) and Lambda'.  The two steps' partial sums
+// and occurrence arrays reuse the two sub-key buffers (the host checks that they fit:
+// decode_fused_fits).
+__host__ __device__ inline size_t decode_fused_smem_bytes(int PL) {
+    return score_rows_smem_bytes(128, PL, 32, true) + (size_t)SROW_G * 32 * 12 + SROW_G * 8;
+}
+__host__ __device__ inline bool decode_fused_fits(int W, int R, int d_v) {
+    return 2 * ((decode_smem_bytes(W, R, d_v) + 15) & ~(size_t)15) <= 2 * (size_t)SROW_TC_KBUF;
+}
+
+SDM_DEV uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Every thread of both CTAs arrives; memory before the barrier (release) is visible to the
+// other CTA after it (acquire).
+SDM_DEV void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+// 32-bit word at the same shared-memory offset in CTA `rank` of the cluster
+SDM_DEV uint32_t dsmem_ld(const void* local, uint32_t rank) {
+    const uint32_t a = ptx::smem_u32(local);
+    uint32_t ra, v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(ra) : "memory");
+    return v;
+}
+
+// QPL = 2 (d_v > 128) keeps twice the rows' columns in registers: two CTAs per SM
+template <int PL, typename VT, int QPL>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SROW_THREADS, QPL == 1 ? 4 : 2)
+    decode_fused_kernel(const __grid_constant__ CUtensorMap km0,
+                        const __grid_constant__ CUtensorMap km1, ScoreRowsArgs a, DecArgs dk) {
+    static_assert(SROW_THREADS == DECODE_THREADS, "the step runs on the scorer's CTA");
+    using SM = SrowSmem<PL, 32>;
+    extern __shared__ __align__(16) unsigned char srow_smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.y, n = a.n, kh = a.k_half, B = a.B, H = a.H, N = dk.N, d_v = dk.d_v;
+    const uint32_t rank = cluster_ctarank();  // = the role this CTA scores
+    const int role = (int)rank;
+    const int b0 = (blockIdx.x >> 1) * 4;
+    const int W = a.top[0], R = a.top[1], top = a.top[role];
+    unsigned char* base = srow_smem + ((1024 - (ptx::smem_u32(srow_smem) & 1023)) & 1023);
+    const SM sm(base + SROW_TC_HEAD);
+    int32_t* sel_slot = reinterpret_cast<int32_t*>(sm.ncand + 4);    // [G][32]
+    float* sel_w = reinterpret_cast<float*>(sel_slot + SROW_G * 32);  // [G][32]
+    float* sel_f = sel_w + SROW_G * 32;                               // [G][32]
+    double* lnew = reinterpret_cast<double*>(sel_f + SROW_G * 32);    // [G] Lambda'
+    if (tid < SROW_CAND) {
+        sm.cand[tid] = a.cand[role][tid];
+        if (tid == 0) sm.ncand[0] = a.ncand[role];
+    }
+    // the decay inputs of the rows this CTA selects (warp g: sequence b0 + g) and of the
+    // sequences it steps, read while the scores are computed
+    const int bg = b0 + warp;
+    double Lg = 0.0;
+    float ag = 1.f;
+    if (warp < SROW_G && bg < B) {
+        const size_t bh = (size_t)bg * H + h;
+        ag = dk.alpha[bh];
+        if (!(ag > 0.f) && lane == 0) raise_err(SDM_DEVERR_ALPHA);  // treated as alpha = 1
+        Lg = dk.lambda[bh] + (ag > 0.f ? log((double)ag) : 0.0);
+        if (lane == 0) lnew[warp] = Lg;
+    }
+    float4 vv[2][QPL];
+    float bt[2];
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        const int b = b0 + 2 * role + s;
+        const size_t bh = (size_t)(b < B ? b : 0) * H + h;
+        bt[s] = b < B ? dk.beta[bh] : 0.f;
+#pragma unroll
+        for (int c = 0; c < QPL; ++c) {
+            const int q = lane + 32 * c;
+            vv[s][c] = (b < B && q < d_v / 4)
+                           ? load_v4<VT>(static_cast<const VT*>(dk.v) + bh * d_v + 4 * q)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    const __nv_bfloat16* xr[SROW_G];
+    int rtab[SROW_G];
+#pragma unroll
+    for (int g = 0; g < SROW_G; ++g) {
+        rtab[g] = 0;
+        const int b = b0 + g;
+        xr[g] = b < B ? static_cast<const __nv_bfloat16*>(a.x[role]) + ((size_t)b * H + h) * 128
+                      : nullptr;
+    }
+    const bool ok = srow_tc_dots<32 * PL, 1>(base, sm.segs, SM::SEG, role ? &km1 : &km0, nullptr,
+                                             xr, rtab, h, n);
+    {
+        const int g = warp >> 1, hf = warp & 1;
+        srow_half_topk<PL, 32>(sm.seg(g, hf), n, kh, sm.tv + (g * 2 + hf) * 32,
+                               sm.ti + (g * 2 + hf) * 32, lane);
+    }
+    __syncthreads();
+    if (warp < SROW_G && bg < B) {
+        const int g = warp;
+        int2* scr = reinterpret_cast<int2*>(sm.seg(g, 0) + 32 * PL * 4);
+        uint32_t slot;
+        float wt;
+        srow_combine32(sm.tv + (g * 2) * 32, sm.ti + (g * 2) * 32, sm.tv + (g * 2 + 1) * 32,
+                       sm.ti + (g * 2 + 1) * 32, sm.cand, sm.ncand[0], n, top, scr, lane, slot,
+                       wt);
+        const size_t bh = (size_t)bg * H + h;
+        int sl = ok ? (int)slot : -1;  // a failed dot-product phase selects nothing
+        if (!ok) wt = 0.f;
+        float f = 0.f;
+        if (lane < top) {
+            a.idx[role][bh * top + lane] = sl;
+            a.w[role][bh * top + lane] = wt;
+            if (slot_ok(sl, N)) {
+                f = decode_factor(dk.stamp[bh * (size_t)N + sl], Lg, role == 0, ag, dk.touched);
+            } else {
+                raise_err(SDM_DEVERR_SLOT_RANGE);
+                sl = -1;
+            }
+        }
+        sel_slot[g * 32 + lane] = sl;
+        sel_w[g * 32 + lane] = wt;
+        sel_f[g * 32 + lane] = f;
+    }
+    cluster_sync();  // both roles' selections are complete and visible in the cluster
+    // the occurrences of the two sequences this CTA steps: writes from rank 0's rows, reads
+    // from rank 1's, into the step's arrays (which take the sub-key buffers)
+    const DecSmem d0(base, W, R, d_v), d1(base + ((decode_smem_bytes(W, R, d_v) + 15) & ~(size_t)15), W, R,
+                                                   d_v);
+    for (int e = tid; e < 2 * (W + R); e += SROW_THREADS) {
+        const int s = e / (W + R), o = e % (W + R);
+        const int g = 2 * role + s;
+        const bool rd = o >= W;
+        const int i = rd ? o - W : o, src = rd ? 1 : 0;
+        const int off = g * 32 + i;
+        const DecSmem& dd = s ? d1 : d0;
+        dd.slot[o] = (int)dsmem_ld(sel_slot + off, (uint32_t)src);
+        dd.w[o] = __uint_as_float(dsmem_ld(sel_w + off, (uint32_t)src));
+        dd.f[o] = __uint_as_float(dsmem_ld(sel_f + off, (uint32_t)src));
+    }
+    cluster_sync();  // neither CTA reads the other's shared memory after this
+    for (int s = 0; s < 2; ++s) {
+        const int b = b0 + 2 * role + s;
+        if (b >= B) break;
+        if (s > 0) __syncthreads();  // the first step's partial sums have been read
+        decode_apply<VT, 4, QPL>((size_t)b * H + h, vv[s], bt[s], lnew[2 * role + s], s ? d1 : d0,
+                                 dk.M, dk.stamp, dk.lambda, dk.M0, dk.out, H, N, d_v, W, R);
+    }
 }
 
 }  // namespace sdm

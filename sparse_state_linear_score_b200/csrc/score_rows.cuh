@@ -259,21 +259,376 @@ __host__ __device__ inline size_t score_rows_seg_bytes(int PL, int KP) {
 }
 
 // Shared memory: x rows (CUDA-core dots) or the tensor-core staging (plus 1 KB for its
-// alignment), the score segments, the per-half lists, the selected pairs, the staircase.
+// alignment), the score segments, the per-half lists, the selected pairs, the staircase
+// tables of both roles.
 __host__ __device__ inline size_t score_rows_smem_bytes(int d_k, int PL, int KP, bool tcd) {
     const size_t head = tcd ? SROW_TC_HEAD + 1024 : srow_align16((size_t)SROW_G * d_k * 4);
     return head + (size_t)SROW_G * 2 * score_rows_seg_bytes(PL, KP) + (size_t)SROW_G * 2 * KP * 8 +
-           (size_t)SROW_G * KP * 8 + SROW_CAND * 4 + 16;
+           (size_t)SROW_G * KP * 8 + 2 * SROW_CAND * 4 + 16;
+}
+
+// The common area after the head: score segments, per-half lists, selected pairs, the
+// staircase tables.
+template <int PL, int KP>
+struct SrowSmem {
+    static constexpr size_t SEG = KP == 32 ? (size_t)32 * PL * 4 + 512 : (size_t)32 * PL * 8;
+    unsigned char* segs;  // [G][2] segments of SEG bytes
+    float* tv;            // [G][2][KP] per-half values
+    int* ti;              // [G][2][KP] per-half sub-indices
+    float* sv;            // [G][KP] selected sums (wide combine)
+    uint32_t* ss;         // [G][KP] selected slots (wide combine)
+    int* cand;            // [2][SROW_CAND] staircase pairs per role
+    int* ncand;           // [2]
+    SDM_DEV explicit SrowSmem(unsigned char* p) {
+        segs = p;
+        tv = reinterpret_cast<float*>(segs + (size_t)SROW_G * 2 * SEG);
+        ti = reinterpret_cast<int*>(tv + SROW_G * 2 * KP);
+        sv = reinterpret_cast<float*>(ti + SROW_G * 2 * KP);
+        ss = reinterpret_cast<uint32_t*>(sv + SROW_G * KP);
+        cand = reinterpret_cast<int*>(ss + SROW_G * KP);
+        ncand = cand + 2 * SROW_CAND;
+    }
+    SDM_DEV unsigned char* seg(int g, int hf) const { return segs + (size_t)(g * 2 + hf) * SEG; }
+};
+
+// Phase 1 on the tensor cores for the CTA's SROW_G rows: xr[g] is row g's x (d_k = 128 bf16;
+// null: a zero row), rtab[g] the sub-key table it is scored against (0: km0, 1: km1).  The
+// chunks of the TABLES tables of head h (every table's half 0 then half 1, 128 sub-keys each)
+// stream through the two TMA buffers at `base`; each chunk's scores go to the segments of
+// the rows that use its table.  All threads of the CTA (SROW_THREADS) take part.  Returns
+// false when a bounded wait gave up (the device error word says so).
+template <int NP, int TABLES>
+SDM_DEV bool srow_tc_dots(unsigned char* base, unsigned char* segs, size_t seg_bytes, const CUtensorMap* km0,
+                          const CUtensorMap* km1, const __nv_bfloat16* const (&xr)[SROW_G],
+                          const int (&rtab)[SROW_G], int h, int n) {
+    constexpr uint32_t NEED = TABLES * 2 * ((NP + 127) / 128) * 16;
+    constexpr uint32_t TCOLS = NEED <= 32 ? 32 : (NEED <= 64 ? 64 : (NEED <= 128 ? 128 : 256));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(base + SROW_TC_CTRL);  // [2]
+    uint64_t* bar_mma = bar_tma + 2;                                       // [2]
+    uint64_t* bar_done = bar_mma + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_done + 1);
+    int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+    const int cph = (n + 127) / 128, cpt = 2 * cph, nch = TABLES * cpt;  // chunks per half, table, all
+    auto chunk_map = [&](int c) { return (TABLES == 2 && c >= cpt) ? km1 : km0; };
+    auto chunk_row = [&](int c) {
+        const int cc = c % cpt;
+        return (h * 2 + cc / cph) * n + (cc % cph) * 128;
+    };
+    if (warp == 0) ptx::tmem_alloc(tmem_slot, TCOLS);
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(bar_tma + i, 1);
+            ptx::mbar_init(bar_mma + i, 1);
+        }
+        ptx::mbar_init(bar_done, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+        for (int c = 0; c < 2 && c < nch; ++c) {
+            ptx::mbar_arrive_expect_tx(bar_tma + c, SROW_TC_KBUF);
+            ptx::tma_load_2d(base + c * SROW_TC_KBUF, chunk_map(c), 0, chunk_row(c), bar_tma + c);
+        }
+    }
+    {   // x operand: thread t writes 16 bytes of half t/128, row (t/8)%16 (zero past the
+        // CTA's rows), swizzled: 16-byte chunk index XOR row % 8
+        const int hx = tid >> 7, row = (tid >> 3) & 15, ch = tid & 7;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (row < SROW_G && xr[row] != nullptr)
+            val = __ldg(reinterpret_cast<const uint4*>(xr[row] + hx * 64 + ch * 8));
+        *reinterpret_cast<uint4*>(base + SROW_TC_XT + hx * 2048 + row * 128 +
+                                  ((ch ^ (row & 7)) << 4)) = val;
+    }
+    ptx::fence_proxy_async_smem();  // the x operand is read by the tensor cores
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint64_t deadline = ptx::globaltimer_ns() + 2000000000ull;
+    if (tid == 0) {
+        const uint32_t idesc = ptx::idesc_bf16_f32(128, 16);
+        bool ok = true;
+        for (int c = 0; c < nch && ok; ++c) {
+            const int bf = c & 1;
+            const uint32_t par = (uint32_t)(c >> 1) & 1u;
+            if (!ptx::mbar_wait_bounded(bar_tma + bf, par, deadline)) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            const uint64_t ad = ptx::umma_desc_kmajor_sw128(base + bf * SROW_TC_KBUF);
+            const uint64_t bd =
+                ptx::umma_desc_kmajor_sw128(base + SROW_TC_XT + ((c % cpt) / cph) * 2048);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)  // K = 64 in steps of 16 (32 bytes)
+                ptx::umma_bf16(tmem + 16u * (uint32_t)c, ad + 2 * k, bd + 2 * k, idesc,
+                               k > 0 ? 1u : 0u);
+            ptx::umma_commit(bar_mma + bf);
+            if (c + 2 < nch) {  // buffer bf is free once this chunk's products are done
+                if (!ptx::mbar_wait_bounded(bar_mma + bf, par, deadline)) {
+                    ok = false;
+                    break;
+                }
+                ptx::mbar_arrive_expect_tx(bar_tma + bf, SROW_TC_KBUF);
+                ptx::tma_load_2d(base + bf * SROW_TC_KBUF, chunk_map(c + 2), 0, chunk_row(c + 2),
+                                 bar_tma + bf);
+            }
+        }
+        if (ok) {
+            ptx::umma_commit(bar_done);
+        } else {
+            *abort_flag = 1;
+            raise_err(SDM_DEVERR_TIMEOUT);
+        }
+    }
+    __syncthreads();  // thread 0 has issued everything (or given up)
+    bool aborted = *abort_flag != 0;
+    if (!aborted && !ptx::mbar_wait_bounded(bar_done, 0u, deadline)) {
+        aborted = true;
+        if (tid == 0) raise_err(SDM_DEVERR_TIMEOUT);
+    }
+    ptx::tc_fence_after();
+    if (!aborted) {  // warp w reads TMEM lanes 32 (w % 4) .. + 31 of every other chunk
+        const int q = warp & 3;
+        for (int c = warp >> 2; c < nch; c += 2) {
+            float v[4];
+            tmem_ld4(tmem + ((uint32_t)(32 * q) << 16) + 16u * (uint32_t)c, v);
+            const int tb = c / cpt, cc = c % cpt;
+            const int hf = cc / cph, sidx = (cc % cph) * 128 + 32 * q + lane;
+            if (sidx < n)
+#pragma unroll
+                for (int g = 0; g < SROW_G; ++g)
+                    if (rtab[g] == tb)
+                        reinterpret_cast<float*>(segs + (size_t)(g * 2 + hf) * seg_bytes)[sidx] = v[g];
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, TCOLS);
+    }
+    return !aborted;
+}
+
+// Phase 2 for one warp: the k_half best of one (row, half) score segment into tvo / tio,
+// best first.  The segment's spare bytes are the warp's scratch.
+template <int PL, int KP>
+SDM_DEV void srow_half_topk(unsigned char* seg, int n, int kh, float* tvo, int* tio, int lane) {
+    constexpr int NP = 32 * PL;
+    const float* scf = reinterpret_cast<const float*>(seg);
+    if constexpr (KP == 32) {
+        uint32_t key[PL], id[PL];
+#pragma unroll
+        for (int c = 0; c < PL; ++c) {
+            const int i = c * 32 + lane;
+            id[c] = (uint32_t)i;
+            key[c] = i < n ? order_key(scf[i]) : 0u;
+        }
+        uint32_t bk, bi;
+        if constexpr (PL <= 2) {
+            top32_columns<PL>(key, id, lane);
+            bk = key[0];
+            bi = id[0];
+        } else {  // the segment's second half (NP * 4 >= 512 bytes) is the scratch
+            int2* scr = reinterpret_cast<int2*>(seg + NP * 4);
+            top32_pruned<PL>(key, id, scr, lane, bk, bi);
+        }
+        if (lane < kh) {
+            tvo[lane] = key_value(bk);
+            tio[lane] = (int)bi;
+        }
+    } else {
+        uint32_t key[PL];
+        int id[PL];
+#pragma unroll
+        for (int r = 0; r < PL; ++r) {
+            const int i = lane * PL + r;
+            id[r] = i;
+            key[r] = i < n ? order_key(scf[i]) : 0u;
+        }
+        // bitonic sort of the lane's block, best first (key desc, sub-index asc)
+#pragma unroll
+        for (int k = 2; k <= PL; k <<= 1) {
+#pragma unroll
+            for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll
+                for (int i = 0; i < PL; ++i) {
+                    const int l = i ^ j;
+                    if (l > i) {
+                        const bool l_better =
+                            key[l] > key[i] || (key[l] == key[i] && id[l] < id[i]);
+                        if (((i & k) == 0) == l_better) {
+                            const uint32_t tk = key[i];
+                            key[i] = key[l];
+                            key[l] = tk;
+                            const int tix = id[i];
+                            id[i] = id[l];
+                            id[l] = tix;
+                        }
+                    }
+                }
+            }
+        }
+        __syncwarp();  // every lane has read its scores: the segment now holds the lists
+        int2* lst = reinterpret_cast<int2*>(seg);  // [32][PL]
+#pragma unroll
+        for (int r = 2; r < PL; ++r) lst[lane * PL + r] = make_int2((int)key[r], id[r]);
+        __syncwarp();
+        uint32_t hk = key[0];
+        int hi = id[0];
+        uint32_t nk = PL > 1 ? key[PL > 1 ? 1 : 0] : 0u;
+        int ni = PL > 1 ? id[PL > 1 ? 1 : 0] : 0;
+        int p = 1;  // position of (nk, ni) in the lane's list
+        for (int q = 0; q < kh; ++q) {
+            const uint32_t mx = __reduce_max_sync(0xffffffffu, hk);
+            const uint32_t bal = __ballot_sync(0xffffffffu, hk == mx);
+            if (lane == __ffs(bal) - 1) {
+                tvo[q] = key_value(hk);
+                tio[q] = hi;
+                hk = nk;
+                hi = ni;
+                ++p;
+                if (p < PL) {
+                    const int2 e = lst[lane * PL + p];
+                    nk = (uint32_t)e.x;
+                    ni = e.y;
+                } else {
+                    nk = 0u;
+                    ni = 0;
+                }
+            }
+        }
+    }
+}
+
+// Phase 3 for one warp, k_half and top <= 32: the `top` best staircase pairs (cand, nc) of
+// the row's two half lists, ranked by their sums; lane q < top gets the q-th slot and its
+// softmax weight.  scr: 64 entries of scratch.
+SDM_DEV void srow_combine32(const float* t1, const int* i1, const float* t2, const int* i2,
+                            const int* cand, int nc, int n, int top, int2* scr, int lane,
+                            uint32_t& slot, float& weight) {
+    constexpr int C = SROW_CAND / 32;
+    uint32_t key[C], id[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        const int e = c * 32 + lane;
+        if (e < nc) {
+            const int pr = cand[e], pa = pr >> 8, pb = pr & 255;
+            key[c] = order_key(t1[pa] + t2[pb]);
+            id[c] = (uint32_t)i1[pa] * (uint32_t)n + (uint32_t)i2[pb];
+        } else {
+            key[c] = 0u;
+            id[c] = 0x40000000u + (uint32_t)e;  // padding, distinct from every slot
+        }
+    }
+    uint32_t bk, bi;
+    if (nc <= 64) {
+        uint32_t k2[2] = {key[0], key[1]}, i2c[2] = {id[0], id[1]};
+        top32_columns<2>(k2, i2c, lane);
+        bk = k2[0];
+        bi = i2c[0];
+    } else {
+        top32_pruned<C>(key, id, scr, lane, bk, bi);
+    }
+    const float v = key_value(bk);
+    const float mx = __shfl_sync(0xffffffffu, v, 0);
+    const float ex = lane < top ? expf(v - mx) : 0.f;
+    float z = ex;
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) z += __shfl_xor_sync(0xffffffffu, z, m);
+    slot = bi;
+    weight = ex / z;
+}
+
+// Phase 3 for one warp, k_half or top up to 64: lane l owns staircase columns b = l, l + 32,
+// whose candidates are already sorted along a, and `top` rounds of best-head selection take
+// them in order (equal sums: redux.sync min over slots); svo / sso receive the selection.
+template <int KP>
+SDM_DEV void srow_combine_wide(const float* t1, const int* i1, const float* t2, const int* i2,
+                               int kh, int n, int top, float* svo, uint32_t* sso, int lane,
+                               int32_t* idx_row, float* w_row) {
+    constexpr int CPL = KP / 32;
+    int ca[CPL], lim[CPL];
+    float v2[CPL], cv[CPL];
+    uint32_t j2[CPL], ck[CPL], cs[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+        const int bcol = lane + 32 * c;
+        ca[c] = 0;
+        lim[c] = bcol < kh ? min(kh, top / (bcol + 1)) : 0;
+        v2[c] = bcol < kh ? t2[bcol] : 0.f;
+        j2[c] = bcol < kh ? (uint32_t)i2[bcol] : 0u;
+    }
+    auto head = [&](int c) {
+        if (ca[c] < lim[c]) {
+            cv[c] = t1[ca[c]] + v2[c];
+            ck[c] = order_key(cv[c]);
+            cs[c] = (uint32_t)i1[ca[c]] * (uint32_t)n + j2[c];
+        } else {
+            cv[c] = 0.f;
+            ck[c] = 0u;
+            cs[c] = 0xffffffffu;
+        }
+    };
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) head(c);
+    for (int q = 0; q < top; ++q) {
+        uint32_t bk = ck[0], bs = cs[0];
+        float bv = cv[0];
+        int bc = 0;
+#pragma unroll
+        for (int c = 1; c < CPL; ++c)
+            if (ck[c] > bk || (ck[c] == bk && cs[c] < bs)) {
+                bk = ck[c];
+                bs = cs[c];
+                bv = cv[c];
+                bc = c;
+            }
+        const uint32_t mx = __reduce_max_sync(0xffffffffu, bk);
+        const bool eq = bk == mx;
+        uint32_t bal = __ballot_sync(0xffffffffu, eq);
+        if (__popc(bal) > 1) {  // equal sums: the lower slot first
+            const uint32_t ms = __reduce_min_sync(0xffffffffu, eq ? bs : 0xffffffffu);
+            bal = __ballot_sync(0xffffffffu, eq && bs == ms);
+        }
+        if (lane == __ffs(bal) - 1) {
+            svo[q] = bv;
+            sso[q] = bs;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c)
+                if (c == bc) {
+                    ++ca[c];
+                    head(c);
+                }
+        }
+    }
+    __syncwarp();
+    const float mx = svo[0];
+    float ex[CPL], z = 0.f;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+        const int q = lane + 32 * c;
+        ex[c] = q < top ? expf(svo[q] - mx) : 0.f;
+        z += ex[c];
+    }
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) z += __shfl_xor_sync(0xffffffffu, z, m);
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+        const int q = lane + 32 * c;
+        if (q < top) {
+            idx_row[q] = (int32_t)sso[q];
+            w_row[q] = ex[c] / z;
+        }
+    }
 }
 
 template <typename XT, int PL, int KP, bool TCD>
 __global__ void __launch_bounds__(SROW_THREADS, 4) score_rows_kernel(
     const __grid_constant__ CUtensorMap km0, const __grid_constant__ CUtensorMap km1,
     ScoreRowsArgs a) {
-    constexpr int NP = 32 * PL;    // sub-keys per half, padded to whole lanes
-    constexpr int CPL = KP / 32;   // staircase columns per lane (wide variant)
     constexpr int NB = 2;  // 8-element chunks per load block
-    constexpr size_t SEG = KP == 32 ? NP * 4 + 512 : NP * 8;
+    using SM = SrowSmem<PL, KP>;
     extern __shared__ __align__(16) unsigned char srow_smem[];
     const int role = blockIdx.z;
     const XT* __restrict__ x = static_cast<const XT*>(role ? a.x[1] : a.x[0]);
@@ -291,126 +646,30 @@ __global__ void __launch_bounds__(SROW_THREADS, 4) score_rows_kernel(
     unsigned char* base = srow_smem;
     if constexpr (TCD) base += (1024 - (ptx::smem_u32(srow_smem) & 1023)) & 1023;
     float* xs = reinterpret_cast<float*>(base);  // [G][d_k] (CUDA-core dots)
-    unsigned char* segs =
-        base + (TCD ? (size_t)SROW_TC_HEAD : srow_align16((size_t)SROW_G * d_k * 4));
-    float* tv = reinterpret_cast<float*>(segs + (size_t)SROW_G * 2 * SEG);      // [G][2][KP]
-    int* ti = reinterpret_cast<int*>(tv + SROW_G * 2 * KP);                     // [G][2][KP]
-    float* sv = reinterpret_cast<float*>(ti + SROW_G * 2 * KP);                 // [G][KP]
-    uint32_t* ss = reinterpret_cast<uint32_t*>(sv + SROW_G * KP);               // [G][KP]
-    int* cand = reinterpret_cast<int*>(ss + SROW_G * KP);                       // [SROW_CAND]
-    int* ncand = cand + SROW_CAND;
+    const SM sm(base + (TCD ? (size_t)SROW_TC_HEAD : srow_align16((size_t)SROW_G * d_k * 4)));
     // element offset of row r = b*T + t in the [B,H,T,.] tensors: (b*H + h)*T + t
     auto row_off = [&](long long r) -> size_t {
         const long long b = a.T == 1 ? r : r / a.T;
         return ((size_t)b * a.H + h) * a.T + (size_t)(r - b * a.T);
     };
+    if (KP == 32 && tid < SROW_CAND) {
+        sm.cand[tid] = role ? a.cand[1][tid] : a.cand[0][tid];
+        if (tid == 0) sm.ncand[0] = role ? a.ncand[1] : a.ncand[0];
+    }
 
     if constexpr (TCD) {
         // ---- 1. tensor-core dot products ----------------------------------------------------
-        constexpr uint32_t TCOLS = 2 * ((NP + 127) / 128) * 16 <= 32
-                                       ? 32
-                                       : (2 * ((NP + 127) / 128) * 16 <= 64 ? 64 : 128);
-        uint64_t* bar_tma = reinterpret_cast<uint64_t*>(base + SROW_TC_CTRL);  // [2]
-        uint64_t* bar_mma = bar_tma + 2;                                       // [2]
-        uint64_t* bar_done = bar_mma + 2;
-        uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_done + 1);
-        int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-        const CUtensorMap* km = role ? &km1 : &km0;
-        const int cph = (n + 127) / 128, nch = 2 * cph;  // chunks per half, in all
-        auto chunk_row = [&](int c) { return (h * 2 + c / cph) * n + (c % cph) * 128; };
-        if (warp == 0) ptx::tmem_alloc(tmem_slot, TCOLS);
-        if (tid == 0) {
-            for (int i = 0; i < 2; ++i) {
-                ptx::mbar_init(bar_tma + i, 1);
-                ptx::mbar_init(bar_mma + i, 1);
-            }
-            ptx::mbar_init(bar_done, 1);
-            *abort_flag = 0;
-            ptx::fence_mbar_init();
-            for (int c = 0; c < 2 && c < nch; ++c) {
-                ptx::mbar_arrive_expect_tx(bar_tma + c, SROW_TC_KBUF);
-                ptx::tma_load_2d(base + c * SROW_TC_KBUF, km, 0, chunk_row(c), bar_tma + c);
-            }
-        }
-        {   // x operand: thread t writes 16 bytes of half t/128, row (t/8)%16 (zero past the
-            // CTA's rows), swizzled: 16-byte chunk index XOR row % 8
-            const int hx = tid >> 7, row = (tid >> 3) & 15, ch = tid & 7;
-            uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (row < SROW_G && r0 + row < rows)
-                val = __ldg(reinterpret_cast<const uint4*>(x + row_off(r0 + row) * 128 + hx * 64 +
-                                                           ch * 8));
-            *reinterpret_cast<uint4*>(base + SROW_TC_XT + hx * 2048 + row * 128 +
-                                      ((ch ^ (row & 7)) << 4)) = val;
-        }
-        if (KP == 32 && tid < SROW_CAND) {
-            cand[tid] = role ? a.cand[1][tid] : a.cand[0][tid];
-            if (tid == 0) *ncand = role ? a.ncand[1] : a.ncand[0];
-        }
-        ptx::fence_proxy_async_smem();  // the x operand is read by the tensor cores
-        ptx::tc_fence_before();
-        __syncthreads();
-        ptx::tc_fence_after();
-        const uint32_t tmem = *tmem_slot;
-        const uint64_t deadline = ptx::globaltimer_ns() + 2000000000ull;
-        if (tid == 0) {
-            const uint32_t idesc = ptx::idesc_bf16_f32(128, 16);
-            bool ok = true;
-            for (int c = 0; c < nch && ok; ++c) {
-                const int bf = c & 1;
-                const uint32_t par = (uint32_t)(c >> 1) & 1u;
-                if (!ptx::mbar_wait_bounded(bar_tma + bf, par, deadline)) {
-                    ok = false;
-                    break;
-                }
-                ptx::tc_fence_after();
-                const uint64_t ad = ptx::umma_desc_kmajor_sw128(base + bf * SROW_TC_KBUF);
-                const uint64_t bd = ptx::umma_desc_kmajor_sw128(base + SROW_TC_XT + (c / cph) * 2048);
+        const __nv_bfloat16* xr[SROW_G];
+        int rtab[SROW_G];
 #pragma unroll
-                for (int k = 0; k < 4; ++k)  // K = 64 in steps of 16 (32 bytes)
-                    ptx::umma_bf16(tmem + 16u * (uint32_t)c, ad + 2 * k, bd + 2 * k, idesc,
-                                   k > 0 ? 1u : 0u);
-                ptx::umma_commit(bar_mma + bf);
-                if (c + 2 < nch) {  // buffer bf is free once this chunk's products are done
-                    if (!ptx::mbar_wait_bounded(bar_mma + bf, par, deadline)) {
-                        ok = false;
-                        break;
-                    }
-                    ptx::mbar_arrive_expect_tx(bar_tma + bf, SROW_TC_KBUF);
-                    ptx::tma_load_2d(base + bf * SROW_TC_KBUF, km, 0, chunk_row(c + 2), bar_tma + bf);
-                }
-            }
-            if (ok) {
-                ptx::umma_commit(bar_done);
-            } else {
-                *abort_flag = 1;
-                raise_err(SDM_DEVERR_TIMEOUT);
-            }
+        for (int g = 0; g < SROW_G; ++g) {
+            xr[g] = r0 + g < rows
+                        ? reinterpret_cast<const __nv_bfloat16*>(x) + row_off(r0 + g) * 128
+                        : nullptr;
+            rtab[g] = 0;
         }
-        __syncthreads();  // thread 0 has issued everything (or given up)
-        bool aborted = *abort_flag != 0;
-        if (!aborted && !ptx::mbar_wait_bounded(bar_done, 0u, deadline)) {
-            aborted = true;
-            if (tid == 0) raise_err(SDM_DEVERR_TIMEOUT);
-        }
-        ptx::tc_fence_after();
-        if (!aborted) {  // warp w reads TMEM lanes 32 (w % 4) .. + 31 of every other chunk
-            const int q = warp & 3;
-            for (int c = warp >> 2; c < nch; c += 2) {
-                float v[4];
-                tmem_ld4(tmem + ((uint32_t)(32 * q) << 16) + 16u * (uint32_t)c, v);
-                const int hf = c / cph, sidx = (c % cph) * 128 + 32 * q + lane;
-                if (sidx < n)
-#pragma unroll
-                    for (int g = 0; g < SROW_G; ++g)
-                        reinterpret_cast<float*>(segs + (size_t)(g * 2 + hf) * SEG)[sidx] = v[g];
-            }
-        }
-        ptx::tc_fence_before();
-        __syncthreads();
-        if (warp == 0) {
-            ptx::tc_fence_after();
-            ptx::tmem_dealloc(tmem, TCOLS);
-        }
+        srow_tc_dots<32 * PL, 1>(base, sm.segs, SM::SEG, role ? &km1 : &km0, nullptr, xr, rtab,
+                                 h, n);
     } else {
         // ---- 1a. first sub-key block in flight while x is staged -----------------------------
         const int hf1 = tid >> 7, j1 = tid & 127;  // threads 0..127 half 0, 128..255 half 1
@@ -427,16 +686,12 @@ __global__ void __launch_bounds__(SROW_THREADS, 4) score_rows_kernel(
         };
         if (j1 < n) load_block(j1, 0);
 
-        // ---- 0. x rows (zeros past the last row); the staircase table ------------------------
+        // ---- 0. x rows (zeros past the last row) --------------------------------------------
     #pragma unroll
         for (int g = 0; g < SROW_G; ++g) {
             const bool live = r0 + g < rows;
             for (int c = tid; c < d_k; c += SROW_THREADS)
                 xs[g * d_k + c] = live ? to_f32(x[row_off(r0 + g) * d_k + c]) : 0.f;
-        }
-        if (KP == 32 && tid < SROW_CAND) {
-            cand[tid] = role ? a.cand[1][tid] : a.cand[0][tid];
-            if (tid == 0) *ncand = role ? a.ncand[1] : a.ncand[0];
         }
         __syncthreads();
 
@@ -473,7 +728,7 @@ __global__ void __launch_bounds__(SROW_THREADS, 4) score_rows_kernel(
                 if (s0 + 256 < n) load_block(s0 + 256, 0);
     #pragma unroll
                 for (int g = 0; g < SROW_G; ++g) {
-                    float* scf = reinterpret_cast<float*>(segs + (size_t)(g * 2 + hf1) * SEG);
+                    float* scf = reinterpret_cast<float*>(sm.seg(g, hf1));
                     scf[s0] = acc0[g];
                     if (s1 < n) scf[s1] = acc1[g];
                 }
@@ -485,215 +740,32 @@ __global__ void __launch_bounds__(SROW_THREADS, 4) score_rows_kernel(
     // ---- 2. per-half top-k: warp (g, hf) ---------------------------------------------------
     {
         const int g = warp >> 1, hf = warp & 1;
-        const float* scf = reinterpret_cast<const float*>(segs + (size_t)(g * 2 + hf) * SEG);
-        float* tvo = tv + (g * 2 + hf) * KP;
-        int* tio = ti + (g * 2 + hf) * KP;
-        if constexpr (KP == 32) {
-            uint32_t key[PL], id[PL];
-#pragma unroll
-            for (int c = 0; c < PL; ++c) {
-                const int i = c * 32 + lane;
-                id[c] = (uint32_t)i;
-                key[c] = i < n ? order_key(scf[i]) : 0u;
-            }
-            uint32_t bk, bi;
-            if constexpr (PL <= 2) {
-                top32_columns<PL>(key, id, lane);
-                bk = key[0];
-                bi = id[0];
-            } else {  // the segment's second half (NP * 4 >= 512 bytes) is the scratch
-                int2* scr = reinterpret_cast<int2*>(segs + (size_t)(g * 2 + hf) * SEG + NP * 4);
-                top32_pruned<PL>(key, id, scr, lane, bk, bi);
-            }
-            if (lane < kh) {
-                tvo[lane] = key_value(bk);
-                tio[lane] = (int)bi;
-            }
-        } else {
-            uint32_t key[PL];
-            int id[PL];
-#pragma unroll
-            for (int r = 0; r < PL; ++r) {
-                const int i = lane * PL + r;
-                id[r] = i;
-                key[r] = i < n ? order_key(scf[i]) : 0u;
-            }
-            // bitonic sort of the lane's block, best first (key desc, sub-index asc)
-#pragma unroll
-            for (int k = 2; k <= PL; k <<= 1) {
-#pragma unroll
-                for (int j = k >> 1; j > 0; j >>= 1) {
-#pragma unroll
-                    for (int i = 0; i < PL; ++i) {
-                        const int l = i ^ j;
-                        if (l > i) {
-                            const bool l_better =
-                                key[l] > key[i] || (key[l] == key[i] && id[l] < id[i]);
-                            if (((i & k) == 0) == l_better) {
-                                const uint32_t tk = key[i];
-                                key[i] = key[l];
-                                key[l] = tk;
-                                const int tix = id[i];
-                                id[i] = id[l];
-                                id[l] = tix;
-                            }
-                        }
-                    }
-                }
-            }
-            __syncwarp();  // every lane has read its scores: the segment now holds the lists
-            int2* lst = reinterpret_cast<int2*>(segs + (size_t)(g * 2 + hf) * SEG);  // [32][PL]
-#pragma unroll
-            for (int r = 2; r < PL; ++r) lst[lane * PL + r] = make_int2((int)key[r], id[r]);
-            __syncwarp();
-            uint32_t hk = key[0];
-            int hi = id[0];
-            uint32_t nk = PL > 1 ? key[PL > 1 ? 1 : 0] : 0u;
-            int ni = PL > 1 ? id[PL > 1 ? 1 : 0] : 0;
-            int p = 1;  // position of (nk, ni) in the lane's list
-            for (int q = 0; q < kh; ++q) {
-                const uint32_t mx = __reduce_max_sync(0xffffffffu, hk);
-                const uint32_t bal = __ballot_sync(0xffffffffu, hk == mx);
-                if (lane == __ffs(bal) - 1) {
-                    tvo[q] = key_value(hk);
-                    tio[q] = hi;
-                    hk = nk;
-                    hi = ni;
-                    ++p;
-                    if (p < PL) {
-                        const int2 e = lst[lane * PL + p];
-                        nk = (uint32_t)e.x;
-                        ni = e.y;
-                    } else {
-                        nk = 0u;
-                        ni = 0;
-                    }
-                }
-            }
-        }
+        srow_half_topk<PL, KP>(sm.seg(g, hf), n, kh, sm.tv + (g * 2 + hf) * KP,
+                               sm.ti + (g * 2 + hf) * KP, lane);
     }
     __syncthreads();
 
     // ---- 3. combine and softmax: warp g --------------------------------------------------
     if (warp >= SROW_G || r0 + warp >= rows) return;
     const int g = warp;
-    const float* t1 = tv + (g * 2) * KP;
-    const int* i1 = ti + (g * 2) * KP;
-    const float* t2 = tv + (g * 2 + 1) * KP;
-    const int* i2 = ti + (g * 2 + 1) * KP;
+    const float* t1 = sm.tv + (g * 2) * KP;
+    const int* i1 = sm.ti + (g * 2) * KP;
+    const float* t2 = sm.tv + (g * 2 + 1) * KP;
+    const int* i2 = sm.ti + (g * 2 + 1) * KP;
     const size_t ro = row_off(r0 + g);
     if constexpr (KP == 32) {
-        constexpr int C = SROW_CAND / 32;
-        const int nc = *ncand;
-        uint32_t key[C], id[C];
-#pragma unroll
-        for (int c = 0; c < C; ++c) {
-            const int e = c * 32 + lane;
-            if (e < nc) {
-                const int pr = cand[e], pa = pr >> 8, pb = pr & 255;
-                key[c] = order_key(t1[pa] + t2[pb]);
-                id[c] = (uint32_t)i1[pa] * (uint32_t)n + (uint32_t)i2[pb];
-            } else {
-                key[c] = 0u;
-                id[c] = 0x40000000u + (uint32_t)e;  // padding, distinct from every slot
-            }
-        }
-        uint32_t bk, bi;
-        if (nc <= 64) {
-            uint32_t k2[2] = {key[0], key[1]}, i2c[2] = {id[0], id[1]};
-            top32_columns<2>(k2, i2c, lane);
-            bk = k2[0];
-            bi = i2c[0];
-        } else {  // scratch: the second half of the row's first score segment (free by now)
-            int2* scr = reinterpret_cast<int2*>(segs + (size_t)(g * 2) * SEG + NP * 4);
-            top32_pruned<C>(key, id, scr, lane, bk, bi);
-        }
-        const float v = key_value(bk);
-        const float mx = __shfl_sync(0xffffffffu, v, 0);
-        const float ex = lane < top ? expf(v - mx) : 0.f;
-        float z = ex;
-#pragma unroll
-        for (int m = 16; m > 0; m >>= 1) z += __shfl_xor_sync(0xffffffffu, z, m);
+        // scratch: the second half of the row's first score segment (free by now)
+        int2* scr = reinterpret_cast<int2*>(sm.seg(g, 0) + 32 * PL * 4);
+        uint32_t slot;
+        float wt;
+        srow_combine32(t1, i1, t2, i2, sm.cand, sm.ncand[0], n, top, scr, lane, slot, wt);
         if (lane < top) {
-            idx_out[ro * top + lane] = (int32_t)bi;
-            w_out[ro * top + lane] = ex / z;
+            idx_out[ro * top + lane] = (int32_t)slot;
+            w_out[ro * top + lane] = wt;
         }
     } else {
-        float* svo = sv + g * KP;
-        uint32_t* sso = ss + g * KP;
-        int ca[CPL], lim[CPL];
-        float v2[CPL], cv[CPL];
-        uint32_t j2[CPL], ck[CPL], cs[CPL];
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-            const int bcol = lane + 32 * c;
-            ca[c] = 0;
-            lim[c] = bcol < kh ? min(kh, top / (bcol + 1)) : 0;
-            v2[c] = bcol < kh ? t2[bcol] : 0.f;
-            j2[c] = bcol < kh ? (uint32_t)i2[bcol] : 0u;
-        }
-        auto head = [&](int c) {
-            if (ca[c] < lim[c]) {
-                cv[c] = t1[ca[c]] + v2[c];
-                ck[c] = order_key(cv[c]);
-                cs[c] = (uint32_t)i1[ca[c]] * (uint32_t)n + j2[c];
-            } else {
-                cv[c] = 0.f;
-                ck[c] = 0u;
-                cs[c] = 0xffffffffu;
-            }
-        };
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) head(c);
-        for (int q = 0; q < top; ++q) {
-            uint32_t bk = ck[0], bs = cs[0];
-            float bv = cv[0];
-            int bc = 0;
-#pragma unroll
-            for (int c = 1; c < CPL; ++c)
-                if (ck[c] > bk || (ck[c] == bk && cs[c] < bs)) {
-                    bk = ck[c];
-                    bs = cs[c];
-                    bv = cv[c];
-                    bc = c;
-                }
-            const uint32_t mx = __reduce_max_sync(0xffffffffu, bk);
-            const bool eq = bk == mx;
-            uint32_t bal = __ballot_sync(0xffffffffu, eq);
-            if (__popc(bal) > 1) {  // equal sums: the lower slot first
-                const uint32_t ms = __reduce_min_sync(0xffffffffu, eq ? bs : 0xffffffffu);
-                bal = __ballot_sync(0xffffffffu, eq && bs == ms);
-            }
-            if (lane == __ffs(bal) - 1) {
-                svo[q] = bv;
-                sso[q] = bs;
-#pragma unroll
-                for (int c = 0; c < CPL; ++c)
-                    if (c == bc) {
-                        ++ca[c];
-                        head(c);
-                    }
-            }
-        }
-        __syncwarp();
-        const float mx = svo[0];
-        float ex[CPL], z = 0.f;
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-            const int q = lane + 32 * c;
-            ex[c] = q < top ? expf(svo[q] - mx) : 0.f;
-            z += ex[c];
-        }
-#pragma unroll
-        for (int m = 16; m > 0; m >>= 1) z += __shfl_xor_sync(0xffffffffu, z, m);
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-            const int q = lane + 32 * c;
-            if (q < top) {
-                idx_out[ro * top + q] = (int32_t)sso[q];
-                w_out[ro * top + q] = ex[c] / z;
-            }
-        }
+        srow_combine_wide<KP>(t1, i1, t2, i2, kh, n, top, sm.sv + g * KP, sm.ss + g * KP, lane,
+                              idx_out + ro * top, w_out + ro * top);
     }
 }
 

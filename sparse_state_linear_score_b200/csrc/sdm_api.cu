@@ -326,6 +326,25 @@ struct RowMaps {
     CUtensorMap km[2];
 };
 
+// Tensor maps of two sub-key tables for the row scorer's tensor-core dots: [H*2*n rows][64]
+// bf16, boxes of 128 rows, 128-byte swizzle.
+bool encode_row_maps(const sdm_dims* d, const void* sk0, const void* sk1, RowMaps* m) {
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return false;
+    const void* sk[2] = {sk0, sk1};
+    for (int r = 0; r < 2; ++r) {
+        const cuuint64_t dims[2] = {64, (cuuint64_t)d->H * 2 * d->n_sub};
+        const cuuint64_t strides[1] = {64 * 2};
+        const cuuint32_t box[2] = {64, 128};
+        const cuuint32_t es[2] = {1, 1};
+        if (enc(&m->km[r], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(sk[r]), dims,
+                strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    return true;
+}
+
 template <typename XT, int PL, bool TCD>
 sdm_status launch_score_rows_t(const RowMaps& m, const ScoreRowsArgs& a, int kp, dim3 grid,
                                cudaStream_t s) {
@@ -386,23 +405,81 @@ sdm_status launch_score_rows(const sdm_dims* d, int roles, const void* const* x,
     RowMaps m;
     memset(&m, 0, sizeof(m));
     const bool tcd = d->x_dtype == SDM_BF16 && d->d_k == 128 && d->n_sub > 64;
-    if (tcd) {
-        EncodeTiledFn enc = encode_tiled();
-        if (!enc) return SDM_ERR_CUDA;
-        for (int r = 0; r < 2; ++r) {  // [H*2*n rows][64] bf16, boxes of 128 rows
-            const cuuint64_t dims[2] = {64, (cuuint64_t)d->H * 2 * d->n_sub};
-            const cuuint64_t strides[1] = {64 * 2};
-            const cuuint32_t box[2] = {64, 128};
-            const cuuint32_t es[2] = {1, 1};
-            if (enc(&m.km[r], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.sk[r]), dims,
-                    strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-                return SDM_ERR_CUDA;
-        }
-    }
+    if (tcd && !encode_row_maps(d, a.sk[0], a.sk[1], &m)) return SDM_ERR_CUDA;
     if (d->x_dtype == SDM_F32) return launch_score_rows_x<float>(m, false, a, kp, grid, s);
     return launch_score_rows_x<__nv_bfloat16>(m, tcd, a, kp, grid, s);
+}
+
+// The one-launch decode step (decode_fused_kernel): bf16 keys and queries of d_k = 128, 64 < n
+// <= 512 (the row scorer's tensor-core dot products), k_half, W, R <= 32, d_v <= 256.
+bool decode_fused_eligible(const sdm_dims* d) {
+    return d->x_dtype == SDM_BF16 && d->d_k == 128 && d->n_sub > 64 && d->n_sub <= 512 &&
+           d->k_half <= 32 && d->W <= 32 && d->R <= 32 && d->d_v <= 256 &&
+           decode_fused_fits(d->W, d->R, d->d_v);
+}
+
+template <int PL, typename VT, int QPL>
+sdm_status launch_decode_fused_t(const RowMaps& m, const ScoreRowsArgs& a, const DecArgs& dk,
+                                 dim3 grid, cudaStream_t s) {
+    auto kern = decode_fused_kernel<PL, VT, QPL>;
+    const size_t smem = decode_fused_smem_bytes(PL);
+    if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
+    kern<<<grid, SROW_THREADS, smem, s>>>(m.km[0], m.km[1], a, dk);
+    return launch_status();
+}
+
+template <typename VT>
+sdm_status launch_decode_fused_v(int pl, int qpl, const RowMaps& m, const ScoreRowsArgs& a,
+                                 const DecArgs& dk, dim3 grid, cudaStream_t s) {
+    if (qpl <= 1) {
+        if (pl <= 4) return launch_decode_fused_t<4, VT, 1>(m, a, dk, grid, s);
+        if (pl <= 8) return launch_decode_fused_t<8, VT, 1>(m, a, dk, grid, s);
+        return launch_decode_fused_t<16, VT, 1>(m, a, dk, grid, s);
+    }
+    if (pl <= 4) return launch_decode_fused_t<4, VT, 2>(m, a, dk, grid, s);
+    if (pl <= 8) return launch_decode_fused_t<8, VT, 2>(m, a, dk, grid, s);
+    return launch_decode_fused_t<16, VT, 2>(m, a, dk, grid, s);
+}
+
+sdm_status launch_decode_fused(const sdm_dims* d, const void* q, const void* k, const void* v,
+                               const float* alpha, const float* beta, const void* skw,
+                               const void* skr, const sdm_state* st, int32_t* widx, float* ww,
+                               int32_t* ridx, float* rw, float* out, cudaStream_t s) {
+    ScoreRowsArgs a{};
+    const void* xs[2] = {k, q};
+    const void* sks[2] = {skw, skr};
+    const int tops[2] = {d->W, d->R};
+    int32_t* idxs[2] = {widx, ridx};
+    float* wts[2] = {ww, rw};
+    for (int r = 0; r < 2; ++r) {
+        a.x[r] = xs[r];
+        a.sk[r] = sks[r];
+        a.top[r] = tops[r];
+        a.idx[r] = idxs[r];
+        a.w[r] = wts[r];
+        a.ncand[r] = score_rows_staircase(d->k_half, tops[r], a.cand[r]);
+    }
+    a.B = d->B; a.H = d->H; a.T = 1; a.d_k = d->d_k; a.n = d->n_sub; a.k_half = d->k_half;
+    DecArgs dk{};
+    dk.v = v;
+    dk.alpha = alpha;
+    dk.beta = beta;
+    dk.M = st->M;
+    dk.stamp = st->stamp;
+    dk.lambda = st->Lambda;
+    dk.M0 = st->M0;
+    dk.out = out;
+    dk.N = (int)N_of(d);
+    dk.d_v = d->d_v;
+    dk.touched = d->decay == SDM_DECAY_TOUCHED;
+    RowMaps m;
+    memset(&m, 0, sizeof(m));
+    if (!encode_row_maps(d, skw, skr, &m)) return SDM_ERR_CUDA;
+    const dim3 grid((unsigned)(2 * ((d->B + 3) / 4)), (unsigned)d->H);  // clusters of 2 CTAs
+    const int pl = (d->n_sub + 31) / 32, qpl = (d->d_v / 4 + 31) / 32;
+    if (d->v_dtype == SDM_BF16)
+        return launch_decode_fused_v<__nv_bfloat16>(pl, qpl, m, a, dk, grid, s);
+    return launch_decode_fused_v<float>(pl, qpl, m, a, dk, grid, s);
 }
 
 sdm_status launch_score(const sdm_dims* d, const void* x, const void* sk, int top, int32_t* idx,
@@ -718,6 +795,59 @@ sdm_status sdm_state_materialize(const sdm_dims* dims, const sdm_state* st, floa
     return launch_status();
 }
 
+// Byte offsets of the call log's sections (rows, stamps, Lambda), 16-byte aligned.
+struct CallLog {
+    size_t rows, stamps, lam, total;
+};
+CallLog call_log_layout(const sdm_dims* d) {
+    CallLog L{};
+    const size_t occ = (size_t)BH_of(d) * (size_t)d->T * (size_t)d->W;
+    L.rows = 0;
+    L.stamps = up256(occ * (size_t)d->d_v * 4);
+    L.lam = up256(L.stamps + occ * 8);
+    L.total = up256(L.lam + (size_t)BH_of(d) * 8);
+    return L;
+}
+
+size_t sdm_call_log_bytes(const sdm_dims* dims) {
+    if (check_dims(dims) != SDM_OK) return 0;
+    return call_log_layout(dims).total;
+}
+
+static sdm_status call_log(const sdm_dims* dims, const int32_t* widx, const sdm_state* st,
+                           void* log, size_t log_bytes, bool save, sdm_stream_t stream) {
+    sdm_status e = check_dims(dims);
+    if (e) return e;
+    if ((e = check_state(st))) return e;
+    if (!widx || !log) return SDM_ERR_ARG;
+    if (!aligned16(widx) || !aligned16(log)) return SDM_ERR_ALIGN;
+    const CallLog L = call_log_layout(dims);
+    if (log_bytes < L.total) return SDM_ERR_WORKSPACE;
+    unsigned char* b = static_cast<unsigned char*>(log);
+    const size_t occ = (size_t)BH_of(dims) * (size_t)dims->T * (size_t)dims->W;
+    const size_t total = occ * (size_t)(dims->d_v / 4);
+    const int threads = 256;
+    size_t blocks = (total + threads - 1) / threads;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks == 0) blocks = 1;
+    auto kern = save ? call_log_kernel<true> : call_log_kernel<false>;
+    kern<<<(unsigned)blocks, threads, 0, (cudaStream_t)stream>>>(
+        widx, st->M, st->stamp, st->Lambda, reinterpret_cast<float*>(b + L.rows),
+        reinterpret_cast<double*>(b + L.stamps), reinterpret_cast<double*>(b + L.lam), occ,
+        dims->T * dims->W, (int)N_of(dims), dims->d_v, (int)BH_of(dims));
+    return launch_status();
+}
+
+sdm_status sdm_call_log_save(const sdm_dims* dims, const int32_t* widx, const sdm_state* st,
+                             void* log, size_t log_bytes, sdm_stream_t stream) {
+    return call_log(dims, widx, st, log, log_bytes, true, stream);
+}
+
+sdm_status sdm_call_log_restore(const sdm_dims* dims, const int32_t* widx, const void* log,
+                                size_t log_bytes, const sdm_state* st, sdm_stream_t stream) {
+    return call_log(dims, widx, st, const_cast<void*>(log), log_bytes, false, stream);
+}
+
 sdm_status sdm_score_topk(const sdm_dims* dims, const void* x, const void* subkeys, int32_t top,
                           int32_t* idx, float* w, sdm_stream_t stream) {
     const sdm_status e = check_dims(dims);
@@ -735,6 +865,12 @@ int32_t sdm_score_path(const sdm_dims* dims, int32_t top) {
     if (score_tc_eligible(dims, top)) return SDM_SCORE_TC;
     if (score_rows_eligible(dims)) return SDM_SCORE_ROWS;
     return SDM_SCORE_WARP;
+}
+
+int32_t sdm_decode_path(const sdm_dims* dims) {
+    const sdm_status e = check_dims(dims);
+    if (e) return -(int32_t)e;
+    return decode_fused_eligible(dims) ? SDM_DECODE_FUSED : SDM_DECODE_TWO;
 }
 
 sdm_status sdm_score_qk(const sdm_dims* dims, const void* q, const void* k, const void* skw,
@@ -909,6 +1045,14 @@ sdm_status sdm_decode_step(const sdm_dims* dims, const void* q, const void* k, c
         return SDM_ERR_ARG;
     if (!aligned16(v) || !aligned16(alpha) || !aligned16(beta) || !aligned16(out))
         return SDM_ERR_ALIGN;
+    if (decode_fused_eligible(dims)) {
+        if (!aligned16(q) || !aligned16(k) || !aligned16(skw) || !aligned16(skr) ||
+            !aligned16(widx) || !aligned16(ww) || !aligned16(ridx) || !aligned16(rw))
+            return SDM_ERR_ALIGN;
+        if (dims->B == 0) return SDM_OK;
+        return launch_decode_fused(dims, q, k, v, alpha, beta, skw, skr, st, widx, ww, ridx, rw,
+                                   out, (cudaStream_t)stream);
+    }
     if ((e = score_both_roles(dims, q, k, skw, skr, widx, ww, ridx, rw, stream))) return e;
     const int rpw = ((dims->W > dims->R ? dims->W : dims->R) + DECODE_WARPS - 1) / DECODE_WARPS;
     const int qpl = (dims->d_v / 4 + 31) / 32;

@@ -170,3 +170,28 @@ def test_score_path_dispatch(lib):
     d = sdm.Dims(wl.B, wl.H, wl.T, wl.d_k, wl.n_sub, wl.d_v, wl.k_half, wl.W, wl.R,
                  wl.x_dtype, wl.v_dtype)
     assert sdm.score_path(d, wl.W) == sdm.SCORE_ROWS  # fp32
+
+
+def test_decode_path_dispatch(lib):
+    """The decode workload's step is one launch (scoring and recurrence steps in one cluster of
+    two CTAs); shapes outside the fused kernel's limits (n = 64 or 1024, k = 64, fp32 keys,
+    d_k = 64, d_v = 256 whose two steps' arrays exceed the sub-key buffers) take the scoring
+    launch and the recurrence launch."""
+    import sparse_state_linear_score_b200 as sdm
+    import sdm_synth as S
+    wl = S.DECODE
+    d = sdm.Dims(wl.B, wl.H, 1, wl.d_k, wl.n_sub, wl.d_v, wl.k_half, wl.W, wl.R, wl.x_dtype,
+                 wl.v_dtype)
+    assert sdm.decode_path(d) == sdm.DECODE_FUSED
+    for kw in (dict(n_sub=64), dict(k_half=64, W=64, R=64), dict(x_dtype="f32"), dict(d_k=64),
+               dict(n_sub=1024), dict(d_v=256)):
+        w2 = wl.scaled(**kw)
+        d2 = sdm.Dims(w2.B, w2.H, 1, w2.d_k, w2.n_sub, w2.d_v, w2.k_half, w2.W, w2.R,
+                      w2.x_dtype, w2.v_dtype)
+        assert sdm.decode_path(d2) == sdm.DECODE_TWO, kw
+    for kw in (dict(n_sub=128, d_v=64), dict(n_sub=512, d_v=192, v_dtype="f32"),
+               dict(W=16, R=8, k_half=16)):
+        w2 = wl.scaled(**kw)
+        d2 = sdm.Dims(w2.B, w2.H, 1, w2.d_k, w2.n_sub, w2.d_v, w2.k_half, w2.W, w2.R,
+                      w2.x_dtype, w2.v_dtype)
+        assert sdm.decode_path(d2) == sdm.DECODE_FUSED, kw
