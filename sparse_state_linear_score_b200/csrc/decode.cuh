@@ -396,16 +396,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SROW_THREADS, QPL ==
         if (tid == 0) sm.ncand[0] = a.ncand[role];
     }
     // the decay inputs of the rows this CTA selects (warp g: sequence b0 + g) and of the
-    // sequences it steps, read while the scores are computed
+    // sequences it steps: loads issued now, used after the scores (nothing waits on them
+    // before the sub-key stream is under way)
     const int bg = b0 + warp;
-    double Lg = 0.0;
     float ag = 1.f;
+    double lam = 0.0;
     if (warp < SROW_G && bg < B) {
         const size_t bh = (size_t)bg * H + h;
         ag = dk.alpha[bh];
-        if (!(ag > 0.f) && lane == 0) raise_err(SDM_DEVERR_ALPHA);  // treated as alpha = 1
-        Lg = dk.lambda[bh] + (ag > 0.f ? log((double)ag) : 0.0);
-        if (lane == 0) lnew[warp] = Lg;
+        lam = dk.lambda[bh];
     }
     float4 vv[2][QPL];
     float bt[2];
@@ -441,6 +440,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SROW_THREADS, QPL ==
     __syncthreads();
     if (warp < SROW_G && bg < B) {
         const int g = warp;
+        if (!(ag > 0.f) && lane == 0) raise_err(SDM_DEVERR_ALPHA);  // treated as alpha = 1
+        const double Lg = lam + (ag > 0.f ? log((double)ag) : 0.0);  // Lambda'
+        if (lane == 0) lnew[g] = Lg;
         int2* scr = reinterpret_cast<int2*>(sm.seg(g, 0) + 32 * PL * 4);
         uint32_t slot;
         float wt;
