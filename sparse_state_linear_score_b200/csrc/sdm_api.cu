@@ -1180,7 +1180,8 @@ sdm_status sdm_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* A, const v
     if (M < 1 || N < 1 || K < 8 || K % 8 != 0) return SDM_ERR_SHAPE;
     if (!A || !Bt || !C) return SDM_ERR_ARG;
     if (!aligned16(A) || !aligned16(Bt) || !aligned16(C)) return SDM_ERR_ALIGN;
-    if ((long long)(M + GEMM_BM - 1) / GEMM_BM > 65535) return SDM_ERR_SHAPE;
+    if ((long long)((M + GEMM_BM - 1) / GEMM_BM) * ((N + GEMM_BN - 1) / GEMM_BN) > 0x7fffffffLL)
+        return SDM_ERR_SHAPE;
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return SDM_ERR_CUDA;
     CUtensorMap am, bm;
@@ -1210,15 +1211,22 @@ sdm_status sdm_gemm_bf16(int32_t M, int32_t N, int32_t K, const void* A, const v
     if (N % 4 == 0) {
         const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
         const cuuint64_t strides[1] = {(cuuint64_t)N * 4};
-        const cuuint32_t box[2] = {32, GEMM_BM};
+        const cuuint32_t box[2] = {32, 32};  // one epilogue warp's 32 rows x 32 columns
         cm_ok = enc(&cm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, C, dims, strides, box, es,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     }
-    if (!set_smem(gemm_bf16_tc_kernel, GEMM_SMEM_BYTES)) return SDM_ERR_CUDA;
-    const dim3 grid((unsigned)((N + GEMM_BN - 1) / GEMM_BN), (unsigned)((M + GEMM_BM - 1) / GEMM_BM));
-    gemm_bf16_tc_kernel<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, stream>>>(am, bm, cm, cm_ok, C, M,
-                                                                        N, K);
+    auto kern = gemm_bf16_tc_kernel;
+    const uint32_t smem = GEMM_SMEM_BYTES;
+    if (!set_smem(kern, smem)) return SDM_ERR_CUDA;
+    // persistent: one CTA per SM (or per tile, when there are fewer tiles)
+    const long long tiles = (long long)((M + GEMM_BM - 1) / GEMM_BM) * ((N + GEMM_BN - 1) / GEMM_BN);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return SDM_ERR_CUDA;
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+    kern<<<grid, GEMM_THREADS, smem, stream>>>(am, bm, cm, cm_ok, C, M, N, K);
     return launch_status();
 }
 

@@ -43,7 +43,12 @@ def gemm_check(sdm, M, N, K, seed):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (256, 512, 512), (200, 300, 72), (1, 16, 8),
-                                   (129, 257, 136), (1000, 48, 520)])
+                                   (129, 257, 136), (1000, 48, 520),
+                                   # more tiles than SMs: several tiles per persistent CTA,
+                                   # both TMEM accumulators, the stage ring across tiles
+                                   (2560, 3072, 64), (2048, 2560, 328),
+                                   # K > 1024: the deep-ring configuration
+                                   (300, 520, 1544), (1280, 4096, 2048)])
 def test_gemm_vs_fp64(sdm, M, N, K):
     gemm_check(sdm, M, N, K, seed=M * 7 + N * 3 + K)
 
