@@ -532,6 +532,40 @@ def run_workload(name: str, device, sdm, steps: int = 5, warm: int = 3,
     return res
 
 
+def run_gemm_only(device, sdm, steps: int = 10, warm: int = 3) -> dict:
+    """The layer's two projections (the mid workload's shapes) on their own: the input side's
+    GEMM [B*T, d_model] x [H*hs, d_model]^T and the output side's [B*T, H*d_v] x
+    [d_model, H*d_v]^T, bf16 in, fp32 out, each timed over `steps` back-to-back calls."""
+    import torch
+
+    import sdm_synth as S
+    wl = S.MID
+    dm = 4 * wl.H * wl.n_sub
+    hs = 2 * wl.d_k + 2 * wl.d_v + 2
+    gen = torch.Generator(device=device).manual_seed(11)
+    res = {}
+    pk = measured_peaks()["bf16_tflops"]
+    for name, (M, N, K) in (("gemm_in", (wl.B * wl.T, wl.H * hs, dm)),
+                            ("gemm_out", (wl.B * wl.T, dm, wl.H * wl.d_v))):
+        A = torch.randn(M, K, device=device, generator=gen).to(torch.bfloat16)
+        Bt = torch.randn(N, K, device=device, generator=gen).to(torch.bfloat16)
+        C = torch.empty(M, N, device=device)
+        for _ in range(warm):
+            sdm.gemm_bf16(A, Bt, C)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            sdm.gemm_bf16(A, Bt, C)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        tf = 2.0 * M * N * K / (ms / 1e3) / 1e12
+        res[name] = {"M": M, "N": N, "K": K, "ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / pk}
+        del A, Bt, C
+    res["device_errors"] = sdm.device_error()
+    return res
+
+
 def run_score_only(name: str, device, sdm, tokens: int | None = None, steps: int = 5,
                    warm: int = 3) -> dict:
     """Both roles' scoring of one workload (`sdm_score_qk`) on its own: `tokens` replaces the
@@ -971,7 +1005,17 @@ def main(argv=None):
                          "--warmup) and print its object")
     ap.add_argument("--score-tokens", type=int, default=None,
                     help="tokens per sequence for --score-only (default: the workload's T)")
+    ap.add_argument("--gemm-only", action="store_true",
+                    help="run only the layer's two projection GEMMs (--steps timed calls each) "
+                         "and print their object")
     args = ap.parse_args(argv)
+    if args.gemm_only:
+        import torch
+
+        import sparse_state_linear_score_b200 as sdm
+        print(json.dumps({"gemm": run_gemm_only(torch.device("cuda", 0), sdm, steps=args.steps,
+                                                warm=max(3, args.warmup))}), flush=True)
+        return
     if args.score_only:
         import torch
 

@@ -2,8 +2,9 @@
 // A and B bf16 and K-contiguous, accumulation in fp32 in TMEM.
 //
 // Persistent and warp-specialised: one CTA per SM walks the 128 x 256 output tiles
-// blockIdx.x, blockIdx.x + gridDim.x, ... (m fastest, so the CTAs running together share the
-// B block and sweep A).  Its six warps take three roles:
+// blockIdx.x, blockIdx.x + gridDim.x, ... (n fastest, so the CTAs running together take every
+// column block of a few row blocks: each A block is read from memory about once while the B
+// blocks stay in L2).  Its six warps take three roles:
 //   warp 0      (one lane) TMA producer: the A and B K-blocks (64 wide, 128-byte swizzle) of
 //               every tile into a GEMM_STAGES-deep ring; full[s] completes on the bytes,
 //               empty[s] is the MMA's release of the stage.
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_bf16_tc_kernel(
         // ---- producer ----
         uint32_t it = 0;
         for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
-            const int m0 = (t % num_m) * GEMM_BM, n0 = (t / num_m) * GEMM_BN;
+            const int m0 = (t / num_n) * GEMM_BM, n0 = (t % num_n) * GEMM_BN;
             for (int kb = 0; kb < nk; ++kb, ++it) {
                 const uint32_t s = it % GEMM_STAGES, use = it / GEMM_STAGES;
                 if (use > 0 && !ptx::mbar_wait_bounded(empty + s, (use - 1) & 1u, deadline)) {
@@ -157,7 +158,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_bf16_tc_kernel(
                 break;
             }
             ptx::tc_fence_after();
-            const int m0 = (t % num_m) * GEMM_BM, n0 = (t / num_m) * GEMM_BN;
+            const int m0 = (t / num_n) * GEMM_BM, n0 = (t % num_n) * GEMM_BN;
             const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + acc * GEMM_BN;
             for (int c = 0; c < GEMM_BN; c += 32, ++gc) {
                 float v[32];
