@@ -49,18 +49,42 @@ sdm_status check_dims(const sdm_dims* d) {
 
 inline long long N_of(const sdm_dims* d) { return (long long)d->n_sub * d->n_sub; }
 inline long long BH_of(const sdm_dims* d) { return (long long)d->B * d->H; }
-inline int col_width(const sdm_dims* d) { return d->d_v % 8 == 0 ? 8 : 4; }
-
-// Tokens per chunk of the prefill recurrence: as many as fit the plan's occurrence
-// budget, the run kernel's shared memory and the 256-token scan of plan_local.
-int chunk_tokens(const sdm_dims* d) {
-    const int CW = col_width(d);
+// Tokens per chunk of the prefill recurrence with CW-column slices: as many as fit the plan's
+// occurrence budget, the run kernel's shared memory and the 256-token scan of plan_local.
+int chunk_tokens_cw(const sdm_dims* d, int CW) {
     int C = PLAN_MAX_OCC / (d->W + d->R);
     if (C > PLAN_MAX_C) C = PLAN_MAX_C;
     C &= ~3;  // matrices move in 16-byte rows
     while (C > 4 && run_smem_bytes(C, d->W, d->R, CW, 4) > kSmemBudget) C -= 4;
     return C < 4 ? 4 : C;
 }
+
+int device_sms() {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0, n = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+            sms = n;
+        else
+            return 148;
+    }
+    return sms;
+}
+
+// Value columns per row-pass CTA.  The row pass is bound by the SM's rate of scattered row
+// requests, not by their bytes (4-column slices take as long per chunk as 8-column ones), so
+// wider slices move more bytes per request.  16 columns when the row is a multiple of 16, the
+// chunk size stays what 8 columns allow, and the CTAs still fill the SMs (B*H*d_v/16 of
+// them); else 8, else 4.
+int col_width(const sdm_dims* d) {
+    if (d->d_v % 16 == 0 && chunk_tokens_cw(d, 16) == chunk_tokens_cw(d, 8) &&
+        BH_of(d) * (d->d_v / 16) >= device_sms())
+        return 16;
+    return d->d_v % 8 == 0 ? 8 : 4;
+}
+
+int chunk_tokens(const sdm_dims* d) { return chunk_tokens_cw(d, col_width(d)); }
 
 struct WsLayout {
     int C, J;
@@ -962,6 +986,11 @@ sdm_status forward_run_impl(const sdm_dims* dims, const void* v, const float* be
             return SDM_ERR_CUDA;
     }
     const int CW = col_width(dims);
+    if (CW == 16) {
+        if (dims->v_dtype == SDM_BF16)
+            return launch_run_t<16, __nv_bfloat16>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, ep, stream);
+        return launch_run_t<16, float>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, ep, stream);
+    }
     if (CW == 8) {
         if (dims->v_dtype == SDM_BF16)
             return launch_run_t<8, __nv_bfloat16>(dims, L, P, v, beta, widx, ww, ridx, rw, st, out, ep, stream);

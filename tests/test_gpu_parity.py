@@ -196,6 +196,22 @@ def test_forward_shared_slots(sdm, orc, T, pool, W, R):
     _forward_case(sdm, orc, wl, inp, widx, ww, ridx, rw, TOL["f32"])
 
 
+@pytest.mark.parametrize("vdt,dv", [("f32", 32), ("bf16", 64)])
+def test_forward_sixteen_column_slices(sdm, orc, vdt, dv):
+    """Enough sequences that the row pass takes 16-column slices (B*H*d_v/16 CTAs fill the
+    SMs: 320 and 640 here), ragged last chunk, slots shared within and across chunks."""
+    B, H, T, W, R = 4, 40, 70, 6, 5
+    wl = S.TINY.scaled(B=B, H=H, T=T, n_sub=16, d_v=dv, k_half=8, W=W, R=R, v_dtype=vdt,
+                       alpha=("uniform", 0.6, 1.0))
+    inp = to_dev(S.generate(wl))
+    g = torch.Generator().manual_seed(dv)
+    widx = S.random_indices(B, H, T, wl.N, W, g, pool=60).cuda()
+    ridx = S.random_indices(B, H, T, wl.N, R, g, pool=60).cuda()
+    ww = S.random_weights(B, H, T, W, g).cuda()
+    rw = S.random_weights(B, H, T, R, g).cuda()
+    _forward_case(sdm, orc, wl, inp, widx, ww, ridx, rw, TOL[vdt])
+
+
 def test_forward_long_call_walk_path(sdm, orc):
     """More than 512 chunks in one call: the plan takes its sequential walk instead of the
     per-slot chunk masks; results must not depend on which is used."""
