@@ -53,7 +53,7 @@ namespace sdm {
 
 constexpr int PLAN_MAX_OCC = 2048;  // C*(W+R) never exceeds this
 constexpr int PLAN_MAX_C = 32;      // tokens per chunk
-constexpr int PLAN_HASH = 4096;     // hash buckets (>= 2 * max write occurrences)
+constexpr int PLAN_HASH = 2048;     // hash buckets (>= the write occurrences of a chunk)
 constexpr int PLAN_THREADS = 256;
 constexpr int WALK_THREADS = 512;
 constexpr int WALK_MAXO = PLAN_MAX_OCC / WALK_THREADS;
@@ -67,7 +67,8 @@ constexpr int LK_PREV_SHIFT = 18;  // bits 18..29: 1 + previous chunk's owner of
 SDM_DEV int lk_link(int lk) { return (lk & 0xffff) - 1; }
 SDM_DEV int lk_prev(int lk) { return ((lk >> LK_PREV_SHIFT) & 0xfff) - 1; }
 
-SDM_DEV unsigned slot_hash(int s) { return ((unsigned)s * 2654435761u) >> (32 - 12); }
+SDM_DEV unsigned slot_hash(int s) { return ((unsigned)s * 2654435761u) >> (32 - 11); }
+static_assert(PLAN_HASH == 1 << 11, "slot_hash takes the top 11 bits");
 
 // Dynamic shared memory of plan_local (bytes).
 __host__ __device__ inline size_t plan_local_smem_bytes() {
@@ -159,7 +160,7 @@ __host__ __device__ inline RunImg run_img(int C, int W, int R) {
 
 // TOUCHED: touched-slots decay (PlanPtrs::vfc and vsh are set); the default decays every slot.
 template <bool TOUCHED>
-__global__ void __launch_bounds__(PLAN_THREADS, 2) plan_local_kernel(
+__global__ void __launch_bounds__(PLAN_THREADS, 3) plan_local_kernel(
     const float* __restrict__ alpha, const float* __restrict__ beta,
     const int32_t* __restrict__ widx, const float* __restrict__ ww,
     const int32_t* __restrict__ ridx, const float* __restrict__ rw,
@@ -175,8 +176,8 @@ __global__ void __launch_bounds__(PLAN_THREADS, 2) plan_local_kernel(
     int* s_slot = reinterpret_cast<int*>(s_bet + PLAN_MAX_C); // [2048]
     int* s_slot2 = s_slot + PLAN_MAX_OCC;                     // previous chunk's write slots
     float* s_wt = reinterpret_cast<float*>(s_slot2 + PLAN_MAX_OCC);  // [2048] weights
-    int* s_head = reinterpret_cast<int*>(s_wt + PLAN_MAX_OCC);       // [4096] (32-bit atomics)
-    int* s_head2 = s_head + PLAN_HASH;                               // [4096]
+    int* s_head = reinterpret_cast<int*>(s_wt + PLAN_MAX_OCC);       // [PLAN_HASH] (32-bit atomics)
+    int* s_head2 = s_head + PLAN_HASH;                               // [PLAN_HASH]
     short* s_link = reinterpret_cast<short*>(s_head2 + PLAN_HASH);
     short* s_next = s_link + PLAN_MAX_OCC;
     short* s_next2 = s_next + PLAN_MAX_OCC;
