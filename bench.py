@@ -35,10 +35,9 @@ L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 # the hash of the kernel sources it was taken with; None when not yet measured for the
 # current sources.  Filled from profiles/ (see the summary named there).
 MEASURED_TRAFFIC = {
-    # profiles/recur_run_kernel_mid_prefill.md: dram read 728.85 MB + write 406.16 MB, taken
-    # after the row pass gained its fused layer-output variant (a separate instantiation;
-    # the plain one is unchanged)
-    "e719ce73f5a42202": 1_135_003_648,
+    # profiles/recur_run_kernel_mid_prefill.md: dram read 728.72 MB + write 405.46 MB, taken
+    # after plan_local's hash table was halved (the row pass itself unchanged)
+    "3a393632b1033ab5": 1_134_180_864,
 }
 
 
