@@ -33,10 +33,11 @@ L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 
 # DRAM traffic per launch of the recurrence row pass from an ncu capture (bytes), keyed by
 # the hash of the kernel sources it was taken with; None when not yet measured for the
-# current sources.  Filled from profiles/ (see the summary named there).
+# current sources.  Filled by hand from the capture of the row pass on the mid-size workload
+# (dram__bytes_read.sum + dram__bytes_write.sum of one launch).
 MEASURED_TRAFFIC = {
-    # profiles/recur_run_kernel_mid_prefill.md: dram read 728.72 MB + write 405.46 MB, taken
-    # after plan_local's hash table was halved (the row pass itself unchanged)
+    # dram read 728.72 MB + write 405.46 MB, taken after plan_local's hash table was halved
+    # (the row pass itself unchanged)
     "3a393632b1033ab5": 1_134_180_864,
 }
 
