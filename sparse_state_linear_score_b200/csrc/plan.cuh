@@ -543,8 +543,26 @@ __global__ void __launch_bounds__(WALK_THREADS) plan_walk_kernel(
     const double* Lr = lstart_smem ? s_L : Lg;
     const size_t occ_base = bh * (size_t)T * (W + R);
 
+    // a chunk's write words and read words are two contiguous runs: with W and R multiples of
+    // 4 both start on 16-byte boundaries (here and in the ring) and move in 16-byte pieces
+    const bool vec = (W & 3) == 0 && (R & 3) == 0;
     auto load_stage = [&](int jn) {
-        if (jn < J) {
+        if (jn < J && vec) {
+            uint32_t* dst = s_ring + (jn % WALK_RING) * stage;
+            const int t0 = jn * C, nt = min(C, T - t0), nw = nt * W, nr = nt * R;
+            const uint32_t* wsrc = P.occw + occ_base + (size_t)t0 * W;
+            const uint32_t* rsrc = P.occw + occ_base + (size_t)T * W + (size_t)t0 * R;
+            for (int p = tid; p < (nw + nr) / 4; p += WALK_THREADS) {
+                const int o = 4 * p;  // nw is a multiple of 4: a piece is all writes or all reads
+                cp_async16(dst + o, o < nw ? wsrc + o : rsrc + (o - nw), true);
+            }
+            for (int t = tid; t < nt; t += WALK_THREADS) {
+                const unsigned d = (unsigned)__cvta_generic_to_shared(dst + PLAN_MAX_OCC + t);
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(d),
+                             "l"(P.lam + bh * T + t0 + t)
+                             : "memory");
+            }
+        } else if (jn < J) {
             uint32_t* dst = s_ring + (jn % WALK_RING) * stage;
             const int t0 = jn * C, nt = min(C, T - t0), nw = nt * W, no = nt * (W + R);
             for (int o = tid; o < no; o += WALK_THREADS) {
