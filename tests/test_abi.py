@@ -195,3 +195,33 @@ def test_decode_path_dispatch(lib):
         d2 = sdm.Dims(w2.B, w2.H, 1, w2.d_k, w2.n_sub, w2.d_v, w2.k_half, w2.W, w2.R,
                       w2.x_dtype, w2.v_dtype)
         assert sdm.decode_path(d2) == sdm.DECODE_FUSED, kw
+
+
+def test_call_log_host_checks(lib):
+    """sdm_call_log_bytes covers the rows and stamps of every write occurrence and Lambda;
+    save and restore refuse bad arguments on the host (nothing is launched)."""
+    class State(ctypes.Structure):
+        _fields_ = [("M", ctypes.c_void_p), ("stamp", ctypes.c_void_p), ("Lambda", ctypes.c_void_p),
+                    ("M0", ctypes.c_void_p)]
+    lib.sdm_call_log_bytes.restype = ctypes.c_size_t
+    d = mid_dims()
+    BH, T, W, dv = 2 * 4, 4096, 32, 128
+    nb = lib.sdm_call_log_bytes(ctypes.byref(d))
+    assert nb >= BH * T * W * (dv * 4 + 8) + BH * 8
+    assert nb < BH * T * W * (dv * 4 + 8) + BH * 8 + 3 * 256  # three 256-byte aligned sections
+    # the log grows with the write slots, not with N or R
+    assert lib.sdm_call_log_bytes(ctypes.byref(mid_dims(n_sub=512, R=8))) == nb
+    assert lib.sdm_call_log_bytes(ctypes.byref(mid_dims(W=16))) < nb
+    assert lib.sdm_call_log_bytes(ctypes.byref(mid_dims(W=65))) == 0  # bad dims
+    p = ctypes.c_void_p(0x1000)
+    st = State(0x1000, 0x2000, 0x3000, 0x4000)
+    small = ctypes.c_size_t(nb - 1)
+    assert lib.sdm_call_log_save(ctypes.byref(d), None, ctypes.byref(st), p,
+                                 ctypes.c_size_t(nb), None) == 1                  # SDM_ERR_ARG
+    assert lib.sdm_call_log_save(ctypes.byref(d), p, ctypes.byref(st), p, small, None) == 7
+    assert lib.sdm_call_log_restore(ctypes.byref(d), p, p, small, ctypes.byref(st), None) == 7
+    assert lib.sdm_call_log_restore(ctypes.byref(d), p, ctypes.c_void_p(0x1008),
+                                    ctypes.c_size_t(nb), ctypes.byref(st), None) == 4  # ALIGN
+    st_bad = State(0x1000, 0x2000, 0x3003, 0x4000)
+    assert lib.sdm_call_log_save(ctypes.byref(d), p, ctypes.byref(st_bad), p,
+                                 ctypes.c_size_t(nb), None) == 4
