@@ -28,6 +28,7 @@ namespace {
 constexpr int kMaxTop = 64;
 constexpr size_t kSmemBudget = 220 * 1024;  // dynamic shared memory per CTA we plan for
 constexpr size_t kMaskBudget = size_t(512) << 20;  // workspace bytes for per-slot chunk masks
+                                                     // (or a quarter of the state, if larger)
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -121,9 +122,12 @@ WsLayout ws_layout(const sdm_dims* d) {
     L.off_fe = o;     o = up256(o + BH * occ * 4);
     L.off_lk = o;     o = up256(o + BH * occ * 4);
     L.off_occw = o;   o = up256(o + BH * occ * 4);
-    // per-slot chunk masks replace the sequential walk when they stay small
+    // per-slot chunk masks replace the sequential walk when they stay small: within a fixed
+    // budget, or within a quarter of the state's own rows (whose gathers dwarf their traffic)
     const size_t mw = (size_t)(L.J + 63) / 64;
-    L.MW = (L.J <= 512 && BH * N * mw * 8 <= kMaskBudget) ? (int)mw : 0;
+    const size_t state_rows = BH * N * (size_t)d->d_v * 4;
+    const size_t budget = kMaskBudget > state_rows / 4 ? kMaskBudget : state_rows / 4;
+    L.MW = (L.J <= 512 && BH * N * mw * 8 <= budget) ? (int)mw : 0;
     L.off_mask = o;   o = up256(o + BH * N * (size_t)L.MW * 8);
     L.off_wtab = o;   o = up256(o + (L.MW ? 0 : BH * N * 2));
     L.off_cnt = o;    o = up256(o + BH * (size_t)L.J * 4);
