@@ -1,5 +1,7 @@
-// Single-token step for every (b,h): one CTA per sequence owns full slot rows, so it
-// reads and writes the stamps directly (no plan needed).
+// Single-token step for every (b,h): the CTA that steps a sequence owns its full slot rows,
+// so it reads and writes the stamps directly (no plan needed).  Two forms: decode_kernel (one
+// CTA per sequence, after a separate scoring launch) and decode_fused_kernel (clusters of two
+// CTAs that score four sequences' keys and queries and then step them, one launch per step).
 //
 // Per sequence, following §2 Background "Gated DeltaNet" and §3 Method:
 //   Lambda' = Lambda + log(alpha)
